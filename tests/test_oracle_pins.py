@@ -1,0 +1,502 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Each test checks the oracle against brute force, exact rational arithmetic,
+torch's own float8 conversion, closed forms, invariants, or autograd /
+finite differences of an independently written straight-through surrogate.
+A plausible slip in the oracle (a dropped term, a wrong sign or index, a
+transposed operand, a wrong tie rule) fails at least one of them.
+"""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantization_aware_attention_nvfp4_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _all_finite_bf16():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = W.bf16_bits_to_f32(bits)
+    keep = np.isfinite(vals)
+    return bits[keep], vals[keep].astype(np.float64)
+
+
+# ------------------------------------------------------------ E4M3 scale ----
+
+def test_e4m3_value_table_matches_torch():
+    codes = np.arange(127, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([oracle.e4m3_value(int(c)) for c in codes])
+    assert np.array_equal(ref, mine)
+
+
+def test_e4m3_scale_exhaustive_vs_torch_float8():
+    """(i) every finite bf16 amax: scale = nearest E4M3 to a/6 (torch's RNE
+    float32 -> float8_e4m3fn conversion, saturated at 448)."""
+    _, vals = _all_finite_bf16()
+    a = np.abs(vals)
+    t = np.minimum(a / 6.0, 448.0).astype(np.float32)
+    ref = torch.from_numpy(t).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = np.array([oracle.e4m3_round_div6(x) for x in a], dtype=np.uint8)
+    bad = np.nonzero(ref != mine)[0]
+    assert bad.size == 0, (a[bad[:5]], ref[bad[:5]], mine[bad[:5]])
+
+
+def _e4m3_values_fraction():
+    out = []
+    for code in range(127):
+        e, m = code >> 3, code & 7
+        out.append(Fraction(m, 512) if e == 0 else Fraction(8 + m, 8) * Fraction(2) ** (e - 7))
+    return out
+
+
+def _nearest_fraction(target, values):
+    """Brute force: the nearest of the sorted values, ties to the even index,
+    saturating to the last."""
+    if target >= values[-1]:
+        return len(values) - 1
+    best = None
+    for i, v in enumerate(values):
+        d = abs(v - target)
+        if best is None or d < best[0] or (d == best[0] and i % 2 == 0):
+            best = (d, i)
+    return best[1]
+
+
+def test_e4m3_scale_rational_bruteforce_sample():
+    """Exact rational arithmetic, independent of float64 and of torch."""
+    vals = _e4m3_values_fraction()
+    rng = np.random.default_rng(7)
+    bits, fv = _all_finite_bf16()
+    pick = rng.choice(np.nonzero((np.abs(fv) < 3000) & (fv != 0))[0], 400, replace=False)
+    # plus every exact tie a = 6 * midpoint that bf16 can represent
+    ties = []
+    for i in range(126):
+        mid = (vals[i] + vals[i + 1]) / 2 * 6
+        f = float(mid)
+        if Fraction(f) == mid and W.f32_to_bf16_bits(np.array([f], np.float32))[0] is not None:
+            b = W.f32_to_bf16_bits(np.array([f], np.float32))
+            if Fraction(float(W.bf16_bits_to_f32(b)[0])) == mid:
+                ties.append(f)
+    assert len(ties) > 50
+    for a in list(np.abs(fv[pick])) + ties:
+        want = _nearest_fraction(Fraction(float(a)) / 6, vals)
+        assert oracle.e4m3_round_div6(float(a)) == want, a
+
+
+def test_e4m3_golden_points():
+    g = json.load(open(os.path.join(GOLDEN, "e4m3_e2m1_points.json")))
+    for code, v in g["e4m3_value_of_code"]:
+        assert oracle.e4m3_value(code) == v
+    for a, code in g["e4m3_amax_to_code"]:
+        assert oracle.e4m3_round_div6(a) == code, a
+
+
+# ------------------------------------------------------------- E2M1 code ----
+
+def _e2m1_thresholds(ax, s):
+    """Independent formulation: count the midpoints passed.  Crossing the
+    midpoint between codes k and k+1 needs a strict '>' when k is even (the
+    tie stays on the even k) and '>=' when k is odd (the tie moves up to the
+    even k+1)."""
+    code = np.zeros(ax.shape, np.int32)
+    for k in range(7):
+        mid2 = (GRID[k] + GRID[k + 1]) * s
+        if k % 2 == 0:
+            code += (2 * ax > mid2)
+        else:
+            code += (2 * ax >= mid2)
+    return code
+
+
+def test_e2m1_exhaustive_all_bf16_times_all_scales():
+    """(ii) every finite bf16 x against every positive finite E4M3 scale."""
+    _, fv = _all_finite_bf16()
+    ax = np.abs(fv)
+    for sc in range(1, 127):
+        s = oracle.e4m3_value(sc)
+        mine = oracle.e2m1_round_many(ax, np.float64(s))
+        ref = _e2m1_thresholds(ax, s)
+        bad = np.nonzero(mine != ref)[0]
+        assert bad.size == 0, (sc, ax[bad[:5]], mine[bad[:5]], ref[bad[:5]])
+
+
+def test_e2m1_golden_points():
+    g = json.load(open(os.path.join(GOLDEN, "e4m3_e2m1_points.json")))
+    assert [oracle.e2m1_value(c) for c in range(8)] == g["e2m1_grid"]
+    for ratio, code in g["e2m1_ratio_to_code"]:
+        assert oracle.e2m1_round(ratio, 1.0) == code, ratio
+        assert oracle.e2m1_round(ratio * 0.171875, 0.171875) == code, ratio
+
+
+# ------------------------------------------------------- block quantizer ----
+
+def _fq_block_fraction(xs):
+    """Pure-Python exact fq of one block (Fractions): returns (codes, scale
+    code, dequantized Fractions)."""
+    vals = _e4m3_values_fraction()
+    grid = [Fraction(g) for g in GRID]
+    fx = [Fraction(float(x)) for x in xs]
+    a = max(abs(x) for x in fx)
+    sc = 0 if a == 0 else _nearest_fraction(a / 6, vals)
+    s = vals[sc]
+    codes, deq = [], []
+    for x, raw in zip(fx, xs):
+        neg = 1 if np.signbit(raw) else 0
+        c = 0 if s == 0 else _nearest_fraction(abs(x) / s, grid)
+        codes.append((neg << 3) | c)
+        deq.append((-1 if neg else 1) * grid[c] * s)
+    return codes, sc, deq
+
+
+def _special_blocks(rng):
+    """Random, tie-rich, subnormal-scale, saturating and signed-zero blocks."""
+    blocks = []
+    for _ in range(60):
+        blocks.append(rng.standard_normal(16).astype(np.float32) * np.float32(10 ** rng.uniform(-4, 3)))
+    vals = [float(v) for v in _e4m3_values_fraction()]
+    for _ in range(60):  # elements exactly at g*s midpoints of a normal scale
+        sc = int(rng.integers(8, 120))
+        s = vals[sc]
+        mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+        x = rng.choice(mids, 16) * s * rng.choice([-1, 1], 16)
+        x[0] = 6 * s  # pins the scale at s
+        blocks.append(x.astype(np.float32))
+    for _ in range(30):  # tiny blocks: subnormal or zero scales
+        blocks.append(rng.uniform(-1, 1, 16).astype(np.float32) * np.float32(rng.uniform(0.002, 0.2)))
+    blocks.append(np.full(16, 3000.0, np.float32))  # saturating scale
+    blocks.append(np.array([-0.0, 0.0] * 8, np.float32))  # zero block, signed zeros
+    blocks.append(np.array([-1e-30] + [1.0] * 15, np.float32))  # negative to zero -> 0x8
+    return blocks
+
+
+def test_block_quantizer_vs_exact_rationals():
+    rng = np.random.default_rng(11)
+    blocks = _special_blocks(rng)
+    bits = np.stack([W.f32_to_bf16_bits(b) for b in blocks])
+    codes, scales, deq = oracle.quantize_rows(bits, len(blocks), 16, 16, 1)
+    for r, b in enumerate(bits):
+        xs = W.bf16_bits_to_f32(b)
+        want_codes, want_sc, want_deq = _fq_block_fraction(xs)
+        assert scales[r, 0] == want_sc
+        packed = [want_codes[2 * i] | (want_codes[2 * i + 1] << 4) for i in range(8)]
+        assert list(codes[r]) == packed, r
+        assert [Fraction(float(v)) for v in deq[r]] == want_deq
+
+
+def test_block_quantizer_strided_view_and_packing():
+    """A transposed view (blocks along tokens, stride D) equals quantizing the
+    explicitly transposed array; codes put element 2i in the low nibble."""
+    rng = np.random.default_rng(3)
+    L, D = 64, 32
+    x = W.f32_to_bf16_bits(rng.standard_normal((L, D)).astype(np.float32))
+    c1, s1, d1 = oracle.quantize_rows(x, D, L, 1, D)  # rows = channels, cols = tokens
+    xt = np.ascontiguousarray(x.T)
+    c2, s2, d2 = oracle.quantize_rows(xt, D, L, L, 1)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2) and np.array_equal(d1, d2)
+    lo = c1 & 0xF
+    hi = c1 >> 4
+    mag = np.array(GRID)
+    s = np.array([[oracle.e4m3_value(int(v)) for v in row] for row in s1])
+    for r in range(D):
+        for j in range(L):
+            code = lo[r, j // 2] if j % 2 == 0 else hi[r, j // 2]
+            val = mag[code & 7] * s[r, j // 16] * (-1 if code & 8 else 1)
+            assert val == d1[r, j]
+
+
+def test_sign_symmetry():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((500, 64)).astype(np.float32) * np.float32(3)
+    b = W.f32_to_bf16_bits(x)
+    nb = W.f32_to_bf16_bits(-x)
+    _, s1, d1 = oracle.quantize_rows(b, 500, 64, 64, 1)
+    _, s2, d2 = oracle.quantize_rows(nb, 500, 64, 64, 1)
+    assert np.array_equal(s1, s2)
+    assert np.array_equal(d1, -d2)
+
+
+def test_idempotence_on_normal_scales():
+    """fq(fq(x)) == fq(x) whenever the block scale is a normal E4M3 (>= 2^-6):
+    the block max then lands on code 6, so the rescale reproduces s."""
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((4000, 16)) * 10 ** rng.uniform(-1.5, 2.5, (4000, 1))
+    b = W.f32_to_bf16_bits(x.astype(np.float32))
+    _, sc, d1 = oracle.quantize_rows(b, 4000, 16, 16, 1)
+    normal = sc[:, 0] >= 8
+    assert normal.sum() > 3500
+    d2, sc2 = oracle.fq_f64_rows(d1)
+    assert np.array_equal(d2[normal], d1[normal])
+    assert np.array_equal(sc2[normal], sc[normal])
+
+
+def test_idempotence_predicted_failures_on_subnormal_scales():
+    """Single-element blocks a*[1,0,...]: with a in (3, 3.5]*2^-9 the scale is
+    2^-9 (a/6 just above half of 2^-9), the element rounds to 3*2^-9, and a
+    second pass sees a/6 = 0.5*2^-9, a tie that goes to scale 0."""
+    for a in [3.02 * 2 ** -9, 3.2 * 2 ** -9, 3.49 * 2 ** -9]:
+        x = np.zeros((1, 16))
+        x[0, 0] = a
+        b = W.f32_to_bf16_bits(x.astype(np.float32))
+        _, sc, d1 = oracle.quantize_rows(b, 1, 16, 16, 1)
+        assert sc[0, 0] == 1 and d1[0, 0] == 3 * 2 ** -9
+        d2, sc2 = oracle.fq_f64_rows(d1)
+        assert sc2[0, 0] == 0 and np.all(d2 == 0)
+
+
+# ---------------------------------------------------------- attention ------
+
+def _rand_bits(rng, shape, scale=1.0):
+    return W.f32_to_bf16_bits((rng.standard_normal(shape) * scale).astype(np.float32))
+
+
+def _f(bits):
+    return W.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def test_unquantized_forward_matches_sdpa_and_softmax():
+    rng = np.random.default_rng(21)
+    B, H, Lq, Lk, D = 1, 2, 40, 48, 32
+    q, k, v = (_rand_bits(rng, (B, H, L, D)) for L in (Lq, Lk, Lk))
+    c = 0.3
+    out = oracle.attention(q, k, v, c, flags=0)
+    qt, kt, vt = (torch.from_numpy(_f(x)) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=c).numpy()
+    assert np.max(np.abs(out["O"] - ref)) < 1e-12
+    # second formulation: explicit softmax in float64 numpy
+    S = np.einsum("bhid,bhjd->bhij", _f(q), _f(k)) * c
+    P = np.exp(S - S.max(-1, keepdims=True))
+    P /= P.sum(-1, keepdims=True)
+    assert np.allclose(P.sum(-1), 1.0, atol=1e-14)
+    assert np.max(np.abs(out["O"] - P @ _f(v))) < 1e-12
+    assert np.max(np.abs(out["m"] - S.max(-1))) < 1e-13
+    assert np.max(np.abs(np.exp(out["lse"]) - np.exp(S).sum(-1)) / np.exp(S).sum(-1)) < 1e-13
+
+
+def test_probabilities_sum_to_one():
+    """With V = 1 (unquantized) and quant_p off, O = sum_j P_ij = 1 for every
+    row.  (fq would move a block of ones to 6 * E4M3(1/6) = 1.03125.)"""
+    rng = np.random.default_rng(22)
+    q = _rand_bits(rng, (1, 1, 33, 16), 2.0)
+    k = _rand_bits(rng, (1, 1, 64, 16), 2.0)
+    v = W.f32_to_bf16_bits(np.ones((1, 1, 64, 16), np.float32))
+    out = oracle.attention(q, k, v, 0.5, flags=oracle.QUANT_Q | oracle.QUANT_K)
+    assert np.max(np.abs(out["O"] - 1.0)) < 1e-14
+    out = oracle.attention(q, k, v, 0.5, flags=oracle.QUANT_Q | oracle.QUANT_K | oracle.QUANT_V)
+    assert np.max(np.abs(out["O"] - 1.03125)) < 1e-14
+
+
+def test_identical_keys_closed_form():
+    g = json.load(open(os.path.join(GOLDEN, "identical_keys.json")))
+    rng = np.random.default_rng(23)
+    Lq, Lk, D = 20, 64, 32
+    q = _rand_bits(rng, (1, 1, Lq, D))
+    krow = _rand_bits(rng, (1, 1, 1, D))
+    k = np.repeat(krow, Lk, axis=2)
+    v = _rand_bits(rng, (1, 1, Lk, D))
+    _, _, vdeq = oracle.quantize_rows(v[0, 0], D, Lk, 1, D)  # fq(V) blocks along tokens
+    vmean = vdeq.T.mean(0)
+    out = oracle.attention(q, k, v, 0.125, flags=oracle.QUANT_ALL)
+    assert oracle.e4m3_round_div6(1.0) == g["scale_code"]
+    assert oracle.e4m3_value(g["scale_code"]) == g["scale_value"]
+    assert np.max(np.abs(out["O"][0, 0] - g["p_hat_constant"] * vmean)) < 1e-14
+    out2 = oracle.attention(q, k, v, 0.125, flags=oracle.QUANT_ALL & ~oracle.QUANT_P)
+    assert np.max(np.abs(out2["O"][0, 0] - vmean)) < 1e-14
+
+
+def test_single_block_lk16_matches_bruteforce():
+    """Lk = 16: one P block; everything written out by hand with Fractions
+    for the fq of P~ and float64 elsewhere."""
+    rng = np.random.default_rng(24)
+    Lq, Lk, D = 8, 16, 16
+    q, k, v = _rand_bits(rng, (1, 1, Lq, D)), _rand_bits(rng, (1, 1, Lk, D)), _rand_bits(rng, (1, 1, Lk, D))
+    c = 0.25
+    out = oracle.attention(q, k, v, c, flags=oracle.QUANT_ALL)
+    _, _, qd = oracle.quantize_rows(q[0, 0], Lq, D, D, 1)
+    _, _, kd = oracle.quantize_rows(k[0, 0], Lk, D, D, 1)
+    _, _, vd = oracle.quantize_rows(v[0, 0], D, Lk, 1, D)
+    vd = vd.T
+    for i in range(Lq):
+        S = np.array([c * sum(qd[i, d] * kd[j, d] for d in range(D)) for j in range(Lk)])
+        Pt = np.exp(S - S.max())
+        _, _, ph = _fq_block_fraction(Pt)
+        ph = np.array([float(x) for x in ph])
+        O = ph @ vd / Pt.sum()
+        assert np.max(np.abs(out["O"][0, 0, i] - O)) < 1e-12
+
+
+def test_ragged_lk_zero_padding_equivalence():
+    """Lk not a multiple of 16: zero-padding K/V rows to the next block and
+    masking them out gives the same O (padded keys get P~ = 0)."""
+    rng = np.random.default_rng(25)
+    Lq, Lk, D = 10, 40, 16
+    q, k, v = _rand_bits(rng, (1, 1, Lq, D)), _rand_bits(rng, (1, 1, Lk, D)), _rand_bits(rng, (1, 1, Lk, D))
+    hd = oracle.Head(q[0, 0], k[0, 0], v[0, 0], 0.3, oracle.QUANT_ALL)
+    O, lse, m, l = hd.fwd_rows()
+    # by hand with the oracle's own operands, padding to 48 with exp(-inf) = 0
+    S = hd.Qh @ hd.Kh.T * 0.3
+    Pt = np.exp(S - S.max(1, keepdims=True))
+    Ptp = np.concatenate([Pt, np.zeros((Lq, 8))], 1)
+    Ph, _ = oracle.fq_f64_rows(Ptp)
+    O2 = Ph[:, :Lk] @ hd.Vh / Pt.sum(1, keepdims=True)
+    assert np.max(np.abs(O - O2)) < 1e-13
+
+
+# ------------------------------------------------------------ gradients ----
+
+def _torch_attention_grads(q, k, v, dO, c):
+    qt, kt, vt = (torch.tensor(_f(x), requires_grad=True) for x in (q, k, v))
+    S = qt @ kt.transpose(-1, -2) * c
+    O = torch.softmax(S, -1) @ vt
+    (O * torch.tensor(_f(dO))).sum().backward()
+    return O.detach().numpy(), qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+def test_unquantized_gradients_match_autograd():
+    rng = np.random.default_rng(31)
+    Lq, Lk, D = 24, 32, 16
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for L in (Lq, Lk, Lk, Lq))
+    c = 0.4
+    out = oracle.attention(q, k, v, c, flags=0, do_bits=dO)
+    O, gq, gk, gv = _torch_attention_grads(q[0, 0], k[0, 0], v[0, 0], dO[0, 0], c)
+    for name, ref in (("dQ", gq), ("dK", gk), ("dV", gv)):
+        assert np.max(np.abs(out[name][0, 0] - ref)) < 1e-12, name
+
+
+def test_unquantized_gradients_central_differences():
+    rng = np.random.default_rng(32)
+    Lq, Lk, D = 6, 16, 8
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for L in (Lq, Lk, Lk, Lq))
+    c = 0.7
+    out = oracle.attention(q, k, v, c, flags=0, do_bits=dO)
+    base = {n: _f(x)[0, 0] for n, x in (("q", q), ("k", k), ("v", v))}
+    g = _f(dO)[0, 0]
+
+    def loss(vals):
+        S = vals["q"] @ vals["k"].T * c
+        P = np.exp(S - S.max(1, keepdims=True))
+        P /= P.sum(1, keepdims=True)
+        return float(np.sum((P @ vals["v"]) * g))
+
+    h = 1e-6
+    for name, grad in (("q", out["dQ"]), ("k", out["dK"]), ("v", out["dV"])):
+        for idx in [(0, 0), (1, 3), (3, 7)]:
+            plus = {n: a.copy() for n, a in base.items()}
+            minus = {n: a.copy() for n, a in base.items()}
+            plus[name][idx] += h
+            minus[name][idx] -= h
+            fd = (loss(plus) - loss(minus)) / (2 * h)
+            assert abs(fd - grad[0, 0][idx]) < 1e-7, (name, idx)
+
+
+def _ste_surrogate_grads(hd, q, k, v, dO, c, flags):
+    """Gradient of the straight-through surrogate by torch autograd.
+
+    The offsets d_X = fq(X0) - X0 (X in Q, K, V), d_P = fq(P~0) - P~0 and the
+    row max m0 are frozen at the base point; then
+        O(Q, K, V) = (P~ + d_P)(V + d_V) / l,  P~ = exp((Q + d_Q)(K + d_K)^T c - m0),
+        l = sum_j P~.
+    Its exact gradient is what the straight-through estimator prescribes."""
+    Q0, K0, V0 = (_f(x)[0, 0] for x in (q, k, v))
+    dQo, dKo, dVo = hd.Qh - Q0, hd.Kh - K0, hd.Vh - V0
+    S0 = hd.Qh @ hd.Kh.T * c
+    m0 = S0.max(1, keepdims=True)
+    Pt0 = np.exp(S0 - m0)
+    if flags & oracle.QUANT_P:
+        Ph0, _ = oracle.fq_f64_rows(Pt0)
+    else:
+        Ph0 = Pt0
+    dPo = Ph0 - Pt0
+    qt, kt, vt = (torch.tensor(a, requires_grad=True) for a in (Q0, K0, V0))
+    Pt = torch.exp((qt + torch.tensor(dQo)) @ (kt + torch.tensor(dKo)).T * c - torch.tensor(m0))
+    l = Pt.sum(1, keepdim=True)
+    O = (Pt + torch.tensor(dPo)) @ (vt + torch.tensor(dVo)) / l
+    (O * torch.tensor(_f(dO)[0, 0])).sum().backward()
+    return O.detach().numpy(), qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("flags", [oracle.QUANT_ALL, oracle.QUANT_Q | oracle.QUANT_K,
+                                   oracle.QUANT_V | oracle.QUANT_P])
+def test_quantized_gradients_match_ste_surrogate(flags):
+    rng = np.random.default_rng(33 + flags)
+    Lq, Lk, D = 20, 48, 32
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for L in (Lq, Lk, Lk, Lq))
+    c = 0.35
+    out = oracle.attention(q, k, v, c, flags=flags, do_bits=dO)
+    hd = oracle.Head(q[0, 0], k[0, 0], v[0, 0], c, flags, dO[0, 0])
+    O, gq, gk, gv = _ste_surrogate_grads(hd, q, k, v, dO, c, flags)
+    assert np.max(np.abs(out["O"][0, 0] - O)) < 1e-12
+    for name, ref in (("dQ", gq), ("dK", gk), ("dV", gv)):
+        err = np.max(np.abs(out[name][0, 0] - ref))
+        assert err < 1e-11, (name, err)
+
+
+def test_quantized_gradients_finite_differences_of_surrogate():
+    """Central differences of the frozen-offset surrogate (float64 numpy),
+    independent of autograd."""
+    rng = np.random.default_rng(41)
+    Lq, Lk, D = 8, 32, 16
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for L in (Lq, Lk, Lk, Lq))
+    c, flags = 0.5, oracle.QUANT_ALL
+    out = oracle.attention(q, k, v, c, flags=flags, do_bits=dO)
+    hd = oracle.Head(q[0, 0], k[0, 0], v[0, 0], c, flags, dO[0, 0])
+    Q0, K0, V0 = (_f(x)[0, 0] for x in (q, k, v))
+    off = {"q": hd.Qh - Q0, "k": hd.Kh - K0, "v": hd.Vh - V0}
+    S0 = hd.Qh @ hd.Kh.T * c
+    m0 = S0.max(1, keepdims=True)
+    Pt0 = np.exp(S0 - m0)
+    dP = oracle.fq_f64_rows(Pt0)[0] - Pt0
+    g = _f(dO)[0, 0]
+
+    def loss(vals):
+        Pt = np.exp((vals["q"] + off["q"]) @ (vals["k"] + off["k"]).T * c - m0)
+        return float(np.sum(((Pt + dP) @ (vals["v"] + off["v"]) / Pt.sum(1, keepdims=True)) * g))
+
+    base = {"q": Q0, "k": K0, "v": V0}
+    h = 1e-6
+    for name, grad in (("q", out["dQ"]), ("k", out["dK"]), ("v", out["dV"])):
+        for idx in [(0, 0), (2, 5), (7, 15)]:
+            plus = {n: a.copy() for n, a in base.items()}
+            minus = {n: a.copy() for n, a in base.items()}
+            plus[name][idx] += h
+            minus[name][idx] -= h
+            fd = (loss(plus) - loss(minus)) / (2 * h)
+            assert abs(fd - grad[0, 0][idx]) < 1e-6 * max(1.0, abs(fd)), (name, idx, fd)
+
+
+def test_dv_literal_reading_zeroes_normalised_blocks():
+    """The literal fq(P~/l) reading: with no global scale the normalised blocks
+    of a long row have amax/6 below half the smallest E4M3 subnormal, so every
+    block flushes to zero and dV vanishes (why it is not the default)."""
+    rng = np.random.default_rng(51)
+    Lq, Lk, D = 4, 4096, 16
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D), 0.1) for L in (Lq, Lk, Lk, Lq))
+    out = oracle.attention(q, k, v, 0.25, flags=oracle.QUANT_ALL | oracle.DV_QUANT_NORMALIZED,
+                           do_bits=dO)
+    assert np.all(out["dV"] == 0)
+    out2 = oracle.attention(q, k, v, 0.25, flags=oracle.QUANT_ALL, do_bits=dO)
+    assert np.max(np.abs(out2["dV"])) > 0
+    assert np.array_equal(out["dK"], out2["dK"]) and np.array_equal(out["dQ"], out2["dQ"])
+
+
+def test_sampled_rows_equal_full_computation():
+    """The row/block sampling entry points agree with the full computation."""
+    rng = np.random.default_rng(61)
+    Lq, Lk, D = 40, 64, 16
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for L in (Lq, Lk, Lk, Lq))
+    hd = oracle.Head(q[0, 0], k[0, 0], v[0, 0], 0.3, oracle.QUANT_ALL, dO[0, 0])
+    dQ, dK, dV = hd.backward()
+    rows = np.array([3, 17, 39])
+    O, lse, m, l = hd.fwd_rows(rows)
+    st = hd.stats()
+    assert np.array_equal(O, st["O"][rows])
+    assert np.array_equal(hd.dq_rows(rows), dQ[rows])
+    dKs, dVs = hd.dkdv_blocks(np.array([2]))
+    assert np.array_equal(dKs, dK[32:48]) and np.array_equal(dVs, dV[32:48])
