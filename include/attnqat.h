@@ -1,0 +1,172 @@
+/*
+ * attnqat.h -- C ABI of the B200 (sm_100a) Attn-QAT attention library.
+ *
+ * Attn-QAT training attention: non-causal multi-head attention whose operands
+ * are NVFP4 fake-quantized (fq) inside the op, with a straight-through
+ * backward.  The method and its format come from these pages:
+ *  - FastVideo "Attn-QAT Training" guide, section "Architecture-specific
+ *    Triton routing": non-causal BF16 attention, head dimension 128, query
+ *    and key/value lengths may differ (K and V share one), the optimized
+ *    backward needs a 16-aligned KV length, the backend fails loudly instead
+ *    of falling back to dense attention ("Prerequisites").
+ *  - vsqa-test-1.3b checkpoint metadata.json, "attention.precision": "NVFP4
+ *    fake-quant with BF16 matmul", quant_p and quant_v on, no global scale
+ *    (use_global_sf_p / use_global_sf_qkv false); "linear_quantization.format":
+ *    E2M1 values, 16-element blocks, E4M3 block scales.
+ *  - fastvideo-kernel triton_kernels commit (SM100 Attn-QAT route): full KV
+ *    tiles without bounds masks plus a separate masked tail tile.
+ *  - FastVideo PR #1457 review, finding F1: the softmax scale must be plumbed
+ *    end to end, never replaced by a hidden 1/sqrt(D).
+ *
+ * fq(x) on a block of 16 elements along the contraction axis of the matmul
+ * the operand feeds: s = E4M3(amax/6) (round to nearest even, saturating at
+ * 448, subnormals kept, s = 0 zeroes the block), each element becomes
+ * sign(x) * E2M1(|x|/s) * s (round to nearest even on {0,.5,1,1.5,2,3,4,6}).
+ *
+ * Forward:  S = fq(Q) fq(K)^T * sm_scale, m = exact row max of S,
+ *           P~ = exp(S - m), l = sum_j P~ (unquantized),
+ *           O = fq(P~) fq(V) / l with fq(P~) blocked along keys from key 0,
+ *           LSE = m + ln l.
+ * Backward: dV = (fq(P~)/l)^T dO, dP = dO fq(V)^T, Delta = rowsum(dO o O),
+ *           dS = P o (dP - Delta) with P = P~/l, dQ = dS fq(K) sm_scale,
+ *           dK = dS^T fq(Q) sm_scale.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors are dense, contiguous, row-major bf16 in BHSD order:
+ *    q, o, dO, dq: [B][H][Lq][D]; k, v, dk, dv: [B][H][Lk][D].  m, lse:
+ *    float32 [B][H][Lq].  All pointers are device pointers unless stated.
+ *  - The caller owns every buffer.  The library allocates no device memory and
+ *    keeps no state beyond a once-per-process setup of kernel attributes and
+ *    of the driver entry point used to encode TMA descriptors.  Inputs are
+ *    never written.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Work is enqueued asynchronously; all argument checks run on the
+ *    host before any launch.  There is no CPU fallback.
+ *  - Return value: 0 on success, else a negative ATTNQAT_E* code;
+ *    attnqat_strerror() describes it.  On ATTNQAT_ECUDA the CUDA error is
+ *    kept and returned by attnqat_last_cuda_error().
+ *  - Device-side waits are bounded.  A wait that gives up sets a device flag,
+ *    read (with a device synchronize) by attnqat_device_status().
+ */
+#ifndef ATTNQAT_H
+#define ATTNQAT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+#define ATTNQAT_OK 0
+#define ATTNQAT_EINVAL (-1)       /* null or misaligned pointer, bad shape, bad scale */
+#define ATTNQAT_EUNSUPPORTED (-2) /* device is not sm_100 (B200) or D not in {64,128} */
+#define ATTNQAT_ENOSPC (-3)       /* workspace smaller than attnqat_workspace_size() */
+#define ATTNQAT_ECUDA (-4)        /* a CUDA call or launch failed */
+#define ATTNQAT_ETIMEOUT (-5)     /* a device-side wait gave up (attnqat_device_status) */
+
+/* ---- flags: which operands are fake-quantized (vsqa-test-1.3b
+ * metadata.json, attention.precision: quant_p, quant_v; the fine attention
+ * quantizes q/k as well).  A cleared bit makes that fq the identity. ---- */
+#define ATTNQAT_QUANT_Q 1u
+#define ATTNQAT_QUANT_K 2u
+#define ATTNQAT_QUANT_V 4u
+#define ATTNQAT_QUANT_P 8u
+#define ATTNQAT_QUANT_ALL 15u
+
+/* Text for a status code (static storage). */
+const char *attnqat_strerror(int status);
+
+/* Last CUDA runtime error recorded by a failed call (cudaError_t as int). */
+int attnqat_last_cuda_error(void);
+
+/* Synchronizes the current device, then returns ATTNQAT_OK if no device-side
+ * wait of this library has timed out since the last call, else
+ * ATTNQAT_ETIMEOUT (and clears the flag). */
+int attnqat_device_status(void);
+
+/*
+ * attnqat_quantize -- standalone NVFP4 quantizer (fq of a strided bf16 view).
+ *
+ * Defined by: vsqa-test-1.3b metadata.json, "linear_quantization.format"
+ * (E2M1 values, 16-element blocks, E4M3 block scale) with the attention's
+ * "no global scale" setting (attention.precision.use_global_sf_qkv = false).
+ *
+ * View: for batch index z in [0, batch), row r in [0, rows), column j in
+ * [0, cols), the element is x[z*stride_batch + r*stride_row + j*stride_col]
+ * (strides in elements, >= 0).  Each row is quantized in blocks of 16
+ * consecutive columns; cols % 16 == 0 is required.
+ *  - Q or K ([B,H,L,D] contiguous): batch = 1, rows = B*H*L, cols = D,
+ *    strides (0, D, 1).
+ *  - V blocked along tokens: batch = B*H, rows = D, cols = Lk,
+ *    strides (Lk*D, 1, D)  (the transposed view of each head).
+ * Outputs (device, dense, caller-owned):
+ *  - codes  [batch][rows][cols/2] bytes: element 2i in the low nibble and
+ *    2i+1 in the high nibble; nibble = sign bit (bit 3, the input's sign,
+ *    also for values that round to 0) | 3-bit E2M1 magnitude code.
+ *  - scales [batch][rows][cols/16] bytes: E4M3 codes, sign bit 0.
+ *  - deq    [batch][rows][cols] bf16 (may be NULL): the dequantized values
+ *    sign * E2M1 * scale, which bf16 represents exactly.
+ * Codes and scales are bit-exact round-to-nearest-even results of the exact
+ * quotients amax/6 and |x|/s.  Inputs must be finite.
+ * Errors: EINVAL for null x/codes/scales, cols % 16 != 0, non-positive
+ * rows/cols/batch, negative strides, or sizes above 2^40 elements.
+ */
+int attnqat_quantize(const void *x, int64_t batch, int64_t rows, int64_t cols,
+                     int64_t stride_batch, int64_t stride_row,
+                     int64_t stride_col, uint8_t *codes, uint8_t *scales,
+                     void *deq, void *stream);
+
+/*
+ * attnqat_workspace_size -- bytes of device workspace attnqat_fwd and
+ * attnqat_bwd need for this shape and flag set (0 for invalid shapes).  The
+ * workspace holds the dequantized fq(Q), fq(K), fq(V) operands (bf16, plus an
+ * fp16 copy of fq(V) for the forward's P V product -- every fq'd value is
+ * exact in both), a float32 copy of O written by the forward, and the
+ * backward's Delta; every region is 256-byte aligned.
+ */
+size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D,
+                              uint32_t flags);
+
+/*
+ * attnqat_fwd -- Attn-QAT forward.
+ *
+ * Inputs q [B,H,Lq,D], k and v [B,H,Lk,D] (bf16, 16-byte aligned), softmax
+ * scale sm_scale (finite, > 0; used exactly as given -- FastVideo PR #1457
+ * review F1), flags (ATTNQAT_QUANT_*).  Outputs o [B,H,Lq,D] bf16,
+ * lse [B,H,Lq] float32 (natural-log LSE of the scaled scores), m [B,H,Lq]
+ * float32 (the exact row max of the scaled scores).  ws/ws_bytes: device
+ * workspace of at least attnqat_workspace_size(B,H,Lq,Lk,D,flags) bytes,
+ * 256-byte aligned; it must be passed unchanged to attnqat_bwd.
+ * Shapes: B, H >= 1; Lq >= 1; Lk >= 16 with Lk % 16 == 0 (the pages' SM100
+ * backward needs a 16-aligned KV length); D in {64, 128}; B*H*max(Lq,Lk)*D
+ * below 2^31.  Lq is arbitrary (the last query tile is masked); a partial
+ * last KV tile runs the separate masked tail step.
+ * Errors: EINVAL, EUNSUPPORTED (not sm_100, D unsupported), ENOSPC, ECUDA.
+ */
+int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H,
+                int Lq, int Lk, int D, float sm_scale, uint32_t flags, void *o,
+                float *lse, float *m, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * attnqat_bwd -- Attn-QAT backward (straight-through estimator).
+ *
+ * Inputs: q, k, v as given to attnqat_fwd; lse, m as it returned them;
+ * dO [B,H,Lq,D] bf16; the same shape, sm_scale and flags; ws as left by
+ * attnqat_fwd (it holds fq(Q), fq(K), fq(V) and the float32 O).  Outputs
+ * dq [B,H,Lq,D], dk and dv [B,H,Lk,D], bf16.  Delta = rowsum(dO o O) is
+ * taken from the forward's float32 O, not from the bf16 o: where a softmax
+ * row is peaked, dP - Delta cancels and would amplify the bf16 rounding of
+ * O about thirtyfold.
+ * Errors as attnqat_fwd.
+ */
+int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse,
+                const float *m, const void *dO, int B, int H, int Lq, int Lk,
+                int D, float sm_scale, uint32_t flags, void *dq, void *dk,
+                void *dv, void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ATTNQAT_H */

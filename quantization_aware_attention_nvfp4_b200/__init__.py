@@ -1,0 +1,216 @@
+"""Attn-QAT (NVFP4 fake-quantized training attention) for NVIDIA B200 (sm_100a).
+
+A thin Python binding over the C ABI of ``libattnqat.so`` (``include/attnqat.h``).
+It only marshals arguments: PyTorch supplies device memory and the current CUDA
+stream, and every step of the computation runs in the library's kernels.  There
+is no CPU or library fallback: if the library cannot be loaded or the device is
+not sm_100, the calls raise.
+
+Entry points (same names as the C ABI):
+
+* ``attnqat_quantize(x2d)`` -- NVFP4 codes, E4M3 scales and dequantized values
+  of a bf16 view, blocks of 16 along the last axis (a strided/transposed view is
+  allowed).
+* ``attnqat_fwd(q, k, v, sm_scale=None, flags=QUANT_ALL)`` -- forward; returns
+  ``(o, lse, m, ws)``.
+* ``attnqat_bwd(q, k, v, lse, m, dO, ws, sm_scale=None, flags=QUANT_ALL)`` --
+  straight-through backward; returns ``(dq, dk, dv)``.
+
+``sm_scale=None`` means 1/sqrt(D), chosen here and passed explicitly; the
+library itself never substitutes a default (FastVideo PR #1457 review, F1).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import re
+import threading
+
+from . import build as _build
+
+QUANT_Q = 1
+QUANT_K = 2
+QUANT_V = 4
+QUANT_P = 8
+QUANT_ALL = 15
+
+OK = 0
+EINVAL = -1
+EUNSUPPORTED = -2
+ENOSPC = -3
+ECUDA = -4
+ETIMEOUT = -5
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnQatError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        lib = load()
+        msg = lib.attnqat_strerror(status).decode()
+        if status == ECUDA:
+            msg += " (cudaError %d)" % lib.attnqat_last_cuda_error()
+        super().__init__("%s failed: %s [status %d]" % (what, msg, status))
+        self.status = status
+
+
+def load(build_if_needed: bool = True):
+    """Loads libattnqat.so (building it with nvcc first if it is missing or
+    stale).  Raises if it cannot be built or loaded."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build() if build_if_needed else _build.LIB
+            lib = ctypes.CDLL(path)
+            P, I, I64, U32, SZ, F = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                     ctypes.c_uint32, ctypes.c_size_t, ctypes.c_float)
+            lib.attnqat_strerror.restype = ctypes.c_char_p
+            lib.attnqat_strerror.argtypes = [I]
+            lib.attnqat_last_cuda_error.restype = I
+            lib.attnqat_last_cuda_error.argtypes = []
+            lib.attnqat_device_status.restype = I
+            lib.attnqat_device_status.argtypes = []
+            lib.attnqat_quantize.restype = I
+            lib.attnqat_quantize.argtypes = [P, I64, I64, I64, I64, I64, I64, P, P, P, P]
+            lib.attnqat_workspace_size.restype = SZ
+            lib.attnqat_workspace_size.argtypes = [I, I, I, I, I, U32]
+            lib.attnqat_fwd.restype = I
+            lib.attnqat_fwd.argtypes = [P, P, P, I, I, I, I, I, F, U32, P, P, P, P, SZ, P]
+            lib.attnqat_bwd.restype = I
+            lib.attnqat_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, U32, P, P, P, P, SZ, P]
+            _lib = lib
+    return _lib
+
+
+def header_symbols() -> list:
+    """Names of the functions include/attnqat.h declares."""
+    import os
+    text = open(os.path.join(_build.INCLUDE, "attnqat.h")).read()
+    return sorted(set(re.findall(r"\b(attnqat_[a-z0-9_]+)\s*\(", text)))
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(stream=None):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise AttnQatError(status, what)
+
+
+def _require_bf16_cuda(name, t, ndim=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != torch.bfloat16:
+        raise ValueError("%s must be bfloat16" % name)
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s must have %d dims" % (name, ndim))
+
+
+def attnqat_quantize(x, stream=None):
+    """NVFP4 fq of a 2-D (or 3-D batched) bf16 CUDA view, blocks of 16 along
+    the last axis.  Strides may be arbitrary (e.g. ``v.transpose(-1, -2)``).
+
+    Returns ``(codes uint8 [..., cols/2], scales uint8 [..., cols/16],
+    deq bf16 with x's shape and strides)``."""
+    torch = _torch()
+    _require_bf16_cuda("x", x)
+    if x.dim() == 2:
+        batch, (rows, cols) = 1, x.shape
+        sb, (sr, sc) = 0, x.stride()
+    elif x.dim() == 3:
+        batch, rows, cols = x.shape
+        sb, sr, sc = x.stride()
+    else:
+        raise ValueError("x must be 2-D or 3-D")
+    codes = torch.empty((batch, rows, cols // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((batch, rows, cols // 16), dtype=torch.uint8, device=x.device)
+    deq = torch.empty_strided(x.shape, x.stride(), dtype=torch.bfloat16, device=x.device)
+    st = load().attnqat_quantize(ctypes.c_void_p(x.data_ptr()), batch, rows, cols, sb, sr, sc,
+                                 ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                                 ctypes.c_void_p(deq.data_ptr()), _stream_ptr(stream))
+    _check(st, "attnqat_quantize")
+    if x.dim() == 2:
+        codes, scales = codes[0], scales[0]
+    return codes, scales, deq
+
+
+def attnqat_workspace_size(B, H, Lq, Lk, D, flags=QUANT_ALL) -> int:
+    return int(load().attnqat_workspace_size(B, H, Lq, Lk, D, flags))
+
+
+def _shape(q, k, v):
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _require_bf16_cuda(n, t, 4)
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous [B, H, L, D]" % n)
+    B, H, Lq, D = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[1] != H or k.shape[3] != D:
+        raise ValueError("k and v must be [B, H, Lk, D] matching q [B, H, Lq, D]")
+    return B, H, Lq, k.shape[2], D
+
+
+def attnqat_fwd(q, k, v, sm_scale=None, flags=QUANT_ALL, ws=None, out=None, stream=None):
+    """Attn-QAT forward.  Returns ``(o, lse, m, ws)``; pass ``ws`` unchanged
+    to :func:`attnqat_bwd`."""
+    torch = _torch()
+    B, H, Lq, Lk, D = _shape(q, k, v)
+    c = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    need = attnqat_workspace_size(B, H, Lq, Lk, D, flags)
+    if need == 0:
+        _check(EINVAL, "attnqat_workspace_size")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+        m = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    else:
+        o, lse, m = out
+    st = load().attnqat_fwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                            ctypes.c_void_p(v.data_ptr()), B, H, Lq, Lk, D, c, flags,
+                            ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+                            ctypes.c_void_p(m.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                            ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "attnqat_fwd")
+    return o, lse, m, ws
+
+
+def attnqat_bwd(q, k, v, lse, m, dO, ws, sm_scale=None, flags=QUANT_ALL, out=None, stream=None):
+    """Attn-QAT backward (straight-through).  ``ws`` is the workspace the
+    forward returned.  Returns ``(dq, dk, dv)``."""
+    torch = _torch()
+    B, H, Lq, Lk, D = _shape(q, k, v)
+    _require_bf16_cuda("dO", dO, 4)
+    if dO.shape != q.shape or not dO.is_contiguous():
+        raise ValueError("dO must be contiguous and shaped like q")
+    c = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    st = load().attnqat_bwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                            ctypes.c_void_p(v.data_ptr()),
+                            ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(m.data_ptr()),
+                            ctypes.c_void_p(dO.data_ptr()), B, H, Lq, Lk, D, c, flags,
+                            ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
+                            ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                            ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "attnqat_bwd")
+    return dq, dk, dv
+
+
+def attnqat_device_status() -> int:
+    """Synchronizes the device; raises if a bounded device-side wait timed out."""
+    st = load().attnqat_device_status()
+    _check(st, "attnqat_device_status")
+    return st

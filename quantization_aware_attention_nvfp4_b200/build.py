@@ -1,0 +1,61 @@
+"""Builds libattnqat.so (sm_100a) in-tree with nvcc.
+
+The library is one translation unit (csrc/libattnqat.cu includes the kernel
+sources) linked against the shared CUDA runtime, so it shares the runtime
+that PyTorch loads in the same process.
+"""
+from __future__ import annotations
+
+import glob
+import os
+import shutil
+import subprocess
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libattnqat.so")
+ARCH = "-gencode=arch=compute_100a,code=sm_100a"
+
+
+def _nvcc() -> str:
+    cand = [os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc"),
+            shutil.which("nvcc") or ""]
+    for c in cand:
+        if c and os.path.exists(c):
+            return c
+    raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libattnqat.so")
+
+
+def sources() -> list:
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+                  + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
+
+
+def stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    return any(os.path.getmtime(s) > t for s in sources())
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile the library if it is missing or older than its sources."""
+    if not force and not stale():
+        return LIB
+    cuda_home = os.path.dirname(os.path.dirname(_nvcc()))
+    tmp = LIB + ".tmp%d" % os.getpid()
+    cmd = [_nvcc(), "-shared", "-Xcompiler", "-fPIC", "-O3", "-lineinfo", "-std=c++17", ARCH,
+           "-I" + INCLUDE, "-cudart", "shared",
+           "-Xlinker", "-rpath," + os.path.join(cuda_home, "lib64"),
+           "-o", tmp, os.path.join(CSRC, "libattnqat.cu")]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    subprocess.check_call(cmd)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force=True, verbose=True))

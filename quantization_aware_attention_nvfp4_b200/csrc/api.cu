@@ -1,0 +1,330 @@
+// api.cu -- the extern "C" boundary of libattnqat (declared in attnqat.h):
+// host-side validation, workspace layout, TMA descriptor encoding and kernel
+// launches.  Every step of the computation runs in the kernels of this
+// library; there is no host or library fallback.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "attnqat.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace attnqat {
+
+static thread_local int g_last_cuda_error = 0;
+
+static int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return ATTNQAT_ECUDA;
+}
+
+cudaError_t ensure_smem_attr(const void *kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void *>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({dev, kernel})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert({dev, kernel});
+  return e;
+}
+
+// ----------------------------------------------------------- device check --
+
+static int check_device() {
+  static std::mutex mu;
+  static int verdict[64];  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return ATTNQAT_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (verdict[dev] == 0) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    verdict[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return verdict[dev] == 1 ? ATTNQAT_OK : ATTNQAT_EUNSUPPORTED;
+}
+
+// ------------------------------------------------------------ TMA encode --
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encoder() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a [BH][L][D] tensor of 16-bit elements, 64 x 128 boxes
+// (128 bytes x 128 rows), 128-byte swizzle; rows past L read as zeros.
+static bool encode_bhld(CUtensorMap *map, const void *base, int BH, int L, int D, bool f16) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- workspace --
+
+struct Workspace {
+  size_t qh, kh, vh, vh16, o32, delta, stats, total;
+};
+
+// fq(Q) and fq(K) are exact in fp16 (values sign * E2M1 * E4M3 lie in
+// [2^-10, 2688] with at most 7 significant bits), so when both are quantized
+// they are kept as fp16 and S = fq(Q) fq(K)^T, dQ and dK run as fp16 MMAs,
+// which lets the backward feed dS as fp16 (3 more mantissa bits than bf16).
+static bool qk_f16(uint32_t flags) {
+  return (flags & ATTNQAT_QUANT_Q) && (flags & ATTNQAT_QUANT_K);
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
+  Workspace w{};
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t qbytes = BH * Lq * D * 2, kbytes = BH * Lk * D * 2;
+  size_t off = 0;
+  w.qh = off;
+  if (flags & ATTNQAT_QUANT_Q) off = align256(off + qbytes);
+  w.kh = off;
+  if (flags & ATTNQAT_QUANT_K) off = align256(off + kbytes);
+  w.vh = off;
+  if (flags & ATTNQAT_QUANT_V) off = align256(off + kbytes);
+  w.vh16 = off;
+  if (flags & ATTNQAT_QUANT_V) off = align256(off + kbytes);
+  w.o32 = off;
+  off = align256(off + BH * Lq * D * 4);
+  w.delta = off;
+  off = align256(off + BH * Lq * 4);
+  w.stats = off;  // [0] max_i |dO_i|_1, [1] max_i |Delta_i|, [2] max |fq(V)|
+  off = align256(off + 16);
+  w.total = off;
+  return w;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_shape(int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags) {
+  if (B < 1 || H < 1 || Lq < 1 || Lk < 16 || (Lk % 16) != 0) return ATTNQAT_EINVAL;
+  if (static_cast<int64_t>(B) * H > 65535) return ATTNQAT_EINVAL;  // grid.y
+  const int64_t Lmax = Lq > Lk ? Lq : Lk;
+  if (static_cast<int64_t>(B) * H * Lmax * 128 >= (int64_t(1) << 40)) return ATTNQAT_EINVAL;
+  if (!(std::isfinite(sm_scale) && sm_scale > 0.0f)) return ATTNQAT_EINVAL;
+  if (flags & ~ATTNQAT_QUANT_ALL) return ATTNQAT_EINVAL;
+  if (D != 64 && D != 128) return ATTNQAT_EUNSUPPORTED;
+  return ATTNQAT_OK;
+}
+
+// Writes fq(Q), fq(K), fq(V) into the workspace (as the flags ask) and
+// returns the operand pointers the attention kernels read.
+static int prepare_operands(const void *q, const void *k, const void *v, int B, int H, int Lq, int Lk,
+                            int D, uint32_t flags, uint8_t *ws, const Workspace &w,
+                            cudaStream_t stream) {
+  const int64_t BH = static_cast<int64_t>(B) * H;
+  const bool f16 = qk_f16(flags);
+  float *stats = reinterpret_cast<float *>(ws + w.stats);
+  cudaError_t e = cudaMemsetAsync(stats, 0, 16, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (flags & ATTNQAT_QUANT_Q) {
+    uint16_t *dst = reinterpret_cast<uint16_t *>(ws + w.qh);
+    e = launch_quantize(static_cast<const uint16_t *>(q), 1, BH * Lq, D, 0, D, 1, nullptr, nullptr,
+                        f16 ? nullptr : dst, f16 ? dst : nullptr, nullptr, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (flags & ATTNQAT_QUANT_K) {
+    uint16_t *dst = reinterpret_cast<uint16_t *>(ws + w.kh);
+    e = launch_quantize(static_cast<const uint16_t *>(k), 1, BH * Lk, D, 0, D, 1, nullptr, nullptr,
+                        f16 ? nullptr : dst, f16 ? dst : nullptr, nullptr, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (flags & ATTNQAT_QUANT_V) {
+    // blocks of 16 consecutive tokens per channel: the transposed view
+    e = launch_quantize(static_cast<const uint16_t *>(v), BH, D, Lk, static_cast<int64_t>(Lk) * D, 1, D,
+                        nullptr, nullptr, reinterpret_cast<uint16_t *>(ws + w.vh),
+                        reinterpret_cast<uint16_t *>(ws + w.vh16), stats + 2, stream);
+  } else {
+    e = launch_absmax(static_cast<const __nv_bfloat16 *>(v), BH * Lk * D, stats + 2, stream);
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ATTNQAT_OK;
+}
+
+}  // namespace attnqat
+
+using namespace attnqat;
+
+extern "C" {
+
+const char *attnqat_strerror(int status) {
+  switch (status) {
+    case ATTNQAT_OK: return "success";
+    case ATTNQAT_EINVAL: return "invalid argument (null or misaligned pointer, bad shape or scale)";
+    case ATTNQAT_EUNSUPPORTED: return "unsupported (device is not sm_100 or head dimension not 64/128)";
+    case ATTNQAT_ENOSPC: return "workspace too small";
+    case ATTNQAT_ECUDA: return "CUDA error (see attnqat_last_cuda_error)";
+    case ATTNQAT_ETIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int attnqat_last_cuda_error(void) { return g_last_cuda_error; }
+
+int attnqat_device_status(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof v);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (v == 0) return ATTNQAT_OK;
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return ATTNQAT_ETIMEOUT;
+}
+
+int attnqat_quantize(const void *x, int64_t batch, int64_t rows, int64_t cols, int64_t stride_batch,
+                     int64_t stride_row, int64_t stride_col, uint8_t *codes, uint8_t *scales, void *deq,
+                     void *stream) {
+  if (!x || !codes || !scales) return ATTNQAT_EINVAL;
+  if (batch < 1 || rows < 1 || cols < 16 || (cols % 16) != 0) return ATTNQAT_EINVAL;
+  if (stride_batch < 0 || stride_row < 0 || stride_col < 0) return ATTNQAT_EINVAL;
+  const int64_t lim = int64_t(1) << 40;
+  if (batch > lim || rows > lim || cols > lim || batch * rows > lim / cols) return ATTNQAT_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) & 1u) || (deq && (reinterpret_cast<uintptr_t>(deq) & 1u)))
+    return ATTNQAT_EINVAL;
+  const int st = check_device();
+  if (st != ATTNQAT_OK) return st;
+  cudaError_t e = launch_quantize(static_cast<const uint16_t *>(x), batch, rows, cols, stride_batch,
+                                  stride_row, stride_col, codes, scales, static_cast<uint16_t *>(deq),
+                                  nullptr, nullptr, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
+}
+
+size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
+  if (check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
+  return layout(B, H, Lq, Lk, D, flags).total;
+}
+
+int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int Lq, int Lk, int D,
+                float sm_scale, uint32_t flags, void *o, float *lse, float *m, void *ws, size_t ws_bytes,
+                void *stream) {
+  int st = check_shape(B, H, Lq, Lk, D, sm_scale, flags);
+  if (st != ATTNQAT_OK) return st;
+  if (!q || !k || !v || !o || !lse || !m || !ws) return ATTNQAT_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(m) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return ATTNQAT_EINVAL;
+  const Workspace w = layout(B, H, Lq, Lk, D, flags);
+  if (ws_bytes < w.total) return ATTNQAT_ENOSPC;
+  st = check_device();
+  if (st != ATTNQAT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  st = prepare_operands(q, k, v, B, H, Lq, Lk, D, flags, wsb, w, s);
+  if (st != ATTNQAT_OK) return st;
+  const int BH = B * H;
+  const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
+  const void *kh = (flags & ATTNQAT_QUANT_K) ? static_cast<const void *>(wsb + w.kh) : k;
+  const bool pv_f16 = (flags & ATTNQAT_QUANT_V) != 0;
+  const void *vh = pv_f16 ? static_cast<const void *>(wsb + w.vh16) : v;
+  const bool f16 = qk_f16(flags);
+  CUtensorMap tq, tk, tv;
+  if (!encode_bhld(&tq, qh, BH, Lq, D, f16) || !encode_bhld(&tk, kh, BH, Lk, D, f16) ||
+      !encode_bhld(&tv, vh, BH, Lk, D, pv_f16))
+    return cuda_fail(cudaErrorInvalidValue);
+  FwdArgs a;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.nq_tiles = (Lq + kBM - 1) / kBM;
+  a.nk_tiles = (Lk + kBN - 1) / kBN;
+  a.sm_scale = sm_scale;
+  a.scale_log2 = sm_scale * kLog2e;
+  a.o = static_cast<__nv_bfloat16 *>(o);
+  a.o32 = reinterpret_cast<float *>(wsb + w.o32);
+  a.lse = lse;
+  a.m = m;
+  cudaError_t e = launch_fwd(D, f16, pv_f16, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, a, BH, s);
+  return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
+}
+
+int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, const float *m, const void *dO,
+                int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags, void *dq, void *dk, void *dv,
+                void *ws, size_t ws_bytes, void *stream) {
+  int st = check_shape(B, H, Lq, Lk, D, sm_scale, flags);
+  if (st != ATTNQAT_OK) return st;
+  if (!q || !k || !v || !lse || !m || !dO || !dq || !dk || !dv || !ws) return ATTNQAT_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(lse) || !aligned16(m) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return ATTNQAT_EINVAL;
+  const Workspace w = layout(B, H, Lq, Lk, D, flags);
+  if (ws_bytes < w.total) return ATTNQAT_ENOSPC;
+  st = check_device();
+  if (st != ATTNQAT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  const int BH = B * H;
+  float *delta = reinterpret_cast<float *>(wsb + w.delta);
+  float *stats = reinterpret_cast<float *>(wsb + w.stats);
+  cudaError_t e = cudaMemsetAsync(stats, 0, 8, s);  // keeps stats[2] from the forward
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_delta(reinterpret_cast<const float *>(wsb + w.o32), static_cast<const __nv_bfloat16 *>(dO), delta,
+                   static_cast<int64_t>(BH) * Lq, D, stats, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const bool f16 = qk_f16(flags);
+  const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
+  const void *kh = (flags & ATTNQAT_QUANT_K) ? static_cast<const void *>(wsb + w.kh) : k;
+  const void *vh = (flags & ATTNQAT_QUANT_V) ? static_cast<const void *>(wsb + w.vh) : v;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bhld(&tq, qh, BH, Lq, D, f16) || !encode_bhld(&tk, kh, BH, Lk, D, f16) ||
+      !encode_bhld(&tv, vh, BH, Lk, D, false) || !encode_bhld(&tdo, dO, BH, Lq, D, false))
+    return cuda_fail(cudaErrorInvalidValue);
+  BwdArgs a;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.nq_tiles = (Lq + kBM - 1) / kBM;
+  a.nk_tiles = (Lk + kBN - 1) / kBN;
+  a.sm_scale = sm_scale;
+  a.scale_log2 = sm_scale * kLog2e;
+  a.m = m;
+  a.lse = lse;
+  a.delta = delta;
+  a.stats = stats;
+  a.dq = static_cast<__nv_bfloat16 *>(dq);
+  a.dk = static_cast<__nv_bfloat16 *>(dk);
+  a.dv = static_cast<__nv_bfloat16 *>(dv);
+  e = launch_bwd_dkdv(D, f16, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, tdo, a, BH, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_bwd_dq(D, f16, tq, tk, tv, tdo, a, BH, s);
+  return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,577 @@
+// bwd.cu -- Attn-QAT backward kernels for sm_100a (straight-through
+// estimator: every fq is the identity for the gradient).
+//
+//   dK/dV kernel: one CTA per (128-key tile, batch*head), looping over query
+//     tiles.  Per query tile: S = fq(Q) fq(K)^T and dP = dO fq(V)^T into TMEM;
+//     one thread per query row rebuilds P~ = exp(S - m) and fq(P~) exactly as
+//     the forward does (same bits, same blocks of 16 keys), forms
+//     (fq(P~)/l)^T and dS^T = (P o (dP - Delta))^T in shared memory, and the
+//     tensor cores accumulate dV += (fq(P~)/l)^T dO and dK += dS^T fq(Q) in
+//     TMEM.
+//   dQ kernel: one CTA per (128-query tile, batch*head), looping over key
+//     tiles: S, dP as above, dS = P o (dP - Delta) with P = exp(S - LSE),
+//     dQ += dS fq(K).
+//
+// The split into a dK/dV and a dQ kernel follows the fastvideo-kernel
+// triton_kernels commit (SM100 Attn-QAT route: separate dQ and dK/dV tiles);
+// the tiles here are 128 x 128 tcgen05 tiles with TMEM accumulators.
+// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 2..5
+// one thread per query row (TMEM lane).
+#include "common.cuh"
+#include "internal.h"
+
+namespace attnqat {
+
+template <int D>
+struct DkdvLayout {
+  static constexpr int kTile = Tile<D>::kBytes;
+  static constexpr int kXBytes = kBM * kBN * 2;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTile;
+  static constexpr int kQ = kV + kTile;          // 2 stages
+  static constexpr int kDO = kQ + 2 * kTile;     // 2 stages
+  static constexpr int kX = kDO + 2 * kTile;     // P^T, then dS^T
+  static constexpr int kBar = kX + kXBytes;
+  static constexpr int kBytes = kBar + 256;
+  static constexpr int kDynSmem = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDV = 256, kTmemDK = 256 + D;
+};
+
+struct BwdBars {
+  uint64_t kvfull;
+  uint64_t afull[2], aempty[2];   // Q tiles (dK/dV kernel) or K tiles (dQ kernel)
+  uint64_t bfull[2], bempty[2];   // dO tiles (dK/dV kernel) or V tiles (dQ kernel)
+  uint64_t sfull, sempty;   // S and dP in TMEM: filled together, released together
+  uint64_t xfull, xempty;
+  uint64_t done;
+  uint32_t tmem_slot;
+  int abort;
+};
+
+__device__ __forceinline__ void init_bwd_bars(BwdBars *b) {
+  mbar_init(&b->kvfull, 1);
+  for (int s = 0; s < 2; ++s) {
+    mbar_init(&b->afull[s], 1);
+    mbar_init(&b->aempty[s], 1);
+    mbar_init(&b->bfull[s], 1);
+    mbar_init(&b->bempty[s], 1);
+  }
+  mbar_init(&b->sfull, 1);
+  mbar_init(&b->sempty, 4);
+  mbar_init(&b->xfull, 4);
+  mbar_init(&b->xempty, 1);
+  mbar_init(&b->done, 1);
+  b->abort = 0;
+  fence_mbar_init();
+}
+
+// Loads one 128-row x D tile (D/64 swizzled chunks) with TMA.
+template <int D>
+__device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int row0,
+                                          int bh) {
+  for (int c = 0; c < Tile<D>::kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, map, bar, c * 64, row0, bh);
+}
+
+// ----------------------------------------------------------- dK / dV ------
+
+// Power-of-two scale for the f16 dS operand: 2^e with e chosen so that the
+// bound |dS| <= max_i|dO_i|_1 * max|fq(V)| + max_i|Delta_i| maps to at most
+// 2^14 (fp16 max is 65504); the float range of dS below that keeps full fp16
+// precision over 29 binades.  Returns 1 for the bf16 path or a zero bound.
+template <int QKF16>
+__device__ __forceinline__ float ds_scale(const float *stats) {
+  if (!QKF16) return 1.0f;
+  const float bound = fmaf(stats[0], stats[2], stats[1]);
+  if (!(bound > 0.0f)) return 1.0f;
+  int e = 14 - (static_cast<int>((__float_as_uint(bound) >> 23) & 0xFF) - 127) - 1;
+  e = e < -120 ? -120 : (e > 120 ? 120 : e);
+  return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+}
+
+template <int QKF16>
+__device__ __forceinline__ uint32_t pack_ds(float a, float b) {
+  return QKF16 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
+}
+
+// One query tile for one row of the dK/dV kernel, 32 keys at a time: S and
+// dP from TMEM, P~ = exp(S - m) and fq(P~)/l (bf16, a row of the transposed
+// dV operand), and dS = (P~/l)(dP - Delta) in float32, scaled by dsc and
+// packed for the dK operand.  P never leaves float32.
+template <int QP, int QKF16, bool MASKED>
+__device__ __forceinline__ void dkdv_tile(uint32_t tS, uint32_t tDP, int valid_k, bool vq, float cl, float nml,
+                                          float inv_l, float delta, float dsc, uint32_t (&pw)[64],
+                                          uint32_t (&dsw)[64]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tS + c * 32, r);
+    tmem_ld_wait();
+    float p[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float e = ex2_approx(fmaf(__uint_as_float(r[i]), cl, nml));
+      p[i] = (vq && (!MASKED || c * 32 + i < valid_k)) ? e : 0.0f;
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      if (QP) {
+        uint32_t rr[8];
+        const float s = fq16_probs(p + 16 * b, rr);
+        const float f = s * inv_l;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 g = unpack_f16x2(rr[i]);
+          pw[16 * c + 8 * b + i] = pack_bf16x2(g.x * f, g.y * f);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          pw[16 * c + 8 * b + i] = pack_bf16x2(p[16 * b + 2 * i] * inv_l, p[16 * b + 2 * i + 1] * inv_l);
+      }
+    }
+    tmem_ld32(tDP + c * 32, r);
+    tmem_ld_wait();
+    const float pf = inv_l * dsc;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float d0 = p[2 * i] * pf * (__uint_as_float(r[2 * i]) - delta);
+      const float d1 = p[2 * i + 1] * pf * (__uint_as_float(r[2 * i + 1]) - delta);
+      dsw[16 * c + i] = pack_ds<QKF16>(d0, d1);
+    }
+  }
+}
+
+template <int D, int QP, int QKF16>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                         const BwdArgs a) {
+  using L = DkdvLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  BwdBars *bars = reinterpret_cast<BwdBars *>(smem + L::kBar);
+  volatile int *abort = &bars->abort;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kt = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int nq = a.nq_tiles;
+
+  if (threadIdx.x == 0) init_bwd_bars(bars);
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmDO);
+      mbar_arrive_expect_tx(&bars->kvfull, 2 * L::kTile);
+      load_tile<D>(smem + L::kK, &tmK, &bars->kvfull, kt * kBN, bh);
+      load_tile<D>(smem + L::kV, &tmV, &bars->kvfull, kt * kBN, bh);
+      int issued = 0;
+      for (int i = 0; i < nq; ++i) {
+        const int st = i & 1;
+        if (i >= 2 && !mbar_wait(&bars->aempty[st], ((i >> 1) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
+        load_tile<D>(smem + L::kQ + st * L::kTile, &tmQ, &bars->afull[st], i * kBM, bh);
+        if (i >= 2 && !mbar_wait(&bars->bempty[st], ((i >> 1) - 1) & 1, abort)) {
+          issued = i + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars->bfull[st], L::kTile);
+        load_tile<D>(smem + L::kDO + st * L::kTile, &tmDO, &bars->bfull[st], i * kBM, bh);
+        issued = i + 1;
+      }
+      if (*abort) {
+        mbar_wait_drain(&bars->kvfull, 0);
+        for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) {
+          mbar_wait_drain(&bars->afull[i & 1], (i >> 1) & 1);
+          mbar_wait_drain(&bars->bfull[i & 1], (i >> 1) & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(kBM, kBN, !QKF16, false, false);   // Q K^T
+      constexpr uint32_t idDP = idesc_f16(kBM, kBN, true, false, false);    // dO V^T (bf16)
+      constexpr uint32_t idV = idesc_f16(kBN, D, true, true, true);         // P^T dO (bf16)
+      constexpr uint32_t idK = idesc_f16(kBN, D, !QKF16, true, true);       // dS^T Q
+      const uint32_t kaddr = sbase + L::kK, vaddr = sbase + L::kV, xaddr = sbase + L::kX;
+      bool ok = mbar_wait(&bars->kvfull, 0, abort);
+      // S_i and dP_i into TMEM; one commit signals both
+      auto issue_sdp = [&](int i) -> bool {
+        if (!mbar_wait(&bars->afull[i & 1], (i >> 1) & 1, abort)) return false;
+        if (!mbar_wait(&bars->bfull[i & 1], (i >> 1) & 1, abort)) return false;
+        tc_fence_after();
+        mma_kmajor(tmem + L::kTmemS, sbase + L::kQ + (i & 1) * L::kTile, kaddr, D / 16, idS, false);
+        mma_kmajor(tmem + L::kTmemDP, sbase + L::kDO + (i & 1) * L::kTile, vaddr, D / 16, idDP, false);
+        umma_commit(&bars->sfull);
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      for (int i = 0; ok && i < nq; ++i) {
+        const int st = i & 1;
+        if (i + 1 < nq) {
+          ok = mbar_wait(&bars->sempty, i & 1, abort) && issue_sdp(i + 1);
+          if (!ok) break;
+        }
+        // dV += (fq(P~)/l)^T dO_i : A = X (M = keys, MN-major), B = dO (N = D, MN-major)
+        if (!mbar_wait(&bars->xfull, (2 * i) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        mma_mn_mn(tmem + L::kTmemDV, xaddr, sbase + L::kDO + st * L::kTile, kBM / 16, idV, i > 0);
+        umma_commit(&bars->xempty);
+        umma_commit(&bars->bempty[st]);
+        // dK += dS^T Q_i
+        if (!mbar_wait(&bars->xfull, (2 * i + 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        mma_mn_mn(tmem + L::kTmemDK, xaddr, sbase + L::kQ + st * L::kTile, kBM / 16, idK, i > 0);
+        umma_commit(&bars->xempty);
+        umma_commit(&bars->aempty[st]);
+      }
+      umma_commit(&bars->done);
+    }
+  } else {
+    const int wq = warp & 3;
+    const uint32_t row = static_cast<uint32_t>(wq * 32 + lane);
+    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const int valid_k = a.Lk - kt * kBN;  // >= 128 for full key tiles
+    const float cl = a.scale_log2;
+    const float dsc = ds_scale<QKF16>(a.stats);
+    const uint32_t xaddr = sbase + L::kX;
+    bool ok = true;
+    for (int i = 0; i < nq; ++i) {
+      const int qg = i * kBM + static_cast<int>(row);
+      const bool vq = qg < a.Lq;
+      const size_t si = static_cast<size_t>(bh) * a.Lq + (vq ? qg : 0);
+      const float m = vq ? a.m[si] : 0.0f;
+      const float lse = vq ? a.lse[si] : 0.0f;
+      const float delta = vq ? a.delta[si] : 0.0f;
+      const float nml = -(m * kLog2e);
+      const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
+      uint32_t pw[64], dsw[64];
+      if (!mbar_wait(&bars->sfull, i & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      if (valid_k < kBN)
+        dkdv_tile<QP, QKF16, true>(tmem + lane_addr + L::kTmemS, tmem + lane_addr + L::kTmemDP, valid_k, vq,
+                                   cl, nml, inv_l, delta, dsc, pw, dsw);
+      else
+        dkdv_tile<QP, QKF16, false>(tmem + lane_addr + L::kTmemS, tmem + lane_addr + L::kTmemDP, valid_k, vq,
+                                    cl, nml, inv_l, delta, dsc, pw, dsw);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->sempty);
+      if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
+      store_row128(xaddr, row, pw);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->xfull);
+      if (!mbar_wait(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
+      store_row128(xaddr, row, dsw);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->xfull);
+    }
+    if (ok && mbar_wait(&bars->done, 0, abort)) {
+      tc_fence_after();
+      const int kg = kt * kBN + static_cast<int>(row);
+      const size_t rowoff = (static_cast<size_t>(bh) * a.Lk + kg) * D;
+      const float kscale = a.sm_scale / ds_scale<QKF16>(a.stats);  // exact: power-of-two divisor
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32], s[32];
+        tmem_ld32(tmem + lane_addr + L::kTmemDV + c * 32, r);
+        tmem_ld32(tmem + lane_addr + L::kTmemDK + c * 32, s);
+        tmem_ld_wait();
+        if (kg < a.Lk) {
+          uint4 *dv = reinterpret_cast<uint4 *>(a.dv + rowoff + c * 32);
+          uint4 *dk = reinterpret_cast<uint4 *>(a.dk + rowoff + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4], x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              w[k] = pack_bf16x2(__uint_as_float(r[8 * i + 2 * k]), __uint_as_float(r[8 * i + 2 * k + 1]));
+              x[k] = pack_bf16x2(__uint_as_float(s[8 * i + 2 * k]) * kscale,
+                                 __uint_as_float(s[8 * i + 2 * k + 1]) * kscale);
+            }
+            dv[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            dk[i] = make_uint4(x[0], x[1], x[2], x[3]);
+          }
+        }
+      }
+    } else {
+      mbar_wait_drain(&bars->done, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------- dQ -----
+
+template <int D>
+struct DqLayout {
+  static constexpr int kTile = Tile<D>::kBytes;
+  static constexpr int kXBytes = kBM * kBN * 2;
+  static constexpr int kQ = 0;
+  static constexpr int kDO = kQ + kTile;
+  static constexpr int kK = kDO + kTile;        // 2 stages
+  static constexpr int kV = kK + 2 * kTile;     // 2 stages
+  static constexpr int kX = kV + 2 * kTile;     // dS
+  static constexpr int kBar = kX + kXBytes;
+  static constexpr int kBytes = kBar + 256;
+  static constexpr int kDynSmem = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDQ = 256;
+};
+
+// One key tile for one row of the dQ kernel, 32 keys at a time:
+// P = exp(S - LSE) in float32 and dS = P (dP - Delta), scaled by dsc and
+// packed for the dQ operand.
+template <int QKF16, bool MASKED>
+__device__ __forceinline__ void dq_tile(uint32_t tS, uint32_t tDP, int valid_k, bool vq, float cl, float nlse,
+                                        float delta, float dsc, uint32_t (&dsw)[64]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r[32], d[32];
+    tmem_ld32(tS + c * 32, r);
+    tmem_ld32(tDP + c * 32, d);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * i]), cl, nlse));
+      float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), cl, nlse));
+      if (!vq || (MASKED && c * 32 + 2 * i >= valid_k)) p0 = 0.0f;
+      if (!vq || (MASKED && c * 32 + 2 * i + 1 >= valid_k)) p1 = 0.0f;
+      dsw[16 * c + i] = pack_ds<QKF16>(p0 * dsc * (__uint_as_float(d[2 * i]) - delta),
+                                       p1 * dsc * (__uint_as_float(d[2 * i + 1]) - delta));
+    }
+  }
+}
+
+template <int D, int QKF16>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                       const BwdArgs a) {
+  using L = DqLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  BwdBars *bars = reinterpret_cast<BwdBars *>(smem + L::kBar);
+  volatile int *abort = &bars->abort;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qt = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int nk = a.nk_tiles;
+
+  if (threadIdx.x == 0) init_bwd_bars(bars);
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmDO);
+      mbar_arrive_expect_tx(&bars->kvfull, 2 * L::kTile);
+      load_tile<D>(smem + L::kQ, &tmQ, &bars->kvfull, qt * kBM, bh);
+      load_tile<D>(smem + L::kDO, &tmDO, &bars->kvfull, qt * kBM, bh);
+      int issued = 0;
+      for (int j = 0; j < nk; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait(&bars->aempty[st], ((j >> 1) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
+        load_tile<D>(smem + L::kK + st * L::kTile, &tmK, &bars->afull[st], j * kBN, bh);
+        if (j >= 2 && !mbar_wait(&bars->bempty[st], ((j >> 1) - 1) & 1, abort)) {
+          issued = j + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars->bfull[st], L::kTile);
+        load_tile<D>(smem + L::kV + st * L::kTile, &tmV, &bars->bfull[st], j * kBN, bh);
+        issued = j + 1;
+      }
+      if (*abort) {
+        mbar_wait_drain(&bars->kvfull, 0);
+        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
+          mbar_wait_drain(&bars->afull[j & 1], (j >> 1) & 1);
+          mbar_wait_drain(&bars->bfull[j & 1], (j >> 1) & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(kBM, kBN, !QKF16, false, false);  // Q K^T
+      constexpr uint32_t idDP = idesc_f16(kBM, kBN, true, false, false);   // dO V^T
+      constexpr uint32_t idQ = idesc_f16(kBM, D, !QKF16, false, true);     // dS (K-major) * K (MN-major)
+      const uint32_t qaddr = sbase + L::kQ, doaddr = sbase + L::kDO, xaddr = sbase + L::kX;
+      bool ok = mbar_wait(&bars->kvfull, 0, abort);
+      auto issue_sdp = [&](int j) -> bool {
+        if (!mbar_wait(&bars->afull[j & 1], (j >> 1) & 1, abort)) return false;
+        if (!mbar_wait(&bars->bfull[j & 1], (j >> 1) & 1, abort)) return false;
+        tc_fence_after();
+        mma_kmajor(tmem + L::kTmemS, qaddr, sbase + L::kK + (j & 1) * L::kTile, D / 16, idS, false);
+        mma_kmajor(tmem + L::kTmemDP, doaddr, sbase + L::kV + (j & 1) * L::kTile, D / 16, idDP, false);
+        umma_commit(&bars->bempty[j & 1]);
+        umma_commit(&bars->sfull);
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      for (int j = 0; ok && j < nk; ++j) {
+        if (j + 1 < nk) {
+          ok = mbar_wait(&bars->sempty, j & 1, abort) && issue_sdp(j + 1);
+          if (!ok) break;
+        }
+        if (!mbar_wait(&bars->xfull, j & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        mma_a_k_b_mn(tmem + L::kTmemDQ, xaddr, sbase + L::kK + (j & 1) * L::kTile, kBN / 16, idQ, j > 0);
+        umma_commit(&bars->xempty);
+        umma_commit(&bars->aempty[j & 1]);
+      }
+      umma_commit(&bars->done);
+    }
+  } else {
+    const int wq = warp & 3;
+    const uint32_t row = static_cast<uint32_t>(wq * 32 + lane);
+    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const int q = qt * kBM + static_cast<int>(row);
+    const bool vq = q < a.Lq;
+    const size_t si = static_cast<size_t>(bh) * a.Lq + (vq ? q : 0);
+    const float lse = vq ? a.lse[si] : 0.0f;
+    const float delta = vq ? a.delta[si] : 0.0f;
+    const float nlse = -(lse * kLog2e);
+    const float cl = a.scale_log2;
+    const float dsc = ds_scale<QKF16>(a.stats);
+    const int last_valid = a.Lk - (nk - 1) * kBN;
+    const uint32_t xaddr = sbase + L::kX;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      uint32_t dsw[64];
+      if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      if (j == nk - 1 && last_valid < kBN)
+        dq_tile<QKF16, true>(tmem + lane_addr + L::kTmemS, tmem + lane_addr + L::kTmemDP, last_valid, vq, cl,
+                             nlse, delta, dsc, dsw);
+      else
+        dq_tile<QKF16, false>(tmem + lane_addr + L::kTmemS, tmem + lane_addr + L::kTmemDP, kBN, vq, cl, nlse,
+                              delta, dsc, dsw);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->sempty);
+      if (j >= 1 && !mbar_wait(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
+      store_row128(xaddr, row, dsw);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->xfull);
+    }
+    if (ok && mbar_wait(&bars->done, 0, abort)) {
+      tc_fence_after();
+      const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
+      const float qscale = a.sm_scale / dsc;  // exact: power-of-two divisor
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + L::kTmemDQ + c * 32, r);
+        tmem_ld_wait();
+        if (vq) {
+          uint4 *dst = reinterpret_cast<uint4 *>(a.dq + rowoff + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              w[k] = pack_bf16x2(__uint_as_float(r[8 * i + 2 * k]) * qscale,
+                                 __uint_as_float(r[8 * i + 2 * k + 1]) * qscale);
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    } else {
+      mbar_wait_drain(&bars->done, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------- launchers --
+
+template <int D, int QP, int QKF16>
+static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                 const CUtensorMap &tdo, const BwdArgs &a, int BH, cudaStream_t stream) {
+  using L = DkdvLayout<D>;
+  auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16>;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(a.nk_tiles, BH), 192, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t dkdv_dispatch(bool qk_f16, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+                                 const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
+                                 cudaStream_t stream) {
+  if (qk_f16)
+    return quant_p ? launch_dkdv_t<D, 1, 1>(tq, tk, tv, tdo, a, BH, stream)
+                   : launch_dkdv_t<D, 0, 1>(tq, tk, tv, tdo, a, BH, stream);
+  return quant_p ? launch_dkdv_t<D, 1, 0>(tq, tk, tv, tdo, a, BH, stream)
+                 : launch_dkdv_t<D, 0, 0>(tq, tk, tv, tdo, a, BH, stream);
+}
+
+cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+                            const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
+                            cudaStream_t stream) {
+  return D == 128 ? dkdv_dispatch<128>(qk_f16, quant_p, tq, tk, tv, tdo, a, BH, stream)
+                  : dkdv_dispatch<64>(qk_f16, quant_p, tq, tk, tv, tdo, a, BH, stream);
+}
+
+template <int D, int QKF16>
+static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                               const CUtensorMap &tdo, const BwdArgs &a, int BH, cudaStream_t stream) {
+  using L = DqLayout<D>;
+  auto kern = attn_bwd_dq_kernel<D, QKF16>;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(a.nq_tiles, BH), 192, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dq(int D, bool qk_f16, const CUtensorMap &tq, const CUtensorMap &tk,
+                          const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
+                          cudaStream_t stream) {
+  if (D == 128)
+    return qk_f16 ? launch_dq_t<128, 1>(tq, tk, tv, tdo, a, BH, stream)
+                  : launch_dq_t<128, 0>(tq, tk, tv, tdo, a, BH, stream);
+  return qk_f16 ? launch_dq_t<64, 1>(tq, tk, tv, tdo, a, BH, stream)
+                : launch_dq_t<64, 0>(tq, tk, tv, tdo, a, BH, stream);
+}
+
+}  // namespace attnqat

@@ -1,0 +1,109 @@
+// common.cuh -- tile geometry, the in-register NVFP4 fake quantization of
+// probability blocks, and small GEMM-issue helpers shared by the forward and
+// backward attention kernels.
+#pragma once
+
+#include "device.cuh"
+
+namespace attnqat {
+
+constexpr int kBM = 128;                  // query rows per tile (TMEM lanes)
+constexpr int kBN = 128;                  // keys per tile
+constexpr int kChunkBytes = 128 * 128;    // one 128-row x 128-byte swizzled chunk
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Bytes of a 128-row x D tile of 16-bit elements (D/64 swizzled chunks).
+template <int D>
+struct Tile {
+  static constexpr int kBytes = 128 * D * 2;
+  static constexpr int kChunks = D / 64;
+};
+
+// fq of one block of 16 non-negative probabilities held in registers (one
+// query row, 16 consecutive keys): s = E4M3(amax/6), each element rounded to
+// the E2M1 grid of p/s (round to nearest even, saturating at 6).  Returns the
+// 8 f16x2 words of r (the grid values, sign-free) and the block scale s as a
+// float.  With s == 0 every r is 0.
+//
+// amax/6 is formed as amax * (1/6) and p/s as p * rcp(s): for probabilities
+// (exp of a float) exact ties have measure zero, so this selects the same
+// codes as the exact quotients except within one float ulp of a rounding
+// boundary.  Forward and backward use this same routine on the same bits, so
+// they agree bit for bit.
+__device__ __forceinline__ float fq16_probs(const float *p, uint32_t (&r)[8]) {
+  float amax = fmaxf(fmaxf(fmaxf(p[0], p[1]), fmaxf(p[2], p[3])),
+                     fmaxf(fmaxf(p[4], p[5]), fmaxf(p[6], p[7])));
+  amax = fmaxf(amax, fmaxf(fmaxf(fmaxf(p[8], p[9]), fmaxf(p[10], p[11])),
+                           fmaxf(fmaxf(p[12], p[13]), fmaxf(p[14], p[15]))));
+  const uint16_t code = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.0f);
+  const float s = unpack_f16x2(cvt_f16x2_from_e4m3x2(code)).x;
+  const float inv = s > 0.0f ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r[i] = e2m1_round_f16x2(p[2 * i] * inv, p[2 * i + 1] * inv);
+  return s;
+}
+
+// f16x2 word with the f16 value of s (an E4M3 value, exact in f16) in both
+// halves.
+__device__ __forceinline__ uint32_t f16x2_broadcast(float s) {
+  const uint32_t h = __half_as_ushort(__float2half_rn(s));
+  return h | (h << 16);
+}
+
+// Issues D[tmem] (+)= A * B^T for two K-major 128-row tiles (128-byte swizzle,
+// chunks of 64 K-elements kChunkBytes apart) over `ksteps` slices of K = 16.
+__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
+                                           int ksteps, uint32_t idesc, bool accumulate) {
+  for (int kk = 0; kk < ksteps; ++kk) {
+    const uint32_t off = static_cast<uint32_t>(kk >> 2) * kChunkBytes + static_cast<uint32_t>(kk & 3) * 32u;
+    umma_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
+            idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Issues D[tmem] (+)= A * B where A is a K-major 128-row tile and B an
+// MN-major tile (K rows of 128 bytes, N in chunks of 64 elements kChunkBytes
+// apart), K = 16 * ksteps.
+__device__ __forceinline__ void mma_a_k_b_mn(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
+                                             int ksteps, uint32_t idesc, bool accumulate) {
+  for (int kk = 0; kk < ksteps; ++kk) {
+    const uint32_t aoff = static_cast<uint32_t>(kk >> 2) * kChunkBytes + static_cast<uint32_t>(kk & 3) * 32u;
+    const uint32_t boff = static_cast<uint32_t>(kk) * 2048u;
+    umma_ss(d_tmem, sdesc_sw128(a_base + aoff, 16, 1024),
+            sdesc_sw128(b_base + boff, kChunkBytes, 1024), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Issues D[tmem] (+)= A * B where both are MN-major tiles (K rows of 128
+// bytes; M and N in chunks of 64 elements kChunkBytes apart).
+__device__ __forceinline__ void mma_mn_mn(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
+                                          int ksteps, uint32_t idesc, bool accumulate) {
+  for (int kk = 0; kk < ksteps; ++kk) {
+    const uint32_t off = static_cast<uint32_t>(kk) * 2048u;
+    umma_ss(d_tmem, sdesc_sw128(a_base + off, kChunkBytes, 1024),
+            sdesc_sw128(b_base + off, kChunkBytes, 1024), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Writes 128 16-bit values (64 packed words, element 2i in the low half of
+// w[i]) as row `row` of a 128 x 128 swizzled tile at `base` (two chunks of 64
+// elements).  Conflict-free when the 32 lanes of a warp write 32 consecutive
+// rows.
+__device__ __forceinline__ void store_row128(uint32_t base, uint32_t row, const uint32_t *w) {
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const uint32_t addr = base + static_cast<uint32_t>(u >> 3) * kChunkBytes + sw128_offset(row, u & 7);
+    st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+  }
+}
+
+// Advances a dynamic shared-memory pointer to the next 1024-byte boundary of
+// the shared window (the swizzle atoms and UMMA descriptors need it).
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+  const uint32_t pad = (1024u - (smem_u32(p) & 1023u)) & 1023u;
+  return p + pad;
+}
+
+}  // namespace attnqat

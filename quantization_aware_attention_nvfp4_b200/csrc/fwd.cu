@@ -1,0 +1,369 @@
+// fwd.cu -- Attn-QAT forward kernel for sm_100a.
+//
+// One CTA per (128-query tile, batch*head).  192 threads in three roles:
+//   warp 0      TMA producer: the fq(Q) tile once, then fq(K) tiles for the
+//               row-max sweep and fq(K), fq(V) tiles for the output sweep
+//               (2-stage rings, 128-byte swizzle);
+//   warp 1      TMEM owner and single-thread tcgen05.mma issuer;
+//   warps 2..5  one thread per query row (TMEM lane): row max, exp, row sum,
+//               in-register NVFP4 fq of P~ in 16-key blocks, the P tile to
+//               shared memory, and the O epilogue.
+// TMEM columns: S double buffer [0,256), O accumulator [256, 256+D).
+//
+// The row max is exact over all keys, taken in a first sweep of S = Q K^T,
+// so fq(P~) sees the reference-order statistics and O needs no rescaling
+// (FastVideo "Attn-QAT Training" guide, "Architecture-specific Triton
+// routing": FWD_EXACT_M recomputes reference-order softmax statistics).  Full
+// KV tiles run without bounds masks; the partial last KV tile runs a
+// separate masked step (fastvideo-kernel triton_kernels commit, SM100
+// Attn-QAT route).
+#include "common.cuh"
+#include "internal.h"
+
+namespace attnqat {
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kNS = 2;                         // K and V ring stages
+  static constexpr int kTile = Tile<D>::kBytes;
+  static constexpr int kPBytes = kBM * kBN * 2;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTile;
+  static constexpr int kV = kK + kNS * kTile;
+  static constexpr int kP = kV + kNS * kTile;
+  static constexpr int kBar = kP + 2 * kPBytes;
+  static constexpr int kBytes = kBar + 256;
+  static constexpr int kDynSmem = kBytes + 1024;        // slack for 1024-byte alignment
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemO = 256;
+};
+
+struct FwdBars {
+  uint64_t qfull;
+  uint64_t kfull[2], kempty[2], vfull[2], vempty[2];
+  uint64_t sfull[2], sempty[2], pfull[2], pempty[2];
+  uint64_t ofull;
+  uint32_t tmem_slot;
+  int abort;
+};
+
+// One S tile of one row: 128 fp32 values in 4 chunks of 32 TMEM columns.
+template <bool MASKED>
+__device__ __forceinline__ float row_max_tile(uint32_t taddr, int valid) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (MASKED && c * 32 >= valid) break;
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float v = __uint_as_float(r[i]);
+      if (!MASKED || c * 32 + i < valid) mx = fmaxf(mx, v);
+    }
+  }
+  return mx;
+}
+
+// Sweep-2 work for one S tile of one row: P~ = exp2(S*cl + nml), row sum,
+// fq(P~) (or P~ itself), packed into 16-bit pairs and stored as row `row`
+// of the P tile at `pbase`.
+template <int PV_F16, int QP, bool MASKED>
+__device__ __forceinline__ float prob_tile(uint32_t taddr, int valid, float cl, float nml,
+                                           uint32_t pbase, uint32_t row) {
+  float lsum = 0.0f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_ld_wait();
+    float p[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float e = ex2_approx(fmaf(__uint_as_float(r[i]), cl, nml));
+      p[i] = (!MASKED || c * 32 + i < valid) ? e : 0.0f;
+      lsum += p[i];
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      if (QP) {
+        uint32_t rr[8];
+        const float s = fq16_probs(p + 16 * b, rr);
+        if (PV_F16) {
+          const uint32_t s2 = f16x2_broadcast(s);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[8 * b + i] = hmul2_u32(rr[i], s2);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float2 g = unpack_f16x2(rr[i]);
+            w[8 * b + i] = pack_bf16x2(g.x * s, g.y * s);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          w[8 * b + i] = PV_F16 ? pack_f16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1])
+                                : pack_bf16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1]);
+      }
+    }
+    // 32 keys = units 4c .. 4c+3 of the 128-key row
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int unit = 4 * c + u;
+      const uint32_t addr = pbase + static_cast<uint32_t>(unit >> 3) * kChunkBytes + sw128_offset(row, unit & 7);
+      st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+    }
+  }
+  return lsum;
+}
+
+template <int D, int QKF16, int PV_F16, int QP>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+  using L = FwdLayout<D>;
+  constexpr int kNS = L::kNS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  FwdBars *bars = reinterpret_cast<FwdBars *>(smem + L::kBar);
+  volatile int *abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qt = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int nk = a.nk_tiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->qfull, 1);
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&bars->kfull[s], 1);
+      mbar_init(&bars->kempty[s], 1);
+      mbar_init(&bars->vfull[s], 1);
+      mbar_init(&bars->vempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->sfull[b], 1);
+      mbar_init(&bars->sempty[b], 4);
+      mbar_init(&bars->pfull[b], 4);
+      mbar_init(&bars->pempty[b], 1);
+    }
+    mbar_init(&bars->ofull, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(&bars->qfull, L::kTile);
+      for (int c = 0; c < Tile<D>::kChunks; ++c)
+        tma_load_3d(smem + L::kQ + c * kChunkBytes, &tmQ, &bars->qfull, c * 64, qt * kBM, bh);
+      int kissued = 0, vissued = 0;
+      for (int t = 0; t < 2 * nk; ++t) {
+        const int j = t < nk ? t : t - nk;
+        const int st = t % kNS;
+        if (t >= kNS && !mbar_wait(&bars->kempty[st], ((t / kNS) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->kfull[st], L::kTile);
+        for (int c = 0; c < Tile<D>::kChunks; ++c)
+          tma_load_3d(smem + L::kK + st * L::kTile + c * kChunkBytes, &tmK, &bars->kfull[st], c * 64,
+                      j * kBN, bh);
+        kissued = t + 1;
+        if (t >= nk) {
+          const int u = t - nk;
+          const int vs = u % kNS;
+          if (u >= kNS && !mbar_wait(&bars->vempty[vs], ((u / kNS) - 1) & 1, abort)) break;
+          mbar_arrive_expect_tx(&bars->vfull[vs], L::kTile);
+          for (int c = 0; c < Tile<D>::kChunks; ++c)
+            tma_load_3d(smem + L::kV + vs * L::kTile + c * kChunkBytes, &tmV, &bars->vfull[vs],
+                        c * 64, j * kBN, bh);
+          vissued = u + 1;
+        }
+      }
+      if (*abort) {
+        // let the copies already issued land before the CTA exits
+        for (int t = (kissued > kNS ? kissued - kNS : 0); t < kissued; ++t)
+          mbar_wait_drain(&bars->kfull[t % kNS], (t / kNS) & 1);
+        for (int u = (vissued > kNS ? vissued - kNS : 0); u < vissued; ++u)
+          mbar_wait_drain(&bars->vfull[u % kNS], (u / kNS) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA --
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(kBM, kBN, !QKF16, false, false);
+      constexpr uint32_t idPV = idesc_f16(kBM, D, !PV_F16, false, true);
+      const uint32_t qaddr = sbase + L::kQ;
+      bool ok = mbar_wait(&bars->qfull, 0, abort);
+      int nS = 0;  // S tiles issued so far (both sweeps)
+      auto issue_s = [&](int t) -> bool {
+        const int st = t % kNS;
+        const int sb = nS & 1;
+        if (nS >= 2 && !mbar_wait(&bars->sempty[sb], ((nS >> 1) - 1) & 1, abort)) return false;
+        if (!mbar_wait(&bars->kfull[st], (t / kNS) & 1, abort)) return false;
+        tc_fence_after();
+        mma_kmajor(tmem + sb * kBN, qaddr, sbase + L::kK + st * L::kTile, D / 16, idS, false);
+        umma_commit(&bars->kempty[st]);
+        umma_commit(&bars->sfull[sb]);
+        ++nS;
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int pb = j & 1;
+        const int vs = j % kNS;
+        if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, abort)) return false;
+        if (!mbar_wait(&bars->vfull[vs], (j / kNS) & 1, abort)) return false;
+        tc_fence_after();
+        mma_a_k_b_mn(tmem + L::kTmemO, sbase + L::kP + pb * L::kPBytes,
+                     sbase + L::kV + vs * L::kTile, kBN / 16, idPV, j > 0);
+        umma_commit(&bars->vempty[vs]);
+        umma_commit(&bars->pempty[pb]);
+        return true;
+      };
+      for (int j = 0; ok && j < nk; ++j) ok = issue_s(j);
+      for (int j = 0; ok && j < nk; ++j) {
+        ok = issue_s(nk + j);
+        if (ok && j >= 1) ok = issue_pv(j - 1);
+      }
+      if (ok) ok = issue_pv(nk - 1);
+      // ofull also tracks completion of everything issued above, so the
+      // epilogue and the TMEM release never race an MMA in flight
+      umma_commit(&bars->ofull);
+    }
+  } else {
+    // ------------------------------------------------------- softmax rows --
+    const int wq = warp & 3;
+    const uint32_t row = static_cast<uint32_t>(wq * 32 + lane);
+    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const int last_valid = a.Lk - (nk - 1) * kBN;  // keys in the last KV tile
+    float mrow = -INFINITY;
+    bool ok = true;
+    int nS = 0;
+    for (int j = 0; j < nk; ++j, ++nS) {
+      const int sb = nS & 1;
+      if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem + lane_addr + sb * kBN;
+      const float mx = (j == nk - 1 && last_valid < kBN) ? row_max_tile<true>(taddr, last_valid)
+                                                         : row_max_tile<false>(taddr, kBN);
+      mrow = fmaxf(mrow, mx);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->sempty[sb]);
+    }
+    const float m_scaled = mrow * a.sm_scale;
+    const float nml = -(m_scaled * kLog2e);
+    const float cl = a.scale_log2;
+    float lsum = 0.0f;
+    for (int j = 0; ok && j < nk; ++j, ++nS) {
+      const int sb = nS & 1;
+      const int pb = j & 1;
+      if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
+      if (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem + lane_addr + sb * kBN;
+      const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
+      if (j == nk - 1 && last_valid < kBN)
+        lsum += prob_tile<PV_F16, QP, true>(taddr, last_valid, cl, nml, pbase, row);
+      else
+        lsum += prob_tile<PV_F16, QP, false>(taddr, kBN, cl, nml, pbase, row);
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->sempty[sb]);
+        mbar_arrive(&bars->pfull[pb]);
+      }
+    }
+    // ------------------------------------------------------------ epilogue --
+    if (ok && mbar_wait(&bars->ofull, 0, abort)) {
+      tc_fence_after();
+      const int q = qt * kBM + static_cast<int>(row);
+      const float inv_l = 1.0f / lsum;
+      const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + L::kTmemO + c * 32, r);
+        tmem_ld_wait();
+        if (q < a.Lq) {
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]) * inv_l;
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+          uint4 *dst = reinterpret_cast<uint4 *>(a.o + rowoff + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          float4 *d32 = reinterpret_cast<float4 *>(a.o32 + rowoff + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) d32[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+        }
+      }
+      if (q < a.Lq) {
+        a.m[static_cast<size_t>(bh) * a.Lq + q] = m_scaled;
+        a.lse[static_cast<size_t>(bh) * a.Lq + q] = m_scaled + logf(lsum);
+      }
+    } else if (!ok || *abort) {
+      // keep the MMA issuer's final commit from outliving the CTA
+      mbar_wait_drain(&bars->ofull, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+template <int D, int QKF16, int PV_F16, int QP>
+static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                const FwdArgs &a, int BH, cudaStream_t stream) {
+  using L = FwdLayout<D>;
+  auto kern = attn_fwd_kernel<D, QKF16, PV_F16, QP>;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.nq_tiles, BH);
+  kern<<<grid, 192, L::kDynSmem, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+template <int D, int QKF16>
+static cudaError_t fwd_dispatch(bool pv_f16, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+                                const CUtensorMap &tv, const FwdArgs &a, int BH, cudaStream_t stream) {
+  if (pv_f16)
+    return quant_p ? launch_fwd_t<D, QKF16, 1, 1>(tq, tk, tv, a, BH, stream)
+                   : launch_fwd_t<D, QKF16, 1, 0>(tq, tk, tv, a, BH, stream);
+  return quant_p ? launch_fwd_t<D, QKF16, 0, 1>(tq, tk, tv, a, BH, stream)
+                 : launch_fwd_t<D, QKF16, 0, 0>(tq, tk, tv, a, BH, stream);
+}
+
+cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUtensorMap &tq,
+                       const CUtensorMap &tk, const CUtensorMap &tv, const FwdArgs &a, int BH,
+                       cudaStream_t stream) {
+  if (D == 128)
+    return qk_f16 ? fwd_dispatch<128, 1>(pv_f16, quant_p, tq, tk, tv, a, BH, stream)
+                  : fwd_dispatch<128, 0>(pv_f16, quant_p, tq, tk, tv, a, BH, stream);
+  return qk_f16 ? fwd_dispatch<64, 1>(pv_f16, quant_p, tq, tk, tv, a, BH, stream)
+                : fwd_dispatch<64, 0>(pv_f16, quant_p, tq, tk, tv, a, BH, stream);
+}
+
+}  // namespace attnqat

@@ -1,0 +1,75 @@
+// internal.h -- host-side interfaces between the C-ABI layer and the kernel
+// translation units.  Not installed; not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace attnqat {
+
+struct FwdArgs {
+  int Lq, Lk, nq_tiles, nk_tiles;
+  float sm_scale;     // c
+  float scale_log2;   // c * log2(e)
+  __nv_bfloat16 *o;
+  float *o32;   // float32 copy of O kept in the workspace for the backward's Delta
+  float *lse;
+  float *m;
+};
+
+struct BwdArgs {
+  int Lq, Lk, nq_tiles, nk_tiles;
+  float sm_scale;
+  float scale_log2;
+  // stats[0] = max_i |dO_i|_1, stats[1] = max_i |Delta_i|, stats[2] = max |fq(V)|:
+  // they bound |dS| and fix the power-of-two scale of the f16 dS operand.
+  const float *stats;
+  const float *m;
+  const float *lse;
+  const float *delta;
+  __nv_bfloat16 *dq;
+  __nv_bfloat16 *dk;
+  __nv_bfloat16 *dv;
+};
+
+// Forward.  tq/tk/tv: 3-D TMA maps {D, L, B*H} with 64 x 128 boxes, 128-byte
+// swizzle, over fq(Q), fq(K) (fp16 when qk_f16, else bf16) and fq(V) (fp16
+// when pv_f16, else bf16).
+cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUtensorMap &tq,
+                       const CUtensorMap &tk, const CUtensorMap &tv, const FwdArgs &a, int BH,
+                       cudaStream_t stream);
+
+// Backward dK/dV kernel (one CTA per 128-key tile) and dQ kernel (one CTA per
+// 128-query tile).  Maps over fq(Q), fq(K) (fp16 when qk_f16, else bf16),
+// fq(V) and dO (bf16).  With qk_f16 the dS operand is fp16 (scaled by a power
+// of two), else bf16.
+cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, const CUtensorMap &tq,
+                            const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
+                            const BwdArgs &a, int BH, cudaStream_t stream);
+cudaError_t launch_bwd_dq(int D, bool qk_f16, const CUtensorMap &tq, const CUtensorMap &tk,
+                          const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
+                          cudaStream_t stream);
+
+// NVFP4 fq of a strided bf16 view (see attnqat_quantize); any of codes,
+// scales, deq (bf16, same strides as x), deq_f16 and absmax (max |fq(x)|,
+// folded in with an atomic max; must start at 0) may be null.
+cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols,
+                            int64_t sb, int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales,
+                            uint16_t *deq, uint16_t *deq_f16, float *absmax, cudaStream_t stream);
+
+// delta[r] = sum_d dO[r][d] * O[r][d] over `rows` rows of D values (O float32,
+// dO bf16); folds max_r |dO_r|_1 into stats[0] and max_r |delta_r| into
+// stats[1] (both must start at 0).
+cudaError_t launch_delta(const float *o32, const __nv_bfloat16 *dO, float *delta, int64_t rows, int D,
+                         float *stats, cudaStream_t stream);
+
+// max |x| over n bf16 values folded into *out (must start at 0).
+cudaError_t launch_absmax(const __nv_bfloat16 *x, int64_t n, float *out, cudaStream_t stream);
+
+// Sets cudaFuncAttributeMaxDynamicSharedMemorySize for `kernel` once per
+// device (thread-safe).
+cudaError_t ensure_smem_attr(const void *kernel, int bytes);
+
+}  // namespace attnqat

@@ -1,0 +1,285 @@
+// quant.cu -- NVFP4 fake quantization of bf16 operands (HBM-bound) and the
+// backward's Delta = rowsum(dO o O) kernel.
+//
+// Format (vsqa-test-1.3b metadata.json, "linear_quantization.format" and
+// "attention.precision" with no global scale): blocks of 16 consecutive
+// elements along the contraction axis, scale s = E4M3(amax/6), element
+// code = E2M1(|x|/s), both rounded to nearest, ties to even.
+//
+// Exactness: amax/6 is formed with a correctly rounded float division and
+// then rounded to E4M3 once.  For bf16 amax (8 significant bits) the exact
+// quotient is either representable (then nothing is lost) or lies further
+// than 2^-16 relative from every E4M3 rounding midpoint, so the double
+// rounding cannot move it across one.  The E2M1 code is chosen by comparing
+// |x| with the products m_k * s at the 7 midpoints m_k of the grid, which
+// are exact in float (at most 7 significant bits), so ties are detected
+// exactly and resolved to the even code.
+#include "common.cuh"
+#include "internal.h"
+
+namespace attnqat {
+
+__device__ __forceinline__ uint32_t e4m3_scale_code(float amax) {
+  const float t = __fdiv_rn(amax, 6.0f);
+  return cvt_e4m3x2(t, 0.0f) & 0xFFu;
+}
+
+// E2M1 magnitude code of |x| at scale s > 0 (round to nearest even,
+// saturating at 6).  Crossing midpoint k (between codes k and k+1) needs '>'
+// when k is even and '>=' when k is odd.
+__device__ __forceinline__ uint32_t e2m1_code_exact(float ax, float s) {
+  uint32_t c = 0;
+  c += ax > 0.25f * s;
+  c += ax >= 0.75f * s;
+  c += ax > 1.25f * s;
+  c += ax >= 1.75f * s;
+  c += ax > 2.5f * s;
+  c += ax >= 3.5f * s;
+  c += ax > 5.0f * s;
+  return c;
+}
+
+// Magnitude of E2M1 code c (0..7): 0, .5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_magnitude(uint32_t c) {
+  const float fc = static_cast<float>(c);
+  return c < 4 ? 0.5f * fc : (c < 6 ? fc - 2.0f : 2.0f * fc - 8.0f);
+}
+
+// fq of 16 bf16 values (bit patterns in v[]): packed nibbles (element 2i in
+// the low nibble of byte i, 8 bytes as two words), the scale code, and the
+// dequantized values as bf16 and f16 bit patterns.  sign * E2M1 * s has at
+// most 7 significant bits and lies in [2^-10, 2688] when nonzero, so the
+// float product and both 16-bit forms are exact.
+__device__ __forceinline__ void fq16_exact(const uint16_t (&v)[16], uint32_t (&nib)[2], uint32_t &scode,
+                                           uint16_t (&deq_bf16)[16], uint16_t (&deq_f16)[16]) {
+  float ax[16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    ax[i] = fabsf(__uint_as_float(static_cast<uint32_t>(v[i]) << 16));
+    amax = fmaxf(amax, ax[i]);
+  }
+  scode = e4m3_scale_code(amax);
+  const uint32_t s_h2 = cvt_f16x2_from_e4m3x2(static_cast<uint16_t>(scode | (scode << 8)));
+  const float s = unpack_f16x2(s_h2).x;
+  nib[0] = nib[1] = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t c = s > 0.0f ? e2m1_code_exact(ax[i], s) : 0u;
+    const uint32_t sign = static_cast<uint32_t>(v[i]) & 0x8000u;
+    nib[i >> 3] |= (c | (sign >> 12)) << (4 * (i & 7));
+    const float mag = e2m1_magnitude(c) * s;
+    const uint32_t f = __float_as_uint(mag) | (sign << 16);
+    deq_bf16[i] = static_cast<uint16_t>(f >> 16);
+    deq_f16[i] = __half_as_ushort(__float2half_rn(__uint_as_float(f)));
+  }
+}
+
+// Max-reduces a non-negative float over the CTA and folds it into *dst with
+// one atomic (non-negative floats order like their bit patterns).
+__device__ __forceinline__ void block_max_to_global(float v, float *dst) {
+  __shared__ float red[32];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < static_cast<int>(blockDim.x >> 5) ? red[lane] : 0.0f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+    if (lane == 0 && v > 0.0f) atomicMax(reinterpret_cast<unsigned int *>(dst), __float_as_uint(v));
+  }
+}
+
+// Stores 16 16-bit values at dst[base + i*sc] (two 16-byte stores when
+// contiguous and aligned).
+__device__ __forceinline__ void store16(uint16_t *dst, int64_t base, int64_t sc, const uint16_t (&h)[16]) {
+  if (sc == 1 && (reinterpret_cast<uintptr_t>(dst + base) & 15u) == 0) {
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = h[2 * i] | (static_cast<uint32_t>(h[2 * i + 1]) << 16);
+    uint4 *p = reinterpret_cast<uint4 *>(dst + base);
+    p[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    p[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) dst[base + i * sc] = h[i];
+  }
+}
+
+// One thread per 16-element block.  ROW_FASTEST selects which index varies
+// fastest across threads: the block index along cols (contiguous rows, e.g.
+// Q/K blocks along D) or the row index (e.g. V blocks along tokens, where
+// neighbouring channels are contiguous).
+template <bool ROW_FASTEST>
+__global__ void __launch_bounds__(256)
+    quantize_view_kernel(const uint16_t *__restrict__ x, int64_t batch, int64_t rows, int64_t cols,
+                         int64_t sb, int64_t sr, int64_t sc, uint8_t *__restrict__ codes,
+                         uint8_t *__restrict__ scales, uint16_t *__restrict__ deq,
+                         uint16_t *__restrict__ deq_f16, float *__restrict__ absmax) {
+  const int64_t nblk = cols / 16;
+  float vmax = 0.0f;  // largest dequantized magnitude this thread produced
+  const int64_t total = batch * rows * nblk;
+  for (int64_t id = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; id < total;
+       id += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t z, r, b;
+    if (ROW_FASTEST) {
+      r = id % rows;
+      const int64_t t = id / rows;
+      b = t % nblk;
+      z = t / nblk;
+    } else {
+      b = id % nblk;
+      const int64_t t = id / nblk;
+      r = t % rows;
+      z = t / rows;
+    }
+    const int64_t base = z * sb + r * sr + b * 16 * sc;
+    uint16_t v[16];
+    const bool vec = (sc == 1) && ((reinterpret_cast<uintptr_t>(x + base) & 15u) == 0);
+    if (vec) {
+      const uint4 *p = reinterpret_cast<const uint4 *>(x + base);
+      const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = static_cast<uint16_t>(w[i] & 0xFFFFu);
+        v[2 * i + 1] = static_cast<uint16_t>(w[i] >> 16);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = __ldg(x + base + i * sc);
+    }
+    uint32_t nib[2], scode;
+    uint16_t bb[16], hb[16];
+    fq16_exact(v, nib, scode, bb, hb);
+    const int64_t blk = (z * rows + r) * nblk + b;
+    if (codes) *reinterpret_cast<uint2 *>(codes + blk * 8) = make_uint2(nib[0], nib[1]);
+    if (scales) scales[blk] = static_cast<uint8_t>(scode);
+    if (deq) store16(deq, base, sc, bb);
+    if (deq_f16) store16(deq_f16, base, sc, hb);
+    if (absmax) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) vmax = fmaxf(vmax, fabsf(__uint_as_float(static_cast<uint32_t>(bb[i]) << 16)));
+    }
+  }
+  if (absmax) block_max_to_global(vmax, absmax);
+}
+
+cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols, int64_t sb,
+                            int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales, uint16_t *deq,
+                            uint16_t *deq_f16, float *absmax, cudaStream_t stream) {
+  const int64_t total = batch * rows * (cols / 16);
+  if (total == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;  // grid-stride beyond 8 CTAs per SM
+  if (blocks > cap) blocks = cap;
+  const bool row_fastest = (sc != 1) && (sr == 1);
+  if (row_fastest)
+    quantize_view_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax);
+  else
+    quantize_view_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ Delta --
+
+// Delta = rowsum(dO o O) with D/8 lanes per row (each lane reads 8 float32
+// of O and 8 bf16 of dO); grid-stride over rows.  Also folds the largest
+// row L1 norm of dO and the largest |Delta| into stats[0], stats[1]: with
+// max |fq(V)| they bound |dS| = P |dP - Delta| <= |dO_i|_1 max|fq(V)| + |Delta_i|,
+// which fixes the power-of-two scale of the backward's f16 dS operand.
+template <int D>
+__global__ void __launch_bounds__(256)
+    delta_kernel(const float4 *__restrict__ o32, const uint4 *__restrict__ dO, float *__restrict__ delta,
+                 int64_t rows, float *__restrict__ stats) {
+  constexpr int kLanes = D / 8;
+  float dmax = 0.0f, gmax = 0.0f;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x / kLanes;
+  for (int64_t row = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) / kLanes;
+       row - ((threadIdx.x & 31) / kLanes) < rows; row += step) {
+    const int sub = static_cast<int>(threadIdx.x % kLanes);
+    float acc = 0.0f, l1 = 0.0f;
+    if (row < rows) {
+      const float4 a0 = __ldg(o32 + (row * kLanes + sub) * 2);
+      const float4 a1 = __ldg(o32 + (row * kLanes + sub) * 2 + 1);
+      const uint4 b = __ldg(dO + row * kLanes + sub);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(bw[i] << 16), hi = __uint_as_float(bw[i] & 0xFFFF0000u);
+        acc = fmaf(av[2 * i], lo, acc);
+        acc = fmaf(av[2 * i + 1], hi, acc);
+        l1 += fabsf(lo) + fabsf(hi);
+      }
+    }
+#pragma unroll
+    for (int off = kLanes / 2; off > 0; off >>= 1) {
+      acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+      l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, off);
+    }
+    if (row < rows) {
+      if (sub == 0) delta[row] = acc;
+      dmax = fmaxf(dmax, l1);
+      gmax = fmaxf(gmax, fabsf(acc));
+    }
+  }
+  block_max_to_global(dmax, stats);
+  block_max_to_global(gmax, stats + 1);
+}
+
+cudaError_t launch_delta(const float *o32, const __nv_bfloat16 *dO, float *delta, int64_t rows, int D,
+                         float *stats, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int threads = 256;
+  const int64_t need = (rows * (D / 8) + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  const unsigned blocks = static_cast<unsigned>(need < cap ? need : cap);
+  if (D == 128)
+    delta_kernel<128><<<blocks, threads, 0, stream>>>(reinterpret_cast<const float4 *>(o32),
+                                                      reinterpret_cast<const uint4 *>(dO), delta, rows, stats);
+  else
+    delta_kernel<64><<<blocks, threads, 0, stream>>>(reinterpret_cast<const float4 *>(o32),
+                                                     reinterpret_cast<const uint4 *>(dO), delta, rows, stats);
+  return cudaGetLastError();
+}
+
+// max |x| over n bf16 values folded into *out (used for V when it is not
+// quantized, so the forward did not record max |fq(V)|).
+__global__ void __launch_bounds__(256) absmax_kernel(const uint4 *__restrict__ x, int64_t n8, float *out) {
+  float m = 0.0f;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 u = __ldg(x + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[k] << 16)), fabsf(__uint_as_float(w[k] & 0xFFFF0000u))));
+  }
+  block_max_to_global(m, out);
+}
+
+cudaError_t launch_absmax(const __nv_bfloat16 *x, int64_t n, float *out, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t n8 = n / 8;  // n is a multiple of 8 (D is 64 or 128)
+  const int64_t need = (n8 + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  absmax_kernel<<<static_cast<unsigned>(need < cap ? need : cap), 256, 0, stream>>>(
+      reinterpret_cast<const uint4 *>(x), n8, out);
+  return cudaGetLastError();
+}
+
+}  // namespace attnqat

@@ -1,0 +1,103 @@
+"""Bit-exact parity of the standalone NVFP4 quantizer (attnqat_quantize)
+against the float64 oracle: FP4 codes and E4M3 scale bytes identical, and the
+dequantized bf16 values identical bit for bit."""
+import numpy as np
+import pytest
+
+import oracle
+from quantization_aware_attention_nvfp4_b200 import workloads as W
+from tests.helpers import bf16_bits, to_gpu_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_quantize(bits2d):
+    import quantization_aware_attention_nvfp4_b200 as A
+    x = to_gpu_bf16(bits2d)
+    codes, scales, deq = A.attnqat_quantize(x)
+    return codes.cpu().numpy(), scales.cpu().numpy(), bf16_bits(deq)
+
+
+def _oracle_deq_bits(deq_f64):
+    # the oracle's dequantized values are exact in bf16: round-trip is exact
+    return W.f32_to_bf16_bits(deq_f64.astype(np.float32))
+
+
+def _check(bits2d):
+    rows, cols = bits2d.shape
+    c_gpu, s_gpu, d_gpu = _gpu_quantize(bits2d)
+    c_ref, s_ref, d_ref = oracle.quantize_rows(bits2d, rows, cols, cols, 1)
+    assert np.array_equal(s_gpu, s_ref), np.argwhere(s_gpu != s_ref)[:5]
+    assert np.array_equal(c_gpu, c_ref), np.argwhere(c_gpu != c_ref)[:5]
+    assert np.array_equal(d_ref.astype(np.float32).astype(np.float64), d_ref)
+    assert np.array_equal(d_gpu, _oracle_deq_bits(d_ref))
+
+
+def test_every_finite_bf16_as_block_amax():
+    """Each finite bf16 value once as the amax of its own block, with random
+    partners at or below it (covers every scale code, subnormal scales, zero
+    scales and saturation)."""
+    rng = np.random.default_rng(101)
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = W.bf16_bits_to_f32(bits)
+    keep = np.isfinite(vals)
+    bits, vals = bits[keep], vals[keep]
+    blocks = rng.uniform(-1, 1, (bits.size, 16)).astype(np.float32) * np.abs(vals)[:, None]
+    b = W.f32_to_bf16_bits(blocks)
+    b[:, 0] = bits
+    _check(b)
+
+
+def test_tie_rich_and_edge_blocks():
+    rng = np.random.default_rng(102)
+    e4m3 = np.array([oracle.e4m3_value(c) for c in range(127)])
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    rows = []
+    for sc in range(1, 127):
+        s = e4m3[sc]
+        for _ in range(8):
+            x = rng.choice(mids, 16) * s * rng.choice([-1, 1], 16)
+            x[0] = 6 * s
+            rows.append(x.astype(np.float32))
+    rows.append(np.full(16, 3000.0, np.float32))
+    rows.append(np.array([-0.0, 0.0] * 8, np.float32))
+    rows.append(np.array([-1e-30] + [1.0] * 15, np.float32))
+    for a in (3.02, 3.2, 3.49, 0.5, 2.99):  # subnormal-scale neighbourhood
+        x = np.zeros(16, np.float32)
+        x[0] = a * 2 ** -9
+        rows.append(x)
+    b = np.stack([W.f32_to_bf16_bits(r) for r in rows])
+    _check(b)
+
+
+@pytest.mark.parametrize("rows,cols,scale", [(4096, 128, 1.0), (513, 64, 30.0), (7, 16, 1e-3)])
+def test_random_rows(rows, cols, scale):
+    rng = np.random.default_rng(rows + cols)
+    x = (rng.standard_normal((rows, cols)) * scale).astype(np.float32)
+    _check(W.f32_to_bf16_bits(x))
+
+
+def test_transposed_view_blocks_along_tokens():
+    """V blocked along tokens: the [BH, D, Lk] view of a [BH, Lk, D] tensor."""
+    import quantization_aware_attention_nvfp4_b200 as A
+    rng = np.random.default_rng(103)
+    BH, Lk, D = 3, 272, 128
+    v = W.f32_to_bf16_bits(rng.standard_normal((BH, Lk, D)).astype(np.float32))
+    vt = to_gpu_bf16(v).transpose(1, 2)  # [BH, D, Lk], strides (Lk*D, 1, D)
+    codes, scales, deq = A.attnqat_quantize(vt)
+    codes, scales = codes.cpu().numpy(), scales.cpu().numpy()
+    deq_bits = bf16_bits(deq.transpose(1, 2))  # back to [BH, Lk, D]
+    for z in range(BH):
+        c_ref, s_ref, d_ref = oracle.quantize_rows(v[z], D, Lk, 1, D)
+        assert np.array_equal(scales[z], s_ref)
+        assert np.array_equal(codes[z], c_ref)
+        assert np.array_equal(deq_bits[z], _oracle_deq_bits(d_ref.T))
+
+
+def test_rejects_bad_arguments():
+    import torch
+    import quantization_aware_attention_nvfp4_b200 as A
+    x = torch.zeros((4, 24), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(A.AttnQatError) as e:
+        A.attnqat_quantize(x)
+    assert e.value.status == A.EINVAL
