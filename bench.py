@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the Attn-QAT training attention step (forward + backward) on B200.
+
+One step = attnqat_fwd + attnqat_bwd over one batch of the pages' shape:
+B=1, H=6, Lq=Lk=31200, D=128, bf16, all four quantizers on, sm_scale=1/sqrt(128)
+(the 6-head, 31200-token shape the fastvideo-kernel commit times).  The step
+runs every kernel of the path: the three operand quantizers, the forward, the
+Delta kernel, the dK/dV kernel and the dQ kernel.
+
+Metric: nominal TFLOP/s of fwd+bwd (forward 4*B*H*Lq*Lk*D, backward 2.5x that),
+also reported as fwd / bwd / fwd+bwd milliseconds and as a fraction of the
+measured B200 BF16 tensor peak.  Inputs are seeded synthetic tensors; L2 is
+flushed (a 256 MiB write) between timed steps, each step is timed with CUDA
+events on the launching stream, and multi-GPU runs report the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the float64 CPU oracle on the host cores instead (the
+pages ship no runnable implementation): each step is a bounded sample of the
+same workload, one head with the first query rows against all keys.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from quantization_aware_attention_nvfp4_b200 import workloads as W  # noqa: E402
+
+WORKLOAD = "wan_6h_31200"
+METRIC = "Attn-QAT fwd+bwd ms & TFLOP/s at H6 L31200 D128; % of B200 BF16 peak"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+# rows of the oracle's bounded samples (query rows of head 0 against all keys):
+# the CPU-baseline leg of the GPU run (~10-30 s on the machine's host cores) and
+# each step of --impl reference
+BASELINE_SAMPLE_ROWS = int(os.environ.get("ATTNQAT_BASELINE_ROWS", "6144"))
+ORACLE_SAMPLE_ROWS = int(os.environ.get("ATTNQAT_ORACLE_SAMPLE_ROWS", "1024"))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p["bf16_tflops_sustained"], source="measured")
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the
+    timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        if self.proc is None or not getattr(self, "out", ""):
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["no samples"])
+        loaded = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return dict(sm_mhz=float(statistics.median(loaded)), sm_max_mhz=float(max(smax)),
+                    reasons=sorted(reasons), samples=len(sm))
+
+
+# ----------------------------------------------------------------- GPU arm --
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+    import quantization_aware_attention_nvfp4_b200 as A
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = W.get(WORKLOAD)
+    flops = w.nominal_flops()
+    peaks = load_peaks()
+
+    # seeded inputs (host), moved to the device once; the timed region starts
+    # with them resident in HBM
+    inp = W.inputs(w)
+    host = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16) for n in inp}
+    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
+    c = w.sm_scale
+    flags = A.QUANT_ALL
+    ws = torch.empty(A.attnqat_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
+    m = torch.empty_like(lse)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        A.attnqat_fwd(q, k, v, sm_scale=c, flags=flags, ws=ws, out=(o, lse, m))
+        A.attnqat_bwd(q, k, v, lse, m, do, ws, sm_scale=c, flags=flags, out=(dq, dk, dv))
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    A.attnqat_device_status()
+
+    # ---- timed region: K steps, L2 flushed between steps, per-step events
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    A.attnqat_profile_enable(True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            A.attnqat_fwd(q, k, v, sm_scale=c, flags=flags, ws=ws, out=(o, lse, m))
+            e1.record(stream)
+            A.attnqat_bwd(q, k, v, lse, m, do, ws, sm_scale=c, flags=flags, out=(dq, dk, dv))
+            e2.record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    kernels = A.attnqat_profile_read(1 << 16)
+    A.attnqat_profile_enable(False)
+    A.attnqat_device_status()
+    fwd_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in ev)
+    bwd_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in ev)
+    tot_ms = fwd_ms + bwd_ms
+    if world > 1:
+        t = torch.tensor([tot_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms, fwd_ms, bwd_ms = (float(x) for x in t.tolist())
+
+    # ---- per-kernel durations inside the timed region (dominant kernel)
+    per = {}
+    for name, ms in kernels:
+        per.setdefault(name, []).append(ms)
+    units = 2.0 * w.B * w.H * w.Lq * w.Lk * w.D  # one matmul unit
+    algo_flops = {"attn_fwd": 2 * units, "attn_bwd_dkdv": 4 * units, "attn_bwd_dq": 1 * units}
+    exec_flops = {"attn_fwd": 3 * units, "attn_bwd_dkdv": 4 * units, "attn_bwd_dq": 3 * units}
+    tensor_kernels = {n: v for n, v in per.items() if n in algo_flops}
+    dom = max(tensor_kernels, key=lambda n: sum(tensor_kernels[n]))
+    dom_ms = statistics.mean(per[dom])
+    achieved = algo_flops[dom] / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    traffic = load_traffic(dom)
+    kernel_table = {n: dict(launches=len(v), mean_ms=round(statistics.mean(v), 4),
+                            share=round(sum(v) / sum(sum(x) for x in per.values()), 4))
+                    for n, v in per.items()}
+    for n in algo_flops:
+        if n in kernel_table:
+            kernel_table[n]["algorithmic_tflops"] = round(algo_flops[n] / (kernel_table[n]["mean_ms"] * 1e-3) / 1e12, 1)
+            kernel_table[n]["executed_tflops"] = round(exec_flops[n] / (kernel_table[n]["mean_ms"] * 1e-3) / 1e12, 1)
+
+    # ---- end to end through the public API with host buffers
+    e2e = e2e_arm(args, A, torch, dev, host, w, c, flags, ws, world)
+
+    value = world * flops["total"] * args.steps / (tot_ms * 1e-3) / 1e12
+    ms_step = tot_ms / args.steps
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, recipe in DESIGN.md)",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
+                   "quantizers": "q,k,v,p", "sm_scale": "1/sqrt(128)", "global_batch": w.B * world,
+                   "seq_len": w.Lq, "parallelism": "replicas x%d (heads independent, no collective)" % world,
+                   "l2": "flushed between steps (256 MiB write); each step timed with CUDA events"},
+        "fwd_ms": round(fwd_ms / args.steps, 4),
+        "bwd_ms": round(bwd_ms / args.steps, 4),
+        "fwd_tflops": round(flops["fwd"] / (fwd_ms / args.steps * 1e-3) / 1e12, 1),
+        "bwd_tflops": round(flops["bwd"] / (bwd_ms / args.steps * 1e-3) / 1e12, 1),
+        "frac_of_bf16_peak": round(value / world / peaks["bf16_tflops"], 4),
+        "frac_of_bf16_peak_sustained": round(value / world / peaks["bf16_tflops_sustained"], 4),
+        "frac_of_datasheet_2250": round(value / world / DATASHEET_BF16_TFLOPS, 4),
+        "peaks": "%s (bf16 %.1f burst / %.1f sustained TFLOP/s)" % (peaks["source"], peaks["bf16_tflops"],
+                                                                  peaks["bf16_tflops_sustained"]),
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic,
+                     "algorithmic_flops_per_launch": algo_flops[dom],
+                     "mean_launch_ms": round(dom_ms, 4),
+                     "peak_kind": "measured bf16 sustained (kernel timed inside a long step)"
+                     if peaks["source"] == "measured" else "fallback"},
+        "kernels": kernel_table,
+        "gpu_launches": len(kernels),
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": round(wall, 3),
+        "e2e": e2e,
+    }
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline_sample(rows=BASELINE_SAMPLE_ROWS)
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_arm(args, A, torch, dev, host, w, c, flags, ws, world):
+    """Same step through the public API with host buffers: every step copies
+    Q, K, V, dO from pinned host memory to the device and O, LSE, m, dQ, dK, dV
+    back, all inside the timed region."""
+    pin = {n: t.pin_memory() for n, t in host.items()}
+    outs = dict(o=torch.empty_like(pin["q"]).pin_memory(), dq=torch.empty_like(pin["q"]).pin_memory(),
+                dk=torch.empty_like(pin["k"]).pin_memory(), dv=torch.empty_like(pin["v"]).pin_memory(),
+                lse=torch.empty((w.B, w.H, w.Lq), dtype=torch.float32).pin_memory(),
+                m=torch.empty((w.B, w.H, w.Lq), dtype=torch.float32).pin_memory())
+    dbuf = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in pin.items()}
+    o = torch.empty_like(dbuf["q"])
+    lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
+    m = torch.empty_like(lse)
+    dq, dk, dv = torch.empty_like(dbuf["q"]), torch.empty_like(dbuf["k"]), torch.empty_like(dbuf["v"])
+    stream = torch.cuda.current_stream(dev)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+
+    def step():
+        for n in pin:
+            dbuf[n].copy_(pin[n], non_blocking=True)
+        A.attnqat_fwd(dbuf["q"], dbuf["k"], dbuf["v"], sm_scale=c, flags=flags, ws=ws, out=(o, lse, m))
+        A.attnqat_bwd(dbuf["q"], dbuf["k"], dbuf["v"], lse, m, dbuf["do"], ws, sm_scale=c, flags=flags,
+                      out=(dq, dk, dv))
+        for name, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv), ("lse", lse), ("m", m)):
+            outs[name].copy_(t, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    n = max(2, args.steps // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * w.nominal_flops()["total"] * n / (ms * 1e-3) / 1e12
+    return {"value": round(value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": round(ms / n, 4)}
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
+    summary was taken on the current kernel sources (else null)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        d = json.load(open(path))
+        from quantization_aware_attention_nvfp4_b200 import build as B
+        rec = d.get(kernel)
+        if not rec or rec.get("sources_sha") != B.sources_digest():
+            return None
+        return rec.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+# -------------------------------------------------------------- CPU oracle --
+
+def cpu_baseline_sample(rows: int):
+    """The float64 oracle on a bounded sample of the workload: head 0, the
+    first `rows` query rows against all 31200 keys, forward and backward
+    (dQ for those rows, their dK/dV contributions for every key).  Returns the
+    nominal TFLOP/s of that sub-problem."""
+    import oracle
+    w = W.get(WORKLOAD)
+    q = W.head_bits(w, "q", 0, 0)[:rows]
+    k = W.head_bits(w, "k", 0, 0)
+    v = W.head_bits(w, "v", 0, 0)
+    do = W.head_bits(w, "do", 0, 0)[:rows]
+    t0 = time.perf_counter()
+    hd = oracle.Head(q, k, v, w.sm_scale, oracle.QUANT_ALL, do)
+    hd.stats()
+    hd.backward()
+    dt = time.perf_counter() - t0
+    flops = 3.5 * 4.0 * rows * w.Lk * w.D
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": "head 0, query rows [0,%d) x all %d keys, fwd+bwd (float64 C oracle)" % (rows, w.Lk)}
+
+
+def reference_arm(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    w = W.get(WORKLOAD)
+    rows = ORACLE_SAMPLE_ROWS
+    for _ in range(max(0, min(args.warmup, 1))):
+        cpu_baseline_sample(rows=64)
+    times = []
+    for _ in range(args.steps):
+        r = cpu_baseline_sample(rows=rows)
+        times.append(r["seconds"])
+    flops = 3.5 * 4.0 * rows * w.Lk * w.D
+    value = flops * len(times) / sum(times) / 1e12
+    sample = "head 0, query rows [0,%d) x all %d keys, fwd+bwd per step (float64 C oracle)" % (rows, w.Lk)
+    out = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(times) / len(times), 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
+                   "quantizers": "q,k,v,p", "sample_rows": rows},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

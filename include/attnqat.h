@@ -81,6 +81,17 @@ const char *attnqat_strerror(int status);
 /* Last CUDA runtime error recorded by a failed call (cudaError_t as int). */
 int attnqat_last_cuda_error(void);
 
+/* Kernel timing (instrumentation).  attnqat_profile_enable(1) makes every
+ * later attnqat_fwd / attnqat_bwd call record a CUDA event on its stream
+ * before and after each kernel it launches (0 turns this off; both calls
+ * discard what was recorded).  attnqat_profile_read() waits for the recorded
+ * events, writes up to max_records kernel names (static strings) and
+ * durations in milliseconds, clears the record and returns how many kernels
+ * were recorded (or a negative status).  Not thread-safe across streams of
+ * different devices; meant for benchmarks. */
+int attnqat_profile_enable(int on);
+int attnqat_profile_read(const char **names, float *ms, int max_records);
+
 /* Synchronizes the current device, then returns ATTNQAT_OK if no device-side
  * wait of this library has timed out since the last call, else
  * ATTNQAT_ETIMEOUT (and clears the flag). */

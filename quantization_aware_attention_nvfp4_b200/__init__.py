@@ -71,6 +71,10 @@ def load(build_if_needed: bool = True):
             lib.attnqat_last_cuda_error.argtypes = []
             lib.attnqat_device_status.restype = I
             lib.attnqat_device_status.argtypes = []
+            lib.attnqat_profile_enable.restype = I
+            lib.attnqat_profile_enable.argtypes = [I]
+            lib.attnqat_profile_read.restype = I
+            lib.attnqat_profile_read.argtypes = [P, P, I]
             lib.attnqat_quantize.restype = I
             lib.attnqat_quantize.argtypes = [P, I64, I64, I64, I64, I64, I64, P, P, P, P]
             lib.attnqat_workspace_size.restype = SZ
@@ -207,6 +211,23 @@ def attnqat_bwd(q, k, v, lse, m, dO, ws, sm_scale=None, flags=QUANT_ALL, out=Non
                             ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(st, "attnqat_bwd")
     return dq, dk, dv
+
+
+def attnqat_profile_enable(on: bool = True) -> None:
+    """Start (or stop) recording CUDA events around each kernel the library
+    launches; see attnqat_profile_read."""
+    _check(load().attnqat_profile_enable(1 if on else 0), "attnqat_profile_enable")
+
+
+def attnqat_profile_read(max_records: int = 4096) -> list:
+    """[(kernel name, milliseconds)] for the kernels launched since the last
+    read (waits for their events)."""
+    names = (ctypes.c_char_p * max_records)()
+    ms = (ctypes.c_float * max_records)()
+    n = load().attnqat_profile_read(names, ms, max_records)
+    if n < 0:
+        _check(n, "attnqat_profile_read")
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n, max_records))]
 
 
 def attnqat_device_status() -> int:

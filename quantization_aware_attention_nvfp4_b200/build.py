@@ -33,6 +33,17 @@ def sources() -> list:
                   + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+def sources_digest() -> str:
+    """SHA-256 over the library's sources (identifies the kernels a profile
+    was taken on)."""
+    import hashlib
+    h = hashlib.sha256()
+    for path in sources():
+        h.update(os.path.basename(path).encode())
+        h.update(open(path, "rb").read())
+    return h.hexdigest()[:16]
+
+
 def stale() -> bool:
     if not os.path.exists(LIB):
         return True

@@ -6,6 +6,7 @@
 #include <cstring>
 #include <mutex>
 #include <set>
+#include <vector>
 #include <utility>
 
 #include "attnqat.h"
@@ -33,6 +34,51 @@ cudaError_t ensure_smem_attr(const void *kernel, int bytes) {
   if (e == cudaSuccess) done.insert({dev, kernel});
   return e;
 }
+
+// ------------------------------------------------------- kernel timing --
+
+// Optional instrumentation: while enabled, every kernel launch of
+// attnqat_fwd / attnqat_bwd is bracketed by two CUDA events recorded on the
+// caller's stream; attnqat_profile_read() returns the durations.
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  struct Rec {
+    const char *name;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  cudaEvent_t take() {
+    if (used == pool.size()) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+};
+static Profiler g_prof;
+
+struct ProfScope {
+  cudaStream_t s;
+  bool on;
+  cudaEvent_t b = nullptr;
+  ProfScope(const char *name, cudaStream_t stream) : s(stream), on(false) {
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    if (!g_prof.on) return;
+    cudaEvent_t a = g_prof.take();
+    b = g_prof.take();
+    if (!a || !b) return;
+    cudaEventRecord(a, s);
+    g_prof.recs.push_back({name, a, b});
+    on = true;
+  }
+  ~ProfScope() {
+    if (on) cudaEventRecord(b, s);
+  }
+};
 
 // ----------------------------------------------------------- device check --
 
@@ -155,22 +201,26 @@ static int prepare_operands(const void *q, const void *k, const void *v, int B, 
   if (e != cudaSuccess) return cuda_fail(e);
   if (flags & ATTNQAT_QUANT_Q) {
     uint16_t *dst = reinterpret_cast<uint16_t *>(ws + w.qh);
+    ProfScope ps("quantize_q", stream);
     e = launch_quantize(static_cast<const uint16_t *>(q), 1, BH * Lq, D, 0, D, 1, nullptr, nullptr,
                         f16 ? nullptr : dst, f16 ? dst : nullptr, nullptr, stream);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   if (flags & ATTNQAT_QUANT_K) {
     uint16_t *dst = reinterpret_cast<uint16_t *>(ws + w.kh);
+    ProfScope ps("quantize_k", stream);
     e = launch_quantize(static_cast<const uint16_t *>(k), 1, BH * Lk, D, 0, D, 1, nullptr, nullptr,
                         f16 ? nullptr : dst, f16 ? dst : nullptr, nullptr, stream);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   if (flags & ATTNQAT_QUANT_V) {
     // blocks of 16 consecutive tokens per channel: the transposed view
+    ProfScope ps("quantize_v", stream);
     e = launch_quantize(static_cast<const uint16_t *>(v), BH, D, Lk, static_cast<int64_t>(Lk) * D, 1, D,
                         nullptr, nullptr, reinterpret_cast<uint16_t *>(ws + w.vh),
                         reinterpret_cast<uint16_t *>(ws + w.vh16), stats + 2, stream);
   } else {
+    ProfScope ps("absmax_v", stream);
     e = launch_absmax(static_cast<const __nv_bfloat16 *>(v), BH * Lk * D, stats + 2, stream);
   }
   if (e != cudaSuccess) return cuda_fail(e);
@@ -196,6 +246,32 @@ const char *attnqat_strerror(int status) {
 }
 
 int attnqat_last_cuda_error(void) { return g_last_cuda_error; }
+
+int attnqat_profile_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  g_prof.on = on != 0;
+  g_prof.recs.clear();
+  g_prof.used = 0;
+  return ATTNQAT_OK;
+}
+
+int attnqat_profile_read(const char **names, float *ms, int max_records) {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  const int n = static_cast<int>(g_prof.recs.size());
+  for (int i = 0; i < n && i < max_records; ++i) {
+    const Profiler::Rec &r = g_prof.recs[i];
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e);
+    float t = 0.0f;
+    e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (names) names[i] = r.name;
+    if (ms) ms[i] = t;
+  }
+  g_prof.recs.clear();
+  g_prof.used = 0;
+  return n;
+}
 
 int attnqat_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
@@ -271,7 +347,11 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   a.o32 = reinterpret_cast<float *>(wsb + w.o32);
   a.lse = lse;
   a.m = m;
-  cudaError_t e = launch_fwd(D, f16, pv_f16, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, a, BH, s);
+  cudaError_t e;
+  {
+    ProfScope ps("attn_fwd", s);
+    e = launch_fwd(D, f16, pv_f16, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, a, BH, s);
+  }
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }
 
@@ -296,8 +376,11 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
   float *stats = reinterpret_cast<float *>(wsb + w.stats);
   cudaError_t e = cudaMemsetAsync(stats, 0, 8, s);  // keeps stats[2] from the forward
   if (e != cudaSuccess) return cuda_fail(e);
-  e = launch_delta(reinterpret_cast<const float *>(wsb + w.o32), static_cast<const __nv_bfloat16 *>(dO), delta,
-                   static_cast<int64_t>(BH) * Lq, D, stats, s);
+  {
+    ProfScope ps("delta", s);
+    e = launch_delta(reinterpret_cast<const float *>(wsb + w.o32), static_cast<const __nv_bfloat16 *>(dO), delta,
+                     static_cast<int64_t>(BH) * Lq, D, stats, s);
+  }
   if (e != cudaSuccess) return cuda_fail(e);
   const bool f16 = qk_f16(flags);
   const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
@@ -321,9 +404,15 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
   a.dq = static_cast<__nv_bfloat16 *>(dq);
   a.dk = static_cast<__nv_bfloat16 *>(dk);
   a.dv = static_cast<__nv_bfloat16 *>(dv);
-  e = launch_bwd_dkdv(D, f16, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, tdo, a, BH, s);
+  {
+    ProfScope ps("attn_bwd_dkdv", s);
+    e = launch_bwd_dkdv(D, f16, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, tdo, a, BH, s);
+  }
   if (e != cudaSuccess) return cuda_fail(e);
-  e = launch_bwd_dq(D, f16, tq, tk, tv, tdo, a, BH, s);
+  {
+    ProfScope ps("attn_bwd_dq", s);
+    e = launch_bwd_dq(D, f16, tq, tk, tv, tdo, a, BH, s);
+  }
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }
 
