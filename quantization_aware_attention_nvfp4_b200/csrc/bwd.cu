@@ -15,8 +15,9 @@
 // The split into a dK/dV and a dQ kernel follows the fastvideo-kernel
 // triton_kernels commit (SM100 Attn-QAT route: separate dQ and dK/dV tiles);
 // the tiles here are 128 x 128 tcgen05 tiles with TMEM accumulators.
-// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 2..5
-// one thread per query row (TMEM lane).
+// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 2..9
+// row warps: two per TMEM lane quarter, so every query row (TMEM lane) has
+// two threads, each owning 64 of the tile's 128 columns.
 #include "common.cuh"
 #include "internal.h"
 
@@ -58,8 +59,8 @@ __device__ __forceinline__ void init_bwd_bars(BwdBars *b) {
     mbar_init(&b->bempty[s], 1);
   }
   mbar_init(&b->sfull, 1);
-  mbar_init(&b->sempty, 4);
-  mbar_init(&b->xfull, 4);
+  mbar_init(&b->sempty, kSoftWarps);
+  mbar_init(&b->xfull, kSoftWarps);
   mbar_init(&b->xempty, 1);
   mbar_init(&b->done, 1);
   b->abort = 0;
@@ -94,25 +95,28 @@ __device__ __forceinline__ uint32_t pack_ds(float a, float b) {
   return QKF16 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
 }
 
-// One query tile for one row of the dK/dV kernel, 32 keys at a time: S and
-// dP from TMEM, P~ = exp(S - m) and fq(P~)/l (bf16, a row of the transposed
-// dV operand), and dS = (P~/l)(dP - Delta) in float32, scaled by dsc and
-// packed for the dK operand.  P never leaves float32.
+// One query tile for one thread of the dK/dV kernel (one query row, 64 key
+// columns starting at col0), 32 keys at a time: S and dP from TMEM,
+// P~ = exp(S - m) and fq(P~)/l (bf16, half a row of the transposed dV
+// operand), and dS = (P~/l)(dP - Delta) in float32, scaled by dsc and packed
+// for the dK operand.  P never leaves float32.
 template <int QP, int QKF16, bool MASKED>
-__device__ __forceinline__ void dkdv_tile(uint32_t tS, uint32_t tDP, int valid_k, bool vq, float cl, float nml,
-                                          float inv_l, float delta, float dsc, uint32_t (&pw)[64],
-                                          uint32_t (&dsw)[64]) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t r[32];
-    tmem_ld32(tS + c * 32, r);
+__device__ __forceinline__ void dkdv_tile(uint32_t tS, uint32_t tDP, int col0, int valid_k, bool vq, float cl,
+                                          float nml, float inv_l, float delta, float dsc, uint32_t (&pw)[32],
+                                          uint32_t (&dsw)[32]) {
+#pragma unroll 1
+  for (int c = 0; c < 2; ++c) {
+    uint32_t r[32], d[32];
+    tmem_ld32(tS + col0 + c * 32, r);
+    tmem_ld32(tDP + col0 + c * 32, d);
     tmem_ld_wait();
     float p[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float e = ex2_approx(fmaf(__uint_as_float(r[i]), cl, nml));
-      p[i] = (vq && (!MASKED || c * 32 + i < valid_k)) ? e : 0.0f;
+      p[i] = (vq && (!MASKED || col0 + c * 32 + i < valid_k)) ? e : 0.0f;
     }
+    uint32_t wv[16], ws[16];
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       if (QP) {
@@ -122,28 +126,37 @@ __device__ __forceinline__ void dkdv_tile(uint32_t tS, uint32_t tDP, int valid_k
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float2 g = unpack_f16x2(rr[i]);
-          pw[16 * c + 8 * b + i] = pack_bf16x2(g.x * f, g.y * f);
+          wv[8 * b + i] = pack_bf16x2(g.x * f, g.y * f);
         }
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          pw[16 * c + 8 * b + i] = pack_bf16x2(p[16 * b + 2 * i] * inv_l, p[16 * b + 2 * i + 1] * inv_l);
+          wv[8 * b + i] = pack_bf16x2(p[16 * b + 2 * i] * inv_l, p[16 * b + 2 * i + 1] * inv_l);
       }
     }
-    tmem_ld32(tDP + c * 32, r);
-    tmem_ld_wait();
     const float pf = inv_l * dsc;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const float d0 = p[2 * i] * pf * (__uint_as_float(r[2 * i]) - delta);
-      const float d1 = p[2 * i + 1] * pf * (__uint_as_float(r[2 * i + 1]) - delta);
-      dsw[16 * c + i] = pack_ds<QKF16>(d0, d1);
+      const float d0 = p[2 * i] * pf * (__uint_as_float(d[2 * i]) - delta);
+      const float d1 = p[2 * i + 1] * pf * (__uint_as_float(d[2 * i + 1]) - delta);
+      ws[i] = pack_ds<QKF16>(d0, d1);
+    }
+    // runtime c: write through a small selector instead of dynamic indexing
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (c == 0) {
+        pw[i] = wv[i];
+        dsw[i] = ws[i];
+      } else {
+        pw[16 + i] = wv[i];
+        dsw[16 + i] = ws[i];
+      }
     }
   }
 }
 
 template <int D, int QP, int QKF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const BwdArgs a) {
@@ -241,60 +254,68 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(&bars->done);
     }
   } else {
-    const int wq = warp & 3;
-    const uint32_t row = static_cast<uint32_t>(wq * 32 + lane);
-    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const RowRole rr(warp, lane);
+    const int col0 = rr.half * 64;
     const int valid_k = a.Lk - kt * kBN;  // >= 128 for full key tiles
     const float cl = a.scale_log2;
     const float dsc = ds_scale<QKF16>(a.stats);
     const uint32_t xaddr = sbase + L::kX;
+    const uint32_t tS = tmem + rr.lane_addr + L::kTmemS, tDP = tmem + rr.lane_addr + L::kTmemDP;
     bool ok = true;
-    for (int i = 0; i < nq; ++i) {
-      const int qg = i * kBM + static_cast<int>(row);
-      const bool vq = qg < a.Lq;
+    // row statistics of the current query tile, prefetched one tile ahead
+    auto load_stats = [&](int i, float &m, float &lse, float &delta) {
+      const int qg = i * kBM + static_cast<int>(rr.row);
+      const bool vq = i < nq && qg < a.Lq;
       const size_t si = static_cast<size_t>(bh) * a.Lq + (vq ? qg : 0);
-      const float m = vq ? a.m[si] : 0.0f;
-      const float lse = vq ? a.lse[si] : 0.0f;
-      const float delta = vq ? a.delta[si] : 0.0f;
+      m = vq ? a.m[si] : 0.0f;
+      lse = vq ? a.lse[si] : 0.0f;
+      delta = vq ? a.delta[si] : 0.0f;
+    };
+    float m_n, lse_n, delta_n;
+    load_stats(0, m_n, lse_n, delta_n);
+    for (int i = 0; i < nq; ++i) {
+      const bool vq = i * kBM + static_cast<int>(rr.row) < a.Lq;
+      const float m = m_n, lse = lse_n, delta = delta_n;
+      load_stats(i + 1, m_n, lse_n, delta_n);
       const float nml = -(m * kLog2e);
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
-      uint32_t pw[64], dsw[64];
+      uint32_t pw[32], dsw[32];
       if (!mbar_wait(&bars->sfull, i & 1, abort)) { ok = false; break; }
       tc_fence_after();
       if (valid_k < kBN)
-        dkdv_tile<QP, QKF16, true>(tmem + lane_addr + L::kTmemS, tmem + lane_addr + L::kTmemDP, valid_k, vq,
-                                   cl, nml, inv_l, delta, dsc, pw, dsw);
+        dkdv_tile<QP, QKF16, true>(tS, tDP, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
       else
-        dkdv_tile<QP, QKF16, false>(tmem + lane_addr + L::kTmemS, tmem + lane_addr + L::kTmemDP, valid_k, vq,
-                                    cl, nml, inv_l, delta, dsc, pw, dsw);
+        dkdv_tile<QP, QKF16, false>(tS, tDP, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
       if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
-      store_row128(xaddr, row, pw);
+      store_row_half(xaddr, rr.row, rr.half, pw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
       if (!mbar_wait(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
-      store_row128(xaddr, row, dsw);
+      store_row_half(xaddr, rr.row, rr.half, dsw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
     }
     if (ok && mbar_wait(&bars->done, 0, abort)) {
       tc_fence_after();
-      const int kg = kt * kBN + static_cast<int>(row);
+      // TMEM lanes of dV/dK are keys; each thread stores D/2 columns of its key row
+      const int kg = kt * kBN + static_cast<int>(rr.row);
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lk + kg) * D;
       const float kscale = a.sm_scale / ds_scale<QKF16>(a.stats);  // exact: power-of-two divisor
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = rr.half * (D / 2) + c * 32;
         uint32_t r[32], s[32];
-        tmem_ld32(tmem + lane_addr + L::kTmemDV + c * 32, r);
-        tmem_ld32(tmem + lane_addr + L::kTmemDK + c * 32, s);
+        tmem_ld32(tmem + rr.lane_addr + L::kTmemDV + col, r);
+        tmem_ld32(tmem + rr.lane_addr + L::kTmemDK + col, s);
         tmem_ld_wait();
         if (kg < a.Lk) {
-          uint4 *dv = reinterpret_cast<uint4 *>(a.dv + rowoff + c * 32);
-          uint4 *dk = reinterpret_cast<uint4 *>(a.dk + rowoff + c * 32);
+          uint4 *dv = reinterpret_cast<uint4 *>(a.dv + rowoff + col);
+          uint4 *dk = reinterpret_cast<uint4 *>(a.dk + rowoff + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint32_t w[4], x[4];
@@ -340,24 +361,24 @@ struct DqLayout {
   static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDQ = 256;
 };
 
-// One key tile for one row of the dQ kernel, 32 keys at a time:
-// P = exp(S - LSE) in float32 and dS = P (dP - Delta), scaled by dsc and
-// packed for the dQ operand.
+// One key tile for one thread of the dQ kernel (one query row, 64 key
+// columns starting at col0), 32 keys at a time: P = exp(S - LSE) in float32
+// and dS = P (dP - Delta), scaled by dsc and packed for the dQ operand.
 template <int QKF16, bool MASKED>
-__device__ __forceinline__ void dq_tile(uint32_t tS, uint32_t tDP, int valid_k, bool vq, float cl, float nlse,
-                                        float delta, float dsc, uint32_t (&dsw)[64]) {
+__device__ __forceinline__ void dq_tile(uint32_t tS, uint32_t tDP, int col0, int valid_k, bool vq, float cl,
+                                        float nlse, float delta, float dsc, uint32_t (&dsw)[32]) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < 2; ++c) {
     uint32_t r[32], d[32];
-    tmem_ld32(tS + c * 32, r);
-    tmem_ld32(tDP + c * 32, d);
+    tmem_ld32(tS + col0 + c * 32, r);
+    tmem_ld32(tDP + col0 + c * 32, d);
     tmem_ld_wait();
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * i]), cl, nlse));
       float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), cl, nlse));
-      if (!vq || (MASKED && c * 32 + 2 * i >= valid_k)) p0 = 0.0f;
-      if (!vq || (MASKED && c * 32 + 2 * i + 1 >= valid_k)) p1 = 0.0f;
+      if (!vq || (MASKED && col0 + c * 32 + 2 * i >= valid_k)) p0 = 0.0f;
+      if (!vq || (MASKED && col0 + c * 32 + 2 * i + 1 >= valid_k)) p1 = 0.0f;
       dsw[16 * c + i] = pack_ds<QKF16>(p0 * dsc * (__uint_as_float(d[2 * i]) - delta),
                                        p1 * dsc * (__uint_as_float(d[2 * i + 1]) - delta));
     }
@@ -365,7 +386,7 @@ __device__ __forceinline__ void dq_tile(uint32_t tS, uint32_t tDP, int valid_k, 
 }
 
 template <int D, int QKF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                        const BwdArgs a) {
@@ -454,10 +475,9 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(&bars->done);
     }
   } else {
-    const int wq = warp & 3;
-    const uint32_t row = static_cast<uint32_t>(wq * 32 + lane);
-    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-    const int q = qt * kBM + static_cast<int>(row);
+    const RowRole rr(warp, lane);
+    const int col0 = rr.half * 64;
+    const int q = qt * kBM + static_cast<int>(rr.row);
     const bool vq = q < a.Lq;
     const size_t si = static_cast<size_t>(bh) * a.Lq + (vq ? q : 0);
     const float lse = vq ? a.lse[si] : 0.0f;
@@ -467,22 +487,21 @@ __global__ void __launch_bounds__(192, 1)
     const float dsc = ds_scale<QKF16>(a.stats);
     const int last_valid = a.Lk - (nk - 1) * kBN;
     const uint32_t xaddr = sbase + L::kX;
+    const uint32_t tS = tmem + rr.lane_addr + L::kTmemS, tDP = tmem + rr.lane_addr + L::kTmemDP;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
-      uint32_t dsw[64];
+      uint32_t dsw[32];
       if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
       tc_fence_after();
       if (j == nk - 1 && last_valid < kBN)
-        dq_tile<QKF16, true>(tmem + lane_addr + L::kTmemS, tmem + lane_addr + L::kTmemDP, last_valid, vq, cl,
-                             nlse, delta, dsc, dsw);
+        dq_tile<QKF16, true>(tS, tDP, col0, last_valid, vq, cl, nlse, delta, dsc, dsw);
       else
-        dq_tile<QKF16, false>(tmem + lane_addr + L::kTmemS, tmem + lane_addr + L::kTmemDP, kBN, vq, cl, nlse,
-                              delta, dsc, dsw);
+        dq_tile<QKF16, false>(tS, tDP, col0, kBN, vq, cl, nlse, delta, dsc, dsw);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
       if (j >= 1 && !mbar_wait(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
-      store_row128(xaddr, row, dsw);
+      store_row_half(xaddr, rr.row, rr.half, dsw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
@@ -492,12 +511,13 @@ __global__ void __launch_bounds__(192, 1)
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
       const float qscale = a.sm_scale / dsc;  // exact: power-of-two divisor
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = rr.half * (D / 2) + c * 32;
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + L::kTmemDQ + c * 32, r);
+        tmem_ld32(tmem + rr.lane_addr + L::kTmemDQ + col, r);
         tmem_ld_wait();
         if (vq) {
-          uint4 *dst = reinterpret_cast<uint4 *>(a.dq + rowoff + c * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(a.dq + rowoff + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint32_t w[4];
@@ -531,7 +551,7 @@ static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, c
   auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(a.nk_tiles, BH), 192, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<dim3(a.nk_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
   return cudaGetLastError();
 }
 
@@ -560,7 +580,7 @@ static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, con
   auto kern = attn_bwd_dq_kernel<D, QKF16>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(a.nq_tiles, BH), 192, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<dim3(a.nq_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
   return cudaGetLastError();
 }
 

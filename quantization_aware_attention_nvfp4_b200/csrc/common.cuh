@@ -8,6 +8,8 @@
 namespace attnqat {
 
 constexpr int kBM = 128;                  // query rows per tile (TMEM lanes)
+constexpr int kSoftWarps = 8;             // row warps: 2 per TMEM lane quarter, each owns 64 columns
+constexpr int kThreads = 64 + 32 * kSoftWarps;  // + producer warp + MMA warp
 constexpr int kBN = 128;                  // keys per tile
 constexpr int kChunkBytes = 128 * 128;    // one 128-row x 128-byte swizzled chunk
 constexpr float kLog2e = 1.4426950408889634f;
@@ -98,6 +100,32 @@ __device__ __forceinline__ void store_row128(uint32_t base, uint32_t row, const 
     st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
   }
 }
+
+// Writes 64 16-bit values (32 packed words) as columns [64*half, 64*half+64)
+// of row `row` of a 128 x 128 swizzled tile at `base` (exactly one chunk).
+__device__ __forceinline__ void store_row_half(uint32_t base, uint32_t row, int half, const uint32_t *w) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const uint32_t addr = base + static_cast<uint32_t>(half) * kChunkBytes + sw128_offset(row, u);
+    st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+  }
+}
+
+// Role of a row warp (warps 2 .. 2+kSoftWarps-1): the TMEM lane quarter it
+// may access (warp id mod 4), its row in the 128-row tile and which 64-column
+// half of a 128-column tile it owns.
+struct RowRole {
+  int wq;           // lane quarter
+  uint32_t row;     // 0..127
+  int half;         // 0 or 1
+  uint32_t lane_addr;
+  __device__ __forceinline__ RowRole(int warp, int lane) {
+    wq = warp & 3;
+    row = static_cast<uint32_t>(wq * 32 + lane);
+    half = (warp - 2) >> 2;
+    lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+  }
+};
 
 // Advances a dynamic shared-memory pointer to the next 1024-byte boundary of
 // the shared window (the swizzle atoms and UMMA descriptors need it).

@@ -1,13 +1,15 @@
 // fwd.cu -- Attn-QAT forward kernel for sm_100a.
 //
-// One CTA per (128-query tile, batch*head).  192 threads in three roles:
+// One CTA per (128-query tile, batch*head).  320 threads in three roles:
 //   warp 0      TMA producer: the fq(Q) tile once, then fq(K) tiles for the
 //               row-max sweep and fq(K), fq(V) tiles for the output sweep
 //               (2-stage rings, 128-byte swizzle);
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer;
-//   warps 2..5  one thread per query row (TMEM lane): row max, exp, row sum,
-//               in-register NVFP4 fq of P~ in 16-key blocks, the P tile to
-//               shared memory, and the O epilogue.
+//   warps 2..9  row warps, two per TMEM lane quarter: each query row (TMEM
+//               lane) has two threads owning 64 columns each -- row max, exp,
+//               row sum, in-register NVFP4 fq of P~ in 16-key blocks, the P
+//               tile to shared memory, and the O epilogue; the pair merges its
+//               partial max and sum through shared memory.
 // TMEM columns: S double buffer [0,256), O accumulator [256, 256+D).
 //
 // The row max is exact over all keys, taken in a first sweep of S = Q K^T,
@@ -32,7 +34,7 @@ struct FwdLayout {
   static constexpr int kV = kK + kNS * kTile;
   static constexpr int kP = kV + kNS * kTile;
   static constexpr int kBar = kP + 2 * kPBytes;
-  static constexpr int kBytes = kBar + 256;
+  static constexpr int kBytes = kBar + 2048;
   static constexpr int kDynSmem = kBytes + 1024;        // slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256;
@@ -45,44 +47,43 @@ struct FwdBars {
   uint64_t ofull;
   uint32_t tmem_slot;
   int abort;
+  float part[2][kBM];   // per-row partial max / sum of the two column halves
 };
 
-// One S tile of one row: 128 fp32 values in 4 chunks of 32 TMEM columns.
+// Row max over this thread's 64 columns (col0..col0+63) of one S tile.
 template <bool MASKED>
-__device__ __forceinline__ float row_max_tile(uint32_t taddr, int valid) {
+__device__ __forceinline__ float row_max_half(uint32_t taddr, int col0, int valid) {
+  uint32_t r[32], t[32];
+  tmem_ld32(taddr + col0, r);
+  tmem_ld32(taddr + col0 + 32, t);
+  tmem_ld_wait();
   float mx = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    if (MASKED && c * 32 >= valid) break;
-    uint32_t r[32];
-    tmem_ld32(taddr + c * 32, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float v = __uint_as_float(r[i]);
-      if (!MASKED || c * 32 + i < valid) mx = fmaxf(mx, v);
-    }
+  for (int i = 0; i < 32; ++i) {
+    if (!MASKED || col0 + i < valid) mx = fmaxf(mx, __uint_as_float(r[i]));
+    if (!MASKED || col0 + 32 + i < valid) mx = fmaxf(mx, __uint_as_float(t[i]));
   }
   return mx;
 }
 
-// Sweep-2 work for one S tile of one row: P~ = exp2(S*cl + nml), row sum,
-// fq(P~) (or P~ itself), packed into 16-bit pairs and stored as row `row`
-// of the P tile at `pbase`.
+// Sweep-2 work for this thread's 64 columns of one S tile: P~ = exp2(S*cl +
+// nml), partial row sum, fq(P~) (or P~ itself) packed into 16-bit pairs and
+// stored as columns col0..col0+63 (one swizzled chunk) of row `row` of the P
+// tile at `pbase`.
 template <int PV_F16, int QP, bool MASKED>
-__device__ __forceinline__ float prob_tile(uint32_t taddr, int valid, float cl, float nml,
+__device__ __forceinline__ float prob_half(uint32_t taddr, int col0, int valid, float cl, float nml,
                                            uint32_t pbase, uint32_t row) {
   float lsum = 0.0f;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < 2; ++c) {
     uint32_t r[32];
-    tmem_ld32(taddr + c * 32, r);
+    tmem_ld32(taddr + col0 + c * 32, r);
     tmem_ld_wait();
     float p[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float e = ex2_approx(fmaf(__uint_as_float(r[i]), cl, nml));
-      p[i] = (!MASKED || c * 32 + i < valid) ? e : 0.0f;
+      p[i] = (!MASKED || col0 + c * 32 + i < valid) ? e : 0.0f;
       lsum += p[i];
     }
     uint32_t w[16];
@@ -109,19 +110,24 @@ __device__ __forceinline__ float prob_tile(uint32_t taddr, int valid, float cl, 
                                 : pack_bf16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1]);
       }
     }
-    // 32 keys = units 4c .. 4c+3 of the 128-key row
+    // 32 keys = 16-byte units 4c .. 4c+3 of this thread's 64-key chunk
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int unit = 4 * c + u;
-      const uint32_t addr = pbase + static_cast<uint32_t>(unit >> 3) * kChunkBytes + sw128_offset(row, unit & 7);
+      const uint32_t addr = pbase + static_cast<uint32_t>(col0 >> 6) * kChunkBytes + sw128_offset(row, 4 * c + u);
       st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     }
   }
   return lsum;
 }
 
+// Merges a per-row partial value with the other column half's through
+// shared memory (named barrier 1 + lane quarter, 64 threads).
+__device__ __forceinline__ void pair_sync(int wq) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + wq) : "memory");
+}
+
 template <int D, int QKF16, int PV_F16, int QP>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using L = FwdLayout<D>;
@@ -148,8 +154,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->sfull[b], 1);
-      mbar_init(&bars->sempty[b], 4);
-      mbar_init(&bars->pfull[b], 4);
+      mbar_init(&bars->sempty[b], kSoftWarps);
+      mbar_init(&bars->pfull[b], kSoftWarps);
       mbar_init(&bars->pempty[b], 1);
     }
     mbar_init(&bars->ofull, 1);
@@ -246,10 +252,9 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(&bars->ofull);
     }
   } else {
-    // ------------------------------------------------------- softmax rows --
-    const int wq = warp & 3;
-    const uint32_t row = static_cast<uint32_t>(wq * 32 + lane);
-    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    // ---------------------------------------------------------- row warps --
+    const RowRole rr(warp, lane);
+    const int col0 = rr.half * 64;
     const int last_valid = a.Lk - (nk - 1) * kBN;  // keys in the last KV tile
     float mrow = -INFINITY;
     bool ok = true;
@@ -258,14 +263,19 @@ __global__ void __launch_bounds__(192, 1)
       const int sb = nS & 1;
       if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t taddr = tmem + lane_addr + sb * kBN;
-      const float mx = (j == nk - 1 && last_valid < kBN) ? row_max_tile<true>(taddr, last_valid)
-                                                         : row_max_tile<false>(taddr, kBN);
+      const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
+      const float mx = (j == nk - 1 && last_valid < kBN) ? row_max_half<true>(taddr, col0, last_valid)
+                                                         : row_max_half<false>(taddr, col0, kBN);
       mrow = fmaxf(mrow, mx);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty[sb]);
     }
+    // both halves of a row see every tile, so both reach this merge
+    bars->part[rr.half][rr.row] = mrow;
+    pair_sync(rr.wq);
+    mrow = fmaxf(mrow, bars->part[rr.half ^ 1][rr.row]);
+    pair_sync(rr.wq);
     const float m_scaled = mrow * a.sm_scale;
     const float nml = -(m_scaled * kLog2e);
     const float cl = a.scale_log2;
@@ -276,12 +286,12 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
       if (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t taddr = tmem + lane_addr + sb * kBN;
+      const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
       if (j == nk - 1 && last_valid < kBN)
-        lsum += prob_tile<PV_F16, QP, true>(taddr, last_valid, cl, nml, pbase, row);
+        lsum += prob_half<PV_F16, QP, true>(taddr, col0, last_valid, cl, nml, pbase, rr.row);
       else
-        lsum += prob_tile<PV_F16, QP, false>(taddr, kBN, cl, nml, pbase, row);
+        lsum += prob_half<PV_F16, QP, false>(taddr, col0, kBN, cl, nml, pbase, rr.row);
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
@@ -292,14 +302,18 @@ __global__ void __launch_bounds__(192, 1)
     }
     // ------------------------------------------------------------ epilogue --
     if (ok && mbar_wait(&bars->ofull, 0, abort)) {
+      bars->part[rr.half][rr.row] = lsum;
+      pair_sync(rr.wq);
+      lsum += bars->part[rr.half ^ 1][rr.row];
       tc_fence_after();
-      const int q = qt * kBM + static_cast<int>(row);
+      const int q = qt * kBM + static_cast<int>(rr.row);
       const float inv_l = 1.0f / lsum;
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = rr.half * (D / 2) + c * 32;
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + L::kTmemO + c * 32, r);
+        tmem_ld32(tmem + rr.lane_addr + L::kTmemO + col, r);
         tmem_ld_wait();
         if (q < a.Lq) {
           float f[32];
@@ -308,19 +322,19 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
-          uint4 *dst = reinterpret_cast<uint4 *>(a.o + rowoff + c * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(a.o + rowoff + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-          float4 *d32 = reinterpret_cast<float4 *>(a.o32 + rowoff + c * 32);
+          float4 *d32 = reinterpret_cast<float4 *>(a.o32 + rowoff + col);
 #pragma unroll
           for (int i = 0; i < 8; ++i) d32[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
         }
       }
-      if (q < a.Lq) {
+      if (q < a.Lq && rr.half == 0) {
         a.m[static_cast<size_t>(bh) * a.Lq + q] = m_scaled;
         a.lse[static_cast<size_t>(bh) * a.Lq + q] = m_scaled + logf(lsum);
       }
-    } else if (!ok || *abort) {
+    } else {
       // keep the MMA issuer's final commit from outliving the CTA
       mbar_wait_drain(&bars->ofull, 0);
     }
@@ -342,7 +356,7 @@ static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, co
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nq_tiles, BH);
-  kern<<<grid, 192, L::kDynSmem, stream>>>(tq, tk, tv, a);
+  kern<<<grid, kThreads, L::kDynSmem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 
