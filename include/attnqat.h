@@ -177,6 +177,37 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse,
                 int D, float sm_scale, uint32_t flags, void *dq, void *dk,
                 void *dv, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * attnqat_fwd_noalloc -- attnqat_fwd for callers that cannot allocate.
+ *
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that cannot hand the library a device workspace -- e.g. a framework whose
+ * caching allocator already holds nearly all device memory, code running
+ * inside an allocator or memory-pressure callback, or a plain C host without
+ * a device allocator.  It computes exactly what attnqat_fwd computes, with the
+ * same arguments minus ws/ws_bytes: the workspace is a fixed block of
+ * ATTNQAT_NOALLOC_WS_MAX bytes of device memory that the library carries as a
+ * static __device__ array (held on every GPU that loads the library, until
+ * the process exits).  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *  - Shapes with attnqat_workspace_size(...) > ATTNQAT_NOALLOC_WS_MAX return
+ *    ATTNQAT_ENOSPC; invalid shapes ATTNQAT_EINVAL (as attnqat_fwd).
+ *  - The first call on each device looks up the block's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before capturing the stream into a CUDA graph.
+ *  - All calls share the block and it keeps the last call's contents (the
+ *    parts that must start at zero are cleared on the caller's stream).
+ *    Calls whose GPU work overlaps -- two streams, or several host threads on
+ *    one device -- race on it: serialise them.
+ *  - The workspace is internal, so the result cannot be passed to
+ *    attnqat_bwd; use attnqat_fwd for training.
+ */
+#define ATTNQAT_NOALLOC_WS_MAX ((size_t)32 << 20)
+int attnqat_fwd_noalloc(const void *q, const void *k, const void *v, int B,
+                        int H, int Lq, int Lk, int D, float sm_scale,
+                        uint32_t flags, void *o, float *lse, float *m,
+                        void *stream);
+
 #ifdef __cplusplus
 }
 #endif

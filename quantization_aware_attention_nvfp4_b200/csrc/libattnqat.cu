@@ -5,3 +5,4 @@
 #include "fwd.cu"
 #include "bwd.cu"
 #include "api.cu"
+#include "noalloc.cu"
