@@ -63,10 +63,23 @@ def dist_env():
         int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings over all ranks of the default
+    process group (identity when there is none).  Every rank must call it the
+    same number of times with the same number of values."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 # ------------------------------------------------------------------ clocks --
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms while the
     timed region runs."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -81,7 +94,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -190,10 +203,7 @@ def gpu_arm(args):
     fwd_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in ev)
     bwd_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in ev)
     tot_ms = fwd_ms + bwd_ms
-    if world > 1:
-        t = torch.tensor([tot_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms, fwd_ms, bwd_ms = (float(x) for x in t.tolist())
+    tot_ms, fwd_ms, bwd_ms = max_over_ranks([tot_ms, fwd_ms, bwd_ms], dev)
 
     # ---- per-kernel durations inside the timed region (dominant kernel)
     per = {}
@@ -306,12 +316,7 @@ def e2e_arm(args, A, torch, dev, host, w, c, flags, ws, world):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
     value = world * w.nominal_flops()["total"] * n / (ms * 1e-3) / 1e12
     return {"value": round(value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": round(ms / n, 4)}
@@ -392,7 +397,7 @@ def reference_arm(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")

@@ -1,0 +1,127 @@
+"""The C ABI on a machine without a GPU: the library builds and loads, exports
+every symbol include/attnqat.h declares, and rejects bad arguments on the host
+before touching the device.  No call here reaches a CUDA launch: every case
+fails validation first (fake pointers are never dereferenced)."""
+import ctypes
+import math
+
+import pytest
+
+import quantization_aware_attention_nvfp4_b200 as A
+
+FAKE = 0x10000  # 256-byte aligned, never dereferenced: validation fails first
+
+
+def P(x):
+    return ctypes.c_void_p(x)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = A.load()
+    names = A.header_symbols()
+    assert {"attnqat_quantize", "attnqat_fwd", "attnqat_bwd", "attnqat_workspace_size",
+            "attnqat_fwd_noalloc"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_strerror_texts():
+    lib = A.load()
+    for st in (A.OK, A.EINVAL, A.EUNSUPPORTED, A.ENOSPC, A.ECUDA, A.ETIMEOUT):
+        assert lib.attnqat_strerror(st)
+    assert lib.attnqat_strerror(-99) == b"unknown status"
+
+
+def _expected_ws(B, H, Lq, Lk, D, flags):
+    """Workspace layout restated: 256-byte aligned regions for fq(Q), fq(K),
+    fq(V) (bf16), fq(V) (fp16), float32 O, Delta and 16 bytes of statistics."""
+    al = lambda x: (x + 255) // 256 * 256
+    BH = B * H
+    n = 0
+    if flags & 1:
+        n += al(BH * Lq * D * 2)
+    if flags & 2:
+        n += al(BH * Lk * D * 2)
+    if flags & 4:
+        n += 2 * al(BH * Lk * D * 2)
+    n += al(BH * Lq * D * 4) + al(BH * Lq * 4) + al(16)
+    return n
+
+
+@pytest.mark.parametrize("shape", [(1, 6, 31200, 31200, 128), (2, 3, 5, 48, 64), (1, 1, 1, 16, 128)])
+@pytest.mark.parametrize("flags", [0, 15, 4, 3])
+def test_workspace_size(shape, flags):
+    assert A.attnqat_workspace_size(*shape, flags) == _expected_ws(*shape, flags)
+
+
+@pytest.mark.parametrize("shape", [(0, 1, 16, 16, 128), (1, 1, 0, 16, 128), (1, 1, 16, 8, 128),
+                                   (1, 1, 16, 24, 128), (1, 1, 16, 16, 96), (1, 70000, 16, 16, 64)])
+def test_workspace_size_rejects_bad_shapes(shape):
+    assert A.attnqat_workspace_size(*shape, 15) == 0
+
+
+def _fwd(lib, q=FAKE, k=FAKE, v=FAKE, B=1, H=1, Lq=128, Lk=128, D=128, c=0.125, flags=15, o=FAKE,
+         lse=FAKE, m=FAKE, ws=FAKE, ws_bytes=0):
+    return lib.attnqat_fwd(P(q), P(k), P(v), B, H, Lq, Lk, D, c, flags, P(o), P(lse), P(m), P(ws),
+                           ws_bytes, None)
+
+
+def test_fwd_host_validation():
+    lib = A.load()
+    big = 1 << 30
+    assert _fwd(lib, q=0, ws_bytes=big) == A.EINVAL               # null input
+    assert _fwd(lib, o=FAKE + 2, ws_bytes=big) == A.EINVAL        # misaligned output
+    assert _fwd(lib, ws=FAKE + 16, ws_bytes=big) == A.EINVAL      # workspace not 256-byte aligned
+    assert _fwd(lib, Lk=120, ws_bytes=big) == A.EINVAL            # Lk % 16 != 0
+    assert _fwd(lib, Lk=0, ws_bytes=big) == A.EINVAL
+    assert _fwd(lib, D=96, ws_bytes=big) == A.EUNSUPPORTED        # head dimension
+    for c in (0.0, -1.0, math.inf, math.nan):                     # sm_scale used as given, must be valid
+        assert _fwd(lib, c=c, ws_bytes=big) == A.EINVAL
+    assert _fwd(lib, flags=16, ws_bytes=big) == A.EINVAL          # unknown flag bit
+    assert _fwd(lib, ws_bytes=A.attnqat_workspace_size(1, 1, 128, 128, 128, 15) - 1) == A.ENOSPC
+
+
+def test_bwd_host_validation():
+    lib = A.load()
+    big = 1 << 30
+
+    def bwd(dO=FAKE, Lk=128, ws_bytes=big, c=0.125):
+        return lib.attnqat_bwd(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(dO), 1, 1, 128, Lk, 128, c, 15,
+                               P(FAKE), P(FAKE), P(FAKE), P(FAKE), ws_bytes, None)
+    assert bwd(dO=0) == A.EINVAL
+    assert bwd(Lk=100) == A.EINVAL
+    assert bwd(c=math.nan) == A.EINVAL
+    assert bwd(ws_bytes=16) == A.ENOSPC
+
+
+def test_quantize_host_validation():
+    lib = A.load()
+
+    def quant(x=FAKE, batch=1, rows=4, cols=32, sb=0, sr=32, sc=1, codes=FAKE, scales=FAKE):
+        return lib.attnqat_quantize(P(x), batch, rows, cols, sb, sr, sc, P(codes), P(scales), None, None)
+    assert quant(x=0) == A.EINVAL
+    assert quant(codes=0) == A.EINVAL
+    assert quant(cols=24) == A.EINVAL
+    assert quant(rows=0) == A.EINVAL
+    assert quant(sr=-1) == A.EINVAL
+    assert quant(x=FAKE + 1) == A.EINVAL
+
+
+def test_noalloc_rejects_oversized_shapes_before_any_device_call():
+    lib = A.load()
+    lib.attnqat_fwd_noalloc.restype = ctypes.c_int
+    lib.attnqat_fwd_noalloc.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5 + \
+        [ctypes.c_float, ctypes.c_uint32] + [ctypes.c_void_p] * 4
+    st = lib.attnqat_fwd_noalloc(P(FAKE), P(FAKE), P(FAKE), 1, 8, 16384, 16384, 128, 0.1, 15,
+                                 P(FAKE), P(FAKE), P(FAKE), None)
+    assert st == A.ENOSPC
+    st = lib.attnqat_fwd_noalloc(P(FAKE), P(FAKE), P(FAKE), 1, 1, 16, 20, 128, 0.1, 15,
+                                 P(FAKE), P(FAKE), P(FAKE), None)
+    assert st == A.EINVAL
+
+
+def test_python_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros((1, 1, 16, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        A.attnqat_fwd(x, x, x)
