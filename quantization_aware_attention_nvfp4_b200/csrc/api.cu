@@ -140,7 +140,7 @@ static bool encode_bhld(CUtensorMap *map, const void *base, int BH, int L, int D
 // ------------------------------------------------------------- workspace --
 
 struct Workspace {
-  size_t qh, kh, vh, vh16, o32, delta, stats, total;
+  size_t qh, kh, vh, vh16, o32, delta, stats, do16, total;
 };
 
 // fq(Q) and fq(K) are exact in fp16 (values sign * E2M1 * E4M3 lie in
@@ -150,6 +150,12 @@ struct Workspace {
 static bool qk_f16(uint32_t flags) {
   return (flags & ATTNQAT_QUANT_Q) && (flags & ATTNQAT_QUANT_K);
 }
+
+// With every operand quantized, fq(V) is exact in fp16 as well, so the
+// backward runs dP and dV as fp16 MMAs on an exact fp16 copy of dO (dO * 2^e:
+// bf16 has 8 significant bits) -- dP stays exact and the dV operand
+// fq(P~)/l gets 11 significant bits instead of bf16's 8.
+static bool do_f16(uint32_t flags) { return (flags & ATTNQAT_QUANT_ALL) == ATTNQAT_QUANT_ALL; }
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -170,8 +176,10 @@ static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
   off = align256(off + BH * Lq * D * 4);
   w.delta = off;
   off = align256(off + BH * Lq * 4);
-  w.stats = off;  // [0] max_i |dO_i|_1, [1] max_i |Delta_i|, [2] max |fq(V)|
+  w.stats = off;  // [0] max_i |dO_i|_1, [1] max_i |Delta_i|, [2] max |fq(V)|, [3] max |dO_i|/l_i
   off = align256(off + 16);
+  w.do16 = off;   // exact fp16 copy dO * 2^e (all-quantized path)
+  if (do_f16(flags)) off = align256(off + BH * Lq * D * 2);
   w.total = off;
   return w;
 }
@@ -374,7 +382,10 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
   const int BH = B * H;
   float *delta = reinterpret_cast<float *>(wsb + w.delta);
   float *stats = reinterpret_cast<float *>(wsb + w.stats);
-  cudaError_t e = cudaMemsetAsync(stats, 0, 8, s);  // keeps stats[2] from the forward
+  const bool dof16 = do_f16(flags);
+  // stats[2] (max |fq(V)|) comes from the forward; the others start at zero
+  cudaError_t e = cudaMemsetAsync(stats, 0, 8, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(stats + 3, 0, 4, s);
   if (e != cudaSuccess) return cuda_fail(e);
   {
     ProfScope ps("delta", s);
@@ -382,13 +393,21 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
                      static_cast<int64_t>(BH) * Lq, D, stats, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
+  if (dof16) {
+    ProfScope ps("scale_do", s);
+    e = launch_scale_do(static_cast<const __nv_bfloat16 *>(dO), reinterpret_cast<uint16_t *>(wsb + w.do16),
+                        static_cast<int64_t>(BH) * Lq * D, stats, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   const bool f16 = qk_f16(flags);
   const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
   const void *kh = (flags & ATTNQAT_QUANT_K) ? static_cast<const void *>(wsb + w.kh) : k;
-  const void *vh = (flags & ATTNQAT_QUANT_V) ? static_cast<const void *>(wsb + w.vh) : v;
+  const void *vh = dof16 ? static_cast<const void *>(wsb + w.vh16)
+                         : (flags & ATTNQAT_QUANT_V) ? static_cast<const void *>(wsb + w.vh) : v;
+  const void *dob = dof16 ? static_cast<const void *>(wsb + w.do16) : dO;
   CUtensorMap tq, tk, tv, tdo;
   if (!encode_bhld(&tq, qh, BH, Lq, D, f16) || !encode_bhld(&tk, kh, BH, Lk, D, f16) ||
-      !encode_bhld(&tv, vh, BH, Lk, D, false) || !encode_bhld(&tdo, dO, BH, Lq, D, false))
+      !encode_bhld(&tv, vh, BH, Lk, D, dof16) || !encode_bhld(&tdo, dob, BH, Lq, D, dof16))
     return cuda_fail(cudaErrorInvalidValue);
   BwdArgs a;
   a.Lq = Lq;
@@ -406,12 +425,12 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
   a.dv = static_cast<__nv_bfloat16 *>(dv);
   {
     ProfScope ps("attn_bwd_dkdv", s);
-    e = launch_bwd_dkdv(D, f16, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, tdo, a, BH, s);
+    e = launch_bwd_dkdv(D, f16, (flags & ATTNQAT_QUANT_P) != 0, dof16, tq, tk, tv, tdo, a, BH, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   {
     ProfScope ps("attn_bwd_dq", s);
-    e = launch_bwd_dq(D, f16, tq, tk, tv, tdo, a, BH, s);
+    e = launch_bwd_dq(D, f16, dof16, tq, tk, tv, tdo, a, BH, s);
   }
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }

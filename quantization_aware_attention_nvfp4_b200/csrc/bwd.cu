@@ -155,7 +155,44 @@ __device__ __forceinline__ void dkdv_tile(uint32_t tS, uint32_t tDP, int col0, i
   }
 }
 
-template <int D, int QP, int QKF16>
+// The same for the all-quantized path with the exact fp16 copy dO * 2^e:
+// dP' = dP 2^e arrives from TMEM; the dV operand is fq(P~)/l * 2^14 in fp16
+// (r times the per-block factor s/l * 2^14: 11 significant bits, and in
+// fp16's normal range for every nonzero value while Lk <= 2^17); and
+// dS * dsc = P~/l * (dP' 2^-e - Delta) * dsc = P~ * fma(dP', a1, b1) with
+// a1 = 2^-e dsc / l, b1 = -Delta dsc / l.  Rows past Lq come in with
+// nml = -inf, so their P~ is 0 without a per-element test.
+template <bool MASKED>
+__device__ __forceinline__ void dkdv_tile_f16(uint32_t tS, uint32_t tDP, int col0, int valid_k, float cl,
+                                              float nml, float vf, float a1, float b1, uint32_t (&pw)[32],
+                                              uint32_t (&dsw)[32]) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t r[32], d[32];
+    tmem_ld32(tS + col0 + c * 32, r);
+    tmem_ld32(tDP + col0 + c * 32, d);
+    tmem_ld_wait();
+    float p[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float e = ex2_approx(fmaf(__uint_as_float(r[i]), cl, nml));
+      p[i] = (!MASKED || col0 + c * 32 + i < valid_k) ? e : 0.0f;
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      uint32_t rr[8];
+      const uint32_t s2 = f16x2_broadcast(fq16_probs(p + 16 * b, rr) * vf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pw[16 * c + 8 * b + i] = hmul2_u32(rr[i], s2);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      dsw[16 * c + i] = pack_f16x2(p[2 * i] * fmaf(__uint_as_float(d[2 * i]), a1, b1),
+                                   p[2 * i + 1] * fmaf(__uint_as_float(d[2 * i + 1]), a1, b1));
+  }
+}
+
+template <int D, int QP, int QKF16, int DOF16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -216,8 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(kBM, kBN, !QKF16, false, false);   // Q K^T
-      constexpr uint32_t idDP = idesc_f16(kBM, kBN, true, false, false);    // dO V^T (bf16)
-      constexpr uint32_t idV = idesc_f16(kBN, D, true, true, true);         // P^T dO (bf16)
+      constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
+      constexpr uint32_t idV = idesc_f16(kBN, D, !DOF16, true, true);       // P^T dO
       constexpr uint32_t idK = idesc_f16(kBN, D, !QKF16, true, true);       // dS^T Q
       const uint32_t kaddr = sbase + L::kK, vaddr = sbase + L::kV, xaddr = sbase + L::kX;
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
@@ -273,39 +310,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     float m_n, lse_n, delta_n;
     load_stats(0, m_n, lse_n, delta_n);
+    const float dos = DOF16 ? do_scale(a.stats) : 1.0f;
     for (int i = 0; i < nq; ++i) {
       const bool vq = i * kBM + static_cast<int>(rr.row) < a.Lq;
       const float m = m_n, lse = lse_n, delta = delta_n;
       load_stats(i + 1, m_n, lse_n, delta_n);
-      const float nml = -(m * kLog2e);
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
       uint32_t pw[32], dsw[32];
-      if (!mbar_wait(&bars->sfull, i & 1, abort)) { ok = false; break; }
+      if (!mbar_wait_warp(&bars->sfull, i & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      if (valid_k < kBN)
-        dkdv_tile<QP, QKF16, true>(tS, tDP, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
-      else
-        dkdv_tile<QP, QKF16, false>(tS, tDP, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
+      if (DOF16) {
+        const float nml = vq ? -(m * kLog2e) : -INFINITY;
+        const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
+        const float a1 = inv_l * dsc / dos, b1 = -delta * inv_l * dsc;
+        if (valid_k < kBN)
+          dkdv_tile_f16<true>(tS, tDP, col0, valid_k, cl, nml, vf, a1, b1, pw, dsw);
+        else
+          dkdv_tile_f16<false>(tS, tDP, col0, valid_k, cl, nml, vf, a1, b1, pw, dsw);
+      } else {
+        const float nml = -(m * kLog2e);
+        if (valid_k < kBN)
+          dkdv_tile<QP, QKF16, true>(tS, tDP, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
+        else
+          dkdv_tile<QP, QKF16, false>(tS, tDP, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
-      if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
+      if (i >= 1 && !mbar_wait_warp(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, pw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
-      if (!mbar_wait(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
+      if (!mbar_wait_warp(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
     }
-    if (ok && mbar_wait(&bars->done, 0, abort)) {
+    if (ok && mbar_wait_warp(&bars->done, 0, abort)) {
       tc_fence_after();
       // TMEM lanes of dV/dK are keys; each thread stores D/2 columns of its key row
       const int kg = kt * kBN + static_cast<int>(rr.row);
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lk + kg) * D;
       const float kscale = a.sm_scale / ds_scale<QKF16>(a.stats);  // exact: power-of-two divisor
+      const float vscale = DOF16 ? (1.0f / 16384.0f) / do_scale(a.stats) : 1.0f;  // exact: powers of two
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         const int col = rr.half * (D / 2) + c * 32;
@@ -321,7 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t w[4], x[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              w[k] = pack_bf16x2(__uint_as_float(r[8 * i + 2 * k]), __uint_as_float(r[8 * i + 2 * k + 1]));
+              w[k] = pack_bf16x2(__uint_as_float(r[8 * i + 2 * k]) * vscale,
+                                 __uint_as_float(r[8 * i + 2 * k + 1]) * vscale);
               x[k] = pack_bf16x2(__uint_as_float(s[8 * i + 2 * k]) * kscale,
                                  __uint_as_float(s[8 * i + 2 * k + 1]) * kscale);
             }
@@ -385,7 +435,31 @@ __device__ __forceinline__ void dq_tile(uint32_t tS, uint32_t tDP, int col0, int
   }
 }
 
-template <int D, int QKF16>
+// dQ-kernel tile for the exact fp16 copy dO * 2^e: dP' = dP 2^e, so
+// dS * dsc = P (dP' 2^-e - Delta) dsc = P * fma(dP', a1, b1) with
+// a1 = 2^-e dsc, b1 = -Delta dsc.  Rows past Lq come in with nlse = -inf.
+template <bool MASKED>
+__device__ __forceinline__ void dq_tile_f16(uint32_t tS, uint32_t tDP, int col0, int valid_k, float cl,
+                                            float nlse, float a1, float b1, uint32_t (&dsw)[32]) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t r[32], d[32];
+    tmem_ld32(tS + col0 + c * 32, r);
+    tmem_ld32(tDP + col0 + c * 32, d);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * i]), cl, nlse));
+      float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), cl, nlse));
+      if (MASKED && col0 + c * 32 + 2 * i >= valid_k) p0 = 0.0f;
+      if (MASKED && col0 + c * 32 + 2 * i + 1 >= valid_k) p1 = 0.0f;
+      dsw[16 * c + i] = pack_f16x2(p0 * fmaf(__uint_as_float(d[2 * i]), a1, b1),
+                                   p1 * fmaf(__uint_as_float(d[2 * i + 1]), a1, b1));
+    }
+  }
+}
+
+template <int D, int QKF16, int DOF16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -446,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(kBM, kBN, !QKF16, false, false);  // Q K^T
-      constexpr uint32_t idDP = idesc_f16(kBM, kBN, true, false, false);   // dO V^T
+      constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
       constexpr uint32_t idQ = idesc_f16(kBM, D, !QKF16, false, true);     // dS (K-major) * K (MN-major)
       const uint32_t qaddr = sbase + L::kQ, doaddr = sbase + L::kDO, xaddr = sbase + L::kX;
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
@@ -482,31 +556,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t si = static_cast<size_t>(bh) * a.Lq + (vq ? q : 0);
     const float lse = vq ? a.lse[si] : 0.0f;
     const float delta = vq ? a.delta[si] : 0.0f;
-    const float nlse = -(lse * kLog2e);
+    const float nlse = DOF16 ? (vq ? -(lse * kLog2e) : -INFINITY) : -(lse * kLog2e);
     const float cl = a.scale_log2;
     const float dsc = ds_scale<QKF16>(a.stats);
+    const float a1 = DOF16 ? dsc / do_scale(a.stats) : 0.0f;
+    const float b1 = -delta * dsc;
     const int last_valid = a.Lk - (nk - 1) * kBN;
     const uint32_t xaddr = sbase + L::kX;
     const uint32_t tS = tmem + rr.lane_addr + L::kTmemS, tDP = tmem + rr.lane_addr + L::kTmemDP;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       uint32_t dsw[32];
-      if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
+      if (!mbar_wait_warp(&bars->sfull, j & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      if (j == nk - 1 && last_valid < kBN)
-        dq_tile<QKF16, true>(tS, tDP, col0, last_valid, vq, cl, nlse, delta, dsc, dsw);
-      else
-        dq_tile<QKF16, false>(tS, tDP, col0, kBN, vq, cl, nlse, delta, dsc, dsw);
+      if (DOF16) {
+        if (j == nk - 1 && last_valid < kBN)
+          dq_tile_f16<true>(tS, tDP, col0, last_valid, cl, nlse, a1, b1, dsw);
+        else
+          dq_tile_f16<false>(tS, tDP, col0, kBN, cl, nlse, a1, b1, dsw);
+      } else {
+        if (j == nk - 1 && last_valid < kBN)
+          dq_tile<QKF16, true>(tS, tDP, col0, last_valid, vq, cl, nlse, delta, dsc, dsw);
+        else
+          dq_tile<QKF16, false>(tS, tDP, col0, kBN, vq, cl, nlse, delta, dsc, dsw);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
-      if (j >= 1 && !mbar_wait(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
+      if (j >= 1 && !mbar_wait_warp(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
     }
-    if (ok && mbar_wait(&bars->done, 0, abort)) {
+    if (ok && mbar_wait_warp(&bars->done, 0, abort)) {
       tc_fence_after();
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
       const float qscale = a.sm_scale / dsc;  // exact: power-of-two divisor
@@ -544,11 +627,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------- launchers --
 
-template <int D, int QP, int QKF16>
+template <int D, int QP, int QKF16, int DOF16>
 static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                  const CUtensorMap &tdo, const BwdArgs &a, int BH, cudaStream_t stream) {
   using L = DkdvLayout<D>;
-  auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16>;
+  auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16, DOF16>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.nk_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
@@ -556,42 +639,49 @@ static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, c
 }
 
 template <int D>
-static cudaError_t dkdv_dispatch(bool qk_f16, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
-                                 const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
-                                 cudaStream_t stream) {
+static cudaError_t dkdv_dispatch(bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
+                                 const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
+                                 const BwdArgs &a, int BH, cudaStream_t stream) {
+  if (do_f16) return launch_dkdv_t<D, 1, 1, 1>(tq, tk, tv, tdo, a, BH, stream);
   if (qk_f16)
-    return quant_p ? launch_dkdv_t<D, 1, 1>(tq, tk, tv, tdo, a, BH, stream)
-                   : launch_dkdv_t<D, 0, 1>(tq, tk, tv, tdo, a, BH, stream);
-  return quant_p ? launch_dkdv_t<D, 1, 0>(tq, tk, tv, tdo, a, BH, stream)
-                 : launch_dkdv_t<D, 0, 0>(tq, tk, tv, tdo, a, BH, stream);
+    return quant_p ? launch_dkdv_t<D, 1, 1, 0>(tq, tk, tv, tdo, a, BH, stream)
+                   : launch_dkdv_t<D, 0, 1, 0>(tq, tk, tv, tdo, a, BH, stream);
+  return quant_p ? launch_dkdv_t<D, 1, 0, 0>(tq, tk, tv, tdo, a, BH, stream)
+                 : launch_dkdv_t<D, 0, 0, 0>(tq, tk, tv, tdo, a, BH, stream);
 }
 
-cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
-                            const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
-                            cudaStream_t stream) {
-  return D == 128 ? dkdv_dispatch<128>(qk_f16, quant_p, tq, tk, tv, tdo, a, BH, stream)
-                  : dkdv_dispatch<64>(qk_f16, quant_p, tq, tk, tv, tdo, a, BH, stream);
+cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
+                            const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
+                            const BwdArgs &a, int BH, cudaStream_t stream) {
+  return D == 128 ? dkdv_dispatch<128>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, a, BH, stream)
+                  : dkdv_dispatch<64>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, a, BH, stream);
 }
 
-template <int D, int QKF16>
+template <int D, int QKF16, int DOF16>
 static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                const CUtensorMap &tdo, const BwdArgs &a, int BH, cudaStream_t stream) {
   using L = DqLayout<D>;
-  auto kern = attn_bwd_dq_kernel<D, QKF16>;
+  auto kern = attn_bwd_dq_kernel<D, QKF16, DOF16>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.nq_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_dq(int D, bool qk_f16, const CUtensorMap &tq, const CUtensorMap &tk,
+template <int D>
+static cudaError_t dq_dispatch(bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
+                               const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
+                               cudaStream_t stream) {
+  if (do_f16) return launch_dq_t<D, 1, 1>(tq, tk, tv, tdo, a, BH, stream);
+  return qk_f16 ? launch_dq_t<D, 1, 0>(tq, tk, tv, tdo, a, BH, stream)
+                : launch_dq_t<D, 0, 0>(tq, tk, tv, tdo, a, BH, stream);
+}
+
+cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
                           const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
                           cudaStream_t stream) {
-  if (D == 128)
-    return qk_f16 ? launch_dq_t<128, 1>(tq, tk, tv, tdo, a, BH, stream)
-                  : launch_dq_t<128, 0>(tq, tk, tv, tdo, a, BH, stream);
-  return qk_f16 ? launch_dq_t<64, 1>(tq, tk, tv, tdo, a, BH, stream)
-                : launch_dq_t<64, 0>(tq, tk, tv, tdo, a, BH, stream);
+  return D == 128 ? dq_dispatch<128>(qk_f16, do_f16, tq, tk, tv, tdo, a, BH, stream)
+                  : dq_dispatch<64>(qk_f16, do_f16, tq, tk, tv, tdo, a, BH, stream);
 }
 
 }  // namespace attnqat

@@ -27,7 +27,7 @@ struct Tile {
 // 8 f16x2 words of r (the grid values, sign-free) and the block scale s as a
 // float.  With s == 0 every r is 0.
 //
-// amax/6 is formed as amax * (1/6) and p/s as p * rcp(s): for probabilities
+// amax/6 is formed as amax * (1/6) and p/s as p * rcp.approx(s): for probabilities
 // (exp of a float) exact ties have measure zero, so this selects the same
 // codes as the exact quotients except within one float ulp of a rounding
 // boundary.  Forward and backward use this same routine on the same bits, so
@@ -39,7 +39,7 @@ __device__ __forceinline__ float fq16_probs(const float *p, uint32_t (&r)[8]) {
                            fmaxf(fmaxf(p[12], p[13]), fmaxf(p[14], p[15]))));
   const uint16_t code = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.0f);
   const float s = unpack_f16x2(cvt_f16x2_from_e4m3x2(code)).x;
-  const float inv = s > 0.0f ? __frcp_rn(s) : 0.0f;
+  const float inv = s > 0.0f ? rcp_approx(s) : 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) r[i] = e2m1_round_f16x2(p[2 * i] * inv, p[2 * i + 1] * inv);
   return s;
@@ -50,6 +50,16 @@ __device__ __forceinline__ float fq16_probs(const float *p, uint32_t (&r)[8]) {
 __device__ __forceinline__ uint32_t f16x2_broadcast(float s) {
   const uint32_t h = __half_as_ushort(__float2half_rn(s));
   return h | (h << 16);
+}
+
+// Power of two 2^e that maps max |dO| (stats[3]) into [2^13, 2^14): the
+// scale of the backward's exact fp16 copy of dO; 1 when dO is 0.
+__device__ __forceinline__ float do_scale(const float *stats) {
+  const float mx = stats[3];
+  if (!(mx > 0.0f)) return 1.0f;
+  int e = 13 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xFF) - 127);
+  e = e < -120 ? -120 : (e > 120 ? 120 : e);
+  return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
 }
 
 // Issues D[tmem] (+)= A * B^T for two K-major 128-row tiles (128-byte swizzle,

@@ -24,7 +24,8 @@ struct BwdArgs {
   float sm_scale;
   float scale_log2;
   // stats[0] = max_i |dO_i|_1, stats[1] = max_i |Delta_i|, stats[2] = max |fq(V)|:
-  // they bound |dS| and fix the power-of-two scale of the f16 dS operand.
+  // they bound |dS| and fix the power-of-two scale of the f16 dS operand;
+  // stats[3] = max |dO| fixes the scale of the fp16 copy of dO.
   const float *stats;
   const float *m;
   const float *lse;
@@ -43,12 +44,15 @@ cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUte
 
 // Backward dK/dV kernel (one CTA per 128-key tile) and dQ kernel (one CTA per
 // 128-query tile).  Maps over fq(Q), fq(K) (fp16 when qk_f16, else bf16),
-// fq(V) and dO (bf16).  With qk_f16 the dS operand is fp16 (scaled by a power
-// of two), else bf16.
-cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, const CUtensorMap &tq,
+// fq(V) and dO.  With qk_f16 the dS operand is fp16 (scaled by a power of
+// two), else bf16.  With do_f16 (requires qk_f16 and quantized V and P) the dO
+// map is over the exact fp16 copy dO * 2^e and the V map over fp16 fq(V): dP
+// is exact as before and dV takes fq(P~)/l * 2^14 as an fp16 operand; else
+// both maps are bf16.
+cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
                             const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
                             const BwdArgs &a, int BH, cudaStream_t stream);
-cudaError_t launch_bwd_dq(int D, bool qk_f16, const CUtensorMap &tq, const CUtensorMap &tk,
+cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
                           const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
                           cudaStream_t stream);
 
@@ -60,10 +64,14 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
                             uint16_t *deq, uint16_t *deq_f16, float *absmax, cudaStream_t stream);
 
 // delta[r] = sum_d dO[r][d] * O[r][d] over `rows` rows of D values (O float32,
-// dO bf16); folds max_r |dO_r|_1 into stats[0] and max_r |delta_r| into
-// stats[1] (both must start at 0).
+// dO bf16); folds max_r |dO_r|_1 into stats[0], max_r |delta_r| into
+// stats[1] and max |dO| into stats[3] (all must start at 0).
 cudaError_t launch_delta(const float *o32, const __nv_bfloat16 *dO, float *delta, int64_t rows, int D,
                          float *stats, cudaStream_t stream);
+
+// out = fp16(dO * 2^e) over n elements (n % 8 == 0), 2^e = do_scale(stats).
+cudaError_t launch_scale_do(const __nv_bfloat16 *dO, uint16_t *out, int64_t n, const float *stats,
+                            cudaStream_t stream);
 
 // max |x| over n bf16 values folded into *out (must start at 0).
 cudaError_t launch_absmax(const __nv_bfloat16 *x, int64_t n, float *out, cudaStream_t stream);

@@ -196,17 +196,19 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
 // row L1 norm of dO and the largest |Delta| into stats[0], stats[1]: with
 // max |fq(V)| they bound |dS| = P |dP - Delta| <= |dO_i|_1 max|fq(V)| + |Delta_i|,
 // which fixes the power-of-two scale of the backward's f16 dS operand.
+// stats[3] receives max |dO|, which fixes the power-of-two scale of the fp16
+// copy of dO.
 template <int D>
 __global__ void __launch_bounds__(256)
     delta_kernel(const float4 *__restrict__ o32, const uint4 *__restrict__ dO, float *__restrict__ delta,
                  int64_t rows, float *__restrict__ stats) {
   constexpr int kLanes = D / 8;
-  float dmax = 0.0f, gmax = 0.0f;
+  float dmax = 0.0f, gmax = 0.0f, smax = 0.0f;
   const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x / kLanes;
   for (int64_t row = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) / kLanes;
        row - ((threadIdx.x & 31) / kLanes) < rows; row += step) {
     const int sub = static_cast<int>(threadIdx.x % kLanes);
-    float acc = 0.0f, l1 = 0.0f;
+    float acc = 0.0f, l1 = 0.0f, amax = 0.0f;
     if (row < rows) {
       const float4 a0 = __ldg(o32 + (row * kLanes + sub) * 2);
       const float4 a1 = __ldg(o32 + (row * kLanes + sub) * 2 + 1);
@@ -219,21 +221,25 @@ __global__ void __launch_bounds__(256)
         acc = fmaf(av[2 * i], lo, acc);
         acc = fmaf(av[2 * i + 1], hi, acc);
         l1 += fabsf(lo) + fabsf(hi);
+        amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
       }
     }
 #pragma unroll
     for (int off = kLanes / 2; off > 0; off >>= 1) {
       acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
       l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, off);
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
     }
     if (row < rows) {
       if (sub == 0) delta[row] = acc;
       dmax = fmaxf(dmax, l1);
       gmax = fmaxf(gmax, fabsf(acc));
+      smax = fmaxf(smax, amax);
     }
   }
   block_max_to_global(dmax, stats);
   block_max_to_global(gmax, stats + 1);
+  block_max_to_global(smax, stats + 3);
 }
 
 cudaError_t launch_delta(const float *o32, const __nv_bfloat16 *dO, float *delta, int64_t rows, int D,
@@ -252,6 +258,40 @@ cudaError_t launch_delta(const float *o32, const __nv_bfloat16 *dO, float *delta
   else
     delta_kernel<64><<<blocks, threads, 0, stream>>>(reinterpret_cast<const float4 *>(o32),
                                                      reinterpret_cast<const uint4 *>(dO), delta, rows, stats);
+  return cudaGetLastError();
+}
+
+// dO' = fp16(dO * 2^e) with 2^e = do_scale(stats) (max |dO| lands in
+// [2^13, 2^14)).  bf16 values carry 8 significant bits, so the fp16 copy is
+// exact for every element within 2^27 of the largest.  8 elements per
+// thread, grid-stride.
+__global__ void __launch_bounds__(256)
+    scale_do_kernel(const uint4 *__restrict__ dO, uint4 *__restrict__ out, int64_t n8,
+                    const float *__restrict__ stats) {
+  const float sc = do_scale(stats);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 b = __ldg(dO + i);
+    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[k] = pack_f16x2(__uint_as_float(bw[k] << 16) * sc, __uint_as_float(bw[k] & 0xFFFF0000u) * sc);
+    out[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+cudaError_t launch_scale_do(const __nv_bfloat16 *dO, uint16_t *out, int64_t n, const float *stats,
+                            cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t n8 = n / 8;
+  const int64_t need = (n8 + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  scale_do_kernel<<<static_cast<unsigned>(need < cap ? need : cap), 256, 0, stream>>>(
+      reinterpret_cast<const uint4 *>(dO), reinterpret_cast<uint4 *>(out), n8, stats);
   return cudaGetLastError();
 }
 

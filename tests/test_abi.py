@@ -34,7 +34,8 @@ def test_strerror_texts():
 
 def _expected_ws(B, H, Lq, Lk, D, flags):
     """Workspace layout restated: 256-byte aligned regions for fq(Q), fq(K),
-    fq(V) (bf16), fq(V) (fp16), float32 O, Delta and 16 bytes of statistics."""
+    fq(V) (bf16), fq(V) (fp16), float32 O, Delta, 16 bytes of statistics and,
+    with every quantizer on, the fp16 copy of dO."""
     al = lambda x: (x + 255) // 256 * 256
     BH = B * H
     n = 0
@@ -45,6 +46,8 @@ def _expected_ws(B, H, Lq, Lk, D, flags):
     if flags & 4:
         n += 2 * al(BH * Lk * D * 2)
     n += al(BH * Lq * D * 4) + al(BH * Lq * 4) + al(16)
+    if flags & 15 == 15:
+        n += al(BH * Lq * D * 2)  # fp16 copy of dO for the all-quantized backward
     return n
 
 
