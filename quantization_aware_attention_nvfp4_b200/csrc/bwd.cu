@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_stats(i + 1, m_n, lse_n, delta_n);
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
       uint32_t pw[32], dsw[32];
-      if (!mbar_wait_warp(&bars->sfull, i & 1, abort)) { ok = false; break; }
+      if (!mbar_wait(&bars->sfull, i & 1, abort)) { ok = false; break; }
       tc_fence_after();
       if (DOF16) {
         const float nml = vq ? -(m * kLog2e) : -INFINITY;
@@ -337,18 +337,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
-      if (i >= 1 && !mbar_wait_warp(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
+      if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, pw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
-      if (!mbar_wait_warp(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
+      if (!mbar_wait(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
     }
-    if (ok && mbar_wait_warp(&bars->done, 0, abort)) {
+    if (ok && mbar_wait(&bars->done, 0, abort)) {
       tc_fence_after();
       // TMEM lanes of dV/dK are keys; each thread stores D/2 columns of its key row
       const int kg = kt * kBN + static_cast<int>(rr.row);
@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       uint32_t dsw[32];
-      if (!mbar_wait_warp(&bars->sfull, j & 1, abort)) { ok = false; break; }
+      if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
       tc_fence_after();
       if (DOF16) {
         if (j == nk - 1 && last_valid < kBN)
@@ -583,13 +583,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
-      if (j >= 1 && !mbar_wait_warp(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
+      if (j >= 1 && !mbar_wait(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
     }
-    if (ok && mbar_wait_warp(&bars->done, 0, abort)) {
+    if (ok && mbar_wait(&bars->done, 0, abort)) {
       tc_fence_after();
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
       const float qscale = a.sm_scale / dsc;  // exact: power-of-two divisor

@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int nS = 0;
     for (int j = 0; j < nk; ++j, ++nS) {
       const int sb = nS & 1;
-      if (!mbar_wait_warp(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
+      if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const float mx = (j == nk - 1 && last_valid < kBN) ? row_max_half<true>(taddr, col0, last_valid)
@@ -283,8 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; ok && j < nk; ++j, ++nS) {
       const int sb = nS & 1;
       const int pb = j & 1;
-      if (!mbar_wait_warp(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
-      if (j >= 2 && !mbar_wait_warp(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
+      if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
+      if (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ------------------------------------------------------------ epilogue --
-    if (ok && mbar_wait_warp(&bars->ofull, 0, abort)) {
+    if (ok && mbar_wait(&bars->ofull, 0, abort)) {
       bars->part[rr.half][rr.row] = lsum;
       pair_sync(rr.wq);
       lsum += bars->part[rr.half ^ 1][rr.row];
