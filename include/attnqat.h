@@ -132,10 +132,14 @@ int attnqat_quantize(const void *x, int64_t batch, int64_t rows, int64_t cols,
 /*
  * attnqat_workspace_size -- bytes of device workspace attnqat_fwd and
  * attnqat_bwd need for this shape and flag set (0 for invalid shapes).  The
- * workspace holds the dequantized fq(Q), fq(K), fq(V) operands (bf16, plus an
- * fp16 copy of fq(V) for the forward's P V product -- every fq'd value is
- * exact in both), a float32 copy of O written by the forward, and the
- * backward's Delta; every region is 256-byte aligned.
+ * workspace holds the dequantized fq(Q), fq(K), fq(V) operands (fp16 when
+ * both Q and K are quantized, else bf16, plus an fp16 copy of fq(V) for the
+ * P V product -- every fq'd value is exact in both), a float32 copy of O
+ * written by the forward, the backward's Delta, 16 bytes of statistics, an
+ * exact fp16 copy of dO * 2^e when all four quantizers are on, and -- with Q
+ * and K quantized -- their packed NVFP4 codes (D/2 bytes per row) with scale
+ * tiles (512 bytes per 128 rows x 64 columns) for the forward's block-scaled
+ * S = fq(Q) fq(K)^T.  Every region is 256-byte aligned.
  */
 size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D,
                               uint32_t flags);

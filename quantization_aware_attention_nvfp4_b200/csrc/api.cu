@@ -137,10 +137,29 @@ static bool encode_bhld(CUtensorMap *map, const void *base, int BH, int L, int D
   return r == CUDA_SUCCESS;
 }
 
+// 3-D map over packed NVFP4 codes [BH][L][D/2 bytes]: whole rows of D/2 bytes
+// x 128 rows per box, swizzled by the row width (64 B for D = 128, 32 B for
+// D = 64) as the block-scaled MMA's K-major descriptors expect; rows past L
+// read as zeros.
+static bool encode_codes(CUtensorMap *map, const void *base, int BH, int L, int D) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(D) / 2;
+  cuuint64_t dims[3] = {row, static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {row, static_cast<cuuint64_t>(L) * row};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(row), 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------- workspace --
 
 struct Workspace {
-  size_t qh, kh, vh, vh16, o32, delta, stats, do16, total;
+  size_t qh, kh, vh, vh16, o32, delta, stats, do16, qc, qsf, kc, ksf, total;
+  size_t qsf_bytes, ksf_bytes;
 };
 
 // fq(Q) and fq(K) are exact in fp16 (values sign * E2M1 * E4M3 lie in
@@ -180,6 +199,20 @@ static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
   off = align256(off + 16);
   w.do16 = off;   // exact fp16 copy dO * 2^e (all-quantized path)
   if (do_f16(flags)) off = align256(off + BH * Lq * D * 2);
+  // packed NVFP4 codes of fq(Q), fq(K) and their scales in 128-row tiles
+  // (512 bytes per 128 rows x 64 columns), read by the forward's S MMA
+  const size_t ntq = (static_cast<size_t>(Lq) + 127) / 128, ntk = (static_cast<size_t>(Lk) + 127) / 128;
+  w.qsf_bytes = BH * ntq * (D / 64) * 512;
+  w.ksf_bytes = BH * ntk * (D / 64) * 512;
+  const bool fp4 = qk_f16(flags);
+  w.qc = off;
+  if (fp4) off = align256(off + BH * Lq * D / 2);
+  w.qsf = off;
+  if (fp4) off = align256(off + w.qsf_bytes);
+  w.kc = off;
+  if (fp4) off = align256(off + BH * Lk * D / 2);
+  w.ksf = off;
+  if (fp4) off = align256(off + w.ksf_bytes);
   w.total = off;
   return w;
 }
@@ -207,19 +240,31 @@ static int prepare_operands(const void *q, const void *k, const void *v, int B, 
   float *stats = reinterpret_cast<float *>(ws + w.stats);
   cudaError_t e = cudaMemsetAsync(stats, 0, 16, stream);
   if (e != cudaSuccess) return cuda_fail(e);
+  // With Q and K both quantized one pass writes the exact fp16 fq (for the
+  // backward) and the packed codes with tiled scales (for the forward's S);
+  // scale tiles are cleared first when the last 128-row tile is partial, so
+  // its padding rows carry zero scales.
+  auto quant_qk = [&](const void *x, int L, size_t deq_off, size_t c_off, size_t sf_off, size_t sf_bytes,
+                      const char *name) -> int {
+    uint16_t *dst = reinterpret_cast<uint16_t *>(ws + deq_off);
+    if (f16 && (L % 128) != 0) {
+      cudaError_t em = cudaMemsetAsync(ws + sf_off, 0, sf_bytes, stream);
+      if (em != cudaSuccess) return cuda_fail(em);
+    }
+    ProfScope ps(name, stream);
+    cudaError_t eq = launch_quantize(static_cast<const uint16_t *>(x), 1, BH * L, D, 0, D, 1,
+                                     f16 ? ws + c_off : nullptr, f16 ? ws + sf_off : nullptr,
+                                     f16 ? nullptr : dst, f16 ? dst : nullptr, nullptr, stream,
+                                     f16 ? L : 0);
+    return eq == cudaSuccess ? ATTNQAT_OK : cuda_fail(eq);
+  };
   if (flags & ATTNQAT_QUANT_Q) {
-    uint16_t *dst = reinterpret_cast<uint16_t *>(ws + w.qh);
-    ProfScope ps("quantize_q", stream);
-    e = launch_quantize(static_cast<const uint16_t *>(q), 1, BH * Lq, D, 0, D, 1, nullptr, nullptr,
-                        f16 ? nullptr : dst, f16 ? dst : nullptr, nullptr, stream);
-    if (e != cudaSuccess) return cuda_fail(e);
+    const int st = quant_qk(q, Lq, w.qh, w.qc, w.qsf, w.qsf_bytes, "quantize_q");
+    if (st != ATTNQAT_OK) return st;
   }
   if (flags & ATTNQAT_QUANT_K) {
-    uint16_t *dst = reinterpret_cast<uint16_t *>(ws + w.kh);
-    ProfScope ps("quantize_k", stream);
-    e = launch_quantize(static_cast<const uint16_t *>(k), 1, BH * Lk, D, 0, D, 1, nullptr, nullptr,
-                        f16 ? nullptr : dst, f16 ? dst : nullptr, nullptr, stream);
-    if (e != cudaSuccess) return cuda_fail(e);
+    const int st = quant_qk(k, Lk, w.kh, w.kc, w.ksf, w.ksf_bytes, "quantize_k");
+    if (st != ATTNQAT_OK) return st;
   }
   if (flags & ATTNQAT_QUANT_V) {
     // blocks of 16 consecutive tokens per channel: the transposed view
@@ -341,9 +386,9 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   const void *vh = pv_f16 ? static_cast<const void *>(wsb + w.vh16) : v;
   const bool f16 = qk_f16(flags);
   CUtensorMap tq, tk, tv;
-  if (!encode_bhld(&tq, qh, BH, Lq, D, f16) || !encode_bhld(&tk, kh, BH, Lk, D, f16) ||
-      !encode_bhld(&tv, vh, BH, Lk, D, pv_f16))
-    return cuda_fail(cudaErrorInvalidValue);
+  const bool maps_ok = f16 ? encode_codes(&tq, wsb + w.qc, BH, Lq, D) && encode_codes(&tk, wsb + w.kc, BH, Lk, D)
+                           : encode_bhld(&tq, qh, BH, Lq, D, false) && encode_bhld(&tk, kh, BH, Lk, D, false);
+  if (!maps_ok || !encode_bhld(&tv, vh, BH, Lk, D, pv_f16)) return cuda_fail(cudaErrorInvalidValue);
   FwdArgs a;
   a.Lq = Lq;
   a.Lk = Lk;
@@ -351,6 +396,8 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   a.nk_tiles = (Lk + kBN - 1) / kBN;
   a.sm_scale = sm_scale;
   a.scale_log2 = sm_scale * kLog2e;
+  a.qsf = wsb + w.qsf;
+  a.ksf = wsb + w.ksf;
   a.o = static_cast<__nv_bfloat16 *>(o);
   a.o32 = reinterpret_cast<float *>(wsb + w.o32);
   a.lse = lse;

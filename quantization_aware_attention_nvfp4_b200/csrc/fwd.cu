@@ -24,25 +24,41 @@
 
 namespace attnqat {
 
-template <int D>
+// Shared-memory and TMEM layout of the forward.  With FP4S the Q and K tiles
+// are packed NVFP4 codes (D/2 bytes per row, TMA swizzle of D/2 bytes) and
+// their 16-element scales (512-byte scale-factor blocks per 64 columns); S is
+// then a block-scaled kind::mxf4nvf4 MMA.  Otherwise Q and K are 16-bit tiles.
+template <int D, int FP4S>
 struct FwdLayout {
-  static constexpr int kNS = 2;                         // K and V ring stages
-  static constexpr int kTile = Tile<D>::kBytes;
+  static constexpr int kNSK = FP4S ? 4 : 2;             // K ring stages
+  static constexpr int kNSV = 2;                        // V ring stages
+  static constexpr int kQKRow = FP4S ? D / 2 : 2 * D;   // bytes per Q/K row
+  static constexpr int kQK = 128 * kQKRow;              // bytes per Q/K tile
+  static constexpr int kSF = FP4S ? (D / 64) * 512 : 0;  // scale-factor bytes per tile
+  static constexpr int kVT = Tile<D>::kBytes;
   static constexpr int kPBytes = kBM * kBN * 2;
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTile;
-  static constexpr int kV = kK + kNS * kTile;
-  static constexpr int kP = kV + kNS * kTile;
-  static constexpr int kBar = kP + 2 * kPBytes;
+  static constexpr int kK = kQ + kQK;
+  static constexpr int kV = (kK + kNSK * kQK + 1023) / 1024 * 1024;
+  static constexpr int kP = kV + kNSV * kVT;
+  static constexpr int kQSF = kP + 2 * kPBytes;
+  static constexpr int kKSF = kQSF + kSF;
+  static constexpr int kBar = kKSF + kNSK * kSF;
   static constexpr int kBytes = kBar + 2048;
   static constexpr int kDynSmem = kBytes + 1024;        // slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256;
+  static constexpr uint32_t kSFCols = (D / 64) * 4;     // TMEM columns of one tile's scales
+  static constexpr uint32_t kTmemSFA = 256 + D;
+  static constexpr uint32_t kTmemSFB = kTmemSFA + kSFCols;  // kNSK stages
+  // UMMA layout of the packed tiles: 64-byte rows swizzle 64B, 32-byte rows 32B
+  static constexpr uint32_t kCodeLayout = (D / 2 == 64) ? 4u : 6u;
+  static constexpr uint32_t kCodeSBO = 8 * (D / 2);
 };
 
 struct FwdBars {
   uint64_t qfull;
-  uint64_t kfull[2], kempty[2], vfull[2], vempty[2];
+  uint64_t kfull[4], kempty[4], vfull[2], vempty[2];
   uint64_t sfull[2], sempty[2], pfull[2], pempty[2];
   uint64_t ofull;
   uint32_t tmem_slot;
@@ -126,12 +142,12 @@ __device__ __forceinline__ void pair_sync(int wq) {
   asm volatile("bar.sync %0, 64;" ::"r"(1 + wq) : "memory");
 }
 
-template <int D, int QKF16, int PV_F16, int QP>
+template <int D, int FP4S, int PV_F16, int QP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
-  using L = FwdLayout<D>;
-  constexpr int kNS = L::kNS;
+  using L = FwdLayout<D, FP4S>;
+  constexpr int kNSK = L::kNSK, kNSV = L::kNSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
@@ -146,9 +162,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
-    for (int s = 0; s < kNS; ++s) {
+    for (int s = 0; s < kNSK; ++s) {
       mbar_init(&bars->kfull[s], 1);
       mbar_init(&bars->kempty[s], 1);
+    }
+    for (int s = 0; s < kNSV; ++s) {
       mbar_init(&bars->vfull[s], 1);
       mbar_init(&bars->vempty[s], 1);
     }
@@ -177,53 +195,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(&bars->qfull, L::kTile);
-      for (int c = 0; c < Tile<D>::kChunks; ++c)
-        tma_load_3d(smem + L::kQ + c * kChunkBytes, &tmQ, &bars->qfull, c * 64, qt * kBM, bh);
+      // Q (or its packed codes and scales) once
+      auto load_qk = [&](uint8_t *dst, const CUtensorMap *map, uint64_t *bar, int row0) {
+        if (FP4S) {
+          tma_load_3d(dst, map, bar, 0, row0, bh);
+        } else {
+          for (int c = 0; c < Tile<D>::kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, map, bar, c * 64, row0, bh);
+        }
+      };
+      mbar_arrive_expect_tx(&bars->qfull, L::kQK + L::kSF);
+      load_qk(smem + L::kQ, &tmQ, &bars->qfull, qt * kBM);
+      if (FP4S)
+        bulk_load(smem + L::kQSF, a.qsf + (static_cast<size_t>(bh) * a.nq_tiles + qt) * L::kSF, L::kSF,
+                  &bars->qfull);
       int kissued = 0, vissued = 0;
       for (int t = 0; t < 2 * nk; ++t) {
         const int j = t < nk ? t : t - nk;
-        const int st = t % kNS;
-        if (t >= kNS && !mbar_wait(&bars->kempty[st], ((t / kNS) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&bars->kfull[st], L::kTile);
-        for (int c = 0; c < Tile<D>::kChunks; ++c)
-          tma_load_3d(smem + L::kK + st * L::kTile + c * kChunkBytes, &tmK, &bars->kfull[st], c * 64,
-                      j * kBN, bh);
+        const int st = t % kNSK;
+        if (t >= kNSK && !mbar_wait(&bars->kempty[st], ((t / kNSK) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->kfull[st], L::kQK + L::kSF);
+        load_qk(smem + L::kK + st * L::kQK, &tmK, &bars->kfull[st], j * kBN);
+        if (FP4S)
+          bulk_load(smem + L::kKSF + st * L::kSF, a.ksf + (static_cast<size_t>(bh) * nk + j) * L::kSF, L::kSF,
+                    &bars->kfull[st]);
         kissued = t + 1;
         if (t >= nk) {
           const int u = t - nk;
-          const int vs = u % kNS;
-          if (u >= kNS && !mbar_wait(&bars->vempty[vs], ((u / kNS) - 1) & 1, abort)) break;
-          mbar_arrive_expect_tx(&bars->vfull[vs], L::kTile);
+          const int vs = u % kNSV;
+          if (u >= kNSV && !mbar_wait(&bars->vempty[vs], ((u / kNSV) - 1) & 1, abort)) break;
+          mbar_arrive_expect_tx(&bars->vfull[vs], L::kVT);
           for (int c = 0; c < Tile<D>::kChunks; ++c)
-            tma_load_3d(smem + L::kV + vs * L::kTile + c * kChunkBytes, &tmV, &bars->vfull[vs],
+            tma_load_3d(smem + L::kV + vs * L::kVT + c * kChunkBytes, &tmV, &bars->vfull[vs],
                         c * 64, j * kBN, bh);
           vissued = u + 1;
         }
       }
       if (*abort) {
         // let the copies already issued land before the CTA exits
-        for (int t = (kissued > kNS ? kissued - kNS : 0); t < kissued; ++t)
-          mbar_wait_drain(&bars->kfull[t % kNS], (t / kNS) & 1);
-        for (int u = (vissued > kNS ? vissued - kNS : 0); u < vissued; ++u)
-          mbar_wait_drain(&bars->vfull[u % kNS], (u / kNS) & 1);
+        for (int t = (kissued > kNSK ? kissued - kNSK : 0); t < kissued; ++t)
+          mbar_wait_drain(&bars->kfull[t % kNSK], (t / kNSK) & 1);
+        for (int u = (vissued > kNSV ? vissued - kNSV : 0); u < vissued; ++u)
+          mbar_wait_drain(&bars->vfull[u % kNSV], (u / kNSV) & 1);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_f16(kBM, kBN, !QKF16, false, false);
+      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);
       constexpr uint32_t idPV = idesc_f16(kBM, D, !PV_F16, false, true);
       const uint32_t qaddr = sbase + L::kQ;
       bool ok = mbar_wait(&bars->qfull, 0, abort);
+      if (ok && FP4S) {
+        // scales of the Q tile into TMEM once (tcgen05 ops of this thread run in order)
+        tc_fence_after();
+        for (int kc = 0; kc < D / 64; ++kc)
+          tmem_cp_32x128b_x4(tmem + L::kTmemSFA + kc * 4, sdesc_make(sbase + L::kQSF + kc * 512, 16, 128, 0));
+      }
       int nS = 0;  // S tiles issued so far (both sweeps)
       auto issue_s = [&](int t) -> bool {
-        const int st = t % kNS;
+        const int st = t % kNSK;
         const int sb = nS & 1;
         if (nS >= 2 && !mbar_wait(&bars->sempty[sb], ((nS >> 1) - 1) & 1, abort)) return false;
-        if (!mbar_wait(&bars->kfull[st], (t / kNS) & 1, abort)) return false;
+        if (!mbar_wait(&bars->kfull[st], (t / kNSK) & 1, abort)) return false;
         tc_fence_after();
-        mma_kmajor(tmem + sb * kBN, qaddr, sbase + L::kK + st * L::kTile, D / 16, idS, false);
+        const uint32_t kaddr = sbase + L::kK + st * L::kQK;
+        if (FP4S) {
+          const uint32_t sfb = tmem + L::kTmemSFB + st * L::kSFCols;
+          for (int kc = 0; kc < D / 64; ++kc)
+            tmem_cp_32x128b_x4(sfb + kc * 4, sdesc_make(sbase + L::kKSF + st * L::kSF + kc * 512, 16, 128, 0));
+          for (int kk = 0; kk < D / 64; ++kk)
+            umma_fp4(tmem + sb * kBN, sdesc_make(qaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout),
+                     sdesc_make(kaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout), idS,
+                     tmem + L::kTmemSFA + kk * 4, sfb + kk * 4, kk > 0 ? 1u : 0u);
+        } else {
+          mma_kmajor(tmem + sb * kBN, qaddr, kaddr, D / 16, idS, false);
+        }
         umma_commit(&bars->kempty[st]);
         umma_commit(&bars->sfull[sb]);
         ++nS;
@@ -231,12 +277,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int j) -> bool {
         const int pb = j & 1;
-        const int vs = j % kNS;
+        const int vs = j % kNSV;
         if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, abort)) return false;
-        if (!mbar_wait(&bars->vfull[vs], (j / kNS) & 1, abort)) return false;
+        if (!mbar_wait(&bars->vfull[vs], (j / kNSV) & 1, abort)) return false;
         tc_fence_after();
         mma_a_k_b_mn(tmem + L::kTmemO, sbase + L::kP + pb * L::kPBytes,
-                     sbase + L::kV + vs * L::kTile, kBN / 16, idPV, j > 0);
+                     sbase + L::kV + vs * L::kVT, kBN / 16, idPV, j > 0);
         umma_commit(&bars->vempty[vs]);
         umma_commit(&bars->pempty[pb]);
         return true;
@@ -348,11 +394,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int QKF16, int PV_F16, int QP>
+template <int D, int FP4S, int PV_F16, int QP>
 static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const FwdArgs &a, int BH, cudaStream_t stream) {
-  using L = FwdLayout<D>;
-  auto kern = attn_fwd_kernel<D, QKF16, PV_F16, QP>;
+  using L = FwdLayout<D, FP4S>;
+  static_assert(L::kDynSmem <= 232448, "forward shared memory over the 227 KB limit");
+  static_assert(!FP4S || L::kTmemSFB + L::kNSK * L::kSFCols <= L::kTmemCols, "forward TMEM over 512 columns");
+  auto kern = attn_fwd_kernel<D, FP4S, PV_F16, QP>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nq_tiles, BH);
@@ -360,19 +408,20 @@ static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, co
   return cudaGetLastError();
 }
 
-template <int D, int QKF16>
+template <int D, int FP4S>
 static cudaError_t fwd_dispatch(bool pv_f16, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, const FwdArgs &a, int BH, cudaStream_t stream) {
   if (pv_f16)
-    return quant_p ? launch_fwd_t<D, QKF16, 1, 1>(tq, tk, tv, a, BH, stream)
-                   : launch_fwd_t<D, QKF16, 1, 0>(tq, tk, tv, a, BH, stream);
-  return quant_p ? launch_fwd_t<D, QKF16, 0, 1>(tq, tk, tv, a, BH, stream)
-                 : launch_fwd_t<D, QKF16, 0, 0>(tq, tk, tv, a, BH, stream);
+    return quant_p ? launch_fwd_t<D, FP4S, 1, 1>(tq, tk, tv, a, BH, stream)
+                   : launch_fwd_t<D, FP4S, 1, 0>(tq, tk, tv, a, BH, stream);
+  return quant_p ? launch_fwd_t<D, FP4S, 0, 1>(tq, tk, tv, a, BH, stream)
+                 : launch_fwd_t<D, FP4S, 0, 0>(tq, tk, tv, a, BH, stream);
 }
 
 cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUtensorMap &tq,
                        const CUtensorMap &tk, const CUtensorMap &tv, const FwdArgs &a, int BH,
                        cudaStream_t stream) {
+  // quantized Q and K: S runs on the NVFP4 tensor-core path
   if (D == 128)
     return qk_f16 ? fwd_dispatch<128, 1>(pv_f16, quant_p, tq, tk, tv, a, BH, stream)
                   : fwd_dispatch<128, 0>(pv_f16, quant_p, tq, tk, tv, a, BH, stream);

@@ -13,6 +13,8 @@ struct FwdArgs {
   int Lq, Lk, nq_tiles, nk_tiles;
   float sm_scale;     // c
   float scale_log2;   // c * log2(e)
+  const uint8_t *qsf;   // scale-factor tiles of fq(Q), fq(K) (NVFP4 S path)
+  const uint8_t *ksf;
   __nv_bfloat16 *o;
   float *o32;   // float32 copy of O kept in the workspace for the backward's Delta
   float *lse;
@@ -35,9 +37,11 @@ struct BwdArgs {
   __nv_bfloat16 *dv;
 };
 
-// Forward.  tq/tk/tv: 3-D TMA maps {D, L, B*H} with 64 x 128 boxes, 128-byte
-// swizzle, over fq(Q), fq(K) (fp16 when qk_f16, else bf16) and fq(V) (fp16
-// when pv_f16, else bf16).
+// Forward.  tv: 3-D TMA map {D, L, B*H} with 64 x 128 boxes, 128-byte swizzle
+// over fq(V) (fp16 when pv_f16, else bf16).  With qk_f16 (Q and K quantized)
+// tq/tk map the packed NVFP4 codes {D/2 bytes, L, B*H} with (D/2) x 128 boxes
+// and a D/2-byte swizzle, a.qsf/a.ksf point at their scale-factor tiles, and S
+// runs as a block-scaled NVFP4 MMA; otherwise tq/tk map the bf16 Q and K.
 cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUtensorMap &tq,
                        const CUtensorMap &tk, const CUtensorMap &tv, const FwdArgs &a, int BH,
                        cudaStream_t stream);
@@ -58,10 +62,14 @@ cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq
 
 // NVFP4 fq of a strided bf16 view (see attnqat_quantize); any of codes,
 // scales, deq (bf16, same strides as x), deq_f16 and absmax (max |fq(x)|,
-// folded in with an atomic max; must start at 0) may be null.
+// folded in with an atomic max; must start at 0) may be null.  With
+// sf_tile_rows = L > 0 (contiguous [heads*L, cols] rows), the scales go to
+// the per-head, per-128-row-tile layout the block-scaled MMA reads from TMEM
+// (padding rows of the last tile are not written).
 cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols,
                             int64_t sb, int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales,
-                            uint16_t *deq, uint16_t *deq_f16, float *absmax, cudaStream_t stream);
+                            uint16_t *deq, uint16_t *deq_f16, float *absmax, cudaStream_t stream,
+                            int64_t sf_tile_rows = 0);
 
 // delta[r] = sum_d dO[r][d] * O[r][d] over `rows` rows of D values (O float32,
 // dO bf16); folds max_r |dO_r|_1 into stats[0], max_r |delta_r| into

@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256)
     quantize_view_kernel(const uint16_t *__restrict__ x, int64_t batch, int64_t rows, int64_t cols,
                          int64_t sb, int64_t sr, int64_t sc, uint8_t *__restrict__ codes,
                          uint8_t *__restrict__ scales, uint16_t *__restrict__ deq,
-                         uint16_t *__restrict__ deq_f16, float *__restrict__ absmax) {
+                         uint16_t *__restrict__ deq_f16, float *__restrict__ absmax, int64_t sf_tile_rows) {
   const int64_t nblk = cols / 16;
   float vmax = 0.0f;  // largest dequantized magnitude this thread produced
   const int64_t total = batch * rows * nblk;
@@ -156,7 +156,21 @@ __global__ void __launch_bounds__(256)
     fq16_exact(v, nib, scode, bb, hb);
     const int64_t blk = (z * rows + r) * nblk + b;
     if (codes) *reinterpret_cast<uint2 *>(codes + blk * 8) = make_uint2(nib[0], nib[1]);
-    if (scales) scales[blk] = static_cast<uint8_t>(scode);
+    if (scales) {
+      if (sf_tile_rows > 0) {
+        // scale-factor tile layout read by tcgen05.cp 32x128b.warpx4: per head,
+        // per 128-row tile, per 64-column chunk a 512-byte block in which row
+        // t (m0 = t % 32, m1 = t / 32 within the tile) holds its four 16-column
+        // scales at bytes m0*16 + m1*4 + (0..3)
+        const int64_t head = r / sf_tile_rows, t = r % sf_tile_rows;
+        const int64_t ntiles = (sf_tile_rows + 127) / 128;
+        const int64_t off = ((head * ntiles + (t >> 7)) * (nblk >> 2) + (b >> 2)) * 512 + (t & 31) * 16 +
+                            ((t & 127) >> 5) * 4 + (b & 3);
+        scales[off] = static_cast<uint8_t>(scode);
+      } else {
+        scales[blk] = static_cast<uint8_t>(scode);
+      }
+    }
     if (deq) store16(deq, base, sc, bb);
     if (deq_f16) store16(deq_f16, base, sc, hb);
     if (absmax) {
@@ -169,7 +183,7 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols, int64_t sb,
                             int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales, uint16_t *deq,
-                            uint16_t *deq_f16, float *absmax, cudaStream_t stream) {
+                            uint16_t *deq_f16, float *absmax, cudaStream_t stream, int64_t sf_tile_rows) {
   const int64_t total = batch * rows * (cols / 16);
   if (total == 0) return cudaSuccess;
   int dev = 0, sms = 148;
@@ -182,10 +196,10 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
   const bool row_fastest = (sc != 1) && (sr == 1);
   if (row_fastest)
     quantize_view_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax);
+        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax, sf_tile_rows);
   else
     quantize_view_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax);
+        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax, sf_tile_rows);
   return cudaGetLastError();
 }
 

@@ -34,8 +34,9 @@ def test_strerror_texts():
 
 def _expected_ws(B, H, Lq, Lk, D, flags):
     """Workspace layout restated: 256-byte aligned regions for fq(Q), fq(K),
-    fq(V) (bf16), fq(V) (fp16), float32 O, Delta, 16 bytes of statistics and,
-    with every quantizer on, the fp16 copy of dO."""
+    fq(V) (bf16), fq(V) (fp16), float32 O, Delta, 16 bytes of statistics,
+    with every quantizer on the fp16 copy of dO and, with Q and K quantized,
+    their packed codes and scale tiles."""
     al = lambda x: (x + 255) // 256 * 256
     BH = B * H
     n = 0
@@ -48,6 +49,11 @@ def _expected_ws(B, H, Lq, Lk, D, flags):
     n += al(BH * Lq * D * 4) + al(BH * Lq * 4) + al(16)
     if flags & 15 == 15:
         n += al(BH * Lq * D * 2)  # fp16 copy of dO for the all-quantized backward
+    if flags & 3 == 3:
+        # packed NVFP4 codes (D/2 bytes per row) and 512-byte scale tiles per
+        # 128 rows x 64 columns, for Q then K
+        for L in (Lq, Lk):
+            n += al(BH * L * D // 2) + al(BH * ((L + 127) // 128) * (D // 64) * 512)
     return n
 
 
