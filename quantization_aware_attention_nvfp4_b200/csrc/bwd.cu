@@ -43,6 +43,7 @@ struct BwdBars {
   uint64_t kvfull;
   uint64_t afull[2], aempty[2];   // Q tiles (dK/dV kernel) or K tiles (dQ kernel)
   uint64_t bfull[2], bempty[2];   // dO tiles (dK/dV kernel) or V tiles (dQ kernel)
+  uint64_t k4full[2], k4empty[2]; // packed NVFP4 K tiles and scales (dQ kernel, NVFP4 S)
   uint64_t sfull, sempty;   // S and dP in TMEM: filled together, released together
   uint64_t xfull, xempty;
   uint64_t done;
@@ -57,6 +58,8 @@ __device__ __forceinline__ void init_bwd_bars(BwdBars *b) {
     mbar_init(&b->aempty[s], 1);
     mbar_init(&b->bfull[s], 1);
     mbar_init(&b->bempty[s], 1);
+    mbar_init(&b->k4full[s], 1);
+    mbar_init(&b->k4empty[s], 1);
   }
   mbar_init(&b->sfull, 1);
   mbar_init(&b->sempty, kSoftWarps);
@@ -95,28 +98,35 @@ __device__ __forceinline__ uint32_t pack_ds(float a, float b) {
   return QKF16 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
 }
 
+// S and dP of one thread's 64 columns (starting at col0) from TMEM into
+// registers.  The caller releases the TMEM tiles right after, so the next
+// tile's S and dP MMAs run while this tile's row math proceeds.
+__device__ __forceinline__ void load_sdp(uint32_t tS, uint32_t tDP, int col0, uint32_t (&sv)[64],
+                                         uint32_t (&dv)[64]) {
+  tmem_ld32(tS + col0, *reinterpret_cast<uint32_t(*)[32]>(sv));
+  tmem_ld32(tS + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+  tmem_ld32(tDP + col0, *reinterpret_cast<uint32_t(*)[32]>(dv));
+  tmem_ld32(tDP + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+  tmem_ld_wait();
+}
+
 // One query tile for one thread of the dK/dV kernel (one query row, 64 key
-// columns starting at col0), 32 keys at a time: S and dP from TMEM,
-// P~ = exp(S - m) and fq(P~)/l (bf16, half a row of the transposed dV
-// operand), and dS = (P~/l)(dP - Delta) in float32, scaled by dsc and packed
-// for the dK operand.  P never leaves float32.
+// columns starting at col0), from S and dP in registers: P~ = exp(S - m) and
+// fq(P~)/l (bf16, half a row of the transposed dV operand), and
+// dS = (P~/l)(dP - Delta) in float32, scaled by dsc and packed for the dK
+// operand.  P never leaves float32.
 template <int QP, int QKF16, bool MASKED>
-__device__ __forceinline__ void dkdv_tile(uint32_t tS, uint32_t tDP, int col0, int valid_k, bool vq, float cl,
-                                          float nml, float inv_l, float delta, float dsc, uint32_t (&pw)[32],
-                                          uint32_t (&dsw)[32]) {
-#pragma unroll 1
+__device__ __forceinline__ void dkdv_tile(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
+                                          int valid_k, bool vq, float cl, float nml, float inv_l, float delta,
+                                          float dsc, uint32_t (&pw)[32], uint32_t (&dsw)[32]) {
+#pragma unroll
   for (int c = 0; c < 2; ++c) {
-    uint32_t r[32], d[32];
-    tmem_ld32(tS + col0 + c * 32, r);
-    tmem_ld32(tDP + col0 + c * 32, d);
-    tmem_ld_wait();
     float p[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float e = ex2_approx(fmaf(__uint_as_float(r[i]), cl, nml));
+      const float e = ex2_approx(fmaf(__uint_as_float(sv[32 * c + i]), cl, nml));
       p[i] = (vq && (!MASKED || col0 + c * 32 + i < valid_k)) ? e : 0.0f;
     }
-    uint32_t wv[16], ws[16];
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       if (QP) {
@@ -126,31 +136,20 @@ __device__ __forceinline__ void dkdv_tile(uint32_t tS, uint32_t tDP, int col0, i
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float2 g = unpack_f16x2(rr[i]);
-          wv[8 * b + i] = pack_bf16x2(g.x * f, g.y * f);
+          pw[16 * c + 8 * b + i] = pack_bf16x2(g.x * f, g.y * f);
         }
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          wv[8 * b + i] = pack_bf16x2(p[16 * b + 2 * i] * inv_l, p[16 * b + 2 * i + 1] * inv_l);
+          pw[16 * c + 8 * b + i] = pack_bf16x2(p[16 * b + 2 * i] * inv_l, p[16 * b + 2 * i + 1] * inv_l);
       }
     }
     const float pf = inv_l * dsc;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const float d0 = p[2 * i] * pf * (__uint_as_float(d[2 * i]) - delta);
-      const float d1 = p[2 * i + 1] * pf * (__uint_as_float(d[2 * i + 1]) - delta);
-      ws[i] = pack_ds<QKF16>(d0, d1);
-    }
-    // runtime c: write through a small selector instead of dynamic indexing
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (c == 0) {
-        pw[i] = wv[i];
-        dsw[i] = ws[i];
-      } else {
-        pw[16 + i] = wv[i];
-        dsw[16 + i] = ws[i];
-      }
+      const float d0 = p[2 * i] * pf * (__uint_as_float(dv[32 * c + 2 * i]) - delta);
+      const float d1 = p[2 * i + 1] * pf * (__uint_as_float(dv[32 * c + 2 * i + 1]) - delta);
+      dsw[16 * c + i] = pack_ds<QKF16>(d0, d1);
     }
   }
 }
@@ -163,19 +162,15 @@ __device__ __forceinline__ void dkdv_tile(uint32_t tS, uint32_t tDP, int col0, i
 // a1 = 2^-e dsc / l, b1 = -Delta dsc / l.  Rows past Lq come in with
 // nml = -inf, so their P~ is 0 without a per-element test.
 template <bool MASKED>
-__device__ __forceinline__ void dkdv_tile_f16(uint32_t tS, uint32_t tDP, int col0, int valid_k, float cl,
-                                              float nml, float vf, float a1, float b1, uint32_t (&pw)[32],
-                                              uint32_t (&dsw)[32]) {
+__device__ __forceinline__ void dkdv_tile_f16(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
+                                              int valid_k, float cl, float nml, float vf, float a1, float b1,
+                                              uint32_t (&pw)[32], uint32_t (&dsw)[32]) {
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    uint32_t r[32], d[32];
-    tmem_ld32(tS + col0 + c * 32, r);
-    tmem_ld32(tDP + col0 + c * 32, d);
-    tmem_ld_wait();
     float p[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float e = ex2_approx(fmaf(__uint_as_float(r[i]), cl, nml));
+      const float e = ex2_approx(fmaf(__uint_as_float(sv[32 * c + i]), cl, nml));
       p[i] = (!MASKED || col0 + c * 32 + i < valid_k) ? e : 0.0f;
     }
 #pragma unroll
@@ -187,8 +182,8 @@ __device__ __forceinline__ void dkdv_tile_f16(uint32_t tS, uint32_t tDP, int col
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i)
-      dsw[16 * c + i] = pack_f16x2(p[2 * i] * fmaf(__uint_as_float(d[2 * i]), a1, b1),
-                                   p[2 * i + 1] * fmaf(__uint_as_float(d[2 * i + 1]), a1, b1));
+      dsw[16 * c + i] = pack_f16x2(p[2 * i] * fmaf(__uint_as_float(dv[32 * c + 2 * i]), a1, b1),
+                                   p[2 * i + 1] * fmaf(__uint_as_float(dv[32 * c + 2 * i + 1]), a1, b1));
   }
 }
 
@@ -259,12 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t kaddr = sbase + L::kK, vaddr = sbase + L::kV, xaddr = sbase + L::kX;
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
       // S_i and dP_i into TMEM; one commit signals both
+      // dP first: the dO slot frees earlier (after dV) than the Q slot (after
+      // dK), so the Q tile's load has dP's duration to land
       auto issue_sdp = [&](int i) -> bool {
-        if (!mbar_wait(&bars->afull[i & 1], (i >> 1) & 1, abort)) return false;
         if (!mbar_wait(&bars->bfull[i & 1], (i >> 1) & 1, abort)) return false;
         tc_fence_after();
-        mma_kmajor(tmem + L::kTmemS, sbase + L::kQ + (i & 1) * L::kTile, kaddr, D / 16, idS, false);
         mma_kmajor(tmem + L::kTmemDP, sbase + L::kDO + (i & 1) * L::kTile, vaddr, D / 16, idDP, false);
+        if (!mbar_wait(&bars->afull[i & 1], (i >> 1) & 1, abort)) return false;
+        tc_fence_after();
+        mma_kmajor(tmem + L::kTmemS, sbase + L::kQ + (i & 1) * L::kTile, kaddr, D / 16, idS, false);
         umma_commit(&bars->sfull);
         return true;
       };
@@ -317,26 +315,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_stats(i + 1, m_n, lse_n, delta_n);
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
       uint32_t pw[32], dsw[32];
+      uint32_t sv[64], dv[64];
       if (!mbar_wait(&bars->sfull, i & 1, abort)) { ok = false; break; }
       tc_fence_after();
+      load_sdp(tS, tDP, col0, sv, dv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->sempty);
       if (DOF16) {
         const float nml = vq ? -(m * kLog2e) : -INFINITY;
         const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
         const float a1 = inv_l * dsc / dos, b1 = -delta * inv_l * dsc;
         if (valid_k < kBN)
-          dkdv_tile_f16<true>(tS, tDP, col0, valid_k, cl, nml, vf, a1, b1, pw, dsw);
+          dkdv_tile_f16<true>(sv, dv, col0, valid_k, cl, nml, vf, a1, b1, pw, dsw);
         else
-          dkdv_tile_f16<false>(tS, tDP, col0, valid_k, cl, nml, vf, a1, b1, pw, dsw);
+          dkdv_tile_f16<false>(sv, dv, col0, valid_k, cl, nml, vf, a1, b1, pw, dsw);
       } else {
         const float nml = -(m * kLog2e);
         if (valid_k < kBN)
-          dkdv_tile<QP, QKF16, true>(tS, tDP, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
+          dkdv_tile<QP, QKF16, true>(sv, dv, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
         else
-          dkdv_tile<QP, QKF16, false>(tS, tDP, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
+          dkdv_tile<QP, QKF16, false>(sv, dv, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sempty);
       if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, pw);
       fence_proxy_async_smem();
@@ -395,43 +395,51 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ----------------------------------------------------------------- dQ -----
 
-template <int D>
+// dQ kernel layout.  With FP4S (Q and K quantized) S = fq(Q) fq(K)^T is a
+// block-scaled NVFP4 MMA: the Q codes and scales stay resident and K codes
+// stream through their own small 2-stage ring, so S never waits on the
+// 16-bit K slot that the dQ MMA holds; the 16-bit Q tile is then not needed.
+template <int D, int FP4S>
 struct DqLayout {
   static constexpr int kTile = Tile<D>::kBytes;
   static constexpr int kXBytes = kBM * kBN * 2;
-  static constexpr int kQ = 0;
-  static constexpr int kDO = kQ + kTile;
-  static constexpr int kK = kDO + kTile;        // 2 stages
+  static constexpr int kCode = 128 * (D / 2);   // one packed NVFP4 tile
+  static constexpr int kSF = (D / 64) * 512;    // its scale-factor blocks
+  static constexpr int kQ = 0;                  // 16-bit Q tile, or Q codes (FP4S)
+  static constexpr int kQSF = kQ + (FP4S ? kCode : kTile);
+  static constexpr int kDO = (kQSF + (FP4S ? kSF : 0) + 1023) / 1024 * 1024;
+  static constexpr int kK = kDO + kTile;        // 2 stages of 16-bit K
   static constexpr int kV = kK + 2 * kTile;     // 2 stages
   static constexpr int kX = kV + 2 * kTile;     // dS
-  static constexpr int kBar = kX + kXBytes;
+  static constexpr int kK4 = kX + kXBytes;      // FP4S: 2 stages of K codes
+  static constexpr int kKSF = kK4 + (FP4S ? 2 * kCode : 0);
+  static constexpr int kBar = kKSF + (FP4S ? 2 * kSF : 0);
   static constexpr int kBytes = kBar + 256;
   static constexpr int kDynSmem = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDQ = 256;
+  static constexpr uint32_t kSFCols = (D / 64) * 4;
+  static constexpr uint32_t kTmemSFA = 256 + D, kTmemSFB = kTmemSFA + kSFCols;  // 2 stages
+  static constexpr uint32_t kCodeLayout = (D / 2 == 64) ? 4u : 6u;  // SW64 / SW32
+  static constexpr uint32_t kCodeSBO = 8 * (D / 2);
 };
 
 // One key tile for one thread of the dQ kernel (one query row, 64 key
-// columns starting at col0), 32 keys at a time: P = exp(S - LSE) in float32
-// and dS = P (dP - Delta), scaled by dsc and packed for the dQ operand.
+// columns starting at col0), from S and dP in registers: P = exp(S - LSE) in
+// float32 and dS = P (dP - Delta), scaled by dsc and packed for the dQ
+// operand.
 template <int QKF16, bool MASKED>
-__device__ __forceinline__ void dq_tile(uint32_t tS, uint32_t tDP, int col0, int valid_k, bool vq, float cl,
-                                        float nlse, float delta, float dsc, uint32_t (&dsw)[32]) {
+__device__ __forceinline__ void dq_tile(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
+                                        int valid_k, bool vq, float cl, float nlse, float delta, float dsc,
+                                        uint32_t (&dsw)[32]) {
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    uint32_t r[32], d[32];
-    tmem_ld32(tS + col0 + c * 32, r);
-    tmem_ld32(tDP + col0 + c * 32, d);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * i]), cl, nlse));
-      float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), cl, nlse));
-      if (!vq || (MASKED && col0 + c * 32 + 2 * i >= valid_k)) p0 = 0.0f;
-      if (!vq || (MASKED && col0 + c * 32 + 2 * i + 1 >= valid_k)) p1 = 0.0f;
-      dsw[16 * c + i] = pack_ds<QKF16>(p0 * dsc * (__uint_as_float(d[2 * i]) - delta),
-                                       p1 * dsc * (__uint_as_float(d[2 * i + 1]) - delta));
-    }
+  for (int i = 0; i < 32; ++i) {
+    float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), cl, nlse));
+    float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), cl, nlse));
+    if (!vq || (MASKED && col0 + 2 * i >= valid_k)) p0 = 0.0f;
+    if (!vq || (MASKED && col0 + 2 * i + 1 >= valid_k)) p1 = 0.0f;
+    dsw[i] = pack_ds<QKF16>(p0 * dsc * (__uint_as_float(dv[2 * i]) - delta),
+                            p1 * dsc * (__uint_as_float(dv[2 * i + 1]) - delta));
   }
 }
 
@@ -439,23 +447,17 @@ __device__ __forceinline__ void dq_tile(uint32_t tS, uint32_t tDP, int col0, int
 // dS * dsc = P (dP' 2^-e - Delta) dsc = P * fma(dP', a1, b1) with
 // a1 = 2^-e dsc, b1 = -Delta dsc.  Rows past Lq come in with nlse = -inf.
 template <bool MASKED>
-__device__ __forceinline__ void dq_tile_f16(uint32_t tS, uint32_t tDP, int col0, int valid_k, float cl,
-                                            float nlse, float a1, float b1, uint32_t (&dsw)[32]) {
+__device__ __forceinline__ void dq_tile_f16(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
+                                            int valid_k, float cl, float nlse, float a1, float b1,
+                                            uint32_t (&dsw)[32]) {
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    uint32_t r[32], d[32];
-    tmem_ld32(tS + col0 + c * 32, r);
-    tmem_ld32(tDP + col0 + c * 32, d);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * i]), cl, nlse));
-      float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * i + 1]), cl, nlse));
-      if (MASKED && col0 + c * 32 + 2 * i >= valid_k) p0 = 0.0f;
-      if (MASKED && col0 + c * 32 + 2 * i + 1 >= valid_k) p1 = 0.0f;
-      dsw[16 * c + i] = pack_f16x2(p0 * fmaf(__uint_as_float(d[2 * i]), a1, b1),
-                                   p1 * fmaf(__uint_as_float(d[2 * i + 1]), a1, b1));
-    }
+  for (int i = 0; i < 32; ++i) {
+    float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), cl, nlse));
+    float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), cl, nlse));
+    if (MASKED && col0 + 2 * i >= valid_k) p0 = 0.0f;
+    if (MASKED && col0 + 2 * i + 1 >= valid_k) p1 = 0.0f;
+    dsw[i] = pack_f16x2(p0 * fmaf(__uint_as_float(dv[2 * i]), a1, b1),
+                        p1 * fmaf(__uint_as_float(dv[2 * i + 1]), a1, b1));
   }
 }
 
@@ -463,8 +465,9 @@ template <int D, int QKF16, int DOF16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                       const BwdArgs a) {
-  using L = DqLayout<D>;
+                       const __grid_constant__ CUtensorMap tmK4, const BwdArgs a) {
+  constexpr int FP4S = QKF16;  // quantized Q and K: S on the NVFP4 path
+  using L = DqLayout<D, FP4S>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
@@ -492,59 +495,97 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmDO);
-      mbar_arrive_expect_tx(&bars->kvfull, 2 * L::kTile);
-      load_tile<D>(smem + L::kQ, &tmQ, &bars->kvfull, qt * kBM, bh);
+      if (FP4S) prefetch_tmap(&tmK4);
+      mbar_arrive_expect_tx(&bars->kvfull, (FP4S ? L::kCode + L::kSF : L::kTile) + L::kTile);
+      if (FP4S) {
+        tma_load_3d(smem + L::kQ, &tmQ, &bars->kvfull, 0, qt * kBM, bh);
+        bulk_load(smem + L::kQSF, a.qsf + (static_cast<size_t>(bh) * a.nq_tiles + qt) * L::kSF, L::kSF,
+                  &bars->kvfull);
+      } else {
+        load_tile<D>(smem + L::kQ, &tmQ, &bars->kvfull, qt * kBM, bh);
+      }
       load_tile<D>(smem + L::kDO, &tmDO, &bars->kvfull, qt * kBM, bh);
-      int issued = 0;
+      int n4 = 0, nv = 0, nkh = 0;  // tiles issued per ring
       for (int j = 0; j < nk; ++j) {
         const int st = j & 1;
-        if (j >= 2 && !mbar_wait(&bars->aempty[st], ((j >> 1) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
-        load_tile<D>(smem + L::kK + st * L::kTile, &tmK, &bars->afull[st], j * kBN, bh);
-        if (j >= 2 && !mbar_wait(&bars->bempty[st], ((j >> 1) - 1) & 1, abort)) {
-          issued = j + 1;
-          break;
+        const int ph = ((j >> 1) - 1) & 1;
+        if (FP4S) {
+          if (j >= 2 && !mbar_wait(&bars->k4empty[st], ph, abort)) break;
+          mbar_arrive_expect_tx(&bars->k4full[st], L::kCode + L::kSF);
+          tma_load_3d(smem + L::kK4 + st * L::kCode, &tmK4, &bars->k4full[st], 0, j * kBN, bh);
+          bulk_load(smem + L::kKSF + st * L::kSF, a.ksf + (static_cast<size_t>(bh) * nk + j) * L::kSF, L::kSF,
+                    &bars->k4full[st]);
+          n4 = j + 1;
         }
+        if (j >= 2 && !mbar_wait(&bars->bempty[st], ph, abort)) break;
         mbar_arrive_expect_tx(&bars->bfull[st], L::kTile);
         load_tile<D>(smem + L::kV + st * L::kTile, &tmV, &bars->bfull[st], j * kBN, bh);
-        issued = j + 1;
+        nv = j + 1;
+        if (j >= 2 && !mbar_wait(&bars->aempty[st], ph, abort)) break;
+        mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
+        load_tile<D>(smem + L::kK + st * L::kTile, &tmK, &bars->afull[st], j * kBN, bh);
+        nkh = j + 1;
       }
       if (*abort) {
         mbar_wait_drain(&bars->kvfull, 0);
-        for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
-          mbar_wait_drain(&bars->afull[j & 1], (j >> 1) & 1);
-          mbar_wait_drain(&bars->bfull[j & 1], (j >> 1) & 1);
-        }
+        for (int j = (n4 > 2 ? n4 - 2 : 0); j < n4; ++j) mbar_wait_drain(&bars->k4full[j & 1], (j >> 1) & 1);
+        for (int j = (nv > 2 ? nv - 2 : 0); j < nv; ++j) mbar_wait_drain(&bars->bfull[j & 1], (j >> 1) & 1);
+        for (int j = (nkh > 2 ? nkh - 2 : 0); j < nkh; ++j) mbar_wait_drain(&bars->afull[j & 1], (j >> 1) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_f16(kBM, kBN, !QKF16, false, false);  // Q K^T
+      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);  // Q K^T
       constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
       constexpr uint32_t idQ = idesc_f16(kBM, D, !QKF16, false, true);     // dS (K-major) * K (MN-major)
       const uint32_t qaddr = sbase + L::kQ, doaddr = sbase + L::kDO, xaddr = sbase + L::kX;
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
-      auto issue_sdp = [&](int j) -> bool {
-        if (!mbar_wait(&bars->afull[j & 1], (j >> 1) & 1, abort)) return false;
-        if (!mbar_wait(&bars->bfull[j & 1], (j >> 1) & 1, abort)) return false;
+      if (ok && FP4S) {
         tc_fence_after();
-        mma_kmajor(tmem + L::kTmemS, qaddr, sbase + L::kK + (j & 1) * L::kTile, D / 16, idS, false);
-        mma_kmajor(tmem + L::kTmemDP, doaddr, sbase + L::kV + (j & 1) * L::kTile, D / 16, idDP, false);
-        umma_commit(&bars->bempty[j & 1]);
+        for (int kc = 0; kc < D / 64; ++kc)
+          tmem_cp_32x128b_x4(tmem + L::kTmemSFA + kc * 4, sdesc_make(sbase + L::kQSF + kc * 512, 16, 128, 0));
+      }
+      // dP_j, then S_j; one commit signals both
+      auto issue_sdp = [&](int j) -> bool {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&bars->bfull[st], ph, abort)) return false;
+        tc_fence_after();
+        mma_kmajor(tmem + L::kTmemDP, doaddr, sbase + L::kV + st * L::kTile, D / 16, idDP, false);
+        umma_commit(&bars->bempty[st]);
+        if (FP4S) {
+          if (!mbar_wait(&bars->k4full[st], ph, abort)) return false;
+          tc_fence_after();
+          const uint32_t sfb = tmem + L::kTmemSFB + st * L::kSFCols;
+          const uint32_t kaddr = sbase + L::kK4 + st * L::kCode;
+          for (int kc = 0; kc < D / 64; ++kc)
+            tmem_cp_32x128b_x4(sfb + kc * 4, sdesc_make(sbase + L::kKSF + st * L::kSF + kc * 512, 16, 128, 0));
+          for (int kk = 0; kk < D / 64; ++kk)
+            umma_fp4(tmem + L::kTmemS, sdesc_make(qaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout),
+                     sdesc_make(kaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout), idS,
+                     tmem + L::kTmemSFA + kk * 4, sfb + kk * 4, kk > 0 ? 1u : 0u);
+          umma_commit(&bars->k4empty[st]);
+        } else {
+          if (!mbar_wait(&bars->afull[st], ph, abort)) return false;
+          tc_fence_after();
+          mma_kmajor(tmem + L::kTmemS, qaddr, sbase + L::kK + st * L::kTile, D / 16, idS, false);
+        }
         umma_commit(&bars->sfull);
         return true;
       };
       if (ok) ok = issue_sdp(0);
       for (int j = 0; ok && j < nk; ++j) {
+        const int st = j & 1;
         if (j + 1 < nk) {
           ok = mbar_wait(&bars->sempty, j & 1, abort) && issue_sdp(j + 1);
           if (!ok) break;
         }
         if (!mbar_wait(&bars->xfull, j & 1, abort)) { ok = false; break; }
+        if (FP4S && !mbar_wait(&bars->afull[st], (j >> 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        mma_a_k_b_mn(tmem + L::kTmemDQ, xaddr, sbase + L::kK + (j & 1) * L::kTile, kBN / 16, idQ, j > 0);
+        mma_a_k_b_mn(tmem + L::kTmemDQ, xaddr, sbase + L::kK + st * L::kTile, kBN / 16, idQ, j > 0);
         umma_commit(&bars->xempty);
-        umma_commit(&bars->aempty[j & 1]);
+        umma_commit(&bars->aempty[st]);
       }
       umma_commit(&bars->done);
     }
@@ -567,22 +608,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       uint32_t dsw[32];
+      uint32_t sv[64], dv[64];
       if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      if (DOF16) {
-        if (j == nk - 1 && last_valid < kBN)
-          dq_tile_f16<true>(tS, tDP, col0, last_valid, cl, nlse, a1, b1, dsw);
-        else
-          dq_tile_f16<false>(tS, tDP, col0, kBN, cl, nlse, a1, b1, dsw);
-      } else {
-        if (j == nk - 1 && last_valid < kBN)
-          dq_tile<QKF16, true>(tS, tDP, col0, last_valid, vq, cl, nlse, delta, dsc, dsw);
-        else
-          dq_tile<QKF16, false>(tS, tDP, col0, kBN, vq, cl, nlse, delta, dsc, dsw);
-      }
+      load_sdp(tS, tDP, col0, sv, dv);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
+      if (DOF16) {
+        if (j == nk - 1 && last_valid < kBN)
+          dq_tile_f16<true>(sv, dv, col0, last_valid, cl, nlse, a1, b1, dsw);
+        else
+          dq_tile_f16<false>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw);
+      } else {
+        if (j == nk - 1 && last_valid < kBN)
+          dq_tile<QKF16, true>(sv, dv, col0, last_valid, vq, cl, nlse, delta, dsc, dsw);
+        else
+          dq_tile<QKF16, false>(sv, dv, col0, kBN, vq, cl, nlse, delta, dsc, dsw);
+      }
       if (j >= 1 && !mbar_wait(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
       fence_proxy_async_smem();
@@ -659,29 +702,32 @@ cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const
 
 template <int D, int QKF16, int DOF16>
 static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                               const CUtensorMap &tdo, const BwdArgs &a, int BH, cudaStream_t stream) {
-  using L = DqLayout<D>;
+                               const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
+                               cudaStream_t stream) {
+  using L = DqLayout<D, QKF16>;
+  static_assert(L::kDynSmem <= 232448, "dQ shared memory over the 227 KB limit");
+  static_assert(L::kTmemSFB + 2 * L::kSFCols <= L::kTmemCols, "dQ TMEM over 512 columns");
   auto kern = attn_bwd_dq_kernel<D, QKF16, DOF16>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(a.nq_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<dim3(a.nq_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, tk4, a);
   return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t dq_dispatch(bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
-                               const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
-                               cudaStream_t stream) {
-  if (do_f16) return launch_dq_t<D, 1, 1>(tq, tk, tv, tdo, a, BH, stream);
-  return qk_f16 ? launch_dq_t<D, 1, 0>(tq, tk, tv, tdo, a, BH, stream)
-                : launch_dq_t<D, 0, 0>(tq, tk, tv, tdo, a, BH, stream);
+                               const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4,
+                               const BwdArgs &a, int BH, cudaStream_t stream) {
+  if (do_f16) return launch_dq_t<D, 1, 1>(tq, tk, tv, tdo, tk4, a, BH, stream);
+  return qk_f16 ? launch_dq_t<D, 1, 0>(tq, tk, tv, tdo, tk4, a, BH, stream)
+                : launch_dq_t<D, 0, 0>(tq, tk, tv, tdo, tk4, a, BH, stream);
 }
 
 cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
-                          const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
-                          cudaStream_t stream) {
-  return D == 128 ? dq_dispatch<128>(qk_f16, do_f16, tq, tk, tv, tdo, a, BH, stream)
-                  : dq_dispatch<64>(qk_f16, do_f16, tq, tk, tv, tdo, a, BH, stream);
+                          const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4,
+                          const BwdArgs &a, int BH, cudaStream_t stream) {
+  return D == 128 ? dq_dispatch<128>(qk_f16, do_f16, tq, tk, tv, tdo, tk4, a, BH, stream)
+                  : dq_dispatch<64>(qk_f16, do_f16, tq, tk, tv, tdo, tk4, a, BH, stream);
 }
 
 }  // namespace attnqat

@@ -32,6 +32,8 @@ struct BwdArgs {
   const float *m;
   const float *lse;
   const float *delta;
+  const uint8_t *qsf;   // scale-factor tiles of fq(Q), fq(K) (NVFP4 S in the dQ kernel)
+  const uint8_t *ksf;
   __nv_bfloat16 *dq;
   __nv_bfloat16 *dk;
   __nv_bfloat16 *dv;
@@ -56,9 +58,12 @@ cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUte
 cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
                             const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
                             const BwdArgs &a, int BH, cudaStream_t stream);
+// dQ.  With qk_f16, tq maps the packed NVFP4 Q codes (as for the forward),
+// tk4 the K codes, a.qsf/a.ksf their scale tiles, and tk the fp16 fq(K) that
+// dQ = dS fq(K) reads; otherwise tq/tk are bf16 and tk4 is unused.
 cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
-                          const CUtensorMap &tv, const CUtensorMap &tdo, const BwdArgs &a, int BH,
-                          cudaStream_t stream);
+                          const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4,
+                          const BwdArgs &a, int BH, cudaStream_t stream);
 
 // NVFP4 fq of a strided bf16 view (see attnqat_quantize); any of codes,
 // scales, deq (bf16, same strides as x), deq_f16 and absmax (max |fq(x)|,
