@@ -119,13 +119,17 @@ template <int QP, int QKF16, bool MASKED>
 __device__ __forceinline__ void dkdv_tile(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
                                           int valid_k, bool vq, float cl, float nml, float inv_l, float delta,
                                           float dsc, uint32_t (&pw)[32], uint32_t (&dsw)[32]) {
+  const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     float p[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float e = ex2_approx(fmaf(__uint_as_float(sv[32 * c + i]), cl, nml));
-      p[i] = (vq && (!MASKED || col0 + c * 32 + i < valid_k)) ? e : 0.0f;
+    for (int i = 0; i < 16; ++i) {
+      const float2 x = fma2(make_float2(__uint_as_float(sv[32 * c + 2 * i]), __uint_as_float(sv[32 * c + 2 * i + 1])),
+                            cl2, nml2);
+      const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
+      p[2 * i] = (vq && (!MASKED || col0 + c * 32 + 2 * i < valid_k)) ? e0 : 0.0f;
+      p[2 * i + 1] = (vq && (!MASKED || col0 + c * 32 + 2 * i + 1 < valid_k)) ? e1 : 0.0f;
     }
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
@@ -165,13 +169,18 @@ template <bool MASKED>
 __device__ __forceinline__ void dkdv_tile_f16(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
                                               int valid_k, float cl, float nml, float vf, float a1, float b1,
                                               uint32_t (&pw)[32], uint32_t (&dsw)[32]) {
+  const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
+  const float2 a12 = make_float2(a1, a1), b12 = make_float2(b1, b1);
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     float p[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float e = ex2_approx(fmaf(__uint_as_float(sv[32 * c + i]), cl, nml));
-      p[i] = (!MASKED || col0 + c * 32 + i < valid_k) ? e : 0.0f;
+    for (int i = 0; i < 16; ++i) {
+      const float2 x = fma2(make_float2(__uint_as_float(sv[32 * c + 2 * i]), __uint_as_float(sv[32 * c + 2 * i + 1])),
+                            cl2, nml2);
+      const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
+      p[2 * i] = (!MASKED || col0 + c * 32 + 2 * i < valid_k) ? e0 : 0.0f;
+      p[2 * i + 1] = (!MASKED || col0 + c * 32 + 2 * i + 1 < valid_k) ? e1 : 0.0f;
     }
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
@@ -181,9 +190,12 @@ __device__ __forceinline__ void dkdv_tile_f16(const uint32_t (&sv)[64], const ui
       for (int i = 0; i < 8; ++i) pw[16 * c + 8 * b + i] = hmul2_u32(rr[i], s2);
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      dsw[16 * c + i] = pack_f16x2(p[2 * i] * fmaf(__uint_as_float(dv[32 * c + 2 * i]), a1, b1),
-                                   p[2 * i + 1] * fmaf(__uint_as_float(dv[32 * c + 2 * i + 1]), a1, b1));
+    for (int i = 0; i < 16; ++i) {
+      const float2 g = fma2(make_float2(__uint_as_float(dv[32 * c + 2 * i]), __uint_as_float(dv[32 * c + 2 * i + 1])),
+                            a12, b12);
+      const float2 d = mul2(make_float2(p[2 * i], p[2 * i + 1]), g);
+      dsw[16 * c + i] = pack_f16x2(d.x, d.y);
+    }
   }
 }
 
@@ -450,14 +462,18 @@ template <bool MASKED>
 __device__ __forceinline__ void dq_tile_f16(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
                                             int valid_k, float cl, float nlse, float a1, float b1,
                                             uint32_t (&dsw)[32]) {
+  const float2 cl2 = make_float2(cl, cl), nl2 = make_float2(nlse, nlse);
+  const float2 a12 = make_float2(a1, a1), b12 = make_float2(b1, b1);
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), cl, nlse));
-    float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), cl, nlse));
+    const float2 x = fma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), cl2, nl2);
+    float p0 = ex2_approx(x.x);
+    float p1 = ex2_approx(x.y);
     if (MASKED && col0 + 2 * i >= valid_k) p0 = 0.0f;
     if (MASKED && col0 + 2 * i + 1 >= valid_k) p1 = 0.0f;
-    dsw[i] = pack_f16x2(p0 * fmaf(__uint_as_float(dv[2 * i]), a1, b1),
-                        p1 * fmaf(__uint_as_float(dv[2 * i + 1]), a1, b1));
+    const float2 g = fma2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), a12, b12);
+    const float2 d = mul2(make_float2(p0, p1), g);
+    dsw[i] = pack_f16x2(d.x, d.y);
   }
 }
 

@@ -33,15 +33,17 @@ struct Tile {
 // boundary.  Forward and backward use this same routine on the same bits, so
 // they agree bit for bit.
 __device__ __forceinline__ float fq16_probs(const float *p, uint32_t (&r)[8]) {
-  float amax = fmaxf(fmaxf(fmaxf(p[0], p[1]), fmaxf(p[2], p[3])),
-                     fmaxf(fmaxf(p[4], p[5]), fmaxf(p[6], p[7])));
-  amax = fmaxf(amax, fmaxf(fmaxf(fmaxf(p[8], p[9]), fmaxf(p[10], p[11])),
-                           fmaxf(fmaxf(p[12], p[13]), fmaxf(p[14], p[15]))));
+  const float amax = fmax3(fmax3(fmax3(p[0], p[1], p[2]), fmax3(p[3], p[4], p[5]), fmax3(p[6], p[7], p[8])),
+                          fmax3(p[9], p[10], p[11]), fmax3(p[12], p[13], fmaxf(p[14], p[15])));
   const uint16_t code = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.0f);
   const float s = unpack_f16x2(cvt_f16x2_from_e4m3x2(code)).x;
   const float inv = s > 0.0f ? rcp_approx(s) : 0.0f;
+  const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) r[i] = e2m1_round_f16x2(p[2 * i] * inv, p[2 * i + 1] * inv);
+  for (int i = 0; i < 8; ++i) {
+    const float2 x = mul2(make_float2(p[2 * i], p[2 * i + 1]), inv2);
+    r[i] = e2m1_round_f16x2(x.x, x.y);
+  }
   return s;
 }
 

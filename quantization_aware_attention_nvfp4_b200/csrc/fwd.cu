@@ -76,8 +76,9 @@ __device__ __forceinline__ float row_max_half(uint32_t taddr, int col0, int vali
   float mx = -INFINITY;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    if (!MASKED || col0 + i < valid) mx = fmaxf(mx, __uint_as_float(r[i]));
-    if (!MASKED || col0 + 32 + i < valid) mx = fmaxf(mx, __uint_as_float(t[i]));
+    const float a = (!MASKED || col0 + i < valid) ? __uint_as_float(r[i]) : -INFINITY;
+    const float b = (!MASKED || col0 + 32 + i < valid) ? __uint_as_float(t[i]) : -INFINITY;
+    mx = fmax3(mx, a, b);
   }
   return mx;
 }
@@ -89,7 +90,8 @@ __device__ __forceinline__ float row_max_half(uint32_t taddr, int col0, int vali
 template <int PV_F16, int QP, bool MASKED>
 __device__ __forceinline__ float prob_half(uint32_t taddr, int col0, int valid, float cl, float nml,
                                            uint32_t pbase, uint32_t row) {
-  float lsum = 0.0f;
+  float2 lsum = make_float2(0.0f, 0.0f);
+  const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     uint32_t r[32];
@@ -97,10 +99,12 @@ __device__ __forceinline__ float prob_half(uint32_t taddr, int col0, int valid, 
     tmem_ld_wait();
     float p[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float e = ex2_approx(fmaf(__uint_as_float(r[i]), cl, nml));
-      p[i] = (!MASKED || col0 + c * 32 + i < valid) ? e : 0.0f;
-      lsum += p[i];
+    for (int i = 0; i < 16; ++i) {
+      const float2 x = fma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), cl2, nml2);
+      const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
+      p[2 * i] = (!MASKED || col0 + c * 32 + 2 * i < valid) ? e0 : 0.0f;
+      p[2 * i + 1] = (!MASKED || col0 + c * 32 + 2 * i + 1 < valid) ? e1 : 0.0f;
+      lsum = add2(lsum, make_float2(p[2 * i], p[2 * i + 1]));
     }
     uint32_t w[16];
 #pragma unroll
@@ -133,7 +137,7 @@ __device__ __forceinline__ float prob_half(uint32_t taddr, int col0, int valid, 
       st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     }
   }
-  return lsum;
+  return lsum.x + lsum.y;
 }
 
 // Merges a per-row partial value with the other column half's through
