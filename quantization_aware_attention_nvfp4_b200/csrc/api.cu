@@ -472,17 +472,18 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
   a.dq = static_cast<__nv_bfloat16 *>(dq);
   a.dk = static_cast<__nv_bfloat16 *>(dk);
   a.dv = static_cast<__nv_bfloat16 *>(dv);
+  // with Q and K quantized, S runs on the packed NVFP4 codes
+  CUtensorMap tq4, tk4;
+  if (f16 && !(encode_codes(&tq4, wsb + w.qc, BH, Lq, D) && encode_codes(&tk4, wsb + w.kc, BH, Lk, D)))
+    return cuda_fail(cudaErrorInvalidValue);
   {
     ProfScope ps("attn_bwd_dkdv", s);
-    e = launch_bwd_dkdv(D, f16, (flags & ATTNQAT_QUANT_P) != 0, dof16, tq, tk, tv, tdo, a, BH, s);
+    e = launch_bwd_dkdv(D, f16, (flags & ATTNQAT_QUANT_P) != 0, dof16, tq, f16 ? tk4 : tk, tv, tdo,
+                        f16 ? tq4 : tq, a, BH, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   {
     ProfScope ps("attn_bwd_dq", s);
-    // with Q and K quantized, S runs on the packed NVFP4 codes
-    CUtensorMap tq4, tk4;
-    if (f16 && !(encode_codes(&tq4, wsb + w.qc, BH, Lq, D) && encode_codes(&tk4, wsb + w.kc, BH, Lk, D)))
-      return cuda_fail(cudaErrorInvalidValue);
     e = launch_bwd_dq(D, f16, dof16, f16 ? tq4 : tq, tk, tv, tdo, f16 ? tk4 : tk, a, BH, s);
   }
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);

@@ -23,28 +23,46 @@
 
 namespace attnqat {
 
-template <int D>
+// dK/dV kernel layout.  One TMEM buffer holds S_i, then dP_i, then S_{i+1}
+// (each released as soon as the row warps have read it into registers), so
+// the TMEM left over holds the scale factors of the NVFP4 S = fq(Q) fq(K)^T
+// (FP4S: Q and K quantized).  With FP4S the K codes stay resident and Q codes
+// stream through their own ring, so S never waits on the 16-bit Q tile,
+// which only dK = dS^T fq(Q) reads, late in the tile.
+template <int D, int FP4S>
 struct DkdvLayout {
   static constexpr int kTile = Tile<D>::kBytes;
   static constexpr int kXBytes = kBM * kBN * 2;
-  static constexpr int kK = 0;
-  static constexpr int kV = kK + kTile;
-  static constexpr int kQ = kV + kTile;          // 2 stages
-  static constexpr int kDO = kQ + 2 * kTile;     // 2 stages
-  static constexpr int kX = kDO + 2 * kTile;     // P^T, then dS^T
+  static constexpr int kCode = 128 * (D / 2);  // one packed NVFP4 tile
+  static constexpr int kSF = (D / 64) * 512;   // its scale-factor blocks
+  static constexpr int kK = 0;                 // 16-bit K, or K codes + scales (FP4S)
+  static constexpr int kKSF = kK + kCode;      // FP4S
+  static constexpr int kV = FP4S ? (kKSF + kSF + 1023) / 1024 * 1024 : kK + kTile;
+  static constexpr int kQ4 = kV + kTile;       // FP4S: 2 stages of Q codes
+  static constexpr int kQSF = kQ4 + (FP4S ? 2 * kCode : 0);
+  static constexpr int kQ = (kQSF + (FP4S ? 2 * kSF : 0) + 1023) / 1024 * 1024;  // 2 stages
+  static constexpr int kDO = kQ + 2 * kTile;   // 2 stages
+  static constexpr int kX = kDO + 2 * kTile;   // P^T, then dS^T
   static constexpr int kBar = kX + kXBytes;
   static constexpr int kBytes = kBar + 256;
   static constexpr int kDynSmem = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDV = 256, kTmemDK = 256 + D;
+  static constexpr uint32_t kTmemBuf = 0, kTmemDV = 128, kTmemDK = 128 + D;
+  static constexpr uint32_t kSFCols = (D / 64) * 4;
+  static constexpr uint32_t kTmemSFA = 128 + 2 * D;         // 2 stages (Q codes)
+  static constexpr uint32_t kTmemSFB = kTmemSFA + 2 * kSFCols;  // K codes
+  static constexpr uint32_t kCodeLayout = (D / 2 == 64) ? 4u : 6u;  // SW64 / SW32
+  static constexpr uint32_t kCodeSBO = 8 * (D / 2);
 };
 
 struct BwdBars {
   uint64_t kvfull;
   uint64_t afull[2], aempty[2];   // Q tiles (dK/dV kernel) or K tiles (dQ kernel)
   uint64_t bfull[2], bempty[2];   // dO tiles (dK/dV kernel) or V tiles (dQ kernel)
-  uint64_t k4full[2], k4empty[2]; // packed NVFP4 K tiles and scales (dQ kernel, NVFP4 S)
-  uint64_t sfull, sempty;   // S and dP in TMEM: filled together, released together
+  uint64_t cfull[2], cempty[2];   // packed NVFP4 Q (dK/dV kernel) or K (dQ kernel) codes + scales
+  // dK/dV kernel: the TMEM buffer's fills S_0, dP_0, S_1, ... one phase each;
+  // dQ kernel: S and dP filled together, released together
+  uint64_t sfull, sempty;
   uint64_t xfull, xempty;
   uint64_t done;
   uint32_t tmem_slot;
@@ -58,8 +76,8 @@ __device__ __forceinline__ void init_bwd_bars(BwdBars *b) {
     mbar_init(&b->aempty[s], 1);
     mbar_init(&b->bfull[s], 1);
     mbar_init(&b->bempty[s], 1);
-    mbar_init(&b->k4full[s], 1);
-    mbar_init(&b->k4empty[s], 1);
+    mbar_init(&b->cfull[s], 1);
+    mbar_init(&b->cempty[s], 1);
   }
   mbar_init(&b->sfull, 1);
   mbar_init(&b->sempty, kSoftWarps);
@@ -110,92 +128,95 @@ __device__ __forceinline__ void load_sdp(uint32_t tS, uint32_t tDP, int col0, ui
   tmem_ld_wait();
 }
 
-// One query tile for one thread of the dK/dV kernel (one query row, 64 key
-// columns starting at col0), from S and dP in registers: P~ = exp(S - m) and
-// fq(P~)/l (bf16, half a row of the transposed dV operand), and
-// dS = (P~/l)(dP - Delta) in float32, scaled by dsc and packed for the dK
-// operand.  P never leaves float32.
-template <int QP, int QKF16, bool MASKED>
-__device__ __forceinline__ void dkdv_tile(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
-                                          int valid_k, bool vq, float cl, float nml, float inv_l, float delta,
-                                          float dsc, uint32_t (&pw)[32], uint32_t (&dsw)[32]) {
+// 64 columns (one thread's half row) of one 32-bit TMEM tile into registers.
+__device__ __forceinline__ void load_cols64(uint32_t taddr, uint32_t (&v)[64]) {
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(v));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+  tmem_ld_wait();
+}
+
+// dK/dV kernel, first half of a query tile for one thread (one query row, 64
+// key columns from col0): P~ = exp(S - m) (rebuilt exactly as the forward
+// builds it: same bits, same blocks of 16 keys) and the dV operand row,
+// fq(P~)/l in bf16 (or P~/l when P is not quantized).  P~ stays in float32
+// for dS.
+template <int QP, bool MASKED>
+__device__ __forceinline__ void dkdv_probs(const uint32_t (&sv)[64], int col0, int valid_k, bool vq, float cl,
+                                           float nml, float inv_l, float (&p)[64], uint32_t (&pw)[32]) {
   const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    float p[32];
+  for (int i = 0; i < 32; ++i) {
+    const float2 x = fma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), cl2, nml2);
+    const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
+    p[2 * i] = (vq && (!MASKED || col0 + 2 * i < valid_k)) ? e0 : 0.0f;
+    p[2 * i + 1] = (vq && (!MASKED || col0 + 2 * i + 1 < valid_k)) ? e1 : 0.0f;
+  }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float2 x = fma2(make_float2(__uint_as_float(sv[32 * c + 2 * i]), __uint_as_float(sv[32 * c + 2 * i + 1])),
-                            cl2, nml2);
-      const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
-      p[2 * i] = (vq && (!MASKED || col0 + c * 32 + 2 * i < valid_k)) ? e0 : 0.0f;
-      p[2 * i + 1] = (vq && (!MASKED || col0 + c * 32 + 2 * i + 1 < valid_k)) ? e1 : 0.0f;
-    }
+  for (int b = 0; b < 4; ++b) {
+    if (QP) {
+      uint32_t rr[8];
+      const float f = fq16_probs(p + 16 * b, rr) * inv_l;
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      if (QP) {
-        uint32_t rr[8];
-        const float s = fq16_probs(p + 16 * b, rr);
-        const float f = s * inv_l;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 g = unpack_f16x2(rr[i]);
-          pw[16 * c + 8 * b + i] = pack_bf16x2(g.x * f, g.y * f);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          pw[16 * c + 8 * b + i] = pack_bf16x2(p[16 * b + 2 * i] * inv_l, p[16 * b + 2 * i + 1] * inv_l);
+      for (int i = 0; i < 8; ++i) {
+        const float2 g = unpack_f16x2(rr[i]);
+        pw[8 * b + i] = pack_bf16x2(g.x * f, g.y * f);
       }
-    }
-    const float pf = inv_l * dsc;
+    } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float d0 = p[2 * i] * pf * (__uint_as_float(dv[32 * c + 2 * i]) - delta);
-      const float d1 = p[2 * i + 1] * pf * (__uint_as_float(dv[32 * c + 2 * i + 1]) - delta);
-      dsw[16 * c + i] = pack_ds<QKF16>(d0, d1);
+      for (int i = 0; i < 8; ++i)
+        pw[8 * b + i] = pack_bf16x2(p[16 * b + 2 * i] * inv_l, p[16 * b + 2 * i + 1] * inv_l);
     }
   }
 }
 
-// The same for the all-quantized path with the exact fp16 copy dO * 2^e:
-// dP' = dP 2^e arrives from TMEM; the dV operand is fq(P~)/l * 2^14 in fp16
-// (r times the per-block factor s/l * 2^14: 11 significant bits, and in
-// fp16's normal range for every nonzero value while Lk <= 2^17); and
+// Second half: dS = (P~/l)(dP - Delta) in float32, scaled by dsc (pf =
+// dsc / l) and packed for the dK operand.
+template <int QKF16>
+__device__ __forceinline__ void dkdv_ds(const float (&p)[64], const uint32_t (&dv)[64], float pf, float delta,
+                                        uint32_t (&dsw)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float d0 = p[2 * i] * pf * (__uint_as_float(dv[2 * i]) - delta);
+    const float d1 = p[2 * i + 1] * pf * (__uint_as_float(dv[2 * i + 1]) - delta);
+    dsw[i] = pack_ds<QKF16>(d0, d1);
+  }
+}
+
+// The same two halves for the all-quantized path with the exact fp16 copy
+// dO * 2^e: the dV operand is fq(P~)/l * 2^14 in fp16 (r times the per-block
+// factor s/l * 2^14: 11 significant bits, and in fp16's normal range for every
+// nonzero value while Lk <= 2^17); dP' = dP 2^e arrives from TMEM and
 // dS * dsc = P~/l * (dP' 2^-e - Delta) * dsc = P~ * fma(dP', a1, b1) with
 // a1 = 2^-e dsc / l, b1 = -Delta dsc / l.  Rows past Lq come in with
 // nml = -inf, so their P~ is 0 without a per-element test.
 template <bool MASKED>
-__device__ __forceinline__ void dkdv_tile_f16(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
-                                              int valid_k, float cl, float nml, float vf, float a1, float b1,
-                                              uint32_t (&pw)[32], uint32_t (&dsw)[32]) {
+__device__ __forceinline__ void dkdv_probs_f16(const uint32_t (&sv)[64], int col0, int valid_k, float cl,
+                                               float nml, float vf, float (&p)[64], uint32_t (&pw)[32]) {
   const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 x = fma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), cl2, nml2);
+    const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
+    p[2 * i] = (!MASKED || col0 + 2 * i < valid_k) ? e0 : 0.0f;
+    p[2 * i + 1] = (!MASKED || col0 + 2 * i + 1 < valid_k) ? e1 : 0.0f;
+  }
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    uint32_t rr[8];
+    const uint32_t s2 = f16x2_broadcast(fq16_probs(p + 16 * b, rr) * vf);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pw[8 * b + i] = hmul2_u32(rr[i], s2);
+  }
+}
+
+__device__ __forceinline__ void dkdv_ds_f16(const float (&p)[64], const uint32_t (&dv)[64], float a1, float b1,
+                                            uint32_t (&dsw)[32]) {
   const float2 a12 = make_float2(a1, a1), b12 = make_float2(b1, b1);
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    float p[32];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float2 x = fma2(make_float2(__uint_as_float(sv[32 * c + 2 * i]), __uint_as_float(sv[32 * c + 2 * i + 1])),
-                            cl2, nml2);
-      const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
-      p[2 * i] = (!MASKED || col0 + c * 32 + 2 * i < valid_k) ? e0 : 0.0f;
-      p[2 * i + 1] = (!MASKED || col0 + c * 32 + 2 * i + 1 < valid_k) ? e1 : 0.0f;
-    }
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      uint32_t rr[8];
-      const uint32_t s2 = f16x2_broadcast(fq16_probs(p + 16 * b, rr) * vf);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) pw[16 * c + 8 * b + i] = hmul2_u32(rr[i], s2);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float2 g = fma2(make_float2(__uint_as_float(dv[32 * c + 2 * i]), __uint_as_float(dv[32 * c + 2 * i + 1])),
-                            a12, b12);
-      const float2 d = mul2(make_float2(p[2 * i], p[2 * i + 1]), g);
-      dsw[16 * c + i] = pack_f16x2(d.x, d.y);
-    }
+  for (int i = 0; i < 32; ++i) {
+    const float2 g = fma2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), a12, b12);
+    const float2 d = mul2(make_float2(p[2 * i], p[2 * i + 1]), g);
+    dsw[i] = pack_f16x2(d.x, d.y);
   }
 }
 
@@ -203,8 +224,9 @@ template <int D, int QP, int QKF16, int DOF16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                         const BwdArgs a) {
-  using L = DkdvLayout<D>;
+                         const __grid_constant__ CUtensorMap tmQ4, const BwdArgs a) {
+  constexpr int FP4S = QKF16;  // quantized Q and K: S on the NVFP4 path
+  using L = DkdvLayout<D, FP4S>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
@@ -232,67 +254,110 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmDO);
-      mbar_arrive_expect_tx(&bars->kvfull, 2 * L::kTile);
-      load_tile<D>(smem + L::kK, &tmK, &bars->kvfull, kt * kBN, bh);
+      if (FP4S) prefetch_tmap(&tmQ4);
+      mbar_arrive_expect_tx(&bars->kvfull, (FP4S ? L::kCode + L::kSF : L::kTile) + L::kTile);
+      if (FP4S) {
+        tma_load_3d(smem + L::kK, &tmK, &bars->kvfull, 0, kt * kBN, bh);
+        bulk_load(smem + L::kKSF, a.ksf + (static_cast<size_t>(bh) * a.nk_tiles + kt) * L::kSF, L::kSF,
+                  &bars->kvfull);
+      } else {
+        load_tile<D>(smem + L::kK, &tmK, &bars->kvfull, kt * kBN, bh);
+      }
       load_tile<D>(smem + L::kV, &tmV, &bars->kvfull, kt * kBN, bh);
-      int issued = 0;
+      // per query tile, in the order the MMAs need them: Q codes (S), dO (dP,
+      // then dV), 16-bit Q (dK; with !FP4S also S)
+      int nc = 0, nd = 0, nqh = 0;  // tiles issued per ring
       for (int i = 0; i < nq; ++i) {
         const int st = i & 1;
-        if (i >= 2 && !mbar_wait(&bars->aempty[st], ((i >> 1) - 1) & 1, abort)) break;
-        mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
-        load_tile<D>(smem + L::kQ + st * L::kTile, &tmQ, &bars->afull[st], i * kBM, bh);
-        if (i >= 2 && !mbar_wait(&bars->bempty[st], ((i >> 1) - 1) & 1, abort)) {
-          issued = i + 1;
-          break;
+        const int ph = ((i >> 1) - 1) & 1;
+        if (FP4S) {
+          if (i >= 2 && !mbar_wait(&bars->cempty[st], ph, abort)) break;
+          mbar_arrive_expect_tx(&bars->cfull[st], L::kCode + L::kSF);
+          tma_load_3d(smem + L::kQ4 + st * L::kCode, &tmQ4, &bars->cfull[st], 0, i * kBM, bh);
+          bulk_load(smem + L::kQSF + st * L::kSF, a.qsf + (static_cast<size_t>(bh) * nq + i) * L::kSF, L::kSF,
+                    &bars->cfull[st]);
+          nc = i + 1;
         }
+        if (i >= 2 && !mbar_wait(&bars->bempty[st], ph, abort)) break;
         mbar_arrive_expect_tx(&bars->bfull[st], L::kTile);
         load_tile<D>(smem + L::kDO + st * L::kTile, &tmDO, &bars->bfull[st], i * kBM, bh);
-        issued = i + 1;
+        nd = i + 1;
+        if (i >= 2 && !mbar_wait(&bars->aempty[st], ph, abort)) break;
+        mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
+        load_tile<D>(smem + L::kQ + st * L::kTile, &tmQ, &bars->afull[st], i * kBM, bh);
+        nqh = i + 1;
       }
       if (*abort) {
         mbar_wait_drain(&bars->kvfull, 0);
-        for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) {
-          mbar_wait_drain(&bars->afull[i & 1], (i >> 1) & 1);
-          mbar_wait_drain(&bars->bfull[i & 1], (i >> 1) & 1);
-        }
+        for (int i = (nc > 2 ? nc - 2 : 0); i < nc; ++i) mbar_wait_drain(&bars->cfull[i & 1], (i >> 1) & 1);
+        for (int i = (nd > 2 ? nd - 2 : 0); i < nd; ++i) mbar_wait_drain(&bars->bfull[i & 1], (i >> 1) & 1);
+        for (int i = (nqh > 2 ? nqh - 2 : 0); i < nqh; ++i) mbar_wait_drain(&bars->afull[i & 1], (i >> 1) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_f16(kBM, kBN, !QKF16, false, false);   // Q K^T
+      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);  // Q K^T
       constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
       constexpr uint32_t idV = idesc_f16(kBN, D, !DOF16, true, true);       // P^T dO
       constexpr uint32_t idK = idesc_f16(kBN, D, !QKF16, true, true);       // dS^T Q
       const uint32_t kaddr = sbase + L::kK, vaddr = sbase + L::kV, xaddr = sbase + L::kX;
+      const uint32_t tbuf = tmem + L::kTmemBuf;
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
-      // S_i and dP_i into TMEM; one commit signals both
-      // dP first: the dO slot frees earlier (after dV) than the Q slot (after
-      // dK), so the Q tile's load has dP's duration to land
-      auto issue_sdp = [&](int i) -> bool {
-        if (!mbar_wait(&bars->bfull[i & 1], (i >> 1) & 1, abort)) return false;
+      if (ok && FP4S) {
         tc_fence_after();
-        mma_kmajor(tmem + L::kTmemDP, sbase + L::kDO + (i & 1) * L::kTile, vaddr, D / 16, idDP, false);
-        if (!mbar_wait(&bars->afull[i & 1], (i >> 1) & 1, abort)) return false;
-        tc_fence_after();
-        mma_kmajor(tmem + L::kTmemS, sbase + L::kQ + (i & 1) * L::kTile, kaddr, D / 16, idS, false);
+        for (int kc = 0; kc < D / 64; ++kc)
+          tmem_cp_32x128b_x4(tmem + L::kTmemSFB + kc * 4, sdesc_make(sbase + L::kKSF + kc * 512, 16, 128, 0));
+      }
+      // S_i into the TMEM buffer (fill 2i); the buffer's previous fill (dP_{i-1})
+      // has been released by the caller's wait
+      auto issue_s = [&](int i) -> bool {
+        const int st = i & 1;
+        const uint32_t ph = (i >> 1) & 1;
+        if (FP4S) {
+          if (!mbar_wait(&bars->cfull[st], ph, abort)) return false;
+          tc_fence_after();
+          const uint32_t sfa = tmem + L::kTmemSFA + st * L::kSFCols;
+          const uint32_t qaddr = sbase + L::kQ4 + st * L::kCode;
+          for (int kc = 0; kc < D / 64; ++kc)
+            tmem_cp_32x128b_x4(sfa + kc * 4, sdesc_make(sbase + L::kQSF + st * L::kSF + kc * 512, 16, 128, 0));
+          for (int kk = 0; kk < D / 64; ++kk)
+            umma_fp4(tbuf, sdesc_make(qaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout),
+                     sdesc_make(kaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout), idS, sfa + kk * 4,
+                     tmem + L::kTmemSFB + kk * 4, kk > 0 ? 1u : 0u);
+          umma_commit(&bars->cempty[st]);
+        } else {
+          if (!mbar_wait(&bars->afull[st], ph, abort)) return false;
+          tc_fence_after();
+          mma_kmajor(tbuf, sbase + L::kQ + st * L::kTile, kaddr, D / 16, idS, false);
+        }
         umma_commit(&bars->sfull);
         return true;
       };
-      if (ok) ok = issue_sdp(0);
+      if (ok) ok = issue_s(0);
       for (int i = 0; ok && i < nq; ++i) {
         const int st = i & 1;
-        if (i + 1 < nq) {
-          ok = mbar_wait(&bars->sempty, i & 1, abort) && issue_sdp(i + 1);
-          if (!ok) break;
+        const uint32_t ph = (i >> 1) & 1;
+        // dP_i once the rows have read S_i (fill 2i)
+        if (!mbar_wait(&bars->sempty, (2 * i) & 1, abort) || !mbar_wait(&bars->bfull[st], ph, abort)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        mma_kmajor(tbuf, sbase + L::kDO + st * L::kTile, vaddr, D / 16, idDP, false);
+        umma_commit(&bars->sfull);
         // dV += (fq(P~)/l)^T dO_i : A = X (M = keys, MN-major), B = dO (N = D, MN-major)
         if (!mbar_wait(&bars->xfull, (2 * i) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         mma_mn_mn(tmem + L::kTmemDV, xaddr, sbase + L::kDO + st * L::kTile, kBM / 16, idV, i > 0);
         umma_commit(&bars->xempty);
         umma_commit(&bars->bempty[st]);
+        // S_{i+1} once the rows have read dP_i (fill 2i+1)
+        if (i + 1 < nq) {
+          if (!mbar_wait(&bars->sempty, (2 * i + 1) & 1, abort) || !issue_s(i + 1)) { ok = false; break; }
+        }
         // dK += dS^T Q_i
         if (!mbar_wait(&bars->xfull, (2 * i + 1) & 1, abort)) { ok = false; break; }
+        if (FP4S && !mbar_wait(&bars->afull[st], ph, abort)) { ok = false; break; }
         tc_fence_after();
         mma_mn_mn(tmem + L::kTmemDK, xaddr, sbase + L::kQ + st * L::kTile, kBM / 16, idK, i > 0);
         umma_commit(&bars->xempty);
@@ -307,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float cl = a.scale_log2;
     const float dsc = ds_scale<QKF16>(a.stats);
     const uint32_t xaddr = sbase + L::kX;
-    const uint32_t tS = tmem + rr.lane_addr + L::kTmemS, tDP = tmem + rr.lane_addr + L::kTmemDP;
+    const uint32_t tbuf = tmem + rr.lane_addr + L::kTmemBuf + col0;
     bool ok = true;
     // row statistics of the current query tile, prefetched one tile ahead
     auto load_stats = [&](int i, float &m, float &lse, float &delta) {
@@ -326,34 +391,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m = m_n, lse = lse_n, delta = delta_n;
       load_stats(i + 1, m_n, lse_n, delta_n);
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
+      float p[64];
       uint32_t pw[32], dsw[32];
-      uint32_t sv[64], dv[64];
-      if (!mbar_wait(&bars->sfull, i & 1, abort)) { ok = false; break; }
-      tc_fence_after();
-      load_sdp(tS, tDP, col0, sv, dv);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sempty);
-      if (DOF16) {
-        const float nml = vq ? -(m * kLog2e) : -INFINITY;
-        const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
-        const float a1 = inv_l * dsc / dos, b1 = -delta * inv_l * dsc;
-        if (valid_k < kBN)
-          dkdv_tile_f16<true>(sv, dv, col0, valid_k, cl, nml, vf, a1, b1, pw, dsw);
-        else
-          dkdv_tile_f16<false>(sv, dv, col0, valid_k, cl, nml, vf, a1, b1, pw, dsw);
-      } else {
-        const float nml = -(m * kLog2e);
-        if (valid_k < kBN)
-          dkdv_tile<QP, QKF16, true>(sv, dv, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
-        else
-          dkdv_tile<QP, QKF16, false>(sv, dv, col0, valid_k, vq, cl, nml, inv_l, delta, dsc, pw, dsw);
+      {
+        // S_i: read, release the buffer for dP_i, build P~ and the dV operand
+        uint32_t sv[64];
+        if (!mbar_wait(&bars->sfull, (2 * i) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        load_cols64(tbuf, sv);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->sempty);
+        if (DOF16) {
+          const float nml = vq ? -(m * kLog2e) : -INFINITY;
+          const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
+          if (valid_k < kBN)
+            dkdv_probs_f16<true>(sv, col0, valid_k, cl, nml, vf, p, pw);
+          else
+            dkdv_probs_f16<false>(sv, col0, valid_k, cl, nml, vf, p, pw);
+        } else {
+          const float nml = -(m * kLog2e);
+          if (valid_k < kBN)
+            dkdv_probs<QP, true>(sv, col0, valid_k, vq, cl, nml, inv_l, p, pw);
+          else
+            dkdv_probs<QP, false>(sv, col0, valid_k, vq, cl, nml, inv_l, p, pw);
+        }
       }
+      // X = (fq(P~)/l)^T once dK_{i-1} has read the previous dS^T
       if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, pw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
+      {
+        // dP_i: read, release the buffer for S_{i+1}, build dS
+        uint32_t dv[64];
+        if (!mbar_wait(&bars->sfull, (2 * i + 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        load_cols64(tbuf, dv);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->sempty);
+        if (DOF16)
+          dkdv_ds_f16(p, dv, inv_l * dsc / dos, -delta * inv_l * dsc, dsw);
+        else
+          dkdv_ds<QKF16>(p, dv, inv_l * dsc, delta, dsw);
+      }
+      // X = dS^T once dV_i has read the P^T
       if (!mbar_wait(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
       fence_proxy_async_smem();
@@ -526,11 +610,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = j & 1;
         const int ph = ((j >> 1) - 1) & 1;
         if (FP4S) {
-          if (j >= 2 && !mbar_wait(&bars->k4empty[st], ph, abort)) break;
-          mbar_arrive_expect_tx(&bars->k4full[st], L::kCode + L::kSF);
-          tma_load_3d(smem + L::kK4 + st * L::kCode, &tmK4, &bars->k4full[st], 0, j * kBN, bh);
+          if (j >= 2 && !mbar_wait(&bars->cempty[st], ph, abort)) break;
+          mbar_arrive_expect_tx(&bars->cfull[st], L::kCode + L::kSF);
+          tma_load_3d(smem + L::kK4 + st * L::kCode, &tmK4, &bars->cfull[st], 0, j * kBN, bh);
           bulk_load(smem + L::kKSF + st * L::kSF, a.ksf + (static_cast<size_t>(bh) * nk + j) * L::kSF, L::kSF,
-                    &bars->k4full[st]);
+                    &bars->cfull[st]);
           n4 = j + 1;
         }
         if (j >= 2 && !mbar_wait(&bars->bempty[st], ph, abort)) break;
@@ -544,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort) {
         mbar_wait_drain(&bars->kvfull, 0);
-        for (int j = (n4 > 2 ? n4 - 2 : 0); j < n4; ++j) mbar_wait_drain(&bars->k4full[j & 1], (j >> 1) & 1);
+        for (int j = (n4 > 2 ? n4 - 2 : 0); j < n4; ++j) mbar_wait_drain(&bars->cfull[j & 1], (j >> 1) & 1);
         for (int j = (nv > 2 ? nv - 2 : 0); j < nv; ++j) mbar_wait_drain(&bars->bfull[j & 1], (j >> 1) & 1);
         for (int j = (nkh > 2 ? nkh - 2 : 0); j < nkh; ++j) mbar_wait_drain(&bars->afull[j & 1], (j >> 1) & 1);
       }
@@ -570,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_kmajor(tmem + L::kTmemDP, doaddr, sbase + L::kV + st * L::kTile, D / 16, idDP, false);
         umma_commit(&bars->bempty[st]);
         if (FP4S) {
-          if (!mbar_wait(&bars->k4full[st], ph, abort)) return false;
+          if (!mbar_wait(&bars->cfull[st], ph, abort)) return false;
           tc_fence_after();
           const uint32_t sfb = tmem + L::kTmemSFB + st * L::kSFCols;
           const uint32_t kaddr = sbase + L::kK4 + st * L::kCode;
@@ -580,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_fp4(tmem + L::kTmemS, sdesc_make(qaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout),
                      sdesc_make(kaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout), idS,
                      tmem + L::kTmemSFA + kk * 4, sfb + kk * 4, kk > 0 ? 1u : 0u);
-          umma_commit(&bars->k4empty[st]);
+          umma_commit(&bars->cempty[st]);
         } else {
           if (!mbar_wait(&bars->afull[st], ph, abort)) return false;
           tc_fence_after();
@@ -688,32 +772,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, int QP, int QKF16, int DOF16>
 static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                 const CUtensorMap &tdo, const BwdArgs &a, int BH, cudaStream_t stream) {
-  using L = DkdvLayout<D>;
+                                 const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
+                                 cudaStream_t stream) {
+  using L = DkdvLayout<D, QKF16>;
+  static_assert(L::kDynSmem <= 232448, "dK/dV shared memory over the 227 KB limit");
+  static_assert(L::kTmemSFB + L::kSFCols <= L::kTmemCols, "dK/dV TMEM over 512 columns");
   auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16, DOF16>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(a.nk_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<dim3(a.nk_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, tq4, a);
   return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t dkdv_dispatch(bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
                                  const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
-                                 const BwdArgs &a, int BH, cudaStream_t stream) {
-  if (do_f16) return launch_dkdv_t<D, 1, 1, 1>(tq, tk, tv, tdo, a, BH, stream);
+                                 const CUtensorMap &tq4, const BwdArgs &a, int BH, cudaStream_t stream) {
+  if (do_f16) return launch_dkdv_t<D, 1, 1, 1>(tq, tk, tv, tdo, tq4, a, BH, stream);
   if (qk_f16)
-    return quant_p ? launch_dkdv_t<D, 1, 1, 0>(tq, tk, tv, tdo, a, BH, stream)
-                   : launch_dkdv_t<D, 0, 1, 0>(tq, tk, tv, tdo, a, BH, stream);
-  return quant_p ? launch_dkdv_t<D, 1, 0, 0>(tq, tk, tv, tdo, a, BH, stream)
-                 : launch_dkdv_t<D, 0, 0, 0>(tq, tk, tv, tdo, a, BH, stream);
+    return quant_p ? launch_dkdv_t<D, 1, 1, 0>(tq, tk, tv, tdo, tq4, a, BH, stream)
+                   : launch_dkdv_t<D, 0, 1, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
+  return quant_p ? launch_dkdv_t<D, 1, 0, 0>(tq, tk, tv, tdo, tq4, a, BH, stream)
+                 : launch_dkdv_t<D, 0, 0, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
 cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
                             const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
-                            const BwdArgs &a, int BH, cudaStream_t stream) {
-  return D == 128 ? dkdv_dispatch<128>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, a, BH, stream)
-                  : dkdv_dispatch<64>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, a, BH, stream);
+                            const CUtensorMap &tq4, const BwdArgs &a, int BH, cudaStream_t stream) {
+  return D == 128 ? dkdv_dispatch<128>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, tq4, a, BH, stream)
+                  : dkdv_dispatch<64>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
 template <int D, int QKF16, int DOF16>

@@ -63,37 +63,40 @@ struct FwdBars {
   uint64_t ofull;
   uint32_t tmem_slot;
   int abort;
-  float part[2][kBM];   // per-row partial max / sum of the two column halves
+  float part[4][kBM];   // per-row partial max / sum of the column groups
 };
 
-// Row max over this thread's 64 columns (col0..col0+63) of one S tile.
-template <bool MASKED>
-__device__ __forceinline__ float row_max_half(uint32_t taddr, int col0, int valid) {
-  uint32_t r[32], t[32];
-  tmem_ld32(taddr + col0, r);
-  tmem_ld32(taddr + col0 + 32, t);
-  tmem_ld_wait();
+// Row max over this thread's NC columns (col0..col0+NC-1) of one S tile.
+template <bool MASKED, int NC>
+__device__ __forceinline__ float row_max_cols(uint32_t taddr, int col0, int valid) {
   float mx = -INFINITY;
+  uint32_t r[NC / 32][32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float a = (!MASKED || col0 + i < valid) ? __uint_as_float(r[i]) : -INFINITY;
-    const float b = (!MASKED || col0 + 32 + i < valid) ? __uint_as_float(t[i]) : -INFINITY;
-    mx = fmax3(mx, a, b);
+  for (int c = 0; c < NC / 32; ++c) tmem_ld32(taddr + col0 + 32 * c, r[c]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int c = 0; c < NC / 32; ++c) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float a = (!MASKED || col0 + 32 * c + i < valid) ? __uint_as_float(r[c][i]) : -INFINITY;
+      const float b = (!MASKED || col0 + 32 * c + i + 1 < valid) ? __uint_as_float(r[c][i + 1]) : -INFINITY;
+      mx = fmax3(mx, a, b);
+    }
   }
   return mx;
 }
 
-// Sweep-2 work for this thread's 64 columns of one S tile: P~ = exp2(S*cl +
+// Sweep-2 work for this thread's NC columns of one S tile: P~ = exp2(S*cl +
 // nml), partial row sum, fq(P~) (or P~ itself) packed into 16-bit pairs and
-// stored as columns col0..col0+63 (one swizzled chunk) of row `row` of the P
-// tile at `pbase`.
-template <int PV_F16, int QP, bool MASKED>
-__device__ __forceinline__ float prob_half(uint32_t taddr, int col0, int valid, float cl, float nml,
+// stored as columns col0..col0+NC-1 of row `row` of the P tile at `pbase`
+// (128-byte swizzled chunks of 64 columns).
+template <int PV_F16, int QP, bool MASKED, int NC>
+__device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, float cl, float nml,
                                            uint32_t pbase, uint32_t row) {
   float2 lsum = make_float2(0.0f, 0.0f);
   const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
+  for (int c = 0; c < NC / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + col0 + c * 32, r);
     tmem_ld_wait();
@@ -130,24 +133,31 @@ __device__ __forceinline__ float prob_half(uint32_t taddr, int col0, int valid, 
                                 : pack_bf16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1]);
       }
     }
-    // 32 keys = 16-byte units 4c .. 4c+3 of this thread's 64-key chunk
+    // 32 keys = four 16-byte units of the 64-key swizzled chunk holding them
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const uint32_t addr = pbase + static_cast<uint32_t>(col0 >> 6) * kChunkBytes + sw128_offset(row, 4 * c + u);
+      const int cc = col0 + 32 * c;
+      const uint32_t addr = pbase + static_cast<uint32_t>(cc >> 6) * kChunkBytes +
+                            sw128_offset(row, ((cc & 63) >> 3) + u);
       st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     }
   }
   return lsum.x + lsum.y;
 }
 
-// Merges a per-row partial value with the other column half's through
-// shared memory (named barrier 1 + lane quarter, 64 threads).
-__device__ __forceinline__ void pair_sync(int wq) {
-  asm volatile("bar.sync %0, 64;" ::"r"(1 + wq) : "memory");
+// Synchronises the G row warps of one TMEM lane quarter (named barrier
+// 1 + lane quarter), around the shared-memory merge of per-row partials.
+template <int G>
+__device__ __forceinline__ void group_sync(int wq) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + wq), "n"(32 * G) : "memory");
 }
 
-template <int D, int FP4S, int PV_F16, int QP>
-__global__ void __launch_bounds__(kThreads, 1)
+// Threads of a forward CTA with G row warps per TMEM lane quarter.
+template <int G>
+constexpr int fwd_threads() { return 64 + 128 * G; }
+
+template <int D, int FP4S, int PV_F16, int QP, int G>
+__global__ void __launch_bounds__(fwd_threads<G>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using L = FwdLayout<D, FP4S>;
@@ -176,8 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->sfull[b], 1);
-      mbar_init(&bars->sempty[b], kSoftWarps);
-      mbar_init(&bars->pfull[b], kSoftWarps);
+      mbar_init(&bars->sempty[b], 4 * G);
+      mbar_init(&bars->pfull[b], 4 * G);
       mbar_init(&bars->pempty[b], 1);
     }
     mbar_init(&bars->ofull, 1);
@@ -303,8 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- row warps --
+    constexpr int NC = kBN / G;  // columns per thread
     const RowRole rr(warp, lane);
-    const int col0 = rr.half * 64;
+    const int col0 = rr.half * NC;
     const int last_valid = a.Lk - (nk - 1) * kBN;  // keys in the last KV tile
     float mrow = -INFINITY;
     bool ok = true;
@@ -314,18 +325,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
-      const float mx = (j == nk - 1 && last_valid < kBN) ? row_max_half<true>(taddr, col0, last_valid)
-                                                         : row_max_half<false>(taddr, col0, kBN);
+      const float mx = (j == nk - 1 && last_valid < kBN) ? row_max_cols<true, NC>(taddr, col0, last_valid)
+                                                         : row_max_cols<false, NC>(taddr, col0, kBN);
       mrow = fmaxf(mrow, mx);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty[sb]);
     }
-    // both halves of a row see every tile, so both reach this merge
+    // every column group of a row sees every tile, so all reach this merge
     bars->part[rr.half][rr.row] = mrow;
-    pair_sync(rr.wq);
-    mrow = fmaxf(mrow, bars->part[rr.half ^ 1][rr.row]);
-    pair_sync(rr.wq);
+    group_sync<G>(rr.wq);
+#pragma unroll
+    for (int g = 0; g < G; ++g) mrow = fmaxf(mrow, bars->part[g][rr.row]);
+    group_sync<G>(rr.wq);
     const float m_scaled = mrow * a.sm_scale;
     const float nml = -(m_scaled * kLog2e);
     const float cl = a.scale_log2;
@@ -339,9 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
       if (j == nk - 1 && last_valid < kBN)
-        lsum += prob_half<PV_F16, QP, true>(taddr, col0, last_valid, cl, nml, pbase, rr.row);
+        lsum += prob_cols<PV_F16, QP, true, NC>(taddr, col0, last_valid, cl, nml, pbase, rr.row);
       else
-        lsum += prob_half<PV_F16, QP, false>(taddr, col0, kBN, cl, nml, pbase, rr.row);
+        lsum += prob_cols<PV_F16, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, rr.row);
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
@@ -353,31 +365,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue --
     if (ok && mbar_wait(&bars->ofull, 0, abort)) {
       bars->part[rr.half][rr.row] = lsum;
-      pair_sync(rr.wq);
-      lsum += bars->part[rr.half ^ 1][rr.row];
+      group_sync<G>(rr.wq);
+      lsum = 0.0f;
+#pragma unroll
+      for (int g = 0; g < G; ++g) lsum += bars->part[g][rr.row];
       tc_fence_after();
       const int q = qt * kBM + static_cast<int>(rr.row);
       const float inv_l = 1.0f / lsum;
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
+      constexpr int DC = D / G;            // output columns per thread
+      constexpr int W = DC < 32 ? DC : 32;  // columns per TMEM load
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        const int col = rr.half * (D / 2) + c * 32;
+      for (int c = 0; c < DC / W; ++c) {
+        const int col = rr.half * DC + c * W;
         uint32_t r[32];
-        tmem_ld32(tmem + rr.lane_addr + L::kTmemO + col, r);
+        if (W == 32) {
+          tmem_ld32(tmem + rr.lane_addr + L::kTmemO + col, r);
+        } else {
+          tmem_ld16(tmem + rr.lane_addr + L::kTmemO + col, *reinterpret_cast<uint32_t(*)[16]>(r));
+        }
         tmem_ld_wait();
         if (q < a.Lq) {
-          float f[32];
+          float f[W];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]) * inv_l;
-          uint32_t w[16];
+          for (int i = 0; i < W; ++i) f[i] = __uint_as_float(r[i]) * inv_l;
+          uint32_t w[W / 2];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+          for (int i = 0; i < W / 2; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
           uint4 *dst = reinterpret_cast<uint4 *>(a.o + rowoff + col);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int i = 0; i < W / 8; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
           float4 *d32 = reinterpret_cast<float4 *>(a.o32 + rowoff + col);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) d32[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+          for (int i = 0; i < W / 4; ++i) d32[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
         }
       }
       if (q < a.Lq && rr.half == 0) {
@@ -398,17 +418,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Row warps per TMEM lane quarter in the forward: 2, each owning 64 of the
+// 128 columns.  (4 per quarter, 32 columns each, measured no faster: the
+// forward is not limited by how many row warps hide latency.)
+constexpr int kFwdG = 2;
+
 template <int D, int FP4S, int PV_F16, int QP>
 static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const FwdArgs &a, int BH, cudaStream_t stream) {
   using L = FwdLayout<D, FP4S>;
   static_assert(L::kDynSmem <= 232448, "forward shared memory over the 227 KB limit");
   static_assert(!FP4S || L::kTmemSFB + L::kNSK * L::kSFCols <= L::kTmemCols, "forward TMEM over 512 columns");
-  auto kern = attn_fwd_kernel<D, FP4S, PV_F16, QP>;
+  auto kern = attn_fwd_kernel<D, FP4S, PV_F16, QP, kFwdG>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nq_tiles, BH);
-  kern<<<grid, kThreads, L::kDynSmem, stream>>>(tq, tk, tv, a);
+  kern<<<grid, fwd_threads<kFwdG>(), L::kDynSmem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

@@ -55,9 +55,12 @@ cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUte
 // map is over the exact fp16 copy dO * 2^e and the V map over fp16 fq(V): dP
 // is exact as before and dV takes fq(P~)/l * 2^14 as an fp16 operand; else
 // both maps are bf16.
+// With qk_f16, tk maps the packed NVFP4 K codes and tq4 the Q codes (as for
+// the forward; a.ksf/a.qsf their scale tiles) for S, and tq the fp16 fq(Q)
+// that dK = dS^T fq(Q) reads; otherwise tq/tk are bf16 and tq4 is unused.
 cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
                             const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
-                            const BwdArgs &a, int BH, cudaStream_t stream);
+                            const CUtensorMap &tq4, const BwdArgs &a, int BH, cudaStream_t stream);
 // dQ.  With qk_f16, tq maps the packed NVFP4 Q codes (as for the forward),
 // tk4 the K codes, a.qsf/a.ksf their scale tiles, and tk the fp16 fq(K) that
 // dQ = dS fq(K) reads; otherwise tq/tk are bf16 and tk4 is unused.
