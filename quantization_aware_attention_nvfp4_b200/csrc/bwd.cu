@@ -44,7 +44,8 @@ struct DkdvLayout {
   static constexpr int kDO = kQ + 2 * kTile;   // 2 stages
   static constexpr int kX = kDO + 2 * kTile;   // P^T, then dS^T
   static constexpr int kBar = kX + kXBytes;
-  static constexpr int kBytes = kBar + 256;
+  static constexpr int kBarBytes = 256;  // BwdBars (checked at the launch)
+  static constexpr int kBytes = kBar + kBarBytes;
   static constexpr int kDynSmem = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemBuf = 0, kTmemDV = 128, kTmemDK = 128 + D;
@@ -300,8 +301,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
       constexpr uint32_t idV = idesc_f16(kBN, D, !DOF16, true, true);       // P^T dO
       constexpr uint32_t idK = idesc_f16(kBN, D, !QKF16, true, true);       // dS^T Q
-      const uint32_t kaddr = sbase + L::kK, vaddr = sbase + L::kV, xaddr = sbase + L::kX;
+      const uint32_t kaddr = sbase + L::kK;
       const uint32_t tbuf = tmem + L::kTmemBuf;
+      // operand descriptors of the tiles' base addresses
+      const uint64_t dK = FP4S ? sdesc_make(kaddr, 16, L::kCodeSBO, L::kCodeLayout) : desc_k(kaddr);
+      const uint64_t dQ4 = sdesc_make(sbase + L::kQ4, 16, L::kCodeSBO, L::kCodeLayout);
+      const uint64_t dQSF = sdesc_make(sbase + L::kQSF, 16, 128, 0);
+      const uint64_t dQk = desc_k(sbase + L::kQ), dQmn = desc_mn(sbase + L::kQ);
+      const uint64_t dDOk = desc_k(sbase + L::kDO), dDOmn = desc_mn(sbase + L::kDO);
+      const uint64_t dVk = desc_k(sbase + L::kV), dX = desc_mn(sbase + L::kX);
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
       if (ok && FP4S) {
         tc_fence_after();
@@ -317,18 +325,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&bars->cfull[st], ph, abort)) return false;
           tc_fence_after();
           const uint32_t sfa = tmem + L::kTmemSFA + st * L::kSFCols;
-          const uint32_t qaddr = sbase + L::kQ4 + st * L::kCode;
-          for (int kc = 0; kc < D / 64; ++kc)
-            tmem_cp_32x128b_x4(sfa + kc * 4, sdesc_make(sbase + L::kQSF + st * L::kSF + kc * 512, 16, 128, 0));
+          const uint64_t dQs = sdesc_add(dQ4, st * L::kCode);
+#pragma unroll
+          for (int kc = 0; kc < D / 64; ++kc) tmem_cp_32x128b_x4(sfa + kc * 4, sdesc_add(dQSF, st * L::kSF + kc * 512));
+#pragma unroll
           for (int kk = 0; kk < D / 64; ++kk)
-            umma_fp4(tbuf, sdesc_make(qaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout),
-                     sdesc_make(kaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout), idS, sfa + kk * 4,
+            umma_fp4(tbuf, sdesc_add(dQs, kk * 32), sdesc_add(dK, kk * 32), idS, sfa + kk * 4,
                      tmem + L::kTmemSFB + kk * 4, kk > 0 ? 1u : 0u);
           umma_commit(&bars->cempty[st]);
         } else {
           if (!mbar_wait(&bars->afull[st], ph, abort)) return false;
           tc_fence_after();
-          mma_kmajor(tbuf, sbase + L::kQ + st * L::kTile, kaddr, D / 16, idS, false);
+          mma_kmajor<D / 16>(tbuf, sdesc_add(dQk, st * L::kTile), dK, idS, false);
         }
         umma_commit(&bars->sfull);
         return true;
@@ -343,12 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        mma_kmajor(tbuf, sbase + L::kDO + st * L::kTile, vaddr, D / 16, idDP, false);
+        mma_kmajor<D / 16>(tbuf, sdesc_add(dDOk, st * L::kTile), dVk, idDP, false);
         umma_commit(&bars->sfull);
         // dV += (fq(P~)/l)^T dO_i : A = X (M = keys, MN-major), B = dO (N = D, MN-major)
         if (!mbar_wait(&bars->xfull, (2 * i) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        mma_mn_mn(tmem + L::kTmemDV, xaddr, sbase + L::kDO + st * L::kTile, kBM / 16, idV, i > 0);
+        mma_mn_mn<kBM / 16>(tmem + L::kTmemDV, dX, sdesc_add(dDOmn, st * L::kTile), idV, i > 0);
         umma_commit(&bars->xempty);
         umma_commit(&bars->bempty[st]);
         // S_{i+1} once the rows have read dP_i (fill 2i+1)
@@ -359,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bars->xfull, (2 * i + 1) & 1, abort)) { ok = false; break; }
         if (FP4S && !mbar_wait(&bars->afull[st], ph, abort)) { ok = false; break; }
         tc_fence_after();
-        mma_mn_mn(tmem + L::kTmemDK, xaddr, sbase + L::kQ + st * L::kTile, kBM / 16, idK, i > 0);
+        mma_mn_mn<kBM / 16>(tmem + L::kTmemDK, dX, sdesc_add(dQmn, st * L::kTile), idK, i > 0);
         umma_commit(&bars->xempty);
         umma_commit(&bars->aempty[st]);
       }
@@ -510,7 +518,8 @@ struct DqLayout {
   static constexpr int kK4 = kX + kXBytes;      // FP4S: 2 stages of K codes
   static constexpr int kKSF = kK4 + (FP4S ? 2 * kCode : 0);
   static constexpr int kBar = kKSF + (FP4S ? 2 * kSF : 0);
-  static constexpr int kBytes = kBar + 256;
+  static constexpr int kBarBytes = 256;  // BwdBars (checked at the launch)
+  static constexpr int kBytes = kBar + kBarBytes;
   static constexpr int kDynSmem = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDQ = 256;
@@ -638,7 +647,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);  // Q K^T
       constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
       constexpr uint32_t idQ = idesc_f16(kBM, D, !QKF16, false, true);     // dS (K-major) * K (MN-major)
-      const uint32_t qaddr = sbase + L::kQ, doaddr = sbase + L::kDO, xaddr = sbase + L::kX;
+      const uint32_t qaddr = sbase + L::kQ;
+      // operand descriptors of the tiles' base addresses
+      const uint64_t dQ = FP4S ? sdesc_make(qaddr, 16, L::kCodeSBO, L::kCodeLayout) : desc_k(qaddr);
+      const uint64_t dDO = desc_k(sbase + L::kDO), dVk = desc_k(sbase + L::kV);
+      const uint64_t dK4 = sdesc_make(sbase + L::kK4, 16, L::kCodeSBO, L::kCodeLayout);
+      const uint64_t dKSF = sdesc_make(sbase + L::kKSF, 16, 128, 0);
+      const uint64_t dKk = desc_k(sbase + L::kK), dKmn = desc_mn(sbase + L::kK), dX = desc_k(sbase + L::kX);
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
       if (ok && FP4S) {
         tc_fence_after();
@@ -651,24 +666,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (j >> 1) & 1;
         if (!mbar_wait(&bars->bfull[st], ph, abort)) return false;
         tc_fence_after();
-        mma_kmajor(tmem + L::kTmemDP, doaddr, sbase + L::kV + st * L::kTile, D / 16, idDP, false);
+        mma_kmajor<D / 16>(tmem + L::kTmemDP, dDO, sdesc_add(dVk, st * L::kTile), idDP, false);
         umma_commit(&bars->bempty[st]);
         if (FP4S) {
           if (!mbar_wait(&bars->cfull[st], ph, abort)) return false;
           tc_fence_after();
           const uint32_t sfb = tmem + L::kTmemSFB + st * L::kSFCols;
-          const uint32_t kaddr = sbase + L::kK4 + st * L::kCode;
-          for (int kc = 0; kc < D / 64; ++kc)
-            tmem_cp_32x128b_x4(sfb + kc * 4, sdesc_make(sbase + L::kKSF + st * L::kSF + kc * 512, 16, 128, 0));
+          const uint64_t dKs = sdesc_add(dK4, st * L::kCode);
+#pragma unroll
+          for (int kc = 0; kc < D / 64; ++kc) tmem_cp_32x128b_x4(sfb + kc * 4, sdesc_add(dKSF, st * L::kSF + kc * 512));
+#pragma unroll
           for (int kk = 0; kk < D / 64; ++kk)
-            umma_fp4(tmem + L::kTmemS, sdesc_make(qaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout),
-                     sdesc_make(kaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout), idS,
+            umma_fp4(tmem + L::kTmemS, sdesc_add(dQ, kk * 32), sdesc_add(dKs, kk * 32), idS,
                      tmem + L::kTmemSFA + kk * 4, sfb + kk * 4, kk > 0 ? 1u : 0u);
           umma_commit(&bars->cempty[st]);
         } else {
           if (!mbar_wait(&bars->afull[st], ph, abort)) return false;
           tc_fence_after();
-          mma_kmajor(tmem + L::kTmemS, qaddr, sbase + L::kK + st * L::kTile, D / 16, idS, false);
+          mma_kmajor<D / 16>(tmem + L::kTmemS, dQ, sdesc_add(dKk, st * L::kTile), idS, false);
         }
         umma_commit(&bars->sfull);
         return true;
@@ -683,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bars->xfull, j & 1, abort)) { ok = false; break; }
         if (FP4S && !mbar_wait(&bars->afull[st], (j >> 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        mma_a_k_b_mn(tmem + L::kTmemDQ, xaddr, sbase + L::kK + st * L::kTile, kBN / 16, idQ, j > 0);
+        mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemDQ, dX, sdesc_add(dKmn, st * L::kTile), idQ, j > 0);
         umma_commit(&bars->xempty);
         umma_commit(&bars->aempty[st]);
       }
@@ -776,6 +791,7 @@ static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, c
                                  cudaStream_t stream) {
   using L = DkdvLayout<D, QKF16>;
   static_assert(L::kDynSmem <= 232448, "dK/dV shared memory over the 227 KB limit");
+  static_assert(sizeof(BwdBars) <= L::kBarBytes, "dK/dV barrier block larger than its reservation");
   static_assert(L::kTmemSFB + L::kSFCols <= L::kTmemCols, "dK/dV TMEM over 512 columns");
   auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16, DOF16>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
@@ -809,6 +825,7 @@ static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, con
                                cudaStream_t stream) {
   using L = DqLayout<D, QKF16>;
   static_assert(L::kDynSmem <= 232448, "dQ shared memory over the 227 KB limit");
+  static_assert(sizeof(BwdBars) <= L::kBarBytes, "dQ barrier block larger than its reservation");
   static_assert(L::kTmemSFB + 2 * L::kSFCols <= L::kTmemCols, "dQ TMEM over 512 columns");
   auto kern = attn_bwd_dq_kernel<D, QKF16, DOF16>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);

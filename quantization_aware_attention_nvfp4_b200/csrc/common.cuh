@@ -64,40 +64,57 @@ __device__ __forceinline__ float do_scale(const float *stats) {
   return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
 }
 
+// The MMA helpers below take the descriptors of the operand tiles' base
+// addresses and advance them by adding (byte offset >> 4) to the 14-bit
+// address field (tiles sit below 256 KB of shared memory, so the field never
+// carries): the issuing thread does no address arithmetic per instruction.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t byte_off) {
+  return d + static_cast<uint64_t>(byte_off >> 4);
+}
+
+// Descriptors of 128-byte-swizzled 16-bit tiles: K-major, and MN-major with
+// 64-element chunks kChunkBytes apart.
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) { return sdesc_sw128(saddr, 16, 1024); }
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) { return sdesc_sw128(saddr, kChunkBytes, 1024); }
+
 // Issues D[tmem] (+)= A * B^T for two K-major 128-row tiles (128-byte swizzle,
-// chunks of 64 K-elements kChunkBytes apart) over `ksteps` slices of K = 16.
-__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
-                                           int ksteps, uint32_t idesc, bool accumulate) {
-  for (int kk = 0; kk < ksteps; ++kk) {
+// chunks of 64 K-elements kChunkBytes apart) over KSTEPS slices of K = 16.
+// adesc/bdesc: sdesc_sw128(base, 16, 1024) of the two tiles.
+template <int KSTEPS>
+__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < KSTEPS; ++kk) {
     const uint32_t off = static_cast<uint32_t>(kk >> 2) * kChunkBytes + static_cast<uint32_t>(kk & 3) * 32u;
-    umma_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
-            idesc, (accumulate || kk > 0) ? 1u : 0u);
+    umma_ss(d_tmem, sdesc_add(adesc, off), sdesc_add(bdesc, off), idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
 // Issues D[tmem] (+)= A * B where A is a K-major 128-row tile and B an
 // MN-major tile (K rows of 128 bytes, N in chunks of 64 elements kChunkBytes
-// apart), K = 16 * ksteps.
-__device__ __forceinline__ void mma_a_k_b_mn(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
-                                             int ksteps, uint32_t idesc, bool accumulate) {
-  for (int kk = 0; kk < ksteps; ++kk) {
+// apart), K = 16 * KSTEPS.  adesc: sdesc_sw128(a, 16, 1024); bdesc:
+// sdesc_sw128(b, kChunkBytes, 1024).
+template <int KSTEPS>
+__device__ __forceinline__ void mma_a_k_b_mn(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < KSTEPS; ++kk) {
     const uint32_t aoff = static_cast<uint32_t>(kk >> 2) * kChunkBytes + static_cast<uint32_t>(kk & 3) * 32u;
-    const uint32_t boff = static_cast<uint32_t>(kk) * 2048u;
-    umma_ss(d_tmem, sdesc_sw128(a_base + aoff, 16, 1024),
-            sdesc_sw128(b_base + boff, kChunkBytes, 1024), idesc,
+    umma_ss(d_tmem, sdesc_add(adesc, aoff), sdesc_add(bdesc, static_cast<uint32_t>(kk) * 2048u), idesc,
             (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
 // Issues D[tmem] (+)= A * B where both are MN-major tiles (K rows of 128
-// bytes; M and N in chunks of 64 elements kChunkBytes apart).
-__device__ __forceinline__ void mma_mn_mn(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
-                                          int ksteps, uint32_t idesc, bool accumulate) {
-  for (int kk = 0; kk < ksteps; ++kk) {
+// bytes; M and N in chunks of 64 elements kChunkBytes apart).  Descriptors:
+// sdesc_sw128(base, kChunkBytes, 1024).
+template <int KSTEPS>
+__device__ __forceinline__ void mma_mn_mn(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < KSTEPS; ++kk) {
     const uint32_t off = static_cast<uint32_t>(kk) * 2048u;
-    umma_ss(d_tmem, sdesc_sw128(a_base + off, kChunkBytes, 1024),
-            sdesc_sw128(b_base + off, kChunkBytes, 1024), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
+    umma_ss(d_tmem, sdesc_add(adesc, off), sdesc_add(bdesc, off), idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 

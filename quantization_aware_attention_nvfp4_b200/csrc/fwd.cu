@@ -1,16 +1,19 @@
 // fwd.cu -- Attn-QAT forward kernel for sm_100a.
 //
 // One CTA per (128-query tile, batch*head).  320 threads in three roles:
-//   warp 0      TMA producer: the fq(Q) tile once, then fq(K) tiles for the
-//               row-max sweep and fq(K), fq(V) tiles for the output sweep
-//               (2-stage rings, 128-byte swizzle);
+//   warp 0      TMA producer: the Q tile once, then K tiles for the row-max
+//               sweep and K, fq(V) tiles for the output sweep.  With Q and K
+//               quantized these are the packed NVFP4 codes plus their scale
+//               tiles (8-stage K ring) and S is a block-scaled NVFP4 MMA;
+//               otherwise bf16 tiles; fq(V) in a 2-stage ring, 128-byte swizzle;
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer;
 //   warps 2..9  row warps, two per TMEM lane quarter: each query row (TMEM
 //               lane) has two threads owning 64 columns each -- row max, exp,
 //               row sum, in-register NVFP4 fq of P~ in 16-key blocks, the P
 //               tile to shared memory, and the O epilogue; the pair merges its
 //               partial max and sum through shared memory.
-// TMEM columns: S double buffer [0,256), O accumulator [256, 256+D).
+// TMEM columns: S buffers [0,256) (plus [256,384) during the row-max sweep,
+// before O exists), O accumulator [256, 256+D), scale factors from 384.
 //
 // The row max is exact over all keys, taken in a first sweep of S = Q K^T,
 // so fq(P~) sees the reference-order statistics and O needs no rescaling
@@ -30,7 +33,9 @@ namespace attnqat {
 // then a block-scaled kind::mxf4nvf4 MMA.  Otherwise Q and K are 16-bit tiles.
 template <int D, int FP4S>
 struct FwdLayout {
-  static constexpr int kNSK = FP4S ? 4 : 2;             // K ring stages
+  // K ring stages: the row-max sweep consumes a K tile every few hundred ns,
+  // so the 9 KB NVFP4 stages are kept deep enough to cover the TMA latency
+  static constexpr int kNSK = FP4S ? 8 : 2;
   static constexpr int kNSV = 2;                        // V ring stages
   static constexpr int kQKRow = FP4S ? D / 2 : 2 * D;   // bytes per Q/K row
   static constexpr int kQK = 128 * kQKRow;              // bytes per Q/K tile
@@ -44,26 +49,37 @@ struct FwdLayout {
   static constexpr int kQSF = kP + 2 * kPBytes;
   static constexpr int kKSF = kQSF + kSF;
   static constexpr int kBar = kKSF + kNSK * kSF;
-  static constexpr int kBytes = kBar + 2048;
+  static constexpr int kBarBytes = 2048;  // FwdBars (checked at the launch)
+  static constexpr int kBytes = kBar + kBarBytes;
   static constexpr int kDynSmem = kBytes + 1024;        // slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256;
   static constexpr uint32_t kSFCols = (D / 64) * 4;     // TMEM columns of one tile's scales
-  static constexpr uint32_t kTmemSFA = 256 + D;
+  // sweep 1 (row max) rotates S through three buffers: columns 0, 128 and
+  // 256 (the O accumulator's columns, unused until sweep 2's first P V);
+  // sweep 2 uses the first two.  Scale factors sit above all of them.
+  static constexpr int kNS1 = 3;
+  static constexpr uint32_t kTmemSFA = 384;
   static constexpr uint32_t kTmemSFB = kTmemSFA + kSFCols;  // kNSK stages
   // UMMA layout of the packed tiles: 64-byte rows swizzle 64B, 32-byte rows 32B
   static constexpr uint32_t kCodeLayout = (D / 2 == 64) ? 4u : 6u;
   static constexpr uint32_t kCodeSBO = 8 * (D / 2);
 };
 
+// Row warps per TMEM lane quarter in the forward: 2, each owning 64 of the
+// 128 columns.  (4 per quarter, 32 columns each, measured no faster: the
+// forward is not limited by how many row warps hide latency.)
+constexpr int kFwdG = 2;
+
 struct FwdBars {
   uint64_t qfull;
-  uint64_t kfull[4], kempty[4], vfull[2], vempty[2];
+  uint64_t kfull[8], kempty[8], vfull[2], vempty[2];
+  uint64_t sfull1[3], sempty1[3];   // sweep-1 S buffers
   uint64_t sfull[2], sempty[2], pfull[2], pempty[2];
   uint64_t ofull;
   uint32_t tmem_slot;
   int abort;
-  float part[4][kBM];   // per-row partial max / sum of the column groups
+  float part[kFwdG][kBM];   // per-row partial max / sum of the column groups
 };
 
 // Row max over this thread's NC columns (col0..col0+NC-1) of one S tile.
@@ -161,6 +177,7 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using L = FwdLayout<D, FP4S>;
+  static_assert(G <= kFwdG, "column groups beyond the partial-sum block");
   constexpr int kNSK = L::kNSK, kNSV = L::kNSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
@@ -183,6 +200,10 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     for (int s = 0; s < kNSV; ++s) {
       mbar_init(&bars->vfull[s], 1);
       mbar_init(&bars->vempty[s], 1);
+    }
+    for (int b = 0; b < 3; ++b) {
+      mbar_init(&bars->sfull1[b], 1);
+      mbar_init(&bars->sempty1[b], 4 * G);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->sfull[b], 1);
@@ -265,28 +286,30 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         for (int kc = 0; kc < D / 64; ++kc)
           tmem_cp_32x128b_x4(tmem + L::kTmemSFA + kc * 4, sdesc_make(sbase + L::kQSF + kc * 512, 16, 128, 0));
       }
-      int nS = 0;  // S tiles issued so far (both sweeps)
-      auto issue_s = [&](int t) -> bool {
+      // operand descriptors of the tiles' base addresses
+      const uint64_t dQ = FP4S ? sdesc_make(qaddr, 16, L::kCodeSBO, L::kCodeLayout) : desc_k(qaddr);
+      const uint64_t dK = FP4S ? sdesc_make(sbase + L::kK, 16, L::kCodeSBO, L::kCodeLayout) : desc_k(sbase + L::kK);
+      const uint64_t dKSF = sdesc_make(sbase + L::kKSF, 16, 128, 0);
+      const uint64_t dP = desc_k(sbase + L::kP), dV = desc_mn(sbase + L::kV);
+      // S tile t (K tile t mod nk) into TMEM column dcol, signalling `full`
+      auto issue_s = [&](int t, uint32_t dcol, uint64_t *full) -> bool {
         const int st = t % kNSK;
-        const int sb = nS & 1;
-        if (nS >= 2 && !mbar_wait(&bars->sempty[sb], ((nS >> 1) - 1) & 1, abort)) return false;
         if (!mbar_wait(&bars->kfull[st], (t / kNSK) & 1, abort)) return false;
         tc_fence_after();
-        const uint32_t kaddr = sbase + L::kK + st * L::kQK;
+        const uint64_t dKs = sdesc_add(dK, st * L::kQK);
         if (FP4S) {
           const uint32_t sfb = tmem + L::kTmemSFB + st * L::kSFCols;
-          for (int kc = 0; kc < D / 64; ++kc)
-            tmem_cp_32x128b_x4(sfb + kc * 4, sdesc_make(sbase + L::kKSF + st * L::kSF + kc * 512, 16, 128, 0));
+#pragma unroll
+          for (int kc = 0; kc < D / 64; ++kc) tmem_cp_32x128b_x4(sfb + kc * 4, sdesc_add(dKSF, st * L::kSF + kc * 512));
+#pragma unroll
           for (int kk = 0; kk < D / 64; ++kk)
-            umma_fp4(tmem + sb * kBN, sdesc_make(qaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout),
-                     sdesc_make(kaddr + kk * 32, 16, L::kCodeSBO, L::kCodeLayout), idS,
-                     tmem + L::kTmemSFA + kk * 4, sfb + kk * 4, kk > 0 ? 1u : 0u);
+            umma_fp4(tmem + dcol, sdesc_add(dQ, kk * 32), sdesc_add(dKs, kk * 32), idS, tmem + L::kTmemSFA + kk * 4,
+                     sfb + kk * 4, kk > 0 ? 1u : 0u);
         } else {
-          mma_kmajor(tmem + sb * kBN, qaddr, kaddr, D / 16, idS, false);
+          mma_kmajor<D / 16>(tmem + dcol, dQ, dKs, idS, false);
         }
         umma_commit(&bars->kempty[st]);
-        umma_commit(&bars->sfull[sb]);
-        ++nS;
+        umma_commit(full);
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
@@ -295,15 +318,26 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, abort)) return false;
         if (!mbar_wait(&bars->vfull[vs], (j / kNSV) & 1, abort)) return false;
         tc_fence_after();
-        mma_a_k_b_mn(tmem + L::kTmemO, sbase + L::kP + pb * L::kPBytes,
-                     sbase + L::kV + vs * L::kVT, kBN / 16, idPV, j > 0);
+        mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemO, sdesc_add(dP, pb * L::kPBytes), sdesc_add(dV, vs * L::kVT), idPV,
+                               j > 0);
         umma_commit(&bars->vempty[vs]);
         umma_commit(&bars->pempty[pb]);
         return true;
       };
-      for (int j = 0; ok && j < nk; ++j) ok = issue_s(j);
+      // sweep 1: three S buffers
+      for (int t = 0; ok && t < nk; ++t) {
+        const int b = t % L::kNS1;
+        if (t >= L::kNS1 && !mbar_wait(&bars->sempty1[b], ((t / L::kNS1) - 1) & 1, abort)) { ok = false; break; }
+        ok = issue_s(t, b * kBN, &bars->sfull1[b]);
+      }
+      // every sweep-1 buffer read before sweep 2 reuses columns 0..255
+      for (int t = (nk > L::kNS1 ? nk - L::kNS1 : 0); ok && t < nk; ++t)
+        ok = mbar_wait(&bars->sempty1[t % L::kNS1], (t / L::kNS1) & 1, abort);
+      // sweep 2: two S buffers, P V one tile behind
       for (int j = 0; ok && j < nk; ++j) {
-        ok = issue_s(nk + j);
+        const int sb = j & 1;
+        if (j >= 2 && !mbar_wait(&bars->sempty[sb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
+        ok = issue_s(nk + j, sb * kBN, &bars->sfull[sb]);
         if (ok && j >= 1) ok = issue_pv(j - 1);
       }
       if (ok) ok = issue_pv(nk - 1);
@@ -319,18 +353,17 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     const int last_valid = a.Lk - (nk - 1) * kBN;  // keys in the last KV tile
     float mrow = -INFINITY;
     bool ok = true;
-    int nS = 0;
-    for (int j = 0; j < nk; ++j, ++nS) {
-      const int sb = nS & 1;
-      if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
+    for (int j = 0; j < nk; ++j) {
+      const int b = j % L::kNS1;
+      if (!mbar_wait(&bars->sfull1[b], (j / L::kNS1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
+      const uint32_t taddr = tmem + rr.lane_addr + b * kBN;
       const float mx = (j == nk - 1 && last_valid < kBN) ? row_max_cols<true, NC>(taddr, col0, last_valid)
                                                          : row_max_cols<false, NC>(taddr, col0, kBN);
       mrow = fmaxf(mrow, mx);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sempty[sb]);
+      if (lane == 0) mbar_arrive(&bars->sempty1[b]);
     }
     // every column group of a row sees every tile, so all reach this merge
     bars->part[rr.half][rr.row] = mrow;
@@ -342,10 +375,10 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     const float nml = -(m_scaled * kLog2e);
     const float cl = a.scale_log2;
     float lsum = 0.0f;
-    for (int j = 0; ok && j < nk; ++j, ++nS) {
-      const int sb = nS & 1;
+    for (int j = 0; ok && j < nk; ++j) {
+      const int sb = j & 1;
       const int pb = j & 1;
-      if (!mbar_wait(&bars->sfull[sb], (nS >> 1) & 1, abort)) { ok = false; break; }
+      if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, abort)) { ok = false; break; }
       if (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
@@ -418,16 +451,12 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
   }
 }
 
-// Row warps per TMEM lane quarter in the forward: 2, each owning 64 of the
-// 128 columns.  (4 per quarter, 32 columns each, measured no faster: the
-// forward is not limited by how many row warps hide latency.)
-constexpr int kFwdG = 2;
-
 template <int D, int FP4S, int PV_F16, int QP>
 static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const FwdArgs &a, int BH, cudaStream_t stream) {
   using L = FwdLayout<D, FP4S>;
   static_assert(L::kDynSmem <= 232448, "forward shared memory over the 227 KB limit");
+  static_assert(sizeof(FwdBars) <= L::kBarBytes, "forward barrier block larger than its reservation");
   static_assert(!FP4S || L::kTmemSFB + L::kNSK * L::kSFCols <= L::kTmemCols, "forward TMEM over 512 columns");
   auto kern = attn_fwd_kernel<D, FP4S, PV_F16, QP, kFwdG>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
