@@ -2,12 +2,12 @@
 // estimator: every fq is the identity for the gradient).
 //
 //   dK/dV kernel: one CTA per (128-key tile, batch*head), looping over query
-//     tiles.  Per query tile: S = fq(Q) fq(K)^T and dP = dO fq(V)^T into TMEM;
-//     one thread per query row rebuilds P~ = exp(S - m) and fq(P~) exactly as
-//     the forward does (same bits, same blocks of 16 keys), forms
-//     (fq(P~)/l)^T and dS^T = (P o (dP - Delta))^T in shared memory, and the
-//     tensor cores accumulate dV += (fq(P~)/l)^T dO and dK += dS^T fq(Q) in
-//     TMEM.
+//     tiles.  Per query tile: S = fq(Q) fq(K)^T, then dP = dO fq(V)^T, into
+//     one TMEM buffer; the row warps (a query row per TMEM lane) rebuild
+//     P~ = exp(S - m) and fq(P~) exactly as the forward does (same blocks of
+//     16 keys), form (fq(P~)/l)^T and dS^T = (P o (dP - Delta))^T in shared
+//     memory, and the tensor cores accumulate dV += (fq(P~)/l)^T dO and
+//     dK += dS^T fq(Q) in TMEM.
 //   dQ kernel: one CTA per (128-query tile, batch*head), looping over key
 //     tiles: S, dP as above, dS = P o (dP - Delta) with P = exp(S - LSE),
 //     dQ += dS fq(K).
@@ -15,9 +15,13 @@
 // The split into a dK/dV and a dQ kernel follows the fastvideo-kernel
 // triton_kernels commit (SM100 Attn-QAT route: separate dQ and dK/dV tiles);
 // the tiles here are 128 x 128 tcgen05 tiles with TMEM accumulators.
-// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 2..9
-// row warps: two per TMEM lane quarter, so every query row (TMEM lane) has
-// two threads, each owning 64 of the tile's 128 columns.
+// Roles (384 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer
+// (one thread); in the dQ kernel warp 10 is a second MMA-issuing thread, A
+// issuing S and dP and B the dQ products (one thread alone issues a
+// tcgen05.mma only every ~58 cycles, too slowly to keep the tensor pipe busy
+// there); warps 2..9 row warps: two per TMEM lane quarter, so every query row
+// (TMEM lane) has two threads, each owning 64 of the tile's 128 columns; the
+// remaining warps idle.
 #include "common.cuh"
 #include "internal.h"
 
@@ -66,17 +70,20 @@ struct BwdBars {
   uint64_t sfull, sempty;
   uint64_t xfull, xempty;
   uint64_t done;
+  uint64_t adone;   // issuer A's MMAs have completed (drained before TMEM is freed)
   uint32_t tmem_slot;
   int abort;
 };
 
-__device__ __forceinline__ void init_bwd_bars(BwdBars *b) {
+// a_users / b_users: MMA-issuing threads that commit to aempty / bempty (a
+// ring slot is free once every MMA reading it has completed).
+__device__ __forceinline__ void init_bwd_bars(BwdBars *b, int a_users, int b_users) {
   mbar_init(&b->kvfull, 1);
   for (int s = 0; s < 2; ++s) {
     mbar_init(&b->afull[s], 1);
-    mbar_init(&b->aempty[s], 1);
+    mbar_init(&b->aempty[s], a_users);
     mbar_init(&b->bfull[s], 1);
-    mbar_init(&b->bempty[s], 1);
+    mbar_init(&b->bempty[s], b_users);
     mbar_init(&b->cfull[s], 1);
     mbar_init(&b->cempty[s], 1);
   }
@@ -85,6 +92,7 @@ __device__ __forceinline__ void init_bwd_bars(BwdBars *b) {
   mbar_init(&b->xfull, kSoftWarps);
   mbar_init(&b->xempty, 1);
   mbar_init(&b->done, 1);
+  mbar_init(&b->adone, 1);
   b->abort = 0;
   fence_mbar_init();
 }
@@ -239,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = blockIdx.y;
   const int nq = a.nq_tiles;
 
-  if (threadIdx.x == 0) init_bwd_bars(bars);
+  if (threadIdx.x == 0) init_bwd_bars(bars, 1, 1);
   if (warp == 1) {
     tmem_alloc(&bars->tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -310,14 +318,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dQk = desc_k(sbase + L::kQ), dQmn = desc_mn(sbase + L::kQ);
       const uint64_t dDOk = desc_k(sbase + L::kDO), dDOmn = desc_mn(sbase + L::kDO);
       const uint64_t dVk = desc_k(sbase + L::kV), dX = desc_mn(sbase + L::kX);
+      // One issuing thread here (a second one measured slower: this kernel is
+      // bound by its row warps, whose scheduler the second poller shares).
+      // Order per query tile: dP_i (once the rows have read S_i), dV_i,
+      // S_{i+1} (once the rows have read dP_i), dK_i.
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
       if (ok && FP4S) {
         tc_fence_after();
         for (int kc = 0; kc < D / 64; ++kc)
           tmem_cp_32x128b_x4(tmem + L::kTmemSFB + kc * 4, sdesc_make(sbase + L::kKSF + kc * 512, 16, 128, 0));
       }
-      // S_i into the TMEM buffer (fill 2i); the buffer's previous fill (dP_{i-1})
-      // has been released by the caller's wait
+      // S_i into the TMEM buffer (fill 2i); the buffer's previous fill
+      // (dP_{i-1}) has been released by the caller's wait
       auto issue_s = [&](int i) -> bool {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
@@ -327,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sfa = tmem + L::kTmemSFA + st * L::kSFCols;
           const uint64_t dQs = sdesc_add(dQ4, st * L::kCode);
 #pragma unroll
-          for (int kc = 0; kc < D / 64; ++kc) tmem_cp_32x128b_x4(sfa + kc * 4, sdesc_add(dQSF, st * L::kSF + kc * 512));
+          for (int kc = 0; kc < D / 64; ++kc)
+            tmem_cp_32x128b_x4(sfa + kc * 4, sdesc_add(dQSF, st * L::kSF + kc * 512));
 #pragma unroll
           for (int kk = 0; kk < D / 64; ++kk)
             umma_fp4(tbuf, sdesc_add(dQs, kk * 32), sdesc_add(dK, kk * 32), idS, sfa + kk * 4,
@@ -346,26 +359,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
         // dP_i once the rows have read S_i (fill 2i)
-        if (!mbar_wait(&bars->sempty, (2 * i) & 1, abort) || !mbar_wait(&bars->bfull[st], ph, abort)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait(&bars->sempty, (2 * i) & 1, abort) || !mbar_wait(&bars->bfull[st], ph, abort)) break;
         tc_fence_after();
         mma_kmajor<D / 16>(tbuf, sdesc_add(dDOk, st * L::kTile), dVk, idDP, false);
         umma_commit(&bars->sfull);
         // dV += (fq(P~)/l)^T dO_i : A = X (M = keys, MN-major), B = dO (N = D, MN-major)
-        if (!mbar_wait(&bars->xfull, (2 * i) & 1, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars->xfull, (2 * i) & 1, abort)) break;
         tc_fence_after();
         mma_mn_mn<kBM / 16>(tmem + L::kTmemDV, dX, sdesc_add(dDOmn, st * L::kTile), idV, i > 0);
         umma_commit(&bars->xempty);
         umma_commit(&bars->bempty[st]);
         // S_{i+1} once the rows have read dP_i (fill 2i+1)
-        if (i + 1 < nq) {
-          if (!mbar_wait(&bars->sempty, (2 * i + 1) & 1, abort) || !issue_s(i + 1)) { ok = false; break; }
-        }
+        if (i + 1 < nq && !(mbar_wait(&bars->sempty, (2 * i + 1) & 1, abort) && issue_s(i + 1))) break;
         // dK += dS^T Q_i
-        if (!mbar_wait(&bars->xfull, (2 * i + 1) & 1, abort)) { ok = false; break; }
-        if (FP4S && !mbar_wait(&bars->afull[st], ph, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars->xfull, (2 * i + 1) & 1, abort)) break;
+        if (FP4S && !mbar_wait(&bars->afull[st], ph, abort)) break;
         tc_fence_after();
         mma_mn_mn<kBM / 16>(tmem + L::kTmemDK, dX, sdesc_add(dQmn, st * L::kTile), idK, i > 0);
         umma_commit(&bars->xempty);
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma_commit(&bars->done);
     }
-  } else {
+  } else if (warp >= 2 && warp < 2 + kSoftWarps) {
     const RowRole rr(warp, lane);
     const int col0 = rr.half * 64;
     const int valid_k = a.Lk - kt * kBN;  // >= 128 for full key tiles
@@ -588,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = blockIdx.y;
   const int nk = a.nk_tiles;
 
-  if (threadIdx.x == 0) init_bwd_bars(bars);
+  if (threadIdx.x == 0) init_bwd_bars(bars, 1, 1);
   if (warp == 1) {
     tmem_alloc(&bars->tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -642,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = (nkh > 2 ? nkh - 2 : 0); j < nkh; ++j) mbar_wait_drain(&bars->afull[j & 1], (j >> 1) & 1);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == kMmaB2) {
     if (lane == 0) {
       constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);  // Q K^T
       constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
@@ -654,57 +662,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dK4 = sdesc_make(sbase + L::kK4, 16, L::kCodeSBO, L::kCodeLayout);
       const uint64_t dKSF = sdesc_make(sbase + L::kKSF, 16, 128, 0);
       const uint64_t dKk = desc_k(sbase + L::kK), dKmn = desc_mn(sbase + L::kK), dX = desc_k(sbase + L::kX);
-      bool ok = mbar_wait(&bars->kvfull, 0, abort);
-      if (ok && FP4S) {
-        tc_fence_after();
-        for (int kc = 0; kc < D / 64; ++kc)
-          tmem_cp_32x128b_x4(tmem + L::kTmemSFA + kc * 4, sdesc_make(sbase + L::kQSF + kc * 512, 16, 128, 0));
-      }
-      // dP_j, then S_j; one commit signals both
-      auto issue_sdp = [&](int j) -> bool {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&bars->bfull[st], ph, abort)) return false;
-        tc_fence_after();
-        mma_kmajor<D / 16>(tmem + L::kTmemDP, dDO, sdesc_add(dVk, st * L::kTile), idDP, false);
-        umma_commit(&bars->bempty[st]);
-        if (FP4S) {
-          if (!mbar_wait(&bars->cfull[st], ph, abort)) return false;
+      if (warp == 1) {
+        // issuer A: dP_j, then S_j; one commit signals both
+        bool ok = mbar_wait(&bars->kvfull, 0, abort);
+        if (ok && FP4S) {
           tc_fence_after();
-          const uint32_t sfb = tmem + L::kTmemSFB + st * L::kSFCols;
-          const uint64_t dKs = sdesc_add(dK4, st * L::kCode);
-#pragma unroll
-          for (int kc = 0; kc < D / 64; ++kc) tmem_cp_32x128b_x4(sfb + kc * 4, sdesc_add(dKSF, st * L::kSF + kc * 512));
-#pragma unroll
-          for (int kk = 0; kk < D / 64; ++kk)
-            umma_fp4(tmem + L::kTmemS, sdesc_add(dQ, kk * 32), sdesc_add(dKs, kk * 32), idS,
-                     tmem + L::kTmemSFA + kk * 4, sfb + kk * 4, kk > 0 ? 1u : 0u);
-          umma_commit(&bars->cempty[st]);
-        } else {
-          if (!mbar_wait(&bars->afull[st], ph, abort)) return false;
+          for (int kc = 0; kc < D / 64; ++kc)
+            tmem_cp_32x128b_x4(tmem + L::kTmemSFA + kc * 4, sdesc_make(sbase + L::kQSF + kc * 512, 16, 128, 0));
+        }
+        auto issue_sdp = [&](int j) -> bool {
+          const int st = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          if (!mbar_wait(&bars->bfull[st], ph, abort)) return false;
           tc_fence_after();
-          mma_kmajor<D / 16>(tmem + L::kTmemS, dQ, sdesc_add(dKk, st * L::kTile), idS, false);
+          mma_kmajor<D / 16>(tmem + L::kTmemDP, dDO, sdesc_add(dVk, st * L::kTile), idDP, false);
+          umma_commit(&bars->bempty[st]);
+          if (FP4S) {
+            if (!mbar_wait(&bars->cfull[st], ph, abort)) return false;
+            tc_fence_after();
+            const uint32_t sfb = tmem + L::kTmemSFB + st * L::kSFCols;
+            const uint64_t dKs = sdesc_add(dK4, st * L::kCode);
+#pragma unroll
+            for (int kc = 0; kc < D / 64; ++kc)
+              tmem_cp_32x128b_x4(sfb + kc * 4, sdesc_add(dKSF, st * L::kSF + kc * 512));
+#pragma unroll
+            for (int kk = 0; kk < D / 64; ++kk)
+              umma_fp4(tmem + L::kTmemS, sdesc_add(dQ, kk * 32), sdesc_add(dKs, kk * 32), idS,
+                       tmem + L::kTmemSFA + kk * 4, sfb + kk * 4, kk > 0 ? 1u : 0u);
+            umma_commit(&bars->cempty[st]);
+          } else {
+            if (!mbar_wait(&bars->afull[st], ph, abort)) return false;
+            tc_fence_after();
+            mma_kmajor<D / 16>(tmem + L::kTmemS, dQ, sdesc_add(dKk, st * L::kTile), idS, false);
+          }
+          umma_commit(&bars->sfull);
+          return true;
+        };
+        if (ok) ok = issue_sdp(0);
+        for (int j = 1; ok && j < nk; ++j) ok = mbar_wait(&bars->sempty, (j - 1) & 1, abort) && issue_sdp(j);
+        // TMEM is freed by this warp: let its own MMAs finish first
+        umma_commit(&bars->adone);
+        mbar_wait_drain(&bars->adone, 0);
+      } else {
+        // issuer B: dQ += dS_j K_j.  K_j goes back to the producer after dQ_j
+        // (without FP4S, S_j read it too; the rows have read S_j by then).
+        for (int j = 0; j < nk; ++j) {
+          const int st = j & 1;
+          if (!mbar_wait(&bars->xfull, j & 1, abort) || !mbar_wait(&bars->afull[st], (j >> 1) & 1, abort)) break;
+          tc_fence_after();
+          mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemDQ, dX, sdesc_add(dKmn, st * L::kTile), idQ, j > 0);
+          umma_commit(&bars->xempty);
+          umma_commit(&bars->aempty[st]);
         }
-        umma_commit(&bars->sfull);
-        return true;
-      };
-      if (ok) ok = issue_sdp(0);
-      for (int j = 0; ok && j < nk; ++j) {
-        const int st = j & 1;
-        if (j + 1 < nk) {
-          ok = mbar_wait(&bars->sempty, j & 1, abort) && issue_sdp(j + 1);
-          if (!ok) break;
-        }
-        if (!mbar_wait(&bars->xfull, j & 1, abort)) { ok = false; break; }
-        if (FP4S && !mbar_wait(&bars->afull[st], (j >> 1) & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemDQ, dX, sdesc_add(dKmn, st * L::kTile), idQ, j > 0);
-        umma_commit(&bars->xempty);
-        umma_commit(&bars->aempty[st]);
+        umma_commit(&bars->done);
       }
-      umma_commit(&bars->done);
     }
-  } else {
+  } else if (warp >= 2 && warp < 2 + kSoftWarps) {
     const RowRole rr(warp, lane);
     const int col0 = rr.half * 64;
     const int q = qt * kBM + static_cast<int>(rr.row);

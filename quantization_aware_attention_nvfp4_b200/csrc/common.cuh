@@ -9,7 +9,13 @@ namespace attnqat {
 
 constexpr int kBM = 128;                  // query rows per tile (TMEM lanes)
 constexpr int kSoftWarps = 8;             // row warps: 2 per TMEM lane quarter, each owns 64 columns
-constexpr int kThreads = 64 + 32 * kSoftWarps;  // + producer warp + MMA warp
+// Warp roles: 0 TMA producer, 1 and kMmaB2 the two MMA-issuing threads (one
+// thread issues a tcgen05.mma about every 58 cycles, barely faster than the
+// tensor pipe retires a 128x128x16 f16 MMA, so its waits and commits would
+// idle the pipe; two issuers split the MMA streams), 2..9 row warps, 11 idle
+// (12 warps: the register budget per thread is that of 384 threads anyway).
+constexpr int kMmaB2 = 2 + kSoftWarps;
+constexpr int kThreads = 384;
 constexpr int kBN = 128;                  // keys per tile
 constexpr int kChunkBytes = 128 * 128;    // one 128-row x 128-byte swizzled chunk
 constexpr float kLog2e = 1.4426950408889634f;

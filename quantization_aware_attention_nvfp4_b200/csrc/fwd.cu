@@ -1,17 +1,21 @@
 // fwd.cu -- Attn-QAT forward kernel for sm_100a.
 //
-// One CTA per (128-query tile, batch*head).  320 threads in three roles:
+// One CTA per (128-query tile, batch*head).  384 threads in four roles:
 //   warp 0      TMA producer: the Q tile once, then K tiles for the row-max
 //               sweep and K, fq(V) tiles for the output sweep.  With Q and K
 //               quantized these are the packed NVFP4 codes plus their scale
 //               tiles (8-stage K ring) and S is a block-scaled NVFP4 MMA;
 //               otherwise bf16 tiles; fq(V) in a 2-stage ring, 128-byte swizzle;
-//   warp 1      TMEM owner and single-thread tcgen05.mma issuer;
+//   warps 1, 10 tcgen05.mma issuers (one thread each; warp 1 owns TMEM): A
+//               issues even row-max tiles and the output sweep's S, B the odd
+//               row-max tiles and P V (one thread alone cannot issue fast
+//               enough to keep the tensor pipe busy);
 //   warps 2..9  row warps, two per TMEM lane quarter: each query row (TMEM
 //               lane) has two threads owning 64 columns each -- row max, exp,
 //               row sum, in-register NVFP4 fq of P~ in 16-key blocks, the P
 //               tile to shared memory, and the O epilogue; the pair merges its
 //               partial max and sum through shared memory.
+//   warp 11     idle (pads the CTA to whole groups of four warps).
 // TMEM columns: S buffers [0,256) (plus [256,384) during the row-max sweep,
 // before O exists), O accumulator [256, 256+D), scale factors from 384.
 //
@@ -77,6 +81,8 @@ struct FwdBars {
   uint64_t sfull1[3], sempty1[3];   // sweep-1 S buffers
   uint64_t sfull[2], sempty[2], pfull[2], pempty[2];
   uint64_t ofull;
+  uint64_t sfa_ready;   // issuer A's copy of the Q scales into TMEM has landed
+  uint64_t adone;       // issuer A's MMAs have completed (drained before TMEM is freed)
   uint32_t tmem_slot;
   int abort;
   float part[kFwdG][kBM];   // per-row partial max / sum of the column groups
@@ -168,9 +174,11 @@ __device__ __forceinline__ void group_sync(int wq) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + wq), "n"(32 * G) : "memory");
 }
 
-// Threads of a forward CTA with G row warps per TMEM lane quarter.
+// Threads of a forward CTA with G row warps per TMEM lane quarter: producer,
+// MMA issuer A, 4G row warps, MMA issuer B (warp 2 + 4G), padded to whole
+// groups of four warps.
 template <int G>
-constexpr int fwd_threads() { return 64 + 128 * G; }
+constexpr int fwd_threads() { return (2 + 4 * G + 1 + 3) / 4 * 128; }
 
 template <int D, int FP4S, int PV_F16, int QP, int G>
 __global__ void __launch_bounds__(fwd_threads<G>(), 1)
@@ -212,6 +220,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       mbar_init(&bars->pempty[b], 1);
     }
     mbar_init(&bars->ofull, 1);
+    mbar_init(&bars->sfa_ready, 1);
+    mbar_init(&bars->adone, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -273,18 +283,29 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
           mbar_wait_drain(&bars->vfull[u % kNSV], (u / kNSV) & 1);
       }
     }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------------- MMA --
+  } else if (warp == 1 || warp == 2 + 4 * G) {
+    // ---------------------------------------------------------------- MMA --
+    // Two issuing threads (one thread issues a tcgen05 instruction only every
+    // ~50-60 cycles): A issues the even tiles of the row-max sweep and every
+    // S of the output sweep, B the odd row-max tiles and every P V.
     if (lane == 0) {
+      const bool issuer_a = warp == 1;
       constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);
       constexpr uint32_t idPV = idesc_f16(kBM, D, !PV_F16, false, true);
       const uint32_t qaddr = sbase + L::kQ;
       bool ok = mbar_wait(&bars->qfull, 0, abort);
-      if (ok && FP4S) {
-        // scales of the Q tile into TMEM once (tcgen05 ops of this thread run in order)
-        tc_fence_after();
-        for (int kc = 0; kc < D / 64; ++kc)
-          tmem_cp_32x128b_x4(tmem + L::kTmemSFA + kc * 4, sdesc_make(sbase + L::kQSF + kc * 512, 16, 128, 0));
+      if (FP4S) {
+        if (issuer_a) {
+          // scales of the Q tile into TMEM once; B waits for them to land
+          if (ok) {
+            tc_fence_after();
+            for (int kc = 0; kc < D / 64; ++kc)
+              tmem_cp_32x128b_x4(tmem + L::kTmemSFA + kc * 4, sdesc_make(sbase + L::kQSF + kc * 512, 16, 128, 0));
+          }
+          umma_commit(&bars->sfa_ready);
+        } else {
+          ok = ok && mbar_wait(&bars->sfa_ready, 0, abort);
+        }
       }
       // operand descriptors of the tiles' base addresses
       const uint64_t dQ = FP4S ? sdesc_make(qaddr, 16, L::kCodeSBO, L::kCodeLayout) : desc_k(qaddr);
@@ -312,40 +333,48 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         umma_commit(full);
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
-        const int pb = j & 1;
-        const int vs = j % kNSV;
-        if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, abort)) return false;
-        if (!mbar_wait(&bars->vfull[vs], (j / kNSV) & 1, abort)) return false;
-        tc_fence_after();
-        mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemO, sdesc_add(dP, pb * L::kPBytes), sdesc_add(dV, vs * L::kVT), idPV,
-                               j > 0);
-        umma_commit(&bars->vempty[vs]);
-        umma_commit(&bars->pempty[pb]);
-        return true;
-      };
-      // sweep 1: three S buffers
-      for (int t = 0; ok && t < nk; ++t) {
+      // row-max sweep: three S buffers, tiles alternating between A and B
+      for (int t = issuer_a ? 0 : 1; ok && t < nk; t += 2) {
         const int b = t % L::kNS1;
         if (t >= L::kNS1 && !mbar_wait(&bars->sempty1[b], ((t / L::kNS1) - 1) & 1, abort)) { ok = false; break; }
         ok = issue_s(t, b * kBN, &bars->sfull1[b]);
       }
-      // every sweep-1 buffer read before sweep 2 reuses columns 0..255
-      for (int t = (nk > L::kNS1 ? nk - L::kNS1 : 0); ok && t < nk; ++t)
-        ok = mbar_wait(&bars->sempty1[t % L::kNS1], (t / L::kNS1) & 1, abort);
-      // sweep 2: two S buffers, P V one tile behind
-      for (int j = 0; ok && j < nk; ++j) {
-        const int sb = j & 1;
-        if (j >= 2 && !mbar_wait(&bars->sempty[sb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
-        ok = issue_s(nk + j, sb * kBN, &bars->sfull[sb]);
-        if (ok && j >= 1) ok = issue_pv(j - 1);
+      if (issuer_a) {
+        // every row-max buffer read before the output sweep reuses columns 0..255
+        for (int t = (nk > L::kNS1 ? nk - L::kNS1 : 0); ok && t < nk; ++t)
+          ok = mbar_wait(&bars->sempty1[t % L::kNS1], (t / L::kNS1) & 1, abort);
+        // output sweep: S into two buffers
+        for (int j = 0; ok && j < nk; ++j) {
+          const int sb = j & 1;
+          if (j >= 2 && !mbar_wait(&bars->sempty[sb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
+          ok = issue_s(nk + j, sb * kBN, &bars->sfull[sb]);
+        }
+        // TMEM is freed by this warp: let its own MMAs finish first
+        umma_commit(&bars->adone);
+        mbar_wait_drain(&bars->adone, 0);
+      } else {
+        // output sweep: O += fq(P~)_j fq(V)_j as the rows hand over each P tile
+        // (the first P V runs after every row-max tile was read, so it may
+        // overwrite the third S buffer's columns)
+        for (int j = 0; ok && j < nk; ++j) {
+          const int pb = j & 1;
+          const int vs = j % kNSV;
+          if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, abort) || !mbar_wait(&bars->vfull[vs], (j / kNSV) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemO, sdesc_add(dP, pb * L::kPBytes), sdesc_add(dV, vs * L::kVT), idPV,
+                                 j > 0);
+          umma_commit(&bars->vempty[vs]);
+          umma_commit(&bars->pempty[pb]);
+        }
+        // ofull tracks completion of every P V, so the epilogue and the TMEM
+        // release never race one in flight (the rows have read every S)
+        umma_commit(&bars->ofull);
       }
-      if (ok) ok = issue_pv(nk - 1);
-      // ofull also tracks completion of everything issued above, so the
-      // epilogue and the TMEM release never race an MMA in flight
-      umma_commit(&bars->ofull);
     }
-  } else {
+  } else if (warp >= 2 && warp < 2 + 4 * G) {
     // ---------------------------------------------------------- row warps --
     constexpr int NC = kBN / G;  // columns per thread
     const RowRole rr(warp, lane);
