@@ -155,11 +155,28 @@ static bool encode_codes(CUtensorMap *map, const void *base, int BH, int L, int 
   return r == CUDA_SUCCESS;
 }
 
+// 3-D map over fq(V)'s packed codes [BH][D][Lk/2 bytes] (blocks of 16 tokens
+// per channel): 128 tokens (64 bytes) x D channels per box, 64-byte swizzle,
+// the K-major B operand of the NVFP4 P V product; tokens past Lk read as zeros.
+static bool encode_vcodes(CUtensorMap *map, const void *base, int BH, int Lk, int D) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(Lk) / 2;
+  cuuint64_t dims[3] = {row, static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {row, row * static_cast<cuuint64_t>(D)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(D), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------- workspace --
 
 struct Workspace {
-  size_t qh, kh, vh, vh16, o32, delta, stats, do16, qc, qsf, kc, ksf, total;
-  size_t qsf_bytes, ksf_bytes;
+  size_t qh, kh, vh, vh16, o32, delta, stats, do16, qc, qsf, kc, ksf, vc, vsf, total;
+  size_t qsf_bytes, ksf_bytes, vsf_bytes;
 };
 
 // fq(Q) and fq(K) are exact in fp16 (values sign * E2M1 * E4M3 lie in
@@ -175,6 +192,13 @@ static bool qk_f16(uint32_t flags) {
 // bf16 has 8 significant bits) -- dP stays exact and the dV operand
 // fq(P~)/l gets 11 significant bits instead of bf16's 8.
 static bool do_f16(uint32_t flags) { return (flags & ATTNQAT_QUANT_ALL) == ATTNQAT_QUANT_ALL; }
+
+// With every quantizer on, fq(P~) fq(V) is also a product of NVFP4 blocks
+// along its K axis (keys for P~, tokens for V), so the forward's P V runs as
+// a block-scaled NVFP4 MMA (M = 128 queries, N = D = 128) on fq(V)'s packed
+// codes [B*H][D][Lk/2] -- whose rows the TMA reads need 16-byte aligned:
+// Lk % 32 == 0.  D = 64 keeps the fp16 P V.
+static bool pv_fp4(uint32_t flags, int Lk, int D) { return do_f16(flags) && (Lk % 32) == 0 && D == 128; }
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -213,6 +237,13 @@ static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
   if (fp4) off = align256(off + BH * Lk * D / 2);
   w.ksf = off;
   if (fp4) off = align256(off + w.ksf_bytes);
+  // fq(V)'s packed codes and its scales in 128-token tiles (1 KB per tile)
+  const bool pv4 = pv_fp4(flags, Lk, D);
+  w.vsf_bytes = BH * ntk * 1024;
+  w.vc = off;
+  if (pv4) off = align256(off + BH * Lk * D / 2);
+  w.vsf = off;
+  if (pv4) off = align256(off + w.vsf_bytes);
   w.total = off;
   return w;
 }
@@ -268,10 +299,16 @@ static int prepare_operands(const void *q, const void *k, const void *v, int B, 
   }
   if (flags & ATTNQAT_QUANT_V) {
     // blocks of 16 consecutive tokens per channel: the transposed view
+    const bool pv4 = pv_fp4(flags, Lk, D);
+    if (pv4 && (Lk % 128) != 0) {
+      e = cudaMemsetAsync(ws + w.vsf, 0, w.vsf_bytes, stream);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
     ProfScope ps("quantize_v", stream);
     e = launch_quantize(static_cast<const uint16_t *>(v), BH, D, Lk, static_cast<int64_t>(Lk) * D, 1, D,
-                        nullptr, nullptr, reinterpret_cast<uint16_t *>(ws + w.vh),
-                        reinterpret_cast<uint16_t *>(ws + w.vh16), stats + 2, stream);
+                        pv4 ? ws + w.vc : nullptr, pv4 ? ws + w.vsf : nullptr,
+                        reinterpret_cast<uint16_t *>(ws + w.vh), reinterpret_cast<uint16_t *>(ws + w.vh16),
+                        stats + 2, stream, 0, pv4);
   } else {
     ProfScope ps("absmax_v", stream);
     e = launch_absmax(static_cast<const __nv_bfloat16 *>(v), BH * Lk * D, stats + 2, stream);
@@ -383,12 +420,14 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
   const void *kh = (flags & ATTNQAT_QUANT_K) ? static_cast<const void *>(wsb + w.kh) : k;
   const bool pv_f16 = (flags & ATTNQAT_QUANT_V) != 0;
+  const bool pv4 = pv_fp4(flags, Lk, D);
   const void *vh = pv_f16 ? static_cast<const void *>(wsb + w.vh16) : v;
   const bool f16 = qk_f16(flags);
   CUtensorMap tq, tk, tv;
   const bool maps_ok = f16 ? encode_codes(&tq, wsb + w.qc, BH, Lq, D) && encode_codes(&tk, wsb + w.kc, BH, Lk, D)
                            : encode_bhld(&tq, qh, BH, Lq, D, false) && encode_bhld(&tk, kh, BH, Lk, D, false);
-  if (!maps_ok || !encode_bhld(&tv, vh, BH, Lk, D, pv_f16)) return cuda_fail(cudaErrorInvalidValue);
+  const bool vmap_ok = pv4 ? encode_vcodes(&tv, wsb + w.vc, BH, Lk, D) : encode_bhld(&tv, vh, BH, Lk, D, pv_f16);
+  if (!maps_ok || !vmap_ok) return cuda_fail(cudaErrorInvalidValue);
   FwdArgs a;
   a.Lq = Lq;
   a.Lk = Lk;
@@ -398,6 +437,7 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   a.scale_log2 = sm_scale * kLog2e;
   a.qsf = wsb + w.qsf;
   a.ksf = wsb + w.ksf;
+  a.vsf = wsb + w.vsf;
   a.o = static_cast<__nv_bfloat16 *>(o);
   a.o32 = reinterpret_cast<float *>(wsb + w.o32);
   a.lse = lse;
@@ -405,7 +445,7 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   cudaError_t e;
   {
     ProfScope ps("attn_fwd", s);
-    e = launch_fwd(D, f16, pv_f16, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, a, BH, s);
+    e = launch_fwd(D, f16, pv4 ? 2 : (pv_f16 ? 1 : 0), (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, a, BH, s);
   }
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }

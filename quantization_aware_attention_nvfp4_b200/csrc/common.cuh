@@ -53,6 +53,25 @@ __device__ __forceinline__ float fq16_probs(const float *p, uint32_t (&r)[8]) {
   return s;
 }
 
+// The same fq of 16 probabilities as fq16_probs, step for step (same amax,
+// same E4M3 scale, same p * rcp(s), same E2M1 rounding), returning the packed
+// E2M1 codes (c[0]: elements 0..7, c[1]: 8..15) and the E4M3 scale byte:
+// the operand of the block-scaled NVFP4 P V product.
+__device__ __forceinline__ uint32_t fq4_probs(const float *p, uint32_t (&c)[2]) {
+  const float amax = fmax3(fmax3(fmax3(p[0], p[1], p[2]), fmax3(p[3], p[4], p[5]), fmax3(p[6], p[7], p[8])),
+                          fmax3(p[9], p[10], p[11]), fmax3(p[12], p[13], fmaxf(p[14], p[15])));
+  const uint16_t code = cvt_e4m3x2(amax * (1.0f / 6.0f), 0.0f);
+  const float s = unpack_f16x2(cvt_f16x2_from_e4m3x2(code)).x;
+  const float inv = s > 0.0f ? rcp_approx(s) : 0.0f;
+  const float2 inv2 = make_float2(inv, inv);
+  float2 x[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = mul2(make_float2(p[2 * i], p[2 * i + 1]), inv2);
+  c[0] = e2m1x8(x[0], x[1], x[2], x[3]);
+  c[1] = e2m1x8(x[4], x[5], x[6], x[7]);
+  return code & 0xFFu;
+}
+
 // f16x2 word with the f16 value of s (an E4M3 value, exact in f16) in both
 // halves.
 __device__ __forceinline__ uint32_t f16x2_broadcast(float s) {

@@ -35,24 +35,32 @@ namespace attnqat {
 // are packed NVFP4 codes (D/2 bytes per row, TMA swizzle of D/2 bytes) and
 // their 16-element scales (512-byte scale-factor blocks per 64 columns); S is
 // then a block-scaled kind::mxf4nvf4 MMA.  Otherwise Q and K are 16-bit tiles.
-template <int D, int FP4S>
+// With PV4 the P V product is block-scaled NVFP4 too: fq(P~) blocks run along
+// keys and fq(V) blocks along tokens, both the K axis of P V, so the P tile
+// holds packed codes (64 bytes per query row, 64-byte swizzle) plus scale
+// blocks, and the V stages hold fq(V)'s codes ([D][128 keys / 2]) and scales.
+template <int D, int FP4S, int PV4>
 struct FwdLayout {
   // K ring stages: the row-max sweep consumes a K tile every few hundred ns,
   // so the 9 KB NVFP4 stages are kept deep enough to cover the TMA latency
   static constexpr int kNSK = FP4S ? 8 : 2;
-  static constexpr int kNSV = 2;                        // V ring stages
+  static constexpr int kNSV = PV4 ? 4 : 2;              // V ring stages
   static constexpr int kQKRow = FP4S ? D / 2 : 2 * D;   // bytes per Q/K row
   static constexpr int kQK = 128 * kQKRow;              // bytes per Q/K tile
   static constexpr int kSF = FP4S ? (D / 64) * 512 : 0;  // scale-factor bytes per tile
-  static constexpr int kVT = Tile<D>::kBytes;
-  static constexpr int kPBytes = kBM * kBN * 2;
+  static constexpr int kVT = PV4 ? D * 64 : Tile<D>::kBytes;
+  static constexpr int kVSF = PV4 ? 1024 : 0;           // 128 keys = two 64-key scale blocks
+  static constexpr int kPBytes = PV4 ? kBM * 64 : kBM * kBN * 2;
+  static constexpr int kPSF = PV4 ? 1024 : 0;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kQK;
   static constexpr int kV = (kK + kNSK * kQK + 1023) / 1024 * 1024;
   static constexpr int kP = kV + kNSV * kVT;
   static constexpr int kQSF = kP + 2 * kPBytes;
   static constexpr int kKSF = kQSF + kSF;
-  static constexpr int kBar = kKSF + kNSK * kSF;
+  static constexpr int kVSFo = kKSF + kNSK * kSF;
+  static constexpr int kPSFo = kVSFo + kNSV * kVSF;
+  static constexpr int kBar = kPSFo + 2 * kPSF;
   static constexpr int kBarBytes = 2048;  // FwdBars (checked at the launch)
   static constexpr int kBytes = kBar + kBarBytes;
   static constexpr int kDynSmem = kBytes + 1024;        // slack for 1024-byte alignment
@@ -64,7 +72,10 @@ struct FwdLayout {
   // sweep 2 uses the first two.  Scale factors sit above all of them.
   static constexpr int kNS1 = 3;
   static constexpr uint32_t kTmemSFA = 384;
-  static constexpr uint32_t kTmemSFB = kTmemSFA + kSFCols;  // kNSK stages
+  static constexpr uint32_t kTmemSFB = kTmemSFA + kSFCols;            // kNSK stages
+  static constexpr uint32_t kTmemSFP = kTmemSFB + kNSK * kSFCols;     // PV4: 2 P buffers x 8
+  static constexpr uint32_t kTmemSFV = kTmemSFP + (PV4 ? 16 : 0);     // PV4: kNSV stages x 8
+  static constexpr uint32_t kTmemEnd = kTmemSFV + (PV4 ? 8 * kNSV : 0);
   // UMMA layout of the packed tiles: 64-byte rows swizzle 64B, 32-byte rows 32B
   static constexpr uint32_t kCodeLayout = (D / 2 == 64) ? 4u : 6u;
   static constexpr uint32_t kCodeSBO = 8 * (D / 2);
@@ -77,7 +88,7 @@ constexpr int kFwdG = 2;
 
 struct FwdBars {
   uint64_t qfull;
-  uint64_t kfull[8], kempty[8], vfull[2], vempty[2];
+  uint64_t kfull[8], kempty[8], vfull[4], vempty[4];   // sized for the deepest rings
   uint64_t sfull1[3], sempty1[3];   // sweep-1 S buffers
   uint64_t sfull[2], sempty[2], pfull[2], pempty[2];
   uint64_t ofull;
@@ -112,9 +123,15 @@ __device__ __forceinline__ float row_max_cols(uint32_t taddr, int col0, int vali
 // nml), partial row sum, fq(P~) (or P~ itself) packed into 16-bit pairs and
 // stored as columns col0..col0+NC-1 of row `row` of the P tile at `pbase`
 // (128-byte swizzled chunks of 64 columns).
-template <int PV_F16, int QP, bool MASKED, int NC>
+// PVM selects the P tile's form: 0 bf16, 1 fp16 (16-bit, 128-byte swizzled
+// chunks), 2 packed NVFP4 codes (64-byte rows, 64-byte swizzle) with the
+// E4M3 scale bytes at `psf` in the layout tcgen05.cp moves into TMEM.
+template <int PVM, int QP, bool MASKED, int NC>
 __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, float cl, float nml,
-                                           uint32_t pbase, uint32_t row) {
+                                           uint32_t pbase, uint32_t psf, uint32_t row) {
+  static_assert(PVM != 2 || (QP && NC == 64), "NVFP4 P V needs quantized P and 64 columns per thread");
+  constexpr int PV_F16 = PVM == 1;
+  uint32_t sfw = 0;  // PVM 2: this thread's four scale bytes
   float2 lsum = make_float2(0.0f, 0.0f);
   const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
 #pragma unroll
@@ -131,38 +148,58 @@ __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, 
       p[2 * i + 1] = (!MASKED || col0 + c * 32 + 2 * i + 1 < valid) ? e1 : 0.0f;
       lsum = add2(lsum, make_float2(p[2 * i], p[2 * i + 1]));
     }
-    uint32_t w[16];
+    if (PVM == 2) {
+      // two 16-key blocks -> 16 bytes of codes (the 16-byte unit cc/32 of the
+      // row's 64 bytes, swizzled as TMA's 64-byte mode) and two scale bytes
+      uint32_t cw[4];
+      const uint32_t s0 = fq4_probs(p, *reinterpret_cast<uint32_t(*)[2]>(cw));
+      const uint32_t s1 = fq4_probs(p + 16, *reinterpret_cast<uint32_t(*)[2]>(cw + 2));
+      sfw |= (s0 | (s1 << 8)) << (16 * c);
+      const int unit = (col0 + 32 * c) >> 5;
+      st_shared_v4(pbase + (row >> 3) * 512 + (row & 7) * 64 + ((unit ^ ((row >> 1) & 3)) << 4), cw[0], cw[1],
+                   cw[2], cw[3]);
+    } else {
+      uint32_t w[16];
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      if (QP) {
-        uint32_t rr[8];
-        const float s = fq16_probs(p + 16 * b, rr);
-        if (PV_F16) {
-          const uint32_t s2 = f16x2_broadcast(s);
+      for (int b = 0; b < 2; ++b) {
+        if (QP) {
+          uint32_t rr[8];
+          const float s = fq16_probs(p + 16 * b, rr);
+          if (PV_F16) {
+            const uint32_t s2 = f16x2_broadcast(s);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w[8 * b + i] = hmul2_u32(rr[i], s2);
+            for (int i = 0; i < 8; ++i) w[8 * b + i] = hmul2_u32(rr[i], s2);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 g = unpack_f16x2(rr[i]);
+              w[8 * b + i] = pack_bf16x2(g.x * s, g.y * s);
+            }
+          }
         } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float2 g = unpack_f16x2(rr[i]);
-            w[8 * b + i] = pack_bf16x2(g.x * s, g.y * s);
-          }
+          for (int i = 0; i < 8; ++i)
+            w[8 * b + i] = PV_F16 ? pack_f16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1])
+                                  : pack_bf16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1]);
         }
-      } else {
+      }
+      // 32 keys = four 16-byte units of the 64-key swizzled chunk holding them
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          w[8 * b + i] = PV_F16 ? pack_f16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1])
-                                : pack_bf16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1]);
+      for (int u = 0; u < 4; ++u) {
+        const int cc = col0 + 32 * c;
+        const uint32_t addr = pbase + static_cast<uint32_t>(cc >> 6) * kChunkBytes +
+                              sw128_offset(row, ((cc & 63) >> 3) + u);
+        st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       }
     }
-    // 32 keys = four 16-byte units of the 64-key swizzled chunk holding them
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int cc = col0 + 32 * c;
-      const uint32_t addr = pbase + static_cast<uint32_t>(cc >> 6) * kChunkBytes +
-                            sw128_offset(row, ((cc & 63) >> 3) + u);
-      st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-    }
+  }
+  if (PVM == 2) {
+    // this thread's 64 keys are one 64-key scale block (k-chunk col0 / 64):
+    // row r's four bytes at (r % 32) * 16 + (r / 32) * 4
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(psf + static_cast<uint32_t>(col0 >> 6) * 512 + (row & 31) * 16 +
+                                                   (row >> 5) * 4),
+                 "r"(sfw)
+                 : "memory");
   }
   return lsum.x + lsum.y;
 }
@@ -180,12 +217,15 @@ __device__ __forceinline__ void group_sync(int wq) {
 template <int G>
 constexpr int fwd_threads() { return (2 + 4 * G + 1 + 3) / 4 * 128; }
 
-template <int D, int FP4S, int PV_F16, int QP, int G>
+template <int D, int FP4S, int PVM, int QP, int G>
 __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
-  using L = FwdLayout<D, FP4S>;
+  constexpr int PV4 = PVM == 2;
+  constexpr int PV_F16 = PVM == 1;
+  using L = FwdLayout<D, FP4S, PV4>;
   static_assert(G <= kFwdG, "column groups beyond the partial-sum block");
+  static_assert(L::kNSK <= 8 && L::kNSV <= 4, "ring deeper than its barrier arrays");
   constexpr int kNSK = L::kNSK, kNSV = L::kNSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
@@ -268,10 +308,17 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
           const int u = t - nk;
           const int vs = u % kNSV;
           if (u >= kNSV && !mbar_wait(&bars->vempty[vs], ((u / kNSV) - 1) & 1, abort)) break;
-          mbar_arrive_expect_tx(&bars->vfull[vs], L::kVT);
-          for (int c = 0; c < Tile<D>::kChunks; ++c)
-            tma_load_3d(smem + L::kV + vs * L::kVT + c * kChunkBytes, &tmV, &bars->vfull[vs],
-                        c * 64, j * kBN, bh);
+          mbar_arrive_expect_tx(&bars->vfull[vs], L::kVT + L::kVSF);
+          if (PV4) {
+            // fq(V) codes [D][128 keys / 2] and the tile's two scale blocks
+            tma_load_3d(smem + L::kV + vs * L::kVT, &tmV, &bars->vfull[vs], j * (kBN / 2), 0, bh);
+            bulk_load(smem + L::kVSFo + vs * L::kVSF, a.vsf + (static_cast<size_t>(bh) * nk + j) * L::kVSF, L::kVSF,
+                      &bars->vfull[vs]);
+          } else {
+            for (int c = 0; c < Tile<D>::kChunks; ++c)
+              tma_load_3d(smem + L::kV + vs * L::kVT + c * kChunkBytes, &tmV, &bars->vfull[vs],
+                          c * 64, j * kBN, bh);
+          }
           vissued = u + 1;
         }
       }
@@ -312,6 +359,9 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       const uint64_t dK = FP4S ? sdesc_make(sbase + L::kK, 16, L::kCodeSBO, L::kCodeLayout) : desc_k(sbase + L::kK);
       const uint64_t dKSF = sdesc_make(sbase + L::kKSF, 16, 128, 0);
       const uint64_t dP = desc_k(sbase + L::kP), dV = desc_mn(sbase + L::kV);
+      const uint64_t dP4 = sdesc_make(sbase + L::kP, 16, 512, 4), dV4 = sdesc_make(sbase + L::kV, 16, 512, 4);
+      const uint64_t dPSF = sdesc_make(sbase + L::kPSFo, 16, 128, 0), dVSF = sdesc_make(sbase + L::kVSFo, 16, 128, 0);
+      constexpr uint32_t idPV4 = idesc_mxf4(kBM, D);
       // S tile t (K tile t mod nk) into TMEM column dcol, signalling `full`
       auto issue_s = [&](int t, uint32_t dcol, uint64_t *full) -> bool {
         const int st = t % kNSK;
@@ -364,8 +414,25 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
             break;
           }
           tc_fence_after();
-          mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemO, sdesc_add(dP, pb * L::kPBytes), sdesc_add(dV, vs * L::kVT), idPV,
-                                 j > 0);
+          if (PV4) {
+            // scales of this P tile and V stage into TMEM (their previous
+            // users, P V two and kNSV tiles back, have completed: the rows
+            // and the producer waited for them before refilling)
+            const uint32_t sfp = tmem + L::kTmemSFP + pb * 8, sfv = tmem + L::kTmemSFV + vs * 8;
+#pragma unroll
+            for (int kc = 0; kc < 2; ++kc) {
+              tmem_cp_32x128b_x4(sfp + kc * 4, sdesc_add(dPSF, pb * L::kPSF + kc * 512));
+              tmem_cp_32x128b_x4(sfv + kc * 4, sdesc_add(dVSF, vs * L::kVSF + kc * 512));
+            }
+            const uint64_t dPs = sdesc_add(dP4, pb * L::kPBytes), dVs = sdesc_add(dV4, vs * L::kVT);
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              umma_fp4(tmem + L::kTmemO, sdesc_add(dPs, kk * 32), sdesc_add(dVs, kk * 32), idPV4, sfp + kk * 4,
+                       sfv + kk * 4, (j > 0 || kk > 0) ? 1u : 0u);
+          } else {
+            mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemO, sdesc_add(dP, pb * L::kPBytes), sdesc_add(dV, vs * L::kVT),
+                                   idPV, j > 0);
+          }
           umma_commit(&bars->vempty[vs]);
           umma_commit(&bars->pempty[pb]);
         }
@@ -412,10 +479,11 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
+      const uint32_t psf = sbase + L::kPSFo + pb * L::kPSF;
       if (j == nk - 1 && last_valid < kBN)
-        lsum += prob_cols<PV_F16, QP, true, NC>(taddr, col0, last_valid, cl, nml, pbase, rr.row);
+        lsum += prob_cols<PVM, QP, true, NC>(taddr, col0, last_valid, cl, nml, pbase, psf, rr.row);
       else
-        lsum += prob_cols<PV_F16, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, rr.row);
+        lsum += prob_cols<PVM, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, psf, rr.row);
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
@@ -480,14 +548,14 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
   }
 }
 
-template <int D, int FP4S, int PV_F16, int QP>
+template <int D, int FP4S, int PVM, int QP>
 static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const FwdArgs &a, int BH, cudaStream_t stream) {
-  using L = FwdLayout<D, FP4S>;
+  using L = FwdLayout<D, FP4S, PVM == 2>;
   static_assert(L::kDynSmem <= 232448, "forward shared memory over the 227 KB limit");
   static_assert(sizeof(FwdBars) <= L::kBarBytes, "forward barrier block larger than its reservation");
-  static_assert(!FP4S || L::kTmemSFB + L::kNSK * L::kSFCols <= L::kTmemCols, "forward TMEM over 512 columns");
-  auto kern = attn_fwd_kernel<D, FP4S, PV_F16, QP, kFwdG>;
+  static_assert(!FP4S || L::kTmemEnd <= L::kTmemCols, "forward TMEM over 512 columns");
+  auto kern = attn_fwd_kernel<D, FP4S, PVM, QP, kFwdG>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nq_tiles, BH);
@@ -496,24 +564,25 @@ static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, co
 }
 
 template <int D, int FP4S>
-static cudaError_t fwd_dispatch(bool pv_f16, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+static cudaError_t fwd_dispatch(int pv_mode, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, const FwdArgs &a, int BH, cudaStream_t stream) {
-  if (pv_f16)
+  if (pv_mode == 2) return launch_fwd_t<D, FP4S, 2, 1>(tq, tk, tv, a, BH, stream);
+  if (pv_mode == 1)
     return quant_p ? launch_fwd_t<D, FP4S, 1, 1>(tq, tk, tv, a, BH, stream)
                    : launch_fwd_t<D, FP4S, 1, 0>(tq, tk, tv, a, BH, stream);
   return quant_p ? launch_fwd_t<D, FP4S, 0, 1>(tq, tk, tv, a, BH, stream)
                  : launch_fwd_t<D, FP4S, 0, 0>(tq, tk, tv, a, BH, stream);
 }
 
-cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUtensorMap &tq,
+cudaError_t launch_fwd(int D, bool qk_f16, int pv_mode, bool quant_p, const CUtensorMap &tq,
                        const CUtensorMap &tk, const CUtensorMap &tv, const FwdArgs &a, int BH,
                        cudaStream_t stream) {
   // quantized Q and K: S runs on the NVFP4 tensor-core path
   if (D == 128)
-    return qk_f16 ? fwd_dispatch<128, 1>(pv_f16, quant_p, tq, tk, tv, a, BH, stream)
-                  : fwd_dispatch<128, 0>(pv_f16, quant_p, tq, tk, tv, a, BH, stream);
-  return qk_f16 ? fwd_dispatch<64, 1>(pv_f16, quant_p, tq, tk, tv, a, BH, stream)
-                : fwd_dispatch<64, 0>(pv_f16, quant_p, tq, tk, tv, a, BH, stream);
+    return qk_f16 ? fwd_dispatch<128, 1>(pv_mode, quant_p, tq, tk, tv, a, BH, stream)
+                  : fwd_dispatch<128, 0>(pv_mode, quant_p, tq, tk, tv, a, BH, stream);
+  return qk_f16 ? fwd_dispatch<64, 1>(pv_mode, quant_p, tq, tk, tv, a, BH, stream)
+                : fwd_dispatch<64, 0>(pv_mode, quant_p, tq, tk, tv, a, BH, stream);
 }
 
 }  // namespace attnqat

@@ -15,6 +15,7 @@ struct FwdArgs {
   float scale_log2;   // c * log2(e)
   const uint8_t *qsf;   // scale-factor tiles of fq(Q), fq(K) (NVFP4 S path)
   const uint8_t *ksf;
+  const uint8_t *vsf;   // scale-factor tiles of fq(V) along tokens (NVFP4 P V path)
   __nv_bfloat16 *o;
   float *o32;   // float32 copy of O kept in the workspace for the backward's Delta
   float *lse;
@@ -40,24 +41,17 @@ struct BwdArgs {
 };
 
 // Forward.  tv: 3-D TMA map {D, L, B*H} with 64 x 128 boxes, 128-byte swizzle
-// over fq(V) (fp16 when pv_f16, else bf16).  With qk_f16 (Q and K quantized)
-// tq/tk map the packed NVFP4 codes {D/2 bytes, L, B*H} with (D/2) x 128 boxes
-// and a D/2-byte swizzle, a.qsf/a.ksf point at their scale-factor tiles, and S
-// runs as a block-scaled NVFP4 MMA; otherwise tq/tk map the bf16 Q and K.
-cudaError_t launch_fwd(int D, bool qk_f16, bool pv_f16, bool quant_p, const CUtensorMap &tq,
+// over fq(V) (pv_mode 1: fp16, 0: bf16); with pv_mode 2 (every quantizer on,
+// Lk % 32 == 0) it maps fq(V)'s packed codes {Lk/2 bytes, D, B*H} with
+// 64-byte x D boxes and 64-byte swizzle, a.vsf their scale tiles, and P V is
+// a block-scaled NVFP4 MMA.  With qk_f16 (Q and K quantized) tq/tk map the
+// packed NVFP4 codes {D/2 bytes, L, B*H} with (D/2) x 128 boxes and a
+// D/2-byte swizzle, a.qsf/a.ksf point at their scale-factor tiles, and S runs
+// as a block-scaled NVFP4 MMA; otherwise tq/tk map the bf16 Q and K.
+cudaError_t launch_fwd(int D, bool qk_f16, int pv_mode, bool quant_p, const CUtensorMap &tq,
                        const CUtensorMap &tk, const CUtensorMap &tv, const FwdArgs &a, int BH,
                        cudaStream_t stream);
 
-// Backward dK/dV kernel (one CTA per 128-key tile) and dQ kernel (one CTA per
-// 128-query tile).  Maps over fq(Q), fq(K) (fp16 when qk_f16, else bf16),
-// fq(V) and dO.  With qk_f16 the dS operand is fp16 (scaled by a power of
-// two), else bf16.  With do_f16 (requires qk_f16 and quantized V and P) the dO
-// map is over the exact fp16 copy dO * 2^e and the V map over fp16 fq(V): dP
-// is exact as before and dV takes fq(P~)/l * 2^14 as an fp16 operand; else
-// both maps are bf16.
-// With qk_f16, tk maps the packed NVFP4 K codes and tq4 the Q codes (as for
-// the forward; a.ksf/a.qsf their scale tiles) for S, and tq the fp16 fq(Q)
-// that dK = dS^T fq(Q) reads; otherwise tq/tk are bf16 and tq4 is unused.
 cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
                             const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
                             const CUtensorMap &tq4, const BwdArgs &a, int BH, cudaStream_t stream);
@@ -73,11 +67,13 @@ cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq
 // folded in with an atomic max; must start at 0) may be null.  With
 // sf_tile_rows = L > 0 (contiguous [heads*L, cols] rows), the scales go to
 // the per-head, per-128-row-tile layout the block-scaled MMA reads from TMEM
-// (padding rows of the last tile are not written).
+// (padding rows of the last tile are not written); with sf_col_tiles (rows
+// <= 128, e.g. V's D channels blocked along tokens) to the per-batch,
+// per-128-column-tile layout of the same kind.
 cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols,
                             int64_t sb, int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales,
                             uint16_t *deq, uint16_t *deq_f16, float *absmax, cudaStream_t stream,
-                            int64_t sf_tile_rows = 0);
+                            int64_t sf_tile_rows = 0, bool sf_col_tiles = false);
 
 // delta[r] = sum_d dO[r][d] * O[r][d] over `rows` rows of D values (O float32,
 // dO bf16); folds max_r |dO_r|_1 into stats[0], max_r |delta_r| into

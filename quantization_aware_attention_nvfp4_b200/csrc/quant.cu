@@ -117,7 +117,8 @@ __global__ void __launch_bounds__(256)
     quantize_view_kernel(const uint16_t *__restrict__ x, int64_t batch, int64_t rows, int64_t cols,
                          int64_t sb, int64_t sr, int64_t sc, uint8_t *__restrict__ codes,
                          uint8_t *__restrict__ scales, uint16_t *__restrict__ deq,
-                         uint16_t *__restrict__ deq_f16, float *__restrict__ absmax, int64_t sf_tile_rows) {
+                         uint16_t *__restrict__ deq_f16, float *__restrict__ absmax, int64_t sf_tile_rows,
+                         bool sf_col_tiles) {
   const int64_t nblk = cols / 16;
   float vmax = 0.0f;  // largest dequantized magnitude this thread produced
   const int64_t total = batch * rows * nblk;
@@ -167,6 +168,15 @@ __global__ void __launch_bounds__(256)
         const int64_t off = ((head * ntiles + (t >> 7)) * (nblk >> 2) + (b >> 2)) * 512 + (t & 31) * 16 +
                             ((t & 127) >> 5) * 4 + (b & 3);
         scales[off] = static_cast<uint8_t>(scode);
+      } else if (sf_col_tiles) {
+        // the same block layout with the roles swapped (V blocked along
+        // tokens as the N x K operand of P V): per batch z, per 128-column
+        // tile, per 64-column chunk a 512-byte block in which row r (r < 128)
+        // holds its four 16-column scales at bytes (r % 32)*16 + (r / 32)*4
+        const int64_t ntiles = (nblk + 7) / 8;
+        const int64_t off = ((z * ntiles + (b >> 3)) * 2 + ((b >> 2) & 1)) * 512 + (r & 31) * 16 + (r >> 5) * 4 +
+                            (b & 3);
+        scales[off] = static_cast<uint8_t>(scode);
       } else {
         scales[blk] = static_cast<uint8_t>(scode);
       }
@@ -183,7 +193,8 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols, int64_t sb,
                             int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales, uint16_t *deq,
-                            uint16_t *deq_f16, float *absmax, cudaStream_t stream, int64_t sf_tile_rows) {
+                            uint16_t *deq_f16, float *absmax, cudaStream_t stream, int64_t sf_tile_rows,
+                            bool sf_col_tiles) {
   const int64_t total = batch * rows * (cols / 16);
   if (total == 0) return cudaSuccess;
   int dev = 0, sms = 148;
@@ -196,10 +207,10 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
   const bool row_fastest = (sc != 1) && (sr == 1);
   if (row_fastest)
     quantize_view_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax, sf_tile_rows);
+        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax, sf_tile_rows, sf_col_tiles);
   else
     quantize_view_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax, sf_tile_rows);
+        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, deq_f16, absmax, sf_tile_rows, sf_col_tiles);
   return cudaGetLastError();
 }
 

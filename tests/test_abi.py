@@ -35,8 +35,9 @@ def test_strerror_texts():
 def _expected_ws(B, H, Lq, Lk, D, flags):
     """Workspace layout restated: 256-byte aligned regions for fq(Q), fq(K),
     fq(V) (bf16), fq(V) (fp16), float32 O, Delta, 16 bytes of statistics,
-    with every quantizer on the fp16 copy of dO and, with Q and K quantized,
-    their packed codes and scale tiles."""
+    with every quantizer on the fp16 copy of dO, with Q and K quantized
+    their packed codes and scale tiles, and with every quantizer on, D = 128
+    and Lk % 32 == 0 fq(V)'s packed codes and scale tiles."""
     al = lambda x: (x + 255) // 256 * 256
     BH = B * H
     n = 0
@@ -54,6 +55,9 @@ def _expected_ws(B, H, Lq, Lk, D, flags):
         # 128 rows x 64 columns, for Q then K
         for L in (Lq, Lk):
             n += al(BH * L * D // 2) + al(BH * ((L + 127) // 128) * (D // 64) * 512)
+    if flags & 15 == 15 and Lk % 32 == 0 and D == 128:
+        # fq(V)'s packed codes and 1 KB of scales per 128-token tile
+        n += al(BH * Lk * D // 2) + al(BH * ((Lk + 127) // 128) * 1024)
     return n
 
 
