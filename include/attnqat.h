@@ -138,8 +138,11 @@ int attnqat_quantize(const void *x, int64_t batch, int64_t rows, int64_t cols,
  * written by the forward, the backward's Delta, 16 bytes of statistics, an
  * exact fp16 copy of dO * 2^e when all four quantizers are on, and -- with Q
  * and K quantized -- their packed NVFP4 codes (D/2 bytes per row) with scale
- * tiles (512 bytes per 128 rows x 64 columns) for the forward's block-scaled
- * S = fq(Q) fq(K)^T.  Every region is 256-byte aligned.
+ * tiles (512 bytes per 128 rows x 64 columns) for the block-scaled
+ * S = fq(Q) fq(K)^T; with all four quantizers on, D = 128 and Lk % 32 == 0
+ * also fq(V)'s packed codes ([B*H][D][Lk/2] bytes, blocks along tokens) and
+ * scale tiles (1 KB per 128 tokens) for the forward's block-scaled
+ * fq(P~) fq(V).  Every region is 256-byte aligned.
  */
 size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D,
                               uint32_t flags);
