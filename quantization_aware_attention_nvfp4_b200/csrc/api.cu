@@ -305,10 +305,12 @@ static int prepare_operands(const void *q, const void *k, const void *v, int B, 
       if (e != cudaSuccess) return cuda_fail(e);
     }
     ProfScope ps("quantize_v", stream);
+    // the bf16 copy feeds only the backward's bf16 dP / dV, unused when every
+    // quantizer is on (the fp16 copy and the codes serve both passes then)
     e = launch_quantize(static_cast<const uint16_t *>(v), BH, D, Lk, static_cast<int64_t>(Lk) * D, 1, D,
                         pv4 ? ws + w.vc : nullptr, pv4 ? ws + w.vsf : nullptr,
-                        reinterpret_cast<uint16_t *>(ws + w.vh), reinterpret_cast<uint16_t *>(ws + w.vh16),
-                        stats + 2, stream, 0, pv4);
+                        do_f16(flags) ? nullptr : reinterpret_cast<uint16_t *>(ws + w.vh),
+                        reinterpret_cast<uint16_t *>(ws + w.vh16), stats + 2, stream, 0, pv4);
   } else {
     ProfScope ps("absmax_v", stream);
     e = launch_absmax(static_cast<const __nv_bfloat16 *>(v), BH * Lk * D, stats + 2, stream);
