@@ -78,6 +78,10 @@ def _load():
             lib.oracle_e2m1_round_many.argtypes = [P, P, L, P]
             lib.oracle_quantize_rows.restype = None
             lib.oracle_quantize_rows.argtypes = [P, L, L, L, L, P, P, P]
+            lib.oracle_global_scale.restype = ctypes.c_float
+            lib.oracle_global_scale.argtypes = [ctypes.c_double]
+            lib.oracle_quantize_rows_gs.restype = None
+            lib.oracle_quantize_rows_gs.argtypes = [P, L, L, L, L, P, P, P, P]
             lib.oracle_fq_f64_rows.restype = None
             lib.oracle_fq_f64_rows.argtypes = [P, L, L, P, P]
             lib.oracle_operands.restype = None
@@ -164,6 +168,29 @@ def quantize_rows(x_bits: np.ndarray, rows: int, cols: int, stride_row: int,
     _load().oracle_quantize_rows(_ptr(x), rows, cols, stride_row, stride_col,
                                  _ptr(codes), _ptr(scales), _ptr(deq))
     return codes, scales, deq
+
+
+def global_scale(amax: float) -> float:
+    """The float32 global scale 2688 / amax (1 for amax = 0)."""
+    return float(_load().oracle_global_scale(float(amax)))
+
+
+def quantize_rows_gs(x_bits: np.ndarray, rows: int, cols: int, stride_row: int,
+                     stride_col: int):
+    """NVFP4 with an FP32 global scale (reading R15) of a strided bf16 view.
+
+    Returns (codes uint8 [rows, cols/2], scales uint8 [rows, cols/16],
+    deq bf16 bits uint16 [rows, cols], global scale float)."""
+    x = _bits(x_bits).reshape(-1)
+    if cols % 16:
+        raise ValueError("cols must be a multiple of 16")
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    deq = np.zeros((rows, cols), np.uint16)
+    g = np.zeros(1, np.float32)
+    _load().oracle_quantize_rows_gs(_ptr(x), rows, cols, stride_row, stride_col, _ptr(codes), _ptr(scales),
+                                    _ptr(deq), _ptr(g))
+    return codes, scales, deq, float(g[0])
 
 
 def fq_f64_rows(x: np.ndarray):

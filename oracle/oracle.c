@@ -214,6 +214,121 @@ void oracle_quantize_rows(const uint16_t *x, long rows, long cols, long srow,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* NVFP4 with an FP32 global scale                                           */
+/* ------------------------------------------------------------------------ */
+
+/* The linear-layer variant of the format (vsqa-test-1.3b metadata.json,
+ * "linear_quantization": "NVFP4 W4A4: E2M1 values, 16-element blocks, FP8
+ * E4M3 block scales, FP32 global scale", with the activation global scale
+ * "dynamic, 448*6/max|X| recomputed every forward").  The reading of the
+ * steps the page leaves open (listed in the design notes as R15):
+ *   G   = the float32 quotient 2688 / max|x| (1 when max|x| = 0; the largest
+ *         finite float32 if the quotient overflows);
+ *   k_b = E4M3 round-to-nearest-even (saturating) of the exact a_b * G / 6,
+ *         a_b the block's max |x|;  s_b = value of k_b;
+ *   c   = E2M1 round-to-nearest-even (saturating) of the exact |x| G / s_b
+ *         (0 when s_b = 0);
+ *   deq = sign * E2M1(c) * s_b / G, rounded once to bfloat16 (nearest, ties
+ *         to even).
+ * a_b * G and |x| * G are exact in float64 (8- and 24-bit significands), so
+ * the roundings above reuse the exact midpoint tests of the plain format.  */
+
+/* The float32 global scale for a tensor whose largest magnitude is amax. */
+float oracle_global_scale(double amax)
+{
+    if (!(amax > 0.0))
+        return 1.0f;
+    volatile float num = 2688.0f;
+    volatile float den = (float)amax; /* amax is a bf16 value: exact */
+    float g = num / den;              /* IEEE float32 division */
+    if (isinf(g))
+        g = 3.40282347e38f;
+    return g;
+}
+
+/* Value of a non-negative bfloat16 bit pattern. */
+static double bf16_bits_value(uint32_t h)
+{
+    return oracle_bf16_value((uint16_t)h);
+}
+
+/* bfloat16 bits of the exact quotient n / g (n >= 0, g > 0, exact doubles;
+ * every product below has at most 33 significant bits, so it is exact),
+ * rounded to nearest, ties to even.  Start from the truncated float64
+ * quotient and step along the (monotonic) bit patterns of positive bfloat16
+ * values until lo <= n/g < next(lo), then compare with the midpoint.        */
+static uint16_t bf16_of_quotient(double n, double g)
+{
+    if (n == 0.0)
+        return 0;
+    float qf = (float)(n / g);
+    uint32_t u;
+    memcpy(&u, &qf, sizeof u);
+    uint32_t h = u >> 16;                          /* truncation: value <= qf */
+    while (h > 0 && bf16_bits_value(h) * g > n)
+        h--;
+    while (bf16_bits_value(h + 1) * g <= n)
+        h++;
+    double mid = 0.5 * (bf16_bits_value(h) + bf16_bits_value(h + 1));
+    if (n < mid * g)
+        return (uint16_t)h;
+    if (n > mid * g)
+        return (uint16_t)(h + 1);
+    return (uint16_t)((h % 2 == 0) ? h : h + 1);    /* tie: even bit pattern */
+}
+
+/* Global-scale fq of a strided bf16 view (same view as oracle_quantize_rows).
+ * Outputs: codes [rows][cols/2] (element 2i in the low nibble, sign in bit 3
+ * of each nibble), scales [rows][cols/16] (E4M3 codes of s_b), deq
+ * [rows][cols] bfloat16 bits, and *gscale (any output may be NULL).         */
+void oracle_quantize_rows_gs(const uint16_t *x, long rows, long cols, long srow,
+                             long scol, uint8_t *codes, uint8_t *scales,
+                             uint16_t *deq, float *gscale)
+{
+    long nblk = cols / BLOCK;
+    double amax = 0.0;
+    for (long r = 0; r < rows; r++)
+        for (long j = 0; j < cols; j++) {
+            double a = fabs(oracle_bf16_value(x[r * srow + j * scol]));
+            if (a > amax)
+                amax = a;
+        }
+    float gf = oracle_global_scale(amax);
+    double g = (double)gf;
+    if (gscale)
+        *gscale = gf;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; r++) {
+        for (long b = 0; b < nblk; b++) {
+            double xb[BLOCK];
+            double ab = 0.0;
+            for (long i = 0; i < BLOCK; i++) {
+                xb[i] = oracle_bf16_value(x[r * srow + (b * BLOCK + i) * scol]);
+                if (fabs(xb[i]) > ab)
+                    ab = fabs(xb[i]);
+            }
+            int k = oracle_e4m3_round_div6(ab * g);   /* exact product */
+            double sb = oracle_e4m3_value(k);
+            if (scales)
+                scales[r * nblk + b] = (uint8_t)k;
+            uint8_t cb[BLOCK];
+            for (long i = 0; i < BLOCK; i++) {
+                int neg = signbit(xb[i]) ? 1 : 0;
+                int c = (sb > 0.0) ? oracle_e2m1_round(fabs(xb[i]) * g, sb) : 0;
+                cb[i] = (uint8_t)((neg << 3) | c);
+                if (deq) {
+                    uint16_t h = bf16_of_quotient(E2M1_GRID[c] * sb, g);
+                    deq[r * cols + b * BLOCK + i] = (uint16_t)(h | (neg ? 0x8000u : 0u));
+                }
+            }
+            if (codes)
+                for (long i = 0; i < BLOCK; i += 2)
+                    codes[r * (cols / 2) + (b * BLOCK + i) / 2] = (uint8_t)(cb[i] | (cb[i + 1] << 4));
+        }
+    }
+}
+
 /* fq of float64 values, blocks of 16 along a row (used for tests of the
  * block rounding on non-bf16 inputs, e.g. probabilities).                   */
 void oracle_fq_f64_rows(const double *x, long rows, long cols, double *y,

@@ -500,3 +500,137 @@ def test_sampled_rows_equal_full_computation():
     assert np.array_equal(hd.dq_rows(rows), dQ[rows])
     dKs, dVs = hd.dkdv_blocks(np.array([2]))
     assert np.array_equal(dKs, dK[32:48]) and np.array_equal(dVs, dV[32:48])
+
+
+# ------------------------------------------ NVFP4 with an FP32 global scale ----
+
+def _bf16_value_fraction(h):
+    return Fraction(float(W.bf16_bits_to_f32(np.array([h], np.uint16))[0]))
+
+
+def _bf16_rne_fraction(v):
+    """bf16 bit pattern nearest to the exact rational v >= 0, ties to the even
+    pattern (a search over neighbouring patterns in exact arithmetic)."""
+    if v == 0:
+        return 0
+    h = int(W.f32_to_bf16_bits(np.array([float(v)], np.float32))[0])
+    while h > 0 and _bf16_value_fraction(h) > v:
+        h -= 1
+    while _bf16_value_fraction(h + 1) <= v:
+        h += 1
+    lo, hi = _bf16_value_fraction(h), _bf16_value_fraction(h + 1)
+    if v - lo != hi - v:
+        return h if v - lo < hi - v else h + 1
+    return h if h % 2 == 0 else h + 1
+
+
+def _fq_gs_fraction(xs):
+    """The global-scale format in exact rationals: G = float32(2688 / max|x|),
+    block scale = nearest E4M3 to a_b G / 6, code = nearest E2M1 to |x| G / s,
+    value = sign * E2M1 * s / G rounded to bf16 (all ties to even)."""
+    amax = float(np.max(np.abs(xs)))
+    g32 = np.float32(1.0) if amax == 0 else np.float32(2688.0) / np.float32(amax)
+    if not np.isfinite(g32):
+        g32 = np.float32(np.finfo(np.float32).max)
+    g = Fraction(float(g32))
+    vals = _e4m3_values_fraction()
+    grid = [Fraction(v) for v in GRID]
+    rows, cols = xs.shape
+    codes = np.zeros((rows, cols), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    deq = np.zeros((rows, cols), np.uint16)
+    for r in range(rows):
+        for b in range(cols // 16):
+            blk = [Fraction(float(v)) for v in xs[r, 16 * b:16 * b + 16]]
+            k = _nearest_fraction(max(abs(v) for v in blk) * g / 6, vals)
+            s = vals[k]
+            scales[r, b] = k
+            for i, v in enumerate(blk):
+                neg = 1 if np.signbit(xs[r, 16 * b + i]) else 0
+                c = 0 if s == 0 else _nearest_fraction(abs(v) * g / s, grid)
+                codes[r, 16 * b + i] = (neg << 3) | c
+                deq[r, 16 * b + i] = _bf16_rne_fraction(grid[c] * s / g) | (0x8000 if neg else 0)
+    return codes, scales, deq, float(g32)
+
+
+def _pack(codes):
+    return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+
+
+@pytest.mark.parametrize("seed,mag", [(1, 1.0), (2, 1e-5), (3, 3e3), (4, 0.37), (5, 1e-30)])
+def test_global_scale_format_vs_exact_rationals(seed, mag):
+    """Exact rational brute force of the global-scale format on random and
+    tie-rich tensors across magnitudes (including tiny ones whose global
+    scale is huge)."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((6, 32)).astype(np.float32) * np.float32(mag)
+    x[1, :16] *= np.float32(1e-3)          # a block far below the tensor max
+    x[2, :] = np.float32(0.0)              # zero blocks
+    bits = W.f32_to_bf16_bits(x)
+    xs = W.bf16_bits_to_f32(bits).reshape(6, 32)
+    codes, scales, deq, g = oracle.quantize_rows_gs(bits, 6, 32, 32, 1)
+    wc, ws, wd, wg = _fq_gs_fraction(xs)
+    assert np.float32(g) == np.float32(wg)
+    assert np.array_equal(scales, ws)
+    assert np.array_equal(codes, _pack(wc))
+    assert np.array_equal(deq, wd)
+
+
+def test_global_scale_one_reduces_to_plain_format():
+    """max|x| = 2688 gives G = 1: codes, scales and values of the plain
+    format (pinned above against torch and exact rationals)."""
+    rng = np.random.default_rng(8)
+    x = (rng.standard_normal((5, 48)) * 300).astype(np.float32)
+    x[3, 7] = -2688.0
+    bits = W.f32_to_bf16_bits(x)
+    c, s, d, g = oracle.quantize_rows_gs(bits, 5, 48, 48, 1)
+    c0, s0, d0 = oracle.quantize_rows(bits, 5, 48, 48, 1)
+    assert g == 1.0
+    assert np.array_equal(c, c0) and np.array_equal(s, s0)
+    assert np.array_equal(W.bf16_bits_to_f32(d.reshape(-1)).astype(np.float64), d0.reshape(-1))
+
+
+@pytest.mark.parametrize("k", [-6, -1, 3, 9])
+def test_global_scale_power_of_two_is_plain_format_of_scaled_input(k):
+    """max|x| = 2688 * 2^-k gives G = 2^k exactly, and the result is the plain
+    format applied to x * 2^k, scaled back by 2^-k."""
+    rng = np.random.default_rng(20 + k)
+    x = (rng.standard_normal((4, 64)) * 100).astype(np.float32)
+    x[0, 0] = 2688.0
+    x = x * np.float32(2.0 ** -k)
+    bits = W.f32_to_bf16_bits(x)
+    c, s, d, g = oracle.quantize_rows_gs(bits, 4, 64, 64, 1)
+    assert g == 2.0 ** k
+    xs = W.bf16_bits_to_f32(bits).reshape(4, 64) * np.float32(2.0 ** k)
+    c0, s0, d0 = oracle.quantize_rows(W.f32_to_bf16_bits(xs), 4, 64, 64, 1)
+    assert np.array_equal(c, c0) and np.array_equal(s, s0)
+    assert np.array_equal(W.bf16_bits_to_f32(d.reshape(-1)).astype(np.float64) * 2.0 ** k, d0.reshape(-1))
+
+
+def test_global_max_round_trips_and_sign_symmetry():
+    """The tensor's largest magnitude gets scale 448 and code 6 and comes back
+    exactly; fq(-x) = -fq(x) with the same scales and global scale."""
+    rng = np.random.default_rng(31)
+    for trial in range(20):
+        x = (rng.standard_normal((3, 32)) * 10 ** rng.uniform(-8, 4)).astype(np.float32)
+        bits = W.f32_to_bf16_bits(x)
+        xs = W.bf16_bits_to_f32(bits).reshape(3, 32)
+        c, s, d, g = oracle.quantize_rows_gs(bits, 3, 32, 32, 1)
+        i = np.unravel_index(np.argmax(np.abs(xs)), xs.shape)
+        assert s[i[0], i[1] // 16] == 126  # E4M3 448
+        assert W.bf16_bits_to_f32(d[i[0], i[1]:i[1] + 1])[0] == xs[i]
+        cn, sn, dn, gn = oracle.quantize_rows_gs(bits ^ np.uint16(0x8000), 3, 32, 32, 1)
+        assert gn == g and np.array_equal(sn, s)
+        assert np.array_equal(cn, c ^ np.uint8(0x88)) and np.array_equal(dn, d ^ np.uint16(0x8000))
+
+
+def test_global_scale_special_cases():
+    """All-zero input: G = 1 and zeros; a max below 2688 / FLT_MAX: the
+    quotient overflows float32 and G saturates to the largest finite float."""
+    z = np.zeros((2, 16), np.uint16)
+    c, s, d, g = oracle.quantize_rows_gs(z, 2, 16, 16, 1)
+    assert g == 1.0 and not c.any() and not s.any() and not d.any()
+    assert oracle.global_scale(0.0) == 1.0
+    tiny = float(W.bf16_bits_to_f32(np.array([1], np.uint16))[0])  # smallest bf16 subnormal
+    assert oracle.global_scale(tiny) == float(np.finfo(np.float32).max)
+    assert oracle.global_scale(2688.0) == 1.0
