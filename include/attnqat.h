@@ -130,6 +130,34 @@ int attnqat_quantize(const void *x, int64_t batch, int64_t rows, int64_t cols,
                      void *deq, void *stream);
 
 /*
+ * attnqat_quantize_gs -- NVFP4 with an FP32 global scale (the format's
+ * linear-layer variant).
+ *
+ * Defined by: vsqa-test-1.3b metadata.json, "linear_quantization": "NVFP4
+ * W4A4: E2M1 values, 16-element blocks, FP8 E4M3 block scales, FP32 global
+ * scale", the activation global scale "dynamic, 448*6/max|X| recomputed every
+ * forward".  The steps the page leaves open are read as:
+ *   G   = float32 2688 / max|x| over the whole view (1 if every element is
+ *         zero; the largest finite float32 if the quotient overflows);
+ *   k_b = E4M3 code nearest to a_b * G / 6 (a_b = the block's max |x|), ties
+ *         to even, saturating at 448;  s_b = its value;
+ *   c   = E2M1 code nearest to |x| * G / s_b, ties to even, saturating at 6;
+ *   deq = sign * E2M1(c) * s_b / G, rounded to bf16 (nearest, ties to even).
+ * Every rounding is exact (a_b G and |x| G are exact in float64).
+ *
+ * View, codes, scales and deq (bf16, may be NULL): as attnqat_quantize, with
+ * scales holding the k_b.  gscale: one device float32, caller-owned, that
+ * receives G; it also holds the max-magnitude reduction while the call runs,
+ * so it must not alias another argument.  The work is three launches on
+ * `stream` (reduce max|x|, quantize, finish G).
+ * Errors: as attnqat_quantize, plus EINVAL for a null or misaligned gscale.
+ */
+int attnqat_quantize_gs(const void *x, int64_t batch, int64_t rows,
+                        int64_t cols, int64_t stride_batch, int64_t stride_row,
+                        int64_t stride_col, uint8_t *codes, uint8_t *scales,
+                        void *deq, float *gscale, void *stream);
+
+/*
  * attnqat_workspace_size -- bytes of device workspace attnqat_fwd and
  * attnqat_bwd need for this shape and flag set (0 for invalid shapes).  The
  * workspace holds the dequantized fq(Q), fq(K), fq(V) operands (fp16 when

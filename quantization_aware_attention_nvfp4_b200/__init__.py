@@ -77,6 +77,8 @@ def load(build_if_needed: bool = True):
             lib.attnqat_profile_read.argtypes = [P, P, I]
             lib.attnqat_quantize.restype = I
             lib.attnqat_quantize.argtypes = [P, I64, I64, I64, I64, I64, I64, P, P, P, P]
+            lib.attnqat_quantize_gs.restype = I
+            lib.attnqat_quantize_gs.argtypes = [P, I64, I64, I64, I64, I64, I64, P, P, P, P, P]
             lib.attnqat_workspace_size.restype = SZ
             lib.attnqat_workspace_size.argtypes = [I, I, I, I, I, U32]
             lib.attnqat_fwd.restype = I
@@ -146,6 +148,36 @@ def attnqat_quantize(x, stream=None):
     if x.dim() == 2:
         codes, scales = codes[0], scales[0]
     return codes, scales, deq
+
+
+def attnqat_quantize_gs(x, stream=None):
+    """NVFP4 with an FP32 global scale (G = 2688 / max|x|) of a 2-D (or 3-D
+    batched) bf16 CUDA view, blocks of 16 along the last axis.
+
+    Returns ``(codes uint8 [..., cols/2], scales uint8 [..., cols/16],
+    deq bf16 with x's shape and strides, gscale float32 CUDA tensor [1])``."""
+    torch = _torch()
+    _require_bf16_cuda("x", x)
+    if x.dim() == 2:
+        batch, (rows, cols) = 1, x.shape
+        sb, (sr, sc) = 0, x.stride()
+    elif x.dim() == 3:
+        batch, rows, cols = x.shape
+        sb, sr, sc = x.stride()
+    else:
+        raise ValueError("x must be 2-D or 3-D")
+    codes = torch.empty((batch, rows, cols // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((batch, rows, cols // 16), dtype=torch.uint8, device=x.device)
+    deq = torch.empty_strided(x.shape, x.stride(), dtype=torch.bfloat16, device=x.device)
+    gscale = torch.empty(1, dtype=torch.float32, device=x.device)
+    st = load().attnqat_quantize_gs(ctypes.c_void_p(x.data_ptr()), batch, rows, cols, sb, sr, sc,
+                                    ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                                    ctypes.c_void_p(deq.data_ptr()), ctypes.c_void_p(gscale.data_ptr()),
+                                    _stream_ptr(stream))
+    _check(st, "attnqat_quantize_gs")
+    if x.dim() == 2:
+        codes, scales = codes[0], scales[0]
+    return codes, scales, deq, gscale
 
 
 def attnqat_workspace_size(B, H, Lq, Lk, D, flags=QUANT_ALL) -> int:

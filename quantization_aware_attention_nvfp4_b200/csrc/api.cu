@@ -396,6 +396,25 @@ int attnqat_quantize(const void *x, int64_t batch, int64_t rows, int64_t cols, i
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }
 
+int attnqat_quantize_gs(const void *x, int64_t batch, int64_t rows, int64_t cols, int64_t stride_batch,
+                        int64_t stride_row, int64_t stride_col, uint8_t *codes, uint8_t *scales, void *deq,
+                        float *gscale, void *stream) {
+  if (!x || !codes || !scales || !gscale) return ATTNQAT_EINVAL;
+  if (batch < 1 || rows < 1 || cols < 16 || (cols % 16) != 0) return ATTNQAT_EINVAL;
+  if (stride_batch < 0 || stride_row < 0 || stride_col < 0) return ATTNQAT_EINVAL;
+  const int64_t lim = int64_t(1) << 40;
+  if (batch > lim || rows > lim || cols > lim || batch * rows > lim / cols) return ATTNQAT_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) & 1u) || (deq && (reinterpret_cast<uintptr_t>(deq) & 1u)) ||
+      (reinterpret_cast<uintptr_t>(gscale) & 3u))
+    return ATTNQAT_EINVAL;
+  const int st = check_device();
+  if (st != ATTNQAT_OK) return st;
+  cudaError_t e = launch_quantize_gs(static_cast<const uint16_t *>(x), batch, rows, cols, stride_batch, stride_row,
+                                     stride_col, codes, scales, static_cast<uint16_t *>(deq), gscale,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
+}
+
 size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
   if (check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
   return layout(B, H, Lq, Lk, D, flags).total;

@@ -75,6 +75,13 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
                             uint16_t *deq, uint16_t *deq_f16, float *absmax, cudaStream_t stream,
                             int64_t sf_tile_rows = 0, bool sf_col_tiles = false);
 
+// NVFP4 with an FP32 global scale (see attnqat_quantize_gs): codes and
+// scales as launch_quantize, deq (bf16 bits, may be null), and *gscale
+// (also the scratch of the max-magnitude reduction).
+cudaError_t launch_quantize_gs(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols, int64_t sb,
+                               int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales, uint16_t *deq,
+                               float *gscale, cudaStream_t stream);
+
 // delta[r] = sum_d dO[r][d] * O[r][d] over `rows` rows of D values (O float32,
 // dO bf16); folds max_r |dO_r|_1 into stats[0], max_r |delta_r| into
 // stats[1] and max |dO| into stats[3] (all must start at 0).

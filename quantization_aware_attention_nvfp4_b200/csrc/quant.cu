@@ -214,6 +214,190 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
   return cudaGetLastError();
 }
 
+// --------------------------------------------- NVFP4 with a global scale --
+//
+// The linear-layer variant of the format (vsqa-test-1.3b metadata.json,
+// "linear_quantization": FP8 E4M3 block scales under an FP32 global scale,
+// the activation scale "dynamic, 448*6/max|X| recomputed every forward"):
+//   G   = float32 2688 / max|x| (1 for an all-zero input, the largest finite
+//         float32 if the quotient overflows);
+//   k_b = E4M3 round-to-nearest-even (saturating) of a_b G / 6;
+//   c   = E2M1 round-to-nearest-even (saturating) of |x| G / s_b;
+//   deq = sign * E2M1(c) * s_b / G rounded once to bf16 (nearest, ties even).
+// a_b G and |x| G are exact in float64 (8- and 24-bit significands), so every
+// rounding decision is an exact float64 comparison with a midpoint.
+
+// max |x| over a strided view, folded into *out (which starts at 0) with an
+// atomic max on the float bits.
+template <bool ROW_FASTEST>
+__global__ void __launch_bounds__(256)
+    view_absmax_kernel(const uint16_t *__restrict__ x, int64_t batch, int64_t rows, int64_t cols, int64_t sb,
+                       int64_t sr, int64_t sc, float *out) {
+  const int64_t nblk = cols / 16;
+  const int64_t total = batch * rows * nblk;
+  float vmax = 0.0f;
+  for (int64_t id = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; id < total;
+       id += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t z, r, b;
+    if (ROW_FASTEST) {
+      r = id % rows;
+      const int64_t t = id / rows;
+      b = t % nblk;
+      z = t / nblk;
+    } else {
+      b = id % nblk;
+      const int64_t t = id / nblk;
+      r = t % rows;
+      z = t / rows;
+    }
+    const int64_t base = z * sb + r * sr + b * 16 * sc;
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i)
+      vmax = fmaxf(vmax, fabsf(__uint_as_float(static_cast<uint32_t>(__ldg(x + base + i * sc)) << 16)));
+  }
+  block_max_to_global(vmax, out);
+}
+
+// The float32 global scale from the tensor's max magnitude.
+__device__ __forceinline__ float global_scale_of(float amax) {
+  if (!(amax > 0.0f)) return 1.0f;
+  const float g = __fdiv_rn(2688.0f, amax);
+  return isinf(g) ? 3.40282347e38f : g;
+}
+
+// Value of E4M3 code k (0..126) in float64.
+__device__ __forceinline__ double e4m3_value_f64(int k) {
+  const int e = k >> 3, m = k & 7;
+  return e == 0 ? ldexp(static_cast<double>(m), -9) : ldexp(static_cast<double>(8 + m), e - 10);
+}
+
+// E4M3 code nearest to a / 6 (a >= 0 exact), ties to the even code,
+// saturating at 448: a float32 conversion gives a candidate within one code,
+// exact midpoint comparisons settle it.
+__device__ __forceinline__ int e4m3_round_div6_exact(double a) {
+  int k = static_cast<int>(cvt_e4m3x2(static_cast<float>(a / 6.0), 0.0f) & 0x7Fu);
+  if (k > 126) k = 126;
+  const double a2 = 2.0 * a;
+  while (k > 0) {
+    const double m2 = 6.0 * (e4m3_value_f64(k - 1) + e4m3_value_f64(k));
+    if (a2 < m2 || (a2 == m2 && (k & 1))) --k;
+    else break;
+  }
+  while (k < 126) {
+    const double m2 = 6.0 * (e4m3_value_f64(k) + e4m3_value_f64(k + 1));
+    if (a2 > m2 || (a2 == m2 && (k & 1))) ++k;
+    else break;
+  }
+  return k;
+}
+
+__device__ __forceinline__ double bf16_bits_f64(uint32_t h) { return static_cast<double>(__uint_as_float(h << 16)); }
+
+// bf16 bits of the exact n / g (n >= 0, g > 0; products below are exact in
+// float64), round to nearest, ties to the even pattern: a candidate from
+// n * (1/g), then a walk over neighbouring bf16 patterns and one exact
+// midpoint comparison.
+__device__ __forceinline__ uint32_t bf16_of_quotient_exact(double n, double g, double ginv) {
+  if (n == 0.0) return 0u;
+  uint32_t h = __float_as_uint(static_cast<float>(n * ginv)) >> 16;
+  while (h > 0 && bf16_bits_f64(h) * g > n) --h;
+  while (bf16_bits_f64(h + 1) * g <= n) ++h;
+  const double mid = 0.5 * (bf16_bits_f64(h) + bf16_bits_f64(h + 1));
+  if (n < mid * g) return h;
+  if (n > mid * g) return h + 1;
+  return (h & 1u) ? h + 1 : h;
+}
+
+template <bool ROW_FASTEST>
+__global__ void __launch_bounds__(256)
+    quantize_gs_kernel(const uint16_t *__restrict__ x, int64_t batch, int64_t rows, int64_t cols, int64_t sb,
+                       int64_t sr, int64_t sc, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                       uint16_t *__restrict__ deq, const float *__restrict__ amax_in) {
+  const int64_t nblk = cols / 16;
+  const int64_t total = batch * rows * nblk;
+  const float gf = global_scale_of(*amax_in);
+  const double g = static_cast<double>(gf), ginv = 1.0 / g;
+  for (int64_t id = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; id < total;
+       id += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t z, r, b;
+    if (ROW_FASTEST) {
+      r = id % rows;
+      const int64_t t = id / rows;
+      b = t % nblk;
+      z = t / nblk;
+    } else {
+      b = id % nblk;
+      const int64_t t = id / nblk;
+      r = t % rows;
+      z = t / rows;
+    }
+    const int64_t base = z * sb + r * sr + b * 16 * sc;
+    uint16_t v[16];
+    float ab = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      v[i] = __ldg(x + base + i * sc);
+      ab = fmaxf(ab, fabsf(__uint_as_float(static_cast<uint32_t>(v[i]) << 16)));
+    }
+    const int k = ab > 0.0f ? e4m3_round_div6_exact(static_cast<double>(ab) * g) : 0;
+    const double s = e4m3_value_f64(k);
+    // midpoints of the E2M1 grid times s (exact): crossing midpoint j needs
+    // '>' for even j and '>=' for odd j (ties to the even code)
+    const double t0 = 0.25 * s, t1 = 0.75 * s, t2 = 1.25 * s, t3 = 1.75 * s, t4 = 2.5 * s, t5 = 3.5 * s,
+                 t6 = 5.0 * s;
+    uint32_t nib[2] = {0u, 0u};
+    uint16_t h[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t sign = static_cast<uint32_t>(v[i]) & 0x8000u;
+      const double y = static_cast<double>(fabsf(__uint_as_float(static_cast<uint32_t>(v[i]) << 16))) * g;
+      uint32_t c = 0;
+      if (s > 0.0)
+        c = (y > t0) + (y >= t1) + (y > t2) + (y >= t3) + (y > t4) + (y >= t5) + (y > t6);
+      nib[i >> 3] |= (c | (sign >> 12)) << (4 * (i & 7));
+      const double mag = (c < 4 ? 0.5 * c : (c < 6 ? c - 2.0 : 2.0 * c - 8.0)) * s;
+      h[i] = static_cast<uint16_t>(bf16_of_quotient_exact(mag, g, ginv) | sign);
+    }
+    const int64_t blk = (z * rows + r) * nblk + b;
+    *reinterpret_cast<uint2 *>(codes + blk * 8) = make_uint2(nib[0], nib[1]);
+    scales[blk] = static_cast<uint8_t>(k);
+    if (deq) store16(deq, base, sc, h);
+  }
+}
+
+// Turns the reduced max magnitude in *g into the global scale.
+__global__ void global_scale_finish_kernel(float *g) { *g = global_scale_of(*g); }
+
+cudaError_t launch_quantize_gs(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols, int64_t sb,
+                               int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales, uint16_t *deq,
+                               float *gscale, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(gscale, 0, sizeof(float), stream);
+  if (e != cudaSuccess) return e;
+  const int64_t total = batch * rows * (cols / 16);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const bool row_fastest = (sc != 1) && (sr == 1);
+  if (row_fastest) {
+    view_absmax_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, batch, rows, cols, sb, sr,
+                                                                                     sc, gscale);
+    quantize_gs_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, gscale);
+  } else {
+    view_absmax_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, batch, rows, cols, sb,
+                                                                                      sr, sc, gscale);
+    quantize_gs_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        x, batch, rows, cols, sb, sr, sc, codes, scales, deq, gscale);
+  }
+  global_scale_finish_kernel<<<1, 1, 0, stream>>>(gscale);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ Delta --
 
 // Delta = rowsum(dO o O) with D/8 lanes per row (each lane reads 8 float32

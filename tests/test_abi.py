@@ -138,3 +138,15 @@ def test_python_binding_refuses_cpu_tensors():
     x = torch.zeros((1, 1, 16, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         A.attnqat_fwd(x, x, x)
+
+
+def test_quantize_gs_host_validation():
+    lib = A.load()
+
+    def quant(x=FAKE, cols=32, codes=FAKE, g=FAKE):
+        return lib.attnqat_quantize_gs(P(x), 1, 4, cols, 0, cols, 1, P(codes), P(FAKE), None, P(g), None)
+    assert quant(g=0) == A.EINVAL
+    assert quant(g=FAKE + 2) == A.EINVAL     # float32 slot misaligned
+    assert quant(x=0) == A.EINVAL
+    assert quant(codes=0) == A.EINVAL
+    assert quant(cols=24) == A.EINVAL

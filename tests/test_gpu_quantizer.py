@@ -101,3 +101,61 @@ def test_rejects_bad_arguments():
     with pytest.raises(A.AttnQatError) as e:
         A.attnqat_quantize(x)
     assert e.value.status == A.EINVAL
+
+
+# ------------------------------------------ NVFP4 with an FP32 global scale ----
+
+def _check_gs(bits, batch, rows, cols, sb, sr, sc, view):
+    """GPU global-scale quantizer vs the oracle on one strided view."""
+    import quantization_aware_attention_nvfp4_b200 as A
+    codes, scales, deq, g = A.attnqat_quantize_gs(view)
+    # the oracle quantizes each batch slice of the same view; G is global, so
+    # fold the batch into rows: rows of every slice share one max
+    flat_rows = []
+    for z in range(batch):
+        for r in range(rows):
+            flat_rows.append(bits.reshape(-1)[z * sb + r * sr + np.arange(cols) * sc])
+    flat = np.stack(flat_rows).astype(np.uint16)
+    c_ref, s_ref, d_ref, g_ref = oracle.quantize_rows_gs(flat, batch * rows, cols, cols, 1)
+    assert np.float32(g.item()) == np.float32(g_ref)
+    assert np.array_equal(scales.cpu().numpy().reshape(batch * rows, -1), s_ref)
+    assert np.array_equal(codes.cpu().numpy().reshape(batch * rows, -1), c_ref)
+    # bf16_bits makes deq contiguous in the view's logical order [batch, rows, cols]
+    assert np.array_equal(bf16_bits(deq).reshape(batch * rows, cols), d_ref)
+
+
+@pytest.mark.parametrize("mag", [1.0, 1e-6, 3e3, 1e-30, 0.0])
+def test_global_scale_rows(mag):
+    """Random rows across magnitudes (a huge G for tiny tensors, G = 1 for an
+    all-zero one), plus a block far below the tensor max."""
+    rng = np.random.default_rng(int(abs(np.log10(mag))) if mag else 5)
+    x = rng.standard_normal((96, 128)).astype(np.float32) * np.float32(mag)
+    x[7, :16] *= np.float32(1e-4)
+    bits = W.f32_to_bf16_bits(x)
+    _check_gs(bits, 1, 96, 128, 0, 128, 1, to_gpu_bf16(bits))
+
+
+def test_global_scale_g_one_and_overflow():
+    """max|x| = 2688 (G = 1: the plain format) and a max below 2688 / FLT_MAX
+    (G saturates to the largest finite float32)."""
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((32, 64)) * 200).astype(np.float32)
+    x[3, 9] = -2688.0
+    bits = W.f32_to_bf16_bits(x)
+    _check_gs(bits, 1, 32, 64, 0, 64, 1, to_gpu_bf16(bits))
+    tiny = np.zeros((4, 32), np.uint16)
+    tiny[1, 5] = 3      # subnormal bf16 values only
+    tiny[2, 17] = 0x8001
+    _check_gs(tiny, 1, 4, 32, 0, 32, 1, to_gpu_bf16(tiny))
+
+
+def test_global_scale_batched_transposed_view():
+    """V-like view: per head, channels as rows and tokens as columns (blocks
+    of 16 tokens), one global scale over all heads."""
+    rng = np.random.default_rng(13)
+    BH, L, D = 3, 96, 64
+    x = rng.standard_normal((BH, L, D)).astype(np.float32)
+    bits = W.f32_to_bf16_bits(x).reshape(BH, L, D)
+    t = to_gpu_bf16(bits)
+    view = t.transpose(-1, -2)  # [BH, D, L] with strides (L*D, 1, D)
+    _check_gs(bits, BH, D, L, L * D, 1, D, view)
