@@ -143,18 +143,6 @@ __device__ __forceinline__ void mma_mn_mn(uint32_t d_tmem, uint64_t adesc, uint6
   }
 }
 
-// Writes 128 16-bit values (64 packed words, element 2i in the low half of
-// w[i]) as row `row` of a 128 x 128 swizzled tile at `base` (two chunks of 64
-// elements).  Conflict-free when the 32 lanes of a warp write 32 consecutive
-// rows.
-__device__ __forceinline__ void store_row128(uint32_t base, uint32_t row, const uint32_t *w) {
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const uint32_t addr = base + static_cast<uint32_t>(u >> 3) * kChunkBytes + sw128_offset(row, u & 7);
-    st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-  }
-}
-
 // Writes 64 16-bit values (32 packed words) as columns [64*half, 64*half+64)
 // of row `row` of a 128 x 128 swizzled tile at `base` (exactly one chunk).
 __device__ __forceinline__ void store_row_half(uint32_t base, uint32_t row, int half, const uint32_t *w) {

@@ -82,17 +82,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
-// mbar_wait for a whole warp: lane 0 polls, the verdict is broadcast, and
-// __syncwarp orders lane 0's acquire before the other lanes' later reads.
-// Must be called by all 32 lanes.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort);
-  ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-  __syncwarp();
-  return ok;
-}
-
 // Like mbar_wait but only bounded by time (used when draining in-flight
 // copies after an abort).
 __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {

@@ -5,7 +5,10 @@
 //               sweep and K, fq(V) tiles for the output sweep.  With Q and K
 //               quantized these are the packed NVFP4 codes plus their scale
 //               tiles (8-stage K ring) and S is a block-scaled NVFP4 MMA;
-//               otherwise bf16 tiles; fq(V) in a 2-stage ring, 128-byte swizzle;
+//               otherwise bf16 tiles.  fq(V): with every quantizer on (D =
+//               128, Lk % 32 == 0) its packed codes and scale tiles (4-stage
+//               ring) for a block-scaled NVFP4 P V, else fp16/bf16 tiles
+//               (2-stage ring, 128-byte swizzle);
 //   warps 1, 10 tcgen05.mma issuers (one thread each; warp 1 owns TMEM): A
 //               issues even row-max tiles and the output sweep's S, B the odd
 //               row-max tiles and P V (one thread alone cannot issue fast
@@ -13,7 +16,8 @@
 //   warps 2..9  row warps, two per TMEM lane quarter: each query row (TMEM
 //               lane) has two threads owning 64 columns each -- row max, exp,
 //               row sum, in-register NVFP4 fq of P~ in 16-key blocks, the P
-//               tile to shared memory, and the O epilogue; the pair merges its
+//               tile (packed codes and scale bytes, or 16-bit values) to
+//               shared memory, and the O epilogue; the pair merges its
 //               partial max and sum through shared memory.
 //   warp 11     idle (pads the CTA to whole groups of four warps).
 // TMEM columns: S buffers [0,256) (plus [256,384) during the row-max sweep,
