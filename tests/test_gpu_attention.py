@@ -162,3 +162,13 @@ def test_workload_scaled_heads_16384_sampled(flags):
 def test_workload_large_40h_75600_sampled():
     w = W.get("large_40h_75600")
     _sampled_compare(w, oracle.QUANT_ALL, heads=[(0, 17)], n_rows=32, n_blocks=40)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("Lq,Lk", [(4160, 12352), (9000, 2080)])
+def test_cross_attention_lengths_sampled(Lq, Lk):
+    """Lq != Lk at scale (K and V share Lk), both orders, with ragged last
+    query and key tiles; Lk % 32 == 0, so the forward's P V runs on the
+    NVFP4 path with a partial last key tile."""
+    w = W.custom(1, 4, Lq, Lk, 128, seed_index=700 + Lq % 97)
+    _sampled_compare(w, oracle.QUANT_ALL, heads=[(0, 0), (0, 3)], tag=" Lq%d Lk%d" % (Lq, Lk))
