@@ -5,7 +5,8 @@ One step = attnqat_fwd + attnqat_bwd over one batch of the pages' shape:
 B=1, H=6, Lq=Lk=31200, D=128, bf16, all four quantizers on, sm_scale=1/sqrt(128)
 (the 6-head, 31200-token shape the fastvideo-kernel commit times).  The step
 runs every kernel of the path: the three operand quantizers, the forward, the
-Delta kernel, the dK/dV kernel and the dQ kernel.
+Delta kernel, the kernel writing the exact fp16 copy of dO, the dK/dV kernel
+and the dQ kernel.
 
 Metric: nominal TFLOP/s of fwd+bwd (forward 4*B*H*Lq*Lk*D, backward 2.5x that),
 also reported as fwd / bwd / fwd+bwd milliseconds and as a fraction of the
