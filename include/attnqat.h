@@ -185,10 +185,12 @@ size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D,
  * float32 (the exact row max of the scaled scores).  ws/ws_bytes: device
  * workspace of at least attnqat_workspace_size(B,H,Lq,Lk,D,flags) bytes,
  * 256-byte aligned; it must be passed unchanged to attnqat_bwd.
- * Shapes: B, H >= 1; Lq >= 1; Lk >= 16 with Lk % 16 == 0 (the pages' SM100
- * backward needs a 16-aligned KV length); D in {64, 128}; B*H*max(Lq,Lk)*D
+ * Shapes: B, H >= 1; Lq >= 1; Lk >= 1; D in {64, 128}; B*H*max(Lq,Lk)*D
  * below 2^31.  Lq is arbitrary (the last query tile is masked); a partial
- * last KV tile runs the separate masked tail step.
+ * last KV tile runs the separate masked tail step.  Lk need not be 16-aligned
+ * (the pages' SM100 backward requires it; here a ragged last block of 16 keys
+ * or tokens is zero-padded: its missing keys get P~ = 0 and its missing V
+ * tokens count as zeros in their fq(V) block).
  * Errors: EINVAL, EUNSUPPORTED (not sm_100, D unsupported), ENOSPC, ECUDA.
  */
 int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H,

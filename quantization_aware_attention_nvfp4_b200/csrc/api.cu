@@ -251,7 +251,7 @@ static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static int check_shape(int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags) {
-  if (B < 1 || H < 1 || Lq < 1 || Lk < 16 || (Lk % 16) != 0) return ATTNQAT_EINVAL;
+  if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return ATTNQAT_EINVAL;
   if (static_cast<int64_t>(B) * H > 65535) return ATTNQAT_EINVAL;  // grid.y
   const int64_t Lmax = Lq > Lk ? Lq : Lk;
   if (static_cast<int64_t>(B) * H * Lmax * 128 >= (int64_t(1) << 40)) return ATTNQAT_EINVAL;

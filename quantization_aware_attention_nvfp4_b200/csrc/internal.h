@@ -62,7 +62,8 @@ cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq
                           const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4,
                           const BwdArgs &a, int BH, cudaStream_t stream);
 
-// NVFP4 fq of a strided bf16 view (see attnqat_quantize); any of codes,
+// NVFP4 fq of a strided bf16 view (see attnqat_quantize; cols need not be a
+// multiple of 16 here: a ragged last block reads zeros); any of codes,
 // scales, deq (bf16, same strides as x), deq_f16 and absmax (max |fq(x)|,
 // folded in with an atomic max; must start at 0) may be null.  With
 // sf_tile_rows = L > 0 (contiguous [heads*L, cols] rows), the scales go to

@@ -92,10 +92,11 @@ __device__ __forceinline__ void block_max_to_global(float v, float *dst) {
   }
 }
 
-// Stores 16 16-bit values at dst[base + i*sc] (two 16-byte stores when
-// contiguous and aligned).
-__device__ __forceinline__ void store16(uint16_t *dst, int64_t base, int64_t sc, const uint16_t (&h)[16]) {
-  if (sc == 1 && (reinterpret_cast<uintptr_t>(dst + base) & 15u) == 0) {
+// Stores the first n (<= 16) of 16 16-bit values at dst[base + i*sc] (two
+// 16-byte stores when all 16 are stored, contiguous and aligned).
+__device__ __forceinline__ void store16(uint16_t *dst, int64_t base, int64_t sc, const uint16_t (&h)[16],
+                                        int n = 16) {
+  if (n == 16 && sc == 1 && (reinterpret_cast<uintptr_t>(dst + base) & 15u) == 0) {
     uint32_t w[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) w[i] = h[2 * i] | (static_cast<uint32_t>(h[2 * i + 1]) << 16);
@@ -104,7 +105,8 @@ __device__ __forceinline__ void store16(uint16_t *dst, int64_t base, int64_t sc,
     p[1] = make_uint4(w[4], w[5], w[6], w[7]);
   } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) dst[base + i * sc] = h[i];
+    for (int i = 0; i < 16; ++i)
+      if (i < n) dst[base + i * sc] = h[i];
   }
 }
 
@@ -119,7 +121,9 @@ __global__ void __launch_bounds__(256)
                          uint8_t *__restrict__ scales, uint16_t *__restrict__ deq,
                          uint16_t *__restrict__ deq_f16, float *__restrict__ absmax, int64_t sf_tile_rows,
                          bool sf_col_tiles) {
-  const int64_t nblk = cols / 16;
+  // a ragged last block along cols (only the attention's V view, cols = Lk)
+  // reads its missing elements as zeros, which leave its amax unchanged
+  const int64_t nblk = (cols + 15) / 16;
   float vmax = 0.0f;  // largest dequantized magnitude this thread produced
   const int64_t total = batch * rows * nblk;
   for (int64_t id = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; id < total;
@@ -137,8 +141,9 @@ __global__ void __launch_bounds__(256)
       z = t / rows;
     }
     const int64_t base = z * sb + r * sr + b * 16 * sc;
+    const int n = static_cast<int>(cols - b * 16 < 16 ? cols - b * 16 : 16);
     uint16_t v[16];
-    const bool vec = (sc == 1) && ((reinterpret_cast<uintptr_t>(x + base) & 15u) == 0);
+    const bool vec = n == 16 && (sc == 1) && ((reinterpret_cast<uintptr_t>(x + base) & 15u) == 0);
     if (vec) {
       const uint4 *p = reinterpret_cast<const uint4 *>(x + base);
       const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
@@ -150,7 +155,7 @@ __global__ void __launch_bounds__(256)
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = __ldg(x + base + i * sc);
+      for (int i = 0; i < 16; ++i) v[i] = i < n ? __ldg(x + base + i * sc) : static_cast<uint16_t>(0);
     }
     uint32_t nib[2], scode;
     uint16_t bb[16], hb[16];
@@ -181,8 +186,8 @@ __global__ void __launch_bounds__(256)
         scales[blk] = static_cast<uint8_t>(scode);
       }
     }
-    if (deq) store16(deq, base, sc, bb);
-    if (deq_f16) store16(deq_f16, base, sc, hb);
+    if (deq) store16(deq, base, sc, bb, n);
+    if (deq_f16) store16(deq_f16, base, sc, hb, n);
     if (absmax) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) vmax = fmaxf(vmax, fabsf(__uint_as_float(static_cast<uint32_t>(bb[i]) << 16)));
@@ -195,7 +200,7 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
                             int64_t sr, int64_t sc, uint8_t *codes, uint8_t *scales, uint16_t *deq,
                             uint16_t *deq_f16, float *absmax, cudaStream_t stream, int64_t sf_tile_rows,
                             bool sf_col_tiles) {
-  const int64_t total = batch * rows * (cols / 16);
+  const int64_t total = batch * rows * ((cols + 15) / 16);
   if (total == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -54,6 +54,7 @@ def test_flag_combinations(flags):
 
 
 @pytest.mark.parametrize("Lq,Lk,D", [(200, 336, 128), (200, 352, 128), (200, 336, 64), (1, 16, 128), (129, 16, 64),
+                                    (200, 100, 128), (130, 1000, 64), (64, 7, 128), (33, 1, 128),
                                      (300, 128, 128), (192, 1040, 128)])
 def test_ragged_and_edge_shapes(Lq, Lk, D):
     """Several tiles with ragged query and key tails, a single key block,
