@@ -16,6 +16,11 @@ citations and the readings taken where the pages are silent):
   O = fq(P~) fq(V) / l; LSE = m + ln l.
 * backward (straight-through): dV = (fq(P~)/l)^T dO; dS = P o (dO fq(V)^T -
   rowsum(dO o O)); dQ = dS fq(K) c; dK = dS^T fq(Q) c.
+* block-sparse fine attention (vsqa-test-1.3b metadata.json, "attention":
+  VSA_QAT_TRAIN_C128, 128-token cubes, selected key blocks per query block):
+  the same computation restricted, per query tile, to the keys of the
+  selected key tiles (``sel`` [n_query_tiles, n_key_tiles], nonzero =
+  selected); a row with no selected key gives O = 0, LSE = m = -inf, dQ = 0.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against brute force, closed forms, torch's own float8 conversion and finite
@@ -88,15 +93,15 @@ def _load():
             lib.oracle_operands.argtypes = [P, P, P, L, L, L, ctypes.c_uint, P, P, P]
             lib.oracle_fwd_rows.restype = None
             lib.oracle_fwd_rows.argtypes = [P, P, P, L, L, L, ctypes.c_double,
-                                            ctypes.c_uint, P, L, P, P, P, P]
+                                            ctypes.c_uint, P, L, P, L, P, P, P, P]
             lib.oracle_delta.restype = None
             lib.oracle_delta.argtypes = [P, P, L, L, P]
             lib.oracle_bwd_dq_rows.restype = None
             lib.oracle_bwd_dq_rows.argtypes = [P, P, P, P, L, L, L, ctypes.c_double,
-                                               ctypes.c_uint, P, P, P, P, L, P]
+                                               ctypes.c_uint, P, L, P, P, P, P, L, P]
             lib.oracle_bwd_dkdv_blocks.restype = None
             lib.oracle_bwd_dkdv_blocks.argtypes = [P, P, P, P, L, L, L, ctypes.c_double,
-                                                   ctypes.c_uint, P, P, P, P, L, P, P]
+                                                   ctypes.c_uint, P, L, P, P, P, P, L, P, P]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -207,9 +212,13 @@ def fq_f64_rows(x: np.ndarray):
 # -------------------------------------------------------------- attention --
 
 class Head:
-    """The fq'd float64 operands of one (b, h) head plus its dO."""
+    """The fq'd float64 operands of one (b, h) head plus its dO.
 
-    def __init__(self, q_bits, k_bits, v_bits, sm_scale, flags, do_bits=None):
+    ``sel`` (optional, uint8 [ceil(Lq/tile), ceil(Lk/tile)]) restricts each
+    query tile to the keys of its selected key tiles (block-sparse fine
+    attention); ``tile`` is the tile length in tokens, a multiple of 16."""
+
+    def __init__(self, q_bits, k_bits, v_bits, sm_scale, flags, do_bits=None, sel=None, tile=128):
         q = _bits(q_bits)
         k = _bits(k_bits)
         v = _bits(v_bits)
@@ -217,6 +226,15 @@ class Head:
         self.Lk = k.shape[0]
         if v.shape != k.shape or k.shape[1] != self.D:
             raise ValueError("q [Lq,D], k and v [Lk,D] expected")
+        if tile < 16 or tile % 16:
+            raise ValueError("tile must be a positive multiple of 16")
+        self.tile = int(tile)
+        if sel is not None:
+            sel = np.ascontiguousarray(sel, dtype=np.uint8)
+            want = (-(-self.Lq // self.tile), -(-self.Lk // self.tile))
+            if sel.shape != want:
+                raise ValueError("sel must be [%d, %d]" % want)
+        self.sel = sel
         self.c = float(sm_scale)
         self.flags = int(flags)
         self.Qh = np.zeros((self.Lq, self.D))
@@ -226,6 +244,9 @@ class Head:
                                 self.flags, _ptr(self.Qh), _ptr(self.Kh), _ptr(self.Vh))
         self.dO = None if do_bits is None else _bits(do_bits)
         self._stats = None
+
+    def _sel_ptr(self):
+        return None if self.sel is None else _ptr(self.sel)
 
     # forward -------------------------------------------------------------
     def fwd_rows(self, rows=None):
@@ -238,8 +259,8 @@ class Head:
         m = np.zeros(n)
         l = np.zeros(n)
         _load().oracle_fwd_rows(_ptr(self.Qh), _ptr(self.Kh), _ptr(self.Vh), self.Lq,
-                                self.Lk, self.D, self.c, self.flags, _ptr(rows), n,
-                                _ptr(O), _ptr(lse), _ptr(m), _ptr(l))
+                                self.Lk, self.D, self.c, self.flags, self._sel_ptr(), self.tile,
+                                _ptr(rows), n, _ptr(O), _ptr(lse), _ptr(m), _ptr(l))
         return O, lse, m, l
 
     def stats(self):
@@ -261,7 +282,7 @@ class Head:
         dQ = np.zeros((n, self.D))
         _load().oracle_bwd_dq_rows(_ptr(self.Qh), _ptr(self.Kh), _ptr(self.Vh),
                                    _ptr(self.dO), self.Lq, self.Lk, self.D, self.c,
-                                   self.flags, _ptr(st["m"]), _ptr(st["l"]),
+                                   self.flags, self._sel_ptr(), self.tile, _ptr(st["m"]), _ptr(st["l"]),
                                    _ptr(st["delta"]), _ptr(rows), n, _ptr(dQ))
         return dQ
 
@@ -277,7 +298,8 @@ class Head:
         dV = np.zeros((n * 16, self.D))
         _load().oracle_bwd_dkdv_blocks(_ptr(self.Qh), _ptr(self.Kh), _ptr(self.Vh),
                                        _ptr(self.dO), self.Lq, self.Lk, self.D, self.c,
-                                       self.flags, _ptr(st["m"]), _ptr(st["l"]),
+                                       self.flags, self._sel_ptr(), self.tile, _ptr(st["m"]),
+                                       _ptr(st["l"]),
                                        _ptr(st["delta"]), _ptr(blocks), n, _ptr(dK),
                                        _ptr(dV))
         return dK, dV
@@ -289,8 +311,9 @@ class Head:
         return dQ, dK[: self.Lk], dV[: self.Lk]
 
 
-def attention(q_bits, k_bits, v_bits, sm_scale, flags=QUANT_ALL, do_bits=None):
-    """Full forward (and backward when dO is given) over [B, H, L, D] inputs.
+def attention(q_bits, k_bits, v_bits, sm_scale, flags=QUANT_ALL, do_bits=None, sel=None, tile=128):
+    """Full forward (and backward when dO is given) over [B, H, L, D] inputs;
+    ``sel`` [B, H, n_query_tiles, n_key_tiles] makes it block-sparse.
 
     Returns a dict of float64 arrays: O, lse, m (and dQ, dK, dV)."""
     q = _bits(q_bits)
@@ -306,7 +329,8 @@ def attention(q_bits, k_bits, v_bits, sm_scale, flags=QUANT_ALL, do_bits=None):
     for b in range(B):
         for h in range(H):
             hd = Head(q[b, h], k[b, h], v[b, h], sm_scale, flags,
-                      None if do_bits is None else dO[b, h])
+                      None if do_bits is None else dO[b, h],
+                      None if sel is None else sel[b, h], tile)
             st = hd.stats()
             out["O"][b, h] = st["O"]
             out["lse"][b, h] = st["lse"]

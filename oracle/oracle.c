@@ -41,6 +41,20 @@
  *    with zeros (which does not change its amax);
  *  - c multiplies the fp64 dot product, never the operands before fq.
  *
+ * Block-sparse fine attention (vsqa-test-1.3b metadata.json, "attention":
+ * backend VSA_QAT_TRAIN_C128, kind "vsa", cube_shape 4 x 4 x 8 = 128 tokens,
+ * "fine": "NVFP4 fake-quant with BF16 matmul", quantize_fine = true, top-k
+ * "selection" of key blocks per query block): every function that takes
+ * `sel` restricts query i to the keys j whose tiles are selected,
+ * sel[(i / T) * nkt + j / T] != 0 with T-token tiles and nkt = ceil(Lk / T);
+ * sel = NULL is dense attention.  Reading: the fine attention is the same
+ * Attn-QAT computation over the selected keys only -- m is their exact max,
+ * l their sum, and a key outside the selection has P~ = 0 (so it adds zero
+ * to its fq(P~) block, which is all zeros when T is a multiple of 16); fq(Q),
+ * fq(K), fq(V) do not depend on the selection.  A query row with no selected
+ * key has O = 0, l = 0, m = LSE = -infinity, dQ = 0, and adds nothing to
+ * dK, dV.
+ *
  * Every arithmetic step is plain float64; the only reorderings are the ones a
  * sum admits.  Loops are parallelised over independent rows with OpenMP.
  */
@@ -59,6 +73,12 @@
 #define ORACLE_DV_QUANT_NORMALIZED 16u
 
 #define BLOCK 16
+
+/* Does query i attend to key j?  (sel == NULL: dense.) */
+static int selected(const uint8_t *sel, long T, long nkt, long i, long j)
+{
+    return sel == NULL || sel[(i / T) * nkt + j / T] != 0;
+}
 
 /* ------------------------------------------------------------------------ */
 /* Number formats                                                            */
@@ -407,20 +427,23 @@ static void score_row(const double *Qi, const double *Kh, long Lk, long D,
         S[j] = c * dot(Qi, Kh + j * D, D);
 }
 
-/* Probability row of one query: P~_j = exp(S_j - m) and, with QUANT_P, the
- * fq'd P^ in blocks of 16 consecutive keys from key 0.  Returns m and l.    */
-static void prob_row(const double *Qi, const double *Kh, long Lk, long D,
-                     double c, unsigned flags, double *S, double *Pt,
-                     double *Phat, double *m_out, double *l_out)
+/* Probability row of query i: P~_j = exp(S_j - m) over the selected keys
+ * (0 elsewhere) and, with QUANT_P, the fq'd P^ in blocks of 16 consecutive
+ * keys from key 0.  Returns m (-inf with no selected key) and l.           */
+static void prob_row(const double *Qi, long i, const double *Kh, long Lk, long D,
+                     double c, unsigned flags, const uint8_t *sel, long T,
+                     double *S, double *Pt, double *Phat, double *m_out,
+                     double *l_out)
 {
+    long nkt = (Lk + T - 1) / T;
     score_row(Qi, Kh, Lk, D, c, S);
     double m = -INFINITY;
     for (long j = 0; j < Lk; j++)
-        if (S[j] > m)
+        if (selected(sel, T, nkt, i, j) && S[j] > m)
             m = S[j];
     double l = 0.0;
     for (long j = 0; j < Lk; j++) {
-        Pt[j] = exp(S[j] - m);
+        Pt[j] = selected(sel, T, nkt, i, j) ? exp(S[j] - m) : 0.0;
         l += Pt[j];
     }
     if (flags & ORACLE_QUANT_P) {
@@ -440,11 +463,12 @@ static void prob_row(const double *Qi, const double *Kh, long Lk, long D,
 /* ------------------------------------------------------------------------ */
 
 /* Forward for the query rows listed in rows[0..nrows): O (float64, [nrows][D]),
- * LSE, m and l per listed row.  Qh/Kh/Vh come from oracle_operands.         */
+ * LSE, m and l per listed row.  Qh/Kh/Vh come from oracle_operands; sel/T
+ * select key tiles per query tile (NULL: dense).                           */
 void oracle_fwd_rows(const double *Qh, const double *Kh, const double *Vh,
                      long Lq, long Lk, long D, double c, unsigned flags,
-                     const long *rows, long nrows, double *O, double *lse,
-                     double *m, double *l)
+                     const uint8_t *sel, long T, const long *rows, long nrows,
+                     double *O, double *lse, double *m, double *l)
 {
     (void)Lq;
 #pragma omp parallel
@@ -456,16 +480,17 @@ void oracle_fwd_rows(const double *Qh, const double *Kh, const double *Vh,
         for (long t = 0; t < nrows; t++) {
             long i = rows[t];
             double mi, li;
-            prob_row(Qh + i * D, Kh, Lk, D, c, flags, S, Pt, Ph, &mi, &li);
+            prob_row(Qh + i * D, i, Kh, Lk, D, c, flags, sel, T, S, Pt, Ph, &mi,
+                     &li);
             for (long d = 0; d < D; d++) {
                 double acc = 0.0;
                 for (long j = 0; j < Lk; j++)
                     acc += Ph[j] * Vh[j * D + d];
-                O[t * D + d] = acc / li;
+                O[t * D + d] = li > 0.0 ? acc / li : 0.0;
             }
             m[t] = mi;
             l[t] = li;
-            lse[t] = mi + log(li);
+            lse[t] = li > 0.0 ? mi + log(li) : -INFINITY;
         }
         free(S);
         free(Pt);
@@ -493,10 +518,12 @@ void oracle_delta(const double *O, const uint16_t *dO, long L, long D,
  * [nrows][D].                                                              */
 void oracle_bwd_dq_rows(const double *Qh, const double *Kh, const double *Vh,
                         const uint16_t *dO, long Lq, long Lk, long D, double c,
-                        unsigned flags, const double *m, const double *l,
+                        unsigned flags, const uint8_t *sel, long T,
+                        const double *m, const double *l,
                         const double *delta, const long *rows, long nrows,
                         double *dQ)
 {
+    long nkt = (Lk + T - 1) / T;
     (void)Lq;
 #pragma omp parallel
     {
@@ -508,7 +535,8 @@ void oracle_bwd_dq_rows(const double *Qh, const double *Kh, const double *Vh,
         for (long t = 0; t < nrows; t++) {
             long i = rows[t];
             double mi, li;
-            prob_row(Qh + i * D, Kh, Lk, D, c, flags, S, Pt, Ph, &mi, &li);
+            prob_row(Qh + i * D, i, Kh, Lk, D, c, flags, sel, T, S, Pt, Ph, &mi,
+                     &li);
             (void)mi;
             (void)li;
             for (long d = 0; d < D; d++)
@@ -516,6 +544,8 @@ void oracle_bwd_dq_rows(const double *Qh, const double *Kh, const double *Vh,
             for (long d = 0; d < D; d++)
                 dQ[t * D + d] = 0.0;
             for (long j = 0; j < Lk; j++) {
+                if (!(l[i] > 0.0) || !selected(sel, T, nkt, i, j))
+                    continue;
                 double P = exp(S[j] - m[i]) / l[i];
                 double dP = dot(dOi, Vh + j * D, D);
                 double dS = P * (dP - delta[i]);
@@ -537,11 +567,13 @@ void oracle_bwd_dq_rows(const double *Qh, const double *Kh, const double *Vh,
  * float64 [nblocks*16][D]; rows past Lk are left zero.                      */
 void oracle_bwd_dkdv_blocks(const double *Qh, const double *Kh, const double *Vh,
                             const uint16_t *dO, long Lq, long Lk, long D,
-                            double c, unsigned flags, const double *m,
+                            double c, unsigned flags, const uint8_t *sel,
+                            long T, const double *m,
                             const double *l, const double *delta,
                             const long *blocks, long nblocks, double *dK,
                             double *dV)
 {
+    long nkt = (Lk + T - 1) / T;
     memset(dK, 0, sizeof(double) * nblocks * BLOCK * D);
     memset(dV, 0, sizeof(double) * nblocks * BLOCK * D);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -551,11 +583,13 @@ void oracle_bwd_dkdv_blocks(const double *Qh, const double *Kh, const double *Vh
         double S[BLOCK], Pt[BLOCK], Ph[BLOCK], dOi[512];
         double *dKt = dK + t * BLOCK * D, *dVt = dV + t * BLOCK * D;
         for (long i = 0; i < Lq; i++) {
+            if (!(l[i] > 0.0))
+                continue; /* no selected key: the row adds nothing */
             for (long d = 0; d < D; d++)
                 dOi[d] = oracle_bf16_value(dO[i * D + d]);
             for (long jj = 0; jj < n; jj++) {
                 S[jj] = c * dot(Qh + i * D, Kh + (j0 + jj) * D, D);
-                Pt[jj] = exp(S[jj] - m[i]);
+                Pt[jj] = selected(sel, T, nkt, i, j0 + jj) ? exp(S[jj] - m[i]) : 0.0;
             }
             /* w_j: the dV weight of key j in this query row */
             double w[BLOCK];

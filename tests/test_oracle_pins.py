@@ -502,6 +502,89 @@ def test_sampled_rows_equal_full_computation():
     assert np.array_equal(dKs, dK[32:48]) and np.array_equal(dVs, dV[32:48])
 
 
+# ------------------------------------------- block-sparse fine attention ----
+# VSA fine attention (vsqa-test-1.3b metadata.json, "attention": backend
+# VSA_QAT_TRAIN_C128, 128-token cubes, selected key blocks per query block,
+# NVFP4 fake-quant on the fine branch).  The oracle takes the selection as a
+# tile mask; small tiles (multiples of 16) keep these pins fast.
+
+def _sparse_case(seed, Lq, Lk, D, T, p=0.5):
+    rng = np.random.default_rng(seed)
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for L in (Lq, Lk, Lk, Lq))
+    nqt, nkt = -(-Lq // T), -(-Lk // T)
+    sel = (rng.random((nqt, nkt)) < p).astype(np.uint8)
+    return q, k, v, dO, sel
+
+
+def test_sparse_all_tiles_selected_is_dense():
+    q, k, v, dO, _ = _sparse_case(71, 70, 90, 32, 32)
+    sel = np.ones((1, 1, 3, 3), np.uint8)
+    a = oracle.attention(q, k, v, 0.2, oracle.QUANT_ALL, dO, sel=sel, tile=32)
+    b = oracle.attention(q, k, v, 0.2, oracle.QUANT_ALL, dO)
+    for key in b:
+        assert np.array_equal(a[key], b[key]), key
+
+
+@pytest.mark.parametrize("flags", [oracle.QUANT_ALL, 0, oracle.QUANT_V | oracle.QUANT_P])
+def test_sparse_equals_dense_attention_on_the_gathered_tiles(flags):
+    """Each query tile's output and dQ equal dense attention of its rows
+    against the concatenation of its selected key tiles (the oracle's dense
+    path, pinned above); dK, dV equal the sum of those per-tile gradients;
+    a query tile with no selection gives O = 0, LSE = m = -inf, dQ = 0; an
+    unselected key tile gets dK = dV = 0.  Tiles are whole 16-blocks (the
+    ragged last key tile comes last in the gather), so fq(V) and fq(P~) see
+    the same blocks either way."""
+    Lq, Lk, D, T = 100, 150, 32, 32
+    q, k, v, dO, sel = _sparse_case(72 + flags, Lq, Lk, D, T)
+    sel[1, :] = 0          # a query tile with nothing selected
+    sel[:, 2] = 0          # a key tile nobody selects
+    sel[0, 4] = sel[3, 4] = 1  # the ragged last key tile, from the ragged last query tile too
+    sel[2, 0] = 1
+    c = 0.21
+    sp = oracle.attention(q, k, v, c, flags, dO, sel=sel[None, None], tile=T)
+    dK = np.zeros((Lk, D))
+    dV = np.zeros((Lk, D))
+    for I in range(sel.shape[0]):
+        rows = np.arange(I * T, min((I + 1) * T, Lq))
+        js = np.nonzero(sel[I])[0]
+        if js.size == 0:
+            assert np.all(sp["O"][0, 0, rows] == 0) and np.all(sp["dQ"][0, 0, rows] == 0)
+            assert np.all(np.isneginf(sp["lse"][0, 0, rows])) and np.all(np.isneginf(sp["m"][0, 0, rows]))
+            continue
+        keys = np.concatenate([np.arange(J * T, min((J + 1) * T, Lk)) for J in js])
+        hd = oracle.Head(q[0, 0, rows], k[0, 0, keys], v[0, 0, keys], c, flags, dO[0, 0, rows])
+        st = hd.stats()
+        dQg, dKg, dVg = hd.backward()
+        assert np.max(np.abs(sp["O"][0, 0, rows] - st["O"])) <= 1e-12 * np.max(np.abs(st["O"]))
+        assert np.max(np.abs(sp["lse"][0, 0, rows] - st["lse"])) <= 1e-12
+        assert np.array_equal(sp["m"][0, 0, rows], st["m"])
+        assert np.max(np.abs(sp["dQ"][0, 0, rows] - dQg)) <= 1e-11 * np.max(np.abs(dQg))
+        dK[keys] += dKg
+        dV[keys] += dVg
+    assert np.all(sp["dK"][0, 0, 64:96] == 0) and np.all(sp["dV"][0, 0, 64:96] == 0)
+    assert np.max(np.abs(sp["dK"][0, 0] - dK)) <= 1e-11 * np.max(np.abs(dK))
+    assert np.max(np.abs(sp["dV"][0, 0] - dV)) <= 1e-11 * np.max(np.abs(dV))
+
+
+def test_sparse_quantizers_off_vs_torch_masked_sdpa():
+    """Quantizers off: block-sparse attention is softmax attention under the
+    token mask the tile selection expands to (torch's masked SDPA and
+    autograd, float64)."""
+    Lq, Lk, D, T = 80, 112, 16, 16
+    q, k, v, dO, sel = _sparse_case(73, Lq, Lk, D, T, p=0.3)
+    sel[np.arange(sel.shape[0]), np.arange(sel.shape[0]) % sel.shape[1]] = 1  # no empty row
+    c = 0.37
+    mask = np.kron(sel, np.ones((T, T), np.uint8))[:Lq, :Lk].astype(bool)
+    qt, kt, vt = (torch.tensor(_f(x[0, 0]), requires_grad=True) for x in (q, k, v))
+    O = torch.nn.functional.scaled_dot_product_attention(qt[None], kt[None], vt[None],
+                                                         attn_mask=torch.tensor(mask)[None], scale=c)[0]
+    (O * torch.tensor(_f(dO[0, 0]))).sum().backward()
+    sp = oracle.attention(q, k, v, c, 0, dO, sel=sel[None, None], tile=T)
+    for name, ref in (("O", O.detach()), ("dQ", qt.grad), ("dK", kt.grad), ("dV", vt.grad)):
+        ref = ref.numpy()
+        assert np.max(np.abs(sp[name][0, 0] - ref)) <= 1e-10 * max(1.0, np.max(np.abs(ref))), name
+
+
 # ------------------------------------------ NVFP4 with an FP32 global scale ----
 
 def _bf16_value_fraction(h):
