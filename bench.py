@@ -14,7 +14,13 @@ measured B200 BF16 tensor peak.  Inputs are seeded synthetic tensors; L2 is
 flushed (a 256 MiB write) between timed steps, each step is timed with CUDA
 events on the launching stream, and multi-GPU runs report the max over ranks.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sparsity S]
+
+--sparsity S times the block-sparse (VSA fine attention) step instead:
+attnqat_sparse_fwd + attnqat_sparse_bwd on the same shape, each 128-query tile
+attending max(1, min(ceil((1-S)*244), 244)) of the 244 key tiles (seeded
+selection; the pages' VSA checkpoint uses S = 0.9), with TFLOP/s counted on
+the selected tiles only.
 
 --impl reference times the float64 CPU oracle on the host cores instead (the
 pages ship no runnable implementation): each step is a bounded sample of the
@@ -41,6 +47,8 @@ from quantization_aware_attention_nvfp4_b200 import workloads as W  # noqa: E402
 
 WORKLOAD = "wan_6h_31200"
 METRIC = "Attn-QAT fwd+bwd ms & TFLOP/s at H6 L31200 D128; % of B200 BF16 peak"
+SPARSE_METRIC = ("Block-sparse (VSA) Attn-QAT fwd+bwd ms & TFLOP/s on the selected tiles at H6 L31200 D128, "
+                 "sparsity %g")
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 # rows of the oracle's bounded samples (query rows of head 0 against all keys):
@@ -81,7 +89,9 @@ def max_over_ranks(values, device=None):
 
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 50 ms while the
-    timed region runs."""
+    timed region runs.  Entering waits (up to 10 s) for a first sample and
+    leaving waits (up to 2 s) for one more, so even a region shorter than the
+    sampling period is bracketed by a sample on each side."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -92,6 +102,8 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        import threading
+        self.lines = []
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
@@ -99,16 +111,34 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        first = threading.Event()
+
+        def reader():
+            for line in self.proc.stdout:
+                self.lines.append(line)
+                first.set()
+            first.set()
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        first.wait(10.0)
+        del self.lines[:-1]  # keep only the latest sample before the region
         return self
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            n0 = len(self.lines)
+            t0 = time.perf_counter()
+            while len(self.lines) <= n0 and time.perf_counter() - t0 < 2.0 and self.proc.poll() is None:
+                time.sleep(0.01)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=10)
+                self.proc.wait(timeout=10)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self.proc.wait()
+            self.thread.join(timeout=10)
+            self.out = "".join(self.lines)
         return False
 
     def summary(self):
@@ -137,6 +167,14 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- GPU arm --
 
+def selected_pairs(w, mask):
+    """Sum over (b, h) of the (query row, key) pairs the tile mask selects."""
+    T = W.SPARSE_TILE
+    rows = np.minimum(T, w.Lq - T * np.arange(mask.shape[2]))
+    keys = np.minimum(T, w.Lk - T * np.arange(mask.shape[3]))
+    return float(np.einsum("bhij,i,j->", mask.astype(np.float64), rows, keys))
+
+
 def gpu_arm(args):
     import torch
     import torch.distributed as dist
@@ -151,6 +189,13 @@ def gpu_arm(args):
     w = W.get(WORKLOAD)
     flops = w.nominal_flops()
     peaks = load_peaks()
+    sparse = args.sparsity is not None
+    pairs = float(w.B * w.H * w.Lq * w.Lk)
+    if sparse:
+        mask_np = W.tile_mask(w, args.sparsity)
+        pairs = selected_pairs(w, mask_np)
+        fwd_f = 4.0 * pairs * w.D
+        flops = dict(fwd=fwd_f, bwd=2.5 * fwd_f, total=3.5 * fwd_f)
 
     # seeded inputs (host), moved to the device once; the timed region starts
     # with them resident in HBM
@@ -159,7 +204,24 @@ def gpu_arm(args):
     q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
     c = w.sm_scale
     flags = A.QUANT_ALL
-    ws = torch.empty(A.attnqat_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags), dtype=torch.uint8, device=dev)
+    if sparse:
+        tm = torch.from_numpy(mask_np).to(dev)
+        ws_bytes = A.attnqat_sparse_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags)
+
+        def fwd(qq, kk, vv, out):
+            return A.attnqat_sparse_fwd(qq, kk, vv, tm, sm_scale=c, flags=flags, ws=ws, out=out)
+
+        def bwd(qq, kk, vv, ll, mm, dd, out):
+            return A.attnqat_sparse_bwd(qq, kk, vv, ll, mm, dd, ws, tm, sm_scale=c, flags=flags, out=out)
+    else:
+        ws_bytes = A.attnqat_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags)
+
+        def fwd(qq, kk, vv, out):
+            return A.attnqat_fwd(qq, kk, vv, sm_scale=c, flags=flags, ws=ws, out=out)
+
+        def bwd(qq, kk, vv, ll, mm, dd, out):
+            return A.attnqat_bwd(qq, kk, vv, ll, mm, dd, ws, sm_scale=c, flags=flags, out=out)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
     m = torch.empty_like(lse)
@@ -168,8 +230,8 @@ def gpu_arm(args):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        A.attnqat_fwd(q, k, v, sm_scale=c, flags=flags, ws=ws, out=(o, lse, m))
-        A.attnqat_bwd(q, k, v, lse, m, do, ws, sm_scale=c, flags=flags, out=(dq, dk, dv))
+        fwd(q, k, v, (o, lse, m))
+        bwd(q, k, v, lse, m, do, (dq, dk, dv))
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -190,9 +252,9 @@ def gpu_arm(args):
             flush.zero_()
             e0, e1, e2 = ev[i]
             e0.record(stream)
-            A.attnqat_fwd(q, k, v, sm_scale=c, flags=flags, ws=ws, out=(o, lse, m))
+            fwd(q, k, v, (o, lse, m))
             e1.record(stream)
-            A.attnqat_bwd(q, k, v, lse, m, do, ws, sm_scale=c, flags=flags, out=(dq, dk, dv))
+            bwd(q, k, v, lse, m, do, (dq, dk, dv))
             e2.record(stream)
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - wall0
@@ -210,7 +272,7 @@ def gpu_arm(args):
     per = {}
     for name, ms in kernels:
         per.setdefault(name, []).append(ms)
-    units = 2.0 * w.B * w.H * w.Lq * w.Lk * w.D  # one matmul unit
+    units = 2.0 * pairs * w.D  # one matmul unit (over the selected pairs when sparse)
     algo_flops = {"attn_fwd": 2 * units, "attn_bwd_dkdv": 4 * units, "attn_bwd_dq": 1 * units}
     exec_flops = {"attn_fwd": 3 * units, "attn_bwd_dkdv": 4 * units, "attn_bwd_dq": 3 * units}
     tensor_kernels = {n: v for n, v in per.items() if n in algo_flops}
@@ -218,7 +280,7 @@ def gpu_arm(args):
     dom_ms = statistics.mean(per[dom])
     achieved = algo_flops[dom] / (dom_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
-    traffic = load_traffic(dom)
+    traffic = None if sparse else load_traffic(dom)  # the committed ncu counters are for the dense step
     kernel_table = {n: dict(launches=len(v), mean_ms=round(statistics.mean(v), 4),
                             share=round(sum(v) / sum(sum(x) for x in per.values()), 4))
                     for n, v in per.items()}
@@ -228,12 +290,21 @@ def gpu_arm(args):
             kernel_table[n]["executed_tflops"] = round(exec_flops[n] / (kernel_table[n]["mean_ms"] * 1e-3) / 1e12, 1)
 
     # ---- end to end through the public API with host buffers
-    e2e = e2e_arm(args, A, torch, dev, host, w, c, flags, ws, world)
+    e2e = e2e_arm(args, torch, dev, host, w, flops, fwd, bwd, world)
 
     value = world * flops["total"] * args.steps / (tot_ms * 1e-3) / 1e12
     ms_step = tot_ms / args.steps
+    config = {"workload": WORKLOAD, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
+              "quantizers": "q,k,v,p", "sm_scale": "1/sqrt(128)", "global_batch": w.B * world,
+              "seq_len": w.Lq, "parallelism": "replicas x%d (heads independent, no collective)" % world,
+              "l2": "flushed between steps (256 MiB write); each step timed with CUDA events"}
+    if sparse:
+        config.update(workload="vsa_" + WORKLOAD, sparsity=args.sparsity, tile=W.SPARSE_TILE,
+                      key_tiles_per_query_tile=int(mask_np.sum(-1).max()),
+                      selected_fraction=round(pairs / (w.B * w.H * w.Lq * w.Lk), 5),
+                      selection="seeded uniform top-k of key tiles per query tile")
     out = {
-        "metric": METRIC,
+        "metric": SPARSE_METRIC % args.sparsity if sparse else METRIC,
         "value": round(value, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -245,10 +316,7 @@ def gpu_arm(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, recipe in DESIGN.md)",
-        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
-                   "quantizers": "q,k,v,p", "sm_scale": "1/sqrt(128)", "global_batch": w.B * world,
-                   "seq_len": w.Lq, "parallelism": "replicas x%d (heads independent, no collective)" % world,
-                   "l2": "flushed between steps (256 MiB write); each step timed with CUDA events"},
+        "config": config,
         "fwd_ms": round(fwd_ms / args.steps, 4),
         "bwd_ms": round(bwd_ms / args.steps, 4),
         "fwd_tflops": round(flops["fwd"] / (fwd_ms / args.steps * 1e-3) / 1e12, 1),
@@ -273,14 +341,15 @@ def gpu_arm(args):
     }
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline_sample(rows=BASELINE_SAMPLE_ROWS)
+            out["cpu_baseline"] = cpu_baseline_sample(rows=BASELINE_SAMPLE_ROWS,
+                                                      sel=mask_np[0, 0] if sparse else None)
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
 
 
-def e2e_arm(args, A, torch, dev, host, w, c, flags, ws, world):
+def e2e_arm(args, torch, dev, host, w, flops, fwd, bwd, world):
     """Same step through the public API with host buffers: every step copies
     Q, K, V, dO from pinned host memory to the device and O, LSE, m, dQ, dK, dV
     back, all inside the timed region."""
@@ -301,9 +370,8 @@ def e2e_arm(args, A, torch, dev, host, w, c, flags, ws, world):
     def step():
         for n in pin:
             dbuf[n].copy_(pin[n], non_blocking=True)
-        A.attnqat_fwd(dbuf["q"], dbuf["k"], dbuf["v"], sm_scale=c, flags=flags, ws=ws, out=(o, lse, m))
-        A.attnqat_bwd(dbuf["q"], dbuf["k"], dbuf["v"], lse, m, dbuf["do"], ws, sm_scale=c, flags=flags,
-                      out=(dq, dk, dv))
+        fwd(dbuf["q"], dbuf["k"], dbuf["v"], (o, lse, m))
+        bwd(dbuf["q"], dbuf["k"], dbuf["v"], lse, m, dbuf["do"], (dq, dk, dv))
         for name, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv), ("lse", lse), ("m", m)):
             outs[name].copy_(t, non_blocking=True)
 
@@ -318,7 +386,7 @@ def e2e_arm(args, A, torch, dev, host, w, c, flags, ws, world):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
-    value = world * w.nominal_flops()["total"] * n / (ms * 1e-3) / 1e12
+    value = world * flops["total"] * n / (ms * 1e-3) / 1e12
     return {"value": round(value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": round(ms / n, 4)}
 
@@ -342,26 +410,37 @@ def load_traffic(kernel):
 
 # -------------------------------------------------------------- CPU oracle --
 
-def cpu_baseline_sample(rows: int):
+def cpu_baseline_sample(rows: int, sel=None):
     """The float64 oracle on a bounded sample of the workload: head 0, the
     first `rows` query rows against all 31200 keys, forward and backward
     (dQ for those rows, their dK/dV contributions for every key).  Returns the
-    nominal TFLOP/s of that sub-problem."""
+    nominal TFLOP/s of that sub-problem (with a tile selection `sel` of head
+    0: block-sparse, counted on the selected keys)."""
     import oracle
     w = W.get(WORKLOAD)
     q = W.head_bits(w, "q", 0, 0)[:rows]
     k = W.head_bits(w, "k", 0, 0)
     v = W.head_bits(w, "v", 0, 0)
     do = W.head_bits(w, "do", 0, 0)[:rows]
+    T = W.SPARSE_TILE
+    if sel is not None:
+        sel = sel[: -(-rows // T)]
     t0 = time.perf_counter()
-    hd = oracle.Head(q, k, v, w.sm_scale, oracle.QUANT_ALL, do)
+    hd = oracle.Head(q, k, v, w.sm_scale, oracle.QUANT_ALL, do, sel=sel, tile=T)
     hd.stats()
     hd.backward()
     dt = time.perf_counter() - t0
-    flops = 3.5 * 4.0 * rows * w.Lk * w.D
+    pairs = float(rows * w.Lk)
+    if sel is not None:
+        keys = np.minimum(T, w.Lk - T * np.arange(sel.shape[1]))
+        rws = np.minimum(T, rows - T * np.arange(sel.shape[0]))
+        pairs = float(rws @ sel.astype(np.float64) @ keys)
+    flops = 3.5 * 4.0 * pairs * w.D
+    what = "block-sparse, selected keys only, " if sel is not None else ""
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": "head 0, query rows [0,%d) x all %d keys, fwd+bwd (float64 C oracle)" % (rows, w.Lk)}
+            "sample": "head 0, query rows [0,%d) x all %d keys, %sfwd+bwd (float64 C oracle)" % (rows, w.Lk,
+                                                                                                what)}
 
 
 def reference_arm(args):
@@ -402,6 +481,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--sparsity", type=float, default=None,
+                    help="time the block-sparse (VSA) step with this key-tile sparsity instead")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3

@@ -215,6 +215,47 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse,
                 void *dv, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Block-sparse fine attention (VSA).
+ *
+ * Defined by: vsqa-test-1.3b metadata.json, "attention": backend
+ * VSA_QAT_TRAIN_C128, kind "vsa", cube_shape 4 x 4 x 8 (128-token cubes),
+ * "fine": "NVFP4 fake-quant with BF16 matmul" (quantize_fine, quant_p,
+ * quant_v), key blocks chosen per query block by a top-k "selection"
+ * (effective_topk = max(1, min(ceil((1 - sparsity) * num_blocks),
+ * num_blocks)), sparsity 0.9).  Each query tile of ATTNQAT_SPARSE_TILE tokens
+ * attends only to the keys of its selected key tiles: the computation above
+ * with the softmax (exact max m, sum l, fq(P~) blocks) over those keys alone;
+ * fq(Q), fq(K), fq(V) do not depend on the selection.  A query tile with no
+ * selected key tile gets O = 0 and m = LSE = -infinity, dQ = 0; a key tile no
+ * query tile selects gets dK = dV = 0.  Choosing the tiles (the coarse
+ * branch), its gates and the token-to-cube layout belong to the caller:
+ * tokens are taken in cube order.
+ *
+ * tile_mask: device bytes [B][H][ceil(Lq/128)][ceil(Lk/128)], caller-owned,
+ * nonzero = the query tile attends the key tile; read, never written.  The
+ * backward must receive the mask the forward used.  Other arguments and
+ * errors are those of attnqat_fwd / attnqat_bwd (plus EINVAL for a null
+ * tile_mask); the workspace is attnqat_sparse_workspace_size() bytes (the
+ * dense workspace plus int32 tile lists, 8 * B*H*nq*nk + 4 * B*H*(nq + nk)
+ * bytes, rebuilt from the mask by every call), passed unchanged from
+ * attnqat_sparse_fwd to attnqat_sparse_bwd.
+ */
+#define ATTNQAT_SPARSE_TILE 128
+size_t attnqat_sparse_workspace_size(int B, int H, int Lq, int Lk, int D,
+                                     uint32_t flags);
+int attnqat_sparse_fwd(const void *q, const void *k, const void *v, int B,
+                       int H, int Lq, int Lk, int D, float sm_scale,
+                       uint32_t flags, const uint8_t *tile_mask, void *o,
+                       float *lse, float *m, void *ws, size_t ws_bytes,
+                       void *stream);
+int attnqat_sparse_bwd(const void *q, const void *k, const void *v,
+                       const float *lse, const float *m, const void *dO, int B,
+                       int H, int Lq, int Lk, int D, float sm_scale,
+                       uint32_t flags, const uint8_t *tile_mask, void *dq,
+                       void *dk, void *dv, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/*
  * attnqat_fwd_noalloc -- attnqat_fwd for callers that cannot allocate.
  *
  * The pages have no counterpart of this entry point; it exists for callers

@@ -15,6 +15,11 @@ Entry points (same names as the C ABI):
   ``(o, lse, m, ws)``.
 * ``attnqat_bwd(q, k, v, lse, m, dO, ws, sm_scale=None, flags=QUANT_ALL)`` --
   straight-through backward; returns ``(dq, dk, dv)``.
+* ``attnqat_sparse_fwd(q, k, v, tile_mask, ...)`` and
+  ``attnqat_sparse_bwd(q, k, v, lse, m, dO, ws, tile_mask, ...)`` -- the
+  block-sparse (VSA fine attention) variants: ``tile_mask`` is a uint8 CUDA
+  tensor [B, H, ceil(Lq/128), ceil(Lk/128)], nonzero where a 128-query tile
+  attends a 128-key tile.
 
 ``sm_scale=None`` means 1/sqrt(D), chosen here and passed explicitly; the
 library itself never substitutes a default (FastVideo PR #1457 review, F1).
@@ -85,6 +90,13 @@ def load(build_if_needed: bool = True):
             lib.attnqat_fwd.argtypes = [P, P, P, I, I, I, I, I, F, U32, P, P, P, P, SZ, P]
             lib.attnqat_bwd.restype = I
             lib.attnqat_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, U32, P, P, P, P, SZ, P]
+            lib.attnqat_sparse_workspace_size.restype = SZ
+            lib.attnqat_sparse_workspace_size.argtypes = [I, I, I, I, I, U32]
+            lib.attnqat_sparse_fwd.restype = I
+            lib.attnqat_sparse_fwd.argtypes = [P, P, P, I, I, I, I, I, F, U32, P, P, P, P, P, SZ, P]
+            lib.attnqat_sparse_bwd.restype = I
+            lib.attnqat_sparse_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, U32, P, P, P, P, P, SZ,
+                                               P]
             _lib = lib
     return _lib
 
@@ -242,6 +254,77 @@ def attnqat_bwd(q, k, v, lse, m, dO, ws, sm_scale=None, flags=QUANT_ALL, out=Non
                             ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
                             ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(st, "attnqat_bwd")
+    return dq, dk, dv
+
+
+SPARSE_TILE = 128
+
+
+def attnqat_sparse_workspace_size(B, H, Lq, Lk, D, flags=QUANT_ALL) -> int:
+    return int(load().attnqat_sparse_workspace_size(B, H, Lq, Lk, D, flags))
+
+
+def _tile_mask(tile_mask, B, H, Lq, Lk, device):
+    torch = _torch()
+    want = (B, H, -(-Lq // SPARSE_TILE), -(-Lk // SPARSE_TILE))
+    if not isinstance(tile_mask, torch.Tensor) or tile_mask.dtype != torch.uint8 or \
+            tile_mask.device != device or tuple(tile_mask.shape) != want or not tile_mask.is_contiguous():
+        raise ValueError("tile_mask must be a contiguous uint8 tensor %s on %s" % (want, device))
+    return ctypes.c_void_p(tile_mask.data_ptr())
+
+
+def attnqat_sparse_fwd(q, k, v, tile_mask, sm_scale=None, flags=QUANT_ALL, ws=None, out=None, stream=None):
+    """Block-sparse Attn-QAT forward (VSA fine attention): each 128-query
+    tile attends only the 128-key tiles ``tile_mask`` selects.  Returns
+    ``(o, lse, m, ws)``; pass ``ws`` and the same mask to
+    :func:`attnqat_sparse_bwd`."""
+    torch = _torch()
+    B, H, Lq, Lk, D = _shape(q, k, v)
+    mp = _tile_mask(tile_mask, B, H, Lq, Lk, q.device)
+    c = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    need = attnqat_sparse_workspace_size(B, H, Lq, Lk, D, flags)
+    if need == 0:
+        _check(EINVAL, "attnqat_sparse_workspace_size")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+        m = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    else:
+        o, lse, m = out
+    st = load().attnqat_sparse_fwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                   ctypes.c_void_p(v.data_ptr()), B, H, Lq, Lk, D, c, flags, mp,
+                                   ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+                                   ctypes.c_void_p(m.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                   ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "attnqat_sparse_fwd")
+    return o, lse, m, ws
+
+
+def attnqat_sparse_bwd(q, k, v, lse, m, dO, ws, tile_mask, sm_scale=None, flags=QUANT_ALL, out=None,
+                       stream=None):
+    """Block-sparse Attn-QAT backward (straight-through) with the forward's
+    ``ws`` and ``tile_mask``.  Returns ``(dq, dk, dv)``."""
+    torch = _torch()
+    B, H, Lq, Lk, D = _shape(q, k, v)
+    mp = _tile_mask(tile_mask, B, H, Lq, Lk, q.device)
+    _require_bf16_cuda("dO", dO, 4)
+    if dO.shape != q.shape or not dO.is_contiguous():
+        raise ValueError("dO must be contiguous and shaped like q")
+    c = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    st = load().attnqat_sparse_bwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                   ctypes.c_void_p(v.data_ptr()),
+                                   ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(m.data_ptr()),
+                                   ctypes.c_void_p(dO.data_ptr()), B, H, Lq, Lk, D, c, flags, mp,
+                                   ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
+                                   ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                   ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "attnqat_sparse_bwd")
     return dq, dk, dv
 
 

@@ -177,6 +177,7 @@ static bool encode_vcodes(CUtensorMap *map, const void *base, int BH, int Lk, in
 struct Workspace {
   size_t qh, kh, vh, vh16, o32, delta, stats, do16, qc, qsf, kc, ksf, vc, vsf, total;
   size_t qsf_bytes, ksf_bytes, vsf_bytes;
+  size_t kv_list, kv_count, q_list, q_count;  // block-sparse tile lists
 };
 
 // fq(Q) and fq(K) are exact in fp16 (values sign * E2M1 * E4M3 lie in
@@ -202,7 +203,7 @@ static bool pv_fp4(uint32_t flags, int Lk, int D) { return do_f16(flags) && (Lk 
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
+static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags, bool sparse = false) {
   Workspace w{};
   const size_t BH = static_cast<size_t>(B) * H;
   const size_t qbytes = BH * Lq * D * 2, kbytes = BH * Lk * D * 2;
@@ -244,6 +245,16 @@ static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
   if (pv4) off = align256(off + BH * Lk * D / 2);
   w.vsf = off;
   if (pv4) off = align256(off + w.vsf_bytes);
+  // block-sparse: the tile lists the attention kernels walk (int32), built
+  // from the caller's tile mask by every sparse call
+  w.kv_list = off;
+  if (sparse) off = align256(off + BH * ntq * ntk * 4);
+  w.kv_count = off;
+  if (sparse) off = align256(off + BH * ntq * 4);
+  w.q_list = off;
+  if (sparse) off = align256(off + BH * ntk * ntq * 4);
+  w.q_count = off;
+  if (sparse) off = align256(off + BH * ntk * 4);
   w.total = off;
   return w;
 }
@@ -420,16 +431,35 @@ size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flag
   return layout(B, H, Lq, Lk, D, flags).total;
 }
 
-int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int Lq, int Lk, int D,
-                float sm_scale, uint32_t flags, void *o, float *lse, float *m, void *ws, size_t ws_bytes,
-                void *stream) {
+}  // extern "C"
+
+namespace attnqat {
+
+// Builds the block-sparse tile lists from the caller's mask into the
+// workspace (no-op for dense calls, mask == nullptr).
+static int plan_sparse(const uint8_t *mask, int BH, int Lq, int Lk, uint8_t *wsb, const Workspace &w,
+                       cudaStream_t s) {
+  if (!mask) return ATTNQAT_OK;
+  ProfScope ps("sparse_plan", s);
+  const cudaError_t e = launch_sparse_plan(mask, BH, (Lq + kBM - 1) / kBM, (Lk + kBN - 1) / kBN,
+                                           reinterpret_cast<int32_t *>(wsb + w.kv_list),
+                                           reinterpret_cast<int32_t *>(wsb + w.kv_count),
+                                           reinterpret_cast<int32_t *>(wsb + w.q_list),
+                                           reinterpret_cast<int32_t *>(wsb + w.q_count), s);
+  return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
+}
+
+// attnqat_fwd (mask == nullptr) and attnqat_sparse_fwd.
+static int run_fwd(const void *q, const void *k, const void *v, int B, int H, int Lq, int Lk, int D,
+                   float sm_scale, uint32_t flags, const uint8_t *mask, void *o, float *lse, float *m, void *ws,
+                   size_t ws_bytes, void *stream) {
   int st = check_shape(B, H, Lq, Lk, D, sm_scale, flags);
   if (st != ATTNQAT_OK) return st;
   if (!q || !k || !v || !o || !lse || !m || !ws) return ATTNQAT_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(m) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
     return ATTNQAT_EINVAL;
-  const Workspace w = layout(B, H, Lq, Lk, D, flags);
+  const Workspace w = layout(B, H, Lq, Lk, D, flags, mask != nullptr);
   if (ws_bytes < w.total) return ATTNQAT_ENOSPC;
   st = check_device();
   if (st != ATTNQAT_OK) return st;
@@ -438,6 +468,8 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   st = prepare_operands(q, k, v, B, H, Lq, Lk, D, flags, wsb, w, s);
   if (st != ATTNQAT_OK) return st;
   const int BH = B * H;
+  st = plan_sparse(mask, BH, Lq, Lk, wsb, w, s);
+  if (st != ATTNQAT_OK) return st;
   const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
   const void *kh = (flags & ATTNQAT_QUANT_K) ? static_cast<const void *>(wsb + w.kh) : k;
   const bool pv_f16 = (flags & ATTNQAT_QUANT_V) != 0;
@@ -463,6 +495,8 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   a.o32 = reinterpret_cast<float *>(wsb + w.o32);
   a.lse = lse;
   a.m = m;
+  a.kv_list = mask ? reinterpret_cast<const int32_t *>(wsb + w.kv_list) : nullptr;
+  a.kv_count = mask ? reinterpret_cast<const int32_t *>(wsb + w.kv_count) : nullptr;
   cudaError_t e;
   {
     ProfScope ps("attn_fwd", s);
@@ -471,9 +505,10 @@ int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int L
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }
 
-int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, const float *m, const void *dO,
-                int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags, void *dq, void *dk, void *dv,
-                void *ws, size_t ws_bytes, void *stream) {
+// attnqat_bwd (mask == nullptr) and attnqat_sparse_bwd.
+static int run_bwd(const void *q, const void *k, const void *v, const float *lse, const float *m, const void *dO,
+                   int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags, const uint8_t *mask,
+                   void *dq, void *dk, void *dv, void *ws, size_t ws_bytes, void *stream) {
   int st = check_shape(B, H, Lq, Lk, D, sm_scale, flags);
   if (st != ATTNQAT_OK) return st;
   if (!q || !k || !v || !lse || !m || !dO || !dq || !dk || !dv || !ws) return ATTNQAT_EINVAL;
@@ -481,13 +516,15 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
       !aligned16(dk) || !aligned16(dv) || !aligned16(lse) || !aligned16(m) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
     return ATTNQAT_EINVAL;
-  const Workspace w = layout(B, H, Lq, Lk, D, flags);
+  const Workspace w = layout(B, H, Lq, Lk, D, flags, mask != nullptr);
   if (ws_bytes < w.total) return ATTNQAT_ENOSPC;
   st = check_device();
   if (st != ATTNQAT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int BH = B * H;
+  st = plan_sparse(mask, BH, Lq, Lk, wsb, w, s);
+  if (st != ATTNQAT_OK) return st;
   float *delta = reinterpret_cast<float *>(wsb + w.delta);
   float *stats = reinterpret_cast<float *>(wsb + w.stats);
   const bool dof16 = do_f16(flags);
@@ -533,6 +570,10 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
   a.dq = static_cast<__nv_bfloat16 *>(dq);
   a.dk = static_cast<__nv_bfloat16 *>(dk);
   a.dv = static_cast<__nv_bfloat16 *>(dv);
+  a.kv_list = mask ? reinterpret_cast<const int32_t *>(wsb + w.kv_list) : nullptr;
+  a.kv_count = mask ? reinterpret_cast<const int32_t *>(wsb + w.kv_count) : nullptr;
+  a.q_list = mask ? reinterpret_cast<const int32_t *>(wsb + w.q_list) : nullptr;
+  a.q_count = mask ? reinterpret_cast<const int32_t *>(wsb + w.q_count) : nullptr;
   // with Q and K quantized, S runs on the packed NVFP4 codes
   CUtensorMap tq4, tk4;
   if (f16 && !(encode_codes(&tq4, wsb + w.qc, BH, Lq, D) && encode_codes(&tk4, wsb + w.kc, BH, Lk, D)))
@@ -548,6 +589,44 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
     e = launch_bwd_dq(D, f16, dof16, f16 ? tq4 : tq, tk, tv, tdo, f16 ? tk4 : tk, a, BH, s);
   }
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
+}
+
+}  // namespace attnqat
+
+extern "C" {
+
+int attnqat_fwd(const void *q, const void *k, const void *v, int B, int H, int Lq, int Lk, int D,
+                float sm_scale, uint32_t flags, void *o, float *lse, float *m, void *ws, size_t ws_bytes,
+                void *stream) {
+  return run_fwd(q, k, v, B, H, Lq, Lk, D, sm_scale, flags, nullptr, o, lse, m, ws, ws_bytes, stream);
+}
+
+int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, const float *m, const void *dO,
+                int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags, void *dq, void *dk, void *dv,
+                void *ws, size_t ws_bytes, void *stream) {
+  return run_bwd(q, k, v, lse, m, dO, B, H, Lq, Lk, D, sm_scale, flags, nullptr, dq, dk, dv, ws, ws_bytes,
+                 stream);
+}
+
+size_t attnqat_sparse_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
+  if (check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
+  return layout(B, H, Lq, Lk, D, flags, true).total;
+}
+
+int attnqat_sparse_fwd(const void *q, const void *k, const void *v, int B, int H, int Lq, int Lk, int D,
+                       float sm_scale, uint32_t flags, const uint8_t *tile_mask, void *o, float *lse, float *m,
+                       void *ws, size_t ws_bytes, void *stream) {
+  if (!tile_mask) return ATTNQAT_EINVAL;
+  return run_fwd(q, k, v, B, H, Lq, Lk, D, sm_scale, flags, tile_mask, o, lse, m, ws, ws_bytes, stream);
+}
+
+int attnqat_sparse_bwd(const void *q, const void *k, const void *v, const float *lse, const float *m,
+                       const void *dO, int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags,
+                       const uint8_t *tile_mask, void *dq, void *dk, void *dv, void *ws, size_t ws_bytes,
+                       void *stream) {
+  if (!tile_mask) return ATTNQAT_EINVAL;
+  return run_bwd(q, k, v, lse, m, dO, B, H, Lq, Lk, D, sm_scale, flags, tile_mask, dq, dk, dv, ws, ws_bytes,
+                 stream);
 }
 
 }  // extern "C"

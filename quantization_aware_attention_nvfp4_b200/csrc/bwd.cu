@@ -22,6 +22,11 @@
 // there); warps 2..9 row warps: two per TMEM lane quarter, so every query row
 // (TMEM lane) has two threads, each owning 64 of the tile's 128 columns; the
 // remaining warps idle.
+//
+// Block-sparse (VSA fine attention): with a.q_list / a.kv_list set, the dK/dV
+// kernel walks only the query tiles that selected its key tile and the dQ
+// kernel only the key tiles its query tile selected; a CTA with an empty list
+// writes zero gradients.
 #include "common.cuh"
 #include "internal.h"
 
@@ -229,7 +234,9 @@ __device__ __forceinline__ void dkdv_ds_f16(const float (&p)[64], const uint32_t
   }
 }
 
-template <int D, int QP, int QKF16, int DOF16>
+// SP: block-sparse (walks a.q_list); a separate instantiation, so the dense
+// kernel carries none of the list handling.
+template <int D, int QP, int QKF16, int DOF16, bool SP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -246,6 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt = blockIdx.x;
   const int bh = blockIdx.y;
   const int nq = a.nq_tiles;
+  // the query tiles this key tile meets: all nq, or those that selected it
+  const size_t krow = static_cast<size_t>(bh) * a.nk_tiles + kt;
+  const int32_t *ql = SP ? a.q_list + krow * nq : nullptr;
+  const int n = SP ? a.q_count[krow] : nq;
+  auto qtile = [&](int i) -> int { return SP ? __ldg(ql + i) : i; };
 
   if (threadIdx.x == 0) init_bwd_bars(bars, 1, 1);
   if (warp == 1) {
@@ -276,24 +288,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // per query tile, in the order the MMAs need them: Q codes (S), dO (dP,
       // then dV), 16-bit Q (dK; with !FP4S also S)
       int nc = 0, nd = 0, nqh = 0;  // tiles issued per ring
-      for (int i = 0; i < nq; ++i) {
+      for (int i = 0; i < n; ++i) {
         const int st = i & 1;
         const int ph = ((i >> 1) - 1) & 1;
+        const int qi = qtile(i);
         if (FP4S) {
           if (i >= 2 && !mbar_wait(&bars->cempty[st], ph, abort)) break;
           mbar_arrive_expect_tx(&bars->cfull[st], L::kCode + L::kSF);
-          tma_load_3d(smem + L::kQ4 + st * L::kCode, &tmQ4, &bars->cfull[st], 0, i * kBM, bh);
-          bulk_load(smem + L::kQSF + st * L::kSF, a.qsf + (static_cast<size_t>(bh) * nq + i) * L::kSF, L::kSF,
+          tma_load_3d(smem + L::kQ4 + st * L::kCode, &tmQ4, &bars->cfull[st], 0, qi * kBM, bh);
+          bulk_load(smem + L::kQSF + st * L::kSF, a.qsf + (static_cast<size_t>(bh) * nq + qi) * L::kSF, L::kSF,
                     &bars->cfull[st]);
           nc = i + 1;
         }
         if (i >= 2 && !mbar_wait(&bars->bempty[st], ph, abort)) break;
         mbar_arrive_expect_tx(&bars->bfull[st], L::kTile);
-        load_tile<D>(smem + L::kDO + st * L::kTile, &tmDO, &bars->bfull[st], i * kBM, bh);
+        load_tile<D>(smem + L::kDO + st * L::kTile, &tmDO, &bars->bfull[st], qi * kBM, bh);
         nd = i + 1;
         if (i >= 2 && !mbar_wait(&bars->aempty[st], ph, abort)) break;
         mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
-        load_tile<D>(smem + L::kQ + st * L::kTile, &tmQ, &bars->afull[st], i * kBM, bh);
+        load_tile<D>(smem + L::kQ + st * L::kTile, &tmQ, &bars->afull[st], qi * kBM, bh);
         nqh = i + 1;
       }
       if (*abort) {
@@ -354,8 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&bars->sfull);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int i = 0; ok && i < nq; ++i) {
+      if (ok && n > 0) ok = issue_s(0);
+      for (int i = 0; ok && i < n; ++i) {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
         // dP_i once the rows have read S_i (fill 2i)
@@ -370,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&bars->xempty);
         umma_commit(&bars->bempty[st]);
         // S_{i+1} once the rows have read dP_i (fill 2i+1)
-        if (i + 1 < nq && !(mbar_wait(&bars->sempty, (2 * i + 1) & 1, abort) && issue_s(i + 1))) break;
+        if (i + 1 < n && !(mbar_wait(&bars->sempty, (2 * i + 1) & 1, abort) && issue_s(i + 1))) break;
         // dK += dS^T Q_i
         if (!mbar_wait(&bars->xfull, (2 * i + 1) & 1, abort)) break;
         if (FP4S && !mbar_wait(&bars->afull[st], ph, abort)) break;
@@ -392,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     // row statistics of the current query tile, prefetched one tile ahead
     auto load_stats = [&](int i, float &m, float &lse, float &delta) {
-      const int qg = i * kBM + static_cast<int>(rr.row);
-      const bool vq = i < nq && qg < a.Lq;
+      const int qg = (i < n ? qtile(i) : 0) * kBM + static_cast<int>(rr.row);
+      const bool vq = i < n && qg < a.Lq;
       const size_t si = static_cast<size_t>(bh) * a.Lq + (vq ? qg : 0);
       m = vq ? a.m[si] : 0.0f;
       lse = vq ? a.lse[si] : 0.0f;
@@ -402,8 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_n, lse_n, delta_n;
     load_stats(0, m_n, lse_n, delta_n);
     const float dos = DOF16 ? do_scale(a.stats) : 1.0f;
-    for (int i = 0; i < nq; ++i) {
-      const bool vq = i * kBM + static_cast<int>(rr.row) < a.Lq;
+    for (int i = 0; i < n; ++i) {
+      const bool vq = qtile(i) * kBM + static_cast<int>(rr.row) < a.Lq;
       const float m = m_n, lse = lse_n, delta = delta_n;
       load_stats(i + 1, m_n, lse_n, delta_n);
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
@@ -487,8 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               x[k] = pack_bf16x2(__uint_as_float(s[8 * i + 2 * k]) * kscale,
                                  __uint_as_float(s[8 * i + 2 * k + 1]) * kscale);
             }
-            dv[i] = make_uint4(w[0], w[1], w[2], w[3]);
-            dk[i] = make_uint4(x[0], x[1], x[2], x[3]);
+            // a key tile no query tile selected: the accumulators were never written
+            dv[i] = n > 0 ? make_uint4(w[0], w[1], w[2], w[3]) : make_uint4(0, 0, 0, 0);
+            dk[i] = n > 0 ? make_uint4(x[0], x[1], x[2], x[3]) : make_uint4(0, 0, 0, 0);
           }
         }
       }
@@ -578,7 +592,8 @@ __device__ __forceinline__ void dq_tile_f16(const uint32_t (&sv)[64], const uint
   }
 }
 
-template <int D, int QKF16, int DOF16>
+// SP: block-sparse (walks a.kv_list), as for the dK/dV kernel.
+template <int D, int QKF16, int DOF16, bool SP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -595,6 +610,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qt = blockIdx.x;
   const int bh = blockIdx.y;
   const int nk = a.nk_tiles;
+  // the key tiles this query tile visits: all nk, or its block-sparse list
+  const size_t qrow = static_cast<size_t>(bh) * a.nq_tiles + qt;
+  const int32_t *kvl = SP ? a.kv_list + qrow * nk : nullptr;
+  const int n = SP ? a.kv_count[qrow] : nk;
+  auto ktile = [&](int j) -> int { return SP ? __ldg(kvl + j) : j; };
 
   if (threadIdx.x == 0) init_bwd_bars(bars, 1, 1);
   if (warp == 1) {
@@ -623,24 +643,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       load_tile<D>(smem + L::kDO, &tmDO, &bars->kvfull, qt * kBM, bh);
       int n4 = 0, nv = 0, nkh = 0;  // tiles issued per ring
-      for (int j = 0; j < nk; ++j) {
+      for (int j = 0; j < n; ++j) {
         const int st = j & 1;
         const int ph = ((j >> 1) - 1) & 1;
+        const int kj = ktile(j);
         if (FP4S) {
           if (j >= 2 && !mbar_wait(&bars->cempty[st], ph, abort)) break;
           mbar_arrive_expect_tx(&bars->cfull[st], L::kCode + L::kSF);
-          tma_load_3d(smem + L::kK4 + st * L::kCode, &tmK4, &bars->cfull[st], 0, j * kBN, bh);
-          bulk_load(smem + L::kKSF + st * L::kSF, a.ksf + (static_cast<size_t>(bh) * nk + j) * L::kSF, L::kSF,
+          tma_load_3d(smem + L::kK4 + st * L::kCode, &tmK4, &bars->cfull[st], 0, kj * kBN, bh);
+          bulk_load(smem + L::kKSF + st * L::kSF, a.ksf + (static_cast<size_t>(bh) * nk + kj) * L::kSF, L::kSF,
                     &bars->cfull[st]);
           n4 = j + 1;
         }
         if (j >= 2 && !mbar_wait(&bars->bempty[st], ph, abort)) break;
         mbar_arrive_expect_tx(&bars->bfull[st], L::kTile);
-        load_tile<D>(smem + L::kV + st * L::kTile, &tmV, &bars->bfull[st], j * kBN, bh);
+        load_tile<D>(smem + L::kV + st * L::kTile, &tmV, &bars->bfull[st], kj * kBN, bh);
         nv = j + 1;
         if (j >= 2 && !mbar_wait(&bars->aempty[st], ph, abort)) break;
         mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
-        load_tile<D>(smem + L::kK + st * L::kTile, &tmK, &bars->afull[st], j * kBN, bh);
+        load_tile<D>(smem + L::kK + st * L::kTile, &tmK, &bars->afull[st], kj * kBN, bh);
         nkh = j + 1;
       }
       if (*abort) {
@@ -698,15 +719,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&bars->sfull);
           return true;
         };
-        if (ok) ok = issue_sdp(0);
-        for (int j = 1; ok && j < nk; ++j) ok = mbar_wait(&bars->sempty, (j - 1) & 1, abort) && issue_sdp(j);
+        if (ok && n > 0) ok = issue_sdp(0);
+        for (int j = 1; ok && j < n; ++j) ok = mbar_wait(&bars->sempty, (j - 1) & 1, abort) && issue_sdp(j);
         // TMEM is freed by this warp: let its own MMAs finish first
         umma_commit(&bars->adone);
         mbar_wait_drain(&bars->adone, 0);
       } else {
         // issuer B: dQ += dS_j K_j.  K_j goes back to the producer after dQ_j
         // (without FP4S, S_j read it too; the rows have read S_j by then).
-        for (int j = 0; j < nk; ++j) {
+        for (int j = 0; j < n; ++j) {
           const int st = j & 1;
           if (!mbar_wait(&bars->xfull, j & 1, abort) || !mbar_wait(&bars->afull[st], (j >> 1) & 1, abort)) break;
           tc_fence_after();
@@ -731,12 +752,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float a1 = DOF16 ? dsc / do_scale(a.stats) : 0.0f;
     const float b1 = -delta * dsc;
     const int last_valid = a.Lk - (nk - 1) * kBN;
+    // the lists ascend, so only the last tile visited can be the partial one
+    const bool tail_last = n > 0 && ktile(n - 1) == nk - 1 && last_valid < kBN;
     const uint32_t xaddr = sbase + L::kX;
     const uint32_t tS = tmem + rr.lane_addr + L::kTmemS, tDP = tmem + rr.lane_addr + L::kTmemDP;
     bool ok = true;
-    for (int j = 0; j < nk; ++j) {
+    for (int j = 0; j < n; ++j) {
       uint32_t dsw[32];
       uint32_t sv[64], dv[64];
+      const bool tail = tail_last && j == n - 1;
       if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
       tc_fence_after();
       load_sdp(tS, tDP, col0, sv, dv);
@@ -744,12 +768,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
       if (DOF16) {
-        if (j == nk - 1 && last_valid < kBN)
+        if (tail)
           dq_tile_f16<true>(sv, dv, col0, last_valid, cl, nlse, a1, b1, dsw);
         else
           dq_tile_f16<false>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw);
       } else {
-        if (j == nk - 1 && last_valid < kBN)
+        if (tail)
           dq_tile<QKF16, true>(sv, dv, col0, last_valid, vq, cl, nlse, delta, dsc, dsw);
         else
           dq_tile<QKF16, false>(sv, dv, col0, kBN, vq, cl, nlse, delta, dsc, dsw);
@@ -779,7 +803,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 4; ++k)
               w[k] = pack_bf16x2(__uint_as_float(r[8 * i + 2 * k]) * qscale,
                                  __uint_as_float(r[8 * i + 2 * k + 1]) * qscale);
-            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            // no key tile selected: the accumulator was never written
+            dst[i] = n > 0 ? make_uint4(w[0], w[1], w[2], w[3]) : make_uint4(0, 0, 0, 0);
           }
         }
       }
@@ -798,19 +823,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------- launchers --
 
-template <int D, int QP, int QKF16, int DOF16>
-static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                 const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
-                                 cudaStream_t stream) {
+template <int D, int QP, int QKF16, int DOF16, bool SP>
+static cudaError_t launch_dkdv_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                  const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
+                                  cudaStream_t stream) {
   using L = DkdvLayout<D, QKF16>;
   static_assert(L::kDynSmem <= 232448, "dK/dV shared memory over the 227 KB limit");
   static_assert(sizeof(BwdBars) <= L::kBarBytes, "dK/dV barrier block larger than its reservation");
   static_assert(L::kTmemSFB + L::kSFCols <= L::kTmemCols, "dK/dV TMEM over 512 columns");
-  auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16, DOF16>;
+  auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16, DOF16, SP>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.nk_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, tq4, a);
   return cudaGetLastError();
+}
+
+template <int D, int QP, int QKF16, int DOF16>
+static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                 const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
+                                 cudaStream_t stream) {
+  return a.q_list ? launch_dkdv_sp<D, QP, QKF16, DOF16, true>(tq, tk, tv, tdo, tq4, a, BH, stream)
+                  : launch_dkdv_sp<D, QP, QKF16, DOF16, false>(tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
 template <int D>
@@ -832,19 +865,27 @@ cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const
                   : dkdv_dispatch<64>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
-template <int D, int QKF16, int DOF16>
-static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                               const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
-                               cudaStream_t stream) {
+template <int D, int QKF16, int DOF16, bool SP>
+static cudaError_t launch_dq_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
+                                cudaStream_t stream) {
   using L = DqLayout<D, QKF16>;
   static_assert(L::kDynSmem <= 232448, "dQ shared memory over the 227 KB limit");
   static_assert(sizeof(BwdBars) <= L::kBarBytes, "dQ barrier block larger than its reservation");
   static_assert(L::kTmemSFB + 2 * L::kSFCols <= L::kTmemCols, "dQ TMEM over 512 columns");
-  auto kern = attn_bwd_dq_kernel<D, QKF16, DOF16>;
+  auto kern = attn_bwd_dq_kernel<D, QKF16, DOF16, SP>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.nq_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, tk4, a);
   return cudaGetLastError();
+}
+
+template <int D, int QKF16, int DOF16>
+static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                               const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
+                               cudaStream_t stream) {
+  return a.kv_list ? launch_dq_sp<D, QKF16, DOF16, true>(tq, tk, tv, tdo, tk4, a, BH, stream)
+                   : launch_dq_sp<D, QKF16, DOF16, false>(tq, tk, tv, tdo, tk4, a, BH, stream);
 }
 
 template <int D>

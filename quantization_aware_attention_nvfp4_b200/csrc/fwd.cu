@@ -30,6 +30,11 @@
 // KV tiles run without bounds masks; the partial last KV tile runs a
 // separate masked step (fastvideo-kernel triton_kernels commit, SM100
 // Attn-QAT route).
+//
+// Block-sparse (VSA fine attention): with a.kv_list set, the CTA walks only
+// the key tiles listed for its query tile, in both sweeps, so m is the exact
+// max over the selected keys; a query tile with no key tile writes O = 0 and
+// m = LSE = -inf.
 #include "common.cuh"
 #include "internal.h"
 
@@ -221,7 +226,9 @@ __device__ __forceinline__ void group_sync(int wq) {
 template <int G>
 constexpr int fwd_threads() { return (2 + 4 * G + 1 + 3) / 4 * 128; }
 
-template <int D, int FP4S, int PVM, int QP, int G>
+// SP: block-sparse (walks a.kv_list); a separate instantiation, so the dense
+// kernel carries none of the list handling.
+template <int D, int FP4S, int PVM, int QP, int G, bool SP>
 __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
@@ -242,6 +249,11 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
   const int qt = blockIdx.x;
   const int bh = blockIdx.y;
   const int nk = a.nk_tiles;
+  // the key tiles this query tile visits: all nk, or its block-sparse list
+  const size_t qrow = static_cast<size_t>(bh) * a.nq_tiles + qt;
+  const int32_t *kvl = SP ? a.kv_list + qrow * nk : nullptr;
+  const int n = SP ? a.kv_count[qrow] : nk;
+  auto ktile = [&](int j) -> int { return SP ? __ldg(kvl + j) : j; };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
@@ -298,8 +310,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         bulk_load(smem + L::kQSF, a.qsf + (static_cast<size_t>(bh) * a.nq_tiles + qt) * L::kSF, L::kSF,
                   &bars->qfull);
       int kissued = 0, vissued = 0;
-      for (int t = 0; t < 2 * nk; ++t) {
-        const int j = t < nk ? t : t - nk;
+      for (int t = 0; t < 2 * n; ++t) {
+        const int j = ktile(t < n ? t : t - n);
         const int st = t % kNSK;
         if (t >= kNSK && !mbar_wait(&bars->kempty[st], ((t / kNSK) - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bars->kfull[st], L::kQK + L::kSF);
@@ -308,8 +320,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
           bulk_load(smem + L::kKSF + st * L::kSF, a.ksf + (static_cast<size_t>(bh) * nk + j) * L::kSF, L::kSF,
                     &bars->kfull[st]);
         kissued = t + 1;
-        if (t >= nk) {
-          const int u = t - nk;
+        if (t >= n) {
+          const int u = t - n;
           const int vs = u % kNSV;
           if (u >= kNSV && !mbar_wait(&bars->vempty[vs], ((u / kNSV) - 1) & 1, abort)) break;
           mbar_arrive_expect_tx(&bars->vfull[vs], L::kVT + L::kVSF);
@@ -366,7 +378,7 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       const uint64_t dP4 = sdesc_make(sbase + L::kP, 16, 512, 4), dV4 = sdesc_make(sbase + L::kV, 16, 512, 4);
       const uint64_t dPSF = sdesc_make(sbase + L::kPSFo, 16, 128, 0), dVSF = sdesc_make(sbase + L::kVSFo, 16, 128, 0);
       constexpr uint32_t idPV4 = idesc_mxf4(kBM, D);
-      // S tile t (K tile t mod nk) into TMEM column dcol, signalling `full`
+      // S tile t (the t-th K tile loaded) into TMEM column dcol, signalling `full`
       auto issue_s = [&](int t, uint32_t dcol, uint64_t *full) -> bool {
         const int st = t % kNSK;
         if (!mbar_wait(&bars->kfull[st], (t / kNSK) & 1, abort)) return false;
@@ -388,20 +400,20 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         return true;
       };
       // row-max sweep: three S buffers, tiles alternating between A and B
-      for (int t = issuer_a ? 0 : 1; ok && t < nk; t += 2) {
+      for (int t = issuer_a ? 0 : 1; ok && t < n; t += 2) {
         const int b = t % L::kNS1;
         if (t >= L::kNS1 && !mbar_wait(&bars->sempty1[b], ((t / L::kNS1) - 1) & 1, abort)) { ok = false; break; }
         ok = issue_s(t, b * kBN, &bars->sfull1[b]);
       }
       if (issuer_a) {
         // every row-max buffer read before the output sweep reuses columns 0..255
-        for (int t = (nk > L::kNS1 ? nk - L::kNS1 : 0); ok && t < nk; ++t)
+        for (int t = (n > L::kNS1 ? n - L::kNS1 : 0); ok && t < n; ++t)
           ok = mbar_wait(&bars->sempty1[t % L::kNS1], (t / L::kNS1) & 1, abort);
         // output sweep: S into two buffers
-        for (int j = 0; ok && j < nk; ++j) {
+        for (int j = 0; ok && j < n; ++j) {
           const int sb = j & 1;
           if (j >= 2 && !mbar_wait(&bars->sempty[sb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
-          ok = issue_s(nk + j, sb * kBN, &bars->sfull[sb]);
+          ok = issue_s(n + j, sb * kBN, &bars->sfull[sb]);
         }
         // TMEM is freed by this warp: let its own MMAs finish first
         umma_commit(&bars->adone);
@@ -410,7 +422,7 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         // output sweep: O += fq(P~)_j fq(V)_j as the rows hand over each P tile
         // (the first P V runs after every row-max tile was read, so it may
         // overwrite the third S buffer's columns)
-        for (int j = 0; ok && j < nk; ++j) {
+        for (int j = 0; ok && j < n; ++j) {
           const int pb = j & 1;
           const int vs = j % kNSV;
           if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, abort) || !mbar_wait(&bars->vfull[vs], (j / kNSV) & 1, abort)) {
@@ -451,15 +463,18 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     const RowRole rr(warp, lane);
     const int col0 = rr.half * NC;
     const int last_valid = a.Lk - (nk - 1) * kBN;  // keys in the last KV tile
+    // the lists ascend, so only the last tile visited can be the partial one
+    const bool tail_last = n > 0 && ktile(n - 1) == nk - 1 && last_valid < kBN;
     float mrow = -INFINITY;
     bool ok = true;
-    for (int j = 0; j < nk; ++j) {
+    for (int j = 0; j < n; ++j) {
       const int b = j % L::kNS1;
+      const bool tail = tail_last && j == n - 1;
       if (!mbar_wait(&bars->sfull1[b], (j / L::kNS1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + b * kBN;
-      const float mx = (j == nk - 1 && last_valid < kBN) ? row_max_cols<true, NC>(taddr, col0, last_valid)
-                                                         : row_max_cols<false, NC>(taddr, col0, kBN);
+      const float mx = tail ? row_max_cols<true, NC>(taddr, col0, last_valid)
+                            : row_max_cols<false, NC>(taddr, col0, kBN);
       mrow = fmaxf(mrow, mx);
       tc_fence_before();
       __syncwarp();
@@ -475,16 +490,17 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     const float nml = -(m_scaled * kLog2e);
     const float cl = a.scale_log2;
     float lsum = 0.0f;
-    for (int j = 0; ok && j < nk; ++j) {
+    for (int j = 0; ok && j < n; ++j) {
       const int sb = j & 1;
       const int pb = j & 1;
+      const bool tail = tail_last && j == n - 1;
       if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, abort)) { ok = false; break; }
       if (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
       const uint32_t psf = sbase + L::kPSFo + pb * L::kPSF;
-      if (j == nk - 1 && last_valid < kBN)
+      if (tail)
         lsum += prob_cols<PVM, QP, true, NC>(taddr, col0, last_valid, cl, nml, pbase, psf, rr.row);
       else
         lsum += prob_cols<PVM, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, psf, rr.row);
@@ -505,6 +521,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       for (int g = 0; g < G; ++g) lsum += bars->part[g][rr.row];
       tc_fence_after();
       const int q = qt * kBM + static_cast<int>(rr.row);
+      // no key tile selected: O = 0 (the accumulator was never written),
+      // m = LSE = -inf
       const float inv_l = 1.0f / lsum;
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
       constexpr int DC = D / G;            // output columns per thread
@@ -522,7 +540,7 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         if (q < a.Lq) {
           float f[W];
 #pragma unroll
-          for (int i = 0; i < W; ++i) f[i] = __uint_as_float(r[i]) * inv_l;
+          for (int i = 0; i < W; ++i) f[i] = n > 0 ? __uint_as_float(r[i]) * inv_l : 0.0f;
           uint32_t w[W / 2];
 #pragma unroll
           for (int i = 0; i < W / 2; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
@@ -535,8 +553,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         }
       }
       if (q < a.Lq && rr.half == 0) {
-        a.m[static_cast<size_t>(bh) * a.Lq + q] = m_scaled;
-        a.lse[static_cast<size_t>(bh) * a.Lq + q] = m_scaled + logf(lsum);
+        a.m[static_cast<size_t>(bh) * a.Lq + q] = n > 0 ? m_scaled : -INFINITY;
+        a.lse[static_cast<size_t>(bh) * a.Lq + q] = n > 0 ? m_scaled + logf(lsum) : -INFINITY;
       }
     } else {
       // keep the MMA issuer's final commit from outliving the CTA
@@ -552,19 +570,26 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
   }
 }
 
-template <int D, int FP4S, int PVM, int QP>
-static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                const FwdArgs &a, int BH, cudaStream_t stream) {
+template <int D, int FP4S, int PVM, int QP, bool SP>
+static cudaError_t launch_fwd_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                 const FwdArgs &a, int BH, cudaStream_t stream) {
   using L = FwdLayout<D, FP4S, PVM == 2>;
   static_assert(L::kDynSmem <= 232448, "forward shared memory over the 227 KB limit");
   static_assert(sizeof(FwdBars) <= L::kBarBytes, "forward barrier block larger than its reservation");
   static_assert(!FP4S || L::kTmemEnd <= L::kTmemCols, "forward TMEM over 512 columns");
-  auto kern = attn_fwd_kernel<D, FP4S, PVM, QP, kFwdG>;
+  auto kern = attn_fwd_kernel<D, FP4S, PVM, QP, kFwdG, SP>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nq_tiles, BH);
   kern<<<grid, fwd_threads<kFwdG>(), L::kDynSmem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
+}
+
+template <int D, int FP4S, int PVM, int QP>
+static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                const FwdArgs &a, int BH, cudaStream_t stream) {
+  return a.kv_list ? launch_fwd_sp<D, FP4S, PVM, QP, true>(tq, tk, tv, a, BH, stream)
+                   : launch_fwd_sp<D, FP4S, PVM, QP, false>(tq, tk, tv, a, BH, stream);
 }
 
 template <int D, int FP4S>

@@ -20,6 +20,10 @@ struct FwdArgs {
   float *o32;   // float32 copy of O kept in the workspace for the backward's Delta
   float *lse;
   float *m;
+  // block-sparse: key tiles of each query tile ([B*H][nq_tiles] rows of
+  // stride nk_tiles, ascending) and their counts; null for dense attention
+  const int32_t *kv_list;
+  const int32_t *kv_count;
 };
 
 struct BwdArgs {
@@ -38,6 +42,13 @@ struct BwdArgs {
   __nv_bfloat16 *dq;
   __nv_bfloat16 *dk;
   __nv_bfloat16 *dv;
+  // block-sparse (null for dense): key tiles per query tile (dQ kernel) and
+  // query tiles per key tile ([B*H][nk_tiles] rows of stride nq_tiles, for
+  // the dK/dV kernel), ascending, with their counts
+  const int32_t *kv_list;
+  const int32_t *kv_count;
+  const int32_t *q_list;
+  const int32_t *q_count;
 };
 
 // Forward.  tv: 3-D TMA map {D, L, B*H} with 64 x 128 boxes, 128-byte swizzle
@@ -92,6 +103,12 @@ cudaError_t launch_delta(const float *o32, const __nv_bfloat16 *dO, float *delta
 // out = fp16(dO * 2^e) over n elements (n % 8 == 0), 2^e = do_scale(stats).
 cudaError_t launch_scale_do(const __nv_bfloat16 *dO, uint16_t *out, int64_t n, const float *stats,
                             cudaStream_t stream);
+
+// Block-sparse tile lists from a tile mask [BH][nq][nk] (nonzero = the
+// query tile attends the key tile): kv_list/kv_count per query tile and
+// q_list/q_count per key tile, ascending (see sparse.cu).
+cudaError_t launch_sparse_plan(const uint8_t *mask, int BH, int nq, int nk, int32_t *kv_list, int32_t *kv_count,
+                               int32_t *q_list, int32_t *q_count, cudaStream_t stream);
 
 // max |x| over n bf16 values folded into *out (must start at 0).
 cudaError_t launch_absmax(const __nv_bfloat16 *x, int64_t n, float *out, cudaStream_t stream);

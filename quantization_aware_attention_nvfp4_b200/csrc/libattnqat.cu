@@ -4,5 +4,6 @@
 #include "quant.cu"
 #include "fwd.cu"
 #include "bwd.cu"
+#include "sparse.cu"
 #include "api.cu"
 #include "noalloc.cu"

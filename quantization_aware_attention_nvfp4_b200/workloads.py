@@ -140,3 +140,44 @@ def inputs(w: Workload, with_grad: bool = True) -> dict:
     if with_grad:
         out["do"] = tensor_bits(w, "do")
     return out
+
+
+# ----------------------------------------------------- block-sparse masks ----
+# Tile masks for the block-sparse (VSA fine attention) entry points:
+# uint8 [B, H, ceil(Lq/128), ceil(Lk/128)], nonzero = the 128-query tile
+# attends the 128-key tile.  The pages' selection keeps, per query cube, the
+# top-k key cubes of a coarse attention with k = max(1, min(ceil((1 -
+# sparsity) * n), n)) and sparsity 0.9 (vsqa-test-1.3b metadata.json,
+# attention.selection); with no trained model the k tiles are drawn here
+# uniformly without replacement, each (b, h) from its own stream
+# [20260 + workload index, 200, b, h].
+
+SPARSE_TILE = 128
+
+
+def topk_tiles(n_tiles: int, sparsity: float) -> int:
+    """Key tiles kept per query tile at the given sparsity."""
+    return max(1, min(math.ceil((1.0 - sparsity) * n_tiles), n_tiles))
+
+
+def tile_mask(w: Workload, sparsity: float = 0.9) -> np.ndarray:
+    """VSA-style selection: topk_tiles(nk, sparsity) distinct key tiles per
+    query tile."""
+    nq, nk = -(-w.Lq // SPARSE_TILE), -(-w.Lk // SPARSE_TILE)
+    k = topk_tiles(nk, sparsity)
+    out = np.zeros((w.B, w.H, nq, nk), np.uint8)
+    for b in range(w.B):
+        for h in range(w.H):
+            rng = np.random.default_rng([w.seed, 200, b, h])
+            for i in range(nq):
+                out[b, h, i, rng.choice(nk, size=k, replace=False)] = 1
+    return out
+
+
+def random_tile_mask(w: Workload, p: float) -> np.ndarray:
+    """Each (query tile, key tile) pair selected independently with
+    probability p (empty rows and columns happen), stream
+    [20260 + workload index, 201]."""
+    nq, nk = -(-w.Lq // SPARSE_TILE), -(-w.Lk // SPARSE_TILE)
+    rng = np.random.default_rng([w.seed, 201])
+    return (rng.random((w.B, w.H, nq, nk)) < p).astype(np.uint8)

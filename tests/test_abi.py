@@ -149,3 +149,34 @@ def test_quantize_gs_host_validation():
     assert quant(x=0) == A.EINVAL
     assert quant(codes=0) == A.EINVAL
     assert quant(cols=24) == A.EINVAL
+
+
+@pytest.mark.parametrize("shape", [(1, 6, 31200, 31200, 128), (2, 3, 5, 300, 64)])
+def test_sparse_workspace_size(shape):
+    """The dense workspace plus int32 tile lists: [BH][nq][nk] and [BH][nk][nq]
+    with their counts, each region 256-byte aligned."""
+    al = lambda x: (x + 255) // 256 * 256
+    B, H, Lq, Lk, D = shape
+    BH, nq, nk = B * H, -(-Lq // 128), -(-Lk // 128)
+    extra = 2 * al(BH * nq * nk * 4) + al(BH * nq * 4) + al(BH * nk * 4)
+    assert A.attnqat_sparse_workspace_size(*shape, 15) == _expected_ws(*shape, 15) + extra
+
+
+def test_sparse_host_validation():
+    lib = A.load()
+    big = 1 << 30
+
+    def fwd(mask=FAKE, q=FAKE, Lk=128, ws_bytes=big):
+        return lib.attnqat_sparse_fwd(P(q), P(FAKE), P(FAKE), 1, 1, 128, Lk, 128, 0.125, 15, P(mask), P(FAKE),
+                                      P(FAKE), P(FAKE), P(FAKE), ws_bytes, None)
+
+    def bwd(mask=FAKE, ws_bytes=big):
+        return lib.attnqat_sparse_bwd(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), 1, 1, 128, 128, 128,
+                                      0.125, 15, P(mask), P(FAKE), P(FAKE), P(FAKE), P(FAKE), ws_bytes, None)
+    assert fwd(mask=0) == A.EINVAL
+    assert fwd(q=0) == A.EINVAL
+    assert fwd(Lk=0) == A.EINVAL
+    # the dense workspace is too small for the tile lists
+    assert fwd(ws_bytes=A.attnqat_workspace_size(1, 1, 128, 128, 128, 15)) == A.ENOSPC
+    assert bwd(mask=0) == A.EINVAL
+    assert bwd(ws_bytes=A.attnqat_sparse_workspace_size(1, 1, 128, 128, 128, 15) - 1) == A.ENOSPC
