@@ -102,6 +102,8 @@ def _load():
             lib.oracle_bwd_dkdv_blocks.restype = None
             lib.oracle_bwd_dkdv_blocks.argtypes = [P, P, P, P, L, L, L, ctypes.c_double,
                                                    ctypes.c_uint, P, L, P, P, P, P, L, P, P]
+            lib.oracle_vsa_select.restype = None
+            lib.oracle_vsa_select.argtypes = [P, P, L, L, L, L, L, P, P]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -309,6 +311,24 @@ class Head:
         dQ = self.dq_rows()
         dK, dV = self.dkdv_blocks()
         return dQ, dK[: self.Lk], dV[: self.Lk]
+
+
+def vsa_select(q_bits, k_bits, topk, tile=128):
+    """Key-tile selection of block-sparse attention for one head (reading
+    R17 in oracle.c): tile means, float32 coarse scores, the topk best key
+    tiles per query tile (ties to the lower index).  q [Lq, D], k [Lk, D]
+    bf16 bits.  Returns (mask uint8 [nq, nk], scores float32 [nq, nk])."""
+    q = _bits(q_bits)
+    k = _bits(k_bits)
+    Lq, D = q.shape
+    Lk = k.shape[0]
+    if k.shape[1] != D or topk < 1 or tile < 1:
+        raise ValueError("q [Lq,D], k [Lk,D], topk >= 1 expected")
+    nq, nk = -(-Lq // tile), -(-Lk // tile)
+    mask = np.zeros((nq, nk), np.uint8)
+    scores = np.zeros((nq, nk), np.float32)
+    _load().oracle_vsa_select(_ptr(q), _ptr(k), Lq, Lk, D, tile, int(topk), _ptr(mask), _ptr(scores))
+    return mask, scores
 
 
 def attention(q_bits, k_bits, v_bits, sm_scale, flags=QUANT_ALL, do_bits=None, sel=None, tile=128):

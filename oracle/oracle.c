@@ -622,6 +622,74 @@ void oracle_bwd_dkdv_blocks(const double *Qh, const double *Kh, const double *Vh
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Block selection of the sparse attention (coarse scores, top-k)             */
+/* ------------------------------------------------------------------------ */
+
+/* VSA key-tile selection for one head (vsqa-test-1.3b metadata.json,
+ * "attention.selection": top-k key cubes per query cube with
+ * effective_topk = max(1, min(ceil((1 - sparsity) * num_blocks), num_blocks);
+ * "attention.precision.coarse": BF16, quantize_coarse false).  Reading (the
+ * page gives the fields, not the arithmetic; listed as R17): each T-token
+ * tile is summarised by the mean of its valid rows; the coarse score of
+ * (query tile I, key tile J) is the dot product of the two means (the softmax
+ * scale and the softmax itself do not change the order); query tile I keeps
+ * the topk key tiles of highest score, ties to the lower J.  The order
+ * decides an integer, so it is taken in the precision a B200 kernel computes
+ * it in, float32, with every step fixed: sum of the rows in token order (one
+ * float32 add per row), mean = sum / count (one correctly rounded float32
+ * division), score = the channels in order d = 0..D-1 accumulated with one
+ * fused multiply-add each from 0.  q: [Lq][D], k: [Lk][D] bf16.  Outputs
+ * mask [nq][nk] (1 = kept) and, if not NULL, the scores [nq][nk].          */
+static void tile_means_f32(const uint16_t *x, long L, long D, long T, float *mean)
+{
+    long nt = (L + T - 1) / T;
+    for (long t = 0; t < nt; t++) {
+        long r0 = t * T, r1 = r0 + T < L ? r0 + T : L;
+        for (long d = 0; d < D; d++) {
+            float s = 0.0f;
+            for (long r = r0; r < r1; r++)
+                s = s + (float)oracle_bf16_value(x[r * D + d]);
+            mean[t * D + d] = s / (float)(r1 - r0);
+        }
+    }
+}
+
+void oracle_vsa_select(const uint16_t *q, const uint16_t *k, long Lq, long Lk,
+                       long D, long T, long topk, uint8_t *mask, float *scores)
+{
+    long nq = (Lq + T - 1) / T, nk = (Lk + T - 1) / T;
+    float *qm = malloc(sizeof(float) * nq * D);
+    float *km = malloc(sizeof(float) * nk * D);
+    float *sc = malloc(sizeof(float) * nk);
+    tile_means_f32(q, Lq, D, T, qm);
+    tile_means_f32(k, Lk, D, T, km);
+    if (topk > nk)
+        topk = nk;
+    for (long i = 0; i < nq; i++) {
+        for (long j = 0; j < nk; j++) {
+            float acc = 0.0f;
+            for (long d = 0; d < D; d++)
+                acc = fmaf(qm[i * D + d], km[j * D + d], acc);
+            sc[j] = acc;
+            if (scores)
+                scores[i * nk + j] = acc;
+            mask[i * nk + j] = 0;
+        }
+        /* topk rounds of "the best tile not yet kept" */
+        for (long r = 0; r < topk; r++) {
+            long best = -1;
+            for (long j = 0; j < nk; j++)
+                if (!mask[i * nk + j] && (best < 0 || sc[j] > sc[best]))
+                    best = j;
+            mask[i * nk + best] = 1;
+        }
+    }
+    free(qm);
+    free(km);
+    free(sc);
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -585,6 +585,58 @@ def test_sparse_quantizers_off_vs_torch_masked_sdpa():
         assert np.max(np.abs(sp[name][0, 0] - ref)) <= 1e-10 * max(1.0, np.max(np.abs(ref))), name
 
 
+# ----------------------------------------------- sparse block selection ----
+
+def test_vsa_select_agrees_with_float64_ranking():
+    """Coarse scores within float32 rounding of the float64 tile-mean dot
+    products, and the kept set equal to the float64 top-k wherever the k-th
+    and (k+1)-th float64 scores are apart by more than the rounding."""
+    rng = np.random.default_rng(91)
+    Lq, Lk, D, T, topk = 300, 700, 64, 32, 5
+    q, k = _rand_bits(rng, (Lq, D)), _rand_bits(rng, (Lk, D))
+    mask, scores = oracle.vsa_select(q, k, topk, tile=T)
+    qf, kf = _f(q), _f(k)
+    qm = np.stack([qf[i:i + T].mean(0) for i in range(0, Lq, T)])
+    km = np.stack([kf[j:j + T].mean(0) for j in range(0, Lk, T)])
+    s64 = qm @ km.T
+    assert np.max(np.abs(scores - s64)) <= 1e-5 * np.max(np.abs(s64))
+    checked = 0
+    for i in range(s64.shape[0]):
+        order = np.argsort(-s64[i], kind="stable")
+        if s64[i, order[topk - 1]] - s64[i, order[topk]] > 1e-4 * np.max(np.abs(s64)):
+            want = np.zeros(s64.shape[1], np.uint8)
+            want[order[:topk]] = 1
+            assert np.array_equal(mask[i], want), i
+            checked += 1
+        assert mask[i].sum() == topk
+    assert checked >= s64.shape[0] - 1
+
+
+def test_vsa_select_ties_go_to_the_lower_tile_and_topk_bounds():
+    """Constant tiles: score = D * a_J exactly; equal scores keep the lower
+    key tile; topk = 1 is the argmax, topk >= the tile count keeps all."""
+    D, T = 16, 16
+    a = [1.0, 3.0, 3.0, 2.0, 3.0]
+    k = W.f32_to_bf16_bits(np.repeat(np.array(a, np.float32), T)[:, None] * np.ones((1, D), np.float32))
+    q = W.f32_to_bf16_bits(np.ones((T, D), np.float32))
+    mask, scores = oracle.vsa_select(q, k, 2, tile=T)
+    assert np.array_equal(scores[0], np.array(a, np.float32) * D)
+    assert np.array_equal(mask[0], [0, 1, 1, 0, 0])
+    assert np.array_equal(oracle.vsa_select(q, k, 1, tile=T)[0][0], [0, 1, 0, 0, 0])
+    assert np.all(oracle.vsa_select(q, k, 9, tile=T)[0] == 1)
+
+
+def test_vsa_select_ragged_tile_mean_uses_its_valid_rows():
+    """A ragged last key tile is averaged over its valid rows only: five rows
+    of 7 beat full tiles of 3 (zero-padding would average them to 2.19)."""
+    D, T = 16, 16
+    vals = np.concatenate([np.full(2 * T, 3.0), np.full(5, 7.0)]).astype(np.float32)
+    k = W.f32_to_bf16_bits(vals[:, None] * np.ones((1, D), np.float32))
+    q = W.f32_to_bf16_bits(np.ones((T, D), np.float32))
+    mask, scores = oracle.vsa_select(q, k, 1, tile=T)
+    assert np.array_equal(mask[0], [0, 0, 1]) and scores[0, 2] == 7.0 * D
+
+
 # ------------------------------------------ NVFP4 with an FP32 global scale ----
 
 def _bf16_value_fraction(h):
