@@ -17,10 +17,10 @@ events on the launching stream, and multi-GPU runs report the max over ranks.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sparsity S]
 
 --sparsity S times the block-sparse (VSA fine attention) step instead:
-attnqat_sparse_fwd + attnqat_sparse_bwd on the same shape, each 128-query tile
-attending max(1, min(ceil((1-S)*244), 244)) of the 244 key tiles (seeded
-selection; the pages' VSA checkpoint uses S = 0.9), with TFLOP/s counted on
-the selected tiles only.
+attnqat_vsa_select (the top max(1, min(ceil((1-S)*244), 244)) of the 244 key
+tiles per 128-query tile by coarse tile-mean scores; the pages' VSA checkpoint
+uses S = 0.9) + attnqat_sparse_fwd + attnqat_sparse_bwd on the same shape,
+with TFLOP/s counted on the selected tiles only.
 
 --impl reference times the float64 CPU oracle on the host cores instead (the
 pages ship no runnable implementation): each step is a bounded sample of the
@@ -191,11 +191,8 @@ def gpu_arm(args):
     peaks = load_peaks()
     sparse = args.sparsity is not None
     pairs = float(w.B * w.H * w.Lq * w.Lk)
-    if sparse:
-        mask_np = W.tile_mask(w, args.sparsity)
-        pairs = selected_pairs(w, mask_np)
-        fwd_f = 4.0 * pairs * w.D
-        flops = dict(fwd=fwd_f, bwd=2.5 * fwd_f, total=3.5 * fwd_f)
+    nq, nk = -(-w.Lq // W.SPARSE_TILE), -(-w.Lk // W.SPARSE_TILE)
+    topk = W.topk_tiles(nk, args.sparsity) if sparse else nk
 
     # seeded inputs (host), moved to the device once; the timed region starts
     # with them resident in HBM
@@ -205,10 +202,14 @@ def gpu_arm(args):
     c = w.sm_scale
     flags = A.QUANT_ALL
     if sparse:
-        tm = torch.from_numpy(mask_np).to(dev)
+        tm = torch.empty((w.B, w.H, nq, nk), dtype=torch.uint8, device=dev)
+        sel_ws = torch.empty(A.load().attnqat_vsa_select_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D),
+                             dtype=torch.uint8, device=dev)
         ws_bytes = A.attnqat_sparse_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags)
 
         def fwd(qq, kk, vv, out):
+            # the selection belongs to the forward: coarse scores, top-k tiles
+            A.attnqat_vsa_select(qq, kk, topk, out=tm, ws=sel_ws)
             return A.attnqat_sparse_fwd(qq, kk, vv, tm, sm_scale=c, flags=flags, ws=ws, out=out)
 
         def bwd(qq, kk, vv, ll, mm, dd, out):
@@ -238,6 +239,12 @@ def gpu_arm(args):
         step()
     torch.cuda.synchronize(dev)
     A.attnqat_device_status()
+    if sparse:
+        # the selection depends only on the inputs: count its pairs once
+        mask_np = tm.cpu().numpy()
+        pairs = selected_pairs(w, mask_np)
+        fwd_f = 4.0 * pairs * w.D
+        flops = dict(fwd=fwd_f, bwd=2.5 * fwd_f, total=3.5 * fwd_f)
 
     # ---- timed region: K steps, L2 flushed between steps, per-step events
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -302,7 +309,7 @@ def gpu_arm(args):
         config.update(workload="vsa_" + WORKLOAD, sparsity=args.sparsity, tile=W.SPARSE_TILE,
                       key_tiles_per_query_tile=int(mask_np.sum(-1).max()),
                       selected_fraction=round(pairs / (w.B * w.H * w.Lq * w.Lk), 5),
-                      selection="seeded uniform top-k of key tiles per query tile")
+                      selection="attnqat_vsa_select in the timed forward (tile means, top-%d coarse scores)" % topk)
     out = {
         "metric": SPARSE_METRIC % args.sparsity if sparse else METRIC,
         "value": round(value, 2),
@@ -334,15 +341,15 @@ def gpu_arm(args):
                      "peak_kind": "measured bf16 sustained (kernel timed inside a long step)"
                      if peaks["source"] == "measured" else "fallback"},
         "kernels": kernel_table,
-        "gpu_launches": len(kernels),
+        # every profiled scope is one kernel launch except the selection (two)
+        "gpu_launches": len(kernels) + sum(1 for n, _ in kernels if n == "vsa_select"),
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall, 3),
         "e2e": e2e,
     }
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline_sample(rows=BASELINE_SAMPLE_ROWS,
-                                                      sel=mask_np[0, 0] if sparse else None)
+            out["cpu_baseline"] = cpu_baseline_sample(rows=BASELINE_SAMPLE_ROWS, topk=topk if sparse else None)
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
@@ -410,12 +417,13 @@ def load_traffic(kernel):
 
 # -------------------------------------------------------------- CPU oracle --
 
-def cpu_baseline_sample(rows: int, sel=None):
+def cpu_baseline_sample(rows: int, topk=None):
     """The float64 oracle on a bounded sample of the workload: head 0, the
     first `rows` query rows against all 31200 keys, forward and backward
     (dQ for those rows, their dK/dV contributions for every key).  Returns the
-    nominal TFLOP/s of that sub-problem (with a tile selection `sel` of head
-    0: block-sparse, counted on the selected keys)."""
+    nominal TFLOP/s of that sub-problem.  With `topk`, block-sparse: the
+    oracle's own selection of head 0 (inside the timed sample), counted on
+    the selected keys."""
     import oracle
     w = W.get(WORKLOAD)
     q = W.head_bits(w, "q", 0, 0)[:rows]
@@ -423,9 +431,10 @@ def cpu_baseline_sample(rows: int, sel=None):
     v = W.head_bits(w, "v", 0, 0)
     do = W.head_bits(w, "do", 0, 0)[:rows]
     T = W.SPARSE_TILE
-    if sel is not None:
-        sel = sel[: -(-rows // T)]
     t0 = time.perf_counter()
+    sel = None
+    if topk is not None:
+        sel = oracle.vsa_select(W.head_bits(w, "q", 0, 0), k, topk, tile=T)[0][: -(-rows // T)]
     hd = oracle.Head(q, k, v, w.sm_scale, oracle.QUANT_ALL, do, sel=sel, tile=T)
     hd.stats()
     hd.backward()

@@ -256,6 +256,37 @@ int attnqat_sparse_bwd(const void *q, const void *k, const void *v,
                        void *stream);
 
 /*
+ * attnqat_vsa_select -- the key tiles each query tile of the block-sparse
+ * attention attends to (the tile mask attnqat_sparse_fwd takes).
+ *
+ * Defined by: vsqa-test-1.3b metadata.json, "attention.selection": top-k key
+ * cubes per query cube, effective_topk = max(1, min(ceil((1 - sparsity) *
+ * num_blocks), num_blocks)) at sparsity 0.9 (the "top-p" mode field stands
+ * beside that count); "attention.precision.coarse": BF16, not quantized.
+ * The page names the fields, not the arithmetic; read as: each 128-token tile
+ * is summarised by the mean of its valid rows; the coarse score of (query tile
+ * I, key tile J) is the dot product of the two means (a softmax and its scale
+ * keep the order); query tile I keeps the `topk` key tiles of highest score,
+ * ties to the lower J (topk above the tile count keeps every tile).  The
+ * ranking is computed in float32 with every step ordered -- rows summed in
+ * token order, one correctly rounded division by the row count, channels
+ * accumulated in order with one fused multiply-add each -- so it is
+ * reproducible bit for bit.
+ *
+ * q [B,H,Lq,D], k [B,H,Lk,D] bf16 (16-byte aligned); topk >= 1 (the caller
+ * evaluates the page's effective_topk); tile_mask: device bytes
+ * [B][H][ceil(Lq/128)][ceil(Lk/128)], written with 0 or 1.  ws: device
+ * workspace of attnqat_vsa_select_workspace_size() bytes, 256-byte aligned
+ * (tile means and scores).  Two launches on `stream`.  Inputs must be finite.
+ * Errors: EINVAL (null or misaligned pointer, bad shape, topk < 1),
+ * EUNSUPPORTED, ENOSPC, ECUDA.
+ */
+size_t attnqat_vsa_select_workspace_size(int B, int H, int Lq, int Lk, int D);
+int attnqat_vsa_select(const void *q, const void *k, int B, int H, int Lq,
+                       int Lk, int D, int topk, uint8_t *tile_mask, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/*
  * attnqat_fwd_noalloc -- attnqat_fwd for callers that cannot allocate.
  *
  * The pages have no counterpart of this entry point; it exists for callers

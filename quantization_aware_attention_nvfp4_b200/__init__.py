@@ -20,6 +20,8 @@ Entry points (same names as the C ABI):
   block-sparse (VSA fine attention) variants: ``tile_mask`` is a uint8 CUDA
   tensor [B, H, ceil(Lq/128), ceil(Lk/128)], nonzero where a 128-query tile
   attends a 128-key tile.
+* ``attnqat_vsa_select(q, k, topk)`` -- that mask from the coarse scores of
+  the tiles' means: the ``topk`` best key tiles per query tile.
 
 ``sm_scale=None`` means 1/sqrt(D), chosen here and passed explicitly; the
 library itself never substitutes a default (FastVideo PR #1457 review, F1).
@@ -90,6 +92,10 @@ def load(build_if_needed: bool = True):
             lib.attnqat_fwd.argtypes = [P, P, P, I, I, I, I, I, F, U32, P, P, P, P, SZ, P]
             lib.attnqat_bwd.restype = I
             lib.attnqat_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, U32, P, P, P, P, SZ, P]
+            lib.attnqat_vsa_select_workspace_size.restype = SZ
+            lib.attnqat_vsa_select_workspace_size.argtypes = [I, I, I, I, I]
+            lib.attnqat_vsa_select.restype = I
+            lib.attnqat_vsa_select.argtypes = [P, P, I, I, I, I, I, I, P, P, SZ, P]
             lib.attnqat_sparse_workspace_size.restype = SZ
             lib.attnqat_sparse_workspace_size.argtypes = [I, I, I, I, I, U32]
             lib.attnqat_sparse_fwd.restype = I
@@ -271,6 +277,38 @@ def _tile_mask(tile_mask, B, H, Lq, Lk, device):
             tile_mask.device != device or tuple(tile_mask.shape) != want or not tile_mask.is_contiguous():
         raise ValueError("tile_mask must be a contiguous uint8 tensor %s on %s" % (want, device))
     return ctypes.c_void_p(tile_mask.data_ptr())
+
+
+def attnqat_vsa_select(q, k, topk, out=None, ws=None, stream=None):
+    """Key tiles per query tile for the block-sparse attention: the ``topk``
+    key tiles whose mean row scores highest against the query tile's mean row
+    (ties to the lower tile).  ``q`` [B, H, Lq, D], ``k`` [B, H, Lk, D] bf16
+    CUDA tensors.  Returns the uint8 tile mask [B, H, ceil(Lq/128),
+    ceil(Lk/128)] (``out`` if given)."""
+    torch = _torch()
+    for n, t in (("q", q), ("k", k)):
+        _require_bf16_cuda(n, t, 4)
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous [B, H, L, D]" % n)
+    B, H, Lq, D = q.shape
+    Lk = k.shape[2]
+    if k.shape[0] != B or k.shape[1] != H or k.shape[3] != D:
+        raise ValueError("k must be [B, H, Lk, D] matching q [B, H, Lq, D]")
+    need = int(load().attnqat_vsa_select_workspace_size(B, H, Lq, Lk, D))
+    if need == 0:
+        _check(EINVAL, "attnqat_vsa_select_workspace_size")
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, H, -(-Lq // SPARSE_TILE), -(-Lk // SPARSE_TILE)), dtype=torch.uint8,
+                          device=q.device)
+    else:
+        _tile_mask(out, B, H, Lq, Lk, q.device)
+    st = load().attnqat_vsa_select(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), B, H, Lq, Lk, D,
+                                   int(topk), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                   ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "attnqat_vsa_select")
+    return out
 
 
 def attnqat_sparse_fwd(q, k, v, tile_mask, sm_scale=None, flags=QUANT_ALL, ws=None, out=None, stream=None):

@@ -620,6 +620,35 @@ int attnqat_sparse_fwd(const void *q, const void *k, const void *v, int B, int H
   return run_fwd(q, k, v, B, H, Lq, Lk, D, sm_scale, flags, tile_mask, o, lse, m, ws, ws_bytes, stream);
 }
 
+size_t attnqat_vsa_select_workspace_size(int B, int H, int Lq, int Lk, int D) {
+  if (check_shape(B, H, Lq, Lk, D, 1.0f, 0) != ATTNQAT_OK) return 0;
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t nq = (static_cast<size_t>(Lq) + kBM - 1) / kBM, nk = (static_cast<size_t>(Lk) + kBN - 1) / kBN;
+  return align256(BH * (nq + nk) * D * 4) + align256(BH * nq * nk * 4);
+}
+
+int attnqat_vsa_select(const void *q, const void *k, int B, int H, int Lq, int Lk, int D, int topk,
+                       uint8_t *tile_mask, void *ws, size_t ws_bytes, void *stream) {
+  int st = check_shape(B, H, Lq, Lk, D, 1.0f, 0);
+  if (st != ATTNQAT_OK) return st;
+  if (!q || !k || !tile_mask || !ws || topk < 1) return ATTNQAT_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return ATTNQAT_EINVAL;
+  const size_t need = attnqat_vsa_select_workspace_size(B, H, Lq, Lk, D);
+  if (ws_bytes < need) return ATTNQAT_ENOSPC;
+  st = check_device();
+  if (st != ATTNQAT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t nq = (static_cast<size_t>(Lq) + kBM - 1) / kBM, nk = (static_cast<size_t>(Lk) + kBN - 1) / kBN;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  float *means = reinterpret_cast<float *>(wsb);
+  float *scores = reinterpret_cast<float *>(wsb + align256(BH * (nq + nk) * D * 4));
+  ProfScope ps("vsa_select", s);
+  const cudaError_t e = launch_vsa_select(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                                          B * H, Lq, Lk, D, topk, means, scores, tile_mask, s);
+  return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
+}
+
 int attnqat_sparse_bwd(const void *q, const void *k, const void *v, const float *lse, const float *m,
                        const void *dO, int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags,
                        const uint8_t *tile_mask, void *dq, void *dk, void *dv, void *ws, size_t ws_bytes,

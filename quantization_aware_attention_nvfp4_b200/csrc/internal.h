@@ -110,6 +110,12 @@ cudaError_t launch_scale_do(const __nv_bfloat16 *dO, uint16_t *out, int64_t n, c
 cudaError_t launch_sparse_plan(const uint8_t *mask, int BH, int nq, int nk, int32_t *kv_list, int32_t *kv_count,
                                int32_t *q_list, int32_t *q_count, cudaStream_t stream);
 
+// VSA key-tile selection (see sparse.cu): tile means of q and k into
+// `means` [BH][nq + nk][D], coarse scores into `scores` [BH][nq][nk], and the
+// tile mask [BH][nq][nk] keeping the topk best key tiles per query tile.
+cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D,
+                              int topk, float *means, float *scores, uint8_t *mask, cudaStream_t stream);
+
 // max |x| over n bf16 values folded into *out (must start at 0).
 cudaError_t launch_absmax(const __nv_bfloat16 *x, int64_t n, float *out, cudaStream_t stream);
 

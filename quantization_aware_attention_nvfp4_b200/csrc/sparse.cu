@@ -67,4 +67,102 @@ cudaError_t launch_sparse_plan(const uint8_t *mask, int BH, int nq, int nk, int3
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------ key-tile selection --
+//
+// VSA selection (vsqa-test-1.3b metadata.json, "attention.selection": top-k
+// key cubes per query cube; "precision.coarse": BF16, unquantized).  Each
+// 128-token tile is summarised by the mean of its valid rows, the coarse
+// score of (query tile I, key tile J) is the dot product of the two means,
+// and query tile I keeps the topk key tiles of highest score, ties to the
+// lower J.  The ranking decides integers, so every step has a fixed float32
+// order: rows summed in token order, one correctly rounded division by the
+// row count, channels accumulated in order with one fused multiply-add each.
+
+// One CTA per (tile, head), one thread per channel: means[bh][t][d], tiles
+// t < nq of q, then nk tiles of k.  The row loop reads one 2*D-byte row per
+// step, coalesced across the CTA.
+__global__ void __launch_bounds__(128) tile_mean_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                        const __nv_bfloat16 *__restrict__ k, int Lq, int Lk,
+                                                        int D, int nq, int nk, float *__restrict__ means) {
+  const int t = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int d = threadIdx.x;
+  const bool isq = t < nq;
+  const int L = isq ? Lq : Lk;
+  const int r0 = (isq ? t : t - nq) * kBM;
+  const int r1 = r0 + kBM < L ? r0 + kBM : L;
+  const __nv_bfloat16 *x = (isq ? q : k) + static_cast<size_t>(bh) * L * D + d;
+  float s = 0.0f;
+#pragma unroll 8
+  for (int r = r0; r < r1; ++r) s = __fadd_rn(s, __bfloat162float(x[static_cast<size_t>(r) * D]));
+  means[(static_cast<size_t>(bh) * (nq + nk) + t) * D + d] = __fdiv_rn(s, static_cast<float>(r1 - r0));
+}
+
+// One warp per (head, query tile): the nk coarse scores into `scores`, then
+// topk rounds of a warp-wide argmax (score descending, tile ascending) over
+// the tiles not yet kept.  The mask row is written here (0 or 1 per tile).
+__global__ void __launch_bounds__(128) tile_select_kernel(const float *__restrict__ means, int BH, int nq, int nk,
+                                                          int D, int topk, float *__restrict__ scores,
+                                                          uint8_t *__restrict__ mask) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<int64_t>(BH) * nq) return;  // warp-uniform
+  const int64_t bh = w / nq;
+  const int I = static_cast<int>(w - bh * nq);
+  const float4 *qm = reinterpret_cast<const float4 *>(means + (bh * (nq + nk) + I) * D);
+  const float *km = means + (bh * (nq + nk) + nq) * D;
+  float *sc = scores + w * nk;
+  uint8_t *mk = mask + w * nk;
+  for (int j = lane; j < nk; j += 32) {
+    const float4 *kr = reinterpret_cast<const float4 *>(km + static_cast<size_t>(j) * D);
+    float acc = 0.0f;
+    for (int c = 0; c < D / 4; ++c) {
+      const float4 a = qm[c], b = kr[c];
+      acc = __fmaf_rn(a.x, b.x, acc);
+      acc = __fmaf_rn(a.y, b.y, acc);
+      acc = __fmaf_rn(a.z, b.z, acc);
+      acc = __fmaf_rn(a.w, b.w, acc);
+    }
+    sc[j] = acc;
+    mk[j] = 0;
+  }
+  __syncwarp();
+  const int kk = topk < nk ? topk : nk;
+  for (int r = 0; r < kk; ++r) {
+    float best = 0.0f;
+    int bj = -1;  // -1: no candidate
+    for (int j = lane; j < nk; j += 32) {
+      if (mk[j]) continue;
+      const float v = sc[j];
+      if (bj < 0 || v > best) {  // ascending j: equal scores keep the lower tile
+        best = v;
+        bj = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      if (oj >= 0 && (bj < 0 || ov > best || (ov == best && oj < bj))) {
+        best = ov;
+        bj = oj;
+      }
+    }
+    if (lane == 0 && bj >= 0 && bj < nk) mk[bj] = 1;
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D,
+                              int topk, float *means, float *scores, uint8_t *mask, cudaStream_t stream) {
+  const int nq = (Lq + kBM - 1) / kBM, nk = (Lk + kBN - 1) / kBN;
+  tile_mean_kernel<<<dim3(nq + nk, BH), D, 0, stream>>>(q, k, Lq, Lk, D, nq, nk, means);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (static_cast<int64_t>(BH) * nq * 32 + 127) / 128;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  tile_select_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(means, BH, nq, nk, D, topk, scores, mask);
+  return cudaGetLastError();
+}
+
 }  // namespace attnqat

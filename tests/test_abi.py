@@ -180,3 +180,23 @@ def test_sparse_host_validation():
     assert fwd(ws_bytes=A.attnqat_workspace_size(1, 1, 128, 128, 128, 15)) == A.ENOSPC
     assert bwd(mask=0) == A.EINVAL
     assert bwd(ws_bytes=A.attnqat_sparse_workspace_size(1, 1, 128, 128, 128, 15) - 1) == A.ENOSPC
+
+
+def test_vsa_select_host_validation_and_workspace():
+    lib = A.load()
+    al = lambda x: (x + 255) // 256 * 256
+    B, H, Lq, Lk, D = 1, 6, 31200, 31200, 128
+    nq = nk = 244
+    assert A.load().attnqat_vsa_select_workspace_size(B, H, Lq, Lk, D) == \
+        al(B * H * (nq + nk) * D * 4) + al(B * H * nq * nk * 4)
+    assert A.load().attnqat_vsa_select_workspace_size(1, 1, 16, 16, 96) == 0
+    big = 1 << 30
+
+    def sel(q=FAKE, topk=3, mask=FAKE, ws=FAKE, ws_bytes=big, D=128):
+        return lib.attnqat_vsa_select(P(q), P(FAKE), 1, 1, 300, 700, D, topk, P(mask), P(ws), ws_bytes, None)
+    assert sel(q=0) == A.EINVAL
+    assert sel(mask=0) == A.EINVAL
+    assert sel(topk=0) == A.EINVAL
+    assert sel(ws=FAKE + 16) == A.EINVAL
+    assert sel(D=96) == A.EUNSUPPORTED
+    assert sel(ws_bytes=lib.attnqat_vsa_select_workspace_size(1, 1, 300, 700, 128) - 1) == A.ENOSPC

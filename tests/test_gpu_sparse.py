@@ -1,6 +1,8 @@
 """Parity of the block-sparse (VSA fine attention) CUDA path --
 attnqat_sparse_fwd / attnqat_sparse_bwd through the C ABI -- with the float64
-oracle restricted to the same tile selection.
+oracle restricted to the same tile selection, and of the key-tile selection
+attnqat_vsa_select with the oracle's (bit-exact: both rank in float32 with
+the same fixed order of operations).
 
 Bar: as for dense attention (relative L2 <= 1e-2, max-abs <= 5e-2 of the
 oracle's RMS).  Rows of a query tile with no selected key tile must be exactly
@@ -149,3 +151,38 @@ def test_vsa_wan_6h_31200_sparsity_09_sampled():
     w = W.get("wan_6h_31200")
     _sampled_compare(w, W.tile_mask(w, 0.9), heads=[(0, 0), (0, w.H - 1)], n_rows=48, n_blocks=48,
                      tag=" vsa")
+
+
+@pytest.mark.parametrize("B,H,Lq,Lk,D,topk", [
+    (1, 2, 1000, 1100, 128, 3),
+    (2, 1, 300, 700, 64, 2),
+    (1, 1, 130, 90, 128, 5),        # topk above the tile count: every tile
+    (1, 6, 31200, 31200, 128, 25),  # the pages' shape at sparsity 0.9
+])
+def test_vsa_select_matches_oracle(B, H, Lq, Lk, D, topk):
+    import torch
+    w = W.custom(B, H, Lq, Lk, D, seed_index=820 + D + topk)
+    inp = W.inputs(w, with_grad=False)
+    q, k = to_gpu_bf16(inp["q"]), to_gpu_bf16(inp["k"])
+    mask = A.attnqat_vsa_select(q, k, topk)
+    torch.cuda.synchronize()
+    got = mask.cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            want, _ = oracle.vsa_select(inp["q"][b, h], inp["k"][b, h], topk, tile=W.SPARSE_TILE)
+            assert np.array_equal(got[b, h], want), (b, h)
+    assert np.all(got.sum(-1) == min(topk, got.shape[-1]))
+
+
+def test_selection_feeds_sparse_attention():
+    """The whole VSA fine path: attnqat_vsa_select's mask into the sparse
+    forward and backward, against the oracle run on the oracle's own mask."""
+    import torch
+    w = W.custom(1, 2, 900, 1000, 128, seed_index=830)
+    inp = W.inputs(w)
+    q, k = to_gpu_bf16(inp["q"]), to_gpu_bf16(inp["k"])
+    topk = W.topk_tiles(-(-w.Lk // W.SPARSE_TILE), 0.7)
+    mask = A.attnqat_vsa_select(q, k, topk).cpu().numpy()
+    want = np.stack([np.stack([oracle.vsa_select(inp["q"][0, h], inp["k"][0, h], topk)[0] for h in range(2)])])
+    assert np.array_equal(mask, want)
+    _full_compare(w, want, oracle.QUANT_ALL)
