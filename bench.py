@@ -400,7 +400,7 @@ def e2e_arm(args, torch, dev, host, w, flops, fwd, bwd, world):
 
 def load_traffic(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
-    summary was taken on the current kernel sources (else null)."""
+    summary was taken on the current attention kernel sources (else null)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -408,7 +408,7 @@ def load_traffic(kernel):
         d = json.load(open(path))
         from quantization_aware_attention_nvfp4_b200 import build as B
         rec = d.get(kernel)
-        if not rec or rec.get("sources_sha") != B.sources_digest():
+        if not rec or rec.get("sources_sha") != B.attention_sources_digest():
             return None
         return rec.get("dram_bytes_per_launch")
     except Exception:

@@ -44,6 +44,21 @@ def sources_digest() -> str:
     return h.hexdigest()[:16]
 
 
+# The files that determine the attention kernels' code (their ncu counters
+# stay valid while these are unchanged).
+ATTENTION_SOURCES = ("fwd.cu", "bwd.cu", "common.cuh", "device.cuh", "internal.h")
+
+
+def attention_sources_digest() -> str:
+    """SHA-256 over the attention kernels' own sources."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ATTENTION_SOURCES:
+        h.update(name.encode())
+        h.update(open(os.path.join(CSRC, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def stale() -> bool:
     if not os.path.exists(LIB):
         return True

@@ -13,7 +13,10 @@
 // rounding cannot move it across one.  The E2M1 code is chosen by comparing
 // |x| with the products m_k * s at the 7 midpoints m_k of the grid, which
 // are exact in float (at most 7 significant bits), so ties are detected
-// exactly and resolved to the even code.
+// exactly and resolved to the even code; three comparisons of a binary search
+// over the midpoints select it.  The dequantized value is the code's E2M1
+// magnitude converted by the hardware (exact) times s in f16 (exact: at most
+// 7 significant bits in [2^-10, 2688]) with the input's sign bit.
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,19 +27,35 @@ __device__ __forceinline__ uint32_t e4m3_scale_code(float amax) {
   return cvt_e4m3x2(t, 0.0f) & 0xFFu;
 }
 
-// E2M1 magnitude code of |x| at scale s > 0 (round to nearest even,
-// saturating at 6).  Crossing midpoint k (between codes k and k+1) needs '>'
-// when k is even and '>=' when k is odd.
-__device__ __forceinline__ uint32_t e2m1_code_exact(float ax, float s) {
-  uint32_t c = 0;
-  c += ax > 0.25f * s;
-  c += ax >= 0.75f * s;
-  c += ax > 1.25f * s;
-  c += ax >= 1.75f * s;
-  c += ax > 2.5f * s;
-  c += ax >= 3.5f * s;
-  c += ax > 5.0f * s;
-  return c;
+// E2M1 magnitude code of |x| (round to nearest even, saturating at 6) from
+// the scaled midpoints t[k] = m_k * s, m = {.25, .75, 1.25, 1.75, 2.5, 3.5,
+// 5}, s > 0: the code is the number of midpoints |x| crosses, and crossing
+// midpoint k (between codes k and k+1) needs '>' when k is even and '>='
+// when k is odd.  Binary search: midpoint 3, then 1 or 5, then the even one.
+__device__ __forceinline__ uint32_t e2m1_code_exact(float ax, const float (&t)[7]) {
+  uint32_t c = ax >= t[3] ? 4u : 0u;
+  c += ax >= (c ? t[5] : t[1]) ? 2u : 0u;
+  const float te = (c & 4u) ? ((c & 2u) ? t[6] : t[4]) : ((c & 2u) ? t[2] : t[0]);
+  return c + (ax > te ? 1u : 0u);
+}
+
+// f16x2 of the two E2M1 codes in the low byte of `byte` (low nibble -> low
+// half); exact.
+__device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "mov.b32 {t0, t1, t2, t3}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t0;\n\t}"
+      : "=r"(r)
+      : "r"(byte));
+  return r;
+}
+
+// bf16x2 bits of an f16x2 word whose values have at most 8 significant bits
+// (exact: the float32 bits truncated to their upper half).
+__device__ __forceinline__ uint32_t bf16x2_from_f16x2_exact(uint32_t h) {
+  const float2 f = unpack_f16x2(h);
+  return (__float_as_uint(f.x) >> 16) | (__float_as_uint(f.y) & 0xFFFF0000u);
 }
 
 // Magnitude of E2M1 code c (0..7): 0, .5, 1, 1.5, 2, 3, 4, 6.
@@ -45,33 +64,53 @@ __device__ __forceinline__ float e2m1_magnitude(uint32_t c) {
   return c < 4 ? 0.5f * fc : (c < 6 ? fc - 2.0f : 2.0f * fc - 8.0f);
 }
 
-// fq of 16 bf16 values (bit patterns in v[]): packed nibbles (element 2i in
-// the low nibble of byte i, 8 bytes as two words), the scale code, and the
-// dequantized values as bf16 and f16 bit patterns.  sign * E2M1 * s has at
-// most 7 significant bits and lies in [2^-10, 2688] when nonzero, so the
-// float product and both 16-bit forms are exact.
-__device__ __forceinline__ void fq16_exact(const uint16_t (&v)[16], uint32_t (&nib)[2], uint32_t &scode,
-                                           uint16_t (&deq_bf16)[16], uint16_t (&deq_f16)[16]) {
+// fq of 16 bf16 values (w[i]: elements 2i and 2i+1 as the low and high
+// halves): packed nibbles (element 2i in the low nibble of byte i, 8 bytes as
+// two words; nibble = the input's sign bit | the magnitude code), the scale
+// code, the dequantized values as f16x2 words (same pairing as w), and the
+// largest dequantized magnitude of the block.
+__device__ __forceinline__ void fq16_exact(const uint32_t (&w)[8], uint32_t (&nib)[2], uint32_t &scode,
+                                           uint32_t (&h16)[8], float &dmax) {
   float ax[16];
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    ax[i] = fabsf(__uint_as_float(static_cast<uint32_t>(v[i]) << 16));
-    amax = fmaxf(amax, ax[i]);
+  for (int i = 0; i < 8; ++i) {
+    ax[2 * i] = __uint_as_float((w[i] << 16) & 0x7FFF0000u);
+    ax[2 * i + 1] = __uint_as_float(w[i] & 0x7FFF0000u);
+    amax = fmax3(amax, ax[2 * i], ax[2 * i + 1]);
   }
   scode = e4m3_scale_code(amax);
   const uint32_t s_h2 = cvt_f16x2_from_e4m3x2(static_cast<uint16_t>(scode | (scode << 8)));
   const float s = unpack_f16x2(s_h2).x;
+  const float t[7] = {0.25f * s, 0.75f * s, 1.25f * s, 1.75f * s, 2.5f * s, 3.5f * s, 5.0f * s};
   nib[0] = nib[1] = 0u;
+  if (s > 0.0f) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t c = s > 0.0f ? e2m1_code_exact(ax[i], s) : 0u;
-    const uint32_t sign = static_cast<uint32_t>(v[i]) & 0x8000u;
-    nib[i >> 3] |= (c | (sign >> 12)) << (4 * (i & 7));
-    const float mag = e2m1_magnitude(c) * s;
-    const uint32_t f = __float_as_uint(mag) | (sign << 16);
-    deq_bf16[i] = static_cast<uint16_t>(f >> 16);
-    deq_f16[i] = __half_as_ushort(__float2half_rn(__uint_as_float(f)));
+    for (int i = 0; i < 16; ++i) nib[i >> 3] |= e2m1_code_exact(ax[i], t) << (4 * (i & 7));
+  }
+  dmax = s > 0.0f ? e2m1_magnitude(e2m1_code_exact(amax, t)) * s : 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t byte = (nib[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+    h16[j] = hmul2_u32(f16x2_from_e2m1x2(byte), s_h2) | (w[j] & 0x80008000u);
+    // the sign bits join the codes: bit 15 -> bit 3, bit 31 -> bit 7 of the byte
+    nib[j >> 2] |= (((w[j] >> 12) & 0x8u) | ((w[j] >> 24) & 0x80u)) << (8 * (j & 3));
+  }
+}
+
+// Stores the first n (<= 16) of the 16 16-bit values held as 8 pairs at
+// dst[base + i*sc] (two 16-byte stores when all 16 are stored, contiguous
+// and aligned).
+__device__ __forceinline__ void store16w(uint16_t *dst, int64_t base, int64_t sc, const uint32_t (&h)[8],
+                                         int n = 16) {
+  if (n == 16 && sc == 1 && (reinterpret_cast<uintptr_t>(dst + base) & 15u) == 0) {
+    uint4 *p = reinterpret_cast<uint4 *>(dst + base);
+    p[0] = make_uint4(h[0], h[1], h[2], h[3]);
+    p[1] = make_uint4(h[4], h[5], h[6], h[7]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < n) dst[base + i * sc] = static_cast<uint16_t>(h[i >> 1] >> (16 * (i & 1)));
   }
 }
 
@@ -142,24 +181,23 @@ __global__ void __launch_bounds__(256)
     }
     const int64_t base = z * sb + r * sr + b * 16 * sc;
     const int n = static_cast<int>(cols - b * 16 < 16 ? cols - b * 16 : 16);
-    uint16_t v[16];
+    uint32_t w[8];
     const bool vec = n == 16 && (sc == 1) && ((reinterpret_cast<uintptr_t>(x + base) & 15u) == 0);
     if (vec) {
       const uint4 *p = reinterpret_cast<const uint4 *>(x + base);
       const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
-      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[2 * i] = static_cast<uint16_t>(w[i] & 0xFFFFu);
-        v[2 * i + 1] = static_cast<uint16_t>(w[i] >> 16);
-      }
+      w[0] = u0.x, w[1] = u0.y, w[2] = u0.z, w[3] = u0.w, w[4] = u1.x, w[5] = u1.y, w[6] = u1.z, w[7] = u1.w;
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = i < n ? __ldg(x + base + i * sc) : static_cast<uint16_t>(0);
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t lo = 2 * i < n ? __ldg(x + base + 2 * i * sc) : 0u;
+        const uint32_t hi = 2 * i + 1 < n ? __ldg(x + base + (2 * i + 1) * sc) : 0u;
+        w[i] = lo | (hi << 16);
+      }
     }
-    uint32_t nib[2], scode;
-    uint16_t bb[16], hb[16];
-    fq16_exact(v, nib, scode, bb, hb);
+    uint32_t nib[2], scode, hb[8];
+    float dmax;
+    fq16_exact(w, nib, scode, hb, dmax);
     const int64_t blk = (z * rows + r) * nblk + b;
     if (codes) *reinterpret_cast<uint2 *>(codes + blk * 8) = make_uint2(nib[0], nib[1]);
     if (scales) {
@@ -186,14 +224,118 @@ __global__ void __launch_bounds__(256)
         scales[blk] = static_cast<uint8_t>(scode);
       }
     }
-    if (deq) store16(deq, base, sc, bb, n);
-    if (deq_f16) store16(deq_f16, base, sc, hb, n);
-    if (absmax) {
+    if (deq) {
+      uint32_t bb[8];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) vmax = fmaxf(vmax, fabsf(__uint_as_float(static_cast<uint32_t>(bb[i]) << 16)));
+      for (int i = 0; i < 8; ++i) bb[i] = bf16x2_from_f16x2_exact(hb[i]);
+      store16w(deq, base, sc, bb, n);
     }
+    if (deq_f16) store16w(deq_f16, base, sc, hb, n);
+    vmax = fmaxf(vmax, dmax);
   }
   if (absmax) block_max_to_global(vmax, absmax);
+}
+
+// The two views the attention quantizes, with the heads on grid.y so that no
+// thread divides by a runtime value (the general kernel above spends more
+// instructions on 64-bit index division than on the quantization).
+//
+// Rows of D contiguous elements, blocks along the row (Q, K: [heads][L][D],
+// 16-byte aligned): one thread per block, 32 contiguous bytes in, the same
+// out.  Scales plain ([row][D/16]) or, with `tiled`, in the per-128-row-tile
+// layout of the general kernel's sf_tile_rows mode (L = sf_tile_rows).
+template <int D>
+__global__ void __launch_bounds__(256)
+    quantize_rows_kernel(const uint16_t *__restrict__ x, int64_t L, uint8_t *__restrict__ codes,
+                         uint8_t *__restrict__ scales, bool tiled, uint16_t *__restrict__ deq,
+                         uint16_t *__restrict__ deq_f16) {
+  constexpr int NB = D / 16;
+  const int64_t id = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const int64_t t = id / NB;
+  const int b = static_cast<int>(id % NB);
+  if (t >= L) return;
+  const int64_t head = blockIdx.y;
+  const int64_t row = head * L + t;
+  const uint4 *p = reinterpret_cast<const uint4 *>(x + row * D + b * 16);
+  const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  uint32_t nib[2], scode, hb[8];
+  float dmax;
+  fq16_exact(w, nib, scode, hb, dmax);
+  if (codes) *reinterpret_cast<uint2 *>(codes + (row * NB + b) * 8) = make_uint2(nib[0], nib[1]);
+  if (scales) {
+    if (tiled) {
+      const int64_t ntiles = (L + 127) >> 7;
+      scales[((head * ntiles + (t >> 7)) * (NB >> 2) + (b >> 2)) * 512 + (t & 31) * 16 + ((t & 127) >> 5) * 4 +
+             (b & 3)] = static_cast<uint8_t>(scode);
+    } else {
+      scales[row * NB + b] = static_cast<uint8_t>(scode);
+    }
+  }
+  if (deq) {
+    uint4 *q = reinterpret_cast<uint4 *>(deq + row * D + b * 16);
+    q[0] = make_uint4(bf16x2_from_f16x2_exact(hb[0]), bf16x2_from_f16x2_exact(hb[1]), bf16x2_from_f16x2_exact(hb[2]),
+                      bf16x2_from_f16x2_exact(hb[3]));
+    q[1] = make_uint4(bf16x2_from_f16x2_exact(hb[4]), bf16x2_from_f16x2_exact(hb[5]), bf16x2_from_f16x2_exact(hb[6]),
+                      bf16x2_from_f16x2_exact(hb[7]));
+  }
+  if (deq_f16) {
+    uint4 *q = reinterpret_cast<uint4 *>(deq_f16 + row * D + b * 16);
+    q[0] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+    q[1] = make_uint4(hb[4], hb[5], hb[6], hb[7]);
+  }
+}
+
+// Blocks of 16 consecutive tokens per channel of a [heads][L][D] tensor (V):
+// thread (channel r, token block b), consecutive threads on consecutive
+// channels, so each of the 16 loads and stores of a warp covers 64
+// contiguous bytes.  A ragged last block reads zeros past L.  Codes and
+// scales plain ([head][r][blocks]) or, with `tiled`, scales in the
+// per-128-token-tile layout of the general kernel's sf_col_tiles mode.
+template <int D>
+__global__ void __launch_bounds__(256)
+    quantize_tokens_kernel(const uint16_t *__restrict__ x, int64_t L, uint8_t *__restrict__ codes,
+                           uint8_t *__restrict__ scales, bool tiled, uint16_t *__restrict__ deq,
+                           uint16_t *__restrict__ deq_f16, float *__restrict__ absmax) {
+  const int64_t nblk = (L + 15) >> 4;
+  const int64_t id = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const int r = static_cast<int>(id % D);
+  const int64_t b = id / D;
+  float dmax = 0.0f;
+  if (b < nblk) {  // no early return: every thread joins the block max below
+    const int64_t z = blockIdx.y;
+    const int64_t base = (z * L + b * 16) * D + r;
+    const int n = static_cast<int>(L - b * 16 < 16 ? L - b * 16 : 16);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t lo = 2 * i < n ? __ldg(x + base + (2 * i) * D) : 0u;
+      const uint32_t hi = 2 * i + 1 < n ? __ldg(x + base + (2 * i + 1) * D) : 0u;
+      w[i] = lo | (hi << 16);
+    }
+    uint32_t nib[2], scode, hb[8];
+    fq16_exact(w, nib, scode, hb, dmax);
+    const int64_t blk = (z * D + r) * nblk + b;
+    if (codes) *reinterpret_cast<uint2 *>(codes + blk * 8) = make_uint2(nib[0], nib[1]);
+    if (scales) {
+      if (tiled) {
+        const int64_t ntiles = (nblk + 7) >> 3;
+        scales[((z * ntiles + (b >> 3)) * 2 + ((b >> 2) & 1)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)] =
+            static_cast<uint8_t>(scode);
+      } else {
+        scales[blk] = static_cast<uint8_t>(scode);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i < n) {
+        const uint32_t h = hb[i >> 1] >> (16 * (i & 1));
+        if (deq) deq[base + i * D] = static_cast<uint16_t>(bf16x2_from_f16x2_exact(h & 0xFFFFu));
+        if (deq_f16) deq_f16[base + i * D] = static_cast<uint16_t>(h);
+      }
+    }
+  }
+  if (absmax) block_max_to_global(dmax, absmax);
 }
 
 cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int64_t cols, int64_t sb,
@@ -202,6 +344,39 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
                             bool sf_col_tiles) {
   const int64_t total = batch * rows * ((cols + 15) / 16);
   if (total == 0) return cudaSuccess;
+  const bool aligned = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 &&
+                       (!deq || (reinterpret_cast<uintptr_t>(deq) & 15u) == 0) &&
+                       (!deq_f16 || (reinterpret_cast<uintptr_t>(deq_f16) & 15u) == 0);
+  // contiguous rows of 64 or 128 elements, blocks along the row
+  if (batch == 1 && sc == 1 && sr == cols && (cols == 64 || cols == 128) && !absmax && !sf_col_tiles && aligned &&
+      (sf_tile_rows <= 0 || rows % sf_tile_rows == 0)) {
+    const int64_t heads = sf_tile_rows > 0 ? rows / sf_tile_rows : 1;
+    const int64_t L = rows / heads;
+    const int64_t gx = (L * (cols / 16) + 255) / 256;
+    if (heads <= 65535 && gx <= 0x7fffffff) {
+      const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(heads));
+      if (cols == 128)
+        quantize_rows_kernel<128><<<grid, 256, 0, stream>>>(x, L, codes, scales, sf_tile_rows > 0, deq, deq_f16);
+      else
+        quantize_rows_kernel<64><<<grid, 256, 0, stream>>>(x, L, codes, scales, sf_tile_rows > 0, deq, deq_f16);
+      return cudaGetLastError();
+    }
+  }
+  // [heads][L][D] blocked along tokens: rows = D channels (stride 1), cols = L
+  // tokens (stride D), batch = heads (stride L*D)
+  if (sr == 1 && (rows == 64 || rows == 128) && sc == rows && sb == rows * cols && sf_tile_rows <= 0) {
+    const int64_t gx = (((cols + 15) / 16) * rows + 255) / 256;
+    if (batch <= 65535 && gx <= 0x7fffffff) {
+      const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(batch));
+      if (rows == 128)
+        quantize_tokens_kernel<128><<<grid, 256, 0, stream>>>(x, cols, codes, scales, sf_col_tiles, deq, deq_f16,
+                                                              absmax);
+      else
+        quantize_tokens_kernel<64><<<grid, 256, 0, stream>>>(x, cols, codes, scales, sf_col_tiles, deq, deq_f16,
+                                                             absmax);
+      return cudaGetLastError();
+    }
+  }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -78,32 +78,48 @@ cudaError_t launch_sparse_plan(const uint8_t *mask, int BH, int nq, int nk, int3
 // order: rows summed in token order, one correctly rounded division by the
 // row count, channels accumulated in order with one fused multiply-add each.
 
-// One CTA per (tile, head), one thread per channel: means[bh][t][d], tiles
-// t < nq of q, then nk tiles of k.  The row loop reads one 2*D-byte row per
-// step, coalesced across the CTA.
-__global__ void __launch_bounds__(128) tile_mean_kernel(const __nv_bfloat16 *__restrict__ q,
-                                                        const __nv_bfloat16 *__restrict__ k, int Lq, int Lk,
-                                                        int D, int nq, int nk, float *__restrict__ means) {
+// One CTA per (tile, head), one thread per pair of channels (D/2 threads):
+// means[bh][t][d], tiles t < nq of q, then nk tiles of k.  Each step of the
+// row loop reads one 2*D-byte row, coalesced across the CTA; the loop is
+// unrolled so that 16 rows are in flight per thread (the sums stay in token
+// order).
+__global__ void __launch_bounds__(64) tile_mean_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                       const __nv_bfloat16 *__restrict__ k, int Lq, int Lk,
+                                                       int D, int nq, int nk, float *__restrict__ means) {
   const int t = blockIdx.x;
   const int64_t bh = blockIdx.y;
-  const int d = threadIdx.x;
+  const int d = 2 * threadIdx.x;
   const bool isq = t < nq;
   const int L = isq ? Lq : Lk;
   const int r0 = (isq ? t : t - nq) * kBM;
   const int r1 = r0 + kBM < L ? r0 + kBM : L;
-  const __nv_bfloat16 *x = (isq ? q : k) + static_cast<size_t>(bh) * L * D + d;
-  float s = 0.0f;
-#pragma unroll 8
-  for (int r = r0; r < r1; ++r) s = __fadd_rn(s, __bfloat162float(x[static_cast<size_t>(r) * D]));
-  means[(static_cast<size_t>(bh) * (nq + nk) + t) * D + d] = __fdiv_rn(s, static_cast<float>(r1 - r0));
+  const uint32_t *x =
+      reinterpret_cast<const uint32_t *>((isq ? q : k) + static_cast<size_t>(bh) * L * D + d);
+  float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 16
+  for (int r = r0; r < r1; ++r) {
+    const uint32_t w = __ldg(x + static_cast<size_t>(r) * (D / 2));
+    s0 = __fadd_rn(s0, __uint_as_float(w << 16));
+    s1 = __fadd_rn(s1, __uint_as_float(w & 0xFFFF0000u));
+  }
+  const float cnt = static_cast<float>(r1 - r0);
+  float2 *dst = reinterpret_cast<float2 *>(means + (static_cast<size_t>(bh) * (nq + nk) + t) * D + d);
+  *dst = make_float2(__fdiv_rn(s0, cnt), __fdiv_rn(s1, cnt));
 }
 
-// One warp per (head, query tile): the nk coarse scores into `scores`, then
-// topk rounds of a warp-wide argmax (score descending, tile ascending) over
-// the tiles not yet kept.  The mask row is written here (0 or 1 per tile).
+// One warp per (head, query tile): the nk coarse scores, then topk rounds of
+// a warp-wide argmax (score descending, tile ascending) over the tiles not
+// yet kept, with the taken tiles marked -inf in the score row (scores are
+// finite for finite inputs).  SM: the score row lives in shared memory
+// (nk <= kSelectSmemTiles), else in `scores` in global memory.  The mask row
+// is written at the end (0 or 1 per tile).
+constexpr int kSelectSmemTiles = 2048;
+
+template <bool SM>
 __global__ void __launch_bounds__(128) tile_select_kernel(const float *__restrict__ means, int BH, int nq, int nk,
                                                           int D, int topk, float *__restrict__ scores,
                                                           uint8_t *__restrict__ mask) {
+  extern __shared__ float sel_smem[];
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= static_cast<int64_t>(BH) * nq) return;  // warp-uniform
@@ -111,30 +127,28 @@ __global__ void __launch_bounds__(128) tile_select_kernel(const float *__restric
   const int I = static_cast<int>(w - bh * nq);
   const float4 *qm = reinterpret_cast<const float4 *>(means + (bh * (nq + nk) + I) * D);
   const float *km = means + (bh * (nq + nk) + nq) * D;
-  float *sc = scores + w * nk;
+  float *sc = SM ? sel_smem + (threadIdx.x >> 5) * nk : scores + w * nk;
   uint8_t *mk = mask + w * nk;
   for (int j = lane; j < nk; j += 32) {
     const float4 *kr = reinterpret_cast<const float4 *>(km + static_cast<size_t>(j) * D);
     float acc = 0.0f;
     for (int c = 0; c < D / 4; ++c) {
-      const float4 a = qm[c], b = kr[c];
+      const float4 a = qm[c], b = __ldg(kr + c);
       acc = __fmaf_rn(a.x, b.x, acc);
       acc = __fmaf_rn(a.y, b.y, acc);
       acc = __fmaf_rn(a.z, b.z, acc);
       acc = __fmaf_rn(a.w, b.w, acc);
     }
     sc[j] = acc;
-    mk[j] = 0;
   }
   __syncwarp();
   const int kk = topk < nk ? topk : nk;
   for (int r = 0; r < kk; ++r) {
-    float best = 0.0f;
+    float best = -INFINITY;
     int bj = -1;  // -1: no candidate
     for (int j = lane; j < nk; j += 32) {
-      if (mk[j]) continue;
       const float v = sc[j];
-      if (bj < 0 || v > best) {  // ascending j: equal scores keep the lower tile
+      if (v != -INFINITY && (bj < 0 || v > best)) {  // ascending j: equal scores keep the lower tile
         best = v;
         bj = j;
       }
@@ -148,20 +162,29 @@ __global__ void __launch_bounds__(128) tile_select_kernel(const float *__restric
         bj = oj;
       }
     }
-    if (lane == 0 && bj >= 0 && bj < nk) mk[bj] = 1;
+    if (lane == 0 && bj >= 0 && bj < nk) sc[bj] = -INFINITY;
     __syncwarp();
   }
+  // kept tiles are the ones marked -inf
+  for (int j = lane; j < nk; j += 32) mk[j] = sc[j] == -INFINITY ? 1 : 0;
 }
 
 cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D,
                               int topk, float *means, float *scores, uint8_t *mask, cudaStream_t stream) {
   const int nq = (Lq + kBM - 1) / kBM, nk = (Lk + kBN - 1) / kBN;
-  tile_mean_kernel<<<dim3(nq + nk, BH), D, 0, stream>>>(q, k, Lq, Lk, D, nq, nk, means);
+  tile_mean_kernel<<<dim3(nq + nk, BH), D / 2, 0, stream>>>(q, k, Lq, Lk, D, nq, nk, means);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t blocks = (static_cast<int64_t>(BH) * nq * 32 + 127) / 128;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
-  tile_select_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(means, BH, nq, nk, D, topk, scores, mask);
+  if (nk <= kSelectSmemTiles) {
+    // 4 warps x nk floats: at most 32 KB
+    tile_select_kernel<true><<<static_cast<unsigned>(blocks), 128, 4 * nk * sizeof(float), stream>>>(
+        means, BH, nq, nk, D, topk, scores, mask);
+  } else {
+    tile_select_kernel<false><<<static_cast<unsigned>(blocks), 128, 0, stream>>>(means, BH, nq, nk, D, topk, scores,
+                                                                                mask);
+  }
   return cudaGetLastError();
 }
 
