@@ -1,0 +1,65 @@
+"""Host logic of the benchmark that needs no GPU: the flop count of the
+block-sparse step (pairs the tile mask selects, ragged last tiles included)
+and the clock sampler's parsing of nvidia-smi samples around a timed region
+shorter than the sampling period (a fake nvidia-smi on PATH)."""
+import os
+import stat
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from quantization_aware_attention_nvfp4_b200 import workloads as W  # noqa: E402
+
+
+def test_selected_pairs_counts_ragged_tiles():
+    w = W.custom(2, 3, 300, 200, 64, seed_index=5)
+    mask = W.random_tile_mask(w, 0.5)
+    T = W.SPARSE_TILE
+    brute = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            for i in range(w.Lq):
+                for j in range(w.Lk):
+                    brute += int(mask[b, h, i // T, j // T])
+    assert bench.selected_pairs(w, mask) == brute
+    assert bench.selected_pairs(w, np.ones_like(mask)) == w.B * w.H * w.Lq * w.Lk
+
+
+def test_topk_tiles_follows_the_selection_formula():
+    # max(1, min(ceil((1 - sparsity) * n), n))
+    assert W.topk_tiles(244, 0.9) == 25
+    assert W.topk_tiles(10, 0.9) == 1
+    assert W.topk_tiles(5, 0.0) == 5
+    assert W.topk_tiles(7, 1.0) == 1
+    m = W.tile_mask(W.get("wan_6h_31200"), 0.9)
+    assert m.shape == (1, 6, 244, 244) and np.all(m.sum(-1) == 25)
+
+
+def _fake_smi(tmp_path, reason):
+    script = tmp_path / "nvidia-smi"
+    script.write_text("#!/bin/sh\nsleep 0.2\nfor i in $(seq 1 200); do echo '0, 1800, 1965, 700.0, 0x4, Not Active, "
+                      "Not Active, Not Active, %s'; sleep 0.05; done\n" % reason)
+    script.chmod(script.stat().st_mode | stat.S_IEXEC)
+    return str(tmp_path)
+
+
+def test_clock_sampler_brackets_a_short_region(tmp_path, monkeypatch):
+    monkeypatch.setenv("PATH", _fake_smi(tmp_path, "Active") + os.pathsep + os.environ["PATH"])
+    with bench.ClockSampler(0) as c:
+        time.sleep(0.01)  # far shorter than the 50 ms sampling period
+    s = c.summary()
+    assert s["samples"] >= 2
+    assert s["sm_mhz"] == 1800.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    monkeypatch.setenv("PATH", str(tmp_path))  # nothing to run
+    with bench.ClockSampler(0) as c:
+        pass
+    assert c.summary()["reasons"] == ["nvidia-smi unavailable"]

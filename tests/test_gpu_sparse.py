@@ -10,8 +10,6 @@ O = 0, m = LSE = -inf, dQ = 0, and keys of a tile nobody selects exactly
 dK = dV = 0.  With every tile selected the sparse path runs the dense kernels'
 schedule on the same tiles, so its outputs must equal the dense call's bit for
 bit."""
-import math
-
 import numpy as np
 import pytest
 
