@@ -21,6 +21,7 @@ citations and the readings taken where the pages are silent):
   the same computation restricted, per query tile, to the keys of the
   selected key tiles (``sel`` [n_query_tiles, n_key_tiles], nonzero =
   selected); a row with no selected key gives O = 0, LSE = m = -inf, dQ = 0.
+* causal masking (flag CAUSAL, Lq == Lk): query i attends to keys j <= i.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against brute force, closed forms, torch's own float8 conversion and finite
@@ -45,6 +46,7 @@ QUANT_V = 4
 QUANT_P = 8
 QUANT_ALL = 15
 DV_QUANT_NORMALIZED = 16
+CAUSAL = 32
 
 _lock = threading.Lock()
 _lib = None
@@ -228,6 +230,8 @@ class Head:
         self.Lk = k.shape[0]
         if v.shape != k.shape or k.shape[1] != self.D:
             raise ValueError("q [Lq,D], k and v [Lk,D] expected")
+        if (flags & CAUSAL) and self.Lq != self.Lk:
+            raise ValueError("causal masking needs Lq == Lk")
         if tile < 16 or tile % 16:
             raise ValueError("tile must be a positive multiple of 16")
         self.tile = int(tile)

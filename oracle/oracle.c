@@ -55,6 +55,11 @@
  * key has O = 0, l = 0, m = LSE = -infinity, dQ = 0, and adds nothing to
  * dK, dV.
  *
+ * Causal masking (flag ORACLE_CAUSAL, Lq == Lk): query i attends to keys
+ * j <= i only.  The pages' training route is non-causal; this is the general
+ * route's masking read the same way as the block selection: masked keys have
+ * P~ = 0 inside their fq(P~) block, and m, l run over the unmasked keys.
+ *
  * Every arithmetic step is plain float64; the only reorderings are the ones a
  * sum admits.  Loops are parallelised over independent rows with OpenMP.
  */
@@ -71,12 +76,17 @@
 #define ORACLE_QUANT_V 4u
 #define ORACLE_QUANT_P 8u
 #define ORACLE_DV_QUANT_NORMALIZED 16u
+#define ORACLE_CAUSAL 32u
 
 #define BLOCK 16
 
-/* Does query i attend to key j?  (sel == NULL: dense.) */
-static int selected(const uint8_t *sel, long T, long nkt, long i, long j)
+/* Does query i attend to key j?  sel == NULL: every tile; ORACLE_CAUSAL:
+ * only keys j <= i (Lq == Lk, query i and key i are the same token).       */
+static int selected(unsigned flags, const uint8_t *sel, long T, long nkt, long i,
+                    long j)
 {
+    if ((flags & ORACLE_CAUSAL) && j > i)
+        return 0;
     return sel == NULL || sel[(i / T) * nkt + j / T] != 0;
 }
 
@@ -439,11 +449,11 @@ static void prob_row(const double *Qi, long i, const double *Kh, long Lk, long D
     score_row(Qi, Kh, Lk, D, c, S);
     double m = -INFINITY;
     for (long j = 0; j < Lk; j++)
-        if (selected(sel, T, nkt, i, j) && S[j] > m)
+        if (selected(flags, sel, T, nkt, i, j) && S[j] > m)
             m = S[j];
     double l = 0.0;
     for (long j = 0; j < Lk; j++) {
-        Pt[j] = selected(sel, T, nkt, i, j) ? exp(S[j] - m) : 0.0;
+        Pt[j] = selected(flags, sel, T, nkt, i, j) ? exp(S[j] - m) : 0.0;
         l += Pt[j];
     }
     if (flags & ORACLE_QUANT_P) {
@@ -544,7 +554,7 @@ void oracle_bwd_dq_rows(const double *Qh, const double *Kh, const double *Vh,
             for (long d = 0; d < D; d++)
                 dQ[t * D + d] = 0.0;
             for (long j = 0; j < Lk; j++) {
-                if (!(l[i] > 0.0) || !selected(sel, T, nkt, i, j))
+                if (!(l[i] > 0.0) || !selected(flags, sel, T, nkt, i, j))
                     continue;
                 double P = exp(S[j] - m[i]) / l[i];
                 double dP = dot(dOi, Vh + j * D, D);
@@ -589,7 +599,7 @@ void oracle_bwd_dkdv_blocks(const double *Qh, const double *Kh, const double *Vh
                 dOi[d] = oracle_bf16_value(dO[i * D + d]);
             for (long jj = 0; jj < n; jj++) {
                 S[jj] = c * dot(Qh + i * D, Kh + (j0 + jj) * D, D);
-                Pt[jj] = selected(sel, T, nkt, i, j0 + jj) ? exp(S[jj] - m[i]) : 0.0;
+                Pt[jj] = selected(flags, sel, T, nkt, i, j0 + jj) ? exp(S[jj] - m[i]) : 0.0;
             }
             /* w_j: the dV weight of key j in this query row */
             double w[BLOCK];

@@ -585,6 +585,61 @@ def test_sparse_quantizers_off_vs_torch_masked_sdpa():
         assert np.max(np.abs(sp[name][0, 0] - ref)) <= 1e-10 * max(1.0, np.max(np.abs(ref))), name
 
 
+# ----------------------------------------------------- causal masking ----
+
+def test_causal_quantizers_off_vs_torch_sdpa():
+    """Quantizers off: causal attention is torch's causal SDPA (float64
+    autograd for the gradients)."""
+    rng = np.random.default_rng(95)
+    L, D, c = 48, 16, 0.31
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for _ in range(4))
+    qt, kt, vt = (torch.tensor(_f(x[0, 0]), requires_grad=True) for x in (q, k, v))
+    O = torch.nn.functional.scaled_dot_product_attention(qt[None], kt[None], vt[None], is_causal=True, scale=c)[0]
+    (O * torch.tensor(_f(dO[0, 0]))).sum().backward()
+    out = oracle.attention(q, k, v, c, oracle.CAUSAL, dO)
+    for name, ref in (("O", O.detach()), ("dQ", qt.grad), ("dK", kt.grad), ("dV", vt.grad)):
+        ref = ref.numpy()
+        assert np.max(np.abs(out[name][0, 0] - ref)) <= 1e-10 * max(1.0, np.max(np.abs(ref))), name
+
+
+def test_causal_rows_equal_dense_attention_on_their_prefix():
+    """With fq on: row i of causal attention is dense attention of row i
+    against keys 0..i (fq(P~)'s ragged last block is zero-padded there, as the
+    masked keys are zeros here); fq(V) runs on the whole V in both (its
+    blocks along tokens do not depend on the mask), so the prefix problems
+    take the oracle's fq(V) as plain bf16 input.  dK, dV sum the prefix
+    problems' gradients."""
+    rng = np.random.default_rng(96)
+    L, D, c = 40, 16, 0.27
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for _ in range(4))
+    flags = oracle.QUANT_ALL | oracle.CAUSAL
+    out = oracle.attention(q, k, v, c, flags, dO)
+    vh = oracle.Head(q[0, 0], k[0, 0], v[0, 0], c, oracle.QUANT_ALL).Vh
+    vq = W.f32_to_bf16_bits(vh.astype(np.float32))
+    assert np.array_equal(W.bf16_bits_to_f32(vq).astype(np.float64), vh)
+    pre = oracle.QUANT_ALL & ~oracle.QUANT_V
+    dK = np.zeros((L, D))
+    dV = np.zeros((L, D))
+    for i in range(L):
+        hd = oracle.Head(q[0, 0, i:i + 1], k[0, 0, : i + 1], vq[: i + 1], c, pre, dO[0, 0, i:i + 1])
+        st = hd.stats()
+        dQi, dKi, dVi = hd.backward()
+        assert np.max(np.abs(out["O"][0, 0, i] - st["O"][0])) <= 1e-12 * np.max(np.abs(st["O"]))
+        assert abs(out["lse"][0, 0, i] - st["lse"][0]) <= 1e-12 and out["m"][0, 0, i] == st["m"][0]
+        assert np.max(np.abs(out["dQ"][0, 0, i] - dQi[0])) <= 1e-11 * max(np.max(np.abs(dQi)), 1e-30)
+        dK[: i + 1] += dKi
+        dV[: i + 1] += dVi
+    assert np.max(np.abs(out["dK"][0, 0] - dK)) <= 1e-11 * np.max(np.abs(dK))
+    assert np.max(np.abs(out["dV"][0, 0] - dV)) <= 1e-11 * np.max(np.abs(dV))
+
+
+def test_causal_needs_equal_lengths():
+    rng = np.random.default_rng(97)
+    q, k = _rand_bits(rng, (8, 16)), _rand_bits(rng, (12, 16))
+    with pytest.raises(ValueError):
+        oracle.Head(q, k, k, 0.3, oracle.CAUSAL)
+
+
 # ----------------------------------------------- sparse block selection ----
 
 def test_vsa_select_agrees_with_float64_ranking():
