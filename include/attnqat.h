@@ -74,6 +74,16 @@ extern "C" {
 #define ATTNQAT_QUANT_V 4u
 #define ATTNQAT_QUANT_P 8u
 #define ATTNQAT_QUANT_ALL 15u
+/* Causal masking (attnqat_fwd / attnqat_bwd / attnqat_workspace_size only;
+ * needs Lq == Lk and every quantizer on, ATTNQAT_QUANT_ALL, whose exact fp16
+ * operands carry dS and the dV operand with 11 significant bits -- with bf16
+ * ones the gradients of the first keys, which every later row feeds, are not
+ * accurate enough): query i attends to keys j <= i.  The pages' training route
+ * is non-causal (FastVideo "Attn-QAT Training" guide, "Architecture-specific
+ * Triton routing"); the mask is applied like a tile selection: masked keys
+ * have P~ = 0 inside their fq(P~) blocks, m and l run over the unmasked keys,
+ * and only the lower triangle of 128 x 128 tiles is computed. */
+#define ATTNQAT_CAUSAL 32u
 
 /* Text for a status code (static storage). */
 const char *attnqat_strerror(int status);
@@ -185,6 +195,8 @@ size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D,
  * float32 (the exact row max of the scaled scores).  ws/ws_bytes: device
  * workspace of at least attnqat_workspace_size(B,H,Lq,Lk,D,flags) bytes,
  * 256-byte aligned; it must be passed unchanged to attnqat_bwd.
+ * flags may add ATTNQAT_CAUSAL (then Lq == Lk and ATTNQAT_QUANT_ALL are
+ * required).
  * Shapes: B, H >= 1; Lq >= 1; Lk >= 1; D in {64, 128}; B*H*max(Lq,Lk)*D
  * below 2^31.  Lq is arbitrary (the last query tile is masked); a partial
  * last KV tile runs the separate masked tail step.  Lk need not be 16-aligned
@@ -238,7 +250,8 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse,
  * tile_mask); the workspace is attnqat_sparse_workspace_size() bytes (the
  * dense workspace plus int32 tile lists, 8 * B*H*nq*nk + 4 * B*H*(nq + nk)
  * bytes, rebuilt from the mask by every call), passed unchanged from
- * attnqat_sparse_fwd to attnqat_sparse_bwd.
+ * attnqat_sparse_fwd to attnqat_sparse_bwd.  ATTNQAT_CAUSAL is not accepted
+ * here (EINVAL; the workspace size is 0).
  */
 #define ATTNQAT_SPARSE_TILE 128
 size_t attnqat_sparse_workspace_size(int B, int H, int Lq, int Lk, int D,

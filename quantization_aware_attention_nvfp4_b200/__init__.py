@@ -40,6 +40,7 @@ QUANT_K = 2
 QUANT_V = 4
 QUANT_P = 8
 QUANT_ALL = 15
+CAUSAL = 32  # causal masking (attnqat_fwd / attnqat_bwd; Lq == Lk, every quantizer on)
 
 OK = 0
 EINVAL = -1

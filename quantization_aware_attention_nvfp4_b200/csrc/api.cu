@@ -263,11 +263,18 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 static int check_shape(int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags) {
   if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return ATTNQAT_EINVAL;
+  if ((flags & ATTNQAT_CAUSAL) && Lq != Lk) return ATTNQAT_EINVAL;  // query i and key i are one token
+  // causal masking runs with every quantizer on, whose exact fp16 operands
+  // carry dS and the dV operand fq(P~)/l with 11 significant bits: with bf16
+  // ones the heavy-tailed gradients of the first keys (fed by every later
+  // row) miss the max-abs bar -- dK 5.3e-2 of RMS with no quantizer, dV
+  // 8.0e-2 with Q and K alone, measured at L = 500
+  if ((flags & ATTNQAT_CAUSAL) && (flags & ATTNQAT_QUANT_ALL) != ATTNQAT_QUANT_ALL) return ATTNQAT_EINVAL;
   if (static_cast<int64_t>(B) * H > 65535) return ATTNQAT_EINVAL;  // grid.y
   const int64_t Lmax = Lq > Lk ? Lq : Lk;
   if (static_cast<int64_t>(B) * H * Lmax * 128 >= (int64_t(1) << 40)) return ATTNQAT_EINVAL;
   if (!(std::isfinite(sm_scale) && sm_scale > 0.0f)) return ATTNQAT_EINVAL;
-  if (flags & ~ATTNQAT_QUANT_ALL) return ATTNQAT_EINVAL;
+  if (flags & ~(ATTNQAT_QUANT_ALL | ATTNQAT_CAUSAL)) return ATTNQAT_EINVAL;
   if (D != 64 && D != 128) return ATTNQAT_EUNSUPPORTED;
   return ATTNQAT_OK;
 }
@@ -428,24 +435,24 @@ int attnqat_quantize_gs(const void *x, int64_t batch, int64_t rows, int64_t cols
 
 size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
   if (check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
-  return layout(B, H, Lq, Lk, D, flags).total;
+  return layout(B, H, Lq, Lk, D, flags, (flags & ATTNQAT_CAUSAL) != 0).total;
 }
 
 }  // extern "C"
 
 namespace attnqat {
 
-// Builds the block-sparse tile lists from the caller's mask into the
-// workspace (no-op for dense calls, mask == nullptr).
-static int plan_sparse(const uint8_t *mask, int BH, int Lq, int Lk, uint8_t *wsb, const Workspace &w,
+// Builds the tile lists into the workspace: from the caller's mask
+// (block-sparse), the lower triangle (causal), or nothing (dense).
+static int plan_sparse(const uint8_t *mask, bool causal, int BH, int Lq, int Lk, uint8_t *wsb, const Workspace &w,
                        cudaStream_t s) {
-  if (!mask) return ATTNQAT_OK;
-  ProfScope ps("sparse_plan", s);
-  const cudaError_t e = launch_sparse_plan(mask, BH, (Lq + kBM - 1) / kBM, (Lk + kBN - 1) / kBN,
-                                           reinterpret_cast<int32_t *>(wsb + w.kv_list),
-                                           reinterpret_cast<int32_t *>(wsb + w.kv_count),
-                                           reinterpret_cast<int32_t *>(wsb + w.q_list),
-                                           reinterpret_cast<int32_t *>(wsb + w.q_count), s);
+  if (!mask && !causal) return ATTNQAT_OK;
+  int32_t *kvl = reinterpret_cast<int32_t *>(wsb + w.kv_list), *kvc = reinterpret_cast<int32_t *>(wsb + w.kv_count);
+  int32_t *ql = reinterpret_cast<int32_t *>(wsb + w.q_list), *qc = reinterpret_cast<int32_t *>(wsb + w.q_count);
+  ProfScope ps(causal ? "causal_plan" : "sparse_plan", s);
+  const cudaError_t e = causal ? launch_causal_plan(BH, (Lq + kBM - 1) / kBM, kvl, kvc, ql, qc, s)
+                               : launch_sparse_plan(mask, BH, (Lq + kBM - 1) / kBM, (Lk + kBN - 1) / kBN, kvl, kvc,
+                                                    ql, qc, s);
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }
 
@@ -455,11 +462,13 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
                    size_t ws_bytes, void *stream) {
   int st = check_shape(B, H, Lq, Lk, D, sm_scale, flags);
   if (st != ATTNQAT_OK) return st;
+  const bool causal = (flags & ATTNQAT_CAUSAL) != 0;
+  if (causal && mask) return ATTNQAT_EINVAL;  // a tile selection and causal masking do not combine
   if (!q || !k || !v || !o || !lse || !m || !ws) return ATTNQAT_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(m) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
     return ATTNQAT_EINVAL;
-  const Workspace w = layout(B, H, Lq, Lk, D, flags, mask != nullptr);
+  const Workspace w = layout(B, H, Lq, Lk, D, flags, mask != nullptr || causal);
   if (ws_bytes < w.total) return ATTNQAT_ENOSPC;
   st = check_device();
   if (st != ATTNQAT_OK) return st;
@@ -468,7 +477,7 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
   st = prepare_operands(q, k, v, B, H, Lq, Lk, D, flags, wsb, w, s);
   if (st != ATTNQAT_OK) return st;
   const int BH = B * H;
-  st = plan_sparse(mask, BH, Lq, Lk, wsb, w, s);
+  st = plan_sparse(mask, causal, BH, Lq, Lk, wsb, w, s);
   if (st != ATTNQAT_OK) return st;
   const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
   const void *kh = (flags & ATTNQAT_QUANT_K) ? static_cast<const void *>(wsb + w.kh) : k;
@@ -495,8 +504,10 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
   a.o32 = reinterpret_cast<float *>(wsb + w.o32);
   a.lse = lse;
   a.m = m;
-  a.kv_list = mask ? reinterpret_cast<const int32_t *>(wsb + w.kv_list) : nullptr;
-  a.kv_count = mask ? reinterpret_cast<const int32_t *>(wsb + w.kv_count) : nullptr;
+  const bool listed = mask != nullptr || causal;
+  a.kv_list = listed ? reinterpret_cast<const int32_t *>(wsb + w.kv_list) : nullptr;
+  a.kv_count = listed ? reinterpret_cast<const int32_t *>(wsb + w.kv_count) : nullptr;
+  a.causal = causal ? 1 : 0;
   cudaError_t e;
   {
     ProfScope ps("attn_fwd", s);
@@ -511,19 +522,21 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
                    void *dq, void *dk, void *dv, void *ws, size_t ws_bytes, void *stream) {
   int st = check_shape(B, H, Lq, Lk, D, sm_scale, flags);
   if (st != ATTNQAT_OK) return st;
+  const bool causal = (flags & ATTNQAT_CAUSAL) != 0;
+  if (causal && mask) return ATTNQAT_EINVAL;
   if (!q || !k || !v || !lse || !m || !dO || !dq || !dk || !dv || !ws) return ATTNQAT_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(lse) || !aligned16(m) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
     return ATTNQAT_EINVAL;
-  const Workspace w = layout(B, H, Lq, Lk, D, flags, mask != nullptr);
+  const Workspace w = layout(B, H, Lq, Lk, D, flags, mask != nullptr || causal);
   if (ws_bytes < w.total) return ATTNQAT_ENOSPC;
   st = check_device();
   if (st != ATTNQAT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int BH = B * H;
-  st = plan_sparse(mask, BH, Lq, Lk, wsb, w, s);
+  st = plan_sparse(mask, causal, BH, Lq, Lk, wsb, w, s);
   if (st != ATTNQAT_OK) return st;
   float *delta = reinterpret_cast<float *>(wsb + w.delta);
   float *stats = reinterpret_cast<float *>(wsb + w.stats);
@@ -570,10 +583,12 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
   a.dq = static_cast<__nv_bfloat16 *>(dq);
   a.dk = static_cast<__nv_bfloat16 *>(dk);
   a.dv = static_cast<__nv_bfloat16 *>(dv);
-  a.kv_list = mask ? reinterpret_cast<const int32_t *>(wsb + w.kv_list) : nullptr;
-  a.kv_count = mask ? reinterpret_cast<const int32_t *>(wsb + w.kv_count) : nullptr;
-  a.q_list = mask ? reinterpret_cast<const int32_t *>(wsb + w.q_list) : nullptr;
-  a.q_count = mask ? reinterpret_cast<const int32_t *>(wsb + w.q_count) : nullptr;
+  const bool listed = mask != nullptr || causal;
+  a.kv_list = listed ? reinterpret_cast<const int32_t *>(wsb + w.kv_list) : nullptr;
+  a.kv_count = listed ? reinterpret_cast<const int32_t *>(wsb + w.kv_count) : nullptr;
+  a.q_list = listed ? reinterpret_cast<const int32_t *>(wsb + w.q_list) : nullptr;
+  a.q_count = listed ? reinterpret_cast<const int32_t *>(wsb + w.q_count) : nullptr;
+  a.causal = causal ? 1 : 0;
   // with Q and K quantized, S runs on the packed NVFP4 codes
   CUtensorMap tq4, tk4;
   if (f16 && !(encode_codes(&tq4, wsb + w.qc, BH, Lq, D) && encode_codes(&tk4, wsb + w.kc, BH, Lk, D)))
@@ -609,7 +624,7 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
 }
 
 size_t attnqat_sparse_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
-  if (check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
+  if ((flags & ATTNQAT_CAUSAL) || check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
   return layout(B, H, Lq, Lk, D, flags, true).total;
 }
 

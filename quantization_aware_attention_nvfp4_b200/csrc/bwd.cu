@@ -26,7 +26,9 @@
 // Block-sparse (VSA fine attention): with a.q_list / a.kv_list set, the dK/dV
 // kernel walks only the query tiles that selected its key tile and the dQ
 // kernel only the key tiles its query tile selected; a CTA with an empty list
-// writes zero gradients.
+// writes zero gradients.  Causal masking walks the lower triangle of tiles and
+// masks the diagonal tile (the dK/dV kernel's first, the dQ kernel's last) to
+// keys <= the query row.
 #include "common.cuh"
 #include "internal.h"
 
@@ -234,9 +236,10 @@ __device__ __forceinline__ void dkdv_ds_f16(const float (&p)[64], const uint32_t
   }
 }
 
-// SP: block-sparse (walks a.q_list); a separate instantiation, so the dense
-// kernel carries none of the list handling.
-template <int D, int QP, int QKF16, int DOF16, bool SP>
+// SP: 0 dense; 1 block-sparse (walks a.q_list); 2 causal (lower-triangle
+// lists, diagonal masked).  Separate instantiations, so the dense kernel
+// carries none of the list handling.
+template <int D, int QP, int QKF16, int DOF16, int SP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -398,6 +401,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const RowRole rr(warp, lane);
     const int col0 = rr.half * 64;
     const int valid_k = a.Lk - kt * kBN;  // >= 128 for full key tiles
+    // causal: the first query tile visited is the diagonal, where query row r
+    // keeps keys 0..r (a partial key tile only ever meets its diagonal)
+    const int diag_k = static_cast<int>(rr.row) + 1;
     const float cl = a.scale_log2;
     const float dsc = ds_scale<QKF16>(a.stats);
     const uint32_t xaddr = sbase + L::kX;
@@ -431,19 +437,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->sempty);
+        const bool masked = SP == 2 ? i == 0 : valid_k < kBN;
+        const int vk = SP == 2 ? diag_k : valid_k;
         if (DOF16) {
           const float nml = vq ? -(m * kLog2e) : -INFINITY;
           const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
-          if (valid_k < kBN)
-            dkdv_probs_f16<true>(sv, col0, valid_k, cl, nml, vf, p, pw);
+          if (masked)
+            dkdv_probs_f16<true>(sv, col0, vk, cl, nml, vf, p, pw);
           else
-            dkdv_probs_f16<false>(sv, col0, valid_k, cl, nml, vf, p, pw);
+            dkdv_probs_f16<false>(sv, col0, vk, cl, nml, vf, p, pw);
         } else {
           const float nml = -(m * kLog2e);
-          if (valid_k < kBN)
-            dkdv_probs<QP, true>(sv, col0, valid_k, vq, cl, nml, inv_l, p, pw);
+          if (masked)
+            dkdv_probs<QP, true>(sv, col0, vk, vq, cl, nml, inv_l, p, pw);
           else
-            dkdv_probs<QP, false>(sv, col0, valid_k, vq, cl, nml, inv_l, p, pw);
+            dkdv_probs<QP, false>(sv, col0, vk, vq, cl, nml, inv_l, p, pw);
         }
       }
       // X = (fq(P~)/l)^T once dK_{i-1} has read the previous dS^T
@@ -592,8 +600,9 @@ __device__ __forceinline__ void dq_tile_f16(const uint32_t (&sv)[64], const uint
   }
 }
 
-// SP: block-sparse (walks a.kv_list), as for the dK/dV kernel.
-template <int D, int QKF16, int DOF16, bool SP>
+// SP: 0 dense, 1 block-sparse (walks a.kv_list), 2 causal, as for the dK/dV
+// kernel.
+template <int D, int QKF16, int DOF16, int SP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -752,8 +761,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float a1 = DOF16 ? dsc / do_scale(a.stats) : 0.0f;
     const float b1 = -delta * dsc;
     const int last_valid = a.Lk - (nk - 1) * kBN;
-    // the lists ascend, so only the last tile visited can be the partial one
-    const bool tail_last = n > 0 && ktile(n - 1) == nk - 1 && last_valid < kBN;
+    // the lists ascend, so only the last tile visited can be the partial one;
+    // with causal masking the last tile is the diagonal, where row r keeps
+    // keys 0..r
+    const bool tail_last = SP == 2 ? true : (n > 0 && ktile(n - 1) == nk - 1 && last_valid < kBN);
+    const int last_cols = SP == 2 ? static_cast<int>(rr.row) + 1 : last_valid;
     const uint32_t xaddr = sbase + L::kX;
     const uint32_t tS = tmem + rr.lane_addr + L::kTmemS, tDP = tmem + rr.lane_addr + L::kTmemDP;
     bool ok = true;
@@ -769,12 +781,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars->sempty);
       if (DOF16) {
         if (tail)
-          dq_tile_f16<true>(sv, dv, col0, last_valid, cl, nlse, a1, b1, dsw);
+          dq_tile_f16<true>(sv, dv, col0, last_cols, cl, nlse, a1, b1, dsw);
         else
           dq_tile_f16<false>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw);
       } else {
         if (tail)
-          dq_tile<QKF16, true>(sv, dv, col0, last_valid, vq, cl, nlse, delta, dsc, dsw);
+          dq_tile<QKF16, true>(sv, dv, col0, last_cols, vq, cl, nlse, delta, dsc, dsw);
         else
           dq_tile<QKF16, false>(sv, dv, col0, kBN, vq, cl, nlse, delta, dsc, dsw);
       }
@@ -823,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------- launchers --
 
-template <int D, int QP, int QKF16, int DOF16, bool SP>
+template <int D, int QP, int QKF16, int DOF16, int SP>
 static cudaError_t launch_dkdv_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
                                   cudaStream_t stream) {
@@ -842,8 +854,9 @@ template <int D, int QP, int QKF16, int DOF16>
 static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                  const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
                                  cudaStream_t stream) {
-  return a.q_list ? launch_dkdv_sp<D, QP, QKF16, DOF16, true>(tq, tk, tv, tdo, tq4, a, BH, stream)
-                  : launch_dkdv_sp<D, QP, QKF16, DOF16, false>(tq, tk, tv, tdo, tq4, a, BH, stream);
+  if (!a.q_list) return launch_dkdv_sp<D, QP, QKF16, DOF16, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
+  return a.causal ? launch_dkdv_sp<D, QP, QKF16, DOF16, 2>(tq, tk, tv, tdo, tq4, a, BH, stream)
+                  : launch_dkdv_sp<D, QP, QKF16, DOF16, 1>(tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
 template <int D>
@@ -865,7 +878,7 @@ cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const
                   : dkdv_dispatch<64>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
-template <int D, int QKF16, int DOF16, bool SP>
+template <int D, int QKF16, int DOF16, int SP>
 static cudaError_t launch_dq_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
                                 cudaStream_t stream) {
@@ -884,8 +897,9 @@ template <int D, int QKF16, int DOF16>
 static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
                                cudaStream_t stream) {
-  return a.kv_list ? launch_dq_sp<D, QKF16, DOF16, true>(tq, tk, tv, tdo, tk4, a, BH, stream)
-                   : launch_dq_sp<D, QKF16, DOF16, false>(tq, tk, tv, tdo, tk4, a, BH, stream);
+  if (!a.kv_list) return launch_dq_sp<D, QKF16, DOF16, 0>(tq, tk, tv, tdo, tk4, a, BH, stream);
+  return a.causal ? launch_dq_sp<D, QKF16, DOF16, 2>(tq, tk, tv, tdo, tk4, a, BH, stream)
+                  : launch_dq_sp<D, QKF16, DOF16, 1>(tq, tk, tv, tdo, tk4, a, BH, stream);
 }
 
 template <int D>

@@ -34,7 +34,8 @@
 // Block-sparse (VSA fine attention): with a.kv_list set, the CTA walks only
 // the key tiles listed for its query tile, in both sweeps, so m is the exact
 // max over the selected keys; a query tile with no key tile writes O = 0 and
-// m = LSE = -inf.
+// m = LSE = -inf.  Causal masking walks the lower triangle the same way and
+// masks its last tile, the diagonal, to keys <= the query row.
 #include "common.cuh"
 #include "internal.h"
 
@@ -226,9 +227,10 @@ __device__ __forceinline__ void group_sync(int wq) {
 template <int G>
 constexpr int fwd_threads() { return (2 + 4 * G + 1 + 3) / 4 * 128; }
 
-// SP: block-sparse (walks a.kv_list); a separate instantiation, so the dense
-// kernel carries none of the list handling.
-template <int D, int FP4S, int PVM, int QP, int G, bool SP>
+// SP: 0 dense; 1 block-sparse (walks a.kv_list); 2 causal (walks the
+// lower-triangle lists and masks the diagonal).  Separate instantiations, so
+// the dense kernel carries none of the list handling.
+template <int D, int FP4S, int PVM, int QP, int G, int SP>
 __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
@@ -463,8 +465,11 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     const RowRole rr(warp, lane);
     const int col0 = rr.half * NC;
     const int last_valid = a.Lk - (nk - 1) * kBN;  // keys in the last KV tile
-    // the lists ascend, so only the last tile visited can be the partial one
-    const bool tail_last = n > 0 && ktile(n - 1) == nk - 1 && last_valid < kBN;
+    // the lists ascend, so only the last tile visited can be the partial one;
+    // with causal masking the last tile is the diagonal, where row r keeps
+    // keys 0..r (which also covers a partial diagonal tile: Lq == Lk)
+    const bool tail_last = SP == 2 ? true : (n > 0 && ktile(n - 1) == nk - 1 && last_valid < kBN);
+    const int last_cols = SP == 2 ? static_cast<int>(rr.row) + 1 : last_valid;
     float mrow = -INFINITY;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -473,7 +478,7 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       if (!mbar_wait(&bars->sfull1[b], (j / L::kNS1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + b * kBN;
-      const float mx = tail ? row_max_cols<true, NC>(taddr, col0, last_valid)
+      const float mx = tail ? row_max_cols<true, NC>(taddr, col0, last_cols)
                             : row_max_cols<false, NC>(taddr, col0, kBN);
       mrow = fmaxf(mrow, mx);
       tc_fence_before();
@@ -501,7 +506,7 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
       const uint32_t psf = sbase + L::kPSFo + pb * L::kPSF;
       if (tail)
-        lsum += prob_cols<PVM, QP, true, NC>(taddr, col0, last_valid, cl, nml, pbase, psf, rr.row);
+        lsum += prob_cols<PVM, QP, true, NC>(taddr, col0, last_cols, cl, nml, pbase, psf, rr.row);
       else
         lsum += prob_cols<PVM, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, psf, rr.row);
       tc_fence_before();
@@ -570,7 +575,7 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
   }
 }
 
-template <int D, int FP4S, int PVM, int QP, bool SP>
+template <int D, int FP4S, int PVM, int QP, int SP>
 static cudaError_t launch_fwd_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                  const FwdArgs &a, int BH, cudaStream_t stream) {
   using L = FwdLayout<D, FP4S, PVM == 2>;
@@ -588,8 +593,9 @@ static cudaError_t launch_fwd_sp(const CUtensorMap &tq, const CUtensorMap &tk, c
 template <int D, int FP4S, int PVM, int QP>
 static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const FwdArgs &a, int BH, cudaStream_t stream) {
-  return a.kv_list ? launch_fwd_sp<D, FP4S, PVM, QP, true>(tq, tk, tv, a, BH, stream)
-                   : launch_fwd_sp<D, FP4S, PVM, QP, false>(tq, tk, tv, a, BH, stream);
+  if (!a.kv_list) return launch_fwd_sp<D, FP4S, PVM, QP, 0>(tq, tk, tv, a, BH, stream);
+  return a.causal ? launch_fwd_sp<D, FP4S, PVM, QP, 2>(tq, tk, tv, a, BH, stream)
+                  : launch_fwd_sp<D, FP4S, PVM, QP, 1>(tq, tk, tv, a, BH, stream);
 }
 
 template <int D, int FP4S>

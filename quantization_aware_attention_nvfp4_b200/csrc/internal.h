@@ -24,6 +24,9 @@ struct FwdArgs {
   // stride nk_tiles, ascending) and their counts; null for dense attention
   const int32_t *kv_list;
   const int32_t *kv_count;
+  // causal masking (Lq == Lk): the lists are the lower triangle of tiles and
+  // each list's diagonal tile keeps keys <= the query row
+  int causal;
 };
 
 struct BwdArgs {
@@ -49,6 +52,7 @@ struct BwdArgs {
   const int32_t *kv_count;
   const int32_t *q_list;
   const int32_t *q_count;
+  int causal;  // as FwdArgs::causal
 };
 
 // Forward.  tv: 3-D TMA map {D, L, B*H} with 64 x 128 boxes, 128-byte swizzle
@@ -109,6 +113,11 @@ cudaError_t launch_scale_do(const __nv_bfloat16 *dO, uint16_t *out, int64_t n, c
 // q_list/q_count per key tile, ascending (see sparse.cu).
 cudaError_t launch_sparse_plan(const uint8_t *mask, int BH, int nq, int nk, int32_t *kv_list, int32_t *kv_count,
                                int32_t *q_list, int32_t *q_count, cudaStream_t stream);
+
+// The same lists for causal masking with nt query and key tiles: key tiles
+// 0..I for query tile I, query tiles J..nt-1 for key tile J.
+cudaError_t launch_causal_plan(int BH, int nt, int32_t *kv_list, int32_t *kv_count, int32_t *q_list,
+                               int32_t *q_count, cudaStream_t stream);
 
 // VSA key-tile selection (see sparse.cu): tile means of q and k into
 // `means` [BH][nq + nk][D], coarse scores into `scores` [BH][nq][nk], and the

@@ -67,6 +67,36 @@ cudaError_t launch_sparse_plan(const uint8_t *mask, int BH, int nq, int nk, int3
   return cudaGetLastError();
 }
 
+// Causal masking walks the lower triangle of tiles: key tiles 0..I for query
+// tile I (the diagonal last), query tiles J..nt-1 for key tile J (the
+// diagonal first).  One warp writes one list.
+__global__ void __launch_bounds__(256) causal_plan_kernel(int BH, int nt, int32_t *__restrict__ kv_list,
+                                                          int32_t *__restrict__ kv_count,
+                                                          int32_t *__restrict__ q_list,
+                                                          int32_t *__restrict__ q_count) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(BH) * nt;
+  if (w < rows) {
+    const int I = static_cast<int>(w % nt);
+    for (int j = lane; j <= I; j += 32) kv_list[w * nt + j] = j;
+    if (lane == 0) kv_count[w] = I + 1;
+  } else if (w < 2 * rows) {
+    const int64_t c = w - rows;
+    const int J = static_cast<int>(c % nt);
+    for (int i = J + lane; i < nt; i += 32) q_list[c * nt + (i - J)] = i;
+    if (lane == 0) q_count[c] = nt - J;
+  }
+}
+
+cudaError_t launch_causal_plan(int BH, int nt, int32_t *kv_list, int32_t *kv_count, int32_t *q_list,
+                               int32_t *q_count, cudaStream_t stream) {
+  const int64_t blocks = (static_cast<int64_t>(BH) * 2 * nt * 32 + 255) / 256;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  causal_plan_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(BH, nt, kv_list, kv_count, q_list, q_count);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------ key-tile selection --
 //
 // VSA selection (vsqa-test-1.3b metadata.json, "attention.selection": top-k

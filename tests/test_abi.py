@@ -200,3 +200,26 @@ def test_vsa_select_host_validation_and_workspace():
     assert sel(ws=FAKE + 16) == A.EINVAL
     assert sel(D=96) == A.EUNSUPPORTED
     assert sel(ws_bytes=lib.attnqat_vsa_select_workspace_size(1, 1, 300, 700, 128) - 1) == A.ENOSPC
+
+
+def test_causal_flag_validation_and_workspace():
+    lib = A.load()
+    big = 1 << 30
+    # causal needs Lq == Lk
+    assert _fwd(lib, Lq=128, Lk=256, flags=15 | A.CAUSAL, ws_bytes=big) == A.EINVAL
+    assert A.attnqat_workspace_size(1, 1, 128, 256, 128, 15 | A.CAUSAL) == 0
+    # the causal workspace adds the tile lists of the lower triangle
+    assert A.attnqat_workspace_size(1, 6, 31200, 31200, 128, 15 | A.CAUSAL) == \
+        A.attnqat_sparse_workspace_size(1, 6, 31200, 31200, 128, 15)
+    assert A.attnqat_sparse_workspace_size(1, 1, 128, 128, 128, 15 | A.CAUSAL) == 0
+    assert _fwd(lib, flags=15 | A.CAUSAL,
+                ws_bytes=A.attnqat_workspace_size(1, 1, 128, 128, 128, 15 | A.CAUSAL) - 1) == A.ENOSPC
+    # no combination with a tile selection
+    st = lib.attnqat_sparse_fwd(P(FAKE), P(FAKE), P(FAKE), 1, 1, 128, 128, 128, 0.125, 15 | A.CAUSAL, P(FAKE),
+                                P(FAKE), P(FAKE), P(FAKE), P(FAKE), big, None)
+    assert st == A.EINVAL
+    assert _fwd(lib, flags=64, ws_bytes=big) == A.EINVAL  # still an unknown bit
+    # causal masking needs every quantizer (fp16 dS and dV operands)
+    for flags in (A.CAUSAL, A.QUANT_Q | A.QUANT_V | A.QUANT_P | A.CAUSAL, A.QUANT_Q | A.QUANT_K | A.CAUSAL):
+        assert _fwd(lib, flags=flags, ws_bytes=big) == A.EINVAL
+    assert _fwd(lib, flags=A.QUANT_ALL | A.CAUSAL, ws_bytes=16) == A.ENOSPC
