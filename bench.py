@@ -14,13 +14,17 @@ measured B200 BF16 tensor peak.  Inputs are seeded synthetic tensors; L2 is
 flushed (a 256 MiB write) between timed steps, each step is timed with CUDA
 events on the launching stream, and multi-GPU runs report the max over ranks.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sparsity S]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sparsity S | --causal]
 
 --sparsity S times the block-sparse (VSA fine attention) step instead:
 attnqat_vsa_select (the top max(1, min(ceil((1-S)*244), 244)) of the 244 key
 tiles per 128-query tile by coarse tile-mean scores; the pages' VSA checkpoint
 uses S = 0.9) + attnqat_sparse_fwd + attnqat_sparse_bwd on the same shape,
 with TFLOP/s counted on the selected tiles only.
+
+--causal times the causal step (ATTNQAT_CAUSAL on attnqat_fwd / attnqat_bwd,
+query i attending keys j <= i) on the same shape, with TFLOP/s counted on the
+unmasked (query, key) pairs, L(L+1)/2 per head.
 
 --impl reference times the float64 CPU oracle on the host cores instead (the
 pages ship no runnable implementation): each step is a bounded sample of the
@@ -49,6 +53,10 @@ WORKLOAD = "wan_6h_31200"
 METRIC = "Attn-QAT fwd+bwd ms & TFLOP/s at H6 L31200 D128; % of B200 BF16 peak"
 SPARSE_METRIC = ("Block-sparse (VSA) Attn-QAT fwd+bwd ms & TFLOP/s on the selected tiles at H6 L31200 D128, "
                  "sparsity %g")
+CAUSAL_METRIC = "Causal Attn-QAT fwd+bwd ms & TFLOP/s on the unmasked pairs at H6 L31200 D128"
+# query rows (= keys) of the oracle's causal sample: its cost grows with the
+# square of the prefix, like the dense sample's rows x all keys
+CAUSAL_SAMPLE_ROWS = int(os.environ.get("ATTNQAT_CAUSAL_BASELINE_ROWS", "15360"))
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 # rows of the oracle's bounded samples (query rows of head 0 against all keys):
@@ -190,7 +198,12 @@ def gpu_arm(args):
     flops = w.nominal_flops()
     peaks = load_peaks()
     sparse = args.sparsity is not None
+    causal = bool(args.causal)
     pairs = float(w.B * w.H * w.Lq * w.Lk)
+    if causal:
+        pairs = float(w.B * w.H) * w.Lq * (w.Lq + 1) / 2.0
+        fwd_f = 4.0 * pairs * w.D
+        flops = dict(fwd=fwd_f, bwd=2.5 * fwd_f, total=3.5 * fwd_f)
     nq, nk = -(-w.Lq // W.SPARSE_TILE), -(-w.Lk // W.SPARSE_TILE)
     topk = W.topk_tiles(nk, args.sparsity) if sparse else nk
 
@@ -200,7 +213,7 @@ def gpu_arm(args):
     host = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16) for n in inp}
     q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
     c = w.sm_scale
-    flags = A.QUANT_ALL
+    flags = A.QUANT_ALL | (A.CAUSAL if causal else 0)
     if sparse:
         tm = torch.empty((w.B, w.H, nq, nk), dtype=torch.uint8, device=dev)
         sel_ws = torch.empty(A.load().attnqat_vsa_select_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D),
@@ -287,7 +300,7 @@ def gpu_arm(args):
     dom_ms = statistics.mean(per[dom])
     achieved = algo_flops[dom] / (dom_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
-    traffic = None if sparse else load_traffic(dom)  # the committed ncu counters are for the dense step
+    traffic = None if (sparse or causal) else load_traffic(dom)  # the committed counters are the dense step's
     kernel_table = {n: dict(launches=len(v), mean_ms=round(statistics.mean(v), 4),
                             share=round(sum(v) / sum(sum(x) for x in per.values()), 4))
                     for n, v in per.items()}
@@ -310,8 +323,11 @@ def gpu_arm(args):
                       key_tiles_per_query_tile=int(mask_np.sum(-1).max()),
                       selected_fraction=round(pairs / (w.B * w.H * w.Lq * w.Lk), 5),
                       selection="attnqat_vsa_select in the timed forward (tile means, top-%d coarse scores)" % topk)
+    if causal:
+        config.update(workload="causal_" + WORKLOAD, mask="causal (query i attends keys j <= i)",
+                      unmasked_fraction=round(pairs / (w.B * w.H * w.Lq * w.Lk), 5))
     out = {
-        "metric": SPARSE_METRIC % args.sparsity if sparse else METRIC,
+        "metric": SPARSE_METRIC % args.sparsity if sparse else (CAUSAL_METRIC if causal else METRIC),
         "value": round(value, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -349,7 +365,8 @@ def gpu_arm(args):
     }
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline_sample(rows=BASELINE_SAMPLE_ROWS, topk=topk if sparse else None)
+            out["cpu_baseline"] = cpu_baseline_sample(rows=CAUSAL_SAMPLE_ROWS if causal else BASELINE_SAMPLE_ROWS,
+                                                      topk=topk if sparse else None, causal=causal)
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
@@ -417,39 +434,44 @@ def load_traffic(kernel):
 
 # -------------------------------------------------------------- CPU oracle --
 
-def cpu_baseline_sample(rows: int, topk=None):
+def cpu_baseline_sample(rows: int, topk=None, causal=False):
     """The float64 oracle on a bounded sample of the workload: head 0, the
     first `rows` query rows against all 31200 keys, forward and backward
     (dQ for those rows, their dK/dV contributions for every key).  Returns the
     nominal TFLOP/s of that sub-problem.  With `topk`, block-sparse: the
     oracle's own selection of head 0 (inside the timed sample), counted on
-    the selected keys."""
+    the selected keys.  With `causal`: the first `rows` tokens of head 0,
+    which attend only to each other, counted on the unmasked pairs."""
     import oracle
     w = W.get(WORKLOAD)
     q = W.head_bits(w, "q", 0, 0)[:rows]
     k = W.head_bits(w, "k", 0, 0)
     v = W.head_bits(w, "v", 0, 0)
+    if causal:
+        k, v = k[:rows], v[:rows]
     do = W.head_bits(w, "do", 0, 0)[:rows]
     T = W.SPARSE_TILE
     t0 = time.perf_counter()
     sel = None
     if topk is not None:
         sel = oracle.vsa_select(W.head_bits(w, "q", 0, 0), k, topk, tile=T)[0][: -(-rows // T)]
-    hd = oracle.Head(q, k, v, w.sm_scale, oracle.QUANT_ALL, do, sel=sel, tile=T)
+    hd = oracle.Head(q, k, v, w.sm_scale, oracle.QUANT_ALL | (oracle.CAUSAL if causal else 0), do, sel=sel, tile=T)
     hd.stats()
     hd.backward()
     dt = time.perf_counter() - t0
     pairs = float(rows * w.Lk)
+    if causal:
+        pairs = rows * (rows + 1) / 2.0
     if sel is not None:
         keys = np.minimum(T, w.Lk - T * np.arange(sel.shape[1]))
         rws = np.minimum(T, rows - T * np.arange(sel.shape[0]))
         pairs = float(rws @ sel.astype(np.float64) @ keys)
     flops = 3.5 * 4.0 * pairs * w.D
-    what = "block-sparse, selected keys only, " if sel is not None else ""
+    what = "block-sparse, selected keys only, " if sel is not None else ("causal, " if causal else "")
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": "head 0, query rows [0,%d) x all %d keys, %sfwd+bwd (float64 C oracle)" % (rows, w.Lk,
-                                                                                                what)}
+            "sample": "head 0, query rows [0,%d) x %s keys, %sfwd+bwd (float64 C oracle)" % (
+                rows, ("the first %d" % rows) if causal else ("all %d" % w.Lk), what)}
 
 
 def reference_arm(args):
@@ -492,7 +514,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--sparsity", type=float, default=None,
                     help="time the block-sparse (VSA) step with this key-tile sparsity instead")
+    ap.add_argument("--causal", action="store_true", help="time the causal step instead")
     args = ap.parse_args()
+    if args.causal and args.sparsity is not None:
+        ap.error("--causal and --sparsity are separate legs")
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
     if args.impl == "reference":
