@@ -475,31 +475,39 @@ def cpu_baseline_sample(rows: int, topk=None, causal=False):
 
 
 def reference_arm(args):
+    """The oracle as the reference arm, on the same leg as the GPU arm (dense,
+    --sparsity or --causal): each step is one bounded sample (see
+    cpu_baseline_sample), timed on the host cores."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     import oracle
     w = W.get(WORKLOAD)
-    rows = ORACLE_SAMPLE_ROWS
+    sparse = args.sparsity is not None
+    causal = bool(args.causal)
+    topk = W.topk_tiles(-(-w.Lk // W.SPARSE_TILE), args.sparsity) if sparse else None
+    # the causal sample's cost grows with the square of its prefix
+    rows = int(ORACLE_SAMPLE_ROWS * 2.5) if causal else ORACLE_SAMPLE_ROWS
     for _ in range(max(0, min(args.warmup, 1))):
-        cpu_baseline_sample(rows=64)
-    times = []
-    for _ in range(args.steps):
-        r = cpu_baseline_sample(rows=rows)
-        times.append(r["seconds"])
-    flops = 3.5 * 4.0 * rows * w.Lk * w.D
-    value = flops * len(times) / sum(times) / 1e12
-    sample = "head 0, query rows [0,%d) x all %d keys, fwd+bwd per step (float64 C oracle)" % (rows, w.Lk)
+        cpu_baseline_sample(rows=64, topk=topk, causal=causal)
+    recs = [cpu_baseline_sample(rows=rows, topk=topk, causal=causal) for _ in range(args.steps)]
+    seconds = sum(r["seconds"] for r in recs)
+    # every step is the same sample: value = its flops over the mean time
+    value = sum(r["value"] * r["seconds"] for r in recs) / seconds
+    metric = SPARSE_METRIC % args.sparsity if sparse else (CAUSAL_METRIC if causal else METRIC)
+    config = {"workload": ("vsa_" if sparse else ("causal_" if causal else "")) + WORKLOAD, "B": w.B, "H": w.H,
+              "Lq": w.Lq, "Lk": w.Lk, "D": w.D, "quantizers": "q,k,v,p", "sample_rows": rows}
+    if sparse:
+        config.update(sparsity=args.sparsity, tile=W.SPARSE_TILE)
     out = {
         "impl": "reference",
-        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sum(times) / len(times), 1),
+        "metric": metric, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * seconds / len(recs), 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16)",
-        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
-                   "quantizers": "q,k,v,p", "sample_rows": rows},
+        "config": config,
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": recs[0]["sample"] + ", one per step"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
