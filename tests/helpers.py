@@ -103,3 +103,26 @@ def run_attention(inp: dict, sm_scale: float, flags: int, backward: bool = True)
     torch.cuda.synchronize()
     A.attnqat_device_status()
     return out
+
+
+CANARY = 0xA5
+
+
+def guarded(shape, dtype, device, guard_bytes=4096):
+    """A contiguous tensor of `shape` inside a larger byte buffer whose
+    `guard_bytes` on each side hold the canary byte (compute-sanitizer is not
+    available: out-of-bounds writes show up as changed guard bytes).
+    Returns (buffer, tensor view)."""
+    import math
+    import torch
+    esize = torch.empty((), dtype=dtype).element_size()
+    nbytes = math.prod(shape) * esize
+    buf = torch.full((2 * guard_bytes + nbytes,), CANARY, dtype=torch.uint8, device=device)
+    view = buf[guard_bytes:guard_bytes + nbytes].view(dtype).view(shape)
+    return buf, view
+
+
+def guards_intact(buf, guard_bytes=4096) -> bool:
+    import torch
+    head, tail = buf[:guard_bytes], buf[buf.numel() - guard_bytes:]
+    return bool(torch.all(head == CANARY)) and bool(torch.all(tail == CANARY))
