@@ -1,9 +1,11 @@
 /*
  * attnqat.h -- C ABI of the B200 (sm_100a) Attn-QAT attention library.
  *
- * Attn-QAT training attention: non-causal multi-head attention whose operands
- * are NVFP4 fake-quantized (fq) inside the op, with a straight-through
- * backward.  The method and its format come from these pages:
+ * Attn-QAT training attention: multi-head attention whose operands are NVFP4
+ * fake-quantized (fq) inside the op, with a straight-through backward --
+ * non-causal as the pages' route (attnqat_fwd / attnqat_bwd), plus the VSA
+ * block-sparse fine attention with its key-tile selection and causal masking
+ * (declared further down).  The method and its format come from these pages:
  *  - FastVideo "Attn-QAT Training" guide, section "Architecture-specific
  *    Triton routing": non-causal BF16 attention, head dimension 128, query
  *    and key/value lengths may differ (K and V share one), the optimized
@@ -197,8 +199,8 @@ size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D,
  * 256-byte aligned; it must be passed unchanged to attnqat_bwd.
  * flags may add ATTNQAT_CAUSAL (then Lq == Lk and ATTNQAT_QUANT_ALL are
  * required).
- * Shapes: B, H >= 1; Lq >= 1; Lk >= 1; D in {64, 128}; B*H*max(Lq,Lk)*D
- * below 2^31.  Lq is arbitrary (the last query tile is masked); a partial
+ * Shapes: B, H >= 1; B*H <= 65535; Lq >= 1; Lk >= 1; D in {64, 128};
+ * B*H*max(Lq,Lk)*128 below 2^40 (offsets are 64-bit).  Lq is arbitrary (the last query tile is masked); a partial
  * last KV tile runs the separate masked tail step.  Lk need not be 16-aligned
  * (the pages' SM100 backward requires it; here a ragged last block of 16 keys
  * or tokens is zero-padded: its missing keys get P~ = 0 and its missing V
