@@ -186,7 +186,11 @@ def global_scale(amax: float) -> float:
 
 def quantize_rows_gs(x_bits: np.ndarray, rows: int, cols: int, stride_row: int,
                      stride_col: int):
-    """NVFP4 with an FP32 global scale (reading R15) of a strided bf16 view.
+    """NVFP4 with an FP32 global scale of a strided bf16 view: G = float32
+    2688 / max|x| (1 for an all-zero view), block scale = E4M3 of the exact
+    a_b G / 6, code = E2M1 of the exact |x| G / s_b, value = sign * E2M1 *
+    s_b / G rounded once to bf16 (the page gives the format, not the order of
+    these steps; exact two-level rounding is the plain reading).
 
     Returns (codes uint8 [rows, cols/2], scales uint8 [rows, cols/16],
     deq bf16 bits uint16 [rows, cols], global scale float)."""
@@ -318,8 +322,9 @@ class Head:
 
 
 def vsa_select(q_bits, k_bits, topk, tile=128):
-    """Key-tile selection of block-sparse attention for one head (reading
-    R17 in oracle.c): tile means, float32 coarse scores, the topk best key
+    """Key-tile selection of block-sparse attention for one head: tile means,
+    float32 coarse scores (mean query row . mean key row, every step in a
+    fixed order, since the ranking decides an integer), the topk best key
     tiles per query tile (ties to the lower index).  q [Lq, D], k [Lk, D]
     bf16 bits.  Returns (mask uint8 [nq, nk], scores float32 [nq, nk])."""
     q = _bits(q_bits)

@@ -27,8 +27,7 @@
  *  dV = (fq(P~)/l)^T dO, dP = dO fq(V)^T, dS = P o (dP - Delta),
  *  Delta = rowsum(dO o O), dQ = dS fq(K) c, dK = dS^T fq(Q) c, P = P~/l.
  *
- * Readings taken where the pages are silent (each is listed with its evidence
- * in the design notes of this repository):
+ * Readings taken where the pages are silent:
  *  - m is the exact row max over all keys (not a running max);
  *  - l sums the unquantized P~;
  *  - dV uses the forward's fq(P~) divided by l (blocks along keys); the literal
@@ -251,8 +250,8 @@ void oracle_quantize_rows(const uint16_t *x, long rows, long cols, long srow,
 /* The linear-layer variant of the format (vsqa-test-1.3b metadata.json,
  * "linear_quantization": "NVFP4 W4A4: E2M1 values, 16-element blocks, FP8
  * E4M3 block scales, FP32 global scale", with the activation global scale
- * "dynamic, 448*6/max|X| recomputed every forward").  The reading of the
- * steps the page leaves open (listed in the design notes as R15):
+ * "dynamic, 448*6/max|X| recomputed every forward").  The page does not fix
+ * the order of the steps; they are read as exact two-level rounding:
  *   G   = the float32 quotient 2688 / max|x| (1 when max|x| = 0; the largest
  *         finite float32 if the quotient overflows);
  *   k_b = E4M3 round-to-nearest-even (saturating) of the exact a_b * G / 6,
@@ -640,7 +639,7 @@ void oracle_bwd_dkdv_blocks(const double *Qh, const double *Kh, const double *Vh
  * "attention.selection": top-k key cubes per query cube with
  * effective_topk = max(1, min(ceil((1 - sparsity) * num_blocks), num_blocks);
  * "attention.precision.coarse": BF16, quantize_coarse false).  Reading (the
- * page gives the fields, not the arithmetic; listed as R17): each T-token
+ * page gives the fields, not the arithmetic): each T-token
  * tile is summarised by the mean of its valid rows; the coarse score of
  * (query tile I, key tile J) is the dot product of the two means (the softmax
  * scale and the softmax itself do not change the order); query tile I keeps
