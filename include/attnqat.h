@@ -37,10 +37,13 @@
  *  - Tensors are dense, contiguous, row-major bf16 in BHSD order:
  *    q, o, dO, dq: [B][H][Lq][D]; k, v, dk, dv: [B][H][Lk][D].  m, lse:
  *    float32 [B][H][Lq].  All pointers are device pointers unless stated.
- *  - The caller owns every buffer.  The library allocates no device memory and
- *    keeps no state beyond a once-per-process setup of kernel attributes and
- *    of the driver entry point used to encode TMA descriptors.  Inputs are
- *    never written.
+ *  - The caller owns every buffer; no call allocates device memory.  The
+ *    library's state is a once-per-process setup of kernel attributes and of
+ *    the driver entry point used to encode TMA descriptors, a per-device
+ *    record of the device check, the device status word below, and one
+ *    static block of ATTNQAT_NOALLOC_WS_MAX bytes per device that only
+ *    attnqat_fwd_noalloc uses (held by every GPU that loads the library).
+ *    Inputs are never written.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Work is enqueued asynchronously; all argument checks run on the
  *    host before any launch.  There is no CPU fallback.
@@ -77,14 +80,14 @@ extern "C" {
 #define ATTNQAT_QUANT_P 8u
 #define ATTNQAT_QUANT_ALL 15u
 /* Causal masking (attnqat_fwd / attnqat_bwd / attnqat_workspace_size only;
- * needs Lq == Lk and every quantizer on, ATTNQAT_QUANT_ALL, whose exact fp16
- * operands carry dS and the dV operand with 11 significant bits -- with bf16
- * ones the gradients of the first keys, which every later row feeds, are not
- * accurate enough): query i attends to keys j <= i.  The pages' training route
- * is non-causal (FastVideo "Attn-QAT Training" guide, "Architecture-specific
- * Triton routing"); the mask is applied like a tile selection: masked keys
- * have P~ = 0 inside their fq(P~) blocks, m and l run over the unmasked keys,
- * and only the lower triangle of 128 x 128 tiles is computed. */
+ * needs Lq == Lk; any quantizer flags): query i attends to keys j <= i.  The
+ * first keys' gradients gather every later row's contribution, which the
+ * backward's fp16 dS and dV operands (11 significant bits) carry accurately.
+ * The pages' training route is non-causal (FastVideo "Attn-QAT Training"
+ * guide, "Architecture-specific Triton routing"); the mask is applied like a
+ * tile selection: masked keys have P~ = 0 inside their fq(P~) blocks, m and l
+ * run over the unmasked keys, and only the lower triangle of 128 x 128 tiles
+ * is computed. */
 #define ATTNQAT_CAUSAL 32u
 
 /* Text for a status code (static storage). */
@@ -109,6 +112,20 @@ int attnqat_profile_read(const char **names, float *ms, int max_records);
  * ATTNQAT_ETIMEOUT (and clears the flag). */
 int attnqat_device_status(void);
 
+/* Self-test of that failure path (no counterpart on the pages: it checks the
+ * library's own fail-loudly machinery).  Launches one small kernel on
+ * `stream` that takes the steps an attention kernel takes when a wait gives
+ * up, on an mbarrier nothing ever arrives at: it allocates TMEM, starts a
+ * bulk copy into shared memory, waits limit_ns nanoseconds (1000 <= limit_ns
+ * <= 2e9), sets its abort flag -- a second waiting role sees it and leaves --
+ * lets the copy land, and frees the TMEM.  Each of the two waits that ends
+ * without its barrier adds 1 to *waits_ended (a device int, 4-byte aligned),
+ * and the device status word is raised, so the next attnqat_device_status()
+ * returns ATTNQAT_ETIMEOUT.  No fault is raised and the context stays usable.
+ * Errors: EINVAL (null or misaligned waits_ended, limit out of range),
+ * EUNSUPPORTED, ECUDA. */
+int attnqat_selftest_wait_timeout(unsigned long long limit_ns, int *waits_ended, void *stream);
+
 /*
  * attnqat_quantize -- standalone NVFP4 quantizer (fq of a strided bf16 view).
  *
@@ -125,7 +142,8 @@ int attnqat_device_status(void);
  *  - V blocked along tokens: batch = B*H, rows = D, cols = Lk,
  *    strides (Lk*D, 1, D)  (the transposed view of each head).
  * Outputs (device, dense, caller-owned):
- *  - codes  [batch][rows][cols/2] bytes: element 2i in the low nibble and
+ *  - codes  [batch][rows][cols/2] bytes, 8-byte aligned (each block's 16
+ *    nibbles are written as one 8-byte group): element 2i in the low nibble and
  *    2i+1 in the high nibble; nibble = sign bit (bit 3, the input's sign,
  *    also for values that round to 0) | 3-bit E2M1 magnitude code.
  *  - scales [batch][rows][cols/16] bytes: E4M3 codes, sign bit 0.
@@ -133,8 +151,9 @@ int attnqat_device_status(void);
  *    sign * E2M1 * scale, which bf16 represents exactly.
  * Codes and scales are bit-exact round-to-nearest-even results of the exact
  * quotients amax/6 and |x|/s.  Inputs must be finite.
- * Errors: EINVAL for null x/codes/scales, cols % 16 != 0, non-positive
- * rows/cols/batch, negative strides, or sizes above 2^40 elements.
+ * Errors: EINVAL for null x/codes/scales, codes not 8-byte aligned, cols % 16
+ * != 0, non-positive rows/cols/batch, negative strides, or sizes above 2^40
+ * elements.
  */
 int attnqat_quantize(const void *x, int64_t batch, int64_t rows, int64_t cols,
                      int64_t stride_batch, int64_t stride_row,
@@ -171,18 +190,20 @@ int attnqat_quantize_gs(const void *x, int64_t batch, int64_t rows,
 
 /*
  * attnqat_workspace_size -- bytes of device workspace attnqat_fwd and
- * attnqat_bwd need for this shape and flag set (0 for invalid shapes).  The
- * workspace holds the dequantized fq(Q), fq(K), fq(V) operands (fp16 when
- * both Q and K are quantized, else bf16, plus an fp16 copy of fq(V) for the
- * P V product -- every fq'd value is exact in both), a float32 copy of O
- * written by the forward, the backward's Delta, 16 bytes of statistics, an
- * exact fp16 copy of dO * 2^e when all four quantizers are on, and -- with Q
- * and K quantized -- their packed NVFP4 codes (D/2 bytes per row) with scale
- * tiles (512 bytes per 128 rows x 64 columns) for the block-scaled
- * S = fq(Q) fq(K)^T; with all four quantizers on, D = 128 and Lk % 32 == 0
- * also fq(V)'s packed codes ([B*H][D][Lk/2] bytes, blocks along tokens) and
- * scale tiles (1 KB per 128 tokens) for the forward's block-scaled
- * fq(P~) fq(V).  Every region is 256-byte aligned.
+ * attnqat_bwd need for this shape and flag set (0 for invalid shapes).  Every
+ * 16-bit operand of the attention's matrix products is fp16, so the
+ * workspace holds fp16 copies of Q, K, V and dO: fq(X) for a quantized
+ * operand (exact: sign * E2M1 * E4M3 values lie in [2^-10, 2688] with at most
+ * 7 significant bits), else X * 2^e with 2^e a power of two that maps max |X|
+ * into [2^13, 2^14) (exact for every element within 2^27 of the largest).  It
+ * also holds a float32 copy of O written by the forward, the backward's Delta,
+ * 32 bytes of statistics (the max magnitudes behind those powers of two and
+ * the bound on |dS|), and -- with Q and K quantized -- their packed NVFP4
+ * codes (D/2 bytes per row) with scale tiles (512 bytes per 128 rows x 64
+ * columns) for the block-scaled S = fq(Q) fq(K)^T; with all four quantizers
+ * on and Lk % 32 == 0 also fq(V)'s packed codes ([B*H][D][Lk/2]
+ * bytes, blocks along tokens) and scale tiles (1 KB per 128 tokens) for the
+ * forward's block-scaled fq(P~) fq(V).  Every region is 256-byte aligned.
  */
 size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D,
                               uint32_t flags);
@@ -197,8 +218,7 @@ size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D,
  * float32 (the exact row max of the scaled scores).  ws/ws_bytes: device
  * workspace of at least attnqat_workspace_size(B,H,Lq,Lk,D,flags) bytes,
  * 256-byte aligned; it must be passed unchanged to attnqat_bwd.
- * flags may add ATTNQAT_CAUSAL (then Lq == Lk and ATTNQAT_QUANT_ALL are
- * required).
+ * flags may add ATTNQAT_CAUSAL (then Lq == Lk is required).
  * Shapes: B, H >= 1; B*H <= 65535; Lq >= 1; Lk >= 1; D in {64, 128};
  * B*H*max(Lq,Lk)*128 below 2^40 (offsets are 64-bit).  Lq is arbitrary (the last query tile is masked); a partial
  * last KV tile runs the separate masked tail step.  Lk need not be 16-aligned
@@ -315,10 +335,14 @@ int attnqat_vsa_select(const void *q, const void *k, int B, int H, int Lq,
  * the process exits).  It calls no cudaMalloc, cudaFree or other allocating
  * routine.
  *  - Shapes with attnqat_workspace_size(...) > ATTNQAT_NOALLOC_WS_MAX return
- *    ATTNQAT_ENOSPC; invalid shapes ATTNQAT_EINVAL (as attnqat_fwd).
+ *    ATTNQAT_ENOSPC; invalid arguments return the code attnqat_fwd returns
+ *    for them (EINVAL, or EUNSUPPORTED for a head dimension it lacks or a
+ *    device that is not sm_100).
  *  - The first call on each device looks up the block's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before capturing the stream into a CUDA graph.
+ *    before capturing the stream into a CUDA graph.  The address is kept per
+ *    device and CUDA context: after a cudaDeviceReset the next call looks it
+ *    up again (so, again, before any capture).
  *  - All calls share the block and it keeps the last call's contents (the
  *    parts that must start at zero are cleared on the caller's stream).
  *    Calls whose GPU work overlaps -- two streams, or several host threads on

@@ -79,6 +79,8 @@ def load(build_if_needed: bool = True):
             lib.attnqat_last_cuda_error.argtypes = []
             lib.attnqat_device_status.restype = I
             lib.attnqat_device_status.argtypes = []
+            lib.attnqat_selftest_wait_timeout.restype = I
+            lib.attnqat_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, P, P]
             lib.attnqat_profile_enable.restype = I
             lib.attnqat_profile_enable.argtypes = [I]
             lib.attnqat_profile_read.restype = I
@@ -389,3 +391,15 @@ def attnqat_device_status() -> int:
     st = load().attnqat_device_status()
     _check(st, "attnqat_device_status")
     return st
+
+
+def attnqat_selftest_wait_timeout(limit_ns: int = 1000000, stream=None) -> int:
+    """Runs the library's timed-out-wait path on purpose (see attnqat.h) and
+    returns how many waits ended without their barrier (2 when it works).
+    Leaves the device status raised: the next attnqat_device_status() call
+    raises ETIMEOUT and clears it."""
+    torch = _torch()
+    ended = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(load().attnqat_selftest_wait_timeout(int(limit_ns), ctypes.c_void_p(ended.data_ptr()),
+                                                _stream_ptr(stream)), "attnqat_selftest_wait_timeout")
+    return int(ended.item())

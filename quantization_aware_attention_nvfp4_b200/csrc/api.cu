@@ -175,61 +175,65 @@ static bool encode_vcodes(CUtensorMap *map, const void *base, int BH, int Lk, in
 // ------------------------------------------------------------- workspace --
 
 struct Workspace {
-  size_t qh, kh, vh, vh16, o32, delta, stats, do16, qc, qsf, kc, ksf, vc, vsf, total;
+  size_t qh, kh, vh16, o32, delta, stats, do16, qc, qsf, kc, ksf, vc, vsf, total;
   size_t qsf_bytes, ksf_bytes, vsf_bytes;
   size_t kv_list, kv_count, q_list, q_count;  // block-sparse tile lists
 };
 
-// fq(Q) and fq(K) are exact in fp16 (values sign * E2M1 * E4M3 lie in
-// [2^-10, 2688] with at most 7 significant bits), so when both are quantized
-// they are kept as fp16 and S = fq(Q) fq(K)^T, dQ and dK run as fp16 MMAs,
-// which lets the backward feed dS as fp16 (3 more mantissa bits than bf16).
-static bool qk_f16(uint32_t flags) {
-  return (flags & ATTNQAT_QUANT_Q) && (flags & ATTNQAT_QUANT_K);
-}
-
-// With every operand quantized, fq(V) is exact in fp16 as well, so the
-// backward runs dP and dV as fp16 MMAs on an exact fp16 copy of dO (dO * 2^e:
-// bf16 has 8 significant bits) -- dP stays exact and the dV operand
-// fq(P~)/l gets 11 significant bits instead of bf16's 8.
-static bool do_f16(uint32_t flags) { return (flags & ATTNQAT_QUANT_ALL) == ATTNQAT_QUANT_ALL; }
+// With Q and K both quantized, S = fq(Q) fq(K)^T runs as a block-scaled NVFP4
+// MMA on their packed codes (every product of two E2M1 codes and two E4M3
+// scales is exact in float32).
+static bool fp4s(uint32_t flags) { return (flags & ATTNQAT_QUANT_Q) && (flags & ATTNQAT_QUANT_K); }
 
 // With every quantizer on, fq(P~) fq(V) is also a product of NVFP4 blocks
 // along its K axis (keys for P~, tokens for V), so the forward's P V runs as
-// a block-scaled NVFP4 MMA (M = 128 queries, N = D = 128) on fq(V)'s packed
-// codes [B*H][D][Lk/2] -- whose rows the TMA reads need 16-byte aligned:
-// Lk % 32 == 0.  D = 64 keeps the fp16 P V.
-static bool pv_fp4(uint32_t flags, int Lk, int D) { return do_f16(flags) && (Lk % 32) == 0 && D == 128; }
+// a block-scaled NVFP4 MMA (M = 128 queries, N = D) on fq(V)'s packed codes
+// [B*H][D][Lk/2] -- whose rows the TMA reads need 16-byte aligned:
+// Lk % 32 == 0.
+static bool pv_fp4(uint32_t flags, int Lk, int D) {
+  (void)D;  // both head dimensions (N = 64 or 128)
+  return (flags & ATTNQAT_QUANT_ALL) == ATTNQAT_QUANT_ALL && (Lk % 32) == 0;
+}
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Statistics block (float32): [0] max_i |dO_i|_1, [1] max_i |Delta_i|,
+// [2] max |fq(V)| (or max |V|), [3] max |dO|, [4] max |Q| and [5] max |K|
+// (only when that operand is not quantized: the scales of their fp16 copies).
+constexpr size_t kStatsBytes = 32;
+
+// Every 16-bit operand of the attention MMAs is fp16: fq(Q), fq(K), fq(V)
+// are exact in fp16 (values sign * E2M1 * E4M3 lie in [2^-10, 2688] with at
+// most 7 significant bits), and an operand whose quantizer is off is copied as
+// X * 2^e, a power of two that maps its max magnitude into [2^13, 2^14) (bf16
+// has 8 significant bits, so the copy is exact for every element within 2^27
+// of the largest).  dO gets the same copy.  So the backward feeds dS and the
+// dV operand P/l as fp16 (11 significant bits) whatever the flags.
 static Workspace layout(int B, int H, int Lq, int Lk, int D, uint32_t flags, bool sparse = false) {
   Workspace w{};
   const size_t BH = static_cast<size_t>(B) * H;
   const size_t qbytes = BH * Lq * D * 2, kbytes = BH * Lk * D * 2;
   size_t off = 0;
   w.qh = off;
-  if (flags & ATTNQAT_QUANT_Q) off = align256(off + qbytes);
+  off = align256(off + qbytes);
   w.kh = off;
-  if (flags & ATTNQAT_QUANT_K) off = align256(off + kbytes);
-  w.vh = off;
-  if (flags & ATTNQAT_QUANT_V) off = align256(off + kbytes);
+  off = align256(off + kbytes);
   w.vh16 = off;
-  if (flags & ATTNQAT_QUANT_V) off = align256(off + kbytes);
+  off = align256(off + kbytes);
   w.o32 = off;
   off = align256(off + BH * Lq * D * 4);
   w.delta = off;
   off = align256(off + BH * Lq * 4);
-  w.stats = off;  // [0] max_i |dO_i|_1, [1] max_i |Delta_i|, [2] max |fq(V)|, [3] max |dO_i|/l_i
-  off = align256(off + 16);
-  w.do16 = off;   // exact fp16 copy dO * 2^e (all-quantized path)
-  if (do_f16(flags)) off = align256(off + BH * Lq * D * 2);
+  w.stats = off;
+  off = align256(off + kStatsBytes);
+  w.do16 = off;   // fp16 copy dO * 2^e
+  off = align256(off + qbytes);
   // packed NVFP4 codes of fq(Q), fq(K) and their scales in 128-row tiles
-  // (512 bytes per 128 rows x 64 columns), read by the forward's S MMA
+  // (512 bytes per 128 rows x 64 columns), read by the S MMAs
   const size_t ntq = (static_cast<size_t>(Lq) + 127) / 128, ntk = (static_cast<size_t>(Lk) + 127) / 128;
   w.qsf_bytes = BH * ntq * (D / 64) * 512;
   w.ksf_bytes = BH * ntk * (D / 64) * 512;
-  const bool fp4 = qk_f16(flags);
+  const bool fp4 = fp4s(flags);
   w.qc = off;
   if (fp4) off = align256(off + BH * Lq * D / 2);
   w.qsf = off;
@@ -264,12 +268,6 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 static int check_shape(int B, int H, int Lq, int Lk, int D, float sm_scale, uint32_t flags) {
   if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return ATTNQAT_EINVAL;
   if ((flags & ATTNQAT_CAUSAL) && Lq != Lk) return ATTNQAT_EINVAL;  // query i and key i are one token
-  // causal masking runs with every quantizer on, whose exact fp16 operands
-  // carry dS and the dV operand fq(P~)/l with 11 significant bits: with bf16
-  // ones the heavy-tailed gradients of the first keys (fed by every later
-  // row) miss the max-abs bar -- dK 5.3e-2 of RMS with no quantizer, dV
-  // 8.0e-2 with Q and K alone, measured at L = 500
-  if ((flags & ATTNQAT_CAUSAL) && (flags & ATTNQAT_QUANT_ALL) != ATTNQAT_QUANT_ALL) return ATTNQAT_EINVAL;
   if (static_cast<int64_t>(B) * H > 65535) return ATTNQAT_EINVAL;  // grid.y
   const int64_t Lmax = Lq > Lk ? Lq : Lk;
   if (static_cast<int64_t>(B) * H * Lmax * 128 >= (int64_t(1) << 40)) return ATTNQAT_EINVAL;
@@ -279,42 +277,55 @@ static int check_shape(int B, int H, int Lq, int Lk, int D, float sm_scale, uint
   return ATTNQAT_OK;
 }
 
-// Writes fq(Q), fq(K), fq(V) into the workspace (as the flags ask) and
-// returns the operand pointers the attention kernels read.
+// Writes the fp16 operands -- fq(Q), fq(K), fq(V), or the scaled copies of
+// the operands whose quantizer is off -- and the packed NVFP4 codes into the
+// workspace, and the max magnitudes that scale the copies into its
+// statistics block.
 static int prepare_operands(const void *q, const void *k, const void *v, int B, int H, int Lq, int Lk,
                             int D, uint32_t flags, uint8_t *ws, const Workspace &w,
                             cudaStream_t stream) {
   const int64_t BH = static_cast<int64_t>(B) * H;
-  const bool f16 = qk_f16(flags);
+  const bool fp4 = fp4s(flags);
   float *stats = reinterpret_cast<float *>(ws + w.stats);
-  cudaError_t e = cudaMemsetAsync(stats, 0, 16, stream);
+  cudaError_t e = cudaMemsetAsync(stats, 0, kStatsBytes, stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  // With Q and K both quantized one pass writes the exact fp16 fq (for the
-  // backward) and the packed codes with tiled scales (for the forward's S);
+  // A quantized operand: one pass writes the exact fp16 fq and, with Q and K
+  // both quantized, the packed codes with tiled scales (for the S MMAs);
   // scale tiles are cleared first when the last 128-row tile is partial, so
-  // its padding rows carry zero scales.
-  auto quant_qk = [&](const void *x, int L, size_t deq_off, size_t c_off, size_t sf_off, size_t sf_bytes,
-                      const char *name) -> int {
+  // its padding rows carry zero scales.  An unquantized one: its max
+  // magnitude, then the scaled fp16 copy.
+  auto prep_qk = [&](const void *x, bool quantized, int L, size_t deq_off, size_t c_off, size_t sf_off,
+                     size_t sf_bytes, float *amax, const char *qname, const char *aname,
+                     const char *cname) -> int {
     uint16_t *dst = reinterpret_cast<uint16_t *>(ws + deq_off);
-    if (f16 && (L % 128) != 0) {
-      cudaError_t em = cudaMemsetAsync(ws + sf_off, 0, sf_bytes, stream);
-      if (em != cudaSuccess) return cuda_fail(em);
+    if (quantized) {
+      if (fp4 && (L % 128) != 0) {
+        cudaError_t em = cudaMemsetAsync(ws + sf_off, 0, sf_bytes, stream);
+        if (em != cudaSuccess) return cuda_fail(em);
+      }
+      ProfScope ps(qname, stream);
+      cudaError_t eq = launch_quantize(static_cast<const uint16_t *>(x), 1, BH * L, D, 0, D, 1,
+                                       fp4 ? ws + c_off : nullptr, fp4 ? ws + sf_off : nullptr, nullptr, dst,
+                                       nullptr, stream, fp4 ? L : 0);
+      return eq == cudaSuccess ? ATTNQAT_OK : cuda_fail(eq);
     }
-    ProfScope ps(name, stream);
-    cudaError_t eq = launch_quantize(static_cast<const uint16_t *>(x), 1, BH * L, D, 0, D, 1,
-                                     f16 ? ws + c_off : nullptr, f16 ? ws + sf_off : nullptr,
-                                     f16 ? nullptr : dst, f16 ? dst : nullptr, nullptr, stream,
-                                     f16 ? L : 0);
-    return eq == cudaSuccess ? ATTNQAT_OK : cuda_fail(eq);
+    cudaError_t ea;
+    {
+      ProfScope ps(aname, stream);
+      ea = launch_absmax(static_cast<const __nv_bfloat16 *>(x), BH * L * D, amax, stream);
+    }
+    if (ea != cudaSuccess) return cuda_fail(ea);
+    ProfScope ps(cname, stream);
+    ea = launch_scale_f16(static_cast<const __nv_bfloat16 *>(x), dst, BH * L * D, amax, stream);
+    return ea == cudaSuccess ? ATTNQAT_OK : cuda_fail(ea);
   };
-  if (flags & ATTNQAT_QUANT_Q) {
-    const int st = quant_qk(q, Lq, w.qh, w.qc, w.qsf, w.qsf_bytes, "quantize_q");
-    if (st != ATTNQAT_OK) return st;
-  }
-  if (flags & ATTNQAT_QUANT_K) {
-    const int st = quant_qk(k, Lk, w.kh, w.kc, w.ksf, w.ksf_bytes, "quantize_k");
-    if (st != ATTNQAT_OK) return st;
-  }
+  int st = prep_qk(q, (flags & ATTNQAT_QUANT_Q) != 0, Lq, w.qh, w.qc, w.qsf, w.qsf_bytes, stats + 4, "quantize_q",
+                   "absmax_q", "scale_q");
+  if (st != ATTNQAT_OK) return st;
+  st = prep_qk(k, (flags & ATTNQAT_QUANT_K) != 0, Lk, w.kh, w.kc, w.ksf, w.ksf_bytes, stats + 5, "quantize_k",
+               "absmax_k", "scale_k");
+  if (st != ATTNQAT_OK) return st;
+  uint16_t *vdst = reinterpret_cast<uint16_t *>(ws + w.vh16);
   if (flags & ATTNQAT_QUANT_V) {
     // blocks of 16 consecutive tokens per channel: the transposed view
     const bool pv4 = pv_fp4(flags, Lk, D);
@@ -323,18 +334,31 @@ static int prepare_operands(const void *q, const void *k, const void *v, int B, 
       if (e != cudaSuccess) return cuda_fail(e);
     }
     ProfScope ps("quantize_v", stream);
-    // the bf16 copy feeds only the backward's bf16 dP / dV, unused when every
-    // quantizer is on (the fp16 copy and the codes serve both passes then)
     e = launch_quantize(static_cast<const uint16_t *>(v), BH, D, Lk, static_cast<int64_t>(Lk) * D, 1, D,
-                        pv4 ? ws + w.vc : nullptr, pv4 ? ws + w.vsf : nullptr,
-                        do_f16(flags) ? nullptr : reinterpret_cast<uint16_t *>(ws + w.vh),
-                        reinterpret_cast<uint16_t *>(ws + w.vh16), stats + 2, stream, 0, pv4);
+                        pv4 ? ws + w.vc : nullptr, pv4 ? ws + w.vsf : nullptr, nullptr, vdst, stats + 2, stream, 0,
+                        pv4);
+    if (e != cudaSuccess) return cuda_fail(e);
   } else {
-    ProfScope ps("absmax_v", stream);
-    e = launch_absmax(static_cast<const __nv_bfloat16 *>(v), BH * Lk * D, stats + 2, stream);
+    {
+      ProfScope ps("absmax_v", stream);
+      e = launch_absmax(static_cast<const __nv_bfloat16 *>(v), BH * Lk * D, stats + 2, stream);
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    ProfScope ps("scale_v", stream);
+    e = launch_scale_f16(static_cast<const __nv_bfloat16 *>(v), vdst, BH * Lk * D, stats + 2, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
   }
-  if (e != cudaSuccess) return cuda_fail(e);
   return ATTNQAT_OK;
+}
+
+// The max magnitudes that scale the fp16 copies of unquantized operands
+// (null for a quantized operand: its fq copy is unscaled).
+static void operand_amax(uint32_t flags, uint8_t *wsb, const Workspace &w, const float **aq, const float **ak,
+                         const float **av) {
+  const float *stats = reinterpret_cast<const float *>(wsb + w.stats);
+  *aq = (flags & ATTNQAT_QUANT_Q) ? nullptr : stats + 4;
+  *ak = (flags & ATTNQAT_QUANT_K) ? nullptr : stats + 5;
+  *av = (flags & ATTNQAT_QUANT_V) ? nullptr : stats + 2;
 }
 
 }  // namespace attnqat
@@ -404,7 +428,9 @@ int attnqat_quantize(const void *x, int64_t batch, int64_t rows, int64_t cols, i
   if (stride_batch < 0 || stride_row < 0 || stride_col < 0) return ATTNQAT_EINVAL;
   const int64_t lim = int64_t(1) << 40;
   if (batch > lim || rows > lim || cols > lim || batch * rows > lim / cols) return ATTNQAT_EINVAL;
-  if ((reinterpret_cast<uintptr_t>(x) & 1u) || (deq && (reinterpret_cast<uintptr_t>(deq) & 1u)))
+  // codes are written as 8-byte groups (one 16-element block each)
+  if ((reinterpret_cast<uintptr_t>(x) & 1u) || (deq && (reinterpret_cast<uintptr_t>(deq) & 1u)) ||
+      (reinterpret_cast<uintptr_t>(codes) & 7u))
     return ATTNQAT_EINVAL;
   const int st = check_device();
   if (st != ATTNQAT_OK) return st;
@@ -423,7 +449,7 @@ int attnqat_quantize_gs(const void *x, int64_t batch, int64_t rows, int64_t cols
   const int64_t lim = int64_t(1) << 40;
   if (batch > lim || rows > lim || cols > lim || batch * rows > lim / cols) return ATTNQAT_EINVAL;
   if ((reinterpret_cast<uintptr_t>(x) & 1u) || (deq && (reinterpret_cast<uintptr_t>(deq) & 1u)) ||
-      (reinterpret_cast<uintptr_t>(gscale) & 3u))
+      (reinterpret_cast<uintptr_t>(gscale) & 3u) || (reinterpret_cast<uintptr_t>(codes) & 7u))
     return ATTNQAT_EINVAL;
   const int st = check_device();
   if (st != ATTNQAT_OK) return st;
@@ -479,16 +505,12 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
   const int BH = B * H;
   st = plan_sparse(mask, causal, BH, Lq, Lk, wsb, w, s);
   if (st != ATTNQAT_OK) return st;
-  const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
-  const void *kh = (flags & ATTNQAT_QUANT_K) ? static_cast<const void *>(wsb + w.kh) : k;
-  const bool pv_f16 = (flags & ATTNQAT_QUANT_V) != 0;
+  const bool fp4 = fp4s(flags);
   const bool pv4 = pv_fp4(flags, Lk, D);
-  const void *vh = pv_f16 ? static_cast<const void *>(wsb + w.vh16) : v;
-  const bool f16 = qk_f16(flags);
   CUtensorMap tq, tk, tv;
-  const bool maps_ok = f16 ? encode_codes(&tq, wsb + w.qc, BH, Lq, D) && encode_codes(&tk, wsb + w.kc, BH, Lk, D)
-                           : encode_bhld(&tq, qh, BH, Lq, D, false) && encode_bhld(&tk, kh, BH, Lk, D, false);
-  const bool vmap_ok = pv4 ? encode_vcodes(&tv, wsb + w.vc, BH, Lk, D) : encode_bhld(&tv, vh, BH, Lk, D, pv_f16);
+  const bool maps_ok = fp4 ? encode_codes(&tq, wsb + w.qc, BH, Lq, D) && encode_codes(&tk, wsb + w.kc, BH, Lk, D)
+                           : encode_bhld(&tq, wsb + w.qh, BH, Lq, D, true) && encode_bhld(&tk, wsb + w.kh, BH, Lk, D, true);
+  const bool vmap_ok = pv4 ? encode_vcodes(&tv, wsb + w.vc, BH, Lk, D) : encode_bhld(&tv, wsb + w.vh16, BH, Lk, D, true);
   if (!maps_ok || !vmap_ok) return cuda_fail(cudaErrorInvalidValue);
   FwdArgs a;
   a.Lq = Lq;
@@ -500,6 +522,7 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
   a.qsf = wsb + w.qsf;
   a.ksf = wsb + w.ksf;
   a.vsf = wsb + w.vsf;
+  operand_amax(flags, wsb, w, &a.amax_q, &a.amax_k, &a.amax_v);
   a.o = static_cast<__nv_bfloat16 *>(o);
   a.o32 = reinterpret_cast<float *>(wsb + w.o32);
   a.lse = lse;
@@ -511,7 +534,7 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
   cudaError_t e;
   {
     ProfScope ps("attn_fwd", s);
-    e = launch_fwd(D, f16, pv4 ? 2 : (pv_f16 ? 1 : 0), (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, a, BH, s);
+    e = launch_fwd(D, fp4, pv4, (flags & ATTNQAT_QUANT_P) != 0, tq, tk, tv, a, BH, s);
   }
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }
@@ -540,8 +563,7 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
   if (st != ATTNQAT_OK) return st;
   float *delta = reinterpret_cast<float *>(wsb + w.delta);
   float *stats = reinterpret_cast<float *>(wsb + w.stats);
-  const bool dof16 = do_f16(flags);
-  // stats[2] (max |fq(V)|) comes from the forward; the others start at zero
+  // stats[2], [4], [5] come from the forward; [0], [1], [3] start at zero
   cudaError_t e = cudaMemsetAsync(stats, 0, 8, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(stats + 3, 0, 4, s);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -551,21 +573,16 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
                      static_cast<int64_t>(BH) * Lq, D, stats, s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dof16) {
+  {
     ProfScope ps("scale_do", s);
-    e = launch_scale_do(static_cast<const __nv_bfloat16 *>(dO), reinterpret_cast<uint16_t *>(wsb + w.do16),
-                        static_cast<int64_t>(BH) * Lq * D, stats, s);
-    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_scale_f16(static_cast<const __nv_bfloat16 *>(dO), reinterpret_cast<uint16_t *>(wsb + w.do16),
+                         static_cast<int64_t>(BH) * Lq * D, stats + 3, s);
   }
-  const bool f16 = qk_f16(flags);
-  const void *qh = (flags & ATTNQAT_QUANT_Q) ? static_cast<const void *>(wsb + w.qh) : q;
-  const void *kh = (flags & ATTNQAT_QUANT_K) ? static_cast<const void *>(wsb + w.kh) : k;
-  const void *vh = dof16 ? static_cast<const void *>(wsb + w.vh16)
-                         : (flags & ATTNQAT_QUANT_V) ? static_cast<const void *>(wsb + w.vh) : v;
-  const void *dob = dof16 ? static_cast<const void *>(wsb + w.do16) : dO;
+  if (e != cudaSuccess) return cuda_fail(e);
+  const bool fp4 = fp4s(flags);
   CUtensorMap tq, tk, tv, tdo;
-  if (!encode_bhld(&tq, qh, BH, Lq, D, f16) || !encode_bhld(&tk, kh, BH, Lk, D, f16) ||
-      !encode_bhld(&tv, vh, BH, Lk, D, dof16) || !encode_bhld(&tdo, dob, BH, Lq, D, dof16))
+  if (!encode_bhld(&tq, wsb + w.qh, BH, Lq, D, true) || !encode_bhld(&tk, wsb + w.kh, BH, Lk, D, true) ||
+      !encode_bhld(&tv, wsb + w.vh16, BH, Lk, D, true) || !encode_bhld(&tdo, wsb + w.do16, BH, Lq, D, true))
     return cuda_fail(cudaErrorInvalidValue);
   BwdArgs a;
   a.Lq = Lq;
@@ -578,6 +595,7 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
   a.lse = lse;
   a.delta = delta;
   a.stats = stats;
+  operand_amax(flags, wsb, w, &a.amax_q, &a.amax_k, &a.amax_v);
   a.qsf = wsb + w.qsf;
   a.ksf = wsb + w.ksf;
   a.dq = static_cast<__nv_bfloat16 *>(dq);
@@ -591,17 +609,21 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
   a.causal = causal ? 1 : 0;
   // with Q and K quantized, S runs on the packed NVFP4 codes
   CUtensorMap tq4, tk4;
-  if (f16 && !(encode_codes(&tq4, wsb + w.qc, BH, Lq, D) && encode_codes(&tk4, wsb + w.kc, BH, Lk, D)))
+  if (fp4 && !(encode_codes(&tq4, wsb + w.qc, BH, Lq, D) && encode_codes(&tk4, wsb + w.kc, BH, Lk, D)))
     return cuda_fail(cudaErrorInvalidValue);
   {
     ProfScope ps("attn_bwd_dkdv", s);
-    e = launch_bwd_dkdv(D, f16, (flags & ATTNQAT_QUANT_P) != 0, dof16, tq, f16 ? tk4 : tk, tv, tdo,
-                        f16 ? tq4 : tq, a, BH, s);
+    e = launch_bwd_dkdv(D, fp4, (flags & ATTNQAT_QUANT_P) != 0, tq, fp4 ? tk4 : tk, tv, tdo, fp4 ? tq4 : tq, a, BH,
+                        s);
   }
   if (e != cudaSuccess) return cuda_fail(e);
   {
     ProfScope ps("attn_bwd_dq", s);
-    e = launch_bwd_dq(D, f16, dof16, f16 ? tq4 : tq, tk, tv, tdo, f16 ? tk4 : tk, a, BH, s);
+    // dS as an fp16 hi + lo pair unless every quantizer is on (measured: a
+    // single fp16 dS keeps the all-quantized dQ within the bar with margin,
+    // and the hot path keeps its one dQ product)
+    const bool dsplit = (flags & ATTNQAT_QUANT_ALL) != ATTNQAT_QUANT_ALL;
+    e = launch_bwd_dq(D, fp4, dsplit, fp4 ? tq4 : tq, tk, tv, tdo, fp4 ? tk4 : tk, a, BH, s);
   }
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }

@@ -113,23 +113,16 @@ __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *map, 
 
 // ----------------------------------------------------------- dK / dV ------
 
-// Power-of-two scale for the f16 dS operand: 2^e with e chosen so that the
+// Power-of-two scale for the fp16 dS operand: 2^e with e chosen so that the
 // bound |dS| <= max_i|dO_i|_1 * max|fq(V)| + max_i|Delta_i| maps to at most
 // 2^14 (fp16 max is 65504); the float range of dS below that keeps full fp16
-// precision over 29 binades.  Returns 1 for the bf16 path or a zero bound.
-template <int QKF16>
+// precision over 29 binades.  Returns 1 for a zero bound.
 __device__ __forceinline__ float ds_scale(const float *stats) {
-  if (!QKF16) return 1.0f;
   const float bound = fmaf(stats[0], stats[2], stats[1]);
   if (!(bound > 0.0f)) return 1.0f;
   int e = 14 - (static_cast<int>((__float_as_uint(bound) >> 23) & 0xFF) - 127) - 1;
   e = e < -120 ? -120 : (e > 120 ? 120 : e);
   return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
-}
-
-template <int QKF16>
-__device__ __forceinline__ uint32_t pack_ds(float a, float b) {
-  return QKF16 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
 }
 
 // S and dP of one thread's 64 columns (starting at col0) from TMEM into
@@ -152,62 +145,16 @@ __device__ __forceinline__ void load_cols64(uint32_t taddr, uint32_t (&v)[64]) {
 }
 
 // dK/dV kernel, first half of a query tile for one thread (one query row, 64
-// key columns from col0): P~ = exp(S - m) (rebuilt exactly as the forward
-// builds it: same bits, same blocks of 16 keys) and the dV operand row,
-// fq(P~)/l in bf16 (or P~/l when P is not quantized).  P~ stays in float32
-// for dS.
+// key columns from col0): P~ = exp2(S cl + nml) -- rebuilt exactly as the
+// forward builds it (same bits, same blocks of 16 keys) -- and the dV
+// operand row in fp16: fq(P~)/l * 2^14 (r times the per-block factor
+// s/l * 2^14), or P~/l * 2^14 when P is not quantized, with 11 significant
+// bits and in fp16's normal range for every value above 2^-28 (all nonzero
+// fq(P~)/l while Lk <= 2^17).  P~ stays in float32 for dS.  Rows past Lq come
+// in with nml = -inf, so their P~ is 0 without a per-element test.
 template <int QP, bool MASKED>
-__device__ __forceinline__ void dkdv_probs(const uint32_t (&sv)[64], int col0, int valid_k, bool vq, float cl,
-                                           float nml, float inv_l, float (&p)[64], uint32_t (&pw)[32]) {
-  const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float2 x = fma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), cl2, nml2);
-    const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
-    p[2 * i] = (vq && (!MASKED || col0 + 2 * i < valid_k)) ? e0 : 0.0f;
-    p[2 * i + 1] = (vq && (!MASKED || col0 + 2 * i + 1 < valid_k)) ? e1 : 0.0f;
-  }
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    if (QP) {
-      uint32_t rr[8];
-      const float f = fq16_probs(p + 16 * b, rr) * inv_l;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float2 g = unpack_f16x2(rr[i]);
-        pw[8 * b + i] = pack_bf16x2(g.x * f, g.y * f);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        pw[8 * b + i] = pack_bf16x2(p[16 * b + 2 * i] * inv_l, p[16 * b + 2 * i + 1] * inv_l);
-    }
-  }
-}
-
-// Second half: dS = (P~/l)(dP - Delta) in float32, scaled by dsc (pf =
-// dsc / l) and packed for the dK operand.
-template <int QKF16>
-__device__ __forceinline__ void dkdv_ds(const float (&p)[64], const uint32_t (&dv)[64], float pf, float delta,
-                                        uint32_t (&dsw)[32]) {
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float d0 = p[2 * i] * pf * (__uint_as_float(dv[2 * i]) - delta);
-    const float d1 = p[2 * i + 1] * pf * (__uint_as_float(dv[2 * i + 1]) - delta);
-    dsw[i] = pack_ds<QKF16>(d0, d1);
-  }
-}
-
-// The same two halves for the all-quantized path with the exact fp16 copy
-// dO * 2^e: the dV operand is fq(P~)/l * 2^14 in fp16 (r times the per-block
-// factor s/l * 2^14: 11 significant bits, and in fp16's normal range for every
-// nonzero value while Lk <= 2^17); dP' = dP 2^e arrives from TMEM and
-// dS * dsc = P~/l * (dP' 2^-e - Delta) * dsc = P~ * fma(dP', a1, b1) with
-// a1 = 2^-e dsc / l, b1 = -Delta dsc / l.  Rows past Lq come in with
-// nml = -inf, so their P~ is 0 without a per-element test.
-template <bool MASKED>
-__device__ __forceinline__ void dkdv_probs_f16(const uint32_t (&sv)[64], int col0, int valid_k, float cl,
-                                               float nml, float vf, float (&p)[64], uint32_t (&pw)[32]) {
+__device__ __forceinline__ void dkdv_probs(const uint32_t (&sv)[64], int col0, int valid_k, float cl, float nml,
+                                           float vf, float (&p)[64], uint32_t (&pw)[32]) {
   const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
@@ -216,17 +163,31 @@ __device__ __forceinline__ void dkdv_probs_f16(const uint32_t (&sv)[64], int col
     p[2 * i] = (!MASKED || col0 + 2 * i < valid_k) ? e0 : 0.0f;
     p[2 * i + 1] = (!MASKED || col0 + 2 * i + 1 < valid_k) ? e1 : 0.0f;
   }
+  if (QP) {
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    uint32_t rr[8];
-    const uint32_t s2 = f16x2_broadcast(fq16_probs(p + 16 * b, rr) * vf);
+    for (int b = 0; b < 4; ++b) {
+      uint32_t rr[8];
+      const uint32_t s2 = f16x2_broadcast(fq16_probs(p + 16 * b, rr) * vf);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) pw[8 * b + i] = hmul2_u32(rr[i], s2);
+      for (int i = 0; i < 8; ++i) pw[8 * b + i] = hmul2_u32(rr[i], s2);
+    }
+  } else {
+    const float2 vf2 = make_float2(vf, vf);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float2 x = mul2(make_float2(p[2 * i], p[2 * i + 1]), vf2);
+      pw[i] = pack_f16x2(x.x, x.y);
+    }
   }
 }
 
-__device__ __forceinline__ void dkdv_ds_f16(const float (&p)[64], const uint32_t (&dv)[64], float a1, float b1,
-                                            uint32_t (&dsw)[32]) {
+// Second half: dS = (P~/l)(dP - Delta) in float32, scaled by the fp16
+// operand's power of two dsc and packed for the dK operand.  dP arrives as
+// dP' = dP 2^e (the fp16 copies of dO and V carry powers of two), so
+// dS * dsc = P~/l * (dP' 2^-e - Delta) * dsc = P~ * fma(dP', a1, b1) with
+// a1 = 2^-e dsc / l, b1 = -Delta dsc / l.
+__device__ __forceinline__ void dkdv_ds(const float (&p)[64], const uint32_t (&dv)[64], float a1, float b1,
+                                        uint32_t (&dsw)[32]) {
   const float2 a12 = make_float2(a1, a1), b12 = make_float2(b1, b1);
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
@@ -239,12 +200,11 @@ __device__ __forceinline__ void dkdv_ds_f16(const float (&p)[64], const uint32_t
 // SP: 0 dense; 1 block-sparse (walks a.q_list); 2 causal (lower-triangle
 // lists, diagonal masked).  Separate instantiations, so the dense kernel
 // carries none of the list handling.
-template <int D, int QP, int QKF16, int DOF16, int SP>
+template <int D, int QP, int FP4S, int SP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const __grid_constant__ CUtensorMap tmQ4, const BwdArgs a) {
-  constexpr int FP4S = QKF16;  // quantized Q and K: S on the NVFP4 path
   using L = DkdvLayout<D, FP4S>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
@@ -321,10 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);  // Q K^T
-      constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
-      constexpr uint32_t idV = idesc_f16(kBN, D, !DOF16, true, true);       // P^T dO
-      constexpr uint32_t idK = idesc_f16(kBN, D, !QKF16, true, true);       // dS^T Q
+      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, false, false, false);  // Q K^T
+      constexpr uint32_t idDP = idesc_f16(kBM, kBN, false, false, false);  // dO V^T
+      constexpr uint32_t idV = idesc_f16(kBN, D, false, true, true);       // P^T dO
+      constexpr uint32_t idK = idesc_f16(kBN, D, false, true, true);       // dS^T Q
       const uint32_t kaddr = sbase + L::kK;
       const uint32_t tbuf = tmem + L::kTmemBuf;
       // operand descriptors of the tiles' base addresses
@@ -404,8 +364,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // causal: the first query tile visited is the diagonal, where query row r
     // keeps keys 0..r (a partial key tile only ever meets its diagonal)
     const int diag_k = static_cast<int>(rr.row) + 1;
-    const float cl = a.scale_log2;
-    const float dsc = ds_scale<QKF16>(a.stats);
+    // the fp16 copies of unquantized operands carry powers of two: S arrives
+    // as S 2^(eq+ek), dP as dP 2^(edo+ev) (all exact to divide out)
+    const float sq = operand_scale(a.amax_q), sk = operand_scale(a.amax_k);
+    const float cl = FP4S ? a.scale_log2 : a.scale_log2 / (sq * sk);
+    const float dsc = ds_scale(a.stats);
+    const float dos = do_scale(a.stats) * operand_scale(a.amax_v);
     const uint32_t xaddr = sbase + L::kX;
     const uint32_t tbuf = tmem + rr.lane_addr + L::kTmemBuf + col0;
     bool ok = true;
@@ -420,7 +384,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     float m_n, lse_n, delta_n;
     load_stats(0, m_n, lse_n, delta_n);
-    const float dos = DOF16 ? do_scale(a.stats) : 1.0f;
     for (int i = 0; i < n; ++i) {
       const bool vq = qtile(i) * kBM + static_cast<int>(rr.row) < a.Lq;
       const float m = m_n, lse = lse_n, delta = delta_n;
@@ -439,20 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&bars->sempty);
         const bool masked = SP == 2 ? i == 0 : valid_k < kBN;
         const int vk = SP == 2 ? diag_k : valid_k;
-        if (DOF16) {
-          const float nml = vq ? -(m * kLog2e) : -INFINITY;
-          const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
-          if (masked)
-            dkdv_probs_f16<true>(sv, col0, vk, cl, nml, vf, p, pw);
-          else
-            dkdv_probs_f16<false>(sv, col0, vk, cl, nml, vf, p, pw);
-        } else {
-          const float nml = -(m * kLog2e);
-          if (masked)
-            dkdv_probs<QP, true>(sv, col0, vk, vq, cl, nml, inv_l, p, pw);
-          else
-            dkdv_probs<QP, false>(sv, col0, vk, vq, cl, nml, inv_l, p, pw);
-        }
+        const float nml = vq ? -(m * kLog2e) : -INFINITY;
+        const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
+        if (masked)
+          dkdv_probs<QP, true>(sv, col0, vk, cl, nml, vf, p, pw);
+        else
+          dkdv_probs<QP, false>(sv, col0, vk, cl, nml, vf, p, pw);
       }
       // X = (fq(P~)/l)^T once dK_{i-1} has read the previous dS^T
       if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
@@ -469,10 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->sempty);
-        if (DOF16)
-          dkdv_ds_f16(p, dv, inv_l * dsc / dos, -delta * inv_l * dsc, dsw);
-        else
-          dkdv_ds<QKF16>(p, dv, inv_l * dsc, delta, dsw);
+        dkdv_ds(p, dv, inv_l * dsc / dos, -delta * inv_l * dsc, dsw);
       }
       // X = dS^T once dV_i has read the P^T
       if (!mbar_wait(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
@@ -486,8 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // TMEM lanes of dV/dK are keys; each thread stores D/2 columns of its key row
       const int kg = kt * kBN + static_cast<int>(rr.row);
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lk + kg) * D;
-      const float kscale = a.sm_scale / ds_scale<QKF16>(a.stats);  // exact: power-of-two divisor
-      const float vscale = DOF16 ? (1.0f / 16384.0f) / do_scale(a.stats) : 1.0f;  // exact: powers of two
+      const float kscale = a.sm_scale / (dsc * sq);  // exact: power-of-two divisors
+      const float vscale = (1.0f / 16384.0f) / do_scale(a.stats);  // exact: powers of two
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         const int col = rr.half * (D / 2) + c * 32;
@@ -533,19 +485,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // block-scaled NVFP4 MMA: the Q codes and scales stay resident and K codes
 // stream through their own small 2-stage ring, so S never waits on the
 // 16-bit K slot that the dQ MMA holds; the 16-bit Q tile is then not needed.
-template <int D, int FP4S>
+// With DSPLIT, dS is fed as two fp16 tiles, hi = fp16(dS) and lo =
+// fp16(dS - hi) (about 22 significant bits: dQ = sum_j dS_ij K_j cancels,
+// since sum_j dS_ij is 0 up to the quantization of P, and amplifies the
+// rounding of an 11-bit dS); the second tile's 32 KB come from running the V
+// ring, which only dP reads, with one stage.
+template <int D, int FP4S, int DSPLIT>
 struct DqLayout {
   static constexpr int kTile = Tile<D>::kBytes;
   static constexpr int kXBytes = kBM * kBN * 2;
   static constexpr int kCode = 128 * (D / 2);   // one packed NVFP4 tile
   static constexpr int kSF = (D / 64) * 512;    // its scale-factor blocks
+  static constexpr int kNV = DSPLIT ? 1 : 2;    // V ring stages
   static constexpr int kQ = 0;                  // 16-bit Q tile, or Q codes (FP4S)
   static constexpr int kQSF = kQ + (FP4S ? kCode : kTile);
   static constexpr int kDO = (kQSF + (FP4S ? kSF : 0) + 1023) / 1024 * 1024;
   static constexpr int kK = kDO + kTile;        // 2 stages of 16-bit K
-  static constexpr int kV = kK + 2 * kTile;     // 2 stages
-  static constexpr int kX = kV + 2 * kTile;     // dS
-  static constexpr int kK4 = kX + kXBytes;      // FP4S: 2 stages of K codes
+  static constexpr int kV = kK + 2 * kTile;     // kNV stages
+  static constexpr int kX = kV + kNV * kTile;   // dS (DSPLIT: its hi part, the lo part follows)
+  static constexpr int kK4 = kX + (DSPLIT ? 2 : 1) * kXBytes;  // FP4S: 2 stages of K codes
   static constexpr int kKSF = kK4 + (FP4S ? 2 * kCode : 0);
   static constexpr int kBar = kKSF + (FP4S ? 2 * kSF : 0);
   static constexpr int kBarBytes = 256;  // BwdBars (checked at the launch)
@@ -560,31 +518,16 @@ struct DqLayout {
 };
 
 // One key tile for one thread of the dQ kernel (one query row, 64 key
-// columns starting at col0), from S and dP in registers: P = exp(S - LSE) in
-// float32 and dS = P (dP - Delta), scaled by dsc and packed for the dQ
-// operand.
-template <int QKF16, bool MASKED>
-__device__ __forceinline__ void dq_tile(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
-                                        int valid_k, bool vq, float cl, float nlse, float delta, float dsc,
-                                        uint32_t (&dsw)[32]) {
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), cl, nlse));
-    float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), cl, nlse));
-    if (!vq || (MASKED && col0 + 2 * i >= valid_k)) p0 = 0.0f;
-    if (!vq || (MASKED && col0 + 2 * i + 1 >= valid_k)) p1 = 0.0f;
-    dsw[i] = pack_ds<QKF16>(p0 * dsc * (__uint_as_float(dv[2 * i]) - delta),
-                            p1 * dsc * (__uint_as_float(dv[2 * i + 1]) - delta));
-  }
-}
-
-// dQ-kernel tile for the exact fp16 copy dO * 2^e: dP' = dP 2^e, so
+// columns starting at col0), from S and dP in registers: P = exp2(S cl +
+// nlse) in float32 and dS = P (dP - Delta), scaled by the fp16 operand's
+// power of two dsc and packed as fp16 for dQ = dS fq(K).  dP arrives as
+// dP' = dP 2^e (the fp16 copies of dO and V carry powers of two), so
 // dS * dsc = P (dP' 2^-e - Delta) dsc = P * fma(dP', a1, b1) with
 // a1 = 2^-e dsc, b1 = -Delta dsc.  Rows past Lq come in with nlse = -inf.
-template <bool MASKED>
-__device__ __forceinline__ void dq_tile_f16(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0,
-                                            int valid_k, float cl, float nlse, float a1, float b1,
-                                            uint32_t (&dsw)[32]) {
+template <bool MASKED, int DSPLIT>
+__device__ __forceinline__ void dq_tile(const uint32_t (&sv)[64], const uint32_t (&dv)[64], int col0, int valid_k,
+                                        float cl, float nlse, float a1, float b1, uint32_t (&dsw)[32],
+                                        uint32_t (&dsl)[32]) {
   const float2 cl2 = make_float2(cl, cl), nl2 = make_float2(nlse, nlse);
   const float2 a12 = make_float2(a1, a1), b12 = make_float2(b1, b1);
 #pragma unroll
@@ -597,18 +540,22 @@ __device__ __forceinline__ void dq_tile_f16(const uint32_t (&sv)[64], const uint
     const float2 g = fma2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), a12, b12);
     const float2 d = mul2(make_float2(p0, p1), g);
     dsw[i] = pack_f16x2(d.x, d.y);
+    if (DSPLIT) {
+      const float2 h = unpack_f16x2(dsw[i]);
+      dsl[i] = pack_f16x2(d.x - h.x, d.y - h.y);  // d - h is exact in float
+    }
   }
 }
 
 // SP: 0 dense, 1 block-sparse (walks a.kv_list), 2 causal, as for the dK/dV
 // kernel.
-template <int D, int QKF16, int DOF16, int SP>
+template <int D, int FP4S, int DSPLIT, int SP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                        const __grid_constant__ CUtensorMap tmK4, const BwdArgs a) {
-  constexpr int FP4S = QKF16;  // quantized Q and K: S on the NVFP4 path
-  using L = DqLayout<D, FP4S>;
+  using L = DqLayout<D, FP4S, DSPLIT>;
+  constexpr int kNV = L::kNV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
@@ -664,9 +611,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     &bars->cfull[st]);
           n4 = j + 1;
         }
-        if (j >= 2 && !mbar_wait(&bars->bempty[st], ph, abort)) break;
-        mbar_arrive_expect_tx(&bars->bfull[st], L::kTile);
-        load_tile<D>(smem + L::kV + st * L::kTile, &tmV, &bars->bfull[st], kj * kBN, bh);
+        const int vs = j % kNV;
+        if (j >= kNV && !mbar_wait(&bars->bempty[vs], ((j / kNV) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->bfull[vs], L::kTile);
+        load_tile<D>(smem + L::kV + vs * L::kTile, &tmV, &bars->bfull[vs], kj * kBN, bh);
         nv = j + 1;
         if (j >= 2 && !mbar_wait(&bars->aempty[st], ph, abort)) break;
         mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
@@ -676,15 +624,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort) {
         mbar_wait_drain(&bars->kvfull, 0);
         for (int j = (n4 > 2 ? n4 - 2 : 0); j < n4; ++j) mbar_wait_drain(&bars->cfull[j & 1], (j >> 1) & 1);
-        for (int j = (nv > 2 ? nv - 2 : 0); j < nv; ++j) mbar_wait_drain(&bars->bfull[j & 1], (j >> 1) & 1);
+        for (int j = (nv > kNV ? nv - kNV : 0); j < nv; ++j) mbar_wait_drain(&bars->bfull[j % kNV], (j / kNV) & 1);
         for (int j = (nkh > 2 ? nkh - 2 : 0); j < nkh; ++j) mbar_wait_drain(&bars->afull[j & 1], (j >> 1) & 1);
       }
     }
   } else if (warp == 1 || warp == kMmaB2) {
     if (lane == 0) {
-      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);  // Q K^T
-      constexpr uint32_t idDP = idesc_f16(kBM, kBN, !DOF16, false, false);  // dO V^T
-      constexpr uint32_t idQ = idesc_f16(kBM, D, !QKF16, false, true);     // dS (K-major) * K (MN-major)
+      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, false, false, false);  // Q K^T
+      constexpr uint32_t idDP = idesc_f16(kBM, kBN, false, false, false);  // dO V^T
+      constexpr uint32_t idQ = idesc_f16(kBM, D, false, false, true);     // dS (K-major) * K (MN-major)
       const uint32_t qaddr = sbase + L::kQ;
       // operand descriptors of the tiles' base addresses
       const uint64_t dQ = FP4S ? sdesc_make(qaddr, 16, L::kCodeSBO, L::kCodeLayout) : desc_k(qaddr);
@@ -703,10 +651,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto issue_sdp = [&](int j) -> bool {
           const int st = j & 1;
           const uint32_t ph = (j >> 1) & 1;
-          if (!mbar_wait(&bars->bfull[st], ph, abort)) return false;
+          const int vs = j % kNV;
+          if (!mbar_wait(&bars->bfull[vs], (j / kNV) & 1, abort)) return false;
           tc_fence_after();
-          mma_kmajor<D / 16>(tmem + L::kTmemDP, dDO, sdesc_add(dVk, st * L::kTile), idDP, false);
-          umma_commit(&bars->bempty[st]);
+          mma_kmajor<D / 16>(tmem + L::kTmemDP, dDO, sdesc_add(dVk, vs * L::kTile), idDP, false);
+          umma_commit(&bars->bempty[vs]);
           if (FP4S) {
             if (!mbar_wait(&bars->cfull[st], ph, abort)) return false;
             tc_fence_after();
@@ -741,6 +690,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&bars->xfull, j & 1, abort) || !mbar_wait(&bars->afull[st], (j >> 1) & 1, abort)) break;
           tc_fence_after();
           mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemDQ, dX, sdesc_add(dKmn, st * L::kTile), idQ, j > 0);
+          if (DSPLIT)  // the lo tile of dS
+            mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemDQ, sdesc_add(dX, L::kXBytes), sdesc_add(dKmn, st * L::kTile), idQ,
+                                   true);
           umma_commit(&bars->xempty);
           umma_commit(&bars->aempty[st]);
         }
@@ -755,10 +707,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t si = static_cast<size_t>(bh) * a.Lq + (vq ? q : 0);
     const float lse = vq ? a.lse[si] : 0.0f;
     const float delta = vq ? a.delta[si] : 0.0f;
-    const float nlse = DOF16 ? (vq ? -(lse * kLog2e) : -INFINITY) : -(lse * kLog2e);
-    const float cl = a.scale_log2;
-    const float dsc = ds_scale<QKF16>(a.stats);
-    const float a1 = DOF16 ? dsc / do_scale(a.stats) : 0.0f;
+    const float nlse = vq ? -(lse * kLog2e) : -INFINITY;
+    // the fp16 copies of unquantized operands carry powers of two: S arrives
+    // as S 2^(eq+ek), dP as dP 2^(edo+ev) (all exact to divide out)
+    const float sk = operand_scale(a.amax_k);
+    const float cl = FP4S ? a.scale_log2 : a.scale_log2 / (operand_scale(a.amax_q) * sk);
+    const float dsc = ds_scale(a.stats);
+    const float a1 = dsc / (do_scale(a.stats) * operand_scale(a.amax_v));
     const float b1 = -delta * dsc;
     const int last_valid = a.Lk - (nk - 1) * kBN;
     // the lists ascend, so only the last tile visited can be the partial one;
@@ -770,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + rr.lane_addr + L::kTmemS, tDP = tmem + rr.lane_addr + L::kTmemDP;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      uint32_t dsw[32];
+      uint32_t dsw[32], dsl[32];
       uint32_t sv[64], dv[64];
       const bool tail = tail_last && j == n - 1;
       if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
@@ -779,19 +734,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
-      if (DOF16) {
-        if (tail)
-          dq_tile_f16<true>(sv, dv, col0, last_cols, cl, nlse, a1, b1, dsw);
-        else
-          dq_tile_f16<false>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw);
-      } else {
-        if (tail)
-          dq_tile<QKF16, true>(sv, dv, col0, last_cols, vq, cl, nlse, delta, dsc, dsw);
-        else
-          dq_tile<QKF16, false>(sv, dv, col0, kBN, vq, cl, nlse, delta, dsc, dsw);
-      }
+      if (tail)
+        dq_tile<true, DSPLIT>(sv, dv, col0, last_cols, cl, nlse, a1, b1, dsw, dsl);
+      else
+        dq_tile<false, DSPLIT>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw, dsl);
       if (j >= 1 && !mbar_wait(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
+      if (DSPLIT) store_row_half(xaddr + L::kXBytes, rr.row, rr.half, dsl);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
@@ -799,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && mbar_wait(&bars->done, 0, abort)) {
       tc_fence_after();
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
-      const float qscale = a.sm_scale / dsc;  // exact: power-of-two divisor
+      const float qscale = a.sm_scale / (dsc * sk);  // exact: power-of-two divisors
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         const int col = rr.half * (D / 2) + c * 32;
@@ -835,87 +784,86 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------- launchers --
 
-template <int D, int QP, int QKF16, int DOF16, int SP>
+template <int D, int QP, int FP4S, int SP>
 static cudaError_t launch_dkdv_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
                                   cudaStream_t stream) {
-  using L = DkdvLayout<D, QKF16>;
+  using L = DkdvLayout<D, FP4S>;
   static_assert(L::kDynSmem <= 232448, "dK/dV shared memory over the 227 KB limit");
   static_assert(sizeof(BwdBars) <= L::kBarBytes, "dK/dV barrier block larger than its reservation");
   static_assert(L::kTmemSFB + L::kSFCols <= L::kTmemCols, "dK/dV TMEM over 512 columns");
-  auto kern = attn_bwd_dkdv_kernel<D, QP, QKF16, DOF16, SP>;
+  auto kern = attn_bwd_dkdv_kernel<D, QP, FP4S, SP>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.nk_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, tq4, a);
   return cudaGetLastError();
 }
 
-template <int D, int QP, int QKF16, int DOF16>
+template <int D, int QP, int FP4S>
 static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                  const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
                                  cudaStream_t stream) {
-  if (!a.q_list) return launch_dkdv_sp<D, QP, QKF16, DOF16, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
-  return a.causal ? launch_dkdv_sp<D, QP, QKF16, DOF16, 2>(tq, tk, tv, tdo, tq4, a, BH, stream)
-                  : launch_dkdv_sp<D, QP, QKF16, DOF16, 1>(tq, tk, tv, tdo, tq4, a, BH, stream);
+  if (!a.q_list) return launch_dkdv_sp<D, QP, FP4S, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
+  return a.causal ? launch_dkdv_sp<D, QP, FP4S, 2>(tq, tk, tv, tdo, tq4, a, BH, stream)
+                  : launch_dkdv_sp<D, QP, FP4S, 1>(tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
 template <int D>
-static cudaError_t dkdv_dispatch(bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
-                                 const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
-                                 const CUtensorMap &tq4, const BwdArgs &a, int BH, cudaStream_t stream) {
-  if (do_f16) return launch_dkdv_t<D, 1, 1, 1>(tq, tk, tv, tdo, tq4, a, BH, stream);
-  if (qk_f16)
-    return quant_p ? launch_dkdv_t<D, 1, 1, 0>(tq, tk, tv, tdo, tq4, a, BH, stream)
-                   : launch_dkdv_t<D, 0, 1, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
-  return quant_p ? launch_dkdv_t<D, 1, 0, 0>(tq, tk, tv, tdo, tq4, a, BH, stream)
-                 : launch_dkdv_t<D, 0, 0, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
+static cudaError_t dkdv_dispatch(bool fp4s, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+                                 const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tq4,
+                                 const BwdArgs &a, int BH, cudaStream_t stream) {
+  if (fp4s)
+    return quant_p ? launch_dkdv_t<D, 1, 1>(tq, tk, tv, tdo, tq4, a, BH, stream)
+                   : launch_dkdv_t<D, 0, 1>(tq, tk, tv, tdo, tq4, a, BH, stream);
+  return quant_p ? launch_dkdv_t<D, 1, 0>(tq, tk, tv, tdo, tq4, a, BH, stream)
+                 : launch_dkdv_t<D, 0, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
-cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
-                            const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
-                            const CUtensorMap &tq4, const BwdArgs &a, int BH, cudaStream_t stream) {
-  return D == 128 ? dkdv_dispatch<128>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, tq4, a, BH, stream)
-                  : dkdv_dispatch<64>(qk_f16, quant_p, do_f16, tq, tk, tv, tdo, tq4, a, BH, stream);
+cudaError_t launch_bwd_dkdv(int D, bool fp4s, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+                            const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tq4,
+                            const BwdArgs &a, int BH, cudaStream_t stream) {
+  return D == 128 ? dkdv_dispatch<128>(fp4s, quant_p, tq, tk, tv, tdo, tq4, a, BH, stream)
+                  : dkdv_dispatch<64>(fp4s, quant_p, tq, tk, tv, tdo, tq4, a, BH, stream);
 }
 
-template <int D, int QKF16, int DOF16, int SP>
+template <int D, int FP4S, int DSPLIT, int SP>
 static cudaError_t launch_dq_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
                                 cudaStream_t stream) {
-  using L = DqLayout<D, QKF16>;
+  using L = DqLayout<D, FP4S, DSPLIT>;
   static_assert(L::kDynSmem <= 232448, "dQ shared memory over the 227 KB limit");
   static_assert(sizeof(BwdBars) <= L::kBarBytes, "dQ barrier block larger than its reservation");
   static_assert(L::kTmemSFB + 2 * L::kSFCols <= L::kTmemCols, "dQ TMEM over 512 columns");
-  auto kern = attn_bwd_dq_kernel<D, QKF16, DOF16, SP>;
+  auto kern = attn_bwd_dq_kernel<D, FP4S, DSPLIT, SP>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.nq_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, tk4, a);
   return cudaGetLastError();
 }
 
-template <int D, int QKF16, int DOF16>
+template <int D, int FP4S, int DSPLIT>
 static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
                                cudaStream_t stream) {
-  if (!a.kv_list) return launch_dq_sp<D, QKF16, DOF16, 0>(tq, tk, tv, tdo, tk4, a, BH, stream);
-  return a.causal ? launch_dq_sp<D, QKF16, DOF16, 2>(tq, tk, tv, tdo, tk4, a, BH, stream)
-                  : launch_dq_sp<D, QKF16, DOF16, 1>(tq, tk, tv, tdo, tk4, a, BH, stream);
+  if (!a.kv_list) return launch_dq_sp<D, FP4S, DSPLIT, 0>(tq, tk, tv, tdo, tk4, a, BH, stream);
+  return a.causal ? launch_dq_sp<D, FP4S, DSPLIT, 2>(tq, tk, tv, tdo, tk4, a, BH, stream)
+                  : launch_dq_sp<D, FP4S, DSPLIT, 1>(tq, tk, tv, tdo, tk4, a, BH, stream);
 }
 
 template <int D>
-static cudaError_t dq_dispatch(bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
+static cudaError_t dq_dispatch(bool fp4s, bool dsplit, const CUtensorMap &tq, const CUtensorMap &tk,
                                const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4,
                                const BwdArgs &a, int BH, cudaStream_t stream) {
-  if (do_f16) return launch_dq_t<D, 1, 1>(tq, tk, tv, tdo, tk4, a, BH, stream);
-  return qk_f16 ? launch_dq_t<D, 1, 0>(tq, tk, tv, tdo, tk4, a, BH, stream)
-                : launch_dq_t<D, 0, 0>(tq, tk, tv, tdo, tk4, a, BH, stream);
+  if (!fp4s) return launch_dq_t<D, 0, 1>(tq, tk, tv, tdo, tk4, a, BH, stream);
+  return dsplit ? launch_dq_t<D, 1, 1>(tq, tk, tv, tdo, tk4, a, BH, stream)
+                : launch_dq_t<D, 1, 0>(tq, tk, tv, tdo, tk4, a, BH, stream);
 }
 
-cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
-                          const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4,
-                          const BwdArgs &a, int BH, cudaStream_t stream) {
-  return D == 128 ? dq_dispatch<128>(qk_f16, do_f16, tq, tk, tv, tdo, tk4, a, BH, stream)
-                  : dq_dispatch<64>(qk_f16, do_f16, tq, tk, tv, tdo, tk4, a, BH, stream);
+cudaError_t launch_bwd_dq(int D, bool fp4s, bool dsplit, const CUtensorMap &tq, const CUtensorMap &tk,
+                          const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a,
+                          int BH, cudaStream_t stream) {
+  return D == 128 ? dq_dispatch<128>(fp4s, dsplit, tq, tk, tv, tdo, tk4, a, BH, stream)
+                  : dq_dispatch<64>(fp4s, dsplit, tq, tk, tv, tdo, tk4, a, BH, stream);
 }
 
 }  // namespace attnqat

@@ -79,15 +79,25 @@ __device__ __forceinline__ uint32_t f16x2_broadcast(float s) {
   return h | (h << 16);
 }
 
-// Power of two 2^e that maps max |dO| (stats[3]) into [2^13, 2^14): the
-// scale of the backward's exact fp16 copy of dO; 1 when dO is 0.
-__device__ __forceinline__ float do_scale(const float *stats) {
-  const float mx = stats[3];
+// Power of two 2^e that maps a tensor's max magnitude `mx` into [2^13, 2^14):
+// the scale of an fp16 copy of a bf16 tensor (dO, and Q, K or V when that
+// operand is not quantized); 1 when mx is 0.  A bf16 value has 8 significant
+// bits, so the copy is exact for every element within 2^27 of the largest,
+// and an element below that moves by at most 2^-25 of the largest.
+__device__ __forceinline__ float pow2_scale(float mx) {
   if (!(mx > 0.0f)) return 1.0f;
   int e = 13 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xFF) - 127);
   e = e < -120 ? -120 : (e > 120 ? 120 : e);
   return __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
 }
+
+// Scale of the fp16 copy of dO (max |dO| is stats[3]).
+__device__ __forceinline__ float do_scale(const float *stats) { return pow2_scale(stats[3]); }
+
+// Scale of an operand's fp16 copy: pow2_scale of the max magnitude `amax`
+// points at, or 1 for a quantized operand (null), whose fq values are exact
+// in fp16 unscaled.
+__device__ __forceinline__ float operand_scale(const float *amax) { return amax ? pow2_scale(*amax) : 1.0f; }
 
 // The MMA helpers below take the descriptors of the operand tiles' base
 // addresses and advance them by adding (byte offset >> 4) to the 14-bit

@@ -67,19 +67,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Gives up
 // (returns false) when *abort is set by another role of the CTA, or after
-// kWaitLimitNs, in which case it sets *abort and the device status flag.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// limit_ns, in which case it sets *abort and the device status flag.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       atomicOr(&g_device_status, 1u);
       return false;
     }
   }
+}
+
+// mbar_wait_for with the library's limit, kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // Like mbar_wait but only bounded by time (used when draining in-flight

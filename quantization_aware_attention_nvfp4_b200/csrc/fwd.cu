@@ -5,10 +5,10 @@
 //               sweep and K, fq(V) tiles for the output sweep.  With Q and K
 //               quantized these are the packed NVFP4 codes plus their scale
 //               tiles (8-stage K ring) and S is a block-scaled NVFP4 MMA;
-//               otherwise bf16 tiles.  fq(V): with every quantizer on (D =
-//               128, Lk % 32 == 0) its packed codes and scale tiles (4-stage
-//               ring) for a block-scaled NVFP4 P V, else fp16/bf16 tiles
-//               (2-stage ring, 128-byte swizzle);
+//               otherwise fp16 tiles.  fq(V): with every quantizer on (Lk %
+//               32 == 0) its packed codes and scale tiles (4-stage ring) for
+//               a block-scaled NVFP4 P V (N = D), else fp16 tiles (2-stage
+//               ring, 128-byte swizzle);
 //   warps 1, 10 tcgen05.mma issuers (one thread each; warp 1 owns TMEM): A
 //               issues even row-max tiles and the output sweep's S, B the odd
 //               row-max tiles and P V (one thread alone cannot issue fast
@@ -16,9 +16,14 @@
 //   warps 2..9  row warps, two per TMEM lane quarter: each query row (TMEM
 //               lane) has two threads owning 64 columns each -- row max, exp,
 //               row sum, in-register NVFP4 fq of P~ in 16-key blocks, the P
-//               tile (packed codes and scale bytes, or 16-bit values) to
+//               tile (packed codes and scale bytes, or fp16 values) to
 //               shared memory, and the O epilogue; the pair merges its
 //               partial max and sum through shared memory.
+// Every 16-bit MMA operand is fp16: fq(Q), fq(K), fq(V) and fq(P~) are exact
+// in fp16 as they are; an operand whose quantizer is off is copied as
+// X * 2^e (a power of two that maps its max magnitude into [2^13, 2^14),
+// exact for every element within 2^27 of the largest), and the powers of two
+// are divided out of S and O.
 //   warp 11     idle (pads the CTA to whole groups of four warps).
 // TMEM columns: S buffers [0,256) (plus [256,384) during the row-max sweep,
 // before O exists), O accumulator [256, 256+D), scale factors from 384.
@@ -44,7 +49,7 @@ namespace attnqat {
 // Shared-memory and TMEM layout of the forward.  With FP4S the Q and K tiles
 // are packed NVFP4 codes (D/2 bytes per row, TMA swizzle of D/2 bytes) and
 // their 16-element scales (512-byte scale-factor blocks per 64 columns); S is
-// then a block-scaled kind::mxf4nvf4 MMA.  Otherwise Q and K are 16-bit tiles.
+// then a block-scaled kind::mxf4nvf4 MMA.  Otherwise Q and K are fp16 tiles.
 // With PV4 the P V product is block-scaled NVFP4 too: fq(P~) blocks run along
 // keys and fq(V) blocks along tokens, both the K axis of P V, so the P tile
 // holds packed codes (64 bytes per query row, 64-byte swizzle) plus scale
@@ -130,18 +135,21 @@ __device__ __forceinline__ float row_max_cols(uint32_t taddr, int col0, int vali
 }
 
 // Sweep-2 work for this thread's NC columns of one S tile: P~ = exp2(S*cl +
-// nml), partial row sum, fq(P~) (or P~ itself) packed into 16-bit pairs and
-// stored as columns col0..col0+NC-1 of row `row` of the P tile at `pbase`
-// (128-byte swizzled chunks of 64 columns).
-// PVM selects the P tile's form: 0 bf16, 1 fp16 (16-bit, 128-byte swizzled
-// chunks), 2 packed NVFP4 codes (64-byte rows, 64-byte swizzle) with the
-// E4M3 scale bytes at `psf` in the layout tcgen05.cp moves into TMEM.
-template <int PVM, int QP, bool MASKED, int NC>
+// nml), partial row sum, and fq(P~) (or P~ itself) written as columns
+// col0..col0+NC-1 of row `row` of the P tile at `pbase`.
+// PV4 selects the P tile's form: packed NVFP4 codes (64-byte rows, 64-byte
+// swizzle) with the E4M3 scale bytes at `psf` in the layout tcgen05.cp moves
+// into TMEM; otherwise fp16 values in 128-byte swizzled chunks of 64 columns.
+// With P unquantized (QP = 0) P~ itself is the operand and fp16 would round
+// it to 11 bits; the product is then taken as hi V + lo V with hi = fp16(P~)
+// and lo = fp16(P~ - hi), stored as two tiles (`lo_off` bytes apart), which
+// carries P~ to about 22 bits.  (Where dP - Delta cancels, Delta = dO . O
+// would otherwise inherit the fp16 rounding of P~ about thirtyfold.)
+template <int PV4, int QP, bool MASKED, int NC>
 __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, float cl, float nml,
-                                           uint32_t pbase, uint32_t psf, uint32_t row) {
-  static_assert(PVM != 2 || (QP && NC == 64), "NVFP4 P V needs quantized P and 64 columns per thread");
-  constexpr int PV_F16 = PVM == 1;
-  uint32_t sfw = 0;  // PVM 2: this thread's four scale bytes
+                                           uint32_t pbase, uint32_t psf, uint32_t row, uint32_t lo_off) {
+  static_assert(!PV4 || (QP && NC == 64), "NVFP4 P V needs quantized P and 64 columns per thread");
+  uint32_t sfw = 0;  // PV4: this thread's four scale bytes
   float2 lsum = make_float2(0.0f, 0.0f);
   const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
 #pragma unroll
@@ -158,7 +166,7 @@ __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, 
       p[2 * i + 1] = (!MASKED || col0 + c * 32 + 2 * i + 1 < valid) ? e1 : 0.0f;
       lsum = add2(lsum, make_float2(p[2 * i], p[2 * i + 1]));
     }
-    if (PVM == 2) {
+    if (PV4) {
       // two 16-key blocks -> 16 bytes of codes (the 16-byte unit cc/32 of the
       // row's 64 bytes, swizzled as TMA's 64-byte mode) and two scale bytes
       uint32_t cw[4];
@@ -169,28 +177,22 @@ __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, 
       st_shared_v4(pbase + (row >> 3) * 512 + (row & 7) * 64 + ((unit ^ ((row >> 1) & 3)) << 4), cw[0], cw[1],
                    cw[2], cw[3]);
     } else {
-      uint32_t w[16];
+      uint32_t w[16], wl[16];
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         if (QP) {
           uint32_t rr[8];
-          const float s = fq16_probs(p + 16 * b, rr);
-          if (PV_F16) {
-            const uint32_t s2 = f16x2_broadcast(s);
+          const uint32_t s2 = f16x2_broadcast(fq16_probs(p + 16 * b, rr));
 #pragma unroll
-            for (int i = 0; i < 8; ++i) w[8 * b + i] = hmul2_u32(rr[i], s2);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float2 g = unpack_f16x2(rr[i]);
-              w[8 * b + i] = pack_bf16x2(g.x * s, g.y * s);
-            }
-          }
+          for (int i = 0; i < 8; ++i) w[8 * b + i] = hmul2_u32(rr[i], s2);
         } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            w[8 * b + i] = PV_F16 ? pack_f16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1])
-                                  : pack_bf16x2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1]);
+          for (int i = 0; i < 8; ++i) {
+            const float2 x = make_float2(p[16 * b + 2 * i], p[16 * b + 2 * i + 1]);
+            w[8 * b + i] = pack_f16x2(x.x, x.y);
+            const float2 h = unpack_f16x2(w[8 * b + i]);
+            wl[8 * b + i] = pack_f16x2(x.x - h.x, x.y - h.y);  // x - h is exact in float
+          }
         }
       }
       // 32 keys = four 16-byte units of the 64-key swizzled chunk holding them
@@ -200,10 +202,11 @@ __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, 
         const uint32_t addr = pbase + static_cast<uint32_t>(cc >> 6) * kChunkBytes +
                               sw128_offset(row, ((cc & 63) >> 3) + u);
         st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        if (!QP) st_shared_v4(addr + lo_off, wl[4 * u], wl[4 * u + 1], wl[4 * u + 2], wl[4 * u + 3]);
       }
     }
   }
-  if (PVM == 2) {
+  if (PV4) {
     // this thread's 64 keys are one 64-key scale block (k-chunk col0 / 64):
     // row r's four bytes at (r % 32) * 16 + (r / 32) * 4
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(psf + static_cast<uint32_t>(col0 >> 6) * 512 + (row & 31) * 16 +
@@ -230,13 +233,15 @@ constexpr int fwd_threads() { return (2 + 4 * G + 1 + 3) / 4 * 128; }
 // SP: 0 dense; 1 block-sparse (walks a.kv_list); 2 causal (walks the
 // lower-triangle lists and masks the diagonal).  Separate instantiations, so
 // the dense kernel carries none of the list handling.
-template <int D, int FP4S, int PVM, int QP, int G, int SP>
+template <int D, int FP4S, int PV4, int QP, int G, int SP>
 __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
-  constexpr int PV4 = PVM == 2;
-  constexpr int PV_F16 = PVM == 1;
   using L = FwdLayout<D, FP4S, PV4>;
+  // unquantized P: one P slot holding the hi and lo tiles (the two P buffers'
+  // space), handed over once per key tile
+  constexpr bool PSPLIT = !QP;
+  static_assert(!(PSPLIT && PV4), "the NVFP4 P V takes quantized P");
   static_assert(G <= kFwdG, "column groups beyond the partial-sum block");
   static_assert(L::kNSK <= 8 && L::kNSV <= 4, "ring deeper than its barrier arrays");
   constexpr int kNSK = L::kNSK, kNSV = L::kNSV;
@@ -355,8 +360,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     // S of the output sweep, B the odd row-max tiles and every P V.
     if (lane == 0) {
       const bool issuer_a = warp == 1;
-      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, true, false, false);
-      constexpr uint32_t idPV = idesc_f16(kBM, D, !PV_F16, false, true);
+      constexpr uint32_t idS = FP4S ? idesc_mxf4(kBM, kBN) : idesc_f16(kBM, kBN, false, false, false);
+      constexpr uint32_t idPV = idesc_f16(kBM, D, false, false, true);
       const uint32_t qaddr = sbase + L::kQ;
       bool ok = mbar_wait(&bars->qfull, 0, abort);
       if (FP4S) {
@@ -425,9 +430,10 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         // (the first P V runs after every row-max tile was read, so it may
         // overwrite the third S buffer's columns)
         for (int j = 0; ok && j < n; ++j) {
-          const int pb = j & 1;
+          const int pb = PSPLIT ? 0 : (j & 1);
           const int vs = j % kNSV;
-          if (!mbar_wait(&bars->pfull[pb], (j >> 1) & 1, abort) || !mbar_wait(&bars->vfull[vs], (j / kNSV) & 1, abort)) {
+          const uint32_t pph = PSPLIT ? (j & 1) : ((j >> 1) & 1);
+          if (!mbar_wait(&bars->pfull[pb], pph, abort) || !mbar_wait(&bars->vfull[vs], (j / kNSV) & 1, abort)) {
             ok = false;
             break;
           }
@@ -450,6 +456,10 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
           } else {
             mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemO, sdesc_add(dP, pb * L::kPBytes), sdesc_add(dV, vs * L::kVT),
                                    idPV, j > 0);
+            // the lo tile (second P buffer): O += lo V
+            if (PSPLIT)
+              mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemO, sdesc_add(dP, L::kPBytes), sdesc_add(dV, vs * L::kVT), idPV,
+                                     true);
           }
           umma_commit(&bars->vempty[vs]);
           umma_commit(&bars->pempty[pb]);
@@ -491,24 +501,32 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
 #pragma unroll
     for (int g = 0; g < G; ++g) mrow = fmaxf(mrow, bars->part[g][rr.row]);
     group_sync<G>(rr.wq);
-    const float m_scaled = mrow * a.sm_scale;
+    // S arrives as S * 2^(eq + ek) when Q or K is a scaled fp16 copy (both
+    // factors are 1 for quantized operands): dividing the powers of two out
+    // of c is exact, so m and P~ are the same bits either way
+    const float sqk = FP4S ? 1.0f : operand_scale(a.amax_q) * operand_scale(a.amax_k);
+    const float m_scaled = mrow * (a.sm_scale / sqk);
     const float nml = -(m_scaled * kLog2e);
-    const float cl = a.scale_log2;
+    const float cl = a.scale_log2 / sqk;
     float lsum = 0.0f;
     for (int j = 0; ok && j < n; ++j) {
       const int sb = j & 1;
-      const int pb = j & 1;
+      const int pb = PSPLIT ? 0 : (j & 1);
       const bool tail = tail_last && j == n - 1;
       if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, abort)) { ok = false; break; }
-      if (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
+      if (PSPLIT ? (j >= 1 && !mbar_wait(&bars->pempty[0], (j - 1) & 1, abort))
+                 : (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
       const uint32_t psf = sbase + L::kPSFo + pb * L::kPSF;
       if (tail)
-        lsum += prob_cols<PVM, QP, true, NC>(taddr, col0, last_cols, cl, nml, pbase, psf, rr.row);
+        lsum += prob_cols<PV4, QP, true, NC>(taddr, col0, last_cols, cl, nml, pbase, psf, rr.row, L::kPBytes);
       else
-        lsum += prob_cols<PVM, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, psf, rr.row);
+        lsum += prob_cols<PV4, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, psf, rr.row, L::kPBytes);
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
@@ -527,8 +545,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       tc_fence_after();
       const int q = qt * kBM + static_cast<int>(rr.row);
       // no key tile selected: O = 0 (the accumulator was never written),
-      // m = LSE = -inf
-      const float inv_l = 1.0f / lsum;
+      // m = LSE = -inf.  A scaled fp16 copy of V leaves O * 2^ev in TMEM.
+      const float inv_l = (1.0f / lsum) / (PV4 ? 1.0f : operand_scale(a.amax_v));
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
       constexpr int DC = D / G;            // output columns per thread
       constexpr int W = DC < 32 ? DC : 32;  // columns per TMEM load
@@ -575,14 +593,14 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
   }
 }
 
-template <int D, int FP4S, int PVM, int QP, int SP>
+template <int D, int FP4S, int PV4, int QP, int SP>
 static cudaError_t launch_fwd_sp(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                  const FwdArgs &a, int BH, cudaStream_t stream) {
-  using L = FwdLayout<D, FP4S, PVM == 2>;
+  using L = FwdLayout<D, FP4S, PV4>;
   static_assert(L::kDynSmem <= 232448, "forward shared memory over the 227 KB limit");
   static_assert(sizeof(FwdBars) <= L::kBarBytes, "forward barrier block larger than its reservation");
   static_assert(!FP4S || L::kTmemEnd <= L::kTmemCols, "forward TMEM over 512 columns");
-  auto kern = attn_fwd_kernel<D, FP4S, PVM, QP, kFwdG, SP>;
+  auto kern = attn_fwd_kernel<D, FP4S, PV4, QP, kFwdG, SP>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nq_tiles, BH);
@@ -590,34 +608,31 @@ static cudaError_t launch_fwd_sp(const CUtensorMap &tq, const CUtensorMap &tk, c
   return cudaGetLastError();
 }
 
-template <int D, int FP4S, int PVM, int QP>
+template <int D, int FP4S, int PV4, int QP>
 static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const FwdArgs &a, int BH, cudaStream_t stream) {
-  if (!a.kv_list) return launch_fwd_sp<D, FP4S, PVM, QP, 0>(tq, tk, tv, a, BH, stream);
-  return a.causal ? launch_fwd_sp<D, FP4S, PVM, QP, 2>(tq, tk, tv, a, BH, stream)
-                  : launch_fwd_sp<D, FP4S, PVM, QP, 1>(tq, tk, tv, a, BH, stream);
+  if (!a.kv_list) return launch_fwd_sp<D, FP4S, PV4, QP, 0>(tq, tk, tv, a, BH, stream);
+  return a.causal ? launch_fwd_sp<D, FP4S, PV4, QP, 2>(tq, tk, tv, a, BH, stream)
+                  : launch_fwd_sp<D, FP4S, PV4, QP, 1>(tq, tk, tv, a, BH, stream);
 }
 
 template <int D, int FP4S>
-static cudaError_t fwd_dispatch(int pv_mode, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+static cudaError_t fwd_dispatch(bool pv4, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
                                 const CUtensorMap &tv, const FwdArgs &a, int BH, cudaStream_t stream) {
-  if (pv_mode == 2) return launch_fwd_t<D, FP4S, 2, 1>(tq, tk, tv, a, BH, stream);
-  if (pv_mode == 1)
-    return quant_p ? launch_fwd_t<D, FP4S, 1, 1>(tq, tk, tv, a, BH, stream)
-                   : launch_fwd_t<D, FP4S, 1, 0>(tq, tk, tv, a, BH, stream);
+  // the NVFP4 P V needs every quantizer (FP4S included)
+  if (FP4S && pv4) return launch_fwd_t<D, FP4S, 1, 1>(tq, tk, tv, a, BH, stream);
   return quant_p ? launch_fwd_t<D, FP4S, 0, 1>(tq, tk, tv, a, BH, stream)
                  : launch_fwd_t<D, FP4S, 0, 0>(tq, tk, tv, a, BH, stream);
 }
 
-cudaError_t launch_fwd(int D, bool qk_f16, int pv_mode, bool quant_p, const CUtensorMap &tq,
-                       const CUtensorMap &tk, const CUtensorMap &tv, const FwdArgs &a, int BH,
-                       cudaStream_t stream) {
+cudaError_t launch_fwd(int D, bool fp4s, bool pv4, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, const FwdArgs &a, int BH, cudaStream_t stream) {
   // quantized Q and K: S runs on the NVFP4 tensor-core path
   if (D == 128)
-    return qk_f16 ? fwd_dispatch<128, 1>(pv_mode, quant_p, tq, tk, tv, a, BH, stream)
-                  : fwd_dispatch<128, 0>(pv_mode, quant_p, tq, tk, tv, a, BH, stream);
-  return qk_f16 ? fwd_dispatch<64, 1>(pv_mode, quant_p, tq, tk, tv, a, BH, stream)
-                : fwd_dispatch<64, 0>(pv_mode, quant_p, tq, tk, tv, a, BH, stream);
+    return fp4s ? fwd_dispatch<128, 1>(pv4, quant_p, tq, tk, tv, a, BH, stream)
+                : fwd_dispatch<128, 0>(pv4, quant_p, tq, tk, tv, a, BH, stream);
+  return fp4s ? fwd_dispatch<64, 1>(pv4, quant_p, tq, tk, tv, a, BH, stream)
+              : fwd_dispatch<64, 0>(pv4, quant_p, tq, tk, tv, a, BH, stream);
 }
 
 }  // namespace attnqat

@@ -16,6 +16,12 @@ struct FwdArgs {
   const uint8_t *qsf;   // scale-factor tiles of fq(Q), fq(K) (NVFP4 S path)
   const uint8_t *ksf;
   const uint8_t *vsf;   // scale-factor tiles of fq(V) along tokens (NVFP4 P V path)
+  // Every 16-bit operand of the MMAs is fp16: fq(X) unscaled (exact), or, for
+  // an operand whose quantizer is off, X * 2^e with 2^e = pow2_scale(*amax_x).
+  // amax_x points at that max magnitude, or is null for a quantized operand.
+  const float *amax_q;
+  const float *amax_k;
+  const float *amax_v;
   __nv_bfloat16 *o;
   float *o32;   // float32 copy of O kept in the workspace for the backward's Delta
   float *lse;
@@ -37,6 +43,9 @@ struct BwdArgs {
   // they bound |dS| and fix the power-of-two scale of the f16 dS operand;
   // stats[3] = max |dO| fixes the scale of the fp16 copy of dO.
   const float *stats;
+  const float *amax_q;   // as FwdArgs: the scales of the fp16 operand copies
+  const float *amax_k;
+  const float *amax_v;
   const float *m;
   const float *lse;
   const float *delta;
@@ -55,27 +64,32 @@ struct BwdArgs {
   int causal;  // as FwdArgs::causal
 };
 
-// Forward.  tv: 3-D TMA map {D, L, B*H} with 64 x 128 boxes, 128-byte swizzle
-// over fq(V) (pv_mode 1: fp16, 0: bf16); with pv_mode 2 (every quantizer on,
-// Lk % 32 == 0) it maps fq(V)'s packed codes {Lk/2 bytes, D, B*H} with
-// 64-byte x D boxes and 64-byte swizzle, a.vsf their scale tiles, and P V is
-// a block-scaled NVFP4 MMA.  With qk_f16 (Q and K quantized) tq/tk map the
-// packed NVFP4 codes {D/2 bytes, L, B*H} with (D/2) x 128 boxes and a
-// D/2-byte swizzle, a.qsf/a.ksf point at their scale-factor tiles, and S runs
-// as a block-scaled NVFP4 MMA; otherwise tq/tk map the bf16 Q and K.
-cudaError_t launch_fwd(int D, bool qk_f16, int pv_mode, bool quant_p, const CUtensorMap &tq,
-                       const CUtensorMap &tk, const CUtensorMap &tv, const FwdArgs &a, int BH,
-                       cudaStream_t stream);
+// Forward.  Every 16-bit operand is fp16 (see FwdArgs::amax_q).  With fp4s
+// (Q and K quantized) tq/tk map the packed NVFP4 codes {D/2 bytes, L, B*H}
+// with (D/2) x 128 boxes and a D/2-byte swizzle, a.qsf/a.ksf point at their
+// scale-factor tiles, and S runs as a block-scaled NVFP4 MMA; otherwise tq/tk
+// map the fp16 copies of Q and K {D, L, B*H} with 64 x 128 boxes and 128-byte
+// swizzle.  With pv4 (every quantizer on, Lk % 32 == 0) tv maps
+// fq(V)'s packed codes {Lk/2 bytes, D, B*H} with 64-byte x D boxes and 64-byte
+// swizzle, a.vsf their scale tiles, and P V is a block-scaled NVFP4 MMA;
+// otherwise tv maps the fp16 copy of V (64 x 128 boxes, 128-byte swizzle) and
+// P V is an fp16 MMA.
+cudaError_t launch_fwd(int D, bool fp4s, bool pv4, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, const FwdArgs &a, int BH, cudaStream_t stream);
 
-cudaError_t launch_bwd_dkdv(int D, bool qk_f16, bool quant_p, bool do_f16, const CUtensorMap &tq,
-                            const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tdo,
-                            const CUtensorMap &tq4, const BwdArgs &a, int BH, cudaStream_t stream);
-// dQ.  With qk_f16, tq maps the packed NVFP4 Q codes (as for the forward),
-// tk4 the K codes, a.qsf/a.ksf their scale tiles, and tk the fp16 fq(K) that
-// dQ = dS fq(K) reads; otherwise tq/tk are bf16 and tk4 is unused.
-cudaError_t launch_bwd_dq(int D, bool qk_f16, bool do_f16, const CUtensorMap &tq, const CUtensorMap &tk,
-                          const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4,
-                          const BwdArgs &a, int BH, cudaStream_t stream);
+// dK/dV.  tq, tk, tv, tdo map the fp16 copies of Q, K, V and dO (64 x 128
+// boxes, 128-byte swizzle); with fp4s tk maps K's packed NVFP4 codes instead
+// and tq4 Q's codes (as for the forward), and S is block-scaled NVFP4.
+cudaError_t launch_bwd_dkdv(int D, bool fp4s, bool quant_p, const CUtensorMap &tq, const CUtensorMap &tk,
+                            const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tq4,
+                            const BwdArgs &a, int BH, cudaStream_t stream);
+// dQ.  With fp4s, tq maps the packed NVFP4 Q codes (as for the forward), tk4
+// the K codes, a.qsf/a.ksf their scale tiles, and tk the fp16 fq(K) that
+// dQ = dS fq(K) reads; otherwise tq/tk map the fp16 copies and tk4 is unused.
+// dsplit feeds dS as an fp16 hi + lo pair (always so without fp4s).
+cudaError_t launch_bwd_dq(int D, bool fp4s, bool dsplit, const CUtensorMap &tq, const CUtensorMap &tk,
+                          const CUtensorMap &tv, const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a,
+                          int BH, cudaStream_t stream);
 
 // NVFP4 fq of a strided bf16 view (see attnqat_quantize; cols need not be a
 // multiple of 16 here: a ragged last block reads zeros); any of codes,
@@ -104,9 +118,10 @@ cudaError_t launch_quantize_gs(const uint16_t *x, int64_t batch, int64_t rows, i
 cudaError_t launch_delta(const float *o32, const __nv_bfloat16 *dO, float *delta, int64_t rows, int D,
                          float *stats, cudaStream_t stream);
 
-// out = fp16(dO * 2^e) over n elements (n % 8 == 0), 2^e = do_scale(stats).
-cudaError_t launch_scale_do(const __nv_bfloat16 *dO, uint16_t *out, int64_t n, const float *stats,
-                            cudaStream_t stream);
+// out = fp16(x * 2^e) over n bf16 elements (n % 8 == 0), 2^e =
+// pow2_scale(*amax) (max |x| lands in [2^13, 2^14)).
+cudaError_t launch_scale_f16(const __nv_bfloat16 *x, uint16_t *out, int64_t n, const float *amax,
+                             cudaStream_t stream);
 
 // Block-sparse tile lists from a tile mask [BH][nq][nk] (nonzero = the
 // query tile attends the key tile): kv_list/kv_count per query tile and

@@ -7,3 +7,4 @@
 #include "sparse.cu"
 #include "api.cu"
 #include "noalloc.cu"
+#include "selftest.cu"

@@ -286,52 +286,82 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Blocks of 16 consecutive tokens per channel of a [heads][L][D] tensor (V):
-// thread (channel r, token block b), consecutive threads on consecutive
-// channels, so each of the 16 loads and stores of a warp covers 64
-// contiguous bytes.  A ragged last block reads zeros past L.  Codes and
-// scales plain ([head][r][blocks]) or, with `tiled`, scales in the
-// per-128-token-tile layout of the general kernel's sf_col_tiles mode.
+// Blocks of 16 consecutive tokens per channel of a [heads][L][D] tensor (V).
+// Thread (channel group g, token block b) quantizes the 8 channels 8g..8g+7
+// over the 16 tokens of block b: 16 loads of 16 bytes (one token row's 8
+// channels each; consecutive threads on consecutive channel groups, so a warp
+// reads whole rows), a byte-permute transpose into 8 per-channel blocks, the
+// exact fq of each, the transpose back, and 16-byte stores of the
+// dequantized rows.  A ragged last block reads zeros past L (and stores only
+// its valid tokens).  Codes ([head][r][blocks], 8 bytes per block) and scales
+// plain ([head][r][blocks]) or, with `tiled`, scales in the per-128-token-tile
+// layout of the general kernel's sf_col_tiles mode.
 template <int D>
 __global__ void __launch_bounds__(256)
     quantize_tokens_kernel(const uint16_t *__restrict__ x, int64_t L, uint8_t *__restrict__ codes,
                            uint8_t *__restrict__ scales, bool tiled, uint16_t *__restrict__ deq,
                            uint16_t *__restrict__ deq_f16, float *__restrict__ absmax) {
+  constexpr int G = D / 8;  // channel groups of 8
   const int64_t nblk = (L + 15) >> 4;
   const int64_t id = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
-  const int r = static_cast<int>(id % D);
-  const int64_t b = id / D;
+  const int g = static_cast<int>(id % G);
+  const int64_t b = id / G;
   float dmax = 0.0f;
   if (b < nblk) {  // no early return: every thread joins the block max below
     const int64_t z = blockIdx.y;
-    const int64_t base = (z * L + b * 16) * D + r;
+    const int64_t row0 = z * L + b * 16;  // first token row of the block
     const int n = static_cast<int>(L - b * 16 < 16 ? L - b * 16 : 16);
-    uint32_t w[8];
+    uint4 t[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t lo = 2 * i < n ? __ldg(x + base + (2 * i) * D) : 0u;
-      const uint32_t hi = 2 * i + 1 < n ? __ldg(x + base + (2 * i + 1) * D) : 0u;
-      w[i] = lo | (hi << 16);
-    }
-    uint32_t nib[2], scode, hb[8];
-    fq16_exact(w, nib, scode, hb, dmax);
-    const int64_t blk = (z * D + r) * nblk + b;
-    if (codes) *reinterpret_cast<uint2 *>(codes + blk * 8) = make_uint2(nib[0], nib[1]);
-    if (scales) {
-      if (tiled) {
-        const int64_t ntiles = (nblk + 7) >> 3;
-        scales[((z * ntiles + (b >> 3)) * 2 + ((b >> 2) & 1)) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)] =
-            static_cast<uint8_t>(scode);
-      } else {
-        scales[blk] = static_cast<uint8_t>(scode);
+    for (int i = 0; i < 16; ++i)
+      t[i] = i < n ? __ldg(reinterpret_cast<const uint4 *>(x + (row0 + i) * D + g * 8)) : make_uint4(0, 0, 0, 0);
+    uint32_t out[16][4];  // dequantized rows (fp16 pairs of channels)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {  // channel pair 2m, 2m+1 (word m of each row)
+      uint32_t wl[8], wh[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t a = (&t[2 * i].x)[m], c = (&t[2 * i + 1].x)[m];
+        wl[i] = __byte_perm(a, c, 0x5410);  // channel 2m: tokens 2i, 2i+1
+        wh[i] = __byte_perm(a, c, 0x7632);  // channel 2m+1
+      }
+      uint32_t nl[2], nh[2], sl, sh, hl[8], hh[8];
+      float dl, dh;
+      fq16_exact(wl, nl, sl, hl, dl);
+      fq16_exact(wh, nh, sh, hh, dh);
+      dmax = fmax3(dmax, dl, dh);
+      const int r = g * 8 + 2 * m;  // channel of wl
+      const int64_t blk = (z * D + r) * nblk + b;
+      if (codes) {
+        *reinterpret_cast<uint2 *>(codes + blk * 8) = make_uint2(nl[0], nl[1]);
+        *reinterpret_cast<uint2 *>(codes + (blk + nblk) * 8) = make_uint2(nh[0], nh[1]);
+      }
+      if (scales) {
+        if (tiled) {
+          const int64_t base = ((z * ((nblk + 7) >> 3) + (b >> 3)) * 2 + ((b >> 2) & 1)) * 512 + (b & 3);
+          scales[base + (r & 31) * 16 + (r >> 5) * 4] = static_cast<uint8_t>(sl);
+          scales[base + ((r + 1) & 31) * 16 + ((r + 1) >> 5) * 4] = static_cast<uint8_t>(sh);
+        } else {
+          scales[blk] = static_cast<uint8_t>(sl);
+          scales[blk + nblk] = static_cast<uint8_t>(sh);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        out[2 * i][m] = __byte_perm(hl[i], hh[i], 0x5410);
+        out[2 * i + 1][m] = __byte_perm(hl[i], hh[i], 0x7632);
       }
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       if (i < n) {
-        const uint32_t h = hb[i >> 1] >> (16 * (i & 1));
-        if (deq) deq[base + i * D] = static_cast<uint16_t>(bf16x2_from_f16x2_exact(h & 0xFFFFu));
-        if (deq_f16) deq_f16[base + i * D] = static_cast<uint16_t>(h);
+        const int64_t off = (row0 + i) * D + g * 8;
+        if (deq_f16)
+          *reinterpret_cast<uint4 *>(deq_f16 + off) = make_uint4(out[i][0], out[i][1], out[i][2], out[i][3]);
+        if (deq)
+          *reinterpret_cast<uint4 *>(deq + off) =
+              make_uint4(bf16x2_from_f16x2_exact(out[i][0]), bf16x2_from_f16x2_exact(out[i][1]),
+                         bf16x2_from_f16x2_exact(out[i][2]), bf16x2_from_f16x2_exact(out[i][3]));
       }
     }
   }
@@ -344,9 +374,11 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
                             bool sf_col_tiles) {
   const int64_t total = batch * rows * ((cols + 15) / 16);
   if (total == 0) return cudaSuccess;
+  // the two fast kernels move 16-byte rows of values and 8-byte groups of codes
   const bool aligned = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 &&
                        (!deq || (reinterpret_cast<uintptr_t>(deq) & 15u) == 0) &&
-                       (!deq_f16 || (reinterpret_cast<uintptr_t>(deq_f16) & 15u) == 0);
+                       (!deq_f16 || (reinterpret_cast<uintptr_t>(deq_f16) & 15u) == 0) &&
+                       (!codes || (reinterpret_cast<uintptr_t>(codes) & 7u) == 0);
   // contiguous rows of 64 or 128 elements, blocks along the row
   if (batch == 1 && sc == 1 && sr == cols && (cols == 64 || cols == 128) && !absmax && !sf_col_tiles && aligned &&
       (sf_tile_rows <= 0 || rows % sf_tile_rows == 0)) {
@@ -364,8 +396,8 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
   }
   // [heads][L][D] blocked along tokens: rows = D channels (stride 1), cols = L
   // tokens (stride D), batch = heads (stride L*D)
-  if (sr == 1 && (rows == 64 || rows == 128) && sc == rows && sb == rows * cols && sf_tile_rows <= 0) {
-    const int64_t gx = (((cols + 15) / 16) * rows + 255) / 256;
+  if (sr == 1 && (rows == 64 || rows == 128) && sc == rows && sb == rows * cols && sf_tile_rows <= 0 && aligned) {
+    const int64_t gx = (((cols + 15) / 16) * (rows / 8) + 255) / 256;
     if (batch <= 65535 && gx <= 0x7fffffff) {
       const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(batch));
       if (rows == 128)
@@ -650,17 +682,18 @@ cudaError_t launch_delta(const float *o32, const __nv_bfloat16 *dO, float *delta
   return cudaGetLastError();
 }
 
-// dO' = fp16(dO * 2^e) with 2^e = do_scale(stats) (max |dO| lands in
-// [2^13, 2^14)).  bf16 values carry 8 significant bits, so the fp16 copy is
-// exact for every element within 2^27 of the largest.  8 elements per
-// thread, grid-stride.
+// x' = fp16(x * 2^e) with 2^e = pow2_scale(*amax) (max |x| lands in
+// [2^13, 2^14)): the backward's copy of dO, and the copy of Q, K or V when
+// that operand is not quantized.  bf16 values carry 8 significant bits, so
+// the fp16 copy is exact for every element within 2^27 of the largest.  8
+// elements per thread, grid-stride.
 __global__ void __launch_bounds__(256)
-    scale_do_kernel(const uint4 *__restrict__ dO, uint4 *__restrict__ out, int64_t n8,
-                    const float *__restrict__ stats) {
-  const float sc = do_scale(stats);
+    scale_f16_kernel(const uint4 *__restrict__ x, uint4 *__restrict__ out, int64_t n8,
+                     const float *__restrict__ amax) {
+  const float sc = pow2_scale(*amax);
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint4 b = __ldg(dO + i);
+    const uint4 b = __ldg(x + i);
     const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
     uint32_t w[4];
 #pragma unroll
@@ -670,8 +703,8 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-cudaError_t launch_scale_do(const __nv_bfloat16 *dO, uint16_t *out, int64_t n, const float *stats,
-                            cudaStream_t stream) {
+cudaError_t launch_scale_f16(const __nv_bfloat16 *x, uint16_t *out, int64_t n, const float *amax,
+                             cudaStream_t stream) {
   if (n == 0) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -679,13 +712,13 @@ cudaError_t launch_scale_do(const __nv_bfloat16 *dO, uint16_t *out, int64_t n, c
   const int64_t n8 = n / 8;
   const int64_t need = (n8 + 255) / 256;
   const int64_t cap = static_cast<int64_t>(sms) * 8;
-  scale_do_kernel<<<static_cast<unsigned>(need < cap ? need : cap), 256, 0, stream>>>(
-      reinterpret_cast<const uint4 *>(dO), reinterpret_cast<uint4 *>(out), n8, stats);
+  scale_f16_kernel<<<static_cast<unsigned>(need < cap ? need : cap), 256, 0, stream>>>(
+      reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(out), n8, amax);
   return cudaGetLastError();
 }
 
-// max |x| over n bf16 values folded into *out (used for V when it is not
-// quantized, so the forward did not record max |fq(V)|).
+// max |x| over n bf16 values folded into *out (for Q, K or V when it is not
+// quantized: the scale of its fp16 copy, and for V the bound on |dS|).
 __global__ void __launch_bounds__(256) absmax_kernel(const uint4 *__restrict__ x, int64_t n8, float *out) {
   float m = 0.0f;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;

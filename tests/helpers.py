@@ -50,9 +50,11 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return np.where(ax > 0, np.exp2(e - 7), 0.0)
 
 
-def _log(name, rel, mx, criterion, floor_mx):
+def _log(name, rel, mx, criterion, floor_mx, literal_mx):
     """Appends the achieved errors to $ATTNQAT_PARITY_LOG (one JSON line per
-    comparison) when that variable is set."""
+    comparison) when that variable is set: the figure the bar was applied to,
+    the literal max |got - ref| / RMS(ref) beside it, and the literal figure
+    of the exact reference rounded to bf16 (the best any bf16 output can do)."""
     import json
     import os
     path = os.environ.get("ATTNQAT_PARITY_LOG")
@@ -60,7 +62,8 @@ def _log(name, rel, mx, criterion, floor_mx):
         test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
         with open(path, "a") as f:
             f.write(json.dumps(dict(test=test, tensor=name, rel_l2=rel, max_abs_over_rms=mx,
-                                    criterion=criterion, bf16_floor_max_abs_over_rms=floor_mx)) + "\n")
+                                    criterion=criterion, literal_max_abs_over_rms=literal_mx,
+                                    bf16_floor_max_abs_over_rms=floor_mx)) + "\n")
 
 
 def assert_close(name, got, ref, rel_tol=REL_L2_TOL, max_tol=MAX_ABS_OVER_RMS_TOL):
@@ -77,15 +80,17 @@ def assert_close(name, got, ref, rel_tol=REL_L2_TOL, max_tol=MAX_ABS_OVER_RMS_TO
     ref = np.asarray(ref, np.float64)
     assert np.all(np.isfinite(got)), "%s has non-finite values" % name
     rel, mx = errors(got, ref)
+    literal = mx
     floor_mx = errors(bf16_round(ref), ref)[1]
     criterion = "max_abs"
     if floor_mx > max_tol:
         criterion = "max_abs_beyond_1ulp"
         rms = np.linalg.norm(ref) / np.sqrt(max(ref.size, 1))
         mx = float(np.max(np.abs(got - ref) - bf16_ulp(ref)) / rms)
-    _log(name, rel, mx, criterion, floor_mx)
-    assert rel <= rel_tol and mx <= max_tol, "%s: rel-L2 %.3e (tol %.0e), %s %.3e (tol %.0e)" % (
-        name, rel, rel_tol, criterion, mx, max_tol)
+    _log(name, rel, mx, criterion, floor_mx, literal)
+    assert rel <= rel_tol and mx <= max_tol, (
+        "%s: rel-L2 %.3e (tol %.0e), %s %.3e (tol %.0e); literal max-abs/RMS %.3e, bf16 floor %.3e" % (
+            name, rel, rel_tol, criterion, mx, max_tol, literal, floor_mx))
     return rel, mx
 
 

@@ -33,29 +33,22 @@ def test_strerror_texts():
 
 
 def _expected_ws(B, H, Lq, Lk, D, flags):
-    """Workspace layout restated: 256-byte aligned regions for fq(Q), fq(K),
-    fq(V) (bf16), fq(V) (fp16), float32 O, Delta, 16 bytes of statistics,
-    with every quantizer on the fp16 copy of dO, with Q and K quantized
-    their packed codes and scale tiles, and with every quantizer on, D = 128
-    and Lk % 32 == 0 fq(V)'s packed codes and scale tiles."""
+    """Workspace layout restated: 256-byte aligned regions for the fp16
+    copies of Q, K and V (fq or scaled), float32 O, Delta, 32 bytes of
+    statistics, the fp16 copy of dO, with Q and K quantized their packed codes
+    and scale tiles, and with every quantizer on and Lk % 32 == 0 fq(V)'s
+    packed codes and scale tiles."""
     al = lambda x: (x + 255) // 256 * 256
     BH = B * H
-    n = 0
-    if flags & 1:
-        n += al(BH * Lq * D * 2)
-    if flags & 2:
-        n += al(BH * Lk * D * 2)
-    if flags & 4:
-        n += 2 * al(BH * Lk * D * 2)
-    n += al(BH * Lq * D * 4) + al(BH * Lq * 4) + al(16)
-    if flags & 15 == 15:
-        n += al(BH * Lq * D * 2)  # fp16 copy of dO for the all-quantized backward
+    n = al(BH * Lq * D * 2) + 2 * al(BH * Lk * D * 2)
+    n += al(BH * Lq * D * 4) + al(BH * Lq * 4) + al(32)
+    n += al(BH * Lq * D * 2)  # fp16 copy of dO
     if flags & 3 == 3:
         # packed NVFP4 codes (D/2 bytes per row) and 512-byte scale tiles per
         # 128 rows x 64 columns, for Q then K
         for L in (Lq, Lk):
             n += al(BH * L * D // 2) + al(BH * ((L + 127) // 128) * (D // 64) * 512)
-    if flags & 15 == 15 and Lk % 32 == 0 and D == 128:
+    if flags & 15 == 15 and Lk % 32 == 0:
         # fq(V)'s packed codes and 1 KB of scales per 128-token tile
         n += al(BH * Lk * D // 2) + al(BH * ((Lk + 127) // 128) * 1024)
     return n
@@ -117,6 +110,7 @@ def test_quantize_host_validation():
     assert quant(rows=0) == A.EINVAL
     assert quant(sr=-1) == A.EINVAL
     assert quant(x=FAKE + 1) == A.EINVAL
+    assert quant(codes=FAKE + 4) == A.EINVAL  # codes are written as 8-byte groups
 
 
 def test_noalloc_rejects_oversized_shapes_before_any_device_call():
@@ -148,6 +142,7 @@ def test_quantize_gs_host_validation():
     assert quant(g=FAKE + 2) == A.EINVAL     # float32 slot misaligned
     assert quant(x=0) == A.EINVAL
     assert quant(codes=0) == A.EINVAL
+    assert quant(codes=FAKE + 4) == A.EINVAL
     assert quant(cols=24) == A.EINVAL
 
 
@@ -219,7 +214,16 @@ def test_causal_flag_validation_and_workspace():
                                 P(FAKE), P(FAKE), P(FAKE), P(FAKE), big, None)
     assert st == A.EINVAL
     assert _fwd(lib, flags=64, ws_bytes=big) == A.EINVAL  # still an unknown bit
-    # causal masking needs every quantizer (fp16 dS and dV operands)
-    for flags in (A.CAUSAL, A.QUANT_Q | A.QUANT_V | A.QUANT_P | A.CAUSAL, A.QUANT_Q | A.QUANT_K | A.CAUSAL):
-        assert _fwd(lib, flags=flags, ws_bytes=big) == A.EINVAL
-    assert _fwd(lib, flags=A.QUANT_ALL | A.CAUSAL, ws_bytes=16) == A.ENOSPC
+    # every flag set takes causal masking (every backward operand is fp16)
+    for flags in range(16):
+        need = A.attnqat_workspace_size(1, 1, 128, 128, 128, flags | A.CAUSAL)
+        assert need > A.attnqat_workspace_size(1, 1, 128, 128, 128, flags) > 0
+        assert _fwd(lib, flags=flags | A.CAUSAL, ws_bytes=need - 1) == A.ENOSPC
+
+
+def test_selftest_wait_timeout_validation():
+    lib = A.load()
+    assert lib.attnqat_selftest_wait_timeout(1000000, None, None) == A.EINVAL       # no counter
+    assert lib.attnqat_selftest_wait_timeout(1000000, P(FAKE + 2), None) == A.EINVAL  # misaligned
+    assert lib.attnqat_selftest_wait_timeout(999, P(FAKE), None) == A.EINVAL         # limit too short
+    assert lib.attnqat_selftest_wait_timeout(3 * 10**9, P(FAKE), None) == A.EINVAL   # above 2 s

@@ -1,8 +1,11 @@
 """Parity of causal masking (flag ATTNQAT_CAUSAL on attnqat_fwd / attnqat_bwd,
 through the C ABI) with the float64 oracle: full comparisons with ragged,
 exact-multiple, single-tile and tiny lengths, both head dimensions and the
-fp16 P V route, all with every quantizer on (the only flag set the library
-accepts causal masking with).  Bar as for dense attention."""
+fp16 P V route with every quantizer on, and the flag sets with some quantizer
+off (whose unquantized operands reach the MMAs as power-of-two-scaled fp16
+copies).  The first keys' gradients gather every later row's contribution, so
+they are heavy-tailed: these cases check that dS and the dV operand keep
+enough precision.  Bar as for dense attention."""
 import pytest
 
 import oracle
@@ -32,6 +35,12 @@ def _full_compare(w, flags):
     (128, 128, oracle.QUANT_ALL),     # the diagonal tile alone
     (7, 128, oracle.QUANT_ALL),
     (1, 64, oracle.QUANT_ALL),
+    (500, 128, 0),                                    # no quantizer
+    (500, 128, oracle.QUANT_Q | oracle.QUANT_K),
+    (500, 128, oracle.QUANT_P),
+    (500, 128, oracle.QUANT_V | oracle.QUANT_P),
+    (1000, 64, oracle.QUANT_Q | oracle.QUANT_V),
+    (1024, 128, oracle.QUANT_ALL & ~oracle.QUANT_P),
 ])
 def test_causal_full(L, D, flags):
     w = W.custom(1, 2, L, L, D, seed_index=900 + L % 97 + D + flags)
