@@ -5,8 +5,8 @@ One step = attnqat_fwd + attnqat_bwd over one batch of the pages' shape:
 B=1, H=6, Lq=Lk=31200, D=128, bf16, all four quantizers on, sm_scale=1/sqrt(128)
 (the 6-head, 31200-token shape the fastvideo-kernel commit times).  The step
 runs every kernel of the path: the three operand quantizers, the forward, the
-Delta kernel, the kernel writing the exact fp16 copy of dO, the dK/dV kernel
-and the dQ kernel.
+Delta kernel, the kernel writing the fp16 copy of dO, the dK/dV kernel and the
+dQ kernel.
 
 Metric: nominal TFLOP/s of fwd+bwd (forward 4*B*H*Lq*Lk*D, backward 2.5x that),
 also reported as fwd / bwd / fwd+bwd milliseconds and as a fraction of the
@@ -14,10 +14,15 @@ measured B200 BF16 tensor peak.  Inputs are seeded synthetic tensors; L2 is
 flushed (a 256 MiB write) between timed steps, each step is timed with CUDA
 events on the launching stream, and multi-GPU runs report the max over ranks.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--sparsity S | --causal]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--workload NAME] [--flags F] [--sparsity S | --causal]
+
+--workload times another of the seeded workloads (tiny, outlier_channels_4096,
+wan_6h_31200, scaled_heads_16384, large_40h_75600) and --flags another set of
+quantizers (bits q=1, k=2, v=4, p=8; default all four).
 
 --sparsity S times the block-sparse (VSA fine attention) step instead:
-attnqat_vsa_select (the top max(1, min(ceil((1-S)*244), 244)) of the 244 key
+attnqat_vsa_select (the top max(1, min(ceil((1-S)*nk), nk)) of the nk key
 tiles per 128-query tile by coarse tile-mean scores; the pages' VSA checkpoint
 uses S = 0.9) + attnqat_sparse_fwd + attnqat_sparse_bwd on the same shape,
 with TFLOP/s counted on the selected tiles only.
@@ -25,6 +30,11 @@ with TFLOP/s counted on the selected tiles only.
 --causal times the causal step (ATTNQAT_CAUSAL on attnqat_fwd / attnqat_bwd,
 query i attending keys j <= i) on the same shape, with TFLOP/s counted on the
 unmasked (query, key) pairs, L(L+1)/2 per head.
+
+The end-to-end leg ("e2e") runs the same step through the public API with the
+inputs in pinned host memory: every step copies Q, K, V, dO to the device and
+O, LSE, m, dQ, dK, dV back, on two copy streams, double-buffered so that one
+step's copies overlap the neighbouring steps' kernels.
 
 --impl reference times the float64 CPU oracle on the host cores instead (the
 pages ship no runnable implementation): each step is a bounded sample of the
@@ -51,9 +61,15 @@ from quantization_aware_attention_nvfp4_b200 import workloads as W  # noqa: E402
 
 WORKLOAD = "wan_6h_31200"
 METRIC = "Attn-QAT fwd+bwd ms & TFLOP/s at H6 L31200 D128; % of B200 BF16 peak"
-SPARSE_METRIC = ("Block-sparse (VSA) Attn-QAT fwd+bwd ms & TFLOP/s on the selected tiles at H6 L31200 D128, "
+SPARSE_METRIC = ("Block-sparse (VSA) Attn-QAT fwd+bwd ms & TFLOP/s on the selected tiles at %s, "
                  "sparsity %g")
-CAUSAL_METRIC = "Causal Attn-QAT fwd+bwd ms & TFLOP/s on the unmasked pairs at H6 L31200 D128"
+CAUSAL_METRIC = "Causal Attn-QAT fwd+bwd ms & TFLOP/s on the unmasked pairs at %s"
+OTHER_METRIC = "Attn-QAT fwd+bwd ms & TFLOP/s at %s; % of B200 BF16 peak"
+FLAG_NAMES = ((1, "q"), (2, "k"), (4, "v"), (8, "p"))
+# nominal dense tensor rates of B200 per input type, relative to bf16/fp16
+# (2.25 PFLOP/s bf16, 9 PFLOP/s fp4): the dK/dV kernel's S unit runs on the
+# block-scaled NVFP4 pipe when Q and K are quantized
+NVFP4_RATE_RATIO = 4.0
 # query rows (= keys) of the oracle's causal sample: its cost grows with the
 # square of the prefix, like the dense sample's rows x all keys
 CAUSAL_SAMPLE_ROWS = int(os.environ.get("ATTNQAT_CAUSAL_BASELINE_ROWS", "15360"))
@@ -64,6 +80,20 @@ FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=
 # each step of --impl reference
 BASELINE_SAMPLE_ROWS = int(os.environ.get("ATTNQAT_BASELINE_ROWS", "6144"))
 ORACLE_SAMPLE_ROWS = int(os.environ.get("ATTNQAT_ORACLE_SAMPLE_ROWS", "1024"))
+
+
+def shape_name(w):
+    return "B%d H%d L%d%s D%d" % (w.B, w.H, w.Lq, "" if w.Lq == w.Lk else "x%d" % w.Lk, w.D)
+
+
+def flag_names(flags):
+    return ",".join(n for b, n in FLAG_NAMES if flags & b) or "none"
+
+
+def sample_rows(w, rows):
+    """Query rows of an oracle sample with about the work of `rows` rows
+    against 31200 keys (the cost of a row grows with Lk)."""
+    return max(1, min(w.Lq, int(rows * 31200 / w.Lk)))
 
 
 def load_peaks():
@@ -183,6 +213,30 @@ def selected_pairs(w, mask):
     return float(np.einsum("bhij,i,j->", mask.astype(np.float64), rows, keys))
 
 
+def dtype_weighted_peak(peak, n_units, fp4_units, ratio=NVFP4_RATE_RATIO):
+    """Peak rate of a kernel whose n_units matmul units run fp4_units on the
+    NVFP4 pipe (ratio times the bf16 rate) and the rest at the bf16 peak: the
+    units over the time floor sum_u (1 / rate_u)."""
+    return peak * n_units / ((n_units - fp4_units) + fp4_units / ratio)
+
+
+def metric_name(args, w):
+    if args.sparsity is not None:
+        return SPARSE_METRIC % (shape_name(w), args.sparsity)
+    if args.causal:
+        return CAUSAL_METRIC % shape_name(w)
+    if w.name == WORKLOAD and args.flags == 15:
+        return METRIC
+    return OTHER_METRIC % shape_name(w)
+
+
+def workload_name(args, w):
+    name = w.name if args.flags == 15 else "%s_flags%d" % (w.name, args.flags)
+    if args.sparsity is not None:
+        return "vsa_" + name
+    return ("causal_" if args.causal else "") + name
+
+
 def gpu_arm(args):
     import torch
     import torch.distributed as dist
@@ -194,7 +248,7 @@ def gpu_arm(args):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
-    w = W.get(WORKLOAD)
+    w = W.get(args.workload)
     flops = w.nominal_flops()
     peaks = load_peaks()
     sparse = args.sparsity is not None
@@ -213,28 +267,29 @@ def gpu_arm(args):
     host = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16) for n in inp}
     q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
     c = w.sm_scale
-    flags = A.QUANT_ALL | (A.CAUSAL if causal else 0)
+    flags = args.flags | (A.CAUSAL if causal else 0)
     if sparse:
         tm = torch.empty((w.B, w.H, nq, nk), dtype=torch.uint8, device=dev)
         sel_ws = torch.empty(A.load().attnqat_vsa_select_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D),
                              dtype=torch.uint8, device=dev)
         ws_bytes = A.attnqat_sparse_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags)
 
-        def fwd(qq, kk, vv, out):
+        def fwd(qq, kk, vv, out, stream=None):
             # the selection belongs to the forward: coarse scores, top-k tiles
-            A.attnqat_vsa_select(qq, kk, topk, out=tm, ws=sel_ws)
-            return A.attnqat_sparse_fwd(qq, kk, vv, tm, sm_scale=c, flags=flags, ws=ws, out=out)
+            A.attnqat_vsa_select(qq, kk, topk, out=tm, ws=sel_ws, stream=stream)
+            return A.attnqat_sparse_fwd(qq, kk, vv, tm, sm_scale=c, flags=flags, ws=ws, out=out, stream=stream)
 
-        def bwd(qq, kk, vv, ll, mm, dd, out):
-            return A.attnqat_sparse_bwd(qq, kk, vv, ll, mm, dd, ws, tm, sm_scale=c, flags=flags, out=out)
+        def bwd(qq, kk, vv, ll, mm, dd, out, stream=None):
+            return A.attnqat_sparse_bwd(qq, kk, vv, ll, mm, dd, ws, tm, sm_scale=c, flags=flags, out=out,
+                                        stream=stream)
     else:
         ws_bytes = A.attnqat_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags)
 
-        def fwd(qq, kk, vv, out):
-            return A.attnqat_fwd(qq, kk, vv, sm_scale=c, flags=flags, ws=ws, out=out)
+        def fwd(qq, kk, vv, out, stream=None):
+            return A.attnqat_fwd(qq, kk, vv, sm_scale=c, flags=flags, ws=ws, out=out, stream=stream)
 
-        def bwd(qq, kk, vv, ll, mm, dd, out):
-            return A.attnqat_bwd(qq, kk, vv, ll, mm, dd, ws, sm_scale=c, flags=flags, out=out)
+        def bwd(qq, kk, vv, ll, mm, dd, out, stream=None):
+            return A.attnqat_bwd(qq, kk, vv, ll, mm, dd, ws, sm_scale=c, flags=flags, out=out, stream=stream)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
@@ -299,8 +354,15 @@ def gpu_arm(args):
     dom = max(tensor_kernels, key=lambda n: sum(tensor_kernels[n]))
     dom_ms = statistics.mean(per[dom])
     achieved = algo_flops[dom] / (dom_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    traffic = None if (sparse or causal) else load_traffic(dom)  # the committed counters are the dense step's
+    # the kernels run inside an ~11 ms step, not a seconds-long loop: the
+    # burst peak is the denominator
+    peak = peaks["bf16_tflops"]
+    # dtype-weighted: with Q and K quantized, one of dK/dV's four units (S)
+    # runs on the NVFP4 pipe, whose nominal rate is 4x bf16's; the time floor
+    # is then 3 units at the bf16 peak plus 1 at 4x it
+    fp4_units = {"attn_bwd_dkdv": 1, "attn_fwd": 0, "attn_bwd_dq": 0}[dom] if (args.flags & 3) == 3 else 0
+    weighted_peak = dtype_weighted_peak(peak, algo_flops[dom] / units, fp4_units)
+    traffic = None if (sparse or causal or w.name != WORKLOAD or args.flags != 15) else load_traffic(dom)
     kernel_table = {n: dict(launches=len(v), mean_ms=round(statistics.mean(v), 4),
                             share=round(sum(v) / sum(sum(x) for x in per.values()), 4))
                     for n, v in per.items()}
@@ -310,24 +372,25 @@ def gpu_arm(args):
             kernel_table[n]["executed_tflops"] = round(exec_flops[n] / (kernel_table[n]["mean_ms"] * 1e-3) / 1e12, 1)
 
     # ---- end to end through the public API with host buffers
-    e2e = e2e_arm(args, torch, dev, host, w, flops, fwd, bwd, world)
+    e2e = None if args.no_e2e else e2e_arm(args, torch, dev, host, w, flops, fwd, bwd, world)
 
     value = world * flops["total"] * args.steps / (tot_ms * 1e-3) / 1e12
     ms_step = tot_ms / args.steps
-    config = {"workload": WORKLOAD, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
-              "quantizers": "q,k,v,p", "sm_scale": "1/sqrt(128)", "global_batch": w.B * world,
-              "seq_len": w.Lq, "parallelism": "replicas x%d (heads independent, no collective)" % world,
+    config = {"workload": workload_name(args, w), "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
+              "quantizers": flag_names(args.flags), "sm_scale": "%.6g" % c, "values": w.description,
+              "global_batch": w.B * world, "seq_len": w.Lq,
+              "parallelism": "replicas x%d (heads independent, no collective)" % world,
               "l2": "flushed between steps (256 MiB write); each step timed with CUDA events"}
     if sparse:
-        config.update(workload="vsa_" + WORKLOAD, sparsity=args.sparsity, tile=W.SPARSE_TILE,
+        config.update(sparsity=args.sparsity, tile=W.SPARSE_TILE,
                       key_tiles_per_query_tile=int(mask_np.sum(-1).max()),
                       selected_fraction=round(pairs / (w.B * w.H * w.Lq * w.Lk), 5),
                       selection="attnqat_vsa_select in the timed forward (tile means, top-%d coarse scores)" % topk)
     if causal:
-        config.update(workload="causal_" + WORKLOAD, mask="causal (query i attends keys j <= i)",
+        config.update(mask="causal (query i attends keys j <= i)",
                       unmasked_fraction=round(pairs / (w.B * w.H * w.Lq * w.Lk), 5))
     out = {
-        "metric": SPARSE_METRIC % args.sparsity if sparse else (CAUSAL_METRIC if causal else METRIC),
+        "metric": metric_name(args, w),
         "value": round(value, 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -338,7 +401,7 @@ def gpu_arm(args):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16, recipe in DESIGN.md)",
+        "data": "synthetic (seeded N(0,1) float32 from numpy PCG64, rounded to bf16; %s)" % w.recipe,
         "config": config,
         "fwd_ms": round(fwd_ms / args.steps, 4),
         "bwd_ms": round(bwd_ms / args.steps, 4),
@@ -354,8 +417,11 @@ def gpu_arm(args):
                      "traffic": traffic,
                      "algorithmic_flops_per_launch": algo_flops[dom],
                      "mean_launch_ms": round(dom_ms, 4),
-                     "peak_kind": "measured bf16 sustained (kernel timed inside a long step)"
-                     if peaks["source"] == "measured" else "fallback"},
+                     "peak_kind": ("measured bf16 burst (cuBLAS 8192^3, best of 10; the kernel runs inside an "
+                                   "~%.0f ms step)" % ms_step) if peaks["source"] == "measured" else "fallback",
+                     "nvfp4_units_per_launch": fp4_units,
+                     "dtype_weighted_peak": round(weighted_peak, 1),
+                     "frac_dtype_weighted": round(achieved / weighted_peak, 4)},
         "kernels": kernel_table,
         # every profiled scope is one kernel launch except the selection (two)
         "gpu_launches": len(kernels) + sum(1 for n, _ in kernels if n == "vsa_select"),
@@ -365,8 +431,9 @@ def gpu_arm(args):
     }
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline_sample(rows=CAUSAL_SAMPLE_ROWS if causal else BASELINE_SAMPLE_ROWS,
-                                                      topk=topk if sparse else None, causal=causal)
+            out["cpu_baseline"] = cpu_baseline_sample(
+                w, args.flags, rows=sample_rows(w, CAUSAL_SAMPLE_ROWS if causal else BASELINE_SAMPLE_ROWS),
+                topk=topk if sparse else None, causal=causal)
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
@@ -375,44 +442,75 @@ def gpu_arm(args):
 
 def e2e_arm(args, torch, dev, host, w, flops, fwd, bwd, world):
     """Same step through the public API with host buffers: every step copies
-    Q, K, V, dO from pinned host memory to the device and O, LSE, m, dQ, dK, dV
-    back, all inside the timed region."""
+    Q, K, V, dO from pinned host memory to the device and O, LSE, m, dQ, dK,
+    dV back, all inside the timed region.
+
+    The copies run on their own streams and are double-buffered: step i's
+    inputs go to device slot i % 2 on the upload stream while step i-1
+    computes, and step i's results leave slot i % 2 on the download stream
+    while step i+1 computes.  Events order each copy against the kernels that
+    read or write its slot (an upload waits until the kernels of step i-2 are
+    done with the slot, the kernels wait for their upload and for the download
+    of step i-2 to have drained their output slot).  The region ends when the
+    last download has landed in host memory."""
     pin = {n: t.pin_memory() for n, t in host.items()}
-    outs = dict(o=torch.empty_like(pin["q"]).pin_memory(), dq=torch.empty_like(pin["q"]).pin_memory(),
-                dk=torch.empty_like(pin["k"]).pin_memory(), dv=torch.empty_like(pin["v"]).pin_memory(),
-                lse=torch.empty((w.B, w.H, w.Lq), dtype=torch.float32).pin_memory(),
-                m=torch.empty((w.B, w.H, w.Lq), dtype=torch.float32).pin_memory())
-    dbuf = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in pin.items()}
-    o = torch.empty_like(dbuf["q"])
-    lse = torch.empty((w.B, w.H, w.Lq), dtype=torch.float32, device=dev)
-    m = torch.empty_like(lse)
-    dq, dk, dv = torch.empty_like(dbuf["q"]), torch.empty_like(dbuf["k"]), torch.empty_like(dbuf["v"])
-    stream = torch.cuda.current_stream(dev)
+    shapes = dict(o=host["q"].shape, dq=host["q"].shape, dk=host["k"].shape, dv=host["v"].shape)
+    stat_shape = (w.B, w.H, w.Lq)
+    h_out = [dict({n: torch.empty(sh, dtype=torch.bfloat16).pin_memory() for n, sh in shapes.items()},
+                  lse=torch.empty(stat_shape, dtype=torch.float32).pin_memory(),
+                  m=torch.empty(stat_shape, dtype=torch.float32).pin_memory()) for _ in range(2)]
+    d_in = [{n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in pin.items()} for _ in range(2)]
+    d_out = [dict({n: torch.empty(sh, dtype=torch.bfloat16, device=dev) for n, sh in shapes.items()},
+                  lse=torch.empty(stat_shape, dtype=torch.float32, device=dev),
+                  m=torch.empty(stat_shape, dtype=torch.float32, device=dev)) for _ in range(2)]
+    comp = torch.cuda.current_stream(dev)
+    up = torch.cuda.Stream(dev)
+    down = torch.cuda.Stream(dev)
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out[0].values())
 
-    def step():
-        for n in pin:
-            dbuf[n].copy_(pin[n], non_blocking=True)
-        fwd(dbuf["q"], dbuf["k"], dbuf["v"], (o, lse, m))
-        bwd(dbuf["q"], dbuf["k"], dbuf["v"], lse, m, dbuf["do"], (dq, dk, dv))
-        for name, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv), ("lse", lse), ("m", m)):
-            outs[name].copy_(t, non_blocking=True)
+    def run(n_steps):
+        uploaded = [torch.cuda.Event() for _ in range(2)]
+        computed = [torch.cuda.Event() for _ in range(2)]
+        drained = [torch.cuda.Event() for _ in range(2)]
+        for i in range(n_steps):
+            b = i % 2
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(computed[b])  # the kernels of step i-2 are done with slot b
+                for n in pin:
+                    d_in[b][n].copy_(pin[n], non_blocking=True)
+                uploaded[b].record(up)
+            comp.wait_event(uploaded[b])
+            if i >= 2:
+                comp.wait_event(drained[b])  # step i-2's results have left slot b
+            x, y = d_in[b], d_out[b]
+            fwd(x["q"], x["k"], x["v"], (y["o"], y["lse"], y["m"]), stream=comp)
+            bwd(x["q"], x["k"], x["v"], y["lse"], y["m"], x["do"], (y["dq"], y["dk"], y["dv"]), stream=comp)
+            computed[b].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[b])
+                for n in h_out[b]:
+                    h_out[b][n].copy_(y[n], non_blocking=True)
+                drained[b].record(down)
+        comp.wait_stream(down)
 
-    for _ in range(2):
-        step()
+    run(2)
     torch.cuda.synchronize(dev)
     n = max(2, args.steps // 2)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n):
-        step()
-    e1.record(stream)
+    # the region opens on the compute stream before the first upload is queued
+    up.wait_stream(comp)
+    e0.record(comp)
+    up.wait_event(e0)
+    run(n)
+    e1.record(comp)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
     value = world * flops["total"] * n / (ms * 1e-3) / 1e12
     return {"value": round(value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": round(ms / n, 4)}
+            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": round(ms / n, 4),
+            "copies": "pinned host <-> device every step, on upload/download streams, double-buffered"}
 
 
 def load_traffic(kernel):
@@ -434,16 +532,15 @@ def load_traffic(kernel):
 
 # -------------------------------------------------------------- CPU oracle --
 
-def cpu_baseline_sample(rows: int, topk=None, causal=False):
+def cpu_baseline_sample(w, flags, rows: int, topk=None, causal=False):
     """The float64 oracle on a bounded sample of the workload: head 0, the
-    first `rows` query rows against all 31200 keys, forward and backward
-    (dQ for those rows, their dK/dV contributions for every key).  Returns the
+    first `rows` query rows against all keys, forward and backward (dQ for
+    those rows, their dK/dV contributions for every key).  Returns the
     nominal TFLOP/s of that sub-problem.  With `topk`, block-sparse: the
     oracle's own selection of head 0 (inside the timed sample), counted on
     the selected keys.  With `causal`: the first `rows` tokens of head 0,
     which attend only to each other, counted on the unmasked pairs."""
     import oracle
-    w = W.get(WORKLOAD)
     q = W.head_bits(w, "q", 0, 0)[:rows]
     k = W.head_bits(w, "k", 0, 0)
     v = W.head_bits(w, "v", 0, 0)
@@ -455,56 +552,56 @@ def cpu_baseline_sample(rows: int, topk=None, causal=False):
     sel = None
     if topk is not None:
         sel = oracle.vsa_select(W.head_bits(w, "q", 0, 0), k, topk, tile=T)[0][: -(-rows // T)]
-    hd = oracle.Head(q, k, v, w.sm_scale, oracle.QUANT_ALL | (oracle.CAUSAL if causal else 0), do, sel=sel, tile=T)
+    hd = oracle.Head(q, k, v, w.sm_scale, flags | (oracle.CAUSAL if causal else 0), do, sel=sel, tile=T)
     hd.stats()
     hd.backward()
     dt = time.perf_counter() - t0
-    pairs = float(rows * w.Lk)
+    nk = k.shape[0]
+    pairs = float(rows * nk)
     if causal:
         pairs = rows * (rows + 1) / 2.0
     if sel is not None:
-        keys = np.minimum(T, w.Lk - T * np.arange(sel.shape[1]))
+        keys = np.minimum(T, nk - T * np.arange(sel.shape[1]))
         rws = np.minimum(T, rows - T * np.arange(sel.shape[0]))
         pairs = float(rws @ sel.astype(np.float64) @ keys)
     flops = 3.5 * 4.0 * pairs * w.D
     what = "block-sparse, selected keys only, " if sel is not None else ("causal, " if causal else "")
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": "head 0, query rows [0,%d) x %s keys, %sfwd+bwd (float64 C oracle)" % (
-                rows, ("the first %d" % rows) if causal else ("all %d" % w.Lk), what)}
+            "sample": "%s head 0, query rows [0,%d) x %s keys, %sfwd+bwd (float64 C oracle)" % (
+                w.name, rows, ("the first %d" % rows) if causal else ("all %d" % nk), what)}
 
 
 def reference_arm(args):
     """The oracle as the reference arm, on the same leg as the GPU arm (dense,
-    --sparsity or --causal): each step is one bounded sample (see
-    cpu_baseline_sample), timed on the host cores."""
+    --sparsity or --causal, the same workload and flags): each step is one
+    bounded sample (see cpu_baseline_sample), timed on the host cores."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     import oracle
-    w = W.get(WORKLOAD)
+    w = W.get(args.workload)
     sparse = args.sparsity is not None
     causal = bool(args.causal)
     topk = W.topk_tiles(-(-w.Lk // W.SPARSE_TILE), args.sparsity) if sparse else None
     # the causal sample's cost grows with the square of its prefix
-    rows = int(ORACLE_SAMPLE_ROWS * 2.5) if causal else ORACLE_SAMPLE_ROWS
+    rows = sample_rows(w, int(ORACLE_SAMPLE_ROWS * 2.5) if causal else ORACLE_SAMPLE_ROWS)
     for _ in range(max(0, min(args.warmup, 1))):
-        cpu_baseline_sample(rows=64, topk=topk, causal=causal)
-    recs = [cpu_baseline_sample(rows=rows, topk=topk, causal=causal) for _ in range(args.steps)]
+        cpu_baseline_sample(w, args.flags, rows=min(64, rows), topk=topk, causal=causal)
+    recs = [cpu_baseline_sample(w, args.flags, rows=rows, topk=topk, causal=causal) for _ in range(args.steps)]
     seconds = sum(r["seconds"] for r in recs)
     # every step is the same sample: value = its flops over the mean time
     value = sum(r["value"] * r["seconds"] for r in recs) / seconds
-    metric = SPARSE_METRIC % args.sparsity if sparse else (CAUSAL_METRIC if causal else METRIC)
-    config = {"workload": ("vsa_" if sparse else ("causal_" if causal else "")) + WORKLOAD, "B": w.B, "H": w.H,
-              "Lq": w.Lq, "Lk": w.Lk, "D": w.D, "quantizers": "q,k,v,p", "sample_rows": rows}
+    config = {"workload": workload_name(args, w), "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
+              "quantizers": flag_names(args.flags), "sample_rows": rows}
     if sparse:
         config.update(sparsity=args.sparsity, tile=W.SPARSE_TILE)
     out = {
         "impl": "reference",
-        "metric": metric, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "metric": metric_name(args, w), "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * seconds / len(recs), 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded N(0,1) bf16)",
+        "data": "synthetic (seeded N(0,1) float32 from numpy PCG64, rounded to bf16; %s)" % w.recipe,
         "config": config,
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": recs[0]["sample"] + ", one per step"},
@@ -519,13 +616,21 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=[x.name for x in W.WORKLOADS],
+                    help="seeded workload to time (default: the pages' H6 L31200 shape)")
+    ap.add_argument("--flags", type=int, default=15,
+                    help="quantizers on (bits q=1, k=2, v=4, p=8; default 15, all four)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (for short profiling runs; the line then has no e2e)")
     ap.add_argument("--sparsity", type=float, default=None,
                     help="time the block-sparse (VSA) step with this key-tile sparsity instead")
     ap.add_argument("--causal", action="store_true", help="time the causal step instead")
     args = ap.parse_args()
     if args.causal and args.sparsity is not None:
         ap.error("--causal and --sparsity are separate legs")
+    if not 0 <= args.flags <= 15:
+        ap.error("--flags takes the quantizer bits 0..15")
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
     if args.impl == "reference":

@@ -63,3 +63,28 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
     with bench.ClockSampler(0) as c:
         pass
     assert c.summary()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_default_metric_and_workload_names():
+    import argparse
+    a = argparse.Namespace(sparsity=None, causal=False, flags=15, workload="wan_6h_31200")
+    w = W.get("wan_6h_31200")
+    assert bench.metric_name(a, w) == bench.METRIC
+    assert bench.workload_name(a, w) == "wan_6h_31200"
+    a.flags = 7
+    assert bench.workload_name(a, w) == "wan_6h_31200_flags7"
+    assert bench.flag_names(7) == "q,k,v" and bench.flag_names(0) == "none"
+    a.causal = True
+    assert bench.metric_name(a, w).startswith("Causal") and bench.workload_name(a, w) == "causal_wan_6h_31200_flags7"
+
+
+def test_dtype_weighted_peak():
+    # four units, one on a pipe four times faster: floor 3 + 1/4 unit-times
+    assert abs(bench.dtype_weighted_peak(1000.0, 4, 1) - 1000.0 * 4 / 3.25) < 1e-9
+    assert bench.dtype_weighted_peak(1000.0, 2, 0) == 1000.0
+
+
+def test_oracle_sample_rows_scale_with_key_length():
+    assert bench.sample_rows(W.get("wan_6h_31200"), 6144) == 6144
+    assert bench.sample_rows(W.get("large_40h_75600"), 6144) == int(6144 * 31200 / 75600)
+    assert bench.sample_rows(W.get("tiny"), 6144) == 256  # capped at Lq
