@@ -64,7 +64,7 @@ METRIC = "Attn-QAT fwd+bwd ms & TFLOP/s at H6 L31200 D128; % of B200 BF16 peak"
 SPARSE_METRIC = ("Block-sparse (VSA) Attn-QAT fwd+bwd ms & TFLOP/s on the selected tiles at %s, "
                  "sparsity %g")
 CAUSAL_METRIC = "Causal Attn-QAT fwd+bwd ms & TFLOP/s on the unmasked pairs at %s"
-OTHER_METRIC = "Attn-QAT fwd+bwd ms & TFLOP/s at %s; % of B200 BF16 peak"
+OTHER_METRIC = "Attn-QAT fwd+bwd ms & TFLOP/s at {}; % of B200 BF16 peak"
 FLAG_NAMES = ((1, "q"), (2, "k"), (4, "v"), (8, "p"))
 # nominal dense tensor rates of B200 per input type, relative to bf16/fp16
 # (2.25 PFLOP/s bf16, 9 PFLOP/s fp4): the dK/dV kernel's S unit runs on the
@@ -227,7 +227,7 @@ def metric_name(args, w):
         return CAUSAL_METRIC % shape_name(w)
     if w.name == WORKLOAD and args.flags == 15:
         return METRIC
-    return OTHER_METRIC % shape_name(w)
+    return OTHER_METRIC.format(shape_name(w))
 
 
 def workload_name(args, w):

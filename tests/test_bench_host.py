@@ -88,3 +88,16 @@ def test_oracle_sample_rows_scale_with_key_length():
     assert bench.sample_rows(W.get("wan_6h_31200"), 6144) == 6144
     assert bench.sample_rows(W.get("large_40h_75600"), 6144) == int(6144 * 31200 / 75600)
     assert bench.sample_rows(W.get("tiny"), 6144) == 256  # capped at Lq
+
+
+def test_metric_names_of_every_leg_and_workload():
+    import argparse
+    for w in W.WORKLOADS:
+        for flags in (15, 7, 0):
+            for sparsity, causal in ((None, False), (0.9, False), (None, True)):
+                a = argparse.Namespace(sparsity=sparsity, causal=causal, flags=flags, workload=w.name)
+                name = bench.metric_name(a, w)
+                assert "B%d H%d L%d" % (w.B, w.H, w.Lq) in name or name == bench.METRIC
+                assert bench.workload_name(a, w).endswith(w.name if flags == 15 else "%s_flags%d" % (w.name, flags))
+    a = argparse.Namespace(sparsity=None, causal=False, flags=15, workload="tiny")
+    assert bench.metric_name(a, W.get("tiny")) == "Attn-QAT fwd+bwd ms & TFLOP/s at B1 H2 L256 D64; % of B200 BF16 peak"
