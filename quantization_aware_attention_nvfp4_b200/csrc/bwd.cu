@@ -84,7 +84,7 @@ struct BwdBars {
 
 // a_users / b_users: MMA-issuing threads that commit to aempty / bempty (a
 // ring slot is free once every MMA reading it has completed).
-__device__ __forceinline__ void init_bwd_bars(BwdBars *b, int a_users, int b_users) {
+__device__ __forceinline__ void init_bwd_bars(BwdBars *b, int a_users, int b_users, int row_warps = kSoftWarps) {
   mbar_init(&b->kvfull, 1);
   for (int s = 0; s < 2; ++s) {
     mbar_init(&b->afull[s], 1);
@@ -95,8 +95,8 @@ __device__ __forceinline__ void init_bwd_bars(BwdBars *b, int a_users, int b_use
     mbar_init(&b->cempty[s], 1);
   }
   mbar_init(&b->sfull, 1);
-  mbar_init(&b->sempty, kSoftWarps);
-  mbar_init(&b->xfull, kSoftWarps);
+  mbar_init(&b->sempty, row_warps);
+  mbar_init(&b->xfull, row_warps);
   mbar_init(&b->xempty, 1);
   mbar_init(&b->done, 1);
   mbar_init(&b->adone, 1);
@@ -144,7 +144,15 @@ __device__ __forceinline__ void load_cols64(uint32_t taddr, uint32_t (&v)[64]) {
   tmem_ld_wait();
 }
 
-// dK/dV kernel, first half of a query tile for one thread (one query row, 64
+// NC (32 or 64) columns of one 32-bit TMEM tile into registers.
+template <int NC>
+__device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&v)[NC]) {
+#pragma unroll
+  for (int c = 0; c < NC / 32; ++c) tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+  tmem_ld_wait();
+}
+
+// dK/dV kernel, first half of a query tile for one thread (one query row, NC
 // key columns from col0): P~ = exp2(S cl + nml) -- rebuilt exactly as the
 // forward builds it (same bits, same blocks of 16 keys) -- and the dV
 // operand row in fp16: fq(P~)/l * 2^14 (r times the per-block factor
@@ -152,12 +160,12 @@ __device__ __forceinline__ void load_cols64(uint32_t taddr, uint32_t (&v)[64]) {
 // bits and in fp16's normal range for every value above 2^-28 (all nonzero
 // fq(P~)/l while Lk <= 2^17).  P~ stays in float32 for dS.  Rows past Lq come
 // in with nml = -inf, so their P~ is 0 without a per-element test.
-template <int QP, bool MASKED>
-__device__ __forceinline__ void dkdv_probs(const uint32_t (&sv)[64], int col0, int valid_k, float cl, float nml,
-                                           float vf, float (&p)[64], uint32_t (&pw)[32]) {
+template <int QP, bool MASKED, int NC>
+__device__ __forceinline__ void dkdv_probs(const uint32_t (&sv)[NC], int col0, int valid_k, float cl, float nml,
+                                           float vf, float (&p)[NC], uint32_t (&pw)[NC / 2]) {
   const float2 cl2 = make_float2(cl, cl), nml2 = make_float2(nml, nml);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NC / 2; ++i) {
     const float2 x = fma2(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), cl2, nml2);
     const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
     p[2 * i] = (!MASKED || col0 + 2 * i < valid_k) ? e0 : 0.0f;
@@ -165,7 +173,7 @@ __device__ __forceinline__ void dkdv_probs(const uint32_t (&sv)[64], int col0, i
   }
   if (QP) {
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
+    for (int b = 0; b < NC / 16; ++b) {
       uint32_t rr[8];
       const uint32_t s2 = f16x2_broadcast(fq16_probs(p + 16 * b, rr) * vf);
 #pragma unroll
@@ -174,7 +182,7 @@ __device__ __forceinline__ void dkdv_probs(const uint32_t (&sv)[64], int col0, i
   } else {
     const float2 vf2 = make_float2(vf, vf);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < NC / 2; ++i) {
       const float2 x = mul2(make_float2(p[2 * i], p[2 * i + 1]), vf2);
       pw[i] = pack_f16x2(x.x, x.y);
     }
@@ -186,22 +194,32 @@ __device__ __forceinline__ void dkdv_probs(const uint32_t (&sv)[64], int col0, i
 // dP' = dP 2^e (the fp16 copies of dO and V carry powers of two), so
 // dS * dsc = P~/l * (dP' 2^-e - Delta) * dsc = P~ * fma(dP', a1, b1) with
 // a1 = 2^-e dsc / l, b1 = -Delta dsc / l.
-__device__ __forceinline__ void dkdv_ds(const float (&p)[64], const uint32_t (&dv)[64], float a1, float b1,
-                                        uint32_t (&dsw)[32]) {
+template <int NC>
+__device__ __forceinline__ void dkdv_ds(const float (&p)[NC], const uint32_t (&dv)[NC], float a1, float b1,
+                                        uint32_t (&dsw)[NC / 2]) {
   const float2 a12 = make_float2(a1, a1), b12 = make_float2(b1, b1);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NC / 2; ++i) {
     const float2 g = fma2(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])), a12, b12);
     const float2 d = mul2(make_float2(p[2 * i], p[2 * i + 1]), g);
     dsw[i] = pack_f16x2(d.x, d.y);
   }
 }
 
+// Row warps per TMEM lane quarter of the dK/dV kernel, and its CTA size
+// (producer, MMA issuer, 4 * RG row warps; 12 warps for RG = 2, the two
+// spare warps idle).  RG = 4 (576 threads, 32 columns per thread) measured
+// slower at the H6 L31200 shape, 5.23 against 5.08 ms: with 18 warps one
+// scheduler holds five of them, which caps registers at 96 per thread.
+constexpr int kDkdvRG = 2;
+template <int RG>
+constexpr int dkdv_threads() { return RG == 2 ? kThreads : 32 * (2 + 4 * RG); }
+
 // SP: 0 dense; 1 block-sparse (walks a.q_list); 2 causal (lower-triangle
 // lists, diagonal masked).  Separate instantiations, so the dense kernel
 // carries none of the list handling.
-template <int D, int QP, int FP4S, int SP>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int QP, int FP4S, int SP, int RG>
+__global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const __grid_constant__ CUtensorMap tmQ4, const BwdArgs a) {
@@ -222,7 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = SP ? a.q_count[krow] : nq;
   auto qtile = [&](int i) -> int { return SP ? __ldg(ql + i) : i; };
 
-  if (threadIdx.x == 0) init_bwd_bars(bars, 1, 1);
+  constexpr int NC = kBN / RG;  // key columns per row-warp thread
+  if (threadIdx.x == 0) init_bwd_bars(bars, 1, 1, 4 * RG);
   if (warp == 1) {
     tmem_alloc(&bars->tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -357,9 +376,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma_commit(&bars->done);
     }
-  } else if (warp >= 2 && warp < 2 + kSoftWarps) {
+  } else if (warp >= 2 && warp < 2 + 4 * RG) {
     const RowRole rr(warp, lane);
-    const int col0 = rr.half * 64;
+    const int col0 = rr.half * NC;
     const int valid_k = a.Lk - kt * kBN;  // >= 128 for full key tiles
     // causal: the first query tile visited is the diagonal, where query row r
     // keeps keys 0..r (a partial key tile only ever meets its diagonal)
@@ -389,14 +408,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m = m_n, lse = lse_n, delta = delta_n;
       load_stats(i + 1, m_n, lse_n, delta_n);
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
-      float p[64];
-      uint32_t pw[32], dsw[32];
+      float p[NC];
+      uint32_t pw[NC / 2], dsw[NC / 2];
       {
         // S_i: read, release the buffer for dP_i, build P~ and the dV operand
-        uint32_t sv[64];
+        uint32_t sv[NC];
         if (!mbar_wait(&bars->sfull, (2 * i) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        load_cols64(tbuf, sv);
+        load_cols<NC>(tbuf, sv);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->sempty);
@@ -405,53 +424,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float nml = vq ? -(m * kLog2e) : -INFINITY;
         const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
         if (masked)
-          dkdv_probs<QP, true>(sv, col0, vk, cl, nml, vf, p, pw);
+          dkdv_probs<QP, true, NC>(sv, col0, vk, cl, nml, vf, p, pw);
         else
-          dkdv_probs<QP, false>(sv, col0, vk, cl, nml, vf, p, pw);
+          dkdv_probs<QP, false, NC>(sv, col0, vk, cl, nml, vf, p, pw);
       }
       // X = (fq(P~)/l)^T once dK_{i-1} has read the previous dS^T
       if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
-      store_row_half(xaddr, rr.row, rr.half, pw);
+      store_row_cols<NC>(xaddr, rr.row, col0, pw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
       {
         // dP_i: read, release the buffer for S_{i+1}, build dS
-        uint32_t dv[64];
+        uint32_t dv[NC];
         if (!mbar_wait(&bars->sfull, (2 * i + 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        load_cols64(tbuf, dv);
+        load_cols<NC>(tbuf, dv);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->sempty);
-        dkdv_ds(p, dv, inv_l * dsc / dos, -delta * inv_l * dsc, dsw);
+        dkdv_ds<NC>(p, dv, inv_l * dsc / dos, -delta * inv_l * dsc, dsw);
       }
       // X = dS^T once dV_i has read the P^T
       if (!mbar_wait(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
-      store_row_half(xaddr, rr.row, rr.half, dsw);
+      store_row_cols<NC>(xaddr, rr.row, col0, dsw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xfull);
     }
     if (ok && mbar_wait(&bars->done, 0, abort)) {
       tc_fence_after();
-      // TMEM lanes of dV/dK are keys; each thread stores D/2 columns of its key row
+      // TMEM lanes of dV/dK are keys; each thread stores D/RG columns of its key row
       const int kg = kt * kBN + static_cast<int>(rr.row);
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lk + kg) * D;
       const float kscale = a.sm_scale / (dsc * sq);  // exact: power-of-two divisors
       const float vscale = (1.0f / 16384.0f) / do_scale(a.stats);  // exact: powers of two
+      constexpr int DC = D / RG;            // output columns per thread
+      constexpr int W = DC < 32 ? DC : 32;  // columns per TMEM load
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        const int col = rr.half * (D / 2) + c * 32;
+      for (int c = 0; c < DC / W; ++c) {
+        const int col = rr.half * DC + c * W;
         uint32_t r[32], s[32];
-        tmem_ld32(tmem + rr.lane_addr + L::kTmemDV + col, r);
-        tmem_ld32(tmem + rr.lane_addr + L::kTmemDK + col, s);
+        if (W == 32) {
+          tmem_ld32(tmem + rr.lane_addr + L::kTmemDV + col, r);
+          tmem_ld32(tmem + rr.lane_addr + L::kTmemDK + col, s);
+        } else {
+          tmem_ld16(tmem + rr.lane_addr + L::kTmemDV + col, *reinterpret_cast<uint32_t(*)[16]>(r));
+          tmem_ld16(tmem + rr.lane_addr + L::kTmemDK + col, *reinterpret_cast<uint32_t(*)[16]>(s));
+        }
         tmem_ld_wait();
         if (kg < a.Lk) {
           uint4 *dv = reinterpret_cast<uint4 *>(a.dv + rowoff + col);
           uint4 *dk = reinterpret_cast<uint4 *>(a.dk + rowoff + col);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < W / 8; ++i) {
             uint32_t w[4], x[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -792,10 +818,10 @@ static cudaError_t launch_dkdv_sp(const CUtensorMap &tq, const CUtensorMap &tk, 
   static_assert(L::kDynSmem <= 232448, "dK/dV shared memory over the 227 KB limit");
   static_assert(sizeof(BwdBars) <= L::kBarBytes, "dK/dV barrier block larger than its reservation");
   static_assert(L::kTmemSFB + L::kSFCols <= L::kTmemCols, "dK/dV TMEM over 512 columns");
-  auto kern = attn_bwd_dkdv_kernel<D, QP, FP4S, SP>;
+  auto kern = attn_bwd_dkdv_kernel<D, QP, FP4S, SP, kDkdvRG>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), L::kDynSmem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(a.nk_tiles, BH), kThreads, L::kDynSmem, stream>>>(tq, tk, tv, tdo, tq4, a);
+  kern<<<dim3(a.nk_tiles, BH), dkdv_threads<kDkdvRG>(), L::kDynSmem, stream>>>(tq, tk, tv, tdo, tq4, a);
   return cudaGetLastError();
 }
 

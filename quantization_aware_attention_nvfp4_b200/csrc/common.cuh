@@ -163,9 +163,23 @@ __device__ __forceinline__ void store_row_half(uint32_t base, uint32_t row, int 
   }
 }
 
-// Role of a row warp (warps 2 .. 2+kSoftWarps-1): the TMEM lane quarter it
-// may access (warp id mod 4), its row in the 128-row tile and which 64-column
-// half of a 128-column tile it owns.
+// Writes NC 16-bit values (NC/2 packed words) as columns [col0, col0 + NC)
+// of row `row` of a 128 x 128 swizzled tile at `base` (NC = 32 or 64, col0 a
+// multiple of NC: within one 64-column chunk).
+template <int NC>
+__device__ __forceinline__ void store_row_cols(uint32_t base, uint32_t row, int col0, const uint32_t *w) {
+#pragma unroll
+  for (int u = 0; u < NC / 8; ++u) {
+    const uint32_t addr = base + static_cast<uint32_t>(col0 >> 6) * kChunkBytes +
+                          sw128_offset(row, static_cast<uint32_t>((col0 & 63) >> 3) + u);
+    st_shared_v4(addr, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+  }
+}
+
+// Role of a row warp (warps 2 .. 2 + 4 G - 1 with G row warps per TMEM lane
+// quarter): the lane quarter it may access (warp id mod 4), its row in the
+// 128-row tile and which of the G column groups of a 128-column tile it owns
+// (`half`: 0 or 1 when G = 2).
 struct RowRole {
   int wq;           // lane quarter
   uint32_t row;     // 0..127
