@@ -21,7 +21,8 @@ events on the launching stream, and multi-GPU runs report the max over ranks.
 wan_6h_31200, scaled_heads_16384, large_40h_75600) and --flags another set of
 quantizers (bits q=1, k=2, v=4, p=8; default all four).
 
---sparsity S times the block-sparse (VSA fine attention) step instead:
+--sparsity S times the block-sparse (VSA fine attention) step instead (with
+--tile 64 the tile-64 profile: 64-token query and key blocks):
 attnqat_vsa_select (the top max(1, min(ceil((1-S)*nk), nk)) of the nk key
 tiles per 128-query tile by coarse tile-mean scores; the pages' VSA checkpoint
 uses S = 0.9) + attnqat_sparse_fwd + attnqat_sparse_bwd on the same shape,
@@ -205,9 +206,9 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- GPU arm --
 
-def selected_pairs(w, mask):
-    """Sum over (b, h) of the (query row, key) pairs the tile mask selects."""
-    T = W.SPARSE_TILE
+def selected_pairs(w, mask, T=W.SPARSE_TILE):
+    """Sum over (b, h) of the (query row, key) pairs the T-token tile mask
+    selects."""
     rows = np.minimum(T, w.Lq - T * np.arange(mask.shape[2]))
     keys = np.minimum(T, w.Lk - T * np.arange(mask.shape[3]))
     return float(np.einsum("bhij,i,j->", mask.astype(np.float64), rows, keys))
@@ -222,7 +223,8 @@ def dtype_weighted_peak(peak, n_units, fp4_units, ratio=NVFP4_RATE_RATIO):
 
 def metric_name(args, w):
     if args.sparsity is not None:
-        return SPARSE_METRIC % (shape_name(w), args.sparsity)
+        return SPARSE_METRIC % (shape_name(w) + ("" if args.tile == 128 else ", %d-token tiles" % args.tile),
+                                args.sparsity)
     if args.causal:
         return CAUSAL_METRIC % shape_name(w)
     if w.name == WORKLOAD and args.flags == 15:
@@ -233,7 +235,7 @@ def metric_name(args, w):
 def workload_name(args, w):
     name = w.name if args.flags == 15 else "%s_flags%d" % (w.name, args.flags)
     if args.sparsity is not None:
-        return "vsa_" + name
+        return ("vsa_" if args.tile == 128 else "vsa%d_" % args.tile) + name
     return ("causal_" if args.causal else "") + name
 
 
@@ -258,7 +260,8 @@ def gpu_arm(args):
         pairs = float(w.B * w.H) * w.Lq * (w.Lq + 1) / 2.0
         fwd_f = 4.0 * pairs * w.D
         flops = dict(fwd=fwd_f, bwd=2.5 * fwd_f, total=3.5 * fwd_f)
-    nq, nk = -(-w.Lq // W.SPARSE_TILE), -(-w.Lk // W.SPARSE_TILE)
+    T = args.tile
+    nq, nk = -(-w.Lq // T), -(-w.Lk // T)
     topk = W.topk_tiles(nk, args.sparsity) if sparse else nk
 
     # seeded inputs (host), moved to the device once; the timed region starts
@@ -270,17 +273,18 @@ def gpu_arm(args):
     flags = args.flags | (A.CAUSAL if causal else 0)
     if sparse:
         tm = torch.empty((w.B, w.H, nq, nk), dtype=torch.uint8, device=dev)
-        sel_ws = torch.empty(A.load().attnqat_vsa_select_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D),
+        sel_ws = torch.empty(A.load().attnqat_vsa_select_tiles_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, T),
                              dtype=torch.uint8, device=dev)
         ws_bytes = A.attnqat_sparse_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags)
 
         def fwd(qq, kk, vv, out, stream=None):
             # the selection belongs to the forward: coarse scores, top-k tiles
-            A.attnqat_vsa_select(qq, kk, topk, out=tm, ws=sel_ws, stream=stream)
-            return A.attnqat_sparse_fwd(qq, kk, vv, tm, sm_scale=c, flags=flags, ws=ws, out=out, stream=stream)
+            A.attnqat_vsa_select(qq, kk, topk, out=tm, ws=sel_ws, stream=stream, tile=T)
+            return A.attnqat_sparse_fwd(qq, kk, vv, tm, sm_scale=c, flags=flags, ws=ws, out=out, stream=stream,
+                                        tile=T)
 
         def bwd(qq, kk, vv, ll, mm, dd, out, stream=None):
-            return A.attnqat_sparse_bwd(qq, kk, vv, ll, mm, dd, ws, tm, sm_scale=c, flags=flags, out=out,
+            return A.attnqat_sparse_bwd(qq, kk, vv, ll, mm, dd, ws, tm, sm_scale=c, flags=flags, out=out, tile=T,
                                         stream=stream)
     else:
         ws_bytes = A.attnqat_workspace_size(w.B, w.H, w.Lq, w.Lk, w.D, flags)
@@ -310,7 +314,7 @@ def gpu_arm(args):
     if sparse:
         # the selection depends only on the inputs: count its pairs once
         mask_np = tm.cpu().numpy()
-        pairs = selected_pairs(w, mask_np)
+        pairs = selected_pairs(w, mask_np, T)
         fwd_f = 4.0 * pairs * w.D
         flops = dict(fwd=fwd_f, bwd=2.5 * fwd_f, total=3.5 * fwd_f)
 
@@ -382,7 +386,7 @@ def gpu_arm(args):
               "parallelism": "replicas x%d (heads independent, no collective)" % world,
               "l2": "flushed between steps (256 MiB write); each step timed with CUDA events"}
     if sparse:
-        config.update(sparsity=args.sparsity, tile=W.SPARSE_TILE,
+        config.update(sparsity=args.sparsity, tile=T,
                       key_tiles_per_query_tile=int(mask_np.sum(-1).max()),
                       selected_fraction=round(pairs / (w.B * w.H * w.Lq * w.Lk), 5),
                       selection="attnqat_vsa_select in the timed forward (tile means, top-%d coarse scores)" % topk)
@@ -433,7 +437,7 @@ def gpu_arm(args):
         if world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline_sample(
                 w, args.flags, rows=sample_rows(w, CAUSAL_SAMPLE_ROWS if causal else BASELINE_SAMPLE_ROWS),
-                topk=topk if sparse else None, causal=causal)
+                topk=topk if sparse else None, causal=causal, T=T)
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
@@ -532,7 +536,7 @@ def load_traffic(kernel):
 
 # -------------------------------------------------------------- CPU oracle --
 
-def cpu_baseline_sample(w, flags, rows: int, topk=None, causal=False):
+def cpu_baseline_sample(w, flags, rows: int, topk=None, causal=False, T=W.SPARSE_TILE):
     """The float64 oracle on a bounded sample of the workload: head 0, the
     first `rows` query rows against all keys, forward and backward (dQ for
     those rows, their dK/dV contributions for every key).  Returns the
@@ -547,7 +551,6 @@ def cpu_baseline_sample(w, flags, rows: int, topk=None, causal=False):
     if causal:
         k, v = k[:rows], v[:rows]
     do = W.head_bits(w, "do", 0, 0)[:rows]
-    T = W.SPARSE_TILE
     t0 = time.perf_counter()
     sel = None
     if topk is not None:
@@ -583,19 +586,20 @@ def reference_arm(args):
     w = W.get(args.workload)
     sparse = args.sparsity is not None
     causal = bool(args.causal)
-    topk = W.topk_tiles(-(-w.Lk // W.SPARSE_TILE), args.sparsity) if sparse else None
+    topk = W.topk_tiles(-(-w.Lk // args.tile), args.sparsity) if sparse else None
     # the causal sample's cost grows with the square of its prefix
     rows = sample_rows(w, int(ORACLE_SAMPLE_ROWS * 2.5) if causal else ORACLE_SAMPLE_ROWS)
     for _ in range(max(0, min(args.warmup, 1))):
-        cpu_baseline_sample(w, args.flags, rows=min(64, rows), topk=topk, causal=causal)
-    recs = [cpu_baseline_sample(w, args.flags, rows=rows, topk=topk, causal=causal) for _ in range(args.steps)]
+        cpu_baseline_sample(w, args.flags, rows=min(64, rows), topk=topk, causal=causal, T=args.tile)
+    recs = [cpu_baseline_sample(w, args.flags, rows=rows, topk=topk, causal=causal, T=args.tile)
+            for _ in range(args.steps)]
     seconds = sum(r["seconds"] for r in recs)
     # every step is the same sample: value = its flops over the mean time
     value = sum(r["value"] * r["seconds"] for r in recs) / seconds
     config = {"workload": workload_name(args, w), "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "D": w.D,
               "quantizers": flag_names(args.flags), "sample_rows": rows}
     if sparse:
-        config.update(sparsity=args.sparsity, tile=W.SPARSE_TILE)
+        config.update(sparsity=args.sparsity, tile=args.tile)
     out = {
         "impl": "reference",
         "metric": metric_name(args, w), "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
@@ -626,6 +630,8 @@ def main():
     ap.add_argument("--sparsity", type=float, default=None,
                     help="time the block-sparse (VSA) step with this key-tile sparsity instead")
     ap.add_argument("--causal", action="store_true", help="time the causal step instead")
+    ap.add_argument("--tile", type=int, default=128, choices=[64, 128],
+                    help="token tile of the block-sparse leg (64: the tile-64 profile)")
     args = ap.parse_args()
     if args.causal and args.sparsity is not None:
         ap.error("--causal and --sparsity are separate legs")

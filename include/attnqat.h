@@ -276,6 +276,15 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse,
  * here (EINVAL; the workspace size is 0).
  */
 #define ATTNQAT_SPARSE_TILE 128
+/* The tile-64 profile (fastvideo-kernel triton_kernels commit: the FP4
+ * sparse-attention emulator's tile-64 and tile-128 profiles; vsqa-test-1.3b
+ * metadata.json, attention.physical_block_tokens = 64): with this flag on the
+ * sparse calls, tile_mask has 64-token granularity,
+ * [B][H][ceil(Lq/64)][ceil(Lk/64)], and query block I attends exactly the
+ * keys of its selected 64-token key blocks; everything else is as for
+ * 128-token tiles (the workspace size is the same).  Not accepted by the
+ * dense calls or with ATTNQAT_CAUSAL (EINVAL). */
+#define ATTNQAT_TILE64 64u
 size_t attnqat_sparse_workspace_size(int B, int H, int Lq, int Lk, int D,
                                      uint32_t flags);
 int attnqat_sparse_fwd(const void *q, const void *k, const void *v, int B,
@@ -320,6 +329,19 @@ size_t attnqat_vsa_select_workspace_size(int B, int H, int Lq, int Lk, int D);
 int attnqat_vsa_select(const void *q, const void *k, int B, int H, int Lq,
                        int Lk, int D, int topk, uint8_t *tile_mask, void *ws,
                        size_t ws_bytes, void *stream);
+
+/* The same selection over `tile`-token tiles, tile = 128 (as above) or 64
+ * (the tile-64 profile, whose mask feeds the sparse calls with
+ * ATTNQAT_TILE64): tile_mask is [B][H][ceil(Lq/tile)][ceil(Lk/tile)] and topk
+ * counts tile-token key tiles.  The workspace (tile means and scores) is
+ * attnqat_vsa_select_tiles_workspace_size() bytes (0 for a tile other than
+ * 64 or 128).  Errors as attnqat_vsa_select, plus EINVAL for another tile. */
+size_t attnqat_vsa_select_tiles_workspace_size(int B, int H, int Lq, int Lk,
+                                               int D, int tile);
+int attnqat_vsa_select_tiles(const void *q, const void *k, int B, int H,
+                             int Lq, int Lk, int D, int tile, int topk,
+                             uint8_t *tile_mask, void *ws, size_t ws_bytes,
+                             void *stream);
 
 /*
  * attnqat_fwd_noalloc -- attnqat_fwd for callers that cannot allocate.

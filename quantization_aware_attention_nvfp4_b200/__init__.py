@@ -22,6 +22,8 @@ Entry points (same names as the C ABI):
   attends a 128-key tile.
 * ``attnqat_vsa_select(q, k, topk)`` -- that mask from the coarse scores of
   the tiles' means: the ``topk`` best key tiles per query tile.
+* ``tile=64`` on these three selects the tile-64 profile: masks of 64-token
+  blocks [B, H, ceil(Lq/64), ceil(Lk/64)].
 
 ``sm_scale=None`` means 1/sqrt(D), chosen here and passed explicitly; the
 library itself never substitutes a default (FastVideo PR #1457 review, F1).
@@ -40,7 +42,8 @@ QUANT_K = 2
 QUANT_V = 4
 QUANT_P = 8
 QUANT_ALL = 15
-CAUSAL = 32  # causal masking (attnqat_fwd / attnqat_bwd; Lq == Lk, every quantizer on)
+CAUSAL = 32  # causal masking (attnqat_fwd / attnqat_bwd; Lq == Lk)
+TILE64 = 64  # 64-token tile masks on the sparse calls (set by their tile=64 argument)
 
 OK = 0
 EINVAL = -1
@@ -99,6 +102,10 @@ def load(build_if_needed: bool = True):
             lib.attnqat_vsa_select_workspace_size.argtypes = [I, I, I, I, I]
             lib.attnqat_vsa_select.restype = I
             lib.attnqat_vsa_select.argtypes = [P, P, I, I, I, I, I, I, P, P, SZ, P]
+            lib.attnqat_vsa_select_tiles_workspace_size.restype = SZ
+            lib.attnqat_vsa_select_tiles_workspace_size.argtypes = [I, I, I, I, I, I]
+            lib.attnqat_vsa_select_tiles.restype = I
+            lib.attnqat_vsa_select_tiles.argtypes = [P, P, I, I, I, I, I, I, I, P, P, SZ, P]
             lib.attnqat_sparse_workspace_size.restype = SZ
             lib.attnqat_sparse_workspace_size.argtypes = [I, I, I, I, I, U32]
             lib.attnqat_sparse_fwd.restype = I
@@ -273,22 +280,30 @@ def attnqat_sparse_workspace_size(B, H, Lq, Lk, D, flags=QUANT_ALL) -> int:
     return int(load().attnqat_sparse_workspace_size(B, H, Lq, Lk, D, flags))
 
 
-def _tile_mask(tile_mask, B, H, Lq, Lk, device):
+def _check_tile(tile):
+    if tile not in (64, 128):
+        raise ValueError("tile must be 64 or 128")
+    return TILE64 if tile == 64 else 0
+
+
+def _tile_mask(tile_mask, B, H, Lq, Lk, device, tile=SPARSE_TILE):
     torch = _torch()
-    want = (B, H, -(-Lq // SPARSE_TILE), -(-Lk // SPARSE_TILE))
+    want = (B, H, -(-Lq // tile), -(-Lk // tile))
     if not isinstance(tile_mask, torch.Tensor) or tile_mask.dtype != torch.uint8 or \
             tile_mask.device != device or tuple(tile_mask.shape) != want or not tile_mask.is_contiguous():
         raise ValueError("tile_mask must be a contiguous uint8 tensor %s on %s" % (want, device))
     return ctypes.c_void_p(tile_mask.data_ptr())
 
 
-def attnqat_vsa_select(q, k, topk, out=None, ws=None, stream=None):
+def attnqat_vsa_select(q, k, topk, out=None, ws=None, stream=None, tile=SPARSE_TILE):
     """Key tiles per query tile for the block-sparse attention: the ``topk``
     key tiles whose mean row scores highest against the query tile's mean row
-    (ties to the lower tile).  ``q`` [B, H, Lq, D], ``k`` [B, H, Lk, D] bf16
-    CUDA tensors.  Returns the uint8 tile mask [B, H, ceil(Lq/128),
-    ceil(Lk/128)] (``out`` if given)."""
+    (ties to the lower tile), over ``tile``-token tiles (128, or 64 for the
+    tile-64 profile).  ``q`` [B, H, Lq, D], ``k`` [B, H, Lk, D] bf16 CUDA
+    tensors.  Returns the uint8 tile mask [B, H, ceil(Lq/tile),
+    ceil(Lk/tile)] (``out`` if given)."""
     torch = _torch()
+    _check_tile(tile)
     for n, t in (("q", q), ("k", k)):
         _require_bf16_cuda(n, t, 4)
         if not t.is_contiguous():
@@ -297,31 +312,33 @@ def attnqat_vsa_select(q, k, topk, out=None, ws=None, stream=None):
     Lk = k.shape[2]
     if k.shape[0] != B or k.shape[1] != H or k.shape[3] != D:
         raise ValueError("k must be [B, H, Lk, D] matching q [B, H, Lq, D]")
-    need = int(load().attnqat_vsa_select_workspace_size(B, H, Lq, Lk, D))
+    need = int(load().attnqat_vsa_select_tiles_workspace_size(B, H, Lq, Lk, D, tile))
     if need == 0:
-        _check(EINVAL, "attnqat_vsa_select_workspace_size")
+        _check(EINVAL, "attnqat_vsa_select_tiles_workspace_size")
     if ws is None:
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     if out is None:
-        out = torch.empty((B, H, -(-Lq // SPARSE_TILE), -(-Lk // SPARSE_TILE)), dtype=torch.uint8,
-                          device=q.device)
+        out = torch.empty((B, H, -(-Lq // tile), -(-Lk // tile)), dtype=torch.uint8, device=q.device)
     else:
-        _tile_mask(out, B, H, Lq, Lk, q.device)
-    st = load().attnqat_vsa_select(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), B, H, Lq, Lk, D,
-                                   int(topk), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
-                                   ws.numel() * ws.element_size(), _stream_ptr(stream))
-    _check(st, "attnqat_vsa_select")
+        _tile_mask(out, B, H, Lq, Lk, q.device, tile)
+    st = load().attnqat_vsa_select_tiles(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), B, H, Lq, Lk,
+                                         D, tile, int(topk), ctypes.c_void_p(out.data_ptr()),
+                                         ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(),
+                                         _stream_ptr(stream))
+    _check(st, "attnqat_vsa_select_tiles")
     return out
 
 
-def attnqat_sparse_fwd(q, k, v, tile_mask, sm_scale=None, flags=QUANT_ALL, ws=None, out=None, stream=None):
-    """Block-sparse Attn-QAT forward (VSA fine attention): each 128-query
-    tile attends only the 128-key tiles ``tile_mask`` selects.  Returns
-    ``(o, lse, m, ws)``; pass ``ws`` and the same mask to
-    :func:`attnqat_sparse_bwd`."""
+def attnqat_sparse_fwd(q, k, v, tile_mask, sm_scale=None, flags=QUANT_ALL, ws=None, out=None, stream=None,
+                       tile=SPARSE_TILE):
+    """Block-sparse Attn-QAT forward (VSA fine attention): each ``tile``-token
+    query tile (128, or 64 for the tile-64 profile) attends only the key tiles
+    ``tile_mask`` selects.  Returns ``(o, lse, m, ws)``; pass ``ws``, the same
+    mask and the same tile to :func:`attnqat_sparse_bwd`."""
     torch = _torch()
     B, H, Lq, Lk, D = _shape(q, k, v)
-    mp = _tile_mask(tile_mask, B, H, Lq, Lk, q.device)
+    flags = (flags & ~TILE64) | _check_tile(tile)
+    mp = _tile_mask(tile_mask, B, H, Lq, Lk, q.device, tile)
     c = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
     need = attnqat_sparse_workspace_size(B, H, Lq, Lk, D, flags)
     if need == 0:
@@ -344,12 +361,13 @@ def attnqat_sparse_fwd(q, k, v, tile_mask, sm_scale=None, flags=QUANT_ALL, ws=No
 
 
 def attnqat_sparse_bwd(q, k, v, lse, m, dO, ws, tile_mask, sm_scale=None, flags=QUANT_ALL, out=None,
-                       stream=None):
+                       stream=None, tile=SPARSE_TILE):
     """Block-sparse Attn-QAT backward (straight-through) with the forward's
-    ``ws`` and ``tile_mask``.  Returns ``(dq, dk, dv)``."""
+    ``ws``, ``tile_mask`` and ``tile``.  Returns ``(dq, dk, dv)``."""
     torch = _torch()
     B, H, Lq, Lk, D = _shape(q, k, v)
-    mp = _tile_mask(tile_mask, B, H, Lq, Lk, q.device)
+    flags = (flags & ~TILE64) | _check_tile(tile)
+    mp = _tile_mask(tile_mask, B, H, Lq, Lk, q.device, tile)
     _require_bf16_cuda("dO", dO, 4)
     if dO.shape != q.shape or not dO.is_contiguous():
         raise ValueError("dO must be contiguous and shaped like q")

@@ -272,7 +272,8 @@ static int check_shape(int B, int H, int Lq, int Lk, int D, float sm_scale, uint
   const int64_t Lmax = Lq > Lk ? Lq : Lk;
   if (static_cast<int64_t>(B) * H * Lmax * 128 >= (int64_t(1) << 40)) return ATTNQAT_EINVAL;
   if (!(std::isfinite(sm_scale) && sm_scale > 0.0f)) return ATTNQAT_EINVAL;
-  if (flags & ~(ATTNQAT_QUANT_ALL | ATTNQAT_CAUSAL)) return ATTNQAT_EINVAL;
+  if (flags & ~(ATTNQAT_QUANT_ALL | ATTNQAT_CAUSAL | ATTNQAT_TILE64)) return ATTNQAT_EINVAL;
+  if ((flags & ATTNQAT_TILE64) && (flags & ATTNQAT_CAUSAL)) return ATTNQAT_EINVAL;  // a mask, or causal
   if (D != 64 && D != 128) return ATTNQAT_EUNSUPPORTED;
   return ATTNQAT_OK;
 }
@@ -460,7 +461,7 @@ int attnqat_quantize_gs(const void *x, int64_t batch, int64_t rows, int64_t cols
 }
 
 size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
-  if (check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
+  if ((flags & ATTNQAT_TILE64) || check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
   return layout(B, H, Lq, Lk, D, flags, (flags & ATTNQAT_CAUSAL) != 0).total;
 }
 
@@ -469,16 +470,22 @@ size_t attnqat_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flag
 namespace attnqat {
 
 // Builds the tile lists into the workspace: from the caller's mask
-// (block-sparse), the lower triangle (causal), or nothing (dense).
-static int plan_sparse(const uint8_t *mask, bool causal, int BH, int Lq, int Lk, uint8_t *wsb, const Workspace &w,
-                       cudaStream_t s) {
+// (block-sparse; with tile64 a 64-token mask whose quadrants ride in the list
+// entries), the lower triangle (causal), or nothing (dense).
+static int plan_sparse(const uint8_t *mask, bool causal, bool tile64, int BH, int Lq, int Lk, uint8_t *wsb,
+                       const Workspace &w, cudaStream_t s) {
   if (!mask && !causal) return ATTNQAT_OK;
   int32_t *kvl = reinterpret_cast<int32_t *>(wsb + w.kv_list), *kvc = reinterpret_cast<int32_t *>(wsb + w.kv_count);
   int32_t *ql = reinterpret_cast<int32_t *>(wsb + w.q_list), *qc = reinterpret_cast<int32_t *>(wsb + w.q_count);
+  const int nq = (Lq + kBM - 1) / kBM, nk = (Lk + kBN - 1) / kBN;
   ProfScope ps(causal ? "causal_plan" : "sparse_plan", s);
-  const cudaError_t e = causal ? launch_causal_plan(BH, (Lq + kBM - 1) / kBM, kvl, kvc, ql, qc, s)
-                               : launch_sparse_plan(mask, BH, (Lq + kBM - 1) / kBM, (Lk + kBN - 1) / kBN, kvl, kvc,
-                                                    ql, qc, s);
+  cudaError_t e;
+  if (causal)
+    e = launch_causal_plan(BH, nq, kvl, kvc, ql, qc, s);
+  else if (tile64)
+    e = launch_sparse64_plan(mask, BH, (Lq + 63) / 64, (Lk + 63) / 64, nq, nk, kvl, kvc, ql, qc, s);
+  else
+    e = launch_sparse_plan(mask, BH, nq, nk, kvl, kvc, ql, qc, s);
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
 }
 
@@ -489,7 +496,9 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
   int st = check_shape(B, H, Lq, Lk, D, sm_scale, flags);
   if (st != ATTNQAT_OK) return st;
   const bool causal = (flags & ATTNQAT_CAUSAL) != 0;
+  const bool tile64 = (flags & ATTNQAT_TILE64) != 0;
   if (causal && mask) return ATTNQAT_EINVAL;  // a tile selection and causal masking do not combine
+  if (tile64 && !mask) return ATTNQAT_EINVAL;  // 64-token tiles describe a mask
   if (!q || !k || !v || !o || !lse || !m || !ws) return ATTNQAT_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(m) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
@@ -503,7 +512,7 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
   st = prepare_operands(q, k, v, B, H, Lq, Lk, D, flags, wsb, w, s);
   if (st != ATTNQAT_OK) return st;
   const int BH = B * H;
-  st = plan_sparse(mask, causal, BH, Lq, Lk, wsb, w, s);
+  st = plan_sparse(mask, causal, tile64, BH, Lq, Lk, wsb, w, s);
   if (st != ATTNQAT_OK) return st;
   const bool fp4 = fp4s(flags);
   const bool pv4 = pv_fp4(flags, Lk, D);
@@ -531,6 +540,7 @@ static int run_fwd(const void *q, const void *k, const void *v, int B, int H, in
   a.kv_list = listed ? reinterpret_cast<const int32_t *>(wsb + w.kv_list) : nullptr;
   a.kv_count = listed ? reinterpret_cast<const int32_t *>(wsb + w.kv_count) : nullptr;
   a.causal = causal ? 1 : 0;
+  a.quad = tile64 ? 1 : 0;
   cudaError_t e;
   {
     ProfScope ps("attn_fwd", s);
@@ -546,7 +556,9 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
   int st = check_shape(B, H, Lq, Lk, D, sm_scale, flags);
   if (st != ATTNQAT_OK) return st;
   const bool causal = (flags & ATTNQAT_CAUSAL) != 0;
+  const bool tile64 = (flags & ATTNQAT_TILE64) != 0;
   if (causal && mask) return ATTNQAT_EINVAL;
+  if (tile64 && !mask) return ATTNQAT_EINVAL;
   if (!q || !k || !v || !lse || !m || !dO || !dq || !dk || !dv || !ws) return ATTNQAT_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(lse) || !aligned16(m) ||
@@ -559,7 +571,7 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const int BH = B * H;
-  st = plan_sparse(mask, causal, BH, Lq, Lk, wsb, w, s);
+  st = plan_sparse(mask, causal, tile64, BH, Lq, Lk, wsb, w, s);
   if (st != ATTNQAT_OK) return st;
   float *delta = reinterpret_cast<float *>(wsb + w.delta);
   float *stats = reinterpret_cast<float *>(wsb + w.stats);
@@ -607,6 +619,7 @@ static int run_bwd(const void *q, const void *k, const void *v, const float *lse
   a.q_list = listed ? reinterpret_cast<const int32_t *>(wsb + w.q_list) : nullptr;
   a.q_count = listed ? reinterpret_cast<const int32_t *>(wsb + w.q_count) : nullptr;
   a.causal = causal ? 1 : 0;
+  a.quad = tile64 ? 1 : 0;
   // with Q and K quantized, S runs on the packed NVFP4 codes
   CUtensorMap tq4, tk4;
   if (fp4 && !(encode_codes(&tq4, wsb + w.qc, BH, Lq, D) && encode_codes(&tk4, wsb + w.kc, BH, Lk, D)))
@@ -647,7 +660,7 @@ int attnqat_bwd(const void *q, const void *k, const void *v, const float *lse, c
 
 size_t attnqat_sparse_workspace_size(int B, int H, int Lq, int Lk, int D, uint32_t flags) {
   if ((flags & ATTNQAT_CAUSAL) || check_shape(B, H, Lq, Lk, D, 1.0f, flags) != ATTNQAT_OK) return 0;
-  return layout(B, H, Lq, Lk, D, flags, true).total;
+  return layout(B, H, Lq, Lk, D, flags & ~ATTNQAT_TILE64, true).total;
 }
 
 int attnqat_sparse_fwd(const void *q, const void *k, const void *v, int B, int H, int Lq, int Lk, int D,
@@ -657,33 +670,42 @@ int attnqat_sparse_fwd(const void *q, const void *k, const void *v, int B, int H
   return run_fwd(q, k, v, B, H, Lq, Lk, D, sm_scale, flags, tile_mask, o, lse, m, ws, ws_bytes, stream);
 }
 
-size_t attnqat_vsa_select_workspace_size(int B, int H, int Lq, int Lk, int D) {
-  if (check_shape(B, H, Lq, Lk, D, 1.0f, 0) != ATTNQAT_OK) return 0;
+size_t attnqat_vsa_select_tiles_workspace_size(int B, int H, int Lq, int Lk, int D, int tile) {
+  if ((tile != 64 && tile != 128) || check_shape(B, H, Lq, Lk, D, 1.0f, 0) != ATTNQAT_OK) return 0;
   const size_t BH = static_cast<size_t>(B) * H;
-  const size_t nq = (static_cast<size_t>(Lq) + kBM - 1) / kBM, nk = (static_cast<size_t>(Lk) + kBN - 1) / kBN;
+  const size_t nq = (static_cast<size_t>(Lq) + tile - 1) / tile, nk = (static_cast<size_t>(Lk) + tile - 1) / tile;
   return align256(BH * (nq + nk) * D * 4) + align256(BH * nq * nk * 4);
 }
 
-int attnqat_vsa_select(const void *q, const void *k, int B, int H, int Lq, int Lk, int D, int topk,
-                       uint8_t *tile_mask, void *ws, size_t ws_bytes, void *stream) {
+size_t attnqat_vsa_select_workspace_size(int B, int H, int Lq, int Lk, int D) {
+  return attnqat_vsa_select_tiles_workspace_size(B, H, Lq, Lk, D, ATTNQAT_SPARSE_TILE);
+}
+
+int attnqat_vsa_select_tiles(const void *q, const void *k, int B, int H, int Lq, int Lk, int D, int tile, int topk,
+                             uint8_t *tile_mask, void *ws, size_t ws_bytes, void *stream) {
   int st = check_shape(B, H, Lq, Lk, D, 1.0f, 0);
   if (st != ATTNQAT_OK) return st;
-  if (!q || !k || !tile_mask || !ws || topk < 1) return ATTNQAT_EINVAL;
+  if (!q || !k || !tile_mask || !ws || topk < 1 || (tile != 64 && tile != 128)) return ATTNQAT_EINVAL;
   if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return ATTNQAT_EINVAL;
-  const size_t need = attnqat_vsa_select_workspace_size(B, H, Lq, Lk, D);
+  const size_t need = attnqat_vsa_select_tiles_workspace_size(B, H, Lq, Lk, D, tile);
   if (ws_bytes < need) return ATTNQAT_ENOSPC;
   st = check_device();
   if (st != ATTNQAT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t BH = static_cast<size_t>(B) * H;
-  const size_t nq = (static_cast<size_t>(Lq) + kBM - 1) / kBM, nk = (static_cast<size_t>(Lk) + kBN - 1) / kBN;
+  const size_t nq = (static_cast<size_t>(Lq) + tile - 1) / tile, nk = (static_cast<size_t>(Lk) + tile - 1) / tile;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   float *means = reinterpret_cast<float *>(wsb);
   float *scores = reinterpret_cast<float *>(wsb + align256(BH * (nq + nk) * D * 4));
   ProfScope ps("vsa_select", s);
   const cudaError_t e = launch_vsa_select(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-                                          B * H, Lq, Lk, D, topk, means, scores, tile_mask, s);
+                                          B * H, Lq, Lk, D, tile, topk, means, scores, tile_mask, s);
   return e == cudaSuccess ? ATTNQAT_OK : cuda_fail(e);
+}
+
+int attnqat_vsa_select(const void *q, const void *k, int B, int H, int Lq, int Lk, int D, int topk,
+                       uint8_t *tile_mask, void *ws, size_t ws_bytes, void *stream) {
+  return attnqat_vsa_select_tiles(q, k, B, H, Lq, Lk, D, ATTNQAT_SPARSE_TILE, topk, tile_mask, ws, ws_bytes, stream);
 }
 
 int attnqat_sparse_bwd(const void *q, const void *k, const void *v, const float *lse, const float *m,

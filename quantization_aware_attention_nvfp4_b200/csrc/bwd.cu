@@ -238,7 +238,8 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
   const size_t krow = static_cast<size_t>(bh) * a.nk_tiles + kt;
   const int32_t *ql = SP ? a.q_list + krow * nq : nullptr;
   const int n = SP ? a.q_count[krow] : nq;
-  auto qtile = [&](int i) -> int { return SP ? __ldg(ql + i) : i; };
+  // SP 3 (64-token masks): list entries carry quadrant bits in the top byte
+  auto qtile = [&](int i) -> int { return SP == 3 ? (__ldg(ql + i) & 0xFFFFFF) : (SP ? __ldg(ql + i) : i); };
 
   constexpr int NC = kBN / RG;  // key columns per row-warp thread
   if (threadIdx.x == 0) init_bwd_bars(bars, 1, 1, 4 * RG);
@@ -401,10 +402,14 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
       lse = vq ? a.lse[si] : 0.0f;
       delta = vq ? a.delta[si] : 0.0f;
     };
+    // SP 3: this thread's quadrant bit (its query half, its 64-key half)
+    const int qbit = (static_cast<int>(rr.row) >> 6) * 2 + (col0 >> 6);
     float m_n, lse_n, delta_n;
     load_stats(0, m_n, lse_n, delta_n);
     for (int i = 0; i < n; ++i) {
-      const bool vq = qtile(i) * kBM + static_cast<int>(rr.row) < a.Lq;
+      // with quadrant masks a row may have selected no key at all (m = -inf):
+      // it contributes nothing, like a row past Lq
+      const bool vq = qtile(i) * kBM + static_cast<int>(rr.row) < a.Lq && (SP != 3 || m_n > -INFINITY);
       const float m = m_n, lse = lse_n, delta = delta_n;
       load_stats(i + 1, m_n, lse_n, delta_n);
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
@@ -419,8 +424,12 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->sempty);
-        const bool masked = SP == 2 ? i == 0 : valid_k < kBN;
-        const int vk = SP == 2 ? diag_k : valid_k;
+        bool masked = SP == 2 ? i == 0 : valid_k < kBN;
+        int vk = SP == 2 ? diag_k : valid_k;
+        if (SP == 3 && !((__ldg(ql + i) >> (24 + qbit)) & 1)) {
+          masked = true;  // an unselected quadrant: every column of this thread
+          vk = col0;
+        }
         const float nml = vq ? -(m * kLog2e) : -INFINITY;
         const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
         if (masked)
@@ -596,7 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const size_t qrow = static_cast<size_t>(bh) * a.nq_tiles + qt;
   const int32_t *kvl = SP ? a.kv_list + qrow * nk : nullptr;
   const int n = SP ? a.kv_count[qrow] : nk;
-  auto ktile = [&](int j) -> int { return SP ? __ldg(kvl + j) : j; };
+  // SP 3 (64-token masks): list entries carry quadrant bits in the top byte
+  auto ktile = [&](int j) -> int { return SP == 3 ? (__ldg(kvl + j) & 0xFFFFFF) : (SP ? __ldg(kvl + j) : j); };
 
   if (threadIdx.x == 0) init_bwd_bars(bars, 1, 1);
   if (warp == 1) {
@@ -729,8 +739,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const RowRole rr(warp, lane);
     const int col0 = rr.half * 64;
     const int q = qt * kBM + static_cast<int>(rr.row);
-    const bool vq = q < a.Lq;
-    const size_t si = static_cast<size_t>(bh) * a.Lq + (vq ? q : 0);
+    const size_t si = static_cast<size_t>(bh) * a.Lq + (q < a.Lq ? q : 0);
+    // with quadrant masks a row may have selected no key at all (LSE = -inf):
+    // its dQ is 0, like a row past Lq
+    const bool vq = q < a.Lq && (SP != 3 || a.lse[si] > -INFINITY);
     const float lse = vq ? a.lse[si] : 0.0f;
     const float delta = vq ? a.delta[si] : 0.0f;
     const float nlse = vq ? -(lse * kLog2e) : -INFINITY;
@@ -747,13 +759,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // keys 0..r
     const bool tail_last = SP == 2 ? true : (n > 0 && ktile(n - 1) == nk - 1 && last_valid < kBN);
     const int last_cols = SP == 2 ? static_cast<int>(rr.row) + 1 : last_valid;
+    const int qbit = (static_cast<int>(rr.row) >> 6) * 2 + (col0 >> 6);  // SP 3: this thread's quadrant
     const uint32_t xaddr = sbase + L::kX;
     const uint32_t tS = tmem + rr.lane_addr + L::kTmemS, tDP = tmem + rr.lane_addr + L::kTmemDP;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       uint32_t dsw[32], dsl[32];
       uint32_t sv[64], dv[64];
-      const bool tail = tail_last && j == n - 1;
+      bool tail = tail_last && j == n - 1;
+      int vk = last_cols;
+      if (SP == 3 && !((__ldg(kvl + j) >> (24 + qbit)) & 1)) {
+        tail = true;  // an unselected quadrant: every column of this thread
+        vk = col0;
+      }
       if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
       tc_fence_after();
       load_sdp(tS, tDP, col0, sv, dv);
@@ -761,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty);
       if (tail)
-        dq_tile<true, DSPLIT>(sv, dv, col0, last_cols, cl, nlse, a1, b1, dsw, dsl);
+        dq_tile<true, DSPLIT>(sv, dv, col0, vk, cl, nlse, a1, b1, dsw, dsl);
       else
         dq_tile<false, DSPLIT>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw, dsl);
       if (j >= 1 && !mbar_wait(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
@@ -781,7 +799,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld32(tmem + rr.lane_addr + L::kTmemDQ + col, r);
         tmem_ld_wait();
-        if (vq) {
+        // every row in range is written; a row with no selected key (SP 3)
+        // accumulated only zeros
+        if (q < a.Lq) {
           uint4 *dst = reinterpret_cast<uint4 *>(a.dq + rowoff + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -830,6 +850,7 @@ static cudaError_t launch_dkdv_t(const CUtensorMap &tq, const CUtensorMap &tk, c
                                  const CUtensorMap &tdo, const CUtensorMap &tq4, const BwdArgs &a, int BH,
                                  cudaStream_t stream) {
   if (!a.q_list) return launch_dkdv_sp<D, QP, FP4S, 0>(tq, tk, tv, tdo, tq4, a, BH, stream);
+  if (a.quad) return launch_dkdv_sp<D, QP, FP4S, 3>(tq, tk, tv, tdo, tq4, a, BH, stream);
   return a.causal ? launch_dkdv_sp<D, QP, FP4S, 2>(tq, tk, tv, tdo, tq4, a, BH, stream)
                   : launch_dkdv_sp<D, QP, FP4S, 1>(tq, tk, tv, tdo, tq4, a, BH, stream);
 }
@@ -872,6 +893,7 @@ static cudaError_t launch_dq_t(const CUtensorMap &tq, const CUtensorMap &tk, con
                                const CUtensorMap &tdo, const CUtensorMap &tk4, const BwdArgs &a, int BH,
                                cudaStream_t stream) {
   if (!a.kv_list) return launch_dq_sp<D, FP4S, DSPLIT, 0>(tq, tk, tv, tdo, tk4, a, BH, stream);
+  if (a.quad) return launch_dq_sp<D, FP4S, DSPLIT, 3>(tq, tk, tv, tdo, tk4, a, BH, stream);
   return a.causal ? launch_dq_sp<D, FP4S, DSPLIT, 2>(tq, tk, tv, tdo, tk4, a, BH, stream)
                   : launch_dq_sp<D, FP4S, DSPLIT, 1>(tq, tk, tv, tdo, tk4, a, BH, stream);
 }

@@ -231,8 +231,9 @@ template <int G>
 constexpr int fwd_threads() { return (2 + 4 * G + 1 + 3) / 4 * 128; }
 
 // SP: 0 dense; 1 block-sparse (walks a.kv_list); 2 causal (walks the
-// lower-triangle lists and masks the diagonal).  Separate instantiations, so
-// the dense kernel carries none of the list handling.
+// lower-triangle lists and masks the diagonal); 3 block-sparse with 64-token
+// masks (list entries carry quadrant bits).  Separate instantiations, so the
+// dense kernel carries none of the list handling.
 template <int D, int FP4S, int PV4, int QP, int G, int SP>
 __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -260,7 +261,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
   const size_t qrow = static_cast<size_t>(bh) * a.nq_tiles + qt;
   const int32_t *kvl = SP ? a.kv_list + qrow * nk : nullptr;
   const int n = SP ? a.kv_count[qrow] : nk;
-  auto ktile = [&](int j) -> int { return SP ? __ldg(kvl + j) : j; };
+  // SP 3 (64-token masks): list entries carry quadrant bits in the top byte
+  auto ktile = [&](int j) -> int { return SP == 3 ? (__ldg(kvl + j) & 0xFFFFFF) : (SP ? __ldg(kvl + j) : j); };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qfull, 1);
@@ -480,16 +482,27 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     // keys 0..r (which also covers a partial diagonal tile: Lq == Lk)
     const bool tail_last = SP == 2 ? true : (n > 0 && ktile(n - 1) == nk - 1 && last_valid < kBN);
     const int last_cols = SP == 2 ? static_cast<int>(rr.row) + 1 : last_valid;
+    // SP 3: this thread's quadrant bit (its query half, its 64-key half); a
+    // clear bit masks every column it owns (valid bound = col0).  The bit is
+    // the same for the 32 rows and the column group of one warp, and so is
+    // "last tile": the branch between the masked and the plain column loops
+    // is taken on those two alone, never on the per-row bound, because both
+    // loops hold warp-collective TMEM loads (a causal diagonal row 127 has
+    // bound kBN but must stay on its warp's masked path).
+    static_assert(SP != 3 || NC == 64, "quadrant masks need 64 columns per thread");
+    const int qbit = (static_cast<int>(rr.row) >> 6) * 2 + (col0 >> 6);
+    auto quad_clear = [&](int j) -> bool { return SP == 3 && !((__ldg(kvl + j) >> (24 + qbit)) & 1); };
     float mrow = -INFINITY;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int b = j % L::kNS1;
-      const bool tail = tail_last && j == n - 1;
+      const bool clear = quad_clear(j);
+      const bool masked = clear || (tail_last && j == n - 1);  // warp-uniform
+      const int vb = clear ? col0 : last_cols;
       if (!mbar_wait(&bars->sfull1[b], (j / L::kNS1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + b * kBN;
-      const float mx = tail ? row_max_cols<true, NC>(taddr, col0, last_cols)
-                            : row_max_cols<false, NC>(taddr, col0, kBN);
+      const float mx = masked ? row_max_cols<true, NC>(taddr, col0, vb) : row_max_cols<false, NC>(taddr, col0, kBN);
       mrow = fmaxf(mrow, mx);
       tc_fence_before();
       __syncwarp();
@@ -512,7 +525,9 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     for (int j = 0; ok && j < n; ++j) {
       const int sb = j & 1;
       const int pb = PSPLIT ? 0 : (j & 1);
-      const bool tail = tail_last && j == n - 1;
+      const bool clear = quad_clear(j);
+      const bool masked = clear || (tail_last && j == n - 1);  // warp-uniform
+      const int vb = clear ? col0 : last_cols;
       if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, abort)) { ok = false; break; }
       if (PSPLIT ? (j >= 1 && !mbar_wait(&bars->pempty[0], (j - 1) & 1, abort))
                  : (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort))) {
@@ -523,8 +538,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
       const uint32_t psf = sbase + L::kPSFo + pb * L::kPSF;
-      if (tail)
-        lsum += prob_cols<PV4, QP, true, NC>(taddr, col0, last_cols, cl, nml, pbase, psf, rr.row, L::kPBytes);
+      if (masked)
+        lsum += prob_cols<PV4, QP, true, NC>(taddr, col0, vb, cl, nml, pbase, psf, rr.row, L::kPBytes);
       else
         lsum += prob_cols<PV4, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, psf, rr.row, L::kPBytes);
       tc_fence_before();
@@ -546,7 +561,10 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       const int q = qt * kBM + static_cast<int>(rr.row);
       // no key tile selected: O = 0 (the accumulator was never written),
       // m = LSE = -inf.  A scaled fp16 copy of V leaves O * 2^ev in TMEM.
+      // With quadrant masks a row may select no key inside its listed tiles:
+      // l = 0 there, and it is treated the same way.
       const float inv_l = (1.0f / lsum) / (PV4 ? 1.0f : operand_scale(a.amax_v));
+      const bool has_keys = SP == 3 ? (n > 0 && lsum > 0.0f) : n > 0;
       const size_t rowoff = (static_cast<size_t>(bh) * a.Lq + q) * D;
       constexpr int DC = D / G;            // output columns per thread
       constexpr int W = DC < 32 ? DC : 32;  // columns per TMEM load
@@ -563,7 +581,7 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         if (q < a.Lq) {
           float f[W];
 #pragma unroll
-          for (int i = 0; i < W; ++i) f[i] = n > 0 ? __uint_as_float(r[i]) * inv_l : 0.0f;
+          for (int i = 0; i < W; ++i) f[i] = has_keys ? __uint_as_float(r[i]) * inv_l : 0.0f;
           uint32_t w[W / 2];
 #pragma unroll
           for (int i = 0; i < W / 2; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
@@ -576,8 +594,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         }
       }
       if (q < a.Lq && rr.half == 0) {
-        a.m[static_cast<size_t>(bh) * a.Lq + q] = n > 0 ? m_scaled : -INFINITY;
-        a.lse[static_cast<size_t>(bh) * a.Lq + q] = n > 0 ? m_scaled + logf(lsum) : -INFINITY;
+        a.m[static_cast<size_t>(bh) * a.Lq + q] = has_keys ? m_scaled : -INFINITY;
+        a.lse[static_cast<size_t>(bh) * a.Lq + q] = has_keys ? m_scaled + logf(lsum) : -INFINITY;
       }
     } else {
       // keep the MMA issuer's final commit from outliving the CTA
@@ -612,6 +630,7 @@ template <int D, int FP4S, int PV4, int QP>
 static cudaError_t launch_fwd_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                 const FwdArgs &a, int BH, cudaStream_t stream) {
   if (!a.kv_list) return launch_fwd_sp<D, FP4S, PV4, QP, 0>(tq, tk, tv, a, BH, stream);
+  if (a.quad) return launch_fwd_sp<D, FP4S, PV4, QP, 3>(tq, tk, tv, a, BH, stream);
   return a.causal ? launch_fwd_sp<D, FP4S, PV4, QP, 2>(tq, tk, tv, a, BH, stream)
                   : launch_fwd_sp<D, FP4S, PV4, QP, 1>(tq, tk, tv, a, BH, stream);
 }

@@ -33,6 +33,8 @@ struct FwdArgs {
   // causal masking (Lq == Lk): the lists are the lower triangle of tiles and
   // each list's diagonal tile keeps keys <= the query row
   int causal;
+  // 64-token block-sparse masks: list entries carry their quadrant bits
+  int quad;
 };
 
 struct BwdArgs {
@@ -62,6 +64,7 @@ struct BwdArgs {
   const int32_t *q_list;
   const int32_t *q_count;
   int causal;  // as FwdArgs::causal
+  int quad;    // as FwdArgs::quad
 };
 
 // Forward.  Every 16-bit operand is fp16 (see FwdArgs::amax_q).  With fp4s
@@ -129,15 +132,24 @@ cudaError_t launch_scale_f16(const __nv_bfloat16 *x, uint16_t *out, int64_t n, c
 cudaError_t launch_sparse_plan(const uint8_t *mask, int BH, int nq, int nk, int32_t *kv_list, int32_t *kv_count,
                                int32_t *q_list, int32_t *q_count, cudaStream_t stream);
 
+// The same lists from a 64-token mask [BH][nq64][nk64] for the nq x nk
+// 128-token tiles: entries tile | bits << 24, bit (qh * 2 + kh) set when the
+// quadrant (query half qh, key half kh) is selected; tiles with no selected
+// quadrant are left out.
+cudaError_t launch_sparse64_plan(const uint8_t *mask, int BH, int nq64, int nk64, int nq, int nk, int32_t *kv_list,
+                                 int32_t *kv_count, int32_t *q_list, int32_t *q_count, cudaStream_t stream);
+
 // The same lists for causal masking with nt query and key tiles: key tiles
 // 0..I for query tile I, query tiles J..nt-1 for key tile J.
 cudaError_t launch_causal_plan(int BH, int nt, int32_t *kv_list, int32_t *kv_count, int32_t *q_list,
                                int32_t *q_count, cudaStream_t stream);
 
-// VSA key-tile selection (see sparse.cu): tile means of q and k into
-// `means` [BH][nq + nk][D], coarse scores into `scores` [BH][nq][nk], and the
-// tile mask [BH][nq][nk] keeping the topk best key tiles per query tile.
-cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D,
+// VSA key-tile selection over T-token tiles (see sparse.cu): tile means into
+// `means` (per head nq + nk rows of D floats: q's [nq][D], then k's stored
+// transposed, [D][nk]), coarse scores into `scores`
+// [BH][nq][nk], and the tile mask [BH][nq][nk] keeping the topk best key
+// tiles per query tile (nq = ceil(Lq / T), nk = ceil(Lk / T)).
+cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D, int T,
                               int topk, float *means, float *scores, uint8_t *mask, cudaStream_t stream);
 
 // max |x| over n bf16 values folded into *out (must start at 0).

@@ -67,6 +67,80 @@ cudaError_t launch_sparse_plan(const uint8_t *mask, int BH, int nq, int nk, int3
   return cudaGetLastError();
 }
 
+// 64-token block-sparse attention runs on the same 128 x 128 kernel tiles:
+// the caller's mask has 64-token granularity [B*H][nq64][nk64], and a 128-
+// token tile pair is listed when any of its four 64 x 64 quadrants is
+// selected.  Each list entry carries those quadrants in its top byte,
+// tile | bits << 24 with bit (qh * 2 + kh) for query half qh and key half kh,
+// and the kernels mask the unselected quadrants (each row-warp thread owns
+// one 64-key half of one query row, so a quadrant is whole threads).
+__device__ __forceinline__ uint32_t quadrant_bits(const uint8_t *m, int nq64, int nk64, int I, int J) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int qh = 0; qh < 2; ++qh) {
+    const int i = 2 * I + qh;
+    if (i >= nq64) break;
+#pragma unroll
+    for (int kh = 0; kh < 2; ++kh) {
+      const int j = 2 * J + kh;
+      if (j < nk64 && m[static_cast<int64_t>(i) * nk64 + j] != 0) bits |= 1u << (qh * 2 + kh);
+    }
+  }
+  return bits;
+}
+
+__global__ void __launch_bounds__(256) sparse64_plan_kernel(const uint8_t *__restrict__ mask, int BH, int nq64,
+                                                            int nk64, int nq, int nk, int32_t *__restrict__ kv_list,
+                                                            int32_t *__restrict__ kv_count,
+                                                            int32_t *__restrict__ q_list,
+                                                            int32_t *__restrict__ q_count) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(BH) * nq;
+  if (w < rows) {
+    // query tile I of head bh: its key tiles with their quadrants
+    const int64_t bh = w / nq;
+    const int I = static_cast<int>(w - bh * nq);
+    const uint8_t *m = mask + bh * nq64 * nk64;
+    int32_t *dst = kv_list + w * nk;
+    int cnt = 0;
+    for (int j0 = 0; j0 < nk; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t bits = j < nk ? quadrant_bits(m, nq64, nk64, I, j) : 0u;
+      const unsigned b = __ballot_sync(0xffffffffu, bits != 0);
+      if (bits) dst[cnt + __popc(b & ((1u << lane) - 1u))] = static_cast<int32_t>(static_cast<uint32_t>(j) | (bits << 24));
+      cnt += __popc(b);
+    }
+    if (lane == 0) kv_count[w] = cnt;
+  } else if (w < rows + static_cast<int64_t>(BH) * nk) {
+    // key tile J of head bh: the query tiles that selected part of it
+    const int64_t c = w - rows;
+    const int64_t bh = c / nk;
+    const int J = static_cast<int>(c - bh * nk);
+    const uint8_t *m = mask + bh * nq64 * nk64;
+    int32_t *dst = q_list + c * nq;
+    int cnt = 0;
+    for (int i0 = 0; i0 < nq; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t bits = i < nq ? quadrant_bits(m, nq64, nk64, i, J) : 0u;
+      const unsigned b = __ballot_sync(0xffffffffu, bits != 0);
+      if (bits) dst[cnt + __popc(b & ((1u << lane) - 1u))] = static_cast<int32_t>(static_cast<uint32_t>(i) | (bits << 24));
+      cnt += __popc(b);
+    }
+    if (lane == 0) q_count[c] = cnt;
+  }
+}
+
+cudaError_t launch_sparse64_plan(const uint8_t *mask, int BH, int nq64, int nk64, int nq, int nk, int32_t *kv_list,
+                                 int32_t *kv_count, int32_t *q_list, int32_t *q_count, cudaStream_t stream) {
+  const int64_t warps = static_cast<int64_t>(BH) * (nq + nk);
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  sparse64_plan_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(mask, BH, nq64, nk64, nq, nk, kv_list,
+                                                                          kv_count, q_list, q_count);
+  return cudaGetLastError();
+}
+
 // Causal masking walks the lower triangle of tiles: key tiles 0..I for query
 // tile I (the diagonal last), query tiles J..nt-1 for key tile J (the
 // diagonal first).  One warp writes one list.
@@ -101,28 +175,31 @@ cudaError_t launch_causal_plan(int BH, int nt, int32_t *kv_list, int32_t *kv_cou
 //
 // VSA selection (vsqa-test-1.3b metadata.json, "attention.selection": top-k
 // key cubes per query cube; "precision.coarse": BF16, unquantized).  Each
-// 128-token tile is summarised by the mean of its valid rows, the coarse
+// T-token tile (T = 128, or 64 for the tile-64 profile) is summarised by the
+// mean of its valid rows, the coarse
 // score of (query tile I, key tile J) is the dot product of the two means,
 // and query tile I keeps the topk key tiles of highest score, ties to the
 // lower J.  The ranking decides integers, so every step has a fixed float32
 // order: rows summed in token order, one correctly rounded division by the
 // row count, channels accumulated in order with one fused multiply-add each.
 
-// One CTA per (tile, head), one thread per pair of channels (D/2 threads):
-// means[bh][t][d], tiles t < nq of q, then nk tiles of k.  Each step of the
-// row loop reads one 2*D-byte row, coalesced across the CTA; the loop is
-// unrolled so that 16 rows are in flight per thread (the sums stay in token
-// order).
+// One CTA per (tile, head), one thread per pair of channels (D/2 threads).
+// The query tiles' means go to means[bh][t][d] (t < nq); the key tiles' means
+// are stored transposed, means[bh][nq * D + d * nk + j] for key tile j, so
+// that the selection's warp, whose lanes score consecutive key tiles, reads
+// one contiguous line per channel.  Each step of the row loop reads one
+// 2*D-byte row, coalesced across the CTA; the loop is unrolled so that 16
+// rows are in flight per thread (the sums stay in token order).
 __global__ void __launch_bounds__(64) tile_mean_kernel(const __nv_bfloat16 *__restrict__ q,
                                                        const __nv_bfloat16 *__restrict__ k, int Lq, int Lk,
-                                                       int D, int nq, int nk, float *__restrict__ means) {
+                                                       int D, int T, int nq, int nk, float *__restrict__ means) {
   const int t = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int d = 2 * threadIdx.x;
   const bool isq = t < nq;
   const int L = isq ? Lq : Lk;
-  const int r0 = (isq ? t : t - nq) * kBM;
-  const int r1 = r0 + kBM < L ? r0 + kBM : L;
+  const int r0 = (isq ? t : t - nq) * T;
+  const int r1 = r0 + T < L ? r0 + T : L;
   const uint32_t *x =
       reinterpret_cast<const uint32_t *>((isq ? q : k) + static_cast<size_t>(bh) * L * D + d);
   float s0 = 0.0f, s1 = 0.0f;
@@ -133,8 +210,15 @@ __global__ void __launch_bounds__(64) tile_mean_kernel(const __nv_bfloat16 *__re
     s1 = __fadd_rn(s1, __uint_as_float(w & 0xFFFF0000u));
   }
   const float cnt = static_cast<float>(r1 - r0);
-  float2 *dst = reinterpret_cast<float2 *>(means + (static_cast<size_t>(bh) * (nq + nk) + t) * D + d);
-  *dst = make_float2(__fdiv_rn(s0, cnt), __fdiv_rn(s1, cnt));
+  float *base = means + static_cast<size_t>(bh) * (nq + nk) * D;
+  if (isq) {
+    *reinterpret_cast<float2 *>(base + static_cast<size_t>(t) * D + d) =
+        make_float2(__fdiv_rn(s0, cnt), __fdiv_rn(s1, cnt));
+  } else {
+    float *kt = base + static_cast<size_t>(nq) * D + (t - nq);
+    kt[static_cast<size_t>(d) * nk] = __fdiv_rn(s0, cnt);
+    kt[static_cast<size_t>(d + 1) * nk] = __fdiv_rn(s1, cnt);
+  }
 }
 
 // One warp per (head, query tile): the nk coarse scores, then topk rounds of
@@ -156,18 +240,18 @@ __global__ void __launch_bounds__(128) tile_select_kernel(const float *__restric
   const int64_t bh = w / nq;
   const int I = static_cast<int>(w - bh * nq);
   const float4 *qm = reinterpret_cast<const float4 *>(means + (bh * (nq + nk) + I) * D);
-  const float *km = means + (bh * (nq + nk) + nq) * D;
+  const float *kmt = means + (bh * (nq + nk) + nq) * D;  // key means, [D][nk]
   float *sc = SM ? sel_smem + (threadIdx.x >> 5) * nk : scores + w * nk;
   uint8_t *mk = mask + w * nk;
   for (int j = lane; j < nk; j += 32) {
-    const float4 *kr = reinterpret_cast<const float4 *>(km + static_cast<size_t>(j) * D);
+    const float *kc = kmt + j;  // channel d of key tile j at kc[d * nk]
     float acc = 0.0f;
     for (int c = 0; c < D / 4; ++c) {
-      const float4 a = qm[c], b = __ldg(kr + c);
-      acc = __fmaf_rn(a.x, b.x, acc);
-      acc = __fmaf_rn(a.y, b.y, acc);
-      acc = __fmaf_rn(a.z, b.z, acc);
-      acc = __fmaf_rn(a.w, b.w, acc);
+      const float4 a = qm[c];
+      acc = __fmaf_rn(a.x, __ldg(kc + static_cast<size_t>(4 * c) * nk), acc);
+      acc = __fmaf_rn(a.y, __ldg(kc + static_cast<size_t>(4 * c + 1) * nk), acc);
+      acc = __fmaf_rn(a.z, __ldg(kc + static_cast<size_t>(4 * c + 2) * nk), acc);
+      acc = __fmaf_rn(a.w, __ldg(kc + static_cast<size_t>(4 * c + 3) * nk), acc);
     }
     sc[j] = acc;
   }
@@ -199,10 +283,10 @@ __global__ void __launch_bounds__(128) tile_select_kernel(const float *__restric
   for (int j = lane; j < nk; j += 32) mk[j] = sc[j] == -INFINITY ? 1 : 0;
 }
 
-cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D,
+cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D, int T,
                               int topk, float *means, float *scores, uint8_t *mask, cudaStream_t stream) {
-  const int nq = (Lq + kBM - 1) / kBM, nk = (Lk + kBN - 1) / kBN;
-  tile_mean_kernel<<<dim3(nq + nk, BH), D / 2, 0, stream>>>(q, k, Lq, Lk, D, nq, nk, means);
+  const int nq = (Lq + T - 1) / T, nk = (Lk + T - 1) / T;
+  tile_mean_kernel<<<dim3(nq + nk, BH), D / 2, 0, stream>>>(q, k, Lq, Lk, D, T, nq, nk, means);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t blocks = (static_cast<int64_t>(BH) * nq * 32 + 127) / 128;

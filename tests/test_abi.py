@@ -227,3 +227,26 @@ def test_selftest_wait_timeout_validation():
     assert lib.attnqat_selftest_wait_timeout(1000000, P(FAKE + 2), None) == A.EINVAL  # misaligned
     assert lib.attnqat_selftest_wait_timeout(999, P(FAKE), None) == A.EINVAL         # limit too short
     assert lib.attnqat_selftest_wait_timeout(3 * 10**9, P(FAKE), None) == A.EINVAL   # above 2 s
+
+
+def test_tile64_flag_validation():
+    lib = A.load()
+    big = 1 << 30
+    # the 64-token profile keeps the 128-token tile lists: the same workspace
+    for flags in (15, 0, 3):
+        assert A.attnqat_sparse_workspace_size(1, 6, 31200, 31200, 128, flags | A.TILE64) == \
+            A.attnqat_sparse_workspace_size(1, 6, 31200, 31200, 128, flags)
+    # a mask-only flag: not for the dense calls, not with causal masking
+    assert A.attnqat_workspace_size(1, 1, 128, 128, 128, 15 | A.TILE64) == 0
+    assert _fwd(lib, flags=15 | A.TILE64, ws_bytes=big) == A.EINVAL
+    assert A.attnqat_sparse_workspace_size(1, 1, 128, 128, 128, 15 | A.TILE64 | A.CAUSAL) == 0
+    # the selection takes 64- or 128-token tiles
+    assert lib.attnqat_vsa_select_tiles_workspace_size(1, 1, 300, 700, 128, 96) == 0
+    assert lib.attnqat_vsa_select_tiles_workspace_size(1, 1, 300, 700, 128, 128) == \
+        lib.attnqat_vsa_select_workspace_size(1, 1, 300, 700, 128)
+    nq, nk = -(-300 // 64), -(-700 // 64)
+    al = lambda x: (x + 255) // 256 * 256
+    assert lib.attnqat_vsa_select_tiles_workspace_size(1, 1, 300, 700, 128, 64) == \
+        al((nq + nk) * 128 * 4) + al(nq * nk * 4)
+    st = lib.attnqat_vsa_select_tiles(P(FAKE), P(FAKE), 1, 1, 300, 700, 128, 96, 3, P(FAKE), P(FAKE), big, None)
+    assert st == A.EINVAL

@@ -67,7 +67,7 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
 
 def test_default_metric_and_workload_names():
     import argparse
-    a = argparse.Namespace(sparsity=None, causal=False, flags=15, workload="wan_6h_31200")
+    a = argparse.Namespace(sparsity=None, causal=False, flags=15, workload="wan_6h_31200", tile=128)
     w = W.get("wan_6h_31200")
     assert bench.metric_name(a, w) == bench.METRIC
     assert bench.workload_name(a, w) == "wan_6h_31200"
@@ -95,9 +95,17 @@ def test_metric_names_of_every_leg_and_workload():
     for w in W.WORKLOADS:
         for flags in (15, 7, 0):
             for sparsity, causal in ((None, False), (0.9, False), (None, True)):
-                a = argparse.Namespace(sparsity=sparsity, causal=causal, flags=flags, workload=w.name)
+                a = argparse.Namespace(sparsity=sparsity, causal=causal, flags=flags, workload=w.name, tile=128)
                 name = bench.metric_name(a, w)
                 assert "B%d H%d L%d" % (w.B, w.H, w.Lq) in name or name == bench.METRIC
                 assert bench.workload_name(a, w).endswith(w.name if flags == 15 else "%s_flags%d" % (w.name, flags))
-    a = argparse.Namespace(sparsity=None, causal=False, flags=15, workload="tiny")
+    a = argparse.Namespace(sparsity=None, causal=False, flags=15, workload="tiny", tile=128)
     assert bench.metric_name(a, W.get("tiny")) == "Attn-QAT fwd+bwd ms & TFLOP/s at B1 H2 L256 D64; % of B200 BF16 peak"
+
+
+def test_selected_pairs_of_64_token_blocks():
+    w = W.custom(1, 2, 300, 200, 64, seed_index=6)
+    rng = np.random.default_rng(1)
+    mask = (rng.random((1, 2, 5, 4)) < 0.5).astype(np.uint8)
+    brute = sum(int(mask[0, h, i // 64, j // 64]) for h in range(2) for i in range(300) for j in range(200))
+    assert bench.selected_pairs(w, mask, 64) == brute

@@ -1,8 +1,9 @@
 """Property check of the oracle's block-sparse and causal masking over random
-shapes, tile sizes and selections (hypothesis): every query tile's outputs
-equal dense attention against its gathered key tiles, and with causal
-masking every row equals dense attention against its key prefix (quantizers
-off there, so the prefix problem needs no fq(V) of the whole V)."""
+shapes, tile sizes (16, 32 and the tile-64 profile's 64) and selections
+(hypothesis): every query tile's outputs equal dense attention against its
+gathered key tiles, and with causal masking every row equals dense attention
+against its key prefix (quantizers off there, so the prefix problem needs no
+fq(V) of the whole V)."""
 import numpy as np
 from hypothesis import given, settings, strategies as st
 
@@ -16,7 +17,7 @@ def _bits(rng, shape):
 
 @settings(max_examples=12, deadline=None)
 @given(seed=st.integers(0, 2 ** 31 - 1), nq=st.integers(1, 3), nk=st.integers(1, 4),
-       tile=st.sampled_from([16, 32]), rq=st.integers(1, 16), rk=st.integers(1, 16),
+       tile=st.sampled_from([16, 32, 64]), rq=st.integers(1, 16), rk=st.integers(1, 16),
        flags=st.sampled_from([oracle.QUANT_ALL, oracle.QUANT_Q | oracle.QUANT_K | oracle.QUANT_P, 0]))
 def test_sparse_tile_outputs_equal_gathered_dense(seed, nq, nk, tile, rq, rk, flags):
     rng = np.random.default_rng(seed)
