@@ -51,11 +51,20 @@ struct DkdvLayout {
   static constexpr int kV = FP4S ? (kKSF + kSF + 1023) / 1024 * 1024 : kK + kTile;
   static constexpr int kQ4 = kV + kTile;       // FP4S: 2 stages of Q codes
   static constexpr int kQSF = kQ4 + (FP4S ? 2 * kCode : 0);
-  static constexpr int kQ = (kQSF + (FP4S ? 2 * kSF : 0) + 1023) / 1024 * 1024;  // 2 stages
-  static constexpr int kDO = kQ + 2 * kTile;   // 2 stages
-  static constexpr int kX = kDO + 2 * kTile;   // P^T, then dS^T
-  static constexpr int kBar = kX + kXBytes;
+  static constexpr int kQ = (kQSF + (FP4S ? 2 * kSF : 0) + 1023) / 1024 * 1024;  // kNQ stages
   static constexpr int kBarBytes = 256;  // BwdBars (checked at the launch)
+  // Two X buffers (P^T in one, dS^T in the other) let the rows store both
+  // operands of a query tile without waiting for dV to finish reading P^T.
+  // Where two of them and two 16-bit Q stages do not fit (D = 128), the
+  // NVFP4-S build keeps one Q stage (its Q tile feeds dK alone, the last MMA
+  // of a query tile, so one stage has a whole tile's row work to refill);
+  // the 16-bit-S build, whose S also reads that tile, keeps one X buffer.
+  static constexpr bool kFitBoth = kQ + 4 * kTile + 2 * kXBytes + kBarBytes + 1024 <= 232448;
+  static constexpr int kNQ = (kFitBoth || !FP4S) ? 2 : 1;  // 16-bit Q stages
+  static constexpr int kXB = (kFitBoth || FP4S) ? 2 : 1;   // X buffers
+  static constexpr int kDO = kQ + kNQ * kTile;  // 2 stages
+  static constexpr int kX = kDO + 2 * kTile;    // kXB buffers: P^T (and dS^T in the last)
+  static constexpr int kBar = kX + kXB * kXBytes;
   static constexpr int kBytes = kBar + kBarBytes;
   static constexpr int kDynSmem = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
@@ -75,7 +84,7 @@ struct BwdBars {
   // dK/dV kernel: the TMEM buffer's fills S_0, dP_0, S_1, ... one phase each;
   // dQ kernel: S and dP filled together, released together
   uint64_t sfull, sempty;
-  uint64_t xfull, xempty;
+  uint64_t xfull[2], xempty[2];   // X buffers (the dQ kernel uses the first)
   uint64_t done;
   uint64_t adone;   // issuer A's MMAs have completed (drained before TMEM is freed)
   uint32_t tmem_slot;
@@ -96,8 +105,10 @@ __device__ __forceinline__ void init_bwd_bars(BwdBars *b, int a_users, int b_use
   }
   mbar_init(&b->sfull, 1);
   mbar_init(&b->sempty, row_warps);
-  mbar_init(&b->xfull, row_warps);
-  mbar_init(&b->xempty, 1);
+  for (int s = 0; s < 2; ++s) {
+    mbar_init(&b->xfull[s], row_warps);
+    mbar_init(&b->xempty[s], 1);
+  }
   mbar_init(&b->done, 1);
   mbar_init(&b->adone, 1);
   b->abort = 0;
@@ -207,13 +218,13 @@ __device__ __forceinline__ void dkdv_ds(const float (&p)[NC], const uint32_t (&d
 }
 
 // Row warps per TMEM lane quarter of the dK/dV kernel, and its CTA size
-// (producer, MMA issuer, 4 * RG row warps; 12 warps for RG = 2, the two
-// spare warps idle).  RG = 4 (576 threads, 32 columns per thread) measured
+// (producer, MMA issuer, 4 * RG row warps, the 16-bit Q producer; 12 warps
+// for RG = 2, one of them idle).  RG = 4 (32 columns per thread) measured
 // slower at the H6 L31200 shape, 5.23 against 5.08 ms: with 18 warps one
 // scheduler holds five of them, which caps registers at 96 per thread.
 constexpr int kDkdvRG = 2;
 template <int RG>
-constexpr int dkdv_threads() { return RG == 2 ? kThreads : 32 * (2 + 4 * RG); }
+constexpr int dkdv_threads() { return RG == 2 ? kThreads : 32 * (3 + 4 * RG); }
 
 // SP: 0 dense; 1 block-sparse (walks a.q_list); 2 causal (lower-triangle
 // lists, diagonal masked).  Separate instantiations, so the dense kernel
@@ -269,8 +280,9 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
       }
       load_tile<D>(smem + L::kV, &tmV, &bars->kvfull, kt * kBN, bh);
       // per query tile, in the order the MMAs need them: Q codes (S), dO (dP,
-      // then dV), 16-bit Q (dK; with !FP4S also S)
-      int nc = 0, nd = 0, nqh = 0;  // tiles issued per ring
+      // then dV); the 16-bit Q ring (dK; with !FP4S also S) has its own
+      // producer warp, so a wait for its slot never holds these back
+      int nc = 0, nd = 0;  // tiles issued per ring
       for (int i = 0; i < n; ++i) {
         const int st = i & 1;
         const int ph = ((i >> 1) - 1) & 1;
@@ -287,17 +299,28 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
         mbar_arrive_expect_tx(&bars->bfull[st], L::kTile);
         load_tile<D>(smem + L::kDO + st * L::kTile, &tmDO, &bars->bfull[st], qi * kBM, bh);
         nd = i + 1;
-        if (i >= 2 && !mbar_wait(&bars->aempty[st], ph, abort)) break;
-        mbar_arrive_expect_tx(&bars->afull[st], L::kTile);
-        load_tile<D>(smem + L::kQ + st * L::kTile, &tmQ, &bars->afull[st], qi * kBM, bh);
-        nqh = i + 1;
       }
       if (*abort) {
         mbar_wait_drain(&bars->kvfull, 0);
         for (int i = (nc > 2 ? nc - 2 : 0); i < nc; ++i) mbar_wait_drain(&bars->cfull[i & 1], (i >> 1) & 1);
         for (int i = (nd > 2 ? nd - 2 : 0); i < nd; ++i) mbar_wait_drain(&bars->bfull[i & 1], (i >> 1) & 1);
-        for (int i = (nqh > 2 ? nqh - 2 : 0); i < nqh; ++i) mbar_wait_drain(&bars->afull[i & 1], (i >> 1) & 1);
       }
+    }
+  } else if (warp == 2 + 4 * RG) {
+    // ------------------------------------------------ 16-bit Q producer --
+    if (lane == 0) {
+      constexpr int NQ = L::kNQ;
+      prefetch_tmap(&tmQ);
+      int nqh = 0;
+      for (int i = 0; i < n; ++i) {
+        const int sq = i % NQ;
+        if (i >= NQ && !mbar_wait(&bars->aempty[sq], ((i / NQ) - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->afull[sq], L::kTile);
+        load_tile<D>(smem + L::kQ + sq * L::kTile, &tmQ, &bars->afull[sq], qtile(i) * kBM, bh);
+        nqh = i + 1;
+      }
+      if (*abort)
+        for (int i = (nqh > NQ ? nqh - NQ : 0); i < nqh; ++i) mbar_wait_drain(&bars->afull[i % NQ], (i / NQ) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -313,11 +336,16 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
       const uint64_t dQSF = sdesc_make(sbase + L::kQSF, 16, 128, 0);
       const uint64_t dQk = desc_k(sbase + L::kQ), dQmn = desc_mn(sbase + L::kQ);
       const uint64_t dDOk = desc_k(sbase + L::kDO), dDOmn = desc_mn(sbase + L::kDO);
-      const uint64_t dVk = desc_k(sbase + L::kV), dX = desc_mn(sbase + L::kX);
+      const uint64_t dVk = desc_k(sbase + L::kV);
+      // X buffers: P^T in the first, dS^T in the last (the same one when
+      // there is one, used twice per query tile)
+      constexpr int XB = L::kXB;
+      const uint64_t dXP = desc_mn(sbase + L::kX), dXS = desc_mn(sbase + L::kX + (XB - 1) * L::kXBytes);
       // One issuing thread here (a second one measured slower: this kernel is
       // bound by its row warps, whose scheduler the second poller shares).
-      // Order per query tile: dP_i (once the rows have read S_i), dV_i,
-      // S_{i+1} (once the rows have read dP_i), dK_i.
+      // Order per query tile: dP_i (once the rows have read S_i), S_{i+1}
+      // (once the rows have read dP_i, ahead of the two accumulations so that
+      // the rows find it ready when they finish tile i), dV_i, dK_i.
       bool ok = mbar_wait(&bars->kvfull, 0, abort);
       if (ok && FP4S) {
         tc_fence_after();
@@ -329,6 +357,7 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
       auto issue_s = [&](int i) -> bool {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
+        static_assert(FP4S || L::kNQ == 2, "16-bit S reads the 16-bit Q ring");
         if (FP4S) {
           if (!mbar_wait(&bars->cfull[st], ph, abort)) return false;
           tc_fence_after();
@@ -354,26 +383,31 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
       for (int i = 0; ok && i < n; ++i) {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
+        const int sq = i % L::kNQ;  // 16-bit Q stage
+        const uint32_t phq = (i / L::kNQ) & 1;
+        // uses of the X buffers so far: P^T_i is use up of the first, dS^T_i
+        // use us of the last
+        const int up = XB == 2 ? i : 2 * i, us = XB == 2 ? i : 2 * i + 1;
         // dP_i once the rows have read S_i (fill 2i)
         if (!mbar_wait(&bars->sempty, (2 * i) & 1, abort) || !mbar_wait(&bars->bfull[st], ph, abort)) break;
         tc_fence_after();
         mma_kmajor<D / 16>(tbuf, sdesc_add(dDOk, st * L::kTile), dVk, idDP, false);
         umma_commit(&bars->sfull);
-        // dV += (fq(P~)/l)^T dO_i : A = X (M = keys, MN-major), B = dO (N = D, MN-major)
-        if (!mbar_wait(&bars->xfull, (2 * i) & 1, abort)) break;
-        tc_fence_after();
-        mma_mn_mn<kBM / 16>(tmem + L::kTmemDV, dX, sdesc_add(dDOmn, st * L::kTile), idV, i > 0);
-        umma_commit(&bars->xempty);
-        umma_commit(&bars->bempty[st]);
         // S_{i+1} once the rows have read dP_i (fill 2i+1)
         if (i + 1 < n && !(mbar_wait(&bars->sempty, (2 * i + 1) & 1, abort) && issue_s(i + 1))) break;
-        // dK += dS^T Q_i
-        if (!mbar_wait(&bars->xfull, (2 * i + 1) & 1, abort)) break;
-        if (FP4S && !mbar_wait(&bars->afull[st], ph, abort)) break;
+        // dV += (fq(P~)/l)^T dO_i : A = X (M = keys, MN-major), B = dO (N = D, MN-major)
+        if (!mbar_wait(&bars->xfull[0], up & 1, abort)) break;
         tc_fence_after();
-        mma_mn_mn<kBM / 16>(tmem + L::kTmemDK, dX, sdesc_add(dQmn, st * L::kTile), idK, i > 0);
-        umma_commit(&bars->xempty);
-        umma_commit(&bars->aempty[st]);
+        mma_mn_mn<kBM / 16>(tmem + L::kTmemDV, dXP, sdesc_add(dDOmn, st * L::kTile), idV, i > 0);
+        umma_commit(&bars->xempty[0]);
+        umma_commit(&bars->bempty[st]);
+        // dK += dS^T Q_i
+        if (!mbar_wait(&bars->xfull[XB - 1], us & 1, abort)) break;
+        if (FP4S && !mbar_wait(&bars->afull[sq], phq, abort)) break;
+        tc_fence_after();
+        mma_mn_mn<kBM / 16>(tmem + L::kTmemDK, dXS, sdesc_add(dQmn, sq * L::kTile), idK, i > 0);
+        umma_commit(&bars->xempty[XB - 1]);
+        umma_commit(&bars->aempty[sq]);
       }
       umma_commit(&bars->done);
     }
@@ -390,7 +424,8 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
     const float cl = FP4S ? a.scale_log2 : a.scale_log2 / (sq * sk);
     const float dsc = ds_scale(a.stats);
     const float dos = do_scale(a.stats) * operand_scale(a.amax_v);
-    const uint32_t xaddr = sbase + L::kX;
+    constexpr int XB = L::kXB;
+    const uint32_t xaddr_p = sbase + L::kX, xaddr_s = sbase + L::kX + (XB - 1) * L::kXBytes;
     const uint32_t tbuf = tmem + rr.lane_addr + L::kTmemBuf + col0;
     bool ok = true;
     // row statistics of the current query tile, prefetched one tile ahead
@@ -407,6 +442,7 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
     float m_n, lse_n, delta_n;
     load_stats(0, m_n, lse_n, delta_n);
     for (int i = 0; i < n; ++i) {
+      const int up = XB == 2 ? i : 2 * i, us = XB == 2 ? i : 2 * i + 1;  // X buffer uses, as the issuer counts them
       // with quadrant masks a row may have selected no key at all (m = -inf):
       // it contributes nothing, like a row past Lq
       const bool vq = qtile(i) * kBM + static_cast<int>(rr.row) < a.Lq && (SP != 3 || m_n > -INFINITY);
@@ -437,12 +473,13 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
         else
           dkdv_probs<QP, false, NC>(sv, col0, vk, cl, nml, vf, p, pw);
       }
-      // X = (fq(P~)/l)^T once dK_{i-1} has read the previous dS^T
-      if (i >= 1 && !mbar_wait(&bars->xempty, (2 * i - 1) & 1, abort)) { ok = false; break; }
-      store_row_cols<NC>(xaddr, rr.row, col0, pw);
+      // X_P = (fq(P~)/l)^T once the buffer's previous use has been read
+      // (dV_{i-1}; with one buffer, dK_{i-1} reading dS^T_{i-1})
+      if (up >= 1 && !mbar_wait(&bars->xempty[0], (up - 1) & 1, abort)) { ok = false; break; }
+      store_row_cols<NC>(xaddr_p, rr.row, col0, pw);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->xfull);
+      if (lane == 0) mbar_arrive(&bars->xfull[0]);
       {
         // dP_i: read, release the buffer for S_{i+1}, build dS
         uint32_t dv[NC];
@@ -454,12 +491,13 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
         if (lane == 0) mbar_arrive(&bars->sempty);
         dkdv_ds<NC>(p, dv, inv_l * dsc / dos, -delta * inv_l * dsc, dsw);
       }
-      // X = dS^T once dV_i has read the P^T
-      if (!mbar_wait(&bars->xempty, (2 * i) & 1, abort)) { ok = false; break; }
-      store_row_cols<NC>(xaddr, rr.row, col0, dsw);
+      // X_S = dS^T once the buffer's previous use has been read (dK_{i-1};
+      // with one buffer, dV_i reading P^T_i)
+      if (us >= 1 && !mbar_wait(&bars->xempty[XB - 1], (us - 1) & 1, abort)) { ok = false; break; }
+      store_row_cols<NC>(xaddr_s, rr.row, col0, dsw);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->xfull);
+      if (lane == 0) mbar_arrive(&bars->xfull[XB - 1]);
     }
     if (ok && mbar_wait(&bars->done, 0, abort)) {
       tc_fence_after();
@@ -723,13 +761,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (without FP4S, S_j read it too; the rows have read S_j by then).
         for (int j = 0; j < n; ++j) {
           const int st = j & 1;
-          if (!mbar_wait(&bars->xfull, j & 1, abort) || !mbar_wait(&bars->afull[st], (j >> 1) & 1, abort)) break;
+          if (!mbar_wait(&bars->xfull[0], j & 1, abort) || !mbar_wait(&bars->afull[st], (j >> 1) & 1, abort)) break;
           tc_fence_after();
           mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemDQ, dX, sdesc_add(dKmn, st * L::kTile), idQ, j > 0);
           if (DSPLIT)  // the lo tile of dS
             mma_a_k_b_mn<kBN / 16>(tmem + L::kTmemDQ, sdesc_add(dX, L::kXBytes), sdesc_add(dKmn, st * L::kTile), idQ,
                                    true);
-          umma_commit(&bars->xempty);
+          umma_commit(&bars->xempty[0]);
           umma_commit(&bars->aempty[st]);
         }
         umma_commit(&bars->done);
@@ -782,12 +820,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         dq_tile<true, DSPLIT>(sv, dv, col0, vk, cl, nlse, a1, b1, dsw, dsl);
       else
         dq_tile<false, DSPLIT>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw, dsl);
-      if (j >= 1 && !mbar_wait(&bars->xempty, (j - 1) & 1, abort)) { ok = false; break; }
+      if (j >= 1 && !mbar_wait(&bars->xempty[0], (j - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
       if (DSPLIT) store_row_half(xaddr + L::kXBytes, rr.row, rr.half, dsl);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->xfull);
+      if (lane == 0) mbar_arrive(&bars->xfull[0]);
     }
     if (ok && mbar_wait(&bars->done, 0, abort)) {
       tc_fence_after();
