@@ -183,13 +183,11 @@ cudaError_t launch_causal_plan(int BH, int nt, int32_t *kv_list, int32_t *kv_cou
 // order: rows summed in token order, one correctly rounded division by the
 // row count, channels accumulated in order with one fused multiply-add each.
 
-// One CTA per (tile, head), one thread per pair of channels (D/2 threads).
-// The query tiles' means go to means[bh][t][d] (t < nq); the key tiles' means
-// are stored transposed, means[bh][nq * D + d * nk + j] for key tile j, so
-// that the selection's warp, whose lanes score consecutive key tiles, reads
-// one contiguous line per channel.  Each step of the row loop reads one
-// 2*D-byte row, coalesced across the CTA; the loop is unrolled so that 16
-// rows are in flight per thread (the sums stay in token order).
+// One CTA per (tile, head), one thread per pair of channels (D/2 threads):
+// means[bh][t][d], tiles t < nq of q, then nk tiles of k.  Each step of the
+// row loop reads one 2*D-byte row, coalesced across the CTA; the loop is
+// unrolled so that 16 rows are in flight per thread (the sums stay in token
+// order).
 __global__ void __launch_bounds__(64) tile_mean_kernel(const __nv_bfloat16 *__restrict__ q,
                                                        const __nv_bfloat16 *__restrict__ k, int Lq, int Lk,
                                                        int D, int T, int nq, int nk, float *__restrict__ means) {
@@ -210,52 +208,75 @@ __global__ void __launch_bounds__(64) tile_mean_kernel(const __nv_bfloat16 *__re
     s1 = __fadd_rn(s1, __uint_as_float(w & 0xFFFF0000u));
   }
   const float cnt = static_cast<float>(r1 - r0);
-  float *base = means + static_cast<size_t>(bh) * (nq + nk) * D;
-  if (isq) {
-    *reinterpret_cast<float2 *>(base + static_cast<size_t>(t) * D + d) =
-        make_float2(__fdiv_rn(s0, cnt), __fdiv_rn(s1, cnt));
-  } else {
-    float *kt = base + static_cast<size_t>(nq) * D + (t - nq);
-    kt[static_cast<size_t>(d) * nk] = __fdiv_rn(s0, cnt);
-    kt[static_cast<size_t>(d + 1) * nk] = __fdiv_rn(s1, cnt);
-  }
+  float2 *dst = reinterpret_cast<float2 *>(means + (static_cast<size_t>(bh) * (nq + nk) + t) * D + d);
+  *dst = make_float2(__fdiv_rn(s0, cnt), __fdiv_rn(s1, cnt));
 }
 
-// One warp per (head, query tile): the nk coarse scores, then topk rounds of
-// a warp-wide argmax (score descending, tile ascending) over the tiles not
-// yet kept, with the taken tiles marked -inf in the score row (scores are
-// finite for finite inputs).  SM: the score row lives in shared memory
-// (nk <= kSelectSmemTiles), else in `scores` in global memory.  The mask row
-// is written at the end (0 or 1 per tile).
+// One CTA per head and group of kSelectWarps query tiles, a warp per query
+// tile: the nk coarse scores, then topk rounds of a warp-wide argmax (score
+// descending, tile ascending) over the tiles not yet kept, with the taken
+// tiles marked -inf in the score row (scores are finite for finite inputs).
+// The key tiles' means pass through shared memory 32 tiles at a time, rows
+// padded to D + 1 floats, so that lane j scoring key tile j0 + j reads its
+// own bank; the CTA's warps share each staged chunk.  Each score is the
+// in-order chain of D fused multiply-adds.  SM: the score rows live in
+// shared memory (nk <= kSelectSmemTiles), else in `scores` in global memory.
+// The mask row is written at the end (0 or 1 per tile).
 constexpr int kSelectSmemTiles = 2048;
+constexpr int kSelectWarps = 8;
+
+__host__ __device__ constexpr int select_smem_floats(int D, int nk, bool sm) {
+  return kSelectWarps * D + 32 * (D + 1) + (sm ? kSelectWarps * nk : 0);
+}
 
 template <bool SM>
-__global__ void __launch_bounds__(128) tile_select_kernel(const float *__restrict__ means, int BH, int nq, int nk,
-                                                          int D, int topk, float *__restrict__ scores,
-                                                          uint8_t *__restrict__ mask) {
+__global__ void __launch_bounds__(32 * kSelectWarps) tile_select_kernel(const float *__restrict__ means, int nq,
+                                                                        int nk, int D, int topk,
+                                                                        float *__restrict__ scores,
+                                                                        uint8_t *__restrict__ mask) {
   extern __shared__ float sel_smem[];
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= static_cast<int64_t>(BH) * nq) return;  // warp-uniform
-  const int64_t bh = w / nq;
-  const int I = static_cast<int>(w - bh * nq);
-  const float4 *qm = reinterpret_cast<const float4 *>(means + (bh * (nq + nk) + I) * D);
-  const float *kmt = means + (bh * (nq + nk) + nq) * D;  // key means, [D][nk]
-  float *sc = SM ? sel_smem + (threadIdx.x >> 5) * nk : scores + w * nk;
-  uint8_t *mk = mask + w * nk;
-  for (int j = lane; j < nk; j += 32) {
-    const float *kc = kmt + j;  // channel d of key tile j at kc[d * nk]
-    float acc = 0.0f;
-    for (int c = 0; c < D / 4; ++c) {
-      const float4 a = qm[c];
-      acc = __fmaf_rn(a.x, __ldg(kc + static_cast<size_t>(4 * c) * nk), acc);
-      acc = __fmaf_rn(a.y, __ldg(kc + static_cast<size_t>(4 * c + 1) * nk), acc);
-      acc = __fmaf_rn(a.z, __ldg(kc + static_cast<size_t>(4 * c + 2) * nk), acc);
-      acc = __fmaf_rn(a.w, __ldg(kc + static_cast<size_t>(4 * c + 3) * nk), acc);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t bh = blockIdx.y;
+  const int I0 = blockIdx.x * kSelectWarps;
+  const int I = I0 + warp;
+  const bool live = I < nq;  // warp-uniform
+  float *qs = sel_smem;                          // [kSelectWarps][D]
+  float *ks = qs + kSelectWarps * D;             // [32][D + 1]
+  const float *qm = means + (bh * (nq + nk) + I0) * D;
+  const float *km = means + (bh * (nq + nk) + nq) * D;
+  for (int x = threadIdx.x; x < kSelectWarps * D; x += blockDim.x) qs[x] = I0 + x / D < nq ? qm[x] : 0.0f;
+  const int64_t row = bh * nq + I;
+  float *sc = SM ? ks + 32 * (D + 1) + warp * nk : scores + row * nk;
+  for (int j0 = 0; j0 < nk; j0 += 32) {
+    const int rows = nk - j0 < 32 ? nk - j0 : 32;
+    // every load of the chunk in flight before any store (32 rows of at most
+    // 128 channels: 16 per thread)
+    constexpr int kPer = 32 * 128 / (32 * kSelectWarps);
+    float v[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int x = threadIdx.x + u * 32 * kSelectWarps;
+      v[u] = x < rows * D ? __ldg(km + static_cast<size_t>(j0) * D + x) : 0.0f;
     }
-    sc[j] = acc;
+    __syncthreads();  // the previous chunk is consumed (and qs is written)
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int x = threadIdx.x + u * 32 * kSelectWarps;
+      const int r = x / D;
+      if (x < rows * D) ks[r * (D + 1) + (x - r * D)] = v[u];
+    }
+    __syncthreads();
+    if (live && lane < rows) {
+      const float *qr = qs + warp * D, *kr = ks + lane * (D + 1);
+      float acc = 0.0f;
+#pragma unroll 16
+      for (int d = 0; d < D; ++d) acc = __fmaf_rn(qr[d], kr[d], acc);
+      sc[j0 + lane] = acc;
+    }
   }
+  if (!live) return;  // warp-uniform, after the CTA's last barrier
   __syncwarp();
+  uint8_t *mk = mask + row * nk;
   const int kk = topk < nk ? topk : nk;
   for (int r = 0; r < kk; ++r) {
     float best = -INFINITY;
@@ -286,19 +307,23 @@ __global__ void __launch_bounds__(128) tile_select_kernel(const float *__restric
 cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D, int T,
                               int topk, float *means, float *scores, uint8_t *mask, cudaStream_t stream) {
   const int nq = (Lq + T - 1) / T, nk = (Lk + T - 1) / T;
+  if (BH > 65535 || D > 128) return cudaErrorInvalidValue;
   tile_mean_kernel<<<dim3(nq + nk, BH), D / 2, 0, stream>>>(q, k, Lq, Lk, D, T, nq, nk, means);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t blocks = (static_cast<int64_t>(BH) * nq * 32 + 127) / 128;
-  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
-  if (nk <= kSelectSmemTiles) {
-    // 4 warps x nk floats: at most 32 KB
-    tile_select_kernel<true><<<static_cast<unsigned>(blocks), 128, 4 * nk * sizeof(float), stream>>>(
-        means, BH, nq, nk, D, topk, scores, mask);
-  } else {
-    tile_select_kernel<false><<<static_cast<unsigned>(blocks), 128, 0, stream>>>(means, BH, nq, nk, D, topk, scores,
-                                                                                mask);
-  }
+  const dim3 grid((nq + kSelectWarps - 1) / kSelectWarps, BH);
+  const bool sm = nk <= kSelectSmemTiles;
+  const int bytes = select_smem_floats(D, nk, sm) * static_cast<int>(sizeof(float));
+  // the attribute is set once per kernel, so to the most any call needs
+  // (head dimension 128, the longest score row kept in shared memory)
+  const void *kern = sm ? reinterpret_cast<const void *>(tile_select_kernel<true>)
+                        : reinterpret_cast<const void *>(tile_select_kernel<false>);
+  e = ensure_smem_attr(kern, select_smem_floats(128, kSelectSmemTiles, sm) * static_cast<int>(sizeof(float)));
+  if (e != cudaSuccess) return e;
+  if (sm)
+    tile_select_kernel<true><<<grid, 32 * kSelectWarps, bytes, stream>>>(means, nq, nk, D, topk, scores, mask);
+  else
+    tile_select_kernel<false><<<grid, 32 * kSelectWarps, bytes, stream>>>(means, nq, nk, D, topk, scores, mask);
   return cudaGetLastError();
 }
 
