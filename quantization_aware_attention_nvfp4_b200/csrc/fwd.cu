@@ -67,15 +67,18 @@ struct FwdLayout {
   static constexpr int kVSF = PV4 ? 1024 : 0;           // 128 keys = two 64-key scale blocks
   static constexpr int kPBytes = PV4 ? kBM * 64 : kBM * kBN * 2;
   static constexpr int kPSF = PV4 ? 1024 : 0;
+  // P slots: three for the 8 KB NVFP4 P tiles (the rows then never wait for
+  // the P V two tiles back), two for fp16 P (or one P split into hi and lo)
+  static constexpr int kNPB = PV4 ? 3 : 2;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kQK;
   static constexpr int kV = (kK + kNSK * kQK + 1023) / 1024 * 1024;
   static constexpr int kP = kV + kNSV * kVT;
-  static constexpr int kQSF = kP + 2 * kPBytes;
+  static constexpr int kQSF = kP + kNPB * kPBytes;
   static constexpr int kKSF = kQSF + kSF;
   static constexpr int kVSFo = kKSF + kNSK * kSF;
   static constexpr int kPSFo = kVSFo + kNSV * kVSF;
-  static constexpr int kBar = kPSFo + 2 * kPSF;
+  static constexpr int kBar = kPSFo + kNPB * kPSF;
   static constexpr int kBarBytes = 2048;  // FwdBars (checked at the launch)
   static constexpr int kBytes = kBar + kBarBytes;
   static constexpr int kDynSmem = kBytes + 1024;        // slack for 1024-byte alignment
@@ -88,8 +91,8 @@ struct FwdLayout {
   static constexpr int kNS1 = 3;
   static constexpr uint32_t kTmemSFA = 384;
   static constexpr uint32_t kTmemSFB = kTmemSFA + kSFCols;            // kNSK stages
-  static constexpr uint32_t kTmemSFP = kTmemSFB + kNSK * kSFCols;     // PV4: 2 P buffers x 8
-  static constexpr uint32_t kTmemSFV = kTmemSFP + (PV4 ? 16 : 0);     // PV4: kNSV stages x 8
+  static constexpr uint32_t kTmemSFP = kTmemSFB + kNSK * kSFCols;     // PV4: kNPB P slots x 8
+  static constexpr uint32_t kTmemSFV = kTmemSFP + (PV4 ? 8 * kNPB : 0);  // PV4: kNSV stages x 8
   static constexpr uint32_t kTmemEnd = kTmemSFV + (PV4 ? 8 * kNSV : 0);
   // UMMA layout of the packed tiles: 64-byte rows swizzle 64B, 32-byte rows 32B
   static constexpr uint32_t kCodeLayout = (D / 2 == 64) ? 4u : 6u;
@@ -105,7 +108,7 @@ struct FwdBars {
   uint64_t qfull;
   uint64_t kfull[8], kempty[8], vfull[4], vempty[4];   // sized for the deepest rings
   uint64_t sfull1[3], sempty1[3];   // sweep-1 S buffers
-  uint64_t sfull[2], sempty[2], pfull[2], pempty[2];
+  uint64_t sfull[2], sempty[2], pfull[3], pempty[3];
   uint64_t ofull;
   uint64_t sfa_ready;   // issuer A's copy of the Q scales into TMEM has landed
   uint64_t adone;       // issuer A's MMAs have completed (drained before TMEM is freed)
@@ -242,6 +245,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
   // unquantized P: one P slot holding the hi and lo tiles (the two P buffers'
   // space), handed over once per key tile
   constexpr bool PSPLIT = !QP;
+  // P slots in use: one (hi at the slot, lo at the next), else the layout's
+  constexpr int kNP = PSPLIT ? 1 : L::kNPB;
   static_assert(!(PSPLIT && PV4), "the NVFP4 P V takes quantized P");
   static_assert(G <= kFwdG, "column groups beyond the partial-sum block");
   static_assert(L::kNSK <= 8 && L::kNSV <= 4, "ring deeper than its barrier arrays");
@@ -281,6 +286,8 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->sfull[b], 1);
       mbar_init(&bars->sempty[b], 4 * G);
+    }
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&bars->pfull[b], 4 * G);
       mbar_init(&bars->pempty[b], 1);
     }
@@ -432,9 +439,9 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
         // (the first P V runs after every row-max tile was read, so it may
         // overwrite the third S buffer's columns)
         for (int j = 0; ok && j < n; ++j) {
-          const int pb = PSPLIT ? 0 : (j & 1);
+          const int pb = j % kNP;
           const int vs = j % kNSV;
-          const uint32_t pph = PSPLIT ? (j & 1) : ((j >> 1) & 1);
+          const uint32_t pph = (j / kNP) & 1;
           if (!mbar_wait(&bars->pfull[pb], pph, abort) || !mbar_wait(&bars->vfull[vs], (j / kNSV) & 1, abort)) {
             ok = false;
             break;
@@ -524,13 +531,12 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
     float lsum = 0.0f;
     for (int j = 0; ok && j < n; ++j) {
       const int sb = j & 1;
-      const int pb = PSPLIT ? 0 : (j & 1);
+      const int pb = j % kNP;
       const bool clear = quad_clear(j);
       const bool masked = clear || (tail_last && j == n - 1);  // warp-uniform
       const int vb = clear ? col0 : last_cols;
       if (!mbar_wait(&bars->sfull[sb], (j >> 1) & 1, abort)) { ok = false; break; }
-      if (PSPLIT ? (j >= 1 && !mbar_wait(&bars->pempty[0], (j - 1) & 1, abort))
-                 : (j >= 2 && !mbar_wait(&bars->pempty[pb], ((j >> 1) - 1) & 1, abort))) {
+      if (j >= kNP && !mbar_wait(&bars->pempty[pb], ((j / kNP) - 1) & 1, abort)) {
         ok = false;
         break;
       }
