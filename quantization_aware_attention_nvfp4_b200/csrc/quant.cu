@@ -10,13 +10,18 @@
 // then rounded to E4M3 once.  For bf16 amax (8 significant bits) the exact
 // quotient is either representable (then nothing is lost) or lies further
 // than 2^-16 relative from every E4M3 rounding midpoint, so the double
-// rounding cannot move it across one.  The E2M1 code is chosen by comparing
-// |x| with the products m_k * s at the 7 midpoints m_k of the grid, which
-// are exact in float (at most 7 significant bits), so ties are detected
-// exactly and resolved to the even code; three comparisons of a binary search
-// over the midpoints select it.  The dequantized value is the code's E2M1
-// magnitude converted by the hardware (exact) times s in f16 (exact: at most
-// 7 significant bits in [2^-10, 2688]) with the input's sign bit.
+// rounding cannot move it across one.  The E2M1 code is the hardware's
+// round-to-nearest-even conversion (cvt.rn.satfinite.e2m1x2) of a quotient
+// q1 = |x|/s formed as q0 = |x| rcp(s), r = |x| - q0 s (exact, one fused
+// multiply-add), q1 = q0 + r rcp(s): q1 is within about 2^-44 of |x|/s, so
+// it equals |x|/s wherever that quotient is a float -- every tie |x| = m s at
+// a grid midpoint m (at most 7 significant bits) among them -- and otherwise
+// lies on the same side of every midpoint, since a bf16 |x| (8 significant
+// bits) that is not m s is at least 2^-9 of it away.  The conversion then
+// picks exactly the code of |x|/s, ties to even, saturating at 6.  The
+// dequantized value is the code's E2M1 magnitude converted by the hardware
+// (exact) times s in f16 (exact: at most 7 significant bits in [2^-10,
+// 2688]) with the input's sign bit.
 #include "common.cuh"
 #include "internal.h"
 
@@ -25,18 +30,6 @@ namespace attnqat {
 __device__ __forceinline__ uint32_t e4m3_scale_code(float amax) {
   const float t = __fdiv_rn(amax, 6.0f);
   return cvt_e4m3x2(t, 0.0f) & 0xFFu;
-}
-
-// E2M1 magnitude code of |x| (round to nearest even, saturating at 6) from
-// the scaled midpoints t[k] = m_k * s, m = {.25, .75, 1.25, 1.75, 2.5, 3.5,
-// 5}, s > 0: the code is the number of midpoints |x| crosses, and crossing
-// midpoint k (between codes k and k+1) needs '>' when k is even and '>='
-// when k is odd.  Binary search: midpoint 3, then 1 or 5, then the even one.
-__device__ __forceinline__ uint32_t e2m1_code_exact(float ax, const float (&t)[7]) {
-  uint32_t c = ax >= t[3] ? 4u : 0u;
-  c += ax >= (c ? t[5] : t[1]) ? 2u : 0u;
-  const float te = (c & 4u) ? ((c & 2u) ? t[6] : t[4]) : ((c & 2u) ? t[2] : t[0]);
-  return c + (ax > te ? 1u : 0u);
 }
 
 // f16x2 of the two E2M1 codes in the low byte of `byte` (low nibble -> low
@@ -58,12 +51,6 @@ __device__ __forceinline__ uint32_t bf16x2_from_f16x2_exact(uint32_t h) {
   return (__float_as_uint(f.x) >> 16) | (__float_as_uint(f.y) & 0xFFFF0000u);
 }
 
-// Magnitude of E2M1 code c (0..7): 0, .5, 1, 1.5, 2, 3, 4, 6.
-__device__ __forceinline__ float e2m1_magnitude(uint32_t c) {
-  const float fc = static_cast<float>(c);
-  return c < 4 ? 0.5f * fc : (c < 6 ? fc - 2.0f : 2.0f * fc - 8.0f);
-}
-
 // fq of 16 bf16 values (w[i]: elements 2i and 2i+1 as the low and high
 // halves): packed nibbles (element 2i in the low nibble of byte i, 8 bytes as
 // two words; nibble = the input's sign bit | the magnitude code), the scale
@@ -82,13 +69,26 @@ __device__ __forceinline__ void fq16_exact(const uint32_t (&w)[8], uint32_t (&ni
   scode = e4m3_scale_code(amax);
   const uint32_t s_h2 = cvt_f16x2_from_e4m3x2(static_cast<uint16_t>(scode | (scode << 8)));
   const float s = unpack_f16x2(s_h2).x;
-  const float t[7] = {0.25f * s, 0.75f * s, 1.25f * s, 1.75f * s, 2.5f * s, 3.5f * s, 5.0f * s};
   nib[0] = nib[1] = 0u;
+  dmax = 0.0f;
   if (s > 0.0f) {
+    // |x|/s to within ~2^-44 (see the file comment), then the hardware's
+    // nearest-even E2M1 conversion of each pair
+    const float inv = rcp_approx(s);
+    const float2 inv2 = make_float2(inv, inv), ns2 = make_float2(-s, -s);
+    float2 q[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) nib[i >> 3] |= e2m1_code_exact(ax[i], t) << (4 * (i & 7));
+    for (int i = 0; i < 8; ++i) {
+      const float2 a = make_float2(ax[2 * i], ax[2 * i + 1]);
+      const float2 q0 = mul2(a, inv2);
+      q[i] = fma2(fma2(q0, ns2, a), inv2, q0);
+    }
+    nib[0] = e2m1x8(q[0], q[1], q[2], q[3]);
+    nib[1] = e2m1x8(q[4], q[5], q[6], q[7]);
+    const float m0 = amax * inv;
+    const float qm = fmaf(fmaf(m0, -s, amax), inv, m0);
+    dmax = unpack_f16x2(e2m1_round_f16x2(qm, 0.0f)).x * s;
   }
-  dmax = s > 0.0f ? e2m1_magnitude(e2m1_code_exact(amax, t)) * s : 0.0f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t byte = (nib[j >> 2] >> (8 * (j & 3))) & 0xFFu;
