@@ -427,8 +427,9 @@ def gpu_arm(args):
                      "dtype_weighted_peak": round(weighted_peak, 1),
                      "frac_dtype_weighted": round(achieved / weighted_peak, 4)},
         "kernels": kernel_table,
-        # every profiled scope is one kernel launch except the selection (two)
-        "gpu_launches": len(kernels) + sum(1 for n, _ in kernels if n == "vsa_select"),
+        # every profiled scope is one kernel launch except the selection
+        # (three: tile means, coarse scores, top-k)
+        "gpu_launches": len(kernels) + 2 * sum(1 for n, _ in kernels if n == "vsa_select"),
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall, 3),
         "e2e": e2e,

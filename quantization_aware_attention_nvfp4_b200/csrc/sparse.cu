@@ -184,10 +184,9 @@ cudaError_t launch_causal_plan(int BH, int nt, int32_t *kv_list, int32_t *kv_cou
 // row count, channels accumulated in order with one fused multiply-add each.
 
 // One CTA per (tile, head), one thread per pair of channels (D/2 threads):
-// means[bh][t][d], tiles t < nq of q, then nk tiles of k.  Each step of the
-// row loop reads one 2*D-byte row, coalesced across the CTA; the loop is
-// unrolled so that 16 rows are in flight per thread (the sums stay in token
-// order).
+// means[bh][t][d], tiles t < nq of q, then nk tiles of k.  Each thread loads
+// 32 rows of its two channels before adding any (2*D-byte rows, coalesced
+// across the CTA), then adds them in token order.
 __global__ void __launch_bounds__(64) tile_mean_kernel(const __nv_bfloat16 *__restrict__ q,
                                                        const __nv_bfloat16 *__restrict__ k, int Lq, int Lk,
                                                        int D, int T, int nq, int nk, float *__restrict__ means) {
@@ -201,82 +200,93 @@ __global__ void __launch_bounds__(64) tile_mean_kernel(const __nv_bfloat16 *__re
   const uint32_t *x =
       reinterpret_cast<const uint32_t *>((isq ? q : k) + static_cast<size_t>(bh) * L * D + d);
   float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll 16
-  for (int r = r0; r < r1; ++r) {
-    const uint32_t w = __ldg(x + static_cast<size_t>(r) * (D / 2));
-    s0 = __fadd_rn(s0, __uint_as_float(w << 16));
-    s1 = __fadd_rn(s1, __uint_as_float(w & 0xFFFF0000u));
+  for (int r = r0; r < r1; r += 32) {
+    uint32_t w[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) w[u] = r + u < r1 ? __ldg(x + static_cast<size_t>(r + u) * (D / 2)) : 0u;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      if (r + u < r1) {
+        s0 = __fadd_rn(s0, __uint_as_float(w[u] << 16));
+        s1 = __fadd_rn(s1, __uint_as_float(w[u] & 0xFFFF0000u));
+      }
+    }
   }
   const float cnt = static_cast<float>(r1 - r0);
   float2 *dst = reinterpret_cast<float2 *>(means + (static_cast<size_t>(bh) * (nq + nk) + t) * D + d);
   *dst = make_float2(__fdiv_rn(s0, cnt), __fdiv_rn(s1, cnt));
 }
 
-// One CTA per head and group of kSelectWarps query tiles, a warp per query
-// tile: the nk coarse scores, then topk rounds of a warp-wide argmax (score
-// descending, tile ascending) over the tiles not yet kept, with the taken
-// tiles marked -inf in the score row (scores are finite for finite inputs).
-// The key tiles' means pass through shared memory 32 tiles at a time, rows
-// padded to D + 1 floats, so that lane j scoring key tile j0 + j reads its
-// own bank; the CTA's warps share each staged chunk.  Each score is the
-// in-order chain of D fused multiply-adds.  SM: the score rows live in
-// shared memory (nk <= kSelectSmemTiles), else in `scores` in global memory.
-// The mask row is written at the end (0 or 1 per tile).
-constexpr int kSelectSmemTiles = 2048;
-constexpr int kSelectWarps = 8;
-
-__host__ __device__ constexpr int select_smem_floats(int D, int nk, bool sm) {
-  return kSelectWarps * D + 32 * (D + 1) + (sm ? kSelectWarps * nk : 0);
+// Coarse scores: one CTA per (32 key tiles, 8 query tiles, head), a warp per
+// query tile and a lane per key tile.  The CTA stages its means in shared
+// memory (key rows padded to D + 1 floats, so that lane j reads its own
+// bank); each score is the in-order chain of D fused multiply-adds.
+constexpr int kScoreQ = 8;
+__global__ void __launch_bounds__(32 * kScoreQ) tile_score_kernel(const float *__restrict__ means, int nq, int nk,
+                                                                   int D, float *__restrict__ scores) {
+  __shared__ float qs[kScoreQ][128];
+  __shared__ float ks[32][129];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t bh = blockIdx.z;
+  const int I0 = blockIdx.y * kScoreQ, j0 = blockIdx.x * 32;
+  const int nqr = nq - I0 < kScoreQ ? nq - I0 : kScoreQ, nkr = nk - j0 < 32 ? nk - j0 : 32;
+  const float *qm = means + (bh * (nq + nk) + I0) * D;
+  const float *km = means + (bh * (nq + nk) + nq + j0) * D;
+  // every load in flight before any store: 32 key rows and 8 query rows of
+  // at most 128 channels (16 and 4 per thread)
+  float kv[16], qv[4];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int x = threadIdx.x + u * 32 * kScoreQ;
+    kv[u] = x < nkr * D ? __ldg(km + x) : 0.0f;
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int x = threadIdx.x + u * 32 * kScoreQ;
+    qv[u] = x < nqr * D ? __ldg(qm + x) : 0.0f;
+  }
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int x = threadIdx.x + u * 32 * kScoreQ;
+    if (x < nkr * D) ks[x / D][x % D] = kv[u];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int x = threadIdx.x + u * 32 * kScoreQ;
+    if (x < nqr * D) qs[x / D][x % D] = qv[u];
+  }
+  __syncthreads();
+  if (warp < nqr && lane < nkr) {
+    const float *qr = qs[warp], *kr = ks[lane];
+    float acc = 0.0f;
+#pragma unroll 16
+    for (int d = 0; d < D; ++d) acc = __fmaf_rn(qr[d], kr[d], acc);
+    scores[(bh * nq + I0 + warp) * nk + j0 + lane] = acc;
+  }
 }
 
+// Top-k: one warp per (head, query tile), topk rounds of a warp-wide argmax
+// (score descending, tile ascending) over the tiles not yet kept, with the
+// taken tiles marked -inf in the score row (scores are finite for finite
+// inputs).  SM: the warp copies its score row into shared memory first
+// (nk <= kSelectSmemTiles); else it works on the row in global memory.  The
+// mask row is written at the end (0 or 1 per tile).
+constexpr int kSelectSmemTiles = 2048;
+constexpr int kTopkWarps = 4;
+
 template <bool SM>
-__global__ void __launch_bounds__(32 * kSelectWarps) tile_select_kernel(const float *__restrict__ means, int nq,
-                                                                        int nk, int D, int topk,
-                                                                        float *__restrict__ scores,
-                                                                        uint8_t *__restrict__ mask) {
+__global__ void __launch_bounds__(32 * kTopkWarps) tile_topk_kernel(float *__restrict__ scores, int rows, int nk,
+                                                                     int topk, uint8_t *__restrict__ mask) {
   extern __shared__ float sel_smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t bh = blockIdx.y;
-  const int I0 = blockIdx.x * kSelectWarps;
-  const int I = I0 + warp;
-  const bool live = I < nq;  // warp-uniform
-  float *qs = sel_smem;                          // [kSelectWarps][D]
-  float *ks = qs + kSelectWarps * D;             // [32][D + 1]
-  const float *qm = means + (bh * (nq + nk) + I0) * D;
-  const float *km = means + (bh * (nq + nk) + nq) * D;
-  for (int x = threadIdx.x; x < kSelectWarps * D; x += blockDim.x) qs[x] = I0 + x / D < nq ? qm[x] : 0.0f;
-  const int64_t row = bh * nq + I;
-  float *sc = SM ? ks + 32 * (D + 1) + warp * nk : scores + row * nk;
-  for (int j0 = 0; j0 < nk; j0 += 32) {
-    const int rows = nk - j0 < 32 ? nk - j0 : 32;
-    // every load of the chunk in flight before any store (32 rows of at most
-    // 128 channels: 16 per thread)
-    constexpr int kPer = 32 * 128 / (32 * kSelectWarps);
-    float v[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int x = threadIdx.x + u * 32 * kSelectWarps;
-      v[u] = x < rows * D ? __ldg(km + static_cast<size_t>(j0) * D + x) : 0.0f;
-    }
-    __syncthreads();  // the previous chunk is consumed (and qs is written)
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int x = threadIdx.x + u * 32 * kSelectWarps;
-      const int r = x / D;
-      if (x < rows * D) ks[r * (D + 1) + (x - r * D)] = v[u];
-    }
-    __syncthreads();
-    if (live && lane < rows) {
-      const float *qr = qs + warp * D, *kr = ks + lane * (D + 1);
-      float acc = 0.0f;
-#pragma unroll 16
-      for (int d = 0; d < D; ++d) acc = __fmaf_rn(qr[d], kr[d], acc);
-      sc[j0 + lane] = acc;
-    }
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kTopkWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;  // warp-uniform; no CTA barrier follows
+  float *g = scores + row * nk;
+  float *sc = SM ? sel_smem + (threadIdx.x >> 5) * nk : g;
+  if (SM) {
+    for (int j = lane; j < nk; j += 32) sc[j] = g[j];
+    __syncwarp();
   }
-  if (!live) return;  // warp-uniform, after the CTA's last barrier
-  __syncwarp();
-  uint8_t *mk = mask + row * nk;
   const int kk = topk < nk ? topk : nk;
   for (int r = 0; r < kk; ++r) {
     float best = -INFINITY;
@@ -301,29 +311,36 @@ __global__ void __launch_bounds__(32 * kSelectWarps) tile_select_kernel(const fl
     __syncwarp();
   }
   // kept tiles are the ones marked -inf
+  uint8_t *mk = mask + row * nk;
   for (int j = lane; j < nk; j += 32) mk[j] = sc[j] == -INFINITY ? 1 : 0;
 }
 
 cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int BH, int Lq, int Lk, int D, int T,
                               int topk, float *means, float *scores, uint8_t *mask, cudaStream_t stream) {
   const int nq = (Lq + T - 1) / T, nk = (Lk + T - 1) / T;
-  if (BH > 65535 || D > 128) return cudaErrorInvalidValue;
+  if (BH > 65535 || D > 128 || (nq + kScoreQ - 1) / kScoreQ > 65535) return cudaErrorInvalidValue;
   tile_mean_kernel<<<dim3(nq + nk, BH), D / 2, 0, stream>>>(q, k, Lq, Lk, D, T, nq, nk, means);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const dim3 grid((nq + kSelectWarps - 1) / kSelectWarps, BH);
-  const bool sm = nk <= kSelectSmemTiles;
-  const int bytes = select_smem_floats(D, nk, sm) * static_cast<int>(sizeof(float));
-  // the attribute is set once per kernel, so to the most any call needs
-  // (head dimension 128, the longest score row kept in shared memory)
-  const void *kern = sm ? reinterpret_cast<const void *>(tile_select_kernel<true>)
-                        : reinterpret_cast<const void *>(tile_select_kernel<false>);
-  e = ensure_smem_attr(kern, select_smem_floats(128, kSelectSmemTiles, sm) * static_cast<int>(sizeof(float)));
+  tile_score_kernel<<<dim3((nk + 31) / 32, (nq + kScoreQ - 1) / kScoreQ, BH), 32 * kScoreQ, 0, stream>>>(
+      means, nq, nk, D, scores);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (sm)
-    tile_select_kernel<true><<<grid, 32 * kSelectWarps, bytes, stream>>>(means, nq, nk, D, topk, scores, mask);
-  else
-    tile_select_kernel<false><<<grid, 32 * kSelectWarps, bytes, stream>>>(means, nq, nk, D, topk, scores, mask);
+  const int64_t rows = static_cast<int64_t>(BH) * nq;
+  const int64_t blocks = (rows + kTopkWarps - 1) / kTopkWarps;
+  if (blocks > 0x7fffffff || rows > 0x7fffffff) return cudaErrorInvalidValue;
+  if (nk <= kSelectSmemTiles) {
+    // the attribute is set once per kernel, so to the most any call needs
+    const int bytes = kTopkWarps * nk * static_cast<int>(sizeof(float));
+    e = ensure_smem_attr(reinterpret_cast<const void *>(tile_topk_kernel<true>),
+                         kTopkWarps * kSelectSmemTiles * static_cast<int>(sizeof(float)));
+    if (e != cudaSuccess) return e;
+    tile_topk_kernel<true><<<static_cast<unsigned>(blocks), 32 * kTopkWarps, bytes, stream>>>(
+        scores, static_cast<int>(rows), nk, topk, mask);
+  } else {
+    tile_topk_kernel<false><<<static_cast<unsigned>(blocks), 32 * kTopkWarps, 0, stream>>>(
+        scores, static_cast<int>(rows), nk, topk, mask);
+  }
   return cudaGetLastError();
 }
 
