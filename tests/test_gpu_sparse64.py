@@ -136,6 +136,22 @@ def test_vsa_select_at_64_token_tiles_bitwise(B, H, Lq, Lk, D, topk):
             assert np.array_equal(got[b, h], want), (b, h)
 
 
+def test_vsa_select_score_rows_in_global_memory_bitwise():
+    """More than 2048 key tiles (Lk = 131200 at 64-token tiles: 2050): the
+    top-k kernel works on its score row in global memory instead of a
+    shared-memory copy.  Bit for bit against the oracle."""
+    import torch
+    w = W.custom(1, 1, 300, 131200, 64, seed_index=860)
+    inp = W.inputs(w, with_grad=False)
+    q, k = to_gpu_bf16(inp["q"]), to_gpu_bf16(inp["k"])
+    assert -(-w.Lk // T) > 2048
+    got = A.attnqat_vsa_select(q, k, 37, tile=T).cpu().numpy()
+    torch.cuda.synchronize()
+    want, _ = oracle.vsa_select(inp["q"][0, 0], inp["k"][0, 0], 37, tile=T)
+    assert np.array_equal(got[0, 0], want)
+    assert np.all(got.sum(-1) == 37)
+
+
 @pytest.mark.slow
 def test_pages_shape_at_sparsity_09_sampled():
     """H6 L31200 with the tile-64 selection at sparsity 0.9 (49 of 488 key
