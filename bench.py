@@ -456,8 +456,10 @@ def e2e_arm(args, torch, dev, host, w, flops, fwd, bwd, world):
     while step i+1 computes.  Events order each copy against the kernels that
     read or write its slot (an upload waits until the kernels of step i-2 are
     done with the slot, the kernels wait for their upload and for the download
-    of step i-2 to have drained their output slot).  The region ends when the
-    last download has landed in host memory."""
+    of step i-2 to have drained their output slot).  Within a step the forward
+    waits only for Q, K, V (dO lands while it runs) and O, LSE, m leave while
+    the backward runs.  The region ends when the last download has landed in
+    host memory."""
     pin = {n: t.pin_memory() for n, t in host.items()}
     shapes = dict(o=host["q"].shape, dq=host["q"].shape, dk=host["k"].shape, dv=host["v"].shape)
     stat_shape = (w.B, w.H, w.Lq)
@@ -474,35 +476,48 @@ def e2e_arm(args, torch, dev, host, w, flops, fwd, bwd, world):
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = sum(t.numel() * t.element_size() for t in h_out[0].values())
 
+    fwd_in, fwd_out = ("q", "k", "v"), ("o", "lse", "m")
+
     def run(n_steps):
-        uploaded = [torch.cuda.Event() for _ in range(2)]
-        computed = [torch.cuda.Event() for _ in range(2)]
-        drained = [torch.cuda.Event() for _ in range(2)]
+        # per slot: the forward's inputs landed, dO landed, the forward done,
+        # the backward done, and every result of the slot downloaded
+        up_f, up_b, fwd_done, computed, drained = ([torch.cuda.Event() for _ in range(2)] for _ in range(5))
         for i in range(n_steps):
             b = i % 2
             with torch.cuda.stream(up):
                 if i >= 2:
                     up.wait_event(computed[b])  # the kernels of step i-2 are done with slot b
-                for n in pin:
+                for n in fwd_in:
                     d_in[b][n].copy_(pin[n], non_blocking=True)
-                uploaded[b].record(up)
-            comp.wait_event(uploaded[b])
+                up_f[b].record(up)
+                d_in[b]["do"].copy_(pin["do"], non_blocking=True)  # lands while the forward runs
+                up_b[b].record(up)
+            comp.wait_event(up_f[b])
             if i >= 2:
                 comp.wait_event(drained[b])  # step i-2's results have left slot b
             x, y = d_in[b], d_out[b]
             fwd(x["q"], x["k"], x["v"], (y["o"], y["lse"], y["m"]), stream=comp)
+            fwd_done[b].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(fwd_done[b])  # O, LSE, m leave while the backward runs
+                for n in fwd_out:
+                    h_out[b][n].copy_(y[n], non_blocking=True)
+            comp.wait_event(up_b[b])
             bwd(x["q"], x["k"], x["v"], y["lse"], y["m"], x["do"], (y["dq"], y["dk"], y["dv"]), stream=comp)
             computed[b].record(comp)
             with torch.cuda.stream(down):
                 down.wait_event(computed[b])
                 for n in h_out[b]:
-                    h_out[b][n].copy_(y[n], non_blocking=True)
+                    if n not in fwd_out:
+                        h_out[b][n].copy_(y[n], non_blocking=True)
                 drained[b].record(down)
         comp.wait_stream(down)
 
     run(2)
     torch.cuda.synchronize(dev)
-    n = max(2, args.steps // 2)
+    # the same number of steps as the device timing: the pipeline's one fill
+    # (the first upload) and one drain (the last download) are spread over them
+    n = max(2, args.steps)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # the region opens on the compute stream before the first upload is queued
     up.wait_stream(comp)
