@@ -451,27 +451,34 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
       const float inv_l = vq ? ex2_approx((m - lse) * kLog2e) : 0.0f;
       float p[NC];
       uint32_t pw[NC / 2], dsw[NC / 2];
+      // SP 3: an unselected quadrant (warp-uniform) reads neither S nor dP
+      // and stores zero operands
+      const bool clear = SP == 3 && !((__ldg(ql + i) >> (24 + qbit)) & 1);
       {
         // S_i: read, release the buffer for dP_i, build P~ and the dV operand
-        uint32_t sv[NC];
         if (!mbar_wait(&bars->sfull, (2 * i) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        load_cols<NC>(tbuf, sv);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->sempty);
-        bool masked = SP == 2 ? i == 0 : valid_k < kBN;
-        int vk = SP == 2 ? diag_k : valid_k;
-        if (SP == 3 && !((__ldg(ql + i) >> (24 + qbit)) & 1)) {
-          masked = true;  // an unselected quadrant: every column of this thread
-          vk = col0;
+        if (clear) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->sempty);
+#pragma unroll
+          for (int k = 0; k < NC / 2; ++k) pw[k] = 0u;
+        } else {
+          uint32_t sv[NC];
+          load_cols<NC>(tbuf, sv);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->sempty);
+          const bool masked = SP == 2 ? i == 0 : valid_k < kBN;
+          const int vk = SP == 2 ? diag_k : valid_k;
+          const float nml = vq ? -(m * kLog2e) : -INFINITY;
+          const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
+          if (masked)
+            dkdv_probs<QP, true, NC>(sv, col0, vk, cl, nml, vf, p, pw);
+          else
+            dkdv_probs<QP, false, NC>(sv, col0, vk, cl, nml, vf, p, pw);
         }
-        const float nml = vq ? -(m * kLog2e) : -INFINITY;
-        const float vf = inv_l * 16384.0f;  // fq(P~)/l scaled by 2^14 for the fp16 dV operand
-        if (masked)
-          dkdv_probs<QP, true, NC>(sv, col0, vk, cl, nml, vf, p, pw);
-        else
-          dkdv_probs<QP, false, NC>(sv, col0, vk, cl, nml, vf, p, pw);
       }
       // X_P = (fq(P~)/l)^T once the buffer's previous use has been read
       // (dV_{i-1}; with one buffer, dK_{i-1} reading dS^T_{i-1})
@@ -482,14 +489,22 @@ __global__ void __launch_bounds__(dkdv_threads<RG>(), 1)
       if (lane == 0) mbar_arrive(&bars->xfull[0]);
       {
         // dP_i: read, release the buffer for S_{i+1}, build dS
-        uint32_t dv[NC];
         if (!mbar_wait(&bars->sfull, (2 * i + 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        load_cols<NC>(tbuf, dv);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->sempty);
-        dkdv_ds<NC>(p, dv, inv_l * dsc / dos, -delta * inv_l * dsc, dsw);
+        if (clear) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->sempty);
+#pragma unroll
+          for (int k = 0; k < NC / 2; ++k) dsw[k] = 0u;
+        } else {
+          uint32_t dv[NC];
+          load_cols<NC>(tbuf, dv);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->sempty);
+          dkdv_ds<NC>(p, dv, inv_l * dsc / dos, -delta * inv_l * dsc, dsw);
+        }
       }
       // X_S = dS^T once the buffer's previous use has been read (dK_{i-1};
       // with one buffer, dV_i reading P^T_i)
@@ -804,22 +819,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n; ++j) {
       uint32_t dsw[32], dsl[32];
       uint32_t sv[64], dv[64];
-      bool tail = tail_last && j == n - 1;
-      int vk = last_cols;
-      if (SP == 3 && !((__ldg(kvl + j) >> (24 + qbit)) & 1)) {
-        tail = true;  // an unselected quadrant: every column of this thread
-        vk = col0;
-      }
+      const bool tail = tail_last && j == n - 1;
+      const int vk = last_cols;
+      // SP 3: an unselected quadrant (warp-uniform) reads neither S nor dP
+      // and stores zero dS
+      const bool clear = SP == 3 && !((__ldg(kvl + j) >> (24 + qbit)) & 1);
       if (!mbar_wait(&bars->sfull, j & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      load_sdp(tS, tDP, col0, sv, dv);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sempty);
-      if (tail)
-        dq_tile<true, DSPLIT>(sv, dv, col0, vk, cl, nlse, a1, b1, dsw, dsl);
-      else
-        dq_tile<false, DSPLIT>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw, dsl);
+      if (clear) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->sempty);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) dsw[k] = dsl[k] = 0u;
+      } else {
+        load_sdp(tS, tDP, col0, sv, dv);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->sempty);
+        if (tail)
+          dq_tile<true, DSPLIT>(sv, dv, col0, vk, cl, nlse, a1, b1, dsw, dsl);
+        else
+          dq_tile<false, DSPLIT>(sv, dv, col0, kBN, cl, nlse, a1, b1, dsw, dsl);
+      }
       if (j >= 1 && !mbar_wait(&bars->xempty[0], (j - 1) & 1, abort)) { ok = false; break; }
       store_row_half(xaddr, rr.row, rr.half, dsw);
       if (DSPLIT) store_row_half(xaddr + L::kXBytes, rr.row, rr.half, dsl);

@@ -148,7 +148,9 @@ __device__ __forceinline__ float row_max_cols(uint32_t taddr, int col0, int vali
 // and lo = fp16(P~ - hi), stored as two tiles (`lo_off` bytes apart), which
 // carries P~ to about 22 bits.  (Where dP - Delta cancels, Delta = dO . O
 // would otherwise inherit the fp16 rounding of P~ about thirtyfold.)
-template <int PV4, int QP, bool MASKED, int NC>
+// ZERO: every column of the thread is masked (an unselected 64 x 64
+// quadrant; warp-uniform): no TMEM load, zeros stored, l += 0.
+template <int PV4, int QP, bool MASKED, int NC, bool ZERO = false>
 __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, float cl, float nml,
                                            uint32_t pbase, uint32_t psf, uint32_t row, uint32_t lo_off) {
   static_assert(!PV4 || (QP && NC == 64), "NVFP4 P V needs quantized P and 64 columns per thread");
@@ -158,11 +160,17 @@ __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, 
 #pragma unroll
   for (int c = 0; c < NC / 32; ++c) {
     uint32_t r[32];
-    tmem_ld32(taddr + col0 + c * 32, r);
-    tmem_ld_wait();
+    if (!ZERO) {
+      tmem_ld32(taddr + col0 + c * 32, r);
+      tmem_ld_wait();
+    }
     float p[32];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
+      if (ZERO) {
+        p[2 * i] = p[2 * i + 1] = 0.0f;
+        continue;
+      }
       const float2 x = fma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), cl2, nml2);
       const float e0 = ex2_approx(x.x), e1 = ex2_approx(x.y);
       p[2 * i] = (!MASKED || col0 + c * 32 + 2 * i < valid) ? e0 : 0.0f;
@@ -172,9 +180,12 @@ __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, 
     if (PV4) {
       // two 16-key blocks -> 16 bytes of codes (the 16-byte unit cc/32 of the
       // row's 64 bytes, swizzled as TMA's 64-byte mode) and two scale bytes
-      uint32_t cw[4];
-      const uint32_t s0 = fq4_probs(p, *reinterpret_cast<uint32_t(*)[2]>(cw));
-      const uint32_t s1 = fq4_probs(p + 16, *reinterpret_cast<uint32_t(*)[2]>(cw + 2));
+      uint32_t cw[4] = {0u, 0u, 0u, 0u};
+      uint32_t s0 = 0u, s1 = 0u;
+      if (!ZERO) {
+        s0 = fq4_probs(p, *reinterpret_cast<uint32_t(*)[2]>(cw));
+        s1 = fq4_probs(p + 16, *reinterpret_cast<uint32_t(*)[2]>(cw + 2));
+      }
       sfw |= (s0 | (s1 << 8)) << (16 * c);
       const int unit = (col0 + 32 * c) >> 5;
       st_shared_v4(pbase + (row >> 3) * 512 + (row & 7) * 64 + ((unit ^ ((row >> 1) & 3)) << 4), cw[0], cw[1],
@@ -183,7 +194,10 @@ __device__ __forceinline__ float prob_cols(uint32_t taddr, int col0, int valid, 
       uint32_t w[16], wl[16];
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
-        if (QP) {
+        if (ZERO) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[8 * b + i] = wl[8 * b + i] = 0u;
+        } else if (QP) {
           uint32_t rr[8];
           const uint32_t s2 = f16x2_broadcast(fq16_probs(p + 16 * b, rr));
 #pragma unroll
@@ -509,7 +523,9 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       if (!mbar_wait(&bars->sfull1[b], (j / L::kNS1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + rr.lane_addr + b * kBN;
-      const float mx = masked ? row_max_cols<true, NC>(taddr, col0, vb) : row_max_cols<false, NC>(taddr, col0, kBN);
+      // an unselected quadrant adds -inf without reading S
+      const float mx = clear ? -INFINITY
+                             : (masked ? row_max_cols<true, NC>(taddr, col0, vb) : row_max_cols<false, NC>(taddr, col0, kBN));
       mrow = fmaxf(mrow, mx);
       tc_fence_before();
       __syncwarp();
@@ -544,7 +560,9 @@ __global__ void __launch_bounds__(fwd_threads<G>(), 1)
       const uint32_t taddr = tmem + rr.lane_addr + sb * kBN;
       const uint32_t pbase = sbase + L::kP + pb * L::kPBytes;
       const uint32_t psf = sbase + L::kPSFo + pb * L::kPSF;
-      if (masked)
+      if (SP == 3 && clear)  // an unselected quadrant: zeros, without reading S
+        lsum += prob_cols<PV4, QP, true, NC, true>(taddr, col0, vb, cl, nml, pbase, psf, rr.row, L::kPBytes);
+      else if (masked)
         lsum += prob_cols<PV4, QP, true, NC>(taddr, col0, vb, cl, nml, pbase, psf, rr.row, L::kPBytes);
       else
         lsum += prob_cols<PV4, QP, false, NC>(taddr, col0, kBN, cl, nml, pbase, psf, rr.row, L::kPBytes);
