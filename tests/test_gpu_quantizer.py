@@ -48,6 +48,33 @@ def test_every_finite_bf16_as_block_amax():
     _check(b)
 
 
+def _e4m3_positive():
+    """The 126 positive finite E4M3 values (4 exponent bits, bias 7, 3
+    mantissa bits; 448 the largest)."""
+    v = [m / 8 * 2.0 ** -6 for m in range(1, 8)]
+    v += [(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8) if not (e == 15 and m == 7)]
+    return v
+
+
+def test_every_bf16_value_under_every_scale():
+    """Every pair of a block scale and an element value the code conversion
+    can meet: for each positive E4M3 scale s, blocks whose amax is exactly
+    6 s (so the scale is s) and whose other 15 elements run through every bf16
+    value of magnitude <= 6 s, both signs (280649 blocks)."""
+    pos_bits = np.arange(0, 0x7F80, dtype=np.uint32).astype(np.uint16)  # every finite bf16 >= 0
+    pos_vals = (pos_bits.astype(np.uint32) << 16).view(np.float32)
+    blocks = []
+    for s in _e4m3_positive():
+        a = np.array([6.0 * s], np.float32)
+        a_bits = np.uint16(a.view(np.uint32)[0] >> 16)
+        assert float((np.uint32(a_bits) << 16).view(np.float32)) == 6.0 * s  # exact in bf16
+        sel = pos_bits[pos_vals <= a[0]]
+        vals = np.concatenate([sel, sel | np.uint16(0x8000)])
+        vals = np.concatenate([vals, np.zeros((-len(vals)) % 15, np.uint16)]).reshape(-1, 15)
+        blocks.append(np.concatenate([np.full((len(vals), 1), a_bits, np.uint16), vals], axis=1))
+    _check(np.ascontiguousarray(np.concatenate(blocks)))
+
+
 def test_tie_rich_and_edge_blocks():
     rng = np.random.default_rng(102)
     e4m3 = np.array([oracle.e4m3_value(c) for c in range(127)])
