@@ -49,13 +49,26 @@ def sources_digest() -> str:
 ATTENTION_SOURCES = ("fwd.cu", "bwd.cu", "common.cuh", "device.cuh", "internal.h")
 
 
-def attention_sources_digest() -> str:
-    """SHA-256 over the attention kernels' own sources."""
+def code_only(text: str) -> str:
+    """C/C++ source with its comments removed and whitespace collapsed (the
+    sources hold no string literal with a comment marker in it)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def attention_sources_digest(read=None) -> str:
+    """SHA-256 over the attention kernels' own sources, comments removed, so
+    that a comment edit keeps the digest of the same code.  `read(name)`
+    returns a file's text (default: the working tree)."""
     import hashlib
+    if read is None:
+        read = lambda name: open(os.path.join(CSRC, name), encoding="utf-8").read()  # noqa: E731
     h = hashlib.sha256()
     for name in ATTENTION_SOURCES:
         h.update(name.encode())
-        h.update(open(os.path.join(CSRC, name), "rb").read())
+        h.update(code_only(read(name)).encode())
     return h.hexdigest()[:16]
 
 

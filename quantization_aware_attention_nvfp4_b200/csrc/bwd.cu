@@ -6,8 +6,8 @@
 //     one TMEM buffer; the row warps (a query row per TMEM lane) rebuild
 //     P~ = exp(S - m) and fq(P~) exactly as the forward does (same blocks of
 //     16 keys), form (fq(P~)/l)^T and dS^T = (P o (dP - Delta))^T in shared
-//     memory, and the tensor cores accumulate dV += (fq(P~)/l)^T dO and
-//     dK += dS^T fq(Q) in TMEM.
+//     memory (two buffers where they fit), and the tensor cores accumulate
+//     dV += (fq(P~)/l)^T dO and dK += dS^T fq(Q) in TMEM.
 //   dQ kernel: one CTA per (128-query tile, batch*head), looping over key
 //     tiles: S, dP as above, dS = P o (dP - Delta) with P = exp(S - LSE),
 //     dQ += dS fq(K).
@@ -19,9 +19,10 @@
 // (one thread); in the dQ kernel warp 10 is a second MMA-issuing thread, A
 // issuing S and dP and B the dQ products (one thread alone issues a
 // tcgen05.mma only every ~58 cycles, too slowly to keep the tensor pipe busy
-// there); warps 2..9 row warps: two per TMEM lane quarter, so every query row
-// (TMEM lane) has two threads, each owning 64 of the tile's 128 columns; the
-// remaining warps idle.
+// there), and in the dK/dV kernel warp 10 loads the 16-bit Q tiles; warps
+// 2..9 row warps: two per TMEM lane quarter, so every query row (TMEM lane)
+// has two threads, each owning 64 of the tile's 128 columns; the remaining
+// warp idles.
 //
 // Block-sparse (VSA fine attention): with a.q_list / a.kv_list set, the dK/dV
 // kernel walks only the query tiles that selected its key tile and the dQ
