@@ -287,21 +287,42 @@ __global__ void __launch_bounds__(256)
 }
 
 // Blocks of 16 consecutive tokens per channel of a [heads][L][D] tensor (V).
-// Thread (channel group g, token block b) quantizes the 8 channels 8g..8g+7
-// over the 16 tokens of block b: 16 loads of 16 bytes (one token row's 8
-// channels each; consecutive threads on consecutive channel groups, so a warp
-// reads whole rows), a byte-permute transpose into 8 per-channel blocks, the
-// exact fq of each, the transpose back, and 16-byte stores of the
-// dequantized rows.  A ragged last block reads zeros past L (and stores only
-// its valid tokens).  Codes ([head][r][blocks], 8 bytes per block) and scales
-// plain ([head][r][blocks]) or, with `tiled`, scales in the per-128-token-tile
+// Thread (channel group g, token block b) quantizes the CH channels
+// CH g..CH g+CH-1 over the 16 tokens of block b: 16 loads of 2 CH bytes (one
+// token row's CH channels each; consecutive threads on consecutive channel
+// groups, so a warp reads whole rows), a byte-permute transpose into CH
+// per-channel blocks, the exact fq of each, the transpose back, and stores of
+// the dequantized rows.  With CH = 4 a thread holds half the data of CH = 8,
+// so three CTAs share an SM and their load, compute and store phases
+// overlap.  A ragged last block reads zeros past L (and stores only its valid
+// tokens).  Codes ([head][r][blocks], 8 bytes per block) and scales plain
+// ([head][r][blocks]) or, with `tiled`, scales in the per-128-token-tile
 // layout of the general kernel's sf_col_tiles mode.
-template <int D>
-__global__ void __launch_bounds__(256)
+constexpr int kTokensCh = 4;
+
+template <int CH>
+struct TokRow;  // one token row's CH channels (CH / 2 words)
+template <>
+struct TokRow<8> {
+  using V = uint4;
+  __device__ static void split(const V &v, uint32_t (&w)[4]) { w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w; }
+  __device__ static V join(const uint32_t (&w)[4]) { return make_uint4(w[0], w[1], w[2], w[3]); }
+};
+template <>
+struct TokRow<4> {
+  using V = uint2;
+  __device__ static void split(const V &v, uint32_t (&w)[2]) { w[0] = v.x; w[1] = v.y; }
+  __device__ static V join(const uint32_t (&w)[2]) { return make_uint2(w[0], w[1]); }
+};
+
+template <int D, int CH>
+__global__ void __launch_bounds__(256, CH == 4 ? 3 : 1)
     quantize_tokens_kernel(const uint16_t *__restrict__ x, int64_t L, uint8_t *__restrict__ codes,
                            uint8_t *__restrict__ scales, bool tiled, uint16_t *__restrict__ deq,
                            uint16_t *__restrict__ deq_f16, float *__restrict__ absmax) {
-  constexpr int G = D / 8;  // channel groups of 8
+  using R = TokRow<CH>;
+  constexpr int G = D / CH;  // channel groups
+  constexpr int NW = CH / 2;  // words (channel pairs) per token row
   const int64_t nblk = (L + 15) >> 4;
   const int64_t id = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   const int g = static_cast<int>(id % G);
@@ -311,17 +332,25 @@ __global__ void __launch_bounds__(256)
     const int64_t z = blockIdx.y;
     const int64_t row0 = z * L + b * 16;  // first token row of the block
     const int n = static_cast<int>(L - b * 16 < 16 ? L - b * 16 : 16);
-    uint4 t[16];
+    uint32_t t[16][NW];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      t[i] = i < n ? __ldg(reinterpret_cast<const uint4 *>(x + (row0 + i) * D + g * 8)) : make_uint4(0, 0, 0, 0);
-    uint32_t out[16][4];  // dequantized rows (fp16 pairs of channels)
+    for (int i = 0; i < 16; ++i) {
+      typename R::V v;
+      if (i < n) {
+        v = __ldg(reinterpret_cast<const typename R::V *>(x + (row0 + i) * D + g * CH));
+      } else {
+        const uint32_t zero[NW] = {};
+        v = R::join(zero);
+      }
+      R::split(v, t[i]);
+    }
+    uint32_t out[16][NW];  // dequantized rows (fp16 pairs of channels)
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {  // channel pair 2m, 2m+1 (word m of each row)
+    for (int m = 0; m < NW; ++m) {  // channel pair 2m, 2m+1 (word m of each row)
       uint32_t wl[8], wh[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint32_t a = (&t[2 * i].x)[m], c = (&t[2 * i + 1].x)[m];
+        const uint32_t a = t[2 * i][m], c = t[2 * i + 1][m];
         wl[i] = __byte_perm(a, c, 0x5410);  // channel 2m: tokens 2i, 2i+1
         wh[i] = __byte_perm(a, c, 0x7632);  // channel 2m+1
       }
@@ -330,7 +359,7 @@ __global__ void __launch_bounds__(256)
       fq16_exact(wl, nl, sl, hl, dl);
       fq16_exact(wh, nh, sh, hh, dh);
       dmax = fmax3(dmax, dl, dh);
-      const int r = g * 8 + 2 * m;  // channel of wl
+      const int r = g * CH + 2 * m;  // channel of wl
       const int64_t blk = (z * D + r) * nblk + b;
       if (codes) {
         *reinterpret_cast<uint2 *>(codes + blk * 8) = make_uint2(nl[0], nl[1]);
@@ -355,13 +384,14 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       if (i < n) {
-        const int64_t off = (row0 + i) * D + g * 8;
-        if (deq_f16)
-          *reinterpret_cast<uint4 *>(deq_f16 + off) = make_uint4(out[i][0], out[i][1], out[i][2], out[i][3]);
-        if (deq)
-          *reinterpret_cast<uint4 *>(deq + off) =
-              make_uint4(bf16x2_from_f16x2_exact(out[i][0]), bf16x2_from_f16x2_exact(out[i][1]),
-                         bf16x2_from_f16x2_exact(out[i][2]), bf16x2_from_f16x2_exact(out[i][3]));
+        const int64_t off = (row0 + i) * D + g * CH;
+        if (deq_f16) *reinterpret_cast<typename R::V *>(deq_f16 + off) = R::join(out[i]);
+        if (deq) {
+          uint32_t bw[NW];
+#pragma unroll
+          for (int m = 0; m < NW; ++m) bw[m] = bf16x2_from_f16x2_exact(out[i][m]);
+          *reinterpret_cast<typename R::V *>(deq + off) = R::join(bw);
+        }
       }
     }
   }
@@ -397,15 +427,15 @@ cudaError_t launch_quantize(const uint16_t *x, int64_t batch, int64_t rows, int6
   // [heads][L][D] blocked along tokens: rows = D channels (stride 1), cols = L
   // tokens (stride D), batch = heads (stride L*D)
   if (sr == 1 && (rows == 64 || rows == 128) && sc == rows && sb == rows * cols && sf_tile_rows <= 0 && aligned) {
-    const int64_t gx = (((cols + 15) / 16) * (rows / 8) + 255) / 256;
+    const int64_t gx = (((cols + 15) / 16) * (rows / kTokensCh) + 255) / 256;
     if (batch <= 65535 && gx <= 0x7fffffff) {
       const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(batch));
       if (rows == 128)
-        quantize_tokens_kernel<128><<<grid, 256, 0, stream>>>(x, cols, codes, scales, sf_col_tiles, deq, deq_f16,
-                                                              absmax);
+        quantize_tokens_kernel<128, kTokensCh><<<grid, 256, 0, stream>>>(x, cols, codes, scales, sf_col_tiles, deq,
+                                                                         deq_f16, absmax);
       else
-        quantize_tokens_kernel<64><<<grid, 256, 0, stream>>>(x, cols, codes, scales, sf_col_tiles, deq, deq_f16,
-                                                             absmax);
+        quantize_tokens_kernel<64, kTokensCh><<<grid, 256, 0, stream>>>(x, cols, codes, scales, sf_col_tiles, deq,
+                                                                        deq_f16, absmax);
       return cudaGetLastError();
     }
   }
