@@ -109,3 +109,19 @@ def test_selected_pairs_of_64_token_blocks():
     mask = (rng.random((1, 2, 5, 4)) < 0.5).astype(np.uint8)
     brute = sum(int(mask[0, h, i // 64, j // 64]) for h in range(2) for i in range(300) for j in range(200))
     assert bench.selected_pairs(w, mask, 64) == brute
+
+
+def test_attention_digest_ignores_comments_not_code():
+    """The digest that ties profiles/traffic.json to the kernels is the same
+    after a comment edit and different after a code edit."""
+    from quantization_aware_attention_nvfp4_b200 import build
+    base = {n: open(os.path.join(build.CSRC, n)).read() for n in build.ATTENTION_SOURCES}
+    d0 = build.attention_sources_digest(lambda n: base[n])
+    assert d0 == build.attention_sources_digest()
+    commented = dict(base)
+    commented["fwd.cu"] = "// a new line comment\n/* and a\n block one */\n" + base["fwd.cu"].replace(";", ";  // note", 1)
+    assert build.attention_sources_digest(lambda n: commented[n]) == d0
+    edited = dict(base)
+    edited["bwd.cu"] = base["bwd.cu"].replace("kBN", "kBM", 1)
+    assert build.attention_sources_digest(lambda n: edited[n]) != d0
+    assert build.code_only("a = 1; // x\n/* y */ b  =\n 2;") == "a = 1; b = 2;"
