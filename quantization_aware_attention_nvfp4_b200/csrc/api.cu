@@ -4,8 +4,8 @@
 // library; there is no host or library fallback.
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
-#include <set>
 #include <vector>
 #include <utility>
 
@@ -22,16 +22,21 @@ static int cuda_fail(cudaError_t e) {
   return ATTNQAT_ECUDA;
 }
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device.  The largest limit set so far is remembered per (device,
+// kernel): a later call asking for more sets it again.
 cudaError_t ensure_smem_attr(const void *kernel, int bytes) {
   static std::mutex mu;
-  static std::set<std::pair<int, const void *>> done;
+  static std::map<std::pair<int, const void *>, int> done;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
-  if (done.count({dev, kernel})) return cudaSuccess;
+  const auto key = std::make_pair(dev, kernel);
+  const auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done.insert({dev, kernel});
+  if (e == cudaSuccess) done[key] = bytes;
   return e;
 }
 

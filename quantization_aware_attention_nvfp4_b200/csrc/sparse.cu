@@ -330,7 +330,7 @@ cudaError_t launch_vsa_select(const __nv_bfloat16 *q, const __nv_bfloat16 *k, in
   const int64_t blocks = (rows + kTopkWarps - 1) / kTopkWarps;
   if (blocks > 0x7fffffff || rows > 0x7fffffff) return cudaErrorInvalidValue;
   if (nk <= kSelectSmemTiles) {
-    // the attribute is set once per kernel, so to the most any call needs
+    // the limit is raised once, to the most any call of this branch needs
     const int bytes = kTopkWarps * nk * static_cast<int>(sizeof(float));
     e = ensure_smem_attr(reinterpret_cast<const void *>(tile_topk_kernel<true>),
                          kTopkWarps * kSelectSmemTiles * static_cast<int>(sizeof(float)));
