@@ -491,12 +491,16 @@ void oracle_fwd_rows(const double *Qh, const double *Kh, const double *Vh,
             double mi, li;
             prob_row(Qh + i * D, i, Kh, Lk, D, c, flags, sel, T, S, Pt, Ph, &mi,
                      &li);
-            for (long d = 0; d < D; d++) {
-                double acc = 0.0;
-                for (long j = 0; j < Lk; j++)
-                    acc += Ph[j] * Vh[j * D + d];
-                O[t * D + d] = li > 0.0 ? acc / li : 0.0;
-            }
+            /* O_d = sum_j P^_j V^_jd / l, each sum taken in key order j =
+             * 0..Lk-1 (the loop over d runs inside, along V's rows)        */
+            double *acc = O + t * D;
+            for (long d = 0; d < D; d++)
+                acc[d] = 0.0;
+            for (long j = 0; j < Lk; j++)
+                for (long d = 0; d < D; d++)
+                    acc[d] += Ph[j] * Vh[j * D + d];
+            for (long d = 0; d < D; d++)
+                acc[d] = li > 0.0 ? acc[d] / li : 0.0;
             m[t] = mi;
             l[t] = li;
             lse[t] = li > 0.0 ? mi + log(li) : -INFINITY;
