@@ -38,12 +38,14 @@
  *    q, o, dO, dq: [B][H][Lq][D]; k, v, dk, dv: [B][H][Lk][D].  m, lse:
  *    float32 [B][H][Lq].  All pointers are device pointers unless stated.
  *  - The caller owns every buffer; no call allocates device memory.  The
- *    library's state is a once-per-process setup of kernel attributes and of
- *    the driver entry point used to encode TMA descriptors, a per-device
+ *    library's state: the driver entry points it looks up once per process
+ *    (to encode TMA descriptors, to identify a context), the largest dynamic
+ *    shared-memory size set so far per kernel and device, a per-device
  *    record of the device check, the device status word below, and one
  *    static block of ATTNQAT_NOALLOC_WS_MAX bytes per device that only
- *    attnqat_fwd_noalloc uses (held by every GPU that loads the library).
- *    Inputs are never written.
+ *    attnqat_fwd_noalloc uses (held by every GPU that loads the library),
+ *    with its device address kept per device and context.  Inputs are never
+ *    written.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Work is enqueued asynchronously; all argument checks run on the
  *    host before any launch.  There is no CPU fallback.
