@@ -129,10 +129,23 @@ def _torch():
     return torch
 
 
-def _stream_ptr(stream=None):
+def _stream_ptr(stream=None, device=None):
+    """The cudaStream_t of `stream` (default: the current stream of `device`),
+    which must belong to `device` when both are given."""
     torch = _torch()
-    s = torch.cuda.current_stream() if stream is None else stream
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    if device is not None and s.device != device:
+        raise ValueError("stream is on %s, the tensors on %s" % (s.device, device))
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _on(device):
+    """Context that makes `device` the current CUDA device for a library call
+    (the library launches on the current device)."""
+    import contextlib
+    if device.type != "cuda":
+        return contextlib.nullcontext()
+    return _torch().cuda.device(device)
 
 
 def _check(status: int, what: str):
@@ -148,6 +161,58 @@ def _require_bf16_cuda(name, t, ndim=None):
         raise ValueError("%s must be bfloat16" % name)
     if ndim is not None and t.dim() != ndim:
         raise ValueError("%s must have %d dims" % (name, ndim))
+
+
+def _require_buffer(name, t, shape, dtype, device):
+    """A caller-supplied tensor the library reads or writes densely: it must
+    have exactly this shape and dtype, be contiguous and sit on `device` (the
+    C ABI receives a bare pointer and cannot check its extent)."""
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or t.device != device or t.dtype != dtype or \
+            tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous %s tensor of shape %s on %s"
+                         % (name, str(dtype).replace("torch.", ""), tuple(shape), device))
+    return t
+
+
+def _require_workspace(ws, device):
+    """A caller-supplied workspace: contiguous, on `device` (its size is
+    checked by the library against the call's need)."""
+    torch = _torch()
+    if not isinstance(ws, torch.Tensor) or ws.device != device or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous tensor on %s" % device)
+    return ws
+
+
+def _fwd_outputs(out, q, B, H, Lq):
+    """(o, lse, m): new tensors, or the caller's after checking them."""
+    torch = _torch()
+    if out is None:
+        return (torch.empty_like(q), torch.empty((B, H, Lq), dtype=torch.float32, device=q.device),
+                torch.empty((B, H, Lq), dtype=torch.float32, device=q.device))
+    o, lse, m = out
+    _require_buffer("o", o, q.shape, torch.bfloat16, q.device)
+    _require_buffer("lse", lse, (B, H, Lq), torch.float32, q.device)
+    _require_buffer("m", m, (B, H, Lq), torch.float32, q.device)
+    return o, lse, m
+
+
+def _bwd_buffers(q, k, v, lse, m, dO, ws, out, B, H, Lq):
+    """Checks the backward's inputs from the forward (lse, m, ws) and dO;
+    returns (dq, dk, dv): new tensors, or the caller's after checking them."""
+    torch = _torch()
+    _require_bf16_cuda("dO", dO, 4)
+    _require_buffer("dO", dO, q.shape, torch.bfloat16, q.device)
+    _require_buffer("lse", lse, (B, H, Lq), torch.float32, q.device)
+    _require_buffer("m", m, (B, H, Lq), torch.float32, q.device)
+    _require_workspace(ws, q.device)
+    if out is None:
+        return torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq, dk, dv = out
+    _require_buffer("dq", dq, q.shape, torch.bfloat16, q.device)
+    _require_buffer("dk", dk, k.shape, torch.bfloat16, q.device)
+    _require_buffer("dv", dv, v.shape, torch.bfloat16, q.device)
+    return dq, dk, dv
 
 
 def attnqat_quantize(x, stream=None):
@@ -169,9 +234,10 @@ def attnqat_quantize(x, stream=None):
     codes = torch.empty((batch, rows, cols // 2), dtype=torch.uint8, device=x.device)
     scales = torch.empty((batch, rows, cols // 16), dtype=torch.uint8, device=x.device)
     deq = torch.empty_strided(x.shape, x.stride(), dtype=torch.bfloat16, device=x.device)
-    st = load().attnqat_quantize(ctypes.c_void_p(x.data_ptr()), batch, rows, cols, sb, sr, sc,
-                                 ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
-                                 ctypes.c_void_p(deq.data_ptr()), _stream_ptr(stream))
+    with _on(x.device):
+        st = load().attnqat_quantize(ctypes.c_void_p(x.data_ptr()), batch, rows, cols, sb, sr, sc,
+                                     ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                                     ctypes.c_void_p(deq.data_ptr()), _stream_ptr(stream, x.device))
     _check(st, "attnqat_quantize")
     if x.dim() == 2:
         codes, scales = codes[0], scales[0]
@@ -198,10 +264,11 @@ def attnqat_quantize_gs(x, stream=None):
     scales = torch.empty((batch, rows, cols // 16), dtype=torch.uint8, device=x.device)
     deq = torch.empty_strided(x.shape, x.stride(), dtype=torch.bfloat16, device=x.device)
     gscale = torch.empty(1, dtype=torch.float32, device=x.device)
-    st = load().attnqat_quantize_gs(ctypes.c_void_p(x.data_ptr()), batch, rows, cols, sb, sr, sc,
-                                    ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
-                                    ctypes.c_void_p(deq.data_ptr()), ctypes.c_void_p(gscale.data_ptr()),
-                                    _stream_ptr(stream))
+    with _on(x.device):
+        st = load().attnqat_quantize_gs(ctypes.c_void_p(x.data_ptr()), batch, rows, cols, sb, sr, sc,
+                                        ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                                        ctypes.c_void_p(deq.data_ptr()), ctypes.c_void_p(gscale.data_ptr()),
+                                        _stream_ptr(stream, x.device))
     _check(st, "attnqat_quantize_gs")
     if x.dim() == 2:
         codes, scales = codes[0], scales[0]
@@ -220,6 +287,8 @@ def _shape(q, k, v):
     B, H, Lq, D = q.shape
     if k.shape != v.shape or k.shape[0] != B or k.shape[1] != H or k.shape[3] != D:
         raise ValueError("k and v must be [B, H, Lk, D] matching q [B, H, Lq, D]")
+    if k.device != q.device or v.device != q.device:
+        raise ValueError("q, k and v must be on one device")
     return B, H, Lq, k.shape[2], D
 
 
@@ -232,19 +301,14 @@ def attnqat_fwd(q, k, v, sm_scale=None, flags=QUANT_ALL, ws=None, out=None, stre
     need = attnqat_workspace_size(B, H, Lq, Lk, D, flags)
     if need == 0:
         _check(EINVAL, "attnqat_workspace_size")
-    if ws is None:
-        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
-    if out is None:
-        o = torch.empty_like(q)
-        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-        m = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-    else:
-        o, lse, m = out
-    st = load().attnqat_fwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                            ctypes.c_void_p(v.data_ptr()), B, H, Lq, Lk, D, c, flags,
-                            ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
-                            ctypes.c_void_p(m.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
-                            ws.numel() * ws.element_size(), _stream_ptr(stream))
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if ws is None else _require_workspace(ws, q.device)
+    o, lse, m = _fwd_outputs(out, q, B, H, Lq)
+    with _on(q.device):
+        st = load().attnqat_fwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                ctypes.c_void_p(v.data_ptr()), B, H, Lq, Lk, D, c, flags,
+                                ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+                                ctypes.c_void_p(m.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                ws.numel() * ws.element_size(), _stream_ptr(stream, q.device))
     _check(st, "attnqat_fwd")
     return o, lse, m, ws
 
@@ -252,23 +316,17 @@ def attnqat_fwd(q, k, v, sm_scale=None, flags=QUANT_ALL, ws=None, out=None, stre
 def attnqat_bwd(q, k, v, lse, m, dO, ws, sm_scale=None, flags=QUANT_ALL, out=None, stream=None):
     """Attn-QAT backward (straight-through).  ``ws`` is the workspace the
     forward returned.  Returns ``(dq, dk, dv)``."""
-    torch = _torch()
     B, H, Lq, Lk, D = _shape(q, k, v)
-    _require_bf16_cuda("dO", dO, 4)
-    if dO.shape != q.shape or not dO.is_contiguous():
-        raise ValueError("dO must be contiguous and shaped like q")
+    dq, dk, dv = _bwd_buffers(q, k, v, lse, m, dO, ws, out, B, H, Lq)
     c = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    if out is None:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    else:
-        dq, dk, dv = out
-    st = load().attnqat_bwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                            ctypes.c_void_p(v.data_ptr()),
-                            ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(m.data_ptr()),
-                            ctypes.c_void_p(dO.data_ptr()), B, H, Lq, Lk, D, c, flags,
-                            ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
-                            ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
-                            ws.numel() * ws.element_size(), _stream_ptr(stream))
+    with _on(q.device):
+        st = load().attnqat_bwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                ctypes.c_void_p(v.data_ptr()),
+                                ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(m.data_ptr()),
+                                ctypes.c_void_p(dO.data_ptr()), B, H, Lq, Lk, D, c, flags,
+                                ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
+                                ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                ws.numel() * ws.element_size(), _stream_ptr(stream, q.device))
     _check(st, "attnqat_bwd")
     return dq, dk, dv
 
@@ -312,19 +370,21 @@ def attnqat_vsa_select(q, k, topk, out=None, ws=None, stream=None, tile=SPARSE_T
     Lk = k.shape[2]
     if k.shape[0] != B or k.shape[1] != H or k.shape[3] != D:
         raise ValueError("k must be [B, H, Lk, D] matching q [B, H, Lq, D]")
+    if k.device != q.device:
+        raise ValueError("q and k must be on one device")
     need = int(load().attnqat_vsa_select_tiles_workspace_size(B, H, Lq, Lk, D, tile))
     if need == 0:
         _check(EINVAL, "attnqat_vsa_select_tiles_workspace_size")
-    if ws is None:
-        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if ws is None else _require_workspace(ws, q.device)
     if out is None:
         out = torch.empty((B, H, -(-Lq // tile), -(-Lk // tile)), dtype=torch.uint8, device=q.device)
     else:
         _tile_mask(out, B, H, Lq, Lk, q.device, tile)
-    st = load().attnqat_vsa_select_tiles(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), B, H, Lq, Lk,
-                                         D, tile, int(topk), ctypes.c_void_p(out.data_ptr()),
-                                         ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(),
-                                         _stream_ptr(stream))
+    with _on(q.device):
+        st = load().attnqat_vsa_select_tiles(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), B, H, Lq,
+                                             Lk, D, tile, int(topk), ctypes.c_void_p(out.data_ptr()),
+                                             ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(),
+                                             _stream_ptr(stream, q.device))
     _check(st, "attnqat_vsa_select_tiles")
     return out
 
@@ -343,19 +403,14 @@ def attnqat_sparse_fwd(q, k, v, tile_mask, sm_scale=None, flags=QUANT_ALL, ws=No
     need = attnqat_sparse_workspace_size(B, H, Lq, Lk, D, flags)
     if need == 0:
         _check(EINVAL, "attnqat_sparse_workspace_size")
-    if ws is None:
-        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
-    if out is None:
-        o = torch.empty_like(q)
-        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-        m = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
-    else:
-        o, lse, m = out
-    st = load().attnqat_sparse_fwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                                   ctypes.c_void_p(v.data_ptr()), B, H, Lq, Lk, D, c, flags, mp,
-                                   ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
-                                   ctypes.c_void_p(m.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
-                                   ws.numel() * ws.element_size(), _stream_ptr(stream))
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if ws is None else _require_workspace(ws, q.device)
+    o, lse, m = _fwd_outputs(out, q, B, H, Lq)
+    with _on(q.device):
+        st = load().attnqat_sparse_fwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                       ctypes.c_void_p(v.data_ptr()), B, H, Lq, Lk, D, c, flags, mp,
+                                       ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+                                       ctypes.c_void_p(m.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                       ws.numel() * ws.element_size(), _stream_ptr(stream, q.device))
     _check(st, "attnqat_sparse_fwd")
     return o, lse, m, ws
 
@@ -364,25 +419,19 @@ def attnqat_sparse_bwd(q, k, v, lse, m, dO, ws, tile_mask, sm_scale=None, flags=
                        stream=None, tile=SPARSE_TILE):
     """Block-sparse Attn-QAT backward (straight-through) with the forward's
     ``ws``, ``tile_mask`` and ``tile``.  Returns ``(dq, dk, dv)``."""
-    torch = _torch()
     B, H, Lq, Lk, D = _shape(q, k, v)
     flags = (flags & ~TILE64) | _check_tile(tile)
     mp = _tile_mask(tile_mask, B, H, Lq, Lk, q.device, tile)
-    _require_bf16_cuda("dO", dO, 4)
-    if dO.shape != q.shape or not dO.is_contiguous():
-        raise ValueError("dO must be contiguous and shaped like q")
+    dq, dk, dv = _bwd_buffers(q, k, v, lse, m, dO, ws, out, B, H, Lq)
     c = 1.0 / math.sqrt(D) if sm_scale is None else float(sm_scale)
-    if out is None:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    else:
-        dq, dk, dv = out
-    st = load().attnqat_sparse_bwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                                   ctypes.c_void_p(v.data_ptr()),
-                                   ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(m.data_ptr()),
-                                   ctypes.c_void_p(dO.data_ptr()), B, H, Lq, Lk, D, c, flags, mp,
-                                   ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
-                                   ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
-                                   ws.numel() * ws.element_size(), _stream_ptr(stream))
+    with _on(q.device):
+        st = load().attnqat_sparse_bwd(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                       ctypes.c_void_p(v.data_ptr()),
+                                       ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(m.data_ptr()),
+                                       ctypes.c_void_p(dO.data_ptr()), B, H, Lq, Lk, D, c, flags, mp,
+                                       ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
+                                       ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                       ws.numel() * ws.element_size(), _stream_ptr(stream, q.device))
     _check(st, "attnqat_sparse_bwd")
     return dq, dk, dv
 
