@@ -29,6 +29,7 @@ differences; none is "parity unpinned".
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -52,64 +53,92 @@ _lock = threading.Lock()
 _lib = None
 
 
+def compile_library(src: str, out: str) -> str:
+    """gcc (OpenMP, no floating-point contraction) of one oracle source file
+    into a shared library at `out`."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+           "-std=c11", "-Wall", src, "-o", out, "-lm"]
+    subprocess.check_call(cmd)
+    return out
+
+
 def build(force: bool = False) -> str:
     """Compile oracle.c into liboracle.so (gcc, OpenMP).  Returns the path."""
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
-           "-std=c11", "-Wall", SRC, "-o", tmp, "-lm"]
-    subprocess.check_call(cmd)
+    compile_library(SRC, tmp)
     os.replace(tmp, LIB)
     return LIB
+
+
+@contextlib.contextmanager
+def library(path: str):
+    """Test hook for the planted-mistake checks: inside the block every call of
+    this module goes through the library at `path` (a build of a modified
+    oracle.c); the previous library is restored on exit."""
+    global _lib
+    lib = _open(path)
+    with _lock:
+        saved, _lib = _lib, lib
+    try:
+        yield
+    finally:
+        with _lock:
+            _lib = saved
 
 
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            P = ctypes.c_void_p
-            L = ctypes.c_long
-            lib.oracle_bf16_value.restype = ctypes.c_double
-            lib.oracle_bf16_value.argtypes = [ctypes.c_uint16]
-            lib.oracle_e4m3_value.restype = ctypes.c_double
-            lib.oracle_e4m3_value.argtypes = [ctypes.c_int]
-            lib.oracle_e2m1_value.restype = ctypes.c_double
-            lib.oracle_e2m1_value.argtypes = [ctypes.c_int]
-            lib.oracle_e4m3_round_div6.restype = ctypes.c_int
-            lib.oracle_e4m3_round_div6.argtypes = [ctypes.c_double]
-            lib.oracle_e2m1_round.restype = ctypes.c_int
-            lib.oracle_e2m1_round.argtypes = [ctypes.c_double, ctypes.c_double]
-            lib.oracle_e2m1_round_many.restype = None
-            lib.oracle_e2m1_round_many.argtypes = [P, P, L, P]
-            lib.oracle_quantize_rows.restype = None
-            lib.oracle_quantize_rows.argtypes = [P, L, L, L, L, P, P, P]
-            lib.oracle_global_scale.restype = ctypes.c_float
-            lib.oracle_global_scale.argtypes = [ctypes.c_double]
-            lib.oracle_quantize_rows_gs.restype = None
-            lib.oracle_quantize_rows_gs.argtypes = [P, L, L, L, L, P, P, P, P]
-            lib.oracle_fq_f64_rows.restype = None
-            lib.oracle_fq_f64_rows.argtypes = [P, L, L, P, P]
-            lib.oracle_operands.restype = None
-            lib.oracle_operands.argtypes = [P, P, P, L, L, L, ctypes.c_uint, P, P, P]
-            lib.oracle_fwd_rows.restype = None
-            lib.oracle_fwd_rows.argtypes = [P, P, P, L, L, L, ctypes.c_double,
-                                            ctypes.c_uint, P, L, P, L, P, P, P, P]
-            lib.oracle_delta.restype = None
-            lib.oracle_delta.argtypes = [P, P, L, L, P]
-            lib.oracle_bwd_dq_rows.restype = None
-            lib.oracle_bwd_dq_rows.argtypes = [P, P, P, P, L, L, L, ctypes.c_double,
-                                               ctypes.c_uint, P, L, P, P, P, P, L, P]
-            lib.oracle_bwd_dkdv_blocks.restype = None
-            lib.oracle_bwd_dkdv_blocks.argtypes = [P, P, P, P, L, L, L, ctypes.c_double,
-                                                   ctypes.c_uint, P, L, P, P, P, P, L, P, P]
-            lib.oracle_vsa_select.restype = None
-            lib.oracle_vsa_select.argtypes = [P, P, L, L, L, L, L, P, P]
-            lib.oracle_num_threads.restype = ctypes.c_int
-            lib.oracle_num_threads.argtypes = []
-            _lib = lib
+            _lib = _open(build())
     return _lib
+
+
+def _open(path: str):
+    """The library at `path` with the argument types of its entry points."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    L = ctypes.c_long
+    lib.oracle_bf16_value.restype = ctypes.c_double
+    lib.oracle_bf16_value.argtypes = [ctypes.c_uint16]
+    lib.oracle_e4m3_value.restype = ctypes.c_double
+    lib.oracle_e4m3_value.argtypes = [ctypes.c_int]
+    lib.oracle_e2m1_value.restype = ctypes.c_double
+    lib.oracle_e2m1_value.argtypes = [ctypes.c_int]
+    lib.oracle_e4m3_round_div6.restype = ctypes.c_int
+    lib.oracle_e4m3_round_div6.argtypes = [ctypes.c_double]
+    lib.oracle_e2m1_round.restype = ctypes.c_int
+    lib.oracle_e2m1_round.argtypes = [ctypes.c_double, ctypes.c_double]
+    lib.oracle_e2m1_round_many.restype = None
+    lib.oracle_e2m1_round_many.argtypes = [P, P, L, P]
+    lib.oracle_quantize_rows.restype = None
+    lib.oracle_quantize_rows.argtypes = [P, L, L, L, L, P, P, P]
+    lib.oracle_global_scale.restype = ctypes.c_float
+    lib.oracle_global_scale.argtypes = [ctypes.c_double]
+    lib.oracle_quantize_rows_gs.restype = None
+    lib.oracle_quantize_rows_gs.argtypes = [P, L, L, L, L, P, P, P, P]
+    lib.oracle_fq_f64_rows.restype = None
+    lib.oracle_fq_f64_rows.argtypes = [P, L, L, P, P]
+    lib.oracle_operands.restype = None
+    lib.oracle_operands.argtypes = [P, P, P, L, L, L, ctypes.c_uint, P, P, P]
+    lib.oracle_fwd_rows.restype = None
+    lib.oracle_fwd_rows.argtypes = [P, P, P, L, L, L, ctypes.c_double,
+                                    ctypes.c_uint, P, L, P, L, P, P, P, P]
+    lib.oracle_delta.restype = None
+    lib.oracle_delta.argtypes = [P, P, L, L, P]
+    lib.oracle_bwd_dq_rows.restype = None
+    lib.oracle_bwd_dq_rows.argtypes = [P, P, P, P, L, L, L, ctypes.c_double,
+                                       ctypes.c_uint, P, L, P, P, P, P, L, P]
+    lib.oracle_bwd_dkdv_blocks.restype = None
+    lib.oracle_bwd_dkdv_blocks.argtypes = [P, P, P, P, L, L, L, ctypes.c_double,
+                                           ctypes.c_uint, P, L, P, P, P, P, L, P, P]
+    lib.oracle_vsa_select.restype = None
+    lib.oracle_vsa_select.argtypes = [P, P, L, L, L, L, L, P, P]
+    lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_num_threads.argtypes = []
+    return lib
 
 
 def _ptr(a: np.ndarray):

@@ -396,6 +396,36 @@ def test_unquantized_gradients_central_differences():
             assert abs(fd - grad[0, 0][idx]) < 1e-7, (name, idx)
 
 
+@pytest.mark.parametrize("flag", [oracle.QUANT_Q, oracle.QUANT_K, oracle.QUANT_V])
+def test_single_quantizer_equals_quantizing_that_operand_first(flag):
+    """One quantizer on its own is plain attention on that operand's fq copy:
+    fq(Q), fq(K) in blocks of 16 along D, fq(V) in blocks of 16 tokens per
+    channel from token 0, each taken from the block quantizer (pinned above
+    against exact rationals; its values are exact in bf16).  Forward and
+    straight-through gradients against torch's float64 softmax attention
+    and autograd on those copies.  A quantizer keyed to the wrong flag bit,
+    or fq(V) blocked along channels, fails this."""
+    rng = np.random.default_rng(60 + flag)
+    Lq, Lk, D = 24, 48, 32
+    q, k, v, dO = (_rand_bits(rng, (1, 1, L, D)) for L in (Lq, Lk, Lk, Lq))
+    c = 0.35
+    pre = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+    name = {oracle.QUANT_Q: "q", oracle.QUANT_K: "k", oracle.QUANT_V: "v"}[flag]
+    x = pre[name][0, 0]
+    if name == "v":
+        _, _, deq = oracle.quantize_rows(x, D, Lk, 1, D)  # the [D, Lk] view: blocks along tokens
+        deq = deq.T
+    else:
+        _, _, deq = oracle.quantize_rows(x, x.shape[0], D, D, 1)
+    fq_bits = W.f32_to_bf16_bits(deq.astype(np.float32))
+    assert np.array_equal(_f(fq_bits), deq)  # exact in bf16
+    pre[name] = fq_bits.reshape(1, 1, -1, D)
+    out = oracle.attention(q, k, v, c, flags=flag, do_bits=dO)
+    O, gq, gk, gv = _torch_attention_grads(pre["q"][0, 0], pre["k"][0, 0], pre["v"][0, 0], dO[0, 0], c)
+    for key, ref in (("O", O), ("dQ", gq), ("dK", gk), ("dV", gv)):
+        assert np.max(np.abs(out[key][0, 0] - ref)) < 1e-12, key
+
+
 def _ste_surrogate_grads(hd, q, k, v, dO, c, flags):
     """Gradient of the straight-through surrogate by torch autograd.
 
