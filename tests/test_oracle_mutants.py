@@ -153,6 +153,36 @@ MUTANTS = [
     ("global-scale value not divided by G",
      "bf16_of_quotient(E2M1_GRID[c] * sb, g);", "bf16_of_quotient(E2M1_GRID[c] * sb, 1.0);",
      "test_global_scale_format_vs_exact_rationals", {"seed": 1, "mag": 1.0}),
+    ("global amax misses the last column",
+     "        for (long j = 0; j < cols; j++) {\n            double a = fabs(oracle_bf16_value(x[r * srow + j * scol]));",
+     "        for (long j = 0; j < cols - 1; j++) {\n            double a = fabs(oracle_bf16_value(x[r * srow + j * scol]));",
+     "test_global_scale_sees_every_element", {}),
+    ("global-scale block scale without G",
+     "int k = oracle_e4m3_round_div6(ab * g);", "int k = oracle_e4m3_round_div6(ab);",
+     "test_global_scale_format_vs_exact_rationals", {"seed": 1, "mag": 1.0}),
+    ("global-scale code without G",
+     "oracle_e2m1_round(fabs(xb[i]) * g, sb)", "oracle_e2m1_round(fabs(xb[i]), sb)",
+     "test_global_scale_format_vs_exact_rationals", {"seed": 1, "mag": 1.0}),
+    ("global scale overflow to 1",
+     "    if (isinf(g))\n        g = 3.40282347e38f;", "    if (isinf(g))\n        g = 1.0f;",
+     "test_global_scale_special_cases", {}),
+    ("global scale of an all-zero tensor 0",
+     "    if (!(amax > 0.0))\n        return 1.0f;", "    if (!(amax > 0.0))\n        return 0.0f;",
+     "test_global_scale_special_cases", {}),
+    ("scores without sm_scale",
+     "        S[j] = c * dot(Qi, Kh + j * D, D);", "        S[j] = dot(Qi, Kh + j * D, D);",
+     "test_unquantized_forward_matches_sdpa_and_softmax", {}),
+    ("dK/dV ignore the mask",
+     "                Pt[jj] = selected(flags, sel, T, nkt, i, j0 + jj) ? exp(S[jj] - m[i]) : 0.0;",
+     "                Pt[jj] = exp(S[jj] - m[i]);",
+     "test_causal_rows_equal_dense_attention_on_their_prefix", {}),
+    ("dK/dV keep rows that select no key",
+     "            if (!(l[i] > 0.0))\n                continue; /* no selected key: the row adds nothing */",
+     "            if (!(l[i] > 0.0) && 0)\n                continue; /* no selected key: the row adds nothing */",
+     "test_sparse_equals_dense_attention_on_the_gathered_tiles", {"flags": ALL}),
+    ("literal dV reading without the division by l",
+     "                    Pn[jj] = Pt[jj] / l[i];", "                    Pn[jj] = Pt[jj];",
+     "test_dv_literal_reading_zeroes_normalised_blocks", {}),
 ]
 
 

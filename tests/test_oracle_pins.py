@@ -844,6 +844,29 @@ def test_global_max_round_trips_and_sign_symmetry():
         assert np.array_equal(cn, c ^ np.uint8(0x88)) and np.array_equal(dn, d ^ np.uint16(0x8000))
 
 
+def test_global_scale_sees_every_element():
+    """G comes from the largest magnitude anywhere in the view: planted at each
+    corner (and inside) of a row-major tensor, and at the last element of a
+    transposed (strided) view, the largest magnitude M gives G =
+    float32(2688 / M)."""
+    rng = np.random.default_rng(41)
+    rows, cols = 5, 48
+    base = (rng.standard_normal((rows, cols)) * 0.5).astype(np.float32)
+    for r, c in [(0, 0), (0, cols - 1), (rows - 1, 0), (rows - 1, cols - 1), (2, 17)]:
+        for big in (np.float32(-37.0), np.float32(9984.0)):  # both exact in bf16
+            x = base.copy()
+            x[r, c] = big
+            bits = W.f32_to_bf16_bits(x)
+            _, _, _, g = oracle.quantize_rows_gs(bits, rows, cols, cols, 1)
+            assert np.float32(g) == np.float32(2688.0) / np.abs(big), (r, c, big)
+    # rows of the view = the 3 columns of a [16, 3] tensor (element (r, j) at
+    # x[j, r]); the largest magnitude is the view's last element
+    x16 = (rng.standard_normal((16, 3)) * 0.5).astype(np.float32)
+    x16[15, 2] = np.float32(-99.0)
+    _, _, _, g16 = oracle.quantize_rows_gs(W.f32_to_bf16_bits(x16), 3, 16, 1, 3)
+    assert np.float32(g16) == np.float32(2688.0) / np.float32(99.0)
+
+
 def test_global_scale_special_cases():
     """All-zero input: G = 1 and zeros; a max below 2688 / FLT_MAX: the
     quotient overflows float32 and G saturates to the largest finite float."""
