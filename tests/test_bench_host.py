@@ -125,3 +125,26 @@ def test_attention_digest_ignores_comments_not_code():
     edited["bwd.cu"] = base["bwd.cu"].replace("kBN", "kBM", 1)
     assert build.attention_sources_digest(lambda n: edited[n]) != d0
     assert build.code_only("a = 1; // x\n/* y */ b  =\n 2;") == "a = 1; b = 2;"
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` (the float64 oracle on the host cores) prints
+    one JSON line with the keys the benchmark contract names."""
+    import json
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    p = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "2",
+                        "--warmup", "1", "--workload", "tiny"], capture_output=True, text=True, timeout=600,
+                       cwd=root)
+    assert p.returncode == 0, p.stderr
+    lines = [ln for ln in p.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 1 and d["value"] > 0
+    assert d["config"]["workload"] == "tiny"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
