@@ -183,6 +183,17 @@ MUTANTS = [
     ("literal dV reading without the division by l",
      "                    Pn[jj] = Pt[jj] / l[i];", "                    Pn[jj] = Pt[jj];",
      "test_dv_literal_reading_zeroes_normalised_blocks", {}),
+    ("sampled forward rows ignored",
+     "            long i = rows[t];\n            double mi, li;\n            prob_row(Qh + i * D, i, Kh, Lk, D, c, flags, sel, T, S, Pt, Ph, &mi,\n                     &li);\n            /* O_d",
+     "            long i = t;\n            double mi, li;\n            prob_row(Qh + i * D, i, Kh, Lk, D, c, flags, sel, T, S, Pt, Ph, &mi,\n                     &li);\n            /* O_d",
+     "test_sampled_rows_equal_full_computation", {}),
+    ("sampled key blocks ignored",
+     "        long j0 = blocks[t] * BLOCK;", "        long j0 = t * BLOCK;",
+     "test_sampled_rows_equal_full_computation", {}),
+    ("tile mask indexed with 128-token tiles whatever the tile",
+     "    return sel == NULL || sel[(i / T) * nkt + j / T] != 0;",
+     "    return sel == NULL || sel[(i / 128) * nkt + j / 128] != 0;",
+     "test_sparse_equals_dense_attention_on_the_gathered_tiles", {"flags": ALL}),
 ]
 
 
